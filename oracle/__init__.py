@@ -1,0 +1,190 @@
+"""Float64 CPU oracle for the Flash EQ-Linear layer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it, and the
+two share no code: the arithmetic lives in ``eqlinear_oracle.c`` (plain C,
+float64, OpenMP), loaded here through ctypes.
+
+What each function computes, and the passage of the "Flash EQ-Linear" summary
+(gist.science/ko/paper/2607.21271) it follows:
+
+* :func:`forward` -- the operator's plain definition,
+  ``Y[n,d,s] = bias[d] + sum_{c,t} W[d,c,(t-s) mod T] X[n,c,t]``, input feature
+  index ``c*T+t`` ("Key insight": group-circulant weights; "Contributions" item 2:
+  the fast method is exact, so the definition is the oracle).
+* :func:`backward_input`, :func:`backward_weight` -- the gradients of that
+  definition ("Implementation", bullet 1 names backward kernels but no formula).
+* :func:`forward_spectral` -- the method's own route ("Algorithmic approach"
+  items 1-3): DFT over the group axis, per-frequency products on the
+  non-redundant half of the spectrum, inverse DFT, with a counter of real MACs
+  ("Specialisation for p4", bullet 3: 6 real GEMMs, 16/6 fewer MACs).
+* :func:`p4_transform_matrices` -- the real 4x4 DFT / inverse-DFT pair for the
+  p4 group ("Specialisation for p4", bullets 1-2: coefficients 0, +-1, +-1/2).
+
+Every function is pinned by tests/test_oracle_pins.py against values fixed by
+something other than this code (dense replicated matmul, numpy FFT, closed
+forms, hand-worked examples, exact MAC counts).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "eqlinear_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile eqlinear_oracle.c into liboracle.so (gcc, -O3, OpenMP)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall",
+           "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            dp = ctypes.POINTER(ctypes.c_double)
+            i64 = ctypes.c_int64
+            lp = ctypes.POINTER(ctypes.c_int64)
+            for name in ("eqlo_forward", "eqlo_forward_spectral"):
+                fn = getattr(lib, name)
+                fn.argtypes = [ctypes.c_int, i64, i64, i64, dp, dp, dp, dp]
+                fn.restype = i64
+            lib.eqlo_backward_input.argtypes = [ctypes.c_int, i64, i64, i64, dp, dp, dp]
+            lib.eqlo_backward_input.restype = i64
+            lib.eqlo_backward_weight.argtypes = [ctypes.c_int, i64, i64, i64, dp, dp, dp, dp]
+            lib.eqlo_backward_weight.restype = i64
+            lib.eqlo_backward_weight_pairs.argtypes = [ctypes.c_int, i64, i64, i64, dp, dp,
+                                                       i64, lp, lp, dp]
+            lib.eqlo_backward_weight_pairs.restype = None
+            lib.eqlo_p4_transform_matrices.argtypes = [dp, dp]
+            lib.eqlo_p4_transform_matrices.restype = None
+            _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _shapes(T: int, X: np.ndarray, W: np.ndarray):
+    D, C, TW = W.shape
+    if TW != T:
+        raise ValueError(f"W has group axis {TW}, expected T={T}")
+    if X.ndim != 2 or X.shape[1] != C * T:
+        raise ValueError(f"X must be [N, C*T] = [N, {C * T}], got {X.shape}")
+    return X.shape[0], C, D
+
+
+def forward(T: int, X, W, bias=None, return_macs: bool = False):
+    """Y[N, D*T] in float64 from X[N, C*T], W[D, C, T], bias[D] or None."""
+    lib = _load()
+    X, W = _f64(X), _f64(W)
+    N, C, D = _shapes(T, X, W)
+    b = None if bias is None else _f64(bias)
+    Y = np.empty((N, D * T), dtype=np.float64)
+    macs = lib.eqlo_forward(T, N, C, D, _ptr(X), _ptr(W), _ptr(b), _ptr(Y))
+    return (Y, macs) if return_macs else Y
+
+
+def forward_spectral(T: int, X, W, bias=None, return_macs: bool = False):
+    """Same output as :func:`forward`, computed through the DFT route."""
+    if T > 126:
+        raise ValueError("forward_spectral supports T <= 126")
+    lib = _load()
+    X, W = _f64(X), _f64(W)
+    N, C, D = _shapes(T, X, W)
+    b = None if bias is None else _f64(bias)
+    Y = np.empty((N, D * T), dtype=np.float64)
+    macs = lib.eqlo_forward_spectral(T, N, C, D, _ptr(X), _ptr(W), _ptr(b), _ptr(Y))
+    return (Y, macs) if return_macs else Y
+
+
+def backward_input(T: int, dY, W):
+    """dX[N, C*T] from dY[N, D*T] and W[D, C, T]."""
+    lib = _load()
+    dY, W = _f64(dY), _f64(W)
+    D, C, _ = W.shape
+    if dY.ndim != 2 or dY.shape[1] != D * T:
+        raise ValueError(f"dY must be [N, {D * T}]")
+    N = dY.shape[0]
+    dX = np.empty((N, C * T), dtype=np.float64)
+    lib.eqlo_backward_input(T, N, C, D, _ptr(dY), _ptr(W), _ptr(dX))
+    return dX
+
+
+def backward_weight(T: int, X, dY, D: int):
+    """(dW[D, C, T], dbias[D]) from X[N, C*T] and dY[N, D*T]."""
+    lib = _load()
+    X, dY = _f64(X), _f64(dY)
+    N = X.shape[0]
+    C = X.shape[1] // T
+    if X.shape[1] != C * T or dY.shape != (N, D * T):
+        raise ValueError("shape mismatch")
+    dW = np.empty((D, C, T), dtype=np.float64)
+    db = np.empty((D,), dtype=np.float64)
+    lib.eqlo_backward_weight(T, N, C, D, _ptr(X), _ptr(dY), _ptr(dW), _ptr(db))
+    return dW, db
+
+
+def backward_weight_pairs(T: int, X, dY, D: int, d_idx, c_idx):
+    """dW[d_i, c_i, :] for sampled pairs, shape [len(d_idx), T]."""
+    lib = _load()
+    X, dY = _f64(X), _f64(dY)
+    N = X.shape[0]
+    C = X.shape[1] // T
+    d_idx = np.ascontiguousarray(np.asarray(d_idx, dtype=np.int64))
+    c_idx = np.ascontiguousarray(np.asarray(c_idx, dtype=np.int64))
+    if d_idx.shape != c_idx.shape or d_idx.ndim != 1:
+        raise ValueError("d_idx and c_idx must be 1-D and the same length")
+    if (d_idx < 0).any() or (d_idx >= D).any() or (c_idx < 0).any() or (c_idx >= C).any():
+        raise ValueError("pair index out of range")
+    out = np.empty((d_idx.shape[0], T), dtype=np.float64)
+    lp = ctypes.POINTER(ctypes.c_int64)
+    lib.eqlo_backward_weight_pairs(T, N, C, D, _ptr(X), _ptr(dY), d_idx.shape[0],
+                                   d_idx.ctypes.data_as(lp), c_idx.ctypes.data_as(lp),
+                                   _ptr(out))
+    return out
+
+
+def p4_transform_matrices():
+    """(F, G): real 4x4 forward DFT (rows Re0, Re2, Re1, Im1) and its inverse."""
+    lib = _load()
+    F = np.empty((4, 4), dtype=np.float64)
+    G = np.empty((4, 4), dtype=np.float64)
+    lib.eqlo_p4_transform_matrices(_ptr(F), _ptr(G))
+    return F, G
+
+
+def threads_used() -> int:
+    """Threads OpenMP will use for the parallel loops (OMP_NUM_THREADS or cores)."""
+    env = os.environ.get("OMP_NUM_THREADS")
+    if env:
+        try:
+            return max(1, int(env.split(",")[0]))
+        except ValueError:
+            pass
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
