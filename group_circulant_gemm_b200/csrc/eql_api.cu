@@ -1,0 +1,248 @@
+// C ABI of the EQ-Linear library: plans, argument checks, kernel dispatch.
+// The operations and their definitions are documented in include/eqlinear.h.
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "../../include/eqlinear.h"
+#include "eql_kernels.h"
+
+using eql::DType;
+
+struct eqlinear_plan_s {
+  int T, C, D;
+  eqlinear_dtype_t dtype;
+  eqlinear_kernel_t kernel;
+  int device;
+  int num_sms;
+  int* status;  // device word written by kernels whose bounded waits give up
+  eql::Twiddles tw;
+};
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+size_t elem_size(eqlinear_dtype_t dt) { return dt == EQL_F32 ? 4 : 2; }
+DType to_dt(eqlinear_dtype_t dt) { return dt == EQL_F32 ? DType::F32 : DType::F16; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void make_twiddles(int T, eql::Twiddles* tw) {
+  std::memset(tw, 0, sizeof(*tw));
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int k = 0; k < T; ++k) {
+    for (int t = 0; t < T; ++t) {
+      // reduce k*t mod T first so the angle is exact-ish and symmetric values match
+      const int m = (k * t) % T;
+      float c = (float)std::cos(two_pi * m / T);
+      float s = (float)std::sin(two_pi * m / T);
+      if (std::fabs(c) < 1e-7f) c = 0.f;
+      if (std::fabs(s) < 1e-7f) s = 0.f;
+      tw->cs[k][t] = c;
+      tw->sn[k][t] = s;
+    }
+  }
+}
+
+eqlinear_status_t from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return EQL_OK;
+  if (e == cudaErrorNotSupported) return EQL_ERR_UNSUPPORTED;
+  return EQL_ERR_CUDA;
+}
+
+size_t plane_elems(const eqlinear_plan_s* p) { return (size_t)p->C * p->D; }
+
+const void* fwd_block(const eqlinear_plan_s* p, const void* W_hat) { return W_hat; }
+const void* adj_block(const eqlinear_plan_s* p, const void* W_hat) {
+  return static_cast<const char*>(W_hat) +
+         (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
+}
+
+// Forward-shaped product used by both eqlinear_forward (Cin=C, Cout=D) and
+// eqlinear_backward_input (Cin=D, Cout=C).
+//   own   : planes [P][Cout][Cin]  (tensor-core operand, K-major)
+//   other : planes [P][Cin][Cout]  (CUDA-core operand)
+eqlinear_status_t run_forward_like(eqlinear_plan_s* p, const void* X, int64_t N, int Cin,
+                                   int Cout, const void* own, const void* other,
+                                   const void* bias, void* Y, cudaStream_t st) {
+  const bool tc_ok = eql::fwd_tc_supported(p->T, to_dt(p->dtype), N, Cin, Cout);
+  if (p->kernel == EQL_KERNEL_TCGEN05 && !tc_ok) return EQL_ERR_UNSUPPORTED;
+  if (p->kernel != EQL_KERNEL_SIMT && tc_ok)
+    return from_cuda(eql::launch_fwd_tc(p->T, X, N, Cin, Cout, own, bias, Y, p->status,
+                                        p->num_sms, st));
+  return from_cuda(eql::launch_fwd_simt(p->T, to_dt(p->dtype), X, N, Cin, Cout, other, bias, Y,
+                                        p->tw, st));
+}
+
+eqlinear_status_t check_plan_device(const eqlinear_plan_s* p) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return EQL_ERR_CUDA;
+  return dev == p->device ? EQL_OK : EQL_ERR_INVALID_ARG;
+}
+
+}  // namespace
+
+extern "C" {
+
+int eqlinear_version(void) { return kVersion; }
+
+const char* eqlinear_status_string(eqlinear_status_t s) {
+  switch (s) {
+    case EQL_OK: return "EQL_OK";
+    case EQL_ERR_INVALID_ARG: return "EQL_ERR_INVALID_ARG: invalid argument";
+    case EQL_ERR_UNSUPPORTED: return "EQL_ERR_UNSUPPORTED: no kernel for this T/dtype/shape";
+    case EQL_ERR_ALIGNMENT: return "EQL_ERR_ALIGNMENT: device pointer not 16-byte aligned";
+    case EQL_ERR_WORKSPACE: return "EQL_ERR_WORKSPACE: workspace missing or too small";
+    case EQL_ERR_CUDA: return "EQL_ERR_CUDA: CUDA runtime error";
+    case EQL_ERR_TIMEOUT: return "EQL_ERR_TIMEOUT: a device-side bounded wait gave up";
+  }
+  return "EQL_ERR_UNKNOWN";
+}
+
+eqlinear_status_t eqlinear_plan_create(int T, int C, int D, eqlinear_dtype_t dtype,
+                                       eqlinear_plan_t* out) {
+  if (!out || C <= 0 || D <= 0 || T <= 0) return EQL_ERR_INVALID_ARG;
+  if (dtype != EQL_F32 && dtype != EQL_F16) return EQL_ERR_INVALID_ARG;
+  if (T > eql::kMaxT) return EQL_ERR_UNSUPPORTED;
+  if ((int64_t)C * T > 0x7fffffff || (int64_t)D * T > 0x7fffffff) return EQL_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return EQL_ERR_CUDA;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return EQL_ERR_CUDA;
+  eqlinear_plan_s* p = new (std::nothrow) eqlinear_plan_s();
+  if (!p) return EQL_ERR_INVALID_ARG;
+  p->T = T;
+  p->C = C;
+  p->D = D;
+  p->dtype = dtype;
+  p->kernel = EQL_KERNEL_AUTO;
+  p->device = dev;
+  p->num_sms = sms;
+  make_twiddles(T, &p->tw);
+  if (cudaMalloc(&p->status, sizeof(int)) != cudaSuccess) {
+    delete p;
+    return EQL_ERR_CUDA;
+  }
+  if (cudaMemset(p->status, 0, sizeof(int)) != cudaSuccess) {
+    cudaFree(p->status);
+    delete p;
+    return EQL_ERR_CUDA;
+  }
+  *out = p;
+  return EQL_OK;
+}
+
+void eqlinear_plan_destroy(eqlinear_plan_t p) {
+  if (!p) return;
+  if (p->status) cudaFree(p->status);
+  delete p;
+}
+
+eqlinear_status_t eqlinear_plan_set_kernel(eqlinear_plan_t p, eqlinear_kernel_t which) {
+  if (!p) return EQL_ERR_INVALID_ARG;
+  if (which != EQL_KERNEL_AUTO && which != EQL_KERNEL_SIMT && which != EQL_KERNEL_TCGEN05)
+    return EQL_ERR_INVALID_ARG;
+  p->kernel = which;
+  return EQL_OK;
+}
+
+const char* eqlinear_forward_kernel_name(eqlinear_plan_t p, int64_t N) {
+  if (!p) return "unsupported";
+  const bool tc_ok = eql::fwd_tc_supported(p->T, to_dt(p->dtype), N, p->C, p->D);
+  if (p->kernel == EQL_KERNEL_TCGEN05) return tc_ok ? "tcgen05" : "unsupported";
+  if (p->kernel == EQL_KERNEL_AUTO && tc_ok) return "tcgen05";
+  return "simt";
+}
+
+const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t p, int64_t N) {
+  (void)N;
+  if (!p) return "unsupported";
+  if (p->kernel == EQL_KERNEL_TCGEN05) return "unsupported";
+  return "simt";
+}
+
+size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t p) {
+  if (!p) return 0;
+  return 2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
+}
+
+eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, void* W_hat,
+                                           void* stream) {
+  if (!p || !W || !W_hat) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(W_hat)) return EQL_ERR_ALIGNMENT;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  void* fwd = W_hat;
+  void* adj = const_cast<void*>(adj_block(p, W_hat));
+  return from_cuda(eql::launch_prepare(p->T, to_dt(p->dtype), W, p->C, p->D, fwd, adj, p->tw,
+                                       (cudaStream_t)stream));
+}
+
+eqlinear_status_t eqlinear_forward(eqlinear_plan_t p, const void* X, int64_t N,
+                                   const void* W_hat, const void* bias, void* Y, void* stream) {
+  if (!p || N < 0) return EQL_ERR_INVALID_ARG;
+  if (N == 0) return EQL_OK;
+  if (!X || !W_hat || !Y) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_hat) || !aligned16(Y) || (bias && !aligned16(bias)))
+    return EQL_ERR_ALIGNMENT;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  return run_forward_like(p, X, N, p->C, p->D, fwd_block(p, W_hat), adj_block(p, W_hat), bias,
+                          Y, (cudaStream_t)stream);
+}
+
+eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int64_t N,
+                                          const void* W_hat, void* dX, void* stream) {
+  if (!p || N < 0) return EQL_ERR_INVALID_ARG;
+  if (N == 0) return EQL_OK;
+  if (!dY || !W_hat || !dX) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(W_hat) || !aligned16(dX)) return EQL_ERR_ALIGNMENT;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  // dX is the forward-shaped product with the adjoint weights: input width D,
+  // output width C; "own" planes are the adjoint block [P][C][D].
+  return run_forward_like(p, dY, N, p->D, p->C, adj_block(p, W_hat), fwd_block(p, W_hat),
+                          nullptr, dX, (cudaStream_t)stream);
+}
+
+size_t eqlinear_backward_weight_workspace_bytes(eqlinear_plan_t p, int64_t N) {
+  if (!p || N < 0) return 0;
+  return eql::wgrad_simt_workspace(p->T, N, p->C, p->D, p->num_sms);
+}
+
+eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t p, const void* X, const void* dY,
+                                           int64_t N, void* dW, void* dbias, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  if (!p || N < 0 || !dW) return EQL_ERR_INVALID_ARG;
+  if (N > 0 && (!X || !dY)) return EQL_ERR_INVALID_ARG;
+  if (p->kernel == EQL_KERNEL_TCGEN05) return EQL_ERR_UNSUPPORTED;
+  if ((X && !aligned16(X)) || (dY && !aligned16(dY)) || !aligned16(dW) ||
+      (dbias && !aligned16(dbias)) || (workspace && !aligned16(workspace)))
+    return EQL_ERR_ALIGNMENT;
+  const size_t need = eql::wgrad_simt_workspace(p->T, N, p->C, p->D, p->num_sms);
+  if (!workspace || workspace_bytes < need) return EQL_ERR_WORKSPACE;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  const int splits = eql::wgrad_simt_splits(p->T, N, p->C, p->D, p->num_sms);
+  return from_cuda(eql::launch_wgrad_simt(p->T, to_dt(p->dtype), X, dY, N, p->C, p->D, dW,
+                                          dbias, static_cast<float*>(workspace), splits, p->tw,
+                                          (cudaStream_t)stream));
+}
+
+eqlinear_status_t eqlinear_get_status(eqlinear_plan_t p, void* stream) {
+  if (!p) return EQL_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return EQL_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, p->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return EQL_ERR_CUDA;
+  if (h != 0) {
+    if (cudaMemset(p->status, 0, sizeof(int)) != cudaSuccess) return EQL_ERR_CUDA;
+    return EQL_ERR_TIMEOUT;
+  }
+  return EQL_OK;
+}
+
+}  // extern "C"

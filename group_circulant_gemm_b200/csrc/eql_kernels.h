@@ -1,0 +1,48 @@
+// Host-side launchers shared between the C ABI (eql_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "eql_common.cuh"
+
+namespace eql {
+
+enum class DType { F32 = 0, F16 = 1 };
+
+// Prepared-weight transform: W[D][C][T] -> forward planes [P][D][C] and
+// adjoint planes [P][C][D] (see eqlinear.h for the plane order).
+cudaError_t launch_prepare(int T, DType dt, const void* W, int C, int D, void* fwd, void* adj,
+                           const Twiddles& tw, cudaStream_t st);
+
+// CUDA-core forward over a group-circulant operator.
+//   X [N][Cin*T] -> Y [N][Cout*T]; Wt = planes [P][Cin][Cout] of the OTHER block
+//   (adjoint block for the forward pass, forward block for dX): the kernel takes
+//   Re from the Re planes and Im from the "-Im" slots, which hold the right sign.
+cudaError_t launch_fwd_simt(int T, DType dt, const void* X, int64_t N, int Cin, int Cout,
+                            const void* Wt, const void* bias, void* Y, const Twiddles& tw,
+                            cudaStream_t st);
+
+// CUDA-core weight gradient: split reduction over rows into FP32 partial spectra,
+// then a finalize kernel (sum in fixed split order, inverse DFT, cast).
+int wgrad_simt_splits(int T, int64_t N, int C, int D, int num_sms);
+size_t wgrad_simt_workspace(int T, int64_t N, int C, int D, int num_sms);
+cudaError_t launch_wgrad_simt(int T, DType dt, const void* X, const void* dY, int64_t N, int C,
+                              int D, void* dW, void* dbias, float* ws, int splits,
+                              const Twiddles& tw, cudaStream_t st);
+
+// Finalize of a split weight-gradient reduction: partial spectra
+// part[split][T planes][D][C] (+ bias partials [split][D]) -> dW[D][C][T], dbias[D].
+cudaError_t launch_wgrad_finalize(int T, DType dt, const float* part, const float* bpart,
+                                  int splits, int C, int D, void* dW, void* dbias,
+                                  const Twiddles& tw, cudaStream_t st);
+
+// tcgen05/TMEM tensor-core forward (FP16 in, FP32 accumulate, FP16 out).
+// Returns cudaErrorNotSupported when the shape does not fit the kernel.
+bool fwd_tc_supported(int T, DType dt, int64_t N, int Cin, int Cout);
+cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
+                          const void* Wplanes /* own block [P][Cout][Cin] */, const void* bias,
+                          void* Y, int* status, int num_sms, cudaStream_t st);
+
+}  // namespace eql

@@ -1,0 +1,96 @@
+"""Torch-tensor convenience wrapper over the C ABI (allocation + marshalling only).
+
+PyTorch provides device memory and streams; every arithmetic step runs in
+libeqlinear.so through the functions of :mod:`group_circulant_gemm_b200.native`.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import native as _n
+
+_DT = {torch.float32: _n.EQL_F32, torch.float16: _n.EQL_F16}
+_KERNEL = {"auto": _n.EQL_KERNEL_AUTO, "simt": _n.EQL_KERNEL_SIMT,
+           "tcgen05": _n.EQL_KERNEL_TCGEN05}
+
+
+class EqLinearPlan:
+    """A plan for the EQ-Linear layer of group order T, C -> D channels."""
+
+    def __init__(self, T: int, C: int, D: int, dtype: torch.dtype, kernel: str = "auto"):
+        if dtype not in _DT:
+            raise ValueError(f"unsupported dtype {dtype}")
+        self.T, self.C, self.D, self.dtype = T, C, D, dtype
+        self.handle = _n.eqlinear_plan_create(T, C, D, _DT[dtype])
+        self.set_kernel(kernel)
+
+    def set_kernel(self, kernel: str) -> None:
+        _n.eqlinear_plan_set_kernel(self.handle, _KERNEL[kernel])
+        self.kernel = kernel
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            _n.eqlinear_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, t: torch.Tensor, shape, name: str) -> None:
+        if not t.is_cuda or t.dtype != self.dtype or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of {self.dtype}")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+    def forward_kernel_name(self, N: int) -> str:
+        return _n.eqlinear_forward_kernel_name(self.handle, N)
+
+    def prepare_weights(self, W: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+        self._check(W, (self.D, self.C, self.T), "W")
+        nbytes = _n.eqlinear_prepared_weight_bytes(self.handle)
+        if out is None:
+            out = torch.empty(nbytes // W.element_size(), dtype=self.dtype, device=W.device)
+        _n.eqlinear_prepare_weights(self.handle, W, out)
+        return out
+
+    def forward(self, X, W_hat, bias=None, out=None) -> torch.Tensor:
+        N = X.shape[0]
+        self._check(X, (N, self.C * self.T), "X")
+        if bias is not None:
+            self._check(bias, (self.D,), "bias")
+        if out is None:
+            out = torch.empty((N, self.D * self.T), dtype=self.dtype, device=X.device)
+        _n.eqlinear_forward(self.handle, X, N, W_hat, bias, out)
+        return out
+
+    def backward_input(self, dY, W_hat, out=None) -> torch.Tensor:
+        N = dY.shape[0]
+        self._check(dY, (N, self.D * self.T), "dY")
+        if out is None:
+            out = torch.empty((N, self.C * self.T), dtype=self.dtype, device=dY.device)
+        _n.eqlinear_backward_input(self.handle, dY, N, W_hat, out)
+        return out
+
+    def workspace_bytes(self, N: int) -> int:
+        return _n.eqlinear_backward_weight_workspace_bytes(self.handle, N)
+
+    def backward_weight(self, X, dY, dW=None, dbias=None, workspace=None, want_bias=True):
+        N = X.shape[0]
+        self._check(X, (N, self.C * self.T), "X")
+        self._check(dY, (N, self.D * self.T), "dY")
+        if dW is None:
+            dW = torch.empty((self.D, self.C, self.T), dtype=self.dtype, device=X.device)
+        if dbias is None and want_bias:
+            dbias = torch.empty((self.D,), dtype=self.dtype, device=X.device)
+        nb = self.workspace_bytes(N)
+        if workspace is None:
+            workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=X.device)
+        _n.eqlinear_backward_weight(self.handle, X, dY, N, dW, dbias, workspace,
+                                    workspace.numel() * workspace.element_size())
+        return dW, dbias
+
+    def status(self) -> int:
+        return _n.eqlinear_get_status(self.handle)

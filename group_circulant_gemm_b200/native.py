@@ -1,0 +1,161 @@
+"""ctypes binding of libeqlinear.so, with the C ABI's own names.
+
+Every function here only marshals arguments (tensor -> device pointer, stream ->
+handle) and checks the returned status; all computation happens in the CUDA
+library.  There is no fallback: if the shared library is missing or was built
+for another architecture, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libeqlinear.so")
+
+EQL_OK, EQL_ERR_INVALID_ARG, EQL_ERR_UNSUPPORTED, EQL_ERR_ALIGNMENT = 0, 1, 2, 3
+EQL_ERR_WORKSPACE, EQL_ERR_CUDA, EQL_ERR_TIMEOUT = 4, 5, 6
+EQL_F32, EQL_F16 = 0, 1
+EQL_KERNEL_AUTO, EQL_KERNEL_SIMT, EQL_KERNEL_TCGEN05 = 0, 1, 2
+
+EXPORTED = (
+    "eqlinear_version", "eqlinear_status_string", "eqlinear_plan_create",
+    "eqlinear_plan_destroy", "eqlinear_plan_set_kernel", "eqlinear_forward_kernel_name",
+    "eqlinear_backward_weight_kernel_name", "eqlinear_prepared_weight_bytes",
+    "eqlinear_prepare_weights", "eqlinear_forward", "eqlinear_backward_input",
+    "eqlinear_backward_weight_workspace_bytes", "eqlinear_backward_weight",
+    "eqlinear_get_status",
+)
+
+
+class EqLinearError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.eqlinear_status_string(status).decode()}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m group_circulant_gemm_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, sz, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+    sig = {
+        "eqlinear_version": ([], i32),
+        "eqlinear_status_string": ([i32], ctypes.c_char_p),
+        "eqlinear_plan_create": ([i32, i32, i32, i32, ctypes.POINTER(vp)], i32),
+        "eqlinear_plan_destroy": ([vp], None),
+        "eqlinear_plan_set_kernel": ([vp, i32], i32),
+        "eqlinear_forward_kernel_name": ([vp, i64], ctypes.c_char_p),
+        "eqlinear_backward_weight_kernel_name": ([vp, i64], ctypes.c_char_p),
+        "eqlinear_prepared_weight_bytes": ([vp], sz),
+        "eqlinear_prepare_weights": ([vp, vp, vp, vp], i32),
+        "eqlinear_forward": ([vp, vp, i64, vp, vp, vp, vp], i32),
+        "eqlinear_backward_input": ([vp, vp, i64, vp, vp, vp], i32),
+        "eqlinear_backward_weight_workspace_bytes": ([vp, i64], sz),
+        "eqlinear_backward_weight": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
+        "eqlinear_get_status": ([vp, vp], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != EQL_OK:
+        raise EqLinearError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# --- the C ABI, name for name --------------------------------------------------
+
+def eqlinear_version() -> int:
+    return _lib.eqlinear_version()
+
+
+def eqlinear_status_string(status: int) -> str:
+    return _lib.eqlinear_status_string(status).decode()
+
+
+def eqlinear_plan_create(T: int, C: int, D: int, dtype: int) -> int:
+    out = ctypes.c_void_p()
+    _check(_lib.eqlinear_plan_create(T, C, D, dtype, ctypes.byref(out)), "eqlinear_plan_create")
+    return out.value
+
+
+def eqlinear_plan_destroy(plan: int) -> None:
+    _lib.eqlinear_plan_destroy(plan)
+
+
+def eqlinear_plan_set_kernel(plan: int, which: int) -> None:
+    _check(_lib.eqlinear_plan_set_kernel(plan, which), "eqlinear_plan_set_kernel")
+
+
+def eqlinear_forward_kernel_name(plan: int, N: int) -> str:
+    return _lib.eqlinear_forward_kernel_name(plan, N).decode()
+
+
+def eqlinear_backward_weight_kernel_name(plan: int, N: int) -> str:
+    return _lib.eqlinear_backward_weight_kernel_name(plan, N).decode()
+
+
+def eqlinear_prepared_weight_bytes(plan: int) -> int:
+    return _lib.eqlinear_prepared_weight_bytes(plan)
+
+
+def eqlinear_prepare_weights(plan: int, W, W_hat, stream=None) -> None:
+    _check(_lib.eqlinear_prepare_weights(plan, _ptr(W), _ptr(W_hat), _stream(stream)),
+           "eqlinear_prepare_weights")
+
+
+def eqlinear_forward(plan: int, X, N: int, W_hat, bias, Y, stream=None) -> None:
+    _check(_lib.eqlinear_forward(plan, _ptr(X), N, _ptr(W_hat), _ptr(bias), _ptr(Y),
+                                 _stream(stream)), "eqlinear_forward")
+
+
+def eqlinear_backward_input(plan: int, dY, N: int, W_hat, dX, stream=None) -> None:
+    _check(_lib.eqlinear_backward_input(plan, _ptr(dY), N, _ptr(W_hat), _ptr(dX),
+                                        _stream(stream)), "eqlinear_backward_input")
+
+
+def eqlinear_backward_weight_workspace_bytes(plan: int, N: int) -> int:
+    return _lib.eqlinear_backward_weight_workspace_bytes(plan, N)
+
+
+def eqlinear_backward_weight(plan: int, X, dY, N: int, dW, dbias, workspace,
+                             workspace_bytes: int, stream=None) -> None:
+    _check(_lib.eqlinear_backward_weight(plan, _ptr(X), _ptr(dY), N, _ptr(dW), _ptr(dbias),
+                                         _ptr(workspace), workspace_bytes, _stream(stream)),
+           "eqlinear_backward_weight")
+
+
+def eqlinear_get_status(plan: int, stream=None) -> int:
+    return _lib.eqlinear_get_status(plan, _stream(stream))
+
+
+def raw_status(fn_name: str, *args) -> int:
+    """Call an ABI function and return its raw status (for error-path tests)."""
+    return getattr(_lib, fn_name)(*args)

@@ -1,0 +1,181 @@
+/*
+ * eqlinear.h -- C ABI of the B200 (sm_100a) Flash EQ-Linear library.
+ *
+ * The layer (Flash EQ-Linear technical summary, gist.science/ko/paper/2607.21271,
+ * "Key insight" and "Algorithmic approach") is the group-equivariant linear map
+ *
+ *     Y[n, d*T+s] = bias[d] + sum_{c<C} sum_{t<T} W[d][c][(t-s) mod T] * X[n, c*T+t]
+ *
+ * over the cyclic group of order T.  Its weight matrix is group-circulant, so the
+ * library computes it exactly through a DFT over the group axis: a real DFT of
+ * every length-T group vector, one real GEMM per real frequency and four per
+ * complex frequency (conjugate symmetry keeps only k = 0..floor(T/2)), then the
+ * inverse DFT.  For the p4 group (T = 4) the transforms use only 0, +-1 and
+ * +-1/2-type coefficients and the products are six real GEMMs ("Specialisation
+ * for p4").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every tensor is a dense row-major array in DEVICE memory, owned by the
+ *    caller, in the plan's dtype (EQL_F32: float, EQL_F16: IEEE binary16),
+ *    accumulation is FP32.  The library never allocates device memory after
+ *    eqlinear_plan_create and never frees caller memory.
+ *  - Every device pointer must be 16-byte aligned, and rows must be a whole
+ *    number of 16-byte units for the tensor-core path (the dispatcher falls
+ *    back to the CUDA-core path when they are not); violations of the 16-byte
+ *    pointer rule return EQL_ERR_ALIGNMENT before anything is launched.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All calls are
+ *    asynchronous on it and return once the work is enqueued; only
+ *    eqlinear_get_status synchronises.
+ *  - The plan is bound to the CUDA device current at eqlinear_plan_create;
+ *    every call must be made with that device current.
+ *  - A plan is immutable after creation except for eqlinear_plan_set_kernel;
+ *    it may be shared by several streams provided each concurrent
+ *    eqlinear_backward_weight call has its own workspace.
+ *  - Argument errors are reported synchronously and nothing is launched.
+ *    Launch failures return EQL_ERR_CUDA.  Device-side failures (a bounded
+ *    wait that gave up) set a sticky status word in the plan, read by
+ *    eqlinear_get_status.
+ */
+#ifndef EQLINEAR_H_
+#define EQLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EQL_API __attribute__((visibility("default")))
+#else
+#define EQL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct eqlinear_plan_s* eqlinear_plan_t;
+
+typedef enum {
+  EQL_OK = 0,
+  EQL_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad enum      */
+  EQL_ERR_UNSUPPORTED = 2, /* T or dtype with no instantiated kernel         */
+  EQL_ERR_ALIGNMENT = 3,   /* device pointer not 16-byte aligned             */
+  EQL_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required     */
+  EQL_ERR_CUDA = 5,        /* CUDA runtime error (launch, allocation, ...)   */
+  EQL_ERR_TIMEOUT = 6      /* a device-side bounded wait gave up             */
+} eqlinear_status_t;
+
+typedef enum { EQL_F32 = 0, EQL_F16 = 1 } eqlinear_dtype_t;
+
+/* Kernel family selection (testing and measurement; AUTO is the default). */
+typedef enum {
+  EQL_KERNEL_AUTO = 0,   /* tensor cores where the shape allows, else CUDA cores */
+  EQL_KERNEL_SIMT = 1,   /* CUDA-core FP32 FMA kernels, any supported shape      */
+  EQL_KERNEL_TCGEN05 = 2 /* tcgen05/TMEM tensor-core kernels; calls whose shape
+                            they cannot take return EQL_ERR_UNSUPPORTED         */
+} eqlinear_kernel_t;
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+EQL_API int eqlinear_version(void);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+EQL_API const char* eqlinear_status_string(eqlinear_status_t status);
+
+/*
+ * Create a plan for group order T, C input channels and D output channels per
+ * group element (input width C*T features, output width D*T), in `dtype`.
+ * Supported T: 1..8.  The plan owns host metadata (DFT twiddles computed in
+ * double on the host, rounded once to float) and a 4-byte device status word
+ * allocated on the current device.  *out is written only on EQL_OK.
+ */
+EQL_API eqlinear_status_t eqlinear_plan_create(int T, int C, int D, eqlinear_dtype_t dtype,
+                                       eqlinear_plan_t* out);
+
+/* Free the plan and its status word.  NULL is ignored.  The caller must make
+ * sure no call using the plan is still running on any stream. */
+EQL_API void eqlinear_plan_destroy(eqlinear_plan_t plan);
+
+/* Choose the kernel family used by later calls (not thread-safe with respect
+ * to calls running concurrently on the same plan). */
+EQL_API eqlinear_status_t eqlinear_plan_set_kernel(eqlinear_plan_t plan, eqlinear_kernel_t which);
+
+/* Name of the kernel eqlinear_forward would launch for N rows with the
+ * current selection ("simt", "tcgen05", or "unsupported"). */
+EQL_API const char* eqlinear_forward_kernel_name(eqlinear_plan_t plan, int64_t N);
+
+/* Same for eqlinear_backward_weight. */
+EQL_API const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t plan, int64_t N);
+
+/*
+ * Size in bytes of the prepared (frequency-domain) weights W_hat.
+ * W_hat layout, plane by plane, each plane a dense matrix in the plan dtype:
+ *   forward planes  [P][D][C]  then  adjoint planes [P][C][D],  P = T + n_cplx,
+ * where n_cplx = number of complex frequencies (T-1)/2 for odd T, T/2-1 for
+ * even T.  Plane order inside each block: real frequency 0; real frequency T/2
+ * (even T); Re and Im of each complex frequency k = 1..n_cplx; then -Im of each
+ * complex frequency.  Forward planes hold conj(DFT(W)) (the correlation form of
+ * the convolution theorem), adjoint planes hold DFT(W) transposed, used for dX.
+ */
+EQL_API size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t plan);
+
+/*
+ * One-time frequency-domain transform of the weights ("Implementation": the
+ * layer replaces a naive EQ-Linear with no retraining; only the parameters are
+ * re-expressed).  W is [D][C][T] in the plan dtype; W_hat receives
+ * eqlinear_prepared_weight_bytes(plan) bytes.  The DFT runs in FP32 and is
+ * rounded once to the plan dtype.
+ */
+EQL_API eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t plan, const void* W, void* W_hat,
+                                           void* stream);
+
+/*
+ * Forward pass ("Algorithmic approach" items 1-3; "Implementation": fused
+ * dataflow with no intermediate global-memory writes).
+ *   X     [N][C*T]  input, feature index c*T+t
+ *   W_hat prepared weights of this plan
+ *   bias  [D] in the plan dtype, or NULL for no bias
+ *   Y     [N][D*T]  output, feature index d*T+s (must not overlap X)
+ * N = 0 is a no-op returning EQL_OK.
+ */
+EQL_API eqlinear_status_t eqlinear_forward(eqlinear_plan_t plan, const void* X, int64_t N,
+                                   const void* W_hat, const void* bias, void* Y, void* stream);
+
+/*
+ * Gradient with respect to the input ("Implementation": backward pass):
+ *   dX[n, c*T+t] = sum_{d,s} dY[n, d*T+s] * W[d][c][(t-s) mod T]
+ * which is the same group-circulant product with the transposed weights and the
+ * opposite conjugation.  dY [N][D*T], dX [N][C*T] (must not overlap).
+ */
+EQL_API eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t plan, const void* dY, int64_t N,
+                                          const void* W_hat, void* dX, void* stream);
+
+/* Workspace bytes eqlinear_backward_weight needs for N rows (FP32 partial
+ * spectra of the split reduction over rows). */
+EQL_API size_t eqlinear_backward_weight_workspace_bytes(eqlinear_plan_t plan, int64_t N);
+
+/*
+ * Gradient with respect to the weights and the bias:
+ *   dW[d][c][u] = sum_{n,s} dY[n, d*T+s] * X[n, c*T + (s+u) mod T]
+ *   dbias[d]    = sum_{n,s} dY[n, d*T+s]
+ * computed per frequency as a reduction over the N rows (FP32, fixed order, so
+ * results are bitwise reproducible for a given N), then one inverse DFT.
+ *   X [N][C*T], dY [N][D*T], dW [D][C][T] (plan dtype, overwritten),
+ *   dbias [D] or NULL, workspace >= eqlinear_backward_weight_workspace_bytes.
+ * N = 0 writes zeros to dW and dbias.
+ */
+EQL_API eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t plan, const void* X, const void* dY,
+                                           int64_t N, void* dW, void* dbias, void* workspace,
+                                           size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the plan's device status word.
+ * Returns EQL_OK, EQL_ERR_TIMEOUT if a kernel's bounded wait gave up since the
+ * last call, or EQL_ERR_CUDA if the stream reports an error.
+ */
+EQL_API eqlinear_status_t eqlinear_get_status(eqlinear_plan_t plan, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EQLINEAR_H_ */
