@@ -130,6 +130,35 @@ def test_edge_shapes_all_ops(T, N, C, D, dtype):
     assert _rel(db.double().cpu().numpy(), rdb) <= TOL[dtype]
 
 
+TC_EDGE = [
+    # N, C, D : ragged rows, channels and out-channels for the tcgen05 p4 path
+    (1, 8, 8), (127, 24, 136), (129, 40, 200), (300, 200, 8), (513, 64, 384), (260, 328, 72),
+]
+
+
+@pytest.mark.parametrize("N,C,D", TC_EDGE)
+def test_tcgen05_edge_shapes(N, C, D):
+    w = Workload("tcedge", 4, N, C, D, "f16", True, 500 + N + C + D)
+    inp = make_inputs(w, need_dy=True)
+    p = _plan(w, "tcgen05")
+    assert p.forward_kernel_name(N) == "tcgen05"
+    Wh = p.prepare_weights(_dev(inp["W"]))
+    Y = p.forward(_dev(inp["X"]), Wh, _dev(inp["bias"])).double().cpu().numpy()
+    assert _rel(Y, oracle.forward(4, inp["X"], inp["W"], inp["bias"])) <= TOL["f16"]
+    dX = p.backward_input(_dev(inp["dY"]), Wh).double().cpu().numpy()
+    assert _rel(dX, oracle.backward_input(4, inp["dY"], inp["W"])) <= TOL["f16"]
+    assert p.status() == 0
+
+
+def test_tcgen05_matches_simt_bitwise_structure():
+    """Same inputs through both kernel families agree to FP16 output rounding."""
+    w = Workload("tcsimt", 4, 1000, 96, 256, "f16", True, 31)
+    inp = make_inputs(w)
+    a, _ = _gpu_forward(w, inp, "tcgen05")
+    b, _ = _gpu_forward(w, inp, "simt")
+    assert _rel(a, b) <= 1e-3
+
+
 def test_no_bias_and_zero_rows():
     w = Workload("nb", 4, 40, 8, 8, "f32", True, 5)
     inp = make_inputs(w, need_dy=True)
