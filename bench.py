@@ -91,7 +91,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -233,15 +233,16 @@ def run_ours(args, workload):
             x = outs[i % nsets][li]
 
     kernel_names = [p.forward_kernel_name(N) for p in plans]
+    # the clock sampler runs from the start of warm-up to the end of the timed region
+    clocks = ClockSampler(local)
+    if rank == 0:
+        clocks.start()
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
     for p in plans:
         assert p.status() == 0
 
-    clocks = ClockSampler(local)
-    if rank == 0:
-        clocks.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()

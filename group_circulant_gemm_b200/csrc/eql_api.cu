@@ -6,18 +6,9 @@
 
 #include "../../include/eqlinear.h"
 #include "eql_kernels.h"
+#include "eql_plan.h"
 
 using eql::DType;
-
-struct eqlinear_plan_s {
-  int T, C, D;
-  eqlinear_dtype_t dtype;
-  eqlinear_kernel_t kernel;
-  int device;
-  int num_sms;
-  int* status;  // device word written by kernels whose bounded waits give up
-  eql::Twiddles tw;
-};
 
 namespace {
 

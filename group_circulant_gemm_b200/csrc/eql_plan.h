@@ -1,0 +1,15 @@
+// Internal definition of the opaque plan handle of include/eqlinear.h.
+#pragma once
+
+#include "../../include/eqlinear.h"
+#include "eql_common.cuh"
+
+struct eqlinear_plan_s {
+  int T, C, D;
+  eqlinear_dtype_t dtype;
+  eqlinear_kernel_t kernel;
+  int device;
+  int num_sms;
+  int* status;  // device word written by kernels whose bounded waits give up
+  eql::Twiddles tw;
+};
