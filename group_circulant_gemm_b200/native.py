@@ -26,7 +26,7 @@ EXPORTED = (
     "eqlinear_backward_weight_kernel_name", "eqlinear_prepared_weight_bytes",
     "eqlinear_prepare_weights", "eqlinear_forward", "eqlinear_backward_input",
     "eqlinear_backward_weight_workspace_bytes", "eqlinear_backward_weight",
-    "eqlinear_get_status",
+    "eqlinear_get_status", "eqlinear_backward_weight_noalloc",
 )
 
 
@@ -58,6 +58,7 @@ def _load() -> ctypes.CDLL:
         "eqlinear_backward_weight_workspace_bytes": ([vp, i64], sz),
         "eqlinear_backward_weight": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
         "eqlinear_get_status": ([vp, vp], i32),
+        "eqlinear_backward_weight_noalloc": ([vp, vp, vp, i64, vp, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -150,6 +151,13 @@ def eqlinear_backward_weight(plan: int, X, dY, N: int, dW, dbias, workspace,
     _check(_lib.eqlinear_backward_weight(plan, _ptr(X), _ptr(dY), N, _ptr(dW), _ptr(dbias),
                                          _ptr(workspace), workspace_bytes, _stream(stream)),
            "eqlinear_backward_weight")
+
+
+def eqlinear_backward_weight_noalloc(plan: int, X, dY, N: int, dW, dbias, stream=None) -> None:
+    """dW/dbias with the library's own built-in scratch (no workspace argument)."""
+    _check(_lib.eqlinear_backward_weight_noalloc(plan, _ptr(X), _ptr(dY), N, _ptr(dW),
+                                                 _ptr(dbias), _stream(stream)),
+           "eqlinear_backward_weight_noalloc")
 
 
 def eqlinear_get_status(plan: int, stream=None) -> int:

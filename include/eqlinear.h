@@ -168,6 +168,34 @@ EQL_API eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t plan, const v
                                            size_t workspace_bytes, void* stream);
 
 /*
+ * Weight gradient for callers that cannot allocate device memory.  The page
+ * describing the layer has no counterpart to this call; it exists for users of
+ * this library whose device memory is all owned by another allocator or fixed
+ * at start-up, or who must not call cudaMalloc/cudaFree (those calls can
+ * synchronise the whole device) on a latency-critical path.
+ *
+ * Computes exactly what eqlinear_backward_weight computes (same arguments minus
+ * the workspace), but keeps the FP32 partial spectra of the split reduction in a
+ * scratch array that the library reserves statically: 16 MiB (4,194,304 floats)
+ * per GPU on which the library is loaded, held until the process exits.
+ *   - Size limit: one row split needs T*C*D + D floats; plans above 4,194,304
+ *     floats are rejected with EQL_ERR_WORKSPACE before anything is launched.
+ *     When the usual number of splits does not fit, fewer splits are used, so
+ *     results can differ from eqlinear_backward_weight in rounding only.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on each device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a GPU shares the one scratch array and leaves its contents
+ *     behind; each call writes every scratch element before reading it, so no
+ *     clearing is needed, but calls whose executions overlap on the GPU (other
+ *     streams, other plans, other host threads) race on it: serialise them.
+ */
+EQL_API eqlinear_status_t eqlinear_backward_weight_noalloc(eqlinear_plan_t plan, const void* X,
+                                                           const void* dY, int64_t N, void* dW,
+                                                           void* dbias, void* stream);
+
+/*
  * Synchronise `stream`, then read and clear the plan's device status word.
  * Returns EQL_OK, EQL_ERR_TIMEOUT if a kernel's bounded wait gave up since the
  * last call, or EQL_ERR_CUDA if the stream reports an error.
