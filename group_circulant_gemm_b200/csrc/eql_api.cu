@@ -49,18 +49,29 @@ const void* adj_block(const eqlinear_plan_s* p, const void* W_hat) {
   return static_cast<const char*>(W_hat) +
          (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
 }
+bool has_tiles(const eqlinear_plan_s* p) {
+  return eql::tc_tiles_wanted(p->T, to_dt(p->dtype), p->C, p->D);
+}
+// tensor-core operand tiles: forward (Cin = C, Cout = D) then adjoint (Cin = D, Cout = C)
+const void* fwd_tiles(const eqlinear_plan_s* p, const void* W_hat) {
+  return static_cast<const char*>(W_hat) +
+         2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
+}
+const void* adj_tiles(const eqlinear_plan_s* p, const void* W_hat) {
+  return static_cast<const char*>(fwd_tiles(p, W_hat)) + eql::tc_tile_bytes(p->C, p->D);
+}
 
 // Forward-shaped product used by both eqlinear_forward (Cin=C, Cout=D) and
 // eqlinear_backward_input (Cin=D, Cout=C).
-//   own   : planes [P][Cout][Cin]  (tensor-core operand, K-major)
+//   tiles : tensor-core operand tiles of this direction (or null)
 //   other : planes [P][Cin][Cout]  (CUDA-core operand)
 eqlinear_status_t run_forward_like(eqlinear_plan_s* p, const void* X, int64_t N, int Cin,
-                                   int Cout, const void* own, const void* other,
+                                   int Cout, const void* tiles, const void* other,
                                    const void* bias, void* Y, cudaStream_t st) {
-  const bool tc_ok = eql::fwd_tc_supported(p->T, to_dt(p->dtype), N, Cin, Cout);
+  const bool tc_ok = has_tiles(p) && eql::fwd_tc_supported(p->T, to_dt(p->dtype), N, Cin, Cout);
   if (p->kernel == EQL_KERNEL_TCGEN05 && !tc_ok) return EQL_ERR_UNSUPPORTED;
   if (p->kernel != EQL_KERNEL_SIMT && tc_ok)
-    return from_cuda(eql::launch_fwd_tc(p->T, X, N, Cin, Cout, own, bias, Y, p->status,
+    return from_cuda(eql::launch_fwd_tc(p->T, X, N, Cin, Cout, tiles, bias, Y, p->status,
                                         p->num_sms, st));
   return from_cuda(eql::launch_fwd_simt(p->T, to_dt(p->dtype), X, N, Cin, Cout, other, bias, Y,
                                         p->tw, st));
@@ -141,7 +152,7 @@ eqlinear_status_t eqlinear_plan_set_kernel(eqlinear_plan_t p, eqlinear_kernel_t 
 
 const char* eqlinear_forward_kernel_name(eqlinear_plan_t p, int64_t N) {
   if (!p) return "unsupported";
-  const bool tc_ok = eql::fwd_tc_supported(p->T, to_dt(p->dtype), N, p->C, p->D);
+  const bool tc_ok = has_tiles(p) && eql::fwd_tc_supported(p->T, to_dt(p->dtype), N, p->C, p->D);
   if (p->kernel == EQL_KERNEL_TCGEN05) return tc_ok ? "tcgen05" : "unsupported";
   if (p->kernel == EQL_KERNEL_AUTO && tc_ok) return "tcgen05";
   return "simt";
@@ -156,7 +167,9 @@ const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t p, int64_t N) {
 
 size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t p) {
   if (!p) return 0;
-  return 2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
+  size_t bytes = 2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
+  if (has_tiles(p)) bytes += eql::tc_tile_bytes(p->C, p->D) + eql::tc_tile_bytes(p->D, p->C);
+  return bytes;
 }
 
 eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, void* W_hat,
@@ -167,8 +180,14 @@ eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, voi
   if (s != EQL_OK) return s;
   void* fwd = W_hat;
   void* adj = const_cast<void*>(adj_block(p, W_hat));
-  return from_cuda(eql::launch_prepare(p->T, to_dt(p->dtype), W, p->C, p->D, fwd, adj, p->tw,
-                                       (cudaStream_t)stream));
+  cudaStream_t st = (cudaStream_t)stream;
+  s = from_cuda(eql::launch_prepare(p->T, to_dt(p->dtype), W, p->C, p->D, fwd, adj, p->tw, st));
+  if (s != EQL_OK || !has_tiles(p)) return s;
+  s = from_cuda(eql::launch_tile_weights(fwd, p->C, p->D, const_cast<void*>(fwd_tiles(p, W_hat)),
+                                         st));
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_tile_weights(adj, p->D, p->C,
+                                            const_cast<void*>(adj_tiles(p, W_hat)), st));
 }
 
 eqlinear_status_t eqlinear_forward(eqlinear_plan_t p, const void* X, int64_t N,
@@ -180,7 +199,7 @@ eqlinear_status_t eqlinear_forward(eqlinear_plan_t p, const void* X, int64_t N,
     return EQL_ERR_ALIGNMENT;
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
-  return run_forward_like(p, X, N, p->C, p->D, fwd_block(p, W_hat), adj_block(p, W_hat), bias,
+  return run_forward_like(p, X, N, p->C, p->D, fwd_tiles(p, W_hat), adj_block(p, W_hat), bias,
                           Y, (cudaStream_t)stream);
 }
 
@@ -193,8 +212,8 @@ eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
   // dX is the forward-shaped product with the adjoint weights: input width D,
-  // output width C; "own" planes are the adjoint block [P][C][D].
-  return run_forward_like(p, dY, N, p->D, p->C, adj_block(p, W_hat), fwd_block(p, W_hat),
+  // output width C; the CUDA-core path reads the forward block [P][D][C].
+  return run_forward_like(p, dY, N, p->D, p->C, adj_tiles(p, W_hat), fwd_block(p, W_hat),
                           nullptr, dX, (cudaStream_t)stream);
 }
 

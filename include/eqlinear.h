@@ -115,6 +115,10 @@ EQL_API const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t plan, i
  * (even T); Re and Im of each complex frequency k = 1..n_cplx; then -Im of each
  * complex frequency.  Forward planes hold conj(DFT(W)) (the correlation form of
  * the convolution theorem), adjoint planes hold DFT(W) transposed, used for dX.
+ * For T = 4 FP16 plans with C and D multiples of 8 two more blocks follow: the
+ * forward and adjoint planes re-arranged as the tensor-core kernel's operand
+ * tiles (one contiguous blob per 128 out-channels x 16 in-channels, in the
+ * kernel's swizzled shared-memory order), so each pipeline stage is one copy.
  */
 EQL_API size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t plan);
 

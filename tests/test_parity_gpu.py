@@ -132,7 +132,7 @@ def test_edge_shapes_all_ops(T, N, C, D, dtype):
 
 TC_EDGE = [
     # N, C, D : ragged rows, channels and out-channels for the tcgen05 p4 path
-    (1, 8, 8), (127, 24, 136), (129, 40, 200), (300, 200, 8), (513, 64, 384), (260, 328, 72),
+    (1, 16, 16), (127, 48, 144), (129, 80, 208), (300, 208, 16), (513, 64, 384), (260, 336, 80),
 ]
 
 
