@@ -41,7 +41,7 @@ constexpr int kT = 4;
 constexpr int BM = 128;          // rows per tile = MMA M
 constexpr int BD = 128;          // out-channels per tile
 constexpr int BK = 32;           // in-channels per pipeline stage = two MMA K steps
-constexpr int X_ST = 3;          // X ring: raw tile in, transformed operand planes out (in place)
+constexpr int X_ST = 4;          // X ring: raw tile in, transformed operand planes out (in place)
 constexpr int W_ST = 3;          // weight-tile ring (L2-resident source)
 constexpr int kPlanes = 4;       // A0, A2, Br, Bi
 constexpr int kThreads = 640;
