@@ -1,6 +1,7 @@
 // C ABI of the EQ-Linear library: plans, argument checks, kernel dispatch.
 // The operations and their definitions are documented in include/eqlinear.h.
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 
@@ -72,7 +73,7 @@ eqlinear_status_t run_forward_like(eqlinear_plan_s* p, const void* X, int64_t N,
   if (p->kernel == EQL_KERNEL_TCGEN05 && !tc_ok) return EQL_ERR_UNSUPPORTED;
   if (p->kernel != EQL_KERNEL_SIMT && tc_ok)
     return from_cuda(eql::launch_fwd_tc(p->T, X, N, Cin, Cout, tiles, bias, Y, p->status,
-                                        p->num_sms, st));
+                                        p->num_sms, p->debug_drop_w_stage, st));
   return from_cuda(eql::launch_fwd_simt(p->T, to_dt(p->dtype), X, N, Cin, Cout, other, bias, Y,
                                         p->tw, st));
 }
@@ -122,6 +123,12 @@ eqlinear_status_t eqlinear_plan_create(int T, int C, int D, eqlinear_dtype_t dty
   p->kernel = EQL_KERNEL_AUTO;
   p->device = dev;
   p->num_sms = sms;
+  // Test hook for the failure-detection path: with EQL_DEBUG_DROP_W_STAGE=k in the
+  // environment at plan creation, the tensor-core kernel's CTA 0 skips weight
+  // stage k; its bounded waits then expire and eqlinear_get_status reports
+  // EQL_ERR_TIMEOUT.  Unset (the normal case) it is off.
+  p->debug_drop_w_stage = -1;
+  if (const char* e = std::getenv("EQL_DEBUG_DROP_W_STAGE")) p->debug_drop_w_stage = std::atoi(e);
   make_twiddles(T, &p->tw);
   if (cudaMalloc(&p->status, sizeof(int)) != cudaSuccess) {
     delete p;

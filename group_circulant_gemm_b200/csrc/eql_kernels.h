@@ -48,8 +48,10 @@ cudaError_t launch_tile_weights(const void* planes /* [P][Cout][Cin] */, int Cin
                                 void* tiles, cudaStream_t st);
 // Returns cudaErrorNotSupported when the shape does not fit the kernel.
 bool fwd_tc_supported(int T, DType dt, int64_t N, int Cin, int Cout);
+// drop_w_stage >= 0 is a test-only fault: CTA 0 never issues that weight stage,
+// so its bounded waits expire and the kernel reports a timeout.
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
-                          int num_sms, cudaStream_t st);
+                          int num_sms, int drop_w_stage, cudaStream_t st);
 
 }  // namespace eql

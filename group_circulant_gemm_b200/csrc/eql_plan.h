@@ -11,5 +11,6 @@ struct eqlinear_plan_s {
   int device;
   int num_sms;
   int* status;  // device word written by kernels whose bounded waits give up
+  int debug_drop_w_stage;  // test-only fault injection (EQL_DEBUG_DROP_W_STAGE), -1 = off
   eql::Twiddles tw;
 };

@@ -236,6 +236,7 @@ struct TileInfo {
   int n_dt;       // d tiles
   int num_tiles;  // row tiles x d tiles
   int k_stages;   // ceil(Cin / BK)
+  int drop_w;     // fault injection for tests: CTA 0 never issues weight stage drop_w (-1: off)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -298,6 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = it % depth;
           const uint32_t ph = (it / depth) & 1;
           if (!(ok = wait_bounded(&empty[s], ph ^ 1, bars, status))) break;
+          if (!is_raw && blockIdx.x == 0 && (int)it == ti.drop_w) continue;  // injected fault
           if (is_raw) {
             mbar_expect_tx(&full[s], X_STAGE_BYTES);
             // 3-D view of X: (64 halves, 128-byte chunk of the row, row); a stage is
@@ -581,7 +583,7 @@ cudaError_t launch_tile_weights(const void* planes, int Cin, int Cout, void* til
 
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
-                          int num_sms, cudaStream_t st) {
+                          int num_sms, int drop_w_stage, cudaStream_t st) {
   if (!fwd_tc_supported(T, DType::F16, N, Cin, Cout)) return cudaErrorNotSupported;
   if (!Wtiles) return cudaErrorNotSupported;
   auto encode = encode_fn();
@@ -606,6 +608,7 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
   if (n_rt * ti.n_dt > 0x7fffffffLL) return cudaErrorInvalidValue;
   ti.num_tiles = (int)(n_rt * ti.n_dt);
   ti.k_stages = (Cin + BK - 1) / BK;
+  ti.drop_w = drop_w_stage;
 
   static bool attr_set = false;
   if (!attr_set) {
