@@ -66,6 +66,26 @@ def layer_bytes(w) -> float:
     return es * (w.N * w.C * w.T + w.N * w.D * w.T + planes * w.C * w.D + w.D)
 
 
+# DRAM traffic per forward launch (dram__bytes_read.sum + dram__bytes_write.sum),
+# from the ncu captures summarised in profiles/, valid only for the kernel source
+# they were taken on (SHA-256 prefix of csrc/eql_tc_fwd.cu); any other source
+# reports null.
+NCU_TRAFFIC = {
+    "86ba56eb36e4696e": {"p4_vitb_mlp_f16": 64.73e6, "c8_1024_f16": 34.20e6},
+}
+
+
+def kernel_traffic(workload: str):
+    import hashlib
+    path = os.path.join(ROOT, "group_circulant_gemm_b200", "csrc", "eql_tc_fwd.cu")
+    try:
+        with open(path, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return NCU_TRAFFIC.get(h, {}).get(workload)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -302,7 +322,7 @@ def run_ours(args, workload):
             peak = peaks["bf16_tflops"]
             achieved = flops_per_launch / (mean_launch_ms / 1e3) / 1e12
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None,
+                    "frac": achieved / peak, "traffic": kernel_traffic(workload),
                     "peak_source": f"{peak_src} dense bf16 burst (fp16 runs at the same rate)"}
         else:
             # CUDA-core FP32 FMA peak: 148 SMs x 128 FMA/clk x 2 FLOP x max SM clock

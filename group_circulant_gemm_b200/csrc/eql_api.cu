@@ -59,7 +59,7 @@ const void* fwd_tiles(const eqlinear_plan_s* p, const void* W_hat) {
          2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
 }
 const void* adj_tiles(const eqlinear_plan_s* p, const void* W_hat) {
-  return static_cast<const char*>(fwd_tiles(p, W_hat)) + eql::tc_tile_bytes(p->C, p->D);
+  return static_cast<const char*>(fwd_tiles(p, W_hat)) + eql::tc_tile_bytes(p->T, p->C, p->D);
 }
 
 // Forward-shaped product used by both eqlinear_forward (Cin=C, Cout=D) and
@@ -175,7 +175,7 @@ const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t p, int64_t N) {
 size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t p) {
   if (!p) return 0;
   size_t bytes = 2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
-  if (has_tiles(p)) bytes += eql::tc_tile_bytes(p->C, p->D) + eql::tc_tile_bytes(p->D, p->C);
+  if (has_tiles(p)) bytes += eql::tc_tile_bytes(p->T, p->C, p->D) + eql::tc_tile_bytes(p->T, p->D, p->C);
   return bytes;
 }
 
@@ -190,10 +190,10 @@ eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, voi
   cudaStream_t st = (cudaStream_t)stream;
   s = from_cuda(eql::launch_prepare(p->T, to_dt(p->dtype), W, p->C, p->D, fwd, adj, p->tw, st));
   if (s != EQL_OK || !has_tiles(p)) return s;
-  s = from_cuda(eql::launch_tile_weights(fwd, p->C, p->D, const_cast<void*>(fwd_tiles(p, W_hat)),
+  s = from_cuda(eql::launch_tile_weights(p->T, fwd, p->C, p->D, const_cast<void*>(fwd_tiles(p, W_hat)),
                                          st));
   if (s != EQL_OK) return s;
-  return from_cuda(eql::launch_tile_weights(adj, p->D, p->C,
+  return from_cuda(eql::launch_tile_weights(p->T, adj, p->D, p->C,
                                             const_cast<void*>(adj_tiles(p, W_hat)), st));
 }
 

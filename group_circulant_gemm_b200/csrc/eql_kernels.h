@@ -38,14 +38,15 @@ cudaError_t launch_wgrad_finalize(int T, DType dt, const float* part, const floa
                                   int splits, int C, int D, void* dW, void* dbias,
                                   const Twiddles& tw, cudaStream_t st);
 
-// tcgen05/TMEM tensor-core forward (FP16 in, FP32 accumulate, FP16 out).
+// tcgen05/TMEM tensor-core forward for T = 4 and T = 8 (FP16 in, FP32
+// accumulate, FP16 out).
 // The kernel reads its weights as operand tiles pre-arranged in its own
 // shared-memory image (one contiguous blob per out-channel tile and K stage),
 // written once by launch_tile_weights from a block of prepared planes.
 bool tc_tiles_wanted(int T, DType dt, int C, int D);
-size_t tc_tile_bytes(int Cin, int Cout);
-cudaError_t launch_tile_weights(const void* planes /* [P][Cout][Cin] */, int Cin, int Cout,
-                                void* tiles, cudaStream_t st);
+size_t tc_tile_bytes(int T, int Cin, int Cout);
+cudaError_t launch_tile_weights(int T, const void* planes /* [P][Cout][Cin] */, int Cin,
+                                int Cout, void* tiles, cudaStream_t st);
 // Returns cudaErrorNotSupported when the shape does not fit the kernel.
 bool fwd_tc_supported(int T, DType dt, int64_t N, int Cin, int Cout);
 // drop_w_stage >= 0 is a test-only fault: CTA 0 never issues that weight stage,

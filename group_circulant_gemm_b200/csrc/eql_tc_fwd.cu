@@ -1,82 +1,108 @@
-// tcgen05/TMEM tensor-core forward of the p4 (T = 4) EQ-Linear layer, FP16 in,
-// FP32 accumulate, FP16 out, for sm_100a.
+// tcgen05/TMEM tensor-core forward of the cyclic-group EQ-Linear layer for
+// T = 4 (the p4 rotation group) and T = 8, FP16 in, FP32 accumulate, FP16 out,
+// for sm_100a.
 //
-// What it computes (Flash EQ-Linear summary, "Algorithmic approach" and
-// "Specialisation for p4"): per row n and input channel c the group DFT
-//   X0 = x0+x1+x2+x3,  X2 = x0-x1+x2-x3,  Xr = x0-x2,  Xi = x3-x1
-// (adds only), six real GEMMs against the prepared weight planes
-//   Y0 = X0 A0^T,  Y2 = X2 A2^T,
-//   Y1r = Xr Br^T - Xi Bi^T,  Y1i = Xr Bi^T + Xi Br^T
-// and the inverse DFT with the dyadic factors 1/4 and 1/2, plus bias:
-//   y0 = (Y0+Y2)/4 + Y1r/2,  y1 = (Y0-Y2)/4 - Y1i/2,
-//   y2 = (Y0+Y2)/4 - Y1r/2,  y3 = (Y0-Y2)/4 + Y1i/2.
+// What it computes (Flash EQ-Linear summary, "Algorithmic approach" items 1-3
+// and "Specialisation for p4"): per row n and input channel c the real DFT of
+// the group vector x[0..T) (FP32, one rounding to FP16), one real GEMM per real
+// frequency and four per complex frequency against the prepared weight planes
+// (conjugated spectrum of W), and the inverse DFT plus bias:
+//   real k:     Y_k  = X_k A_k^T
+//   complex k:  Y_kr = Xr_k Br_k^T - Xi_k Bi_k^T,  Y_ki = Xr_k Bi_k^T + Xi_k Br_k^T
+//   y[s] = (Y_0 + (-1)^s Y_{T/2}) / T + (2/T) sum_k (Y_kr cos(2 pi k s/T) - Y_ki sin(2 pi k s/T))
+// For T = 4 the transforms are adds only (X0 = x0+x1+x2+x3, X2 = x0-x1+x2-x3,
+// Xr = x0-x2, Xi = x3-x1) and the inverse uses the factors 1/4 and 1/2; for
+// T = 8 a radix-2 split leaves one non-dyadic twiddle, sqrt(2)/2.
 //
-// Design (one persistent CTA per SM, tile = 128 rows x 128 out-channels, K
-// stages of 16 input channels = one MMA K step):
-//   warp 0      TMA producer: the raw X tile of a stage (128 rows x 16 channels
-//               x 4, one 128B-swizzled box) into the X ring.
-//   warp 2      weight producer: one bulk copy per stage of a 16 KB blob that
-//               prepare_weights pre-arranged in the operand layout (A0, A2, Br, Bi).
-//   warp 1      TMEM allocator; lane 0 issues the five tcgen05.mma of a stage:
-//               N = 128 for Y0 and Y2, N = 256 for Xr [Br|Bi], and two N = 128
-//               for -Xi Bi (negate-A bit) and Xi Br.
+// Design (one persistent CTA per SM; tile = 128 rows x BD out-channels; K stage
+// = BK input channels, whose raw X tile is always 128 rows x 256 B = 32 KB):
+//   warp 0      TMA producer: the raw X tile of a stage, one 3-D box
+//               (64 halves x 2 row chunks x 128 rows, 128B-swizzled).
+//   warp 2      weight producer: one bulk copy per stage of a blob that
+//               prepare_weights pre-arranged in the MMA operand layout.
+//   warp 1      TMEM allocator; lane 0 issues the MMAs of each K step:
+//               N = BD for each real frequency, N = 2 BD for Xr_k [Br_k|Bi_k],
+//               and N = BD for -Xi_k Bi_k (negate-A bit) and Xi_k Br_k.
 //   warps 12-19 transform: group DFT in FP32, one rounding to FP16, written as
-//               four K-major 32B-swizzled operand planes over the raw tile of the
-//               same slot (the planes take exactly the raw tile's 16 KB).
-//   warps 4-11  epilogue: tcgen05.ld of the four accumulators, inverse DFT, bias,
+//               T K-major swizzled operand planes over the raw tile of the same
+//               slot (the planes take exactly the raw tile's 32 KB).
+//   warps 4-11  epilogue: tcgen05.ld of the T accumulators, inverse DFT, bias,
 //               FP16 pack, 16-byte global stores.
-// Accumulators in TMEM: Y0 at columns [0,128), Y2 [128,256), Y1r [256,384),
-// Y1i [384,512).  Every mbarrier wait is bounded (about 2 s of %globaltimer); on
-// expiry the CTA sets a shared abort flag and the plan's status word, drains
-// what it issued and returns, so a stuck pipeline never hangs the GPU.
+// TMEM (T * BD = 512 columns): real frequency 0 at [0, BD), real frequency T/2
+// at [BD, 2 BD), complex frequency k at [2 BD k, 2 BD k + 2 BD) as (re | im).
+// Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the CTA
+// sets a shared abort flag and the plan's status word, drains what it issued and
+// returns, so a stuck pipeline never hangs the GPU.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <type_traits>
 
 #include "eql_kernels.h"
 
 namespace eql {
 namespace {
 
-constexpr int kT = 4;
 constexpr int BM = 128;          // rows per tile = MMA M
-constexpr int BD = 128;          // out-channels per tile
-constexpr int BK = 32;           // in-channels per pipeline stage = two MMA K steps
 constexpr int X_ST = 4;          // X ring: raw tile in, transformed operand planes out (in place)
-constexpr int W_ST = 3;          // weight-tile ring (L2-resident source)
-constexpr int kPlanes = 4;       // A0, A2, Br, Bi
+constexpr uint32_t X_STAGE_BYTES = BM * 256;   // 128 rows x 256 B raw X per stage
 constexpr int kThreads = 640;
 constexpr int kEpiWarp0 = 4;     // warps 4..11: two per TMEM lane quarter
 constexpr int kEpiWarps = 8;
 constexpr int kXfWarp0 = 12;     // warps 12..19
 constexpr int kXfWarps = 8;
-constexpr uint32_t kTmemCols = 4 * BD;  // 512
+constexpr uint32_t kTmemCols = 512;
 
-// One 32 KB TMA op per stage for X and one 32 KB bulk op for the weights: the
-// per-SM load rate grows with the bytes each operation carries.
-constexpr uint32_t X_STAGE_BYTES = BM * BK * kT * 2;      // 128 rows x 32 channels x 4 x 2 B
-constexpr uint32_t PLANE_BYTES = BM * BK * 2;             // 128 rows x 64 B
-static_assert(4 * PLANE_BYTES == X_STAGE_BYTES, "the four planes replace the raw tile in place");
-constexpr uint32_t WREG_BYTES = BD * BK * 2;              // BD rows x 64 B
-constexpr uint32_t W_STAGE_BYTES = kPlanes * WREG_BYTES;
-constexpr uint32_t OFF_X = 0;
-constexpr uint32_t OFF_W = OFF_X + X_ST * X_STAGE_BYTES;
-constexpr uint32_t OFF_BAR = OFF_W + W_ST * W_STAGE_BYTES;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;     // barriers + alignment slack
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// Per-group shape of the pipeline.
+template <int T>
+struct Cfg;
+template <>
+struct Cfg<4> {
+  static constexpr int BD = 128;        // out-channels per tile
+  static constexpr int BK = 32;         // in-channels per stage (two MMA K steps)
+  static constexpr int W_ST = 3;        // weight-tile ring depth
+};
+template <>
+struct Cfg<8> {
+  static constexpr int BD = 64;
+  static constexpr int BK = 16;         // one MMA K step
+  static constexpr int W_ST = 6;
+};
+template <int T>
+struct Shape : Cfg<T> {
+  using Cfg<T>::BD;
+  using Cfg<T>::BK;
+  using Cfg<T>::W_ST;
+  static constexpr int NPL = T;                           // operand planes = weight regions
+  static constexpr int NC = T / 2 - 1;                    // complex frequencies
+  static constexpr int ROWB = BK * 2;                     // bytes per operand row
+  static constexpr int KSTEPS = BK / 16;
+  static constexpr uint32_t PLANE_BYTES = BM * ROWB;
+  static constexpr uint32_t WREG_BYTES = BD * ROWB;
+  static constexpr uint32_t W_STAGE_BYTES = NPL * WREG_BYTES;
+  static constexpr uint32_t OFF_X = 0;
+  static constexpr uint32_t OFF_W = OFF_X + X_ST * X_STAGE_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_W + W_ST * W_STAGE_BYTES;
+  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers + alignment slack
+  static_assert(NPL * PLANE_BYTES == X_STAGE_BYTES, "planes replace the raw tile in place");
+  static_assert(BK * T * 2 == 256, "a raw stage row is two 128-byte chunks");
+  static_assert(T * BD == (int)kTmemCols, "accumulators fill TMEM");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
 
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 // status word codes
 constexpr int kErrTimeout = 1;
 
+template <int T>
 struct Bars {
   uint64_t x_full[X_ST], x_read[X_ST], x_ready[X_ST], x_empty[X_ST];
-  uint64_t w_full[W_ST], w_empty[W_ST];
+  uint64_t w_full[Shape<T>::W_ST], w_empty[Shape<T>::W_ST];
   uint64_t acc_full, acc_empty, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Bars) <= 512, "barrier block");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -123,14 +149,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* b, uint32_t parity
   return ok != 0;
 }
 // Bounded wait: false if the CTA aborted or the wait timed out (then aborts it).
-__device__ __noinline__ bool wait_bounded(uint64_t* b, uint32_t parity, Bars* bars, int* status) {
+__device__ __noinline__ bool wait_bounded(uint64_t* b, uint32_t parity, int* abort_flag, int* status) {
   if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = gtimer();
   while (true) {
     if (mbar_try_wait_sleep(b, parity, 200000u)) return true;
-    if (*(volatile int*)&bars->abort_flag) return false;
+    if (*(volatile int*)abort_flag) return false;
     if (gtimer() - t0 > kTimeoutNs) {
-      *(volatile int*)&bars->abort_flag = 1;
+      *(volatile int*)abort_flag = 1;
       atomicExch(status, kErrTimeout);
       return false;
     }
@@ -138,8 +164,8 @@ __device__ __noinline__ bool wait_bounded(uint64_t* b, uint32_t parity, Bars* ba
 }
 // Warp-uniform bounded wait: every lane polls, then the warp agrees, so a lane
 // that gave up cannot leave the others waiting at a warp-synchronous point.
-__device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, Bars* bars, int* status) {
-  const bool ok = wait_bounded(b, parity, bars, status);
+__device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, int* abort_flag, int* status) {
+  const bool ok = wait_bounded(b, parity, abort_flag, status);
   return __all_sync(0xffffffffu, ok);
 }
 // Bounded wait used while draining after an abort (ignores the abort flag).
@@ -168,17 +194,19 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// K-major, 64-byte-swizzled operand tile: rows of 64 B (32 fp16 of K), 8-row
-// groups 512 B apart (SBO), descriptor version 1 (sm_100), layout type 4
-// (SWIZZLE_64B: 16-byte chunk index ^= (row / 2) % 4).  The second MMA K step of
-// a stage starts 32 B into the rows.
-__device__ __forceinline__ uint64_t desc_kmajor_sw64(uint32_t saddr) {
+// K-major swizzled operand tile descriptor: rows of `row_bytes` (32 or 64 B of
+// K), 8-row groups 8 * row_bytes apart (SBO), descriptor version 1 (sm_100);
+// layout type 4 = SWIZZLE_64B (16-byte piece ^= (row / 2) % 4), 6 = SWIZZLE_32B
+// (piece ^= (row / 4) % 2).  A later K step inside a row starts 32 B further.
+template <int kRowBytes>
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) {
+  static_assert(kRowBytes == 32 || kRowBytes == 64, "operand row width");
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1u << 16;              // leading byte offset (unused when swizzled)
-  d |= (uint64_t)(512u >> 4) << 32;     // stride byte offset: 8 rows x 64 B
-  d |= (uint64_t)1u << 46;              // descriptor version for sm_100
-  d |= (uint64_t)4u << 61;              // SWIZZLE_64B
+  d |= (uint64_t)1u << 16;                          // leading byte offset (unused)
+  d |= (uint64_t)((8u * kRowBytes) >> 4) << 32;     // stride byte offset
+  d |= (uint64_t)1u << 46;                          // descriptor version for sm_100
+  d |= (uint64_t)(kRowBytes == 64 ? 4u : 6u) << 61; // SWIZZLE_64B / SWIZZLE_32B
   return d;
 }
 // Instruction descriptor, kind::f16: A = B = F16, D = F32, both K-major;
@@ -213,6 +241,10 @@ __device__ __forceinline__ void tc_fence_after() {
 // 16 TMEM lanes x 256 bits: thread t gets lanes (t/4) and (t/4 + 8) of the
 // addressed 16-lane group, columns 2*(t%4) and 2*(t%4)+1 -> regs
 // {lane t/4: col, col+1, lane t/4+8: col, col+1}.
+#define EQL_TMEM_LD_16x256(taddr, r)                                                   \
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0, %1, %2, %3}, [%4];"         \
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])                         \
+               : "r"(taddr))
 // The .x2 form repeats the pattern for the next 8 columns in regs 4..7.
 #define EQL_TMEM_LD_16x256_X2(taddr, r)                                                    \
   asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"    \
@@ -232,6 +264,7 @@ __device__ __forceinline__ float2 unpack_h2(uint32_t u) {
   return __half22float2(h);
 }
 
+
 struct TileInfo {
   int n_dt;       // d tiles
   int num_tiles;  // row tiles x d tiles
@@ -239,27 +272,195 @@ struct TileInfo {
   int drop_w;     // fault injection for tests: CTA 0 never issues weight stage drop_w (-1: off)
 };
 
+// ---------------------------------------------------------------------------
+// Transform: the raw stage is [row][128-byte chunk c][128 B], every 128-byte
+// line L = 2r + c swizzled by (L % 8).  A thread reads eight 16-byte pieces and,
+// once every transform warp holds its pieces, writes its share of the planes.
+// Lane mapping: an 8-lane phase covers 4 rows x both chunks, so its swizzled
+// reads and writes hit 8 distinct bank groups.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 f2(uint32_t u) { return unpack_h2(u); }
+
+// T = 4: a chunk holds 16 channels (2 per piece); a unit is one row x 8 channels
+// (half hq of chunk c), two units per thread.
+template <int T>
+__device__ __forceinline__ void xf_read(const uint8_t* slot, int xt, uint4 (&v)[8]) {
+  if constexpr (T == 4) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int unit = xt + 256 * u;
+      const int c = unit & 1, r = (unit >> 1) & (BM - 1), hq = unit >> 8;
+      const int line = 2 * r + c;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int j = hq * 4 + i;
+        v[4 * u + i] = *reinterpret_cast<const uint4*>(slot + line * 128 + ((j ^ (line & 7)) << 4));
+      }
+    }
+  } else {
+    // T = 8: a chunk holds 8 channels (1 per piece); one unit = one line per thread
+    const int c = xt & 1, r = (xt >> 1) & (BM - 1);
+    const int line = 2 * r + c;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      v[j] = *reinterpret_cast<const uint4*>(slot + line * 128 + ((j ^ (line & 7)) << 4));
+  }
+}
+
+template <int T>
+__device__ __forceinline__ void xf_write(uint8_t* slot, int xt, const uint4 (&v)[8]) {
+  using S = Shape<T>;
+  if constexpr (T == 4) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int unit = xt + 256 * u;
+      const int c = unit & 1, r = (unit >> 1) & (BM - 1), hq = unit >> 8;
+      const int q = 2 * c + hq;
+      // piece i holds channels 2i (.x = x0,x1  .y = x2,x3) and 2i+1 (.z, .w)
+      uint32_t o0[4], o2[4], orr[4], oi[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float f0[2], fh[2], fr[2], fi[2];
+        const uint32_t w4[4] = {v[4 * u + i].x, v[4 * u + i].y, v[4 * u + i].z, v[4 * u + i].w};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const float2 lo = f2(w4[2 * hh]), hi = f2(w4[2 * hh + 1]);
+          const float x0 = lo.x, x1 = lo.y, x2 = hi.x, x3 = hi.y;
+          const float a = x0 + x2, b = x1 + x3;
+          f0[hh] = a + b;
+          fh[hh] = a - b;
+          fr[hh] = x0 - x2;
+          fi[hh] = x3 - x1;
+        }
+        o0[i] = pack_h2(f0[0], f0[1]);
+        o2[i] = pack_h2(fh[0], fh[1]);
+        orr[i] = pack_h2(fr[0], fr[1]);
+        oi[i] = pack_h2(fi[0], fi[1]);
+      }
+      // K-major 64 B rows: 16-byte piece q at (q ^ ((r / 2) % 4))
+      const uint32_t off = r * 64 + ((q ^ ((r >> 1) & 3)) << 4);
+      *reinterpret_cast<uint4*>(slot + 0 * S::PLANE_BYTES + off) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+      *reinterpret_cast<uint4*>(slot + 1 * S::PLANE_BYTES + off) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+      *reinterpret_cast<uint4*>(slot + 2 * S::PLANE_BYTES + off) =
+          make_uint4(orr[0], orr[1], orr[2], orr[3]);
+      *reinterpret_cast<uint4*>(slot + 3 * S::PLANE_BYTES + off) = make_uint4(oi[0], oi[1], oi[2], oi[3]);
+    }
+  } else {
+    // T = 8: piece j = channel j of the chunk, x0..x7 in .x .y .z .w (pairs).
+    // Radix-2: a_t = x_t + x_{t+4}, b_t = x_t - x_{t+4};
+    //   X0 = a0+a1+a2+a3, X4 = a0-a1+a2-a3, X2 = (a0-a2) + i (a3-a1),
+    //   X1 = b0 + h(b1-b3) + i(-b2 - h(b1+b3)),  X3 = b0 - h(b1-b3) + i(b2 - h(b1+b3)),
+    // h = sqrt(2)/2; plane order X0, X4, Re X1, Im X1, Re X2, Im X2, Re X3, Im X3.
+    const float h = 0.70710678118654752f;
+    const int c = xt & 1, r = (xt >> 1) & (BM - 1);
+    uint32_t o[8][4];  // [plane][channel pair]
+#pragma unroll
+    for (int pr = 0; pr < 4; ++pr) {
+      float val[8][2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint4 w = v[2 * pr + hh];
+        const float2 p01 = f2(w.x), p23 = f2(w.y), p45 = f2(w.z), p67 = f2(w.w);
+        const float a0 = p01.x + p45.x, a1 = p01.y + p45.y, a2 = p23.x + p67.x, a3 = p23.y + p67.y;
+        const float b0 = p01.x - p45.x, b1 = p01.y - p45.y, b2 = p23.x - p67.x, b3 = p23.y - p67.y;
+        const float s13 = h * (b1 - b3), t13 = h * (b1 + b3);
+        val[0][hh] = (a0 + a2) + (a1 + a3);
+        val[1][hh] = (a0 + a2) - (a1 + a3);
+        val[2][hh] = b0 + s13;
+        val[3][hh] = -b2 - t13;
+        val[4][hh] = a0 - a2;
+        val[5][hh] = a3 - a1;
+        val[6][hh] = b0 - s13;
+        val[7][hh] = b2 - t13;
+      }
+#pragma unroll
+      for (int p = 0; p < 8; ++p) o[p][pr] = pack_h2(val[p][0], val[p][1]);
+    }
+    // K-major 32 B rows: 16-byte piece c at (c ^ ((r / 4) % 2))
+    const uint32_t off = r * 32 + ((c ^ ((r >> 2) & 1)) << 4);
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+      *reinterpret_cast<uint4*>(slot + p * S::PLANE_BYTES + off) =
+          make_uint4(o[p][0], o[p][1], o[p][2], o[p][3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue of one 8-column group for the two rows (ra, rb) and the out-channel
+// pair (d, d+1) this lane owns; acc[plane][k]: k = 2*rr + hh (row rr, channel hh).
+// ---------------------------------------------------------------------------
+template <int T>
+__device__ __forceinline__ void epi_store(const uint32_t (&acc)[T][4], int64_t ra, int64_t rb,
+                                          int d, float2 bb, __half* __restrict__ Y, int64_t ldy,
+                                          int64_t N) {
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int64_t row = rr ? rb : ra;
+    if (row >= N) continue;
+    if constexpr (T == 4) {
+      uint32_t packed[4];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int k = 2 * rr + hh;
+        const float y0 = __uint_as_float(acc[0][k]), y2 = __uint_as_float(acc[1][k]);
+        const float yr = __uint_as_float(acc[2][k]), yi = __uint_as_float(acc[3][k]);
+        const float b = hh ? bb.y : bb.x;
+        const float e = (y0 + y2) * 0.25f, o = (y0 - y2) * 0.25f;
+        const float re = yr * 0.5f, im = yi * 0.5f;
+        packed[2 * hh + 0] = pack_h2(e + re + b, o - im + b);
+        packed[2 * hh + 1] = pack_h2(e - re + b, o + im + b);
+      }
+      *reinterpret_cast<uint4*>(Y + row * ldy + (int64_t)d * T) =
+          make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    } else {
+      const float h4 = 0.70710678118654752f * 0.25f;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int k = 2 * rr + hh;
+        float Yv[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) Yv[p] = __uint_as_float(acc[p][k]);
+        const float b = hh ? bb.y : bb.x;
+        // y_s = A_s + B_s, y_{s+4} = A_s - B_s (A: frequencies 0, 2, 4; B: 1, 3)
+        const float E = (Yv[0] + Yv[1]) * 0.125f, O = (Yv[0] - Yv[1]) * 0.125f;
+        const float A0 = E + 0.25f * Yv[4], A2 = E - 0.25f * Yv[4];
+        const float A1 = O - 0.25f * Yv[5], A3 = O + 0.25f * Yv[5];
+        const float B0 = 0.25f * (Yv[2] + Yv[6]);
+        const float B1 = h4 * (Yv[2] - Yv[3] - Yv[6] - Yv[7]);
+        const float B2 = 0.25f * (Yv[7] - Yv[3]);
+        const float B3 = h4 * (-Yv[2] - Yv[3] + Yv[6] - Yv[7]);
+        const uint4 out = make_uint4(pack_h2(A0 + B0 + b, A1 + B1 + b), pack_h2(A2 + B2 + b, A3 + B3 + b),
+                                     pack_h2(A0 - B0 + b, A1 - B1 + b), pack_h2(A2 - B2 + b, A3 - B3 + b));
+        *reinterpret_cast<uint4*>(Y + row * ldy + (int64_t)(d + hh) * T) = out;
+      }
+    }
+  }
+}
+
+template <int T>
 __global__ void __launch_bounds__(kThreads, 1)
-    p4_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x,
-                     const uint8_t* __restrict__ wtiles, const __half* __restrict__ bias,
-                     __half* __restrict__ Y, int64_t N, int Cin, int Cout, TileInfo ti,
-                     int* status) {
+    eq_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, const uint8_t* __restrict__ wtiles,
+                     const __half* __restrict__ bias, __half* __restrict__ Y, int64_t N, int Cin,
+                     int Cout, TileInfo ti, int* status) {
+  using S = Shape<T>;
+  constexpr int BD = S::BD;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled TMA destinations and operand tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
+  Bars<T>* bars = reinterpret_cast<Bars<T>*>(smem + S::OFF_BAR);
+  int* abort_flag = &bars->abort_flag;
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < X_ST; ++s) {
       mbar_init(&bars->x_full[s], 1);          // raw tile landed (TMA bytes)
-      mbar_init(&bars->x_read[s], kXfWarps);   // every transform warp holds its raw chunks
+      mbar_init(&bars->x_read[s], kXfWarps);   // every transform warp holds its raw pieces
       mbar_init(&bars->x_ready[s], kXfWarps);  // operand planes written (transform warps)
       mbar_init(&bars->x_empty[s], 1);         // MMAs done with the planes (tcgen05.commit)
     }
-    for (int s = 0; s < W_ST; ++s) {
+    for (int s = 0; s < S::W_ST; ++s) {
       mbar_init(&bars->w_full[s], 1);
       mbar_init(&bars->w_empty[s], 1);
     }
@@ -282,36 +483,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0 || warp == 2) {
-    // ------- producers: warp 0 raw X (TMA, 2D box), warp 2 weight tiles (bulk copy) -------
+    // ------- producers: warp 0 raw X (TMA, 3-D box), warp 2 weight tiles (bulk copy) -------
     if (lane == 0) {
       const bool is_raw = (warp == 0);
-      const int depth = is_raw ? X_ST : W_ST;
+      const int depth = is_raw ? X_ST : S::W_ST;
       uint64_t* full = is_raw ? bars->x_full : bars->w_full;
       uint64_t* empty = is_raw ? bars->x_empty : bars->w_empty;
-      int issued_phase[X_ST > W_ST ? X_ST : W_ST];  // last phase issued per slot
+      int issued_phase[X_ST > S::W_ST ? X_ST : S::W_ST];  // last phase issued per slot
       for (int s = 0; s < depth; ++s) issued_phase[s] = -1;
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < ti.num_tiles; tile += gridDim.x) {
         const int row0 = (tile / ti.n_dt) * BM;
-        const int d0 = (tile % ti.n_dt) * BD;
+        const int dt = tile % ti.n_dt;
         for (int ks = 0; ks < ti.k_stages; ++ks, ++it) {
           const int s = it % depth;
           const uint32_t ph = (it / depth) & 1;
-          if (!(ok = wait_bounded(&empty[s], ph ^ 1, bars, status))) break;
+          if (!(ok = wait_bounded(&empty[s], ph ^ 1, abort_flag, status))) break;
           if (!is_raw && blockIdx.x == 0 && (int)it == ti.drop_w) continue;  // injected fault
           if (is_raw) {
             mbar_expect_tx(&full[s], X_STAGE_BYTES);
             // 3-D view of X: (64 halves, 128-byte chunk of the row, row); a stage is
             // chunks 2ks, 2ks+1 of 128 rows
-            tma_load_3d(sbase + OFF_X + s * X_STAGE_BYTES, &map_x, &full[s], 0, 2 * ks, row0);
+            tma_load_3d(sbase + S::OFF_X + s * X_STAGE_BYTES, &map_x, &full[s], 0, 2 * ks, row0);
           } else {
-            // one pre-arranged blob per (out-channel tile, K stage): regions
-            // A0, A2, Br, Bi in the operand layout the MMAs read
-            mbar_expect_tx(&full[s], W_STAGE_BYTES);
-            const size_t blob = (size_t)(d0 / BD) * ti.k_stages + ks;
-            bulk_load(sbase + OFF_W + s * W_STAGE_BYTES, wtiles + blob * W_STAGE_BYTES,
-                      W_STAGE_BYTES, &full[s]);
+            // one pre-arranged blob per (out-channel tile, K stage)
+            mbar_expect_tx(&full[s], S::W_STAGE_BYTES);
+            const size_t blob = (size_t)dt * ti.k_stages + ks;
+            bulk_load(sbase + S::OFF_W + s * S::W_STAGE_BYTES, wtiles + blob * S::W_STAGE_BYTES,
+                      S::W_STAGE_BYTES, &full[s]);
           }
           issued_phase[s] = (int)ph;
         }
@@ -331,31 +531,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_n1_neg = idesc_f16(BM, BD, true);
       const uint32_t id_n2 = idesc_f16(BM, 2 * BD);
       for (int tile = blockIdx.x; ok && tile < ti.num_tiles; tile += gridDim.x, ++tcount) {
-        if (!(ok = wait_bounded(&bars->acc_empty, (tcount & 1) ^ 1, bars, status))) break;
+        if (!(ok = wait_bounded(&bars->acc_empty, (tcount & 1) ^ 1, abort_flag, status))) break;
         tc_fence_after();
         for (int ks = 0; ks < ti.k_stages; ++ks, ++it) {
-          const int sx = it % X_ST, sw = it % W_ST;
-          if (!(ok = wait_bounded(&bars->x_ready[sx], (it / X_ST) & 1, bars, status))) break;
-          if (!(ok = wait_bounded(&bars->w_full[sw], (it / W_ST) & 1, bars, status))) break;
+          const int sx = it % X_ST, sw = it % S::W_ST;
+          if (!(ok = wait_bounded(&bars->x_ready[sx], (it / X_ST) & 1, abort_flag, status))) break;
+          if (!(ok = wait_bounded(&bars->w_full[sw], (it / S::W_ST) & 1, abort_flag, status)))
+            break;
           tc_fence_after();
-          const uint32_t pl = sbase + OFF_X + sx * X_STAGE_BYTES;   // planes X0, X2, Xr, Xi
-          const uint32_t wr = sbase + OFF_W + sw * W_STAGE_BYTES;   // regions A0, A2, Br, Bi
+          const uint32_t pl = sbase + S::OFF_X + sx * X_STAGE_BYTES;     // planes
+          const uint32_t wr = sbase + S::OFF_W + sw * S::W_STAGE_BYTES;  // weight regions
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint32_t ko = 32u * kk;  // byte offset of this K step inside the 64 B rows
+          for (int kk = 0; kk < S::KSTEPS; ++kk) {
+            const uint32_t ko = 32u * kk;  // byte offset of this K step inside the rows
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
-            // Y0 += X0 A0^T ; Y2 += X2 A2^T ; [Y1r|Y1i] += Xr [Br|Bi]^T ;
-            // Y1r += (-Xi) Bi^T ; Y1i += Xi Br^T
-            umma(tmem + 0, desc_kmajor_sw64(pl + 0 * PLANE_BYTES + ko),
-                 desc_kmajor_sw64(wr + 0 * WREG_BYTES + ko), id_n1, acc);
-            umma(tmem + BD, desc_kmajor_sw64(pl + 1 * PLANE_BYTES + ko),
-                 desc_kmajor_sw64(wr + 1 * WREG_BYTES + ko), id_n1, acc);
-            umma(tmem + 2 * BD, desc_kmajor_sw64(pl + 2 * PLANE_BYTES + ko),
-                 desc_kmajor_sw64(wr + 2 * WREG_BYTES + ko), id_n2, acc);
-            umma(tmem + 2 * BD, desc_kmajor_sw64(pl + 3 * PLANE_BYTES + ko),
-                 desc_kmajor_sw64(wr + 3 * WREG_BYTES + ko), id_n1_neg, 1u);
-            umma(tmem + 3 * BD, desc_kmajor_sw64(pl + 3 * PLANE_BYTES + ko),
-                 desc_kmajor_sw64(wr + 2 * WREG_BYTES + ko), id_n1, 1u);
+            auto A = [&](int p) { return desc_kmajor<S::ROWB>(pl + p * S::PLANE_BYTES + ko); };
+            auto B = [&](int p) { return desc_kmajor<S::ROWB>(wr + p * S::WREG_BYTES + ko); };
+            // real frequencies 0 and T/2
+            umma(tmem + 0, A(0), B(0), id_n1, acc);
+            umma(tmem + BD, A(1), B(1), id_n1, acc);
+            // complex frequencies: [Y_kr|Y_ki] += Xr_k [Br_k|Bi_k]^T ;
+            // Y_kr += (-Xi_k) Bi_k^T ; Y_ki += Xi_k Br_k^T
+#pragma unroll
+            for (int k = 1; k <= S::NC; ++k) {
+              const uint32_t col = 2 * BD * k;
+              umma(tmem + col, A(2 * k), B(2 * k), id_n2, acc);
+              umma(tmem + col, A(2 * k + 1), B(2 * k + 1), id_n1_neg, 1u);
+              umma(tmem + col + BD, A(2 * k + 1), B(2 * k), id_n1, 1u);
+            }
           }
           umma_commit(&bars->x_empty[sx]);
           umma_commit(&bars->w_empty[sw]);
@@ -370,64 +573,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiWarps) {
     // ---------------- epilogue ----------------
     // Warp w reads TMEM lane quarter q = w % 4 (rows 32q..32q+31) and column half
-    // ch (out-channels 64ch..64ch+63 of the tile).  16x256b loads give lane t
-    // rows (t/4, t/4 + 8) of a 16-lane group and out-channel pair 2*(t%4) of
-    // each 8-channel group, so each 16-byte store of a warp covers 8 rows x 64
-    // contiguous bytes.
+    // ch (out-channels ch*BD/2 .. of the tile).  16x256b loads give lane t rows
+    // (t/4, t/4 + 8) of a 16-lane group and out-channel pair 2*(t%4) of each
+    // 8-channel group, so each warp store covers 8 rows x (8 channels x T x 2 B).
     const int q = warp & 3;
     const int ch = (warp - kEpiWarp0) >> 2;
     uint32_t tcount = 0;
-    const int64_t ldy = (int64_t)Cout * kT;
+    const int64_t ldy = (int64_t)Cout * T;
     const int tr = lane >> 2, tc = 2 * (lane & 3);
+    constexpr int kGroups = BD / 2 / 8;
     for (int tile = blockIdx.x; tile < ti.num_tiles; tile += gridDim.x, ++tcount) {
       const int64_t rbase = (int64_t)(tile / ti.n_dt) * BM + 32 * q;
-      const int dbase = (tile % ti.n_dt) * BD + 64 * ch;
-      // bias of this lane's 16 out-channels, loaded while the mainloop runs
-      float2 bv[8];
+      const int dbase = (tile % ti.n_dt) * BD + (BD / 2) * ch;
+      // bias of this lane's out-channels, loaded while the mainloop runs
+      float2 bv[kGroups];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < kGroups; ++j) {
         const int d = dbase + 8 * j + tc;
         bv[j] = (bias && d < Cout) ? __half22float2(*reinterpret_cast<const __half2*>(bias + d))
                                    : make_float2(0.f, 0.f);
       }
-      if (!warp_wait(&bars->acc_full, tcount & 1, bars, status)) break;
+      if (!warp_wait(&bars->acc_full, tcount & 1, abort_flag, status)) break;
       tc_fence_after();
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {  // 16-lane groups of the quarter
-        const uint32_t laddr = tmem + ((uint32_t)(32 * q + 16 * h) << 16) + 64 * ch;
+        const uint32_t laddr = tmem + ((uint32_t)(32 * q + 16 * h) << 16) + (BD / 2) * ch;
         const int64_t row_a = rbase + 16 * h + tr, row_b = row_a + 8;
+        // T = 4: 16-column batches (.x2 loads, one wait per batch); T = 8: 8 columns
+        constexpr int kGB = (T == 4) ? 2 : 1;
 #pragma unroll
-        for (int bt = 0; bt < 4; ++bt) {  // 16-column batches
-          uint32_t a0[8], a2[8], ar[8], ai[8];
-          EQL_TMEM_LD_16x256_X2(laddr + 16 * bt, a0);
-          EQL_TMEM_LD_16x256_X2(laddr + BD + 16 * bt, a2);
-          EQL_TMEM_LD_16x256_X2(laddr + 2 * BD + 16 * bt, ar);
-          EQL_TMEM_LD_16x256_X2(laddr + 3 * BD + 16 * bt, ai);
+        for (int jb = 0; jb < kGroups; jb += kGB) {
+          // accumulator columns of out-channel c: frequency plane p sits at
+          // (p / 2) * 2 BD + (p % 2) * BD + c
+          uint32_t raw[T][4 * kGB];
+#pragma unroll
+          for (int p = 0; p < T; ++p) {
+            const uint32_t col = laddr + (p >> 1) * 2 * BD + (p & 1) * BD + 8 * jb;
+            if constexpr (kGB == 2) {
+              EQL_TMEM_LD_16x256_X2(col, raw[p]);
+            } else {
+              EQL_TMEM_LD_16x256(col, raw[p]);
+            }
+          }
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {  // 8-column group inside the batch
-            const int j = 2 * bt + g;
+          for (int g = 0; g < kGB; ++g) {
+            const int j = jb + g;
             const int d = dbase + 8 * j + tc;
-            if (d >= Cout) continue;  // warp-uniform: Cout is a multiple of 8
+            if (d >= Cout) continue;  // warp-uniform: Cout is a multiple of 16
+            uint32_t acc[T][4];
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-              const int64_t row = rr ? row_b : row_a;
-              if (row >= N) continue;
-              uint32_t packed[4];
+            for (int p = 0; p < T; ++p)
 #pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {  // out-channel d + hh
-                const int k = 4 * g + 2 * rr + hh;
-                const float y0 = __uint_as_float(a0[k]), y2 = __uint_as_float(a2[k]);
-                const float yr = __uint_as_float(ar[k]), yi = __uint_as_float(ai[k]);
-                const float bb = hh ? bv[j].y : bv[j].x;
-                const float e = (y0 + y2) * 0.25f, o = (y0 - y2) * 0.25f;
-                const float r = yr * 0.5f, m = yi * 0.5f;
-                packed[2 * hh + 0] = pack_h2(e + r + bb, o - m + bb);
-                packed[2 * hh + 1] = pack_h2(e - r + bb, o + m + bb);
-              }
-              *reinterpret_cast<uint4*>(Y + row * ldy + (int64_t)d * kT) =
-                  make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            }
+              for (int k = 0; k < 4; ++k) acc[p][k] = raw[p][4 * g + k];
+            epi_store<T>(acc, row_a, row_b, d, bv[j], Y, ldy, N);
           }
         }
       }
@@ -436,71 +635,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kXfWarp0) {
     // ---------------- transform: group DFT into the operand planes ----------------
-    // The raw stage is [row][128-byte chunk c of 16 channels][128 B], every
-    // 128-byte line L = 2r + c swizzled by (L % 8).  One unit = one row x 8
-    // channels (half hq of chunk c): four 16-byte raw pieces in, one 16-byte piece
-    // out per plane (K-major 64 B rows, piece q = 2c + hq at (q ^ ((r/2) % 4))).
-    // An 8-lane phase covers 4 rows x both chunks, so its swizzled reads and
-    // writes hit 8 distinct bank groups.  Planes overwrite the raw tile of the
-    // same slot once every transform warp holds its raw pieces.
     const int xt = threadIdx.x - kXfWarp0 * 32;  // 0..255
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < ti.num_tiles; tile += gridDim.x) {
       for (int ks = 0; ks < ti.k_stages; ++ks, ++it) {
         const int sx = it % X_ST;
-        if (!(ok = warp_wait(&bars->x_full[sx], (it / X_ST) & 1, bars, status))) break;
-        uint8_t* slot = smem + OFF_X + sx * X_STAGE_BYTES;
-        uint4 v[2][4];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int unit = xt + 256 * u;
-          const int c = unit & 1, r = (unit >> 1) & (BM - 1), hq = unit >> 8;
-          const int line = 2 * r + c;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int j = hq * 4 + i;
-            v[u][i] = *reinterpret_cast<const uint4*>(slot + line * 128 + ((j ^ (line & 7)) << 4));
-          }
-        }
+        if (!(ok = warp_wait(&bars->x_full[sx], (it / X_ST) & 1, abort_flag, status))) break;
+        uint8_t* slot = smem + S::OFF_X + sx * X_STAGE_BYTES;
+        uint4 v[8];
+        xf_read<T>(slot, xt, v);
         // every raw piece of the slot is in registers before any plane overwrites it
         // (an mbarrier rather than a named barrier, so the wait stays bounded)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->x_read[sx]);
-        if (!(ok = warp_wait(&bars->x_read[sx], (it / X_ST) & 1, bars, status))) break;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int unit = xt + 256 * u;
-          const int c = unit & 1, r = (unit >> 1) & (BM - 1), hq = unit >> 8;
-          const int q = 2 * c + hq;
-          // piece i holds channels 2i (.x = x0,x1  .y = x2,x3) and 2i+1 (.z, .w)
-          uint32_t o0[4], o2[4], orr[4], oi[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float f0[2], f2[2], fr[2], fi[2];
-            const uint32_t w4[4] = {v[u][i].x, v[u][i].y, v[u][i].z, v[u][i].w};
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const float2 lo = unpack_h2(w4[2 * hh]), hi = unpack_h2(w4[2 * hh + 1]);
-              const float x0 = lo.x, x1 = lo.y, x2 = hi.x, x3 = hi.y;
-              const float a = x0 + x2, b = x1 + x3;
-              f0[hh] = a + b;
-              f2[hh] = a - b;
-              fr[hh] = x0 - x2;
-              fi[hh] = x3 - x1;
-            }
-            o0[i] = pack_h2(f0[0], f0[1]);
-            o2[i] = pack_h2(f2[0], f2[1]);
-            orr[i] = pack_h2(fr[0], fr[1]);
-            oi[i] = pack_h2(fi[0], fi[1]);
-          }
-          const uint32_t off = r * 64 + ((q ^ ((r >> 1) & 3)) << 4);
-          *reinterpret_cast<uint4*>(slot + 0 * PLANE_BYTES + off) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-          *reinterpret_cast<uint4*>(slot + 1 * PLANE_BYTES + off) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
-          *reinterpret_cast<uint4*>(slot + 2 * PLANE_BYTES + off) =
-              make_uint4(orr[0], orr[1], orr[2], orr[3]);
-          *reinterpret_cast<uint4*>(slot + 3 * PLANE_BYTES + off) = make_uint4(oi[0], oi[1], oi[2], oi[3]);
-        }
+        if (!(ok = warp_wait(&bars->x_read[sx], (it / X_ST) & 1, abort_flag, status))) break;
+        xf_write<T>(slot, xt, v);
         // make the generic-proxy stores visible to the tensor core (async proxy)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
@@ -531,54 +681,76 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Re-arrange prepared planes [P][Cout][Cin] into the kernel's per-stage weight
+// image: blob (dt, ks) = regions 0..T-1 (prepared planes 0..T-1: real frequency
+// 0, real frequency T/2, then Re and Im of each complex frequency), each BD rows
+// x BK channels in the K-major swizzled layout the MMAs read; rows and channels
+// past the matrix are zero.  One thread per 16-byte piece.
+template <int T>
+__global__ void tile_weights_kernel(const __half* __restrict__ planes, int Cin, int Cout,
+                                    int n_ks, int64_t n_chunks, uint4* __restrict__ tiles) {
+  using S = Shape<T>;
+  constexpr int kPieces = S::ROWB / 16;  // 16-byte pieces per row
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_chunks) return;
+  const int piece = (int)(idx % kPieces);
+  const int r = (int)((idx / kPieces) % S::BD);
+  const int region = (int)((idx / kPieces) / S::BD % S::NPL);
+  const int64_t blob = (idx / kPieces) / S::BD / S::NPL;
+  const int dt = (int)(blob / n_ks), ks = (int)(blob % n_ks);
+  const int d = dt * S::BD + r, c0 = ks * S::BK + piece * 8;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (d < Cout && c0 < Cin)  // Cin % 16 == 0: the 8 channels are all in range
+    v = *reinterpret_cast<const uint4*>(planes + ((int64_t)region * Cout + d) * Cin + c0);
+  // swizzle: piece ^= (byte offset of the row >> 7) within the swizzle span
+  const int swz = ((r * S::ROWB) >> 7) & (kPieces - 1);
+  const int64_t dst_byte = blob * S::W_STAGE_BYTES + (int64_t)region * S::WREG_BYTES +
+                           r * S::ROWB + ((piece ^ swz) << 4);
+  tiles[dst_byte >> 4] = v;
+}
+
+template <typename F>
+cudaError_t dispatch_tc(int T, F&& f) {
+  if (T == 4) return f(std::integral_constant<int, 4>{});
+  if (T == 8) return f(std::integral_constant<int, 8>{});
+  return cudaErrorNotSupported;
+}
+
 }  // namespace
 
 bool fwd_tc_supported(int T, DType dt, int64_t N, int Cin, int Cout) {
-  return T == 4 && dt == DType::F16 && N >= 1 && N <= 0x7fffff80LL && Cin % 16 == 0 &&
-         Cout % 16 == 0 && Cin >= 16 && Cout >= 16;
+  return (T == 4 || T == 8) && dt == DType::F16 && N >= 1 && N <= 0x7fffff80LL &&
+         Cin % 16 == 0 && Cout % 16 == 0 && Cin >= 16 && Cout >= 16;
 }
 
 bool tc_tiles_wanted(int T, DType dt, int C, int D) {
-  return T == 4 && dt == DType::F16 && C % 16 == 0 && D % 16 == 0 && C >= 16 && D >= 16;
+  return (T == 4 || T == 8) && dt == DType::F16 && C % 16 == 0 && D % 16 == 0 && C >= 16 &&
+         D >= 16;
 }
 
-size_t tc_tile_bytes(int Cin, int Cout) {
-  const size_t n_dt = (size_t)(Cout + BD - 1) / BD, n_ks = (size_t)(Cin + BK - 1) / BK;
-  return n_dt * n_ks * W_STAGE_BYTES;
+size_t tc_tile_bytes(int T, int Cin, int Cout) {
+  size_t bytes = 0;
+  dispatch_tc(T, [&](auto tcst) {
+    using S = Shape<decltype(tcst)::value>;
+    const size_t n_dt = (size_t)(Cout + S::BD - 1) / S::BD, n_ks = (size_t)(Cin + S::BK - 1) / S::BK;
+    bytes = n_dt * n_ks * S::W_STAGE_BYTES;
+    return cudaSuccess;
+  });
+  return bytes;
 }
 
-namespace {
-// Re-arrange prepared planes [P][Cout][Cin] into the kernel's per-stage weight
-// image: blob (dt, ks) = regions A0, A2, Br, Bi (prepared planes 0..3), each BD
-// rows x 32 channels in the K-major 64B-swizzled layout; rows and channels past
-// the matrix are zero.  One thread per 16-byte chunk.
-__global__ void tile_weights_kernel(const __half* __restrict__ planes, int Cin, int Cout,
-                                    int n_ks, int64_t n_chunks, uint4* __restrict__ tiles) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= n_chunks) return;
-  const int chunk = (int)(idx & 3);                   // 8-channel piece of the 64 B row
-  const int r = (int)((idx >> 2) % BD);               // row in the region
-  const int region = (int)((idx >> 2) / BD % kPlanes);
-  const int64_t blob = (idx >> 2) / BD / kPlanes;
-  const int dt = (int)(blob / n_ks), ks = (int)(blob % n_ks);
-  const int d = dt * BD + r, c0 = ks * BK + chunk * 8;
-  uint4 v = make_uint4(0u, 0u, 0u, 0u);
-  if (d < Cout && c0 < Cin)  // Cin % 8 == 0: the 8 channels are all in range
-    v = *reinterpret_cast<const uint4*>(planes + ((int64_t)region * Cout + d) * Cin + c0);
-  const int64_t dst_byte = blob * W_STAGE_BYTES + (int64_t)region * WREG_BYTES + r * 64 +
-                           ((chunk ^ ((r >> 1) & 3)) << 4);
-  tiles[dst_byte >> 4] = v;
-}
-}  // namespace
-
-cudaError_t launch_tile_weights(const void* planes, int Cin, int Cout, void* tiles,
+cudaError_t launch_tile_weights(int T, const void* planes, int Cin, int Cout, void* tiles,
                                 cudaStream_t st) {
-  const int n_ks = (Cin + BK - 1) / BK;
-  const int64_t n_chunks = (int64_t)tc_tile_bytes(Cin, Cout) / 16;
-  const unsigned blocks = (unsigned)((n_chunks + 255) / 256);
-  tile_weights_kernel<<<blocks, 256, 0, st>>>(static_cast<const __half*>(planes), Cin, Cout,
-                                               n_ks, n_chunks, static_cast<uint4*>(tiles));
-  return cudaGetLastError();
+  return dispatch_tc(T, [&](auto tcst) {
+    constexpr int TT = decltype(tcst)::value;
+    using S = Shape<TT>;
+    const int n_ks = (Cin + S::BK - 1) / S::BK;
+    const int64_t n_chunks = (int64_t)tc_tile_bytes(TT, Cin, Cout) / 16;
+    const unsigned blocks = (unsigned)((n_chunks + 255) / 256);
+    tile_weights_kernel<TT><<<blocks, 256, 0, st>>>(static_cast<const __half*>(planes), Cin, Cout,
+                                                    n_ks, n_chunks, static_cast<uint4*>(tiles));
+    return cudaGetLastError();
+  });
 }
 
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
@@ -588,12 +760,13 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
   if (!Wtiles) return cudaErrorNotSupported;
   auto encode = encode_fn();
   if (!encode) return cudaErrorNotSupported;
-
-  CUtensorMap mx;
-  {
-    // X row = Cin/16 chunks of 64 halves (128 B); box = 2 chunks x 128 rows
-    cuuint64_t dims[3] = {64, (cuuint64_t)Cin / 16, (cuuint64_t)N};
-    cuuint64_t strides[2] = {128, (cuuint64_t)Cin * kT * 2};
+  return dispatch_tc(T, [&](auto tcst) {
+    constexpr int TT = decltype(tcst)::value;
+    using S = Shape<TT>;
+    CUtensorMap mx;
+    // X row = Cin*T/64 chunks of 64 halves (128 B); box = 2 chunks x 128 rows
+    cuuint64_t dims[3] = {64, (cuuint64_t)Cin * TT / 64, (cuuint64_t)N};
+    cuuint64_t strides[2] = {128, (cuuint64_t)Cin * TT * 2};
     cuuint32_t box[3] = {64, 2, BM};
     cuuint32_t estr[3] = {1, 1, 1};
     if (encode(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(X), dims, strides, box,
@@ -601,27 +774,27 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
-  }
-  TileInfo ti;
-  ti.n_dt = (Cout + BD - 1) / BD;
-  const int64_t n_rt = (N + BM - 1) / BM;
-  if (n_rt * ti.n_dt > 0x7fffffffLL) return cudaErrorInvalidValue;
-  ti.num_tiles = (int)(n_rt * ti.n_dt);
-  ti.k_stages = (Cin + BK - 1) / BK;
-  ti.drop_w = drop_w_stage;
-
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(p4_fwd_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  const int grid = ti.num_tiles < num_sms ? ti.num_tiles : num_sms;
-  p4_fwd_tc_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(
-      mx, static_cast<const uint8_t*>(Wtiles), static_cast<const __half*>(bias),
-      static_cast<__half*>(Y), N, Cin, Cout, ti, status);
-  return cudaGetLastError();
+    TileInfo ti;
+    ti.n_dt = (Cout + S::BD - 1) / S::BD;
+    const int64_t n_rt = (N + BM - 1) / BM;
+    if (n_rt * ti.n_dt > 0x7fffffffLL) return cudaErrorInvalidValue;
+    ti.num_tiles = (int)(n_rt * ti.n_dt);
+    ti.k_stages = (Cin + S::BK - 1) / S::BK;
+    ti.drop_w = drop_w_stage;
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(eq_fwd_tc_kernel<TT>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           S::SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    const int grid = ti.num_tiles < num_sms ? ti.num_tiles : num_sms;
+    eq_fwd_tc_kernel<TT><<<grid, kThreads, S::SMEM_BYTES, st>>>(
+        mx, static_cast<const uint8_t*>(Wtiles), static_cast<const __half*>(bias),
+        static_cast<__half*>(Y), N, Cin, Cout, ti, status);
+    return cudaGetLastError();
+  });
 }
 
 }  // namespace eql

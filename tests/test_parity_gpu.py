@@ -131,22 +131,24 @@ def test_edge_shapes_all_ops(T, N, C, D, dtype):
 
 
 TC_EDGE = [
-    # N, C, D : ragged rows, channels and out-channels for the tcgen05 p4 path
-    (1, 16, 16), (127, 48, 144), (129, 80, 208), (300, 208, 16), (513, 64, 384), (260, 336, 80),
+    # T, N, C, D : ragged rows, channels and out-channels for the tcgen05 path
+    (4, 1, 16, 16), (4, 127, 48, 144), (4, 129, 80, 208), (4, 300, 208, 16), (4, 513, 64, 384),
+    (4, 260, 336, 80),
+    (8, 1, 16, 16), (8, 129, 48, 80), (8, 300, 128, 128), (8, 257, 32, 208), (8, 200, 176, 48),
 ]
 
 
-@pytest.mark.parametrize("N,C,D", TC_EDGE)
-def test_tcgen05_edge_shapes(N, C, D):
-    w = Workload("tcedge", 4, N, C, D, "f16", True, 500 + N + C + D)
+@pytest.mark.parametrize("T,N,C,D", TC_EDGE)
+def test_tcgen05_edge_shapes(T, N, C, D):
+    w = Workload("tcedge", T, N, C, D, "f16", True, 500 + N + C + D)
     inp = make_inputs(w, need_dy=True)
     p = _plan(w, "tcgen05")
     assert p.forward_kernel_name(N) == "tcgen05"
     Wh = p.prepare_weights(_dev(inp["W"]))
     Y = p.forward(_dev(inp["X"]), Wh, _dev(inp["bias"])).double().cpu().numpy()
-    assert _rel(Y, oracle.forward(4, inp["X"], inp["W"], inp["bias"])) <= TOL["f16"]
+    assert _rel(Y, oracle.forward(T, inp["X"], inp["W"], inp["bias"])) <= TOL["f16"]
     dX = p.backward_input(_dev(inp["dY"]), Wh).double().cpu().numpy()
-    assert _rel(dX, oracle.backward_input(4, inp["dY"], inp["W"])) <= TOL["f16"]
+    assert _rel(dX, oracle.backward_input(T, inp["dY"], inp["W"])) <= TOL["f16"]
     assert p.status() == 0
 
 
