@@ -9,7 +9,8 @@ resident in HBM; `e2e` = the same through the C ABI with the step's input copied
 from pinned host memory and the result read back, inside the timed region.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--workload p4_vitb_mlp_f16|p4_vitb_proj_f32|p4_vith_fc1_f16|c8_1024_f16]
+       [--workload p4_vitb_mlp_f16|p4_vitb_proj_f32|p4_vith_fc1_f16|c8_1024_f16|
+                   p4_vith_fc1_fwd_bwd_f16]
 Under torchrun (N > 1) every rank runs its own copy of the workload (weak
 scaling; rows are independent, so no collective is on the data path).
 """
@@ -19,9 +20,8 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
+import threading
 import time
 
 import numpy as np
@@ -41,13 +41,17 @@ PIPELINES = {
     "p4_vitb_proj_f32": ["p4_vitb_proj_f32"],
     "p4_vith_fc1_f16": ["p4_vith_fc1_f16"],
     "c8_1024_f16": ["c8_1024_f16"],
+    "p4_vith_fc1_fwd_bwd_f16": ["p4_vith_fc1_f16"],
 }
+BACKWARD = {"p4_vith_fc1_fwd_bwd_f16"}
 DESCR = {
     "p4_vitb_mlp_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
                        "C=768->D=192, T=4",
     "p4_vitb_proj_f32": "p4 EQ-Linear fp32 ViT-B projection: N=12608, C=D=192, T=4",
     "p4_vith_fc1_f16": "p4 EQ-Linear fp16 ViT-H fc1: N=8224, C=320->D=1280, T=4",
     "c8_1024_f16": "cyclic T=8 EQ-Linear fp16: N=16384, C=D=128",
+    "p4_vith_fc1_fwd_bwd_f16": "p4 EQ-Linear fp16 ViT-H fc1 forward + dX + dW: N=8224, "
+                               "C=320->D=1280, T=4",
 }
 
 
@@ -95,55 +99,81 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks and clock-event (throttle) reasons, polled through NVML every ~2 ms.
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = None
+    `mark()` brackets the timed region (called with the GPU idle, right before the
+    timed launches are queued and right after they completed), so only samples
+    taken while the timed kernels ran are reported.
+    """
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
+               "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []  # (host time, sm MHz, max sm MHz, reason bits)
+        self.window = [None, None]
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+
+    def _handle(self, nv):
+        import torch
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:
+            return
+        self._nvml = nv
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    self.samples.append((time.perf_counter(), sm, mx, int(reasons(h))))
+                except Exception:
+                    pass
+                time.sleep(0.002)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
+
+    def mark(self, which: int):
+        self.window[which] = time.perf_counter()
 
     def stop(self):
-        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        if self.proc is None:
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+               "source": "nvml, 2 ms polling, samples inside the timed region"}
+        if self._thread is None:
+            out["source"] = "unavailable (NVML could not be opened)"
             return out
-        self.proc.terminate()
+        self._stop.set()
+        self._thread.join(timeout=5)
+        t0, t1 = self.window
+        inside = [s for s in self.samples if t0 is not None and t1 is not None and t0 <= s[0] <= t1]
+        if inside:
+            bits = 0
+            for s in inside:
+                bits |= s[3]
+            out.update(sm_mhz=statistics.median(s[1] for s in inside),
+                       sm_max_mhz=max(s[2] for s in inside),
+                       reasons=sorted(k for k, v in self.REASONS.items() if bits & v),
+                       samples=len(inside))
         try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for nm, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(nm)
-        os.unlink(self.path)
-        if sm:
-            out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                   "reasons": sorted(reasons), "samples": len(sm)}
+            self._nvml.nvmlShutdown()
+        except Exception:
+            pass
         return out
 
 
@@ -154,20 +184,25 @@ def dist_init():
     return world, rank, local
 
 
-def oracle_sample(pipeline, rows: int):
-    """Time the float64 oracle on `rows` rows of the pipeline; returns (seconds, rows)."""
+def oracle_sample(pipeline, rows: int, backward: bool = False):
+    """Time the float64 oracle on `rows` rows of the step's ops; returns (seconds, rows)."""
     import oracle
     oracle.build()
-    layers = [(WORKLOADS[name], make_inputs(WORKLOADS[name], rows=rows)) for name in pipeline]
+    layers = [(WORKLOADS[name], make_inputs(WORKLOADS[name], rows=rows, need_dy=backward))
+              for name in pipeline]
     x = layers[0][1]["X"].astype(np.float64)
     t0 = time.perf_counter()
     for w, inp in layers:
         x = oracle.forward(w.T, x, inp["W"], inp["bias"])
+    if backward:
+        w, inp = layers[0]
+        oracle.backward_input(w.T, inp["dY"], inp["W"])
+        oracle.backward_weight(w.T, inp["X"], inp["dY"], w.D)
     return time.perf_counter() - t0, rows
 
 
-def calibrated_oracle_rows(pipeline, target_s: float) -> int:
-    t, r = oracle_sample(pipeline, 16)
+def calibrated_oracle_rows(pipeline, target_s: float, backward: bool = False) -> int:
+    t, r = oracle_sample(pipeline, 16, backward)
     n_full = WORKLOADS[pipeline[0]].N
     return int(max(16, min(n_full, 16 * target_s / max(t, 1e-6))))
 
@@ -179,11 +214,12 @@ def run_reference(args, workload):
     if rank != 0:
         return 0
     pipeline = PIPELINES[workload]
+    backward = workload in BACKWARD
     per_step_s = max(1.0, 120.0 / max(1, args.steps + args.warmup))
-    rows = calibrated_oracle_rows(pipeline, min(per_step_s, 20.0))
+    rows = calibrated_oracle_rows(pipeline, min(per_step_s, 20.0), backward)
     for _ in range(args.warmup):
-        oracle_sample(pipeline, rows)
-    times = [oracle_sample(pipeline, rows)[0] for _ in range(args.steps)]
+        oracle_sample(pipeline, rows, backward)
+    times = [oracle_sample(pipeline, rows, backward)[0] for _ in range(args.steps)]
     total = sum(times)
     value = rows * args.steps / total
     w0 = WORKLOADS[pipeline[0]]
@@ -204,6 +240,10 @@ def run_reference(args, workload):
     return 0
 
 
+def wgrad_flops(w) -> float:
+    return layer_flops(w)  # same per-frequency products, reduced over rows
+
+
 def run_ours(args, workload):
     import torch
     import torch.distributed as dist
@@ -216,6 +256,7 @@ def run_ours(args, workload):
                                 device_id=torch.device("cuda", local))
     from group_circulant_gemm_b200 import EqLinearPlan
 
+    backward = workload in BACKWARD
     pipeline = [WORKLOADS[n] for n in PIPELINES[workload]]
     dt = torch.float16 if pipeline[0].dtype == "f16" else torch.float32
     N = pipeline[0].N
@@ -231,28 +272,59 @@ def run_ours(args, workload):
         plans.append(p)
         whats.append(p.prepare_weights(W))
         biases.append(torch.from_numpy(inp["bias"]).cuda() if w.bias else None)
-    x_host = make_inputs(pipeline[0].with_(seed=pipeline[0].seed + 1000 * rank))["X"]
+    first = make_inputs(pipeline[0].with_(seed=pipeline[0].seed + 1000 * rank), need_dy=backward)
+    x_host = first["X"]
+    dy_host = first.get("dY")
 
     # rotating input/output sets so the step's working set leaves L2 between steps
     per_set = sum(N * w.C * w.T * es + N * w.D * w.T * es for w in pipeline)
+    if backward:
+        per_set += sum(N * w.D * w.T * es + N * w.C * w.T * es for w in pipeline)
     nsets = max(2, int(np.ceil(2 * L2_BYTES / per_set)))
     xs = [torch.from_numpy(x_host).cuda() for _ in range(nsets)]
     outs = [[torch.empty((N, w.D * w.T), dtype=dt, device="cuda") for w in pipeline]
             for _ in range(nsets)]
+    if backward:
+        w0 = pipeline[0]
+        dys = [torch.from_numpy(dy_host).cuda() for _ in range(nsets)]
+        dxs = [torch.empty((N, w0.C * w0.T), dtype=dt, device="cuda") for _ in range(nsets)]
+        dW = torch.empty((w0.D, w0.C, w0.T), dtype=dt, device="cuda")
+        db = torch.empty((w0.D,), dtype=dt, device="cuda")
+        ws = torch.empty(max(16, plans[0].workspace_bytes(N)), dtype=torch.uint8, device="cuda")
+
+    # the ops of one step: (label, kernel, flops, algorithmic bytes, callable(set index))
+    ops = []
+    for li, w in enumerate(pipeline):
+        def fwd(i, li=li):
+            x = xs[i % nsets] if li == 0 else outs[i % nsets][li - 1]
+            plans[li].forward(x, whats[li], biases[li], out=outs[i % nsets][li])
+        ops.append(("forward", plans[li].forward_kernel_name(N), layer_flops(w), layer_bytes(w),
+                    fwd))
+    if backward:
+        w0 = pipeline[0]
+
+        def bwd_x(i):
+            plans[0].backward_input(dys[i % nsets], whats[0], out=dxs[i % nsets])
+
+        def bwd_w(i):
+            plans[0].backward_weight(xs[i % nsets], dys[i % nsets], dW=dW, dbias=db, workspace=ws)
+        nb = es * (N * w0.C * w0.T + N * w0.D * w0.T)
+        ops.append(("backward_input", plans[0].forward_kernel_name(N), layer_flops(w0),
+                    nb + es * 1.25 * w0.C * w0.D * w0.T, bwd_x))
+        ops.append(("backward_weight", plans[0].backward_weight_kernel_name(N), wgrad_flops(w0),
+                    nb + es * w0.D * w0.C * w0.T, bwd_w))
 
     def step(i, events=None):
-        x = xs[i % nsets]
-        for li, (p, wh, b) in enumerate(zip(plans, whats, biases)):
+        for _, _, _, _, fn in ops:
             if events is not None:
                 events.append(torch.cuda.Event(enable_timing=True))
                 events[-1].record(stream)
-            p.forward(x, wh, b, out=outs[i % nsets][li])
+            fn(i)
             if events is not None:
                 events.append(torch.cuda.Event(enable_timing=True))
                 events[-1].record(stream)
-            x = outs[i % nsets][li]
 
-    kernel_names = [p.forward_kernel_name(N) for p in plans]
+    kernel_names = [k for _, k, _, _, _ in ops]
     # the clock sampler runs from the start of warm-up to the end of the timed region
     clocks = ClockSampler(local)
     if rank == 0:
@@ -266,6 +338,7 @@ def run_ours(args, workload):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    clocks.mark(0)
     ev = []
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
@@ -274,19 +347,38 @@ def run_ours(args, workload):
         step(args.warmup + i, ev)
     t1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark(1)
     if world > 1:
         dist.barrier()
     clk = clocks.stop() if rank == 0 else {}
     elapsed_ms = t0.elapsed_time(t1)
-    launch_ms = [ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(len(ev) // 2)]
+    launch_ms = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1])
+                          for j in range(len(ev) // 2)]).reshape(args.steps, len(ops))
 
-    # end to end through the ABI: pinned host input -> device, both layers, result -> host
+    # end to end through the ABI: pinned host inputs -> device, the step, results -> host
     x_pin = torch.from_numpy(x_host).pin_memory()
     y_pin = torch.empty((N, pipeline[-1].D * pipeline[-1].T), dtype=dt).pin_memory()
-    for _ in range(2):
+    h2d = x_pin.numel() * x_pin.element_size()
+    d2h = y_pin.numel() * y_pin.element_size()
+    if backward:
+        dy_pin = torch.from_numpy(dy_host).pin_memory()
+        dx_pin = torch.empty(tuple(dxs[0].shape), dtype=dt).pin_memory()
+        dw_pin = torch.empty(tuple(dW.shape), dtype=dt).pin_memory()
+        h2d += dy_pin.numel() * dy_pin.element_size()
+        d2h += (dx_pin.numel() + dw_pin.numel()) * dx_pin.element_size()
+
+    def e2e_step():
         xs[0].copy_(x_pin, non_blocking=True)
+        if backward:
+            dys[0].copy_(dy_pin, non_blocking=True)
         step(0)
         y_pin.copy_(outs[0][-1], non_blocking=True)
+        if backward:
+            dx_pin.copy_(dxs[0], non_blocking=True)
+            dw_pin.copy_(dW, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -294,9 +386,7 @@ def run_ours(args, workload):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
-        xs[0].copy_(x_pin, non_blocking=True)
-        step(0)
-        y_pin.copy_(outs[0][-1], non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -310,24 +400,32 @@ def run_ours(args, workload):
 
     if rank == 0:
         peaks, peak_src = load_peaks()
-        flops = sum(layer_flops(w) for w in pipeline)
+        flops = sum(f for _, _, f, _, _ in ops)
         value = world * N * args.steps / (elapsed_ms / 1e3)
         e2e_value = world * N * args.steps / (e2e_ms / 1e3)
-        # dominant kernel: the per-layer forward kernel (same kernel for every layer)
-        per_layer = np.array(launch_ms).reshape(args.steps, len(pipeline))
-        mean_launch_ms = float(per_layer.mean())
-        flops_per_launch = flops / len(pipeline)
-        bytes_per_launch = sum(layer_bytes(w) for w in pipeline) / len(pipeline)
-        if kernel_names[0] == "tcgen05":
+        # dominant kernel: the kernel family with the largest share of the step
+        mean_ms = launch_ms.mean(axis=0)
+        fam = {}
+        for j, (label, kern, f, nbytes, _) in enumerate(ops):
+            key = (label if label != "backward_input" else "forward", kern)
+            a = fam.setdefault(key, [0.0, 0.0, 0.0, 0])
+            a[0] += mean_ms[j]
+            a[1] += f
+            a[2] += nbytes
+            a[3] += 1
+        (dlabel, dkern), (dms, dflops, dbytes, dcount) = max(fam.items(), key=lambda kv: kv[1][0])
+        mean_launch_ms = dms / dcount
+        flops_per_launch = dflops / dcount
+        bytes_per_launch = dbytes / dcount
+        achieved = flops_per_launch / (mean_launch_ms / 1e3) / 1e12
+        if dkern == "tcgen05":
             peak = peaks["bf16_tflops"]
-            achieved = flops_per_launch / (mean_launch_ms / 1e3) / 1e12
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": kernel_traffic(workload),
                     "peak_source": f"{peak_src} dense bf16 burst (fp16 runs at the same rate)"}
         else:
             # CUDA-core FP32 FMA peak: 148 SMs x 128 FMA/clk x 2 FLOP x max SM clock
             peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-            achieved = flops_per_launch / (mean_launch_ms / 1e3) / 1e12
             roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": None,
                     "peak_source": "derived: 148 SM x 128 FP32 FMA/clk x 2 x max SM clock"}
@@ -335,15 +433,17 @@ def run_ours(args, workload):
         roof["hbm_gbs"] = hbm
         roof["hbm_frac"] = hbm / peaks["hbm_gbs"]
         roof["launch_ms"] = mean_launch_ms
-        roof["kernel"] = f"eqlinear_forward[{kernel_names[0]}]"
+        roof["kernel"] = f"eqlinear_{dlabel}[{dkern}]"
+        roof["step_share"] = dms / float(mean_ms.sum())
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             import oracle
-            rows = calibrated_oracle_rows(PIPELINES[workload], 10.0)
-            secs, rows = oracle_sample(PIPELINES[workload], rows)
+            rows = calibrated_oracle_rows(PIPELINES[workload], 10.0, backward)
+            secs, rows = oracle_sample(PIPELINES[workload], rows, backward)
             cpu = {"value": rows / secs, "unit": "tokens/s", "cores": oracle.threads_used(),
                    "kind": "oracle",
-                   "sample": f"{rows} of {N} rows through every layer, float64, {secs:.1f} s"}
+                   "sample": f"{rows} of {N} rows through every op of the step, float64, "
+                             f"{secs:.1f} s"}
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -355,13 +455,13 @@ def run_ours(args, workload):
                        "parallelism": f"replicas x{world} (rows independent)",
                        "l2": f"{nsets} rotating input/output sets of {per_set / 2**20:.0f} MiB "
                              "(> 2x L2)",
-                       "kernels": kernel_names},
+                       "kernels": [f"{label}[{k}]" for label, k, _, _, _ in ops]},
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
-                    "h2d_bytes_per_step": int(x_host.nbytes),
-                    "d2h_bytes_per_step": int(y_pin.numel() * y_pin.element_size())},
-            "gpu_launches": args.steps * len(pipeline),
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "gpu_launches": args.steps * sum(2 if label == "backward_weight" else 1
+                                             for label, _, _, _, _ in ops),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
@@ -376,7 +476,7 @@ def run_ours(args, workload):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(PIPELINES), default="p4_vitb_mlp_f16")

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <new>
 
 #include "../../include/eqlinear.h"
@@ -165,10 +166,22 @@ const char* eqlinear_forward_kernel_name(eqlinear_plan_t p, int64_t N) {
   return "simt";
 }
 
+// The tensor-core weight gradient needs 16-byte aligned X and dY (TMA); the
+// name query assumes aligned buffers, as every torch allocation is.
+static bool wgrad_tc_ok(eqlinear_plan_t p, int64_t N, const void* X, const void* dY) {
+  return eql::wgrad_tc_supported(p->T, to_dt(p->dtype), N, p->C, p->D, X, dY);
+}
+
+static bool wgrad_use_tc(eqlinear_plan_t p, int64_t N, const void* X, const void* dY) {
+  return p->kernel != EQL_KERNEL_SIMT && wgrad_tc_ok(p, N, X, dY);
+}
+
 const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t p, int64_t N) {
-  (void)N;
   if (!p) return "unsupported";
-  if (p->kernel == EQL_KERNEL_TCGEN05) return "unsupported";
+  const void* aligned = reinterpret_cast<const void*>(uintptr_t(256));
+  const bool tc_ok = wgrad_tc_ok(p, N, aligned, aligned);
+  if (p->kernel == EQL_KERNEL_TCGEN05) return tc_ok ? "tcgen05" : "unsupported";
+  if (p->kernel == EQL_KERNEL_AUTO && tc_ok) return "tcgen05";
   return "simt";
 }
 
@@ -224,9 +237,14 @@ eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int
                           nullptr, dX, (cudaStream_t)stream);
 }
 
+// Enough for either kernel, so the size does not depend on which one runs.
 size_t eqlinear_backward_weight_workspace_bytes(eqlinear_plan_t p, int64_t N) {
   if (!p || N < 0) return 0;
-  return eql::wgrad_simt_workspace(p->T, N, p->C, p->D, p->num_sms);
+  size_t need = eql::wgrad_simt_workspace(p->T, N, p->C, p->D, p->num_sms);
+  const void* aligned = reinterpret_cast<const void*>(uintptr_t(256));
+  if (wgrad_tc_ok(p, N, aligned, aligned))
+    need = std::max(need, eql::wgrad_tc_workspace(N, p->C, p->D, p->num_sms));
+  return need;
 }
 
 eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t p, const void* X, const void* dY,
@@ -234,18 +252,29 @@ eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t p, const void* X, con
                                            size_t workspace_bytes, void* stream) {
   if (!p || N < 0 || !dW) return EQL_ERR_INVALID_ARG;
   if (N > 0 && (!X || !dY)) return EQL_ERR_INVALID_ARG;
-  if (p->kernel == EQL_KERNEL_TCGEN05) return EQL_ERR_UNSUPPORTED;
   if ((X && !aligned16(X)) || (dY && !aligned16(dY)) || !aligned16(dW) ||
       (dbias && !aligned16(dbias)) || (workspace && !aligned16(workspace)))
     return EQL_ERR_ALIGNMENT;
-  const size_t need = eql::wgrad_simt_workspace(p->T, N, p->C, p->D, p->num_sms);
-  if (!workspace || workspace_bytes < need) return EQL_ERR_WORKSPACE;
+  if (p->kernel == EQL_KERNEL_TCGEN05 && !wgrad_tc_ok(p, N, X, dY)) return EQL_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < eqlinear_backward_weight_workspace_bytes(p, N))
+    return EQL_ERR_WORKSPACE;
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (wgrad_use_tc(p, N, X, dY)) {
+    const int splits = eql::wgrad_tc_splits(N, p->C, p->D, p->num_sms);
+    float* part = static_cast<float*>(workspace);
+    float* bpart = part + (size_t)splits * 4 * p->C * p->D;
+    s = from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, part, bpart, splits, p->status,
+                                       p->num_sms, st));
+    if (s != EQL_OK) return s;
+    return from_cuda(eql::launch_wgrad_finalize(p->T, to_dt(p->dtype), part, bpart, splits,
+                                                p->C, p->D, dW, dbias, p->tw, st));
+  }
   const int splits = eql::wgrad_simt_splits(p->T, N, p->C, p->D, p->num_sms);
   return from_cuda(eql::launch_wgrad_simt(p->T, to_dt(p->dtype), X, dY, N, p->C, p->D, dW,
                                           dbias, static_cast<float*>(workspace), splits, p->tw,
-                                          (cudaStream_t)stream));
+                                          st));
 }
 
 eqlinear_status_t eqlinear_get_status(eqlinear_plan_t p, void* stream) {

@@ -39,9 +39,12 @@
 #include <type_traits>
 
 #include "eql_kernels.h"
+#include "eql_tc_common.cuh"
 
 namespace eql {
 namespace {
+
+using namespace tc;
 
 constexpr int BM = 128;          // rows per tile = MMA M
 constexpr int X_ST = 4;          // X ring: raw tile in, transformed operand planes out (in place)
@@ -90,11 +93,6 @@ struct Shape : Cfg<T> {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-constexpr unsigned long long kTimeoutNs = 2000000000ull;
-
-// status word codes
-constexpr int kErrTimeout = 1;
-
 template <int T>
 struct Bars {
   uint64_t x_full[X_ST], x_read[X_ST], x_ready[X_ST], x_empty[X_ST];
@@ -103,166 +101,6 @@ struct Bars {
   uint32_t tmem_base;
   int abort_flag;
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t gtimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// try_wait with a suspend-time hint: the thread sleeps in hardware until the
-// phase completes or about `ns` nanoseconds pass, instead of spinning on shared
-// memory (which would steal issue slots from the producer and MMA threads).
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* b, uint32_t parity, uint32_t ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity), "r"(ns)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: false if the CTA aborted or the wait timed out (then aborts it).
-__device__ __noinline__ bool wait_bounded(uint64_t* b, uint32_t parity, int* abort_flag, int* status) {
-  if (mbar_try_wait(b, parity)) return true;
-  const uint64_t t0 = gtimer();
-  while (true) {
-    if (mbar_try_wait_sleep(b, parity, 200000u)) return true;
-    if (*(volatile int*)abort_flag) return false;
-    if (gtimer() - t0 > kTimeoutNs) {
-      *(volatile int*)abort_flag = 1;
-      atomicExch(status, kErrTimeout);
-      return false;
-    }
-  }
-}
-// Warp-uniform bounded wait: every lane polls, then the warp agrees, so a lane
-// that gave up cannot leave the others waiting at a warp-synchronous point.
-__device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, int* abort_flag, int* status) {
-  const bool ok = wait_bounded(b, parity, abort_flag, status);
-  return __all_sync(0xffffffffu, ok);
-}
-// Bounded wait used while draining after an abort (ignores the abort flag).
-__device__ __noinline__ void drain_wait(uint64_t* b, uint32_t parity) {
-  const uint64_t t0 = gtimer();
-  while (!mbar_try_wait_sleep(b, parity, 200000u)) {
-    if (gtimer() - t0 > kTimeoutNs) return;
-  }
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
-                                            int x, int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
-// Plain bulk copy global -> shared of `bytes` (multiple of 16, both 16 B aligned).
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// K-major swizzled operand tile descriptor: rows of `row_bytes` (32 or 64 B of
-// K), 8-row groups 8 * row_bytes apart (SBO), descriptor version 1 (sm_100);
-// layout type 4 = SWIZZLE_64B (16-byte piece ^= (row / 2) % 4), 6 = SWIZZLE_32B
-// (piece ^= (row / 4) % 2).  A later K step inside a row starts 32 B further.
-template <int kRowBytes>
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) {
-  static_assert(kRowBytes == 32 || kRowBytes == 64, "operand row width");
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1u << 16;                          // leading byte offset (unused)
-  d |= (uint64_t)((8u * kRowBytes) >> 4) << 32;     // stride byte offset
-  d |= (uint64_t)1u << 46;                          // descriptor version for sm_100
-  d |= (uint64_t)(kRowBytes == 64 ? 4u : 6u) << 61; // SWIZZLE_64B / SWIZZLE_32B
-  return d;
-}
-// Instruction descriptor, kind::f16: A = B = F16, D = F32, both K-major;
-// bit 13 negates A.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool negate_a = false) {
-  return (1u << 4) | (negate_a ? (1u << 13) : 0u) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                     uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// 16 TMEM lanes x 256 bits: thread t gets lanes (t/4) and (t/4 + 8) of the
-// addressed 16-lane group, columns 2*(t%4) and 2*(t%4)+1 -> regs
-// {lane t/4: col, col+1, lane t/4+8: col, col+1}.
-#define EQL_TMEM_LD_16x256(taddr, r)                                                   \
-  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0, %1, %2, %3}, [%4];"         \
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])                         \
-               : "r"(taddr))
-// The .x2 form repeats the pattern for the next 8 columns in regs 4..7.
-#define EQL_TMEM_LD_16x256_X2(taddr, r)                                                    \
-  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"    \
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),    \
-                 "=r"(r[6]), "=r"(r[7])                                                    \
-               : "r"(taddr))
-
-__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-  const __half2 h = __floats2half2_rn(a, b);  // a -> low half, b -> high half
-  uint32_t u;
-  memcpy(&u, &h, 4);
-  return u;
-}
-__device__ __forceinline__ float2 unpack_h2(uint32_t u) {
-  __half2 h;
-  memcpy(&h, &u, 4);
-  return __half22float2(h);
-}
 
 
 struct TileInfo {
@@ -668,18 +506,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
 
 // Re-arrange prepared planes [P][Cout][Cin] into the kernel's per-stage weight
 // image: blob (dt, ks) = regions 0..T-1 (prepared planes 0..T-1: real frequency

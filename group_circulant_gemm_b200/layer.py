@@ -48,6 +48,9 @@ class EqLinearPlan:
     def forward_kernel_name(self, N: int) -> str:
         return _n.eqlinear_forward_kernel_name(self.handle, N)
 
+    def backward_weight_kernel_name(self, N: int) -> str:
+        return _n.eqlinear_backward_weight_kernel_name(self.handle, N)
+
     def prepare_weights(self, W: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
         self._check(W, (self.D, self.C, self.T), "W")
         nbytes = _n.eqlinear_prepared_weight_bytes(self.handle)

@@ -149,7 +149,44 @@ def test_tcgen05_edge_shapes(T, N, C, D):
     assert _rel(Y, oracle.forward(T, inp["X"], inp["W"], inp["bias"])) <= TOL["f16"]
     dX = p.backward_input(_dev(inp["dY"]), Wh).double().cpu().numpy()
     assert _rel(dX, oracle.backward_input(T, inp["dY"], inp["W"])) <= TOL["f16"]
+    if T == 4:
+        assert p.backward_weight_kernel_name(N) == "tcgen05"
+        dW, db = p.backward_weight(_dev(inp["X"]), _dev(inp["dY"]))
+        rdW, rdb = oracle.backward_weight(T, inp["X"], inp["dY"], D)
+        assert _rel(dW.double().cpu().numpy(), rdW) <= TOL["f16"]
+        assert _rel(db.double().cpu().numpy(), rdb) <= TOL["f16"]
     assert p.status() == 0
+
+
+def test_tcgen05_weight_gradient_matches_simt():
+    """Both weight-gradient kernels on the same inputs (several row splits)."""
+    w = Workload("wgsimt", 4, 2000, 144, 272, "f16", True, 41)
+    inp = make_inputs(w, need_dy=True)
+    out = {}
+    for k in ("tcgen05", "simt"):
+        p = _plan(w, k)
+        assert p.backward_weight_kernel_name(w.N) == k
+        dW, db = p.backward_weight(_dev(inp["X"]), _dev(inp["dY"]))
+        assert p.status() == 0
+        out[k] = (dW.double().cpu().numpy(), db.double().cpu().numpy())
+    assert _rel(out["tcgen05"][0], out["simt"][0]) <= 1e-3
+    assert _rel(out["tcgen05"][1], out["simt"][1]) <= 1e-3
+
+
+def test_tcgen05_weight_gradient_many_units():
+    """More work units than SMs: each CTA runs several units back to back."""
+    w = Workload("wgmany", 4, 96, 2048, 2048, "f16", True, 43)
+    inp = make_inputs(w, need_dy=True)
+    p = _plan(w, "tcgen05")
+    dW, db = p.backward_weight(_dev(inp["X"]), _dev(inp["dY"]))
+    assert p.status() == 0
+    rng = np.random.default_rng(3)
+    dd = np.concatenate([rng.integers(0, w.D, 160), [0, w.D - 1]])
+    cc = np.concatenate([rng.integers(0, w.C, 160), [w.C - 1, 0]])
+    ref = oracle.backward_weight_pairs(w.T, inp["X"], inp["dY"], w.D, dd, cc)
+    assert _rel(dW.double().cpu().numpy()[dd, cc, :], ref) <= TOL["f16"]
+    ref_db = inp["dY"].astype(np.float64).reshape(w.N, w.D, w.T).sum(axis=(0, 2))
+    assert _rel(db.double().cpu().numpy(), ref_db) <= TOL["f16"]
 
 
 def test_tcgen05_matches_simt_bitwise_structure():
@@ -197,6 +234,7 @@ def test_backward_full_size_sampled():
     w = WORKLOADS["p4_vith_fc1_f16"]
     inp = make_inputs(w, need_dy=True)
     p = _plan(w)
+    assert p.backward_weight_kernel_name(w.N) == "tcgen05"
     Wh = p.prepare_weights(_dev(inp["W"]))
     dX = p.backward_input(_dev(inp["dY"]), Wh).double().cpu().numpy()
     dW, db = p.backward_weight(_dev(inp["X"]), _dev(inp["dY"]))
