@@ -456,6 +456,7 @@ def run_ours(args, workload):
                        "l2": f"{nsets} rotating input/output sets of {per_set / 2**20:.0f} MiB "
                              "(> 2x L2)",
                        "kernels": [f"{label}[{k}]" for label, k, _, _, _ in ops]},
+            "op_ms": [round(float(m), 5) for m in mean_ms],
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s",

@@ -47,7 +47,7 @@ namespace {
 using namespace tc;
 
 constexpr int BM = 128;          // rows per tile = MMA M
-constexpr int X_ST = 4;          // X ring: raw tile in, transformed operand planes out (in place)
+constexpr int X_ST = 3;          // X ring: raw tile in, transformed operand planes out (in place)
 constexpr uint32_t X_STAGE_BYTES = BM * 256;   // 128 rows x 256 B raw X per stage
 constexpr int kThreads = 640;
 constexpr int kEpiWarp0 = 4;     // warps 4..11: two per TMEM lane quarter
@@ -55,6 +55,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kXfWarp0 = 12;     // warps 12..19
 constexpr int kXfWarps = 8;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kStgBytes = 4096;  // per epilogue warp: 32 rows x 128 B of Y
 
 // Per-group shape of the pipeline.
 template <int T>
@@ -85,7 +86,9 @@ struct Shape : Cfg<T> {
   static constexpr uint32_t W_STAGE_BYTES = NPL * WREG_BYTES;
   static constexpr uint32_t OFF_X = 0;
   static constexpr uint32_t OFF_W = OFF_X + X_ST * X_STAGE_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_W + W_ST * W_STAGE_BYTES;
+  static constexpr uint32_t OFF_STG = OFF_W + W_ST * W_STAGE_BYTES;
+  static constexpr uint32_t OFF_BIAS = OFF_STG + kEpiWarps * kStgBytes;
+  static constexpr uint32_t OFF_BAR = OFF_BIAS + kEpiWarps * 128;
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers + alignment slack
   static_assert(NPL * PLANE_BYTES == X_STAGE_BYTES, "planes replace the raw tile in place");
   static_assert(BK * T * 2 == 256, "a raw stage row is two 128-byte chunks");
@@ -224,62 +227,79 @@ __device__ __forceinline__ void xf_write(uint8_t* slot, int xt, const uint4 (&v)
 }
 
 // ---------------------------------------------------------------------------
-// Epilogue of one 8-column group for the two rows (ra, rb) and the out-channel
-// pair (d, d+1) this lane owns; acc[plane][k]: k = 2*rr + hh (row rr, channel hh).
+// Epilogue of 32/T out-channels (starting at tile column c0 = out-channel d0)
+// for this lane's row: T accumulator planes -> inverse DFT + bias -> 64 bytes of
+// FP16 output (four 16-byte pieces, in Y's channel-major, group-minor order).
+// Plane p of out-channel c sits in TMEM column p * BD + c.
 // ---------------------------------------------------------------------------
-template <int T>
-__device__ __forceinline__ void epi_store(const uint32_t (&acc)[T][4], int64_t ra, int64_t rb,
-                                          int d, float2 bb, __half* __restrict__ Y, int64_t ldy,
-                                          int64_t N) {
+template <int T, int BD>
+__device__ __forceinline__ void epi_half(uint32_t lane_addr, int c0, const __half* bsm,
+                                         uint4 (&o)[4]) {
+  constexpr int NCH = 32 / T;
+  uint32_t v[T][NCH];
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int64_t row = rr ? rb : ra;
-    if (row >= N) continue;
-    if constexpr (T == 4) {
-      uint32_t packed[4];
+  for (int p = 0; p < T; ++p) tmem_ld_32x32b<NCH>(lane_addr + p * BD + c0, v[p]);
+  // the slice's biases (staged in shared memory before the accumulators were ready)
+  float b[NCH];
+  if constexpr (NCH == 8) {
+    const uint4 bb = *reinterpret_cast<const uint4*>(bsm);
+    const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int k = 2 * rr + hh;
-        const float y0 = __uint_as_float(acc[0][k]), y2 = __uint_as_float(acc[1][k]);
-        const float yr = __uint_as_float(acc[2][k]), yi = __uint_as_float(acc[3][k]);
-        const float b = hh ? bb.y : bb.x;
-        const float e = (y0 + y2) * 0.25f, o = (y0 - y2) * 0.25f;
-        const float re = yr * 0.5f, im = yi * 0.5f;
-        packed[2 * hh + 0] = pack_h2(e + re + b, o - im + b);
-        packed[2 * hh + 1] = pack_h2(e - re + b, o + im + b);
-      }
-      *reinterpret_cast<uint4*>(Y + row * ldy + (int64_t)d * T) =
-          make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    } else {
-      const float h4 = 0.70710678118654752f * 0.25f;
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = unpack_h2(bw[i]);
+      b[2 * i] = f.x;
+      b[2 * i + 1] = f.y;
+    }
+  } else {
+    const uint2 bb = *reinterpret_cast<const uint2*>(bsm);
+    const float2 f0 = unpack_h2(bb.x), f1 = unpack_h2(bb.y);
+    b[0] = f0.x; b[1] = f0.y; b[2] = f1.x; b[3] = f1.y;
+  }
+  tmem_wait_ld();
+  if constexpr (T == 4) {
+    // accumulators arrive scaled (Y0/4, Y2/4, Yr/2, Yi/2):
+    // y0 = Y0'+Y2'+Yr', y1 = Y0'-Y2'-Yi', y2 = Y0'+Y2'-Yr', y3 = Y0'-Y2'+Yi' (+ bias)
+    uint32_t w[2 * NCH];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int k = 2 * rr + hh;
-        float Yv[8];
+    for (int i = 0; i < NCH; ++i) {
+      const float s = __uint_as_float(v[0][i]) + b[i];
+      const float y2 = __uint_as_float(v[1][i]);
+      const float yr = __uint_as_float(v[2][i]), yi = __uint_as_float(v[3][i]);
+      const float e = s + y2, od = s - y2;
+      w[2 * i] = pack_h2(e + yr, od - yi);
+      w[2 * i + 1] = pack_h2(e - yr, od + yi);
+    }
 #pragma unroll
-        for (int p = 0; p < 8; ++p) Yv[p] = __uint_as_float(acc[p][k]);
-        const float b = hh ? bb.y : bb.x;
-        // y_s = A_s + B_s, y_{s+4} = A_s - B_s (A: frequencies 0, 2, 4; B: 1, 3)
-        const float E = (Yv[0] + Yv[1]) * 0.125f, O = (Yv[0] - Yv[1]) * 0.125f;
-        const float A0 = E + 0.25f * Yv[4], A2 = E - 0.25f * Yv[4];
-        const float A1 = O - 0.25f * Yv[5], A3 = O + 0.25f * Yv[5];
-        const float B0 = 0.25f * (Yv[2] + Yv[6]);
-        const float B1 = h4 * (Yv[2] - Yv[3] - Yv[6] - Yv[7]);
-        const float B2 = 0.25f * (Yv[7] - Yv[3]);
-        const float B3 = h4 * (-Yv[2] - Yv[3] + Yv[6] - Yv[7]);
-        const uint4 out = make_uint4(pack_h2(A0 + B0 + b, A1 + B1 + b), pack_h2(A2 + B2 + b, A3 + B3 + b),
-                                     pack_h2(A0 - B0 + b, A1 - B1 + b), pack_h2(A2 - B2 + b, A3 - B3 + b));
-        *reinterpret_cast<uint4*>(Y + row * ldy + (int64_t)(d + hh) * T) = out;
-      }
+    for (int m = 0; m < 4; ++m) o[m] = make_uint4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
+  } else {
+    // accumulators arrive scaled (frequencies 0 and 4 by 1/8, complex by 1/4);
+    // y_s = A_s + B_s, y_{s+4} = A_s - B_s (A: frequencies 0, 2, 4; B: 1, 3)
+    const float h = 0.70710678118654752f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      float Yv[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p) Yv[p] = __uint_as_float(v[p][i]);
+      const float s = Yv[0] + b[i];
+      const float E = s + Yv[1], O = s - Yv[1];
+      const float A0 = E + Yv[4], A2 = E - Yv[4];
+      const float A1 = O - Yv[5], A3 = O + Yv[5];
+      const float B0 = Yv[2] + Yv[6];
+      const float B1 = h * (Yv[2] - Yv[3] - Yv[6] - Yv[7]);
+      const float B2 = Yv[7] - Yv[3];
+      const float B3 = h * (-Yv[2] - Yv[3] + Yv[6] - Yv[7]);
+      o[i] = make_uint4(pack_h2(A0 + B0, A1 + B1), pack_h2(A2 + B2, A3 + B3),
+                        pack_h2(A0 - B0, A1 - B1), pack_h2(A2 - B2, A3 - B3));
     }
   }
 }
 
 template <int T>
 __global__ void __launch_bounds__(kThreads, 1)
-    eq_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, const uint8_t* __restrict__ wtiles,
-                     const __half* __restrict__ bias, __half* __restrict__ Y, int64_t N, int Cin,
-                     int Cout, TileInfo ti, int* status) {
+    eq_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x,
+                     const __grid_constant__ CUtensorMap map_y, const uint8_t* __restrict__ wtiles,
+                     const __half* __restrict__ bias, int64_t N, int Cin, int Cout, TileInfo ti,
+                     int* status) {
   using S = Shape<T>;
   constexpr int BD = S::BD;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -410,67 +430,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiWarps) {
     // ---------------- epilogue ----------------
-    // Warp w reads TMEM lane quarter q = w % 4 (rows 32q..32q+31) and column half
-    // ch (out-channels ch*BD/2 .. of the tile).  16x256b loads give lane t rows
-    // (t/4, t/4 + 8) of a 16-lane group and out-channel pair 2*(t%4) of each
-    // 8-channel group, so each warp store covers 8 rows x (8 channels x T x 2 B).
+    // Warp w reads TMEM lane quarter q = w % 4 (rows 32q..32q+31 of the tile) and
+    // out-channel half ch.  The half goes out in slices of 64/T out-channels: a
+    // slice row is 128 contiguous bytes of Y, staged in the warp's 4 KB buffer
+    // (128-byte swizzle) and written by one TMA store, so TMEM is free for the
+    // next tile as soon as its last slice is read, while the stores drain.
     const int q = warp & 3;
     const int ch = (warp - kEpiWarp0) >> 2;
+    uint8_t* stg = smem + S::OFF_STG + (warp - kEpiWarp0) * kStgBytes;
+    const uint32_t stg_s = smem_u32(stg);
+    uint8_t* my_row = stg + lane * 128;
+    __half* bsm = reinterpret_cast<__half*>(smem + S::OFF_BIAS + (warp - kEpiWarp0) * 128);
+    constexpr int kSliceCh = 64 / T;
+    constexpr int kSlices = (BD / 2) / kSliceCh;
     uint32_t tcount = 0;
-    const int64_t ldy = (int64_t)Cout * T;
-    const int tr = lane >> 2, tc = 2 * (lane & 3);
-    constexpr int kGroups = BD / 2 / 8;
     for (int tile = blockIdx.x; tile < ti.num_tiles; tile += gridDim.x, ++tcount) {
-      const int64_t rbase = (int64_t)(tile / ti.n_dt) * BM + 32 * q;
+      const int64_t row0 = (int64_t)(tile / ti.n_dt) * BM + 32 * q;
       const int dbase = (tile % ti.n_dt) * BD + (BD / 2) * ch;
-      // bias of this lane's out-channels, loaded while the mainloop runs
-      float2 bv[kGroups];
-#pragma unroll
-      for (int j = 0; j < kGroups; ++j) {
-        const int d = dbase + 8 * j + tc;
-        bv[j] = (bias && d < Cout) ? __half22float2(*reinterpret_cast<const __half2*>(bias + d))
-                                   : make_float2(0.f, 0.f);
+      // stage this warp's BD/2 biases while the mainloop runs (lane l: channels 2l, 2l+1)
+      if (2 * lane < BD / 2) {
+        const int d = dbase + 2 * lane;
+        uint32_t v = 0u;
+        if (bias && d < Cout) v = *reinterpret_cast<const uint32_t*>(bias + d);  // Cout even
+        reinterpret_cast<uint32_t*>(bsm)[lane] = v;
       }
+      __syncwarp();
       if (!warp_wait(&bars->acc_full, tcount & 1, abort_flag, status)) break;
       tc_fence_after();
+      const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {  // 16-lane groups of the quarter
-        const uint32_t laddr = tmem + ((uint32_t)(32 * q + 16 * h) << 16) + (BD / 2) * ch;
-        const int64_t row_a = rbase + 16 * h + tr, row_b = row_a + 8;
-        // T = 4: 16-column batches (.x2 loads, one wait per batch); T = 8: 8 columns
-        constexpr int kGB = (T == 4) ? 2 : 1;
+      for (int sc = 0; sc < kSlices; ++sc) {
+        const int c0 = (BD / 2) * ch + sc * kSliceCh;  // column in the tile
+        const int d0 = dbase + sc * kSliceCh;          // out-channel
+        if (d0 >= Cout) break;  // warp-uniform: Cout is a multiple of 16
+        const __half* bs = bsm + sc * kSliceCh;
+        uint4 o[4];
+        epi_half<T, BD>(lane_addr, c0, bs, o);
+        // the previous slice's store has finished reading the buffer
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
-        for (int jb = 0; jb < kGroups; jb += kGB) {
-          // accumulator columns of out-channel c: frequency plane p sits at
-          // (p / 2) * 2 BD + (p % 2) * BD + c
-          uint32_t raw[T][4 * kGB];
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<uint4*>(my_row + ((m ^ (lane & 7)) << 4)) = o[m];
+        epi_half<T, BD>(lane_addr, c0 + 32 / T, bs + 32 / T, o);
 #pragma unroll
-          for (int p = 0; p < T; ++p) {
-            const uint32_t col = laddr + (p >> 1) * 2 * BD + (p & 1) * BD + 8 * jb;
-            if constexpr (kGB == 2) {
-              EQL_TMEM_LD_16x256_X2(col, raw[p]);
-            } else {
-              EQL_TMEM_LD_16x256(col, raw[p]);
-            }
-          }
-          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-          for (int g = 0; g < kGB; ++g) {
-            const int j = jb + g;
-            const int d = dbase + 8 * j + tc;
-            if (d >= Cout) continue;  // warp-uniform: Cout is a multiple of 16
-            uint32_t acc[T][4];
-#pragma unroll
-            for (int p = 0; p < T; ++p)
-#pragma unroll
-              for (int k = 0; k < 4; ++k) acc[p][k] = raw[p][4 * g + k];
-            epi_store<T>(acc, row_a, row_b, d, bv[j], Y, ldy, N);
-          }
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<uint4*>(my_row + (((4 + m) ^ (lane & 7)) << 4)) = o[m];
+        // generic-proxy writes -> visible to the TMA (async proxy), then one store
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          if (row0 < N) tma_store_3d(&map_y, stg_s, 0, d0 * T / 64, (int)row0);
+          bulk_commit();
         }
       }
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   } else if (warp >= kXfWarp0) {
     // ---------------- transform: group DFT into the operand planes ----------------
     const int xt = threadIdx.x - kXfWarp0 * 32;  // 0..255
@@ -526,8 +544,15 @@ __global__ void tile_weights_kernel(const __half* __restrict__ planes, int Cin, 
   const int dt = (int)(blob / n_ks), ks = (int)(blob % n_ks);
   const int d = dt * S::BD + r, c0 = ks * S::BK + piece * 8;
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
-  if (d < Cout && c0 < Cin)  // Cin % 16 == 0: the 8 channels are all in range
+  if (d < Cout && c0 < Cin) {  // Cin % 16 == 0: the 8 channels are all in range
     v = *reinterpret_cast<const uint4*>(planes + ((int64_t)region * Cout + d) * Cin + c0);
+    // the inverse DFT's factors 1/T (real frequencies) and 2/T (complex), exact
+    // powers of two, applied here so the epilogue needs no multiplies by them
+    const __half2 s = __float2half2_rn(region < 2 ? 1.f / T : 2.f / T);
+    __half2* h = reinterpret_cast<__half2*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __hmul2(h[i], s);
+  }
   // swizzle: piece ^= (byte offset of the row >> 7) within the swizzle span
   const int swz = ((r * S::ROWB) >> 7) & (kPieces - 1);
   const int64_t dst_byte = blob * S::W_STAGE_BYTES + (int64_t)region * S::WREG_BYTES +
@@ -584,6 +609,7 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           int num_sms, int drop_w_stage, cudaStream_t st) {
   if (!fwd_tc_supported(T, DType::F16, N, Cin, Cout)) return cudaErrorNotSupported;
   if (!Wtiles) return cudaErrorNotSupported;
+
   auto encode = encode_fn();
   if (!encode) return cudaErrorNotSupported;
   return dispatch_tc(T, [&](auto tcst) {
@@ -597,6 +623,16 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
     cuuint32_t estr[3] = {1, 1, 1};
     if (encode(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(X), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    // Y row = Cout*T/64 chunks of 128 B; store box = 1 chunk x 32 rows
+    CUtensorMap my;
+    cuuint64_t ydims[3] = {64, (cuuint64_t)Cout * TT / 64, (cuuint64_t)N};
+    cuuint64_t ystrides[2] = {128, (cuuint64_t)Cout * TT * 2};
+    cuuint32_t ybox[3] = {64, 1, 32};
+    if (encode(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, Y, ydims, ystrides, ybox, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
@@ -617,8 +653,8 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
     }
     const int grid = ti.num_tiles < num_sms ? ti.num_tiles : num_sms;
     eq_fwd_tc_kernel<TT><<<grid, kThreads, S::SMEM_BYTES, st>>>(
-        mx, static_cast<const uint8_t*>(Wtiles), static_cast<const __half*>(bias),
-        static_cast<__half*>(Y), N, Cin, Cout, ti, status);
+        mx, my, static_cast<const uint8_t*>(Wtiles), static_cast<const __half*>(bias), N, Cin,
+        Cout, ti, status);
     return cudaGetLastError();
   });
 }
