@@ -268,8 +268,8 @@ eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t p, const void* X, con
     s = from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, part, bpart, splits, p->status,
                                        p->num_sms, st));
     if (s != EQL_OK) return s;
-    return from_cuda(eql::launch_wgrad_finalize(p->T, to_dt(p->dtype), part, bpart, splits,
-                                                p->C, p->D, dW, dbias, p->tw, st));
+    return from_cuda(eql::launch_wgrad_tc_finalize(part, bpart, splits, p->C, p->D, dW, dbias,
+                                                   p->tw, st));
   }
   const int splits = eql::wgrad_simt_splits(p->T, N, p->C, p->D, p->num_sms);
   return from_cuda(eql::launch_wgrad_simt(p->T, to_dt(p->dtype), X, dY, N, p->C, p->D, dW,

@@ -56,12 +56,15 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           int num_sms, int drop_w_stage, cudaStream_t st);
 
 // tcgen05/TMEM tensor-core weight gradient for T = 4, FP16: FP32 partial
-// spectra part[splits][4][D][C] and bias partials bpart[splits][D] (the layout
-// launch_wgrad_finalize reads).  X and dY must be 16-byte aligned (TMA).
+// spectra part[splits][4][C][D] and bias partials bpart[splits][D], finished by
+// launch_wgrad_tc_finalize.  X and dY must be 16-byte aligned (TMA).
 bool wgrad_tc_supported(int T, DType dt, int64_t N, int C, int D, const void* X, const void* dY);
 int wgrad_tc_splits(int64_t N, int C, int D, int num_sms);
 size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms);
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D, float* part,
                             float* bpart, int splits, int* status, int num_sms, cudaStream_t st);
+cudaError_t launch_wgrad_tc_finalize(const float* part, const float* bpart, int splits, int C,
+                                     int D, void* dW, void* dbias, const Twiddles& tw,
+                                     cudaStream_t st);
 
 }  // namespace eql

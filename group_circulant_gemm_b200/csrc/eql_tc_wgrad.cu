@@ -8,9 +8,10 @@
 //   Q0 = G0^T Xh0,  Q2 = G2^T Xh2,
 //   Qr = Gr^T Xr + Gi^T Xi,  Qi = Gr^T Xi - Gi^T Xr        (D x C each, K = rows)
 // summed over the row range of one work unit and stored as the FP32 partial
-// planes part[split][4][D][C]; dbias partials are the FP32 column sums of G0.
-// A finalize kernel (shared with the CUDA-core path) adds the splits in a fixed
-// order, applies the inverse group DFT and casts, so the result is deterministic.
+// planes part[split][4][C][D] (out-channel fastest, so each warp store writes 32
+// consecutive floats); dbias partials are the FP32 column sums of G0.  A
+// finalize kernel adds the splits in a fixed order, applies the inverse group
+// DFT and casts, so the result is deterministic.
 //
 // Design (one persistent CTA per SM; work unit = 128 out-channels x 128
 // in-channels x one row range; stage = 32 rows):
@@ -20,12 +21,14 @@
 //               in-channel, K = row.  Per K step (16 rows): N = 128 for Q0 and
 //               Q2, N = 256 for Gr [Xr|Xi], N = 128 for Gi Xi and (negated A)
 //               Gi Xr.
-//   warps 4-11  epilogue: tcgen05.ld of the four accumulators, FP32 stores of
-//               the partial planes.
-//   warps 12-19 transform: each thread takes 8 rows x one channel pair, forms
-//               the group DFT in FP32, rounds once to FP16 and writes it
-//               transposed (rows become the K dimension) as K-major 64-byte
-//               swizzled operand planes over the raw tile it came from.
+//   warps 4-7   epilogue: tcgen05.ld of the four accumulators (one out-channel
+//               per lane), FP32 stores of the partial planes.
+//   warps 8-23  transform, two groups of 8 warps working on the same stage in
+//               parallel (8-15: the dY tile, 16-23: the X tile): each thread takes
+//               8 rows x one channel pair, forms the group DFT in FP32, rounds once
+//               to FP16 and writes it transposed (rows become the K dimension) as
+//               K-major 64-byte swizzled operand planes over the raw tile it came
+//               from.
 // TMEM (512 columns): Q0 at [0,128), Q2 at [128,256), Qr at [256,384), Qi at
 // [384,512).  Every mbarrier wait is bounded (about 2 s); on expiry the CTA sets
 // the plan's status word, drains what it issued and returns.
@@ -49,9 +52,9 @@ constexpr uint32_t WG_ROWB = WG_BR * 2;      // operand row: 32 rows of K, FP16
 constexpr uint32_t WG_PLANE = 128 * WG_ROWB; // one operand plane (128 channels)
 constexpr uint32_t WG_OFF_BAR = WG_ST * WG_STAGE;
 constexpr uint32_t WG_SMEM = WG_OFF_BAR + 512 + 1024;
-constexpr int WG_THREADS = 640;
-constexpr int WG_EPI0 = 4, WG_EPIW = 8;      // warps 4..11
-constexpr int WG_XF0 = 12, WG_XFW = 8;       // warps 12..19
+constexpr int WG_THREADS = 768;
+constexpr int WG_EPI0 = 4, WG_EPIW = 4;      // warps 4..7: one per TMEM lane quarter
+constexpr int WG_XF0 = 8, WG_XFW = 8;        // warps 8..15 (dY tile), 16..23 (X tile)
 static_assert(4 * WG_PLANE == WG_TILE, "planes replace the raw tile in place");
 static_assert(WG_SMEM <= 232448, "shared memory budget");
 
@@ -165,7 +168,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->read_g[s], WG_XFW);
       mbar_init(&bars->read_x[s], WG_XFW);
-      mbar_init(&bars->ready[s], WG_XFW);
+      mbar_init(&bars->ready[s], 2 * WG_XFW);
       mbar_init(&bars->empty[s], 1);
     }
     mbar_init(&bars->acc_full, 1);
@@ -254,10 +257,10 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     __syncwarp();
   } else if (warp >= WG_EPI0 && warp < WG_EPI0 + WG_EPIW) {
     // ---------------- epilogue: accumulators -> FP32 partial planes ----------------
-    // Warp w reads TMEM lane quarter q = w % 4 (out-channels 32q..32q+31 of the
-    // unit) and planes 2h, 2h+1; 32x32b loads give each lane one out-channel and
-    // 16 consecutive in-channels.
-    const int q = warp & 3, h = (warp - WG_EPI0) >> 2;
+    // Warp w reads TMEM lane quarter q = w % 4: lane l holds out-channel
+    // 32q + l; a 32x32b load gives it 16 consecutive in-channels of one plane,
+    // and each of the 16 stores writes 32 consecutive out-channels (128 B).
+    const int q = warp & 3;
     uint32_t ucount = 0;
     for (int u = blockIdx.x; u < wi.num_units; u += gridDim.x, ++ucount) {
       const Unit un = decode(u, wi, N);
@@ -266,27 +269,19 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       const int d = un.dt * WG_BD + 32 * q + lane;
       const uint32_t lrow = tmem + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
-      for (int pl = 0; pl < 2; ++pl) {
-        const int p = 2 * h + pl;
+      for (int p = 0; p < 4; ++p) {
         float* dst_plane = part + ((int64_t)un.z * 4 + p) * D * C;
 #pragma unroll 1
         for (int gq = 0; gq < WG_BC / 16; ++gq) {
-          uint32_t r[16];
-          asm volatile(
-              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,"
-              "%12,%13,%14,%15}, [%16];"
-              : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
-                "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-              : "r"(lrow + p * WG_BC + 16 * gq));
-          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
           const int c = un.ct * WG_BC + 16 * gq;
-          if (d < D && c < C) {  // C % 16 == 0: the 16 columns are all in range
-            float4* o = reinterpret_cast<float4*>(dst_plane + (int64_t)d * C + c);
+          if (c >= C) break;  // warp-uniform; C % 16 == 0: the 16 columns are all in range
+          uint32_t r[16];
+          tmem_ld_32x32b<16>(lrow + p * WG_BC + 16 * gq, r);
+          tmem_wait_ld();
+          if (d < D) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              o[k] = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
-                                 __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+            for (int k = 0; k < 16; ++k)
+              dst_plane[(int64_t)(c + k) * D + d] = __uint_as_float(r[k]);
           }
         }
       }
@@ -295,7 +290,8 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     }
   } else if (warp >= WG_XF0) {
     // ---------------- transform: group DFT, transposed into the operand planes ----------------
-    const int w = warp - WG_XF0;  // 0..7: raw chunk = channel pairs 8w..8w+7
+    const int grp = (warp - WG_XF0) >> 3;  // 0: dY tile (and the dbias sums), 1: X tile
+    const int w = (warp - WG_XF0) & 7;     // raw chunk = channel pairs 8w..8w+7
     const int j = lane & 7, q = lane >> 3;
     uint32_t it = 0;
     bool ok = true;
@@ -307,10 +303,11 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
         const uint32_t ph = (it / WG_ST) & 1;
         if (!(ok = warp_wait(&bars->full[slot], ph, abort_flag, status))) break;
         uint8_t* st = smem + slot * WG_STAGE;
-        wg_transform<true>(st, w, j, q, &bars->read_g[slot], ph, bsum, ok, abort_flag, status);
-        if (!ok) break;
-        wg_transform<false>(st + WG_TILE, w, j, q, &bars->read_x[slot], ph, unused, ok,
-                            abort_flag, status);
+        if (grp == 0)
+          wg_transform<true>(st, w, j, q, &bars->read_g[slot], ph, bsum, ok, abort_flag, status);
+        else
+          wg_transform<false>(st + WG_TILE, w, j, q, &bars->read_x[slot], ph, unused, ok,
+                              abort_flag, status);
         if (!ok) break;
         // make the generic-proxy stores visible to the tensor core (async proxy)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -324,7 +321,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
         bsum[e] += __shfl_xor_sync(0xffffffffu, bsum[e], 8);
         bsum[e] += __shfl_xor_sync(0xffffffffu, bsum[e], 16);
       }
-      if (un.ct == 0 && q == 0) {
+      if (grp == 0 && un.ct == 0 && q == 0) {
         const int d = un.dt * WG_BD + 2 * (8 * w + j);
         if (d < D) bpart[(int64_t)un.z * D + d] = bsum[0];
         if (d + 1 < D) bpart[(int64_t)un.z * D + d + 1] = bsum[1];
@@ -337,6 +334,34 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+// Sum of the split partials (fixed order), inverse group DFT, cast:
+// dW[d][c][u] from part[split][4][C][D]; dbias[d] from bpart[split][D].
+__global__ void wgrad_tc_finalize_kernel(const float* __restrict__ part,
+                                         const float* __restrict__ bpart, int splits, int C, int D,
+                                         __half* __restrict__ dW, __half* __restrict__ dbias,
+                                         Twiddles tw) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // c * D + d
+  const int64_t plane = (int64_t)D * C;
+  if (idx < plane) {
+    float qv[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int z = 0; z < splits; ++z) {
+#pragma unroll
+      for (int p = 0; p < 4; ++p) qv[p] += part[((int64_t)z * 4 + p) * plane + idx];
+    }
+    float wv[4];
+    group_idft<4>(qv, wv, tw);
+    const int64_t c = idx / D, d = idx % D;
+    __half2* out = reinterpret_cast<__half2*>(dW + (d * C + c) * 4);
+    out[0] = __floats2half2_rn(wv[0], wv[1]);
+    out[1] = __floats2half2_rn(wv[2], wv[3]);
+  }
+  if (dbias && idx < D) {
+    float b = 0.f;
+    for (int z = 0; z < splits; ++z) b += bpart[(int64_t)z * D + idx];
+    dbias[idx] = __float2half_rn(b);
   }
 }
 
@@ -380,6 +405,17 @@ int wgrad_tc_splits(int64_t N, int C, int D, int num_sms) {
 size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms) {
   const int s = wgrad_tc_splits(N, C, D, num_sms);
   return (size_t)std::max(s, 1) * ((size_t)4 * C * D + D) * sizeof(float);
+}
+
+cudaError_t launch_wgrad_tc_finalize(const float* part, const float* bpart, int splits, int C,
+                                     int D, void* dW, void* dbias, const Twiddles& tw,
+                                     cudaStream_t st) {
+  const int64_t total = std::max<int64_t>((int64_t)C * D, D);
+  const unsigned blocks = (unsigned)((total + 255) / 256);
+  wgrad_tc_finalize_kernel<<<blocks, 256, 0, st>>>(part, bpart, splits, C, D,
+                                                    static_cast<__half*>(dW),
+                                                    static_cast<__half*>(dbias), tw);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D, float* part,
