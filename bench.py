@@ -74,20 +74,33 @@ def layer_bytes(w) -> float:
 # from the ncu captures summarised in profiles/, valid only for the kernel source
 # they were taken on (SHA-256 prefix of csrc/eql_tc_fwd.cu); any other source
 # reports null.
+# DRAM bytes (read + write) per launch of the step's dominant kernel, from the
+# ncu captures summarised under profiles/, keyed by a hash of the kernel's
+# sources: a changed kernel reports null until it is captured again.
+KERNEL_SOURCES = {
+    "forward": ("eql_tc_fwd.cu", "eql_tc_common.cuh"),
+    "backward_weight": ("eql_tc_wgrad.cu", "eql_tc_common.cuh"),
+}
 NCU_TRAFFIC = {
-    "86ba56eb36e4696e": {"p4_vitb_mlp_f16": 64.73e6, "c8_1024_f16": 34.20e6},
+    ("forward", "ae950bd8670fee35"): {"p4_vitb_mlp_f16": 61.63e6, "c8_1024_f16": 35.61e6,
+                                      "p4_vith_fc1_fwd_bwd_f16": 69.94e6},
+    ("backward_weight", "bfa7d6c1a4d80534"): {"p4_vith_fc1_fwd_bwd_f16": 108.84e6},
 }
 
 
-def kernel_traffic(workload: str):
+def kernel_traffic(family: str, workload: str):
     import hashlib
-    path = os.path.join(ROOT, "group_circulant_gemm_b200", "csrc", "eql_tc_fwd.cu")
+    files = KERNEL_SOURCES.get(family)
+    if not files:
+        return None
+    m = hashlib.sha256()
     try:
-        with open(path, "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()[:16]
+        for f in files:
+            with open(os.path.join(ROOT, "group_circulant_gemm_b200", "csrc", f), "rb") as fh:
+                m.update(fh.read())
     except OSError:
         return None
-    return NCU_TRAFFIC.get(h, {}).get(workload)
+    return NCU_TRAFFIC.get((family, m.hexdigest()[:16]), {}).get(workload)
 
 
 def load_peaks():
@@ -421,7 +434,7 @@ def run_ours(args, workload):
         if dkern == "tcgen05":
             peak = peaks["bf16_tflops"]
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": kernel_traffic(workload),
+                    "frac": achieved / peak, "traffic": kernel_traffic(dlabel, workload),
                     "peak_source": f"{peak_src} dense bf16 burst (fp16 runs at the same rate)"}
         else:
             # CUDA-core FP32 FMA peak: 148 SMs x 128 FMA/clk x 2 FLOP x max SM clock

@@ -115,10 +115,12 @@ EQL_API const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t plan, i
  * (even T); Re and Im of each complex frequency k = 1..n_cplx; then -Im of each
  * complex frequency.  Forward planes hold conj(DFT(W)) (the correlation form of
  * the convolution theorem), adjoint planes hold DFT(W) transposed, used for dX.
- * For T = 4 FP16 plans with C and D multiples of 8 two more blocks follow: the
- * forward and adjoint planes re-arranged as the tensor-core kernel's operand
- * tiles (one contiguous blob per 128 out-channels x 16 in-channels, in the
- * kernel's swizzled shared-memory order), so each pipeline stage is one copy.
+ * For FP16 plans with T = 4 or 8 and C, D multiples of 16 two more blocks
+ * follow: the forward and adjoint planes re-arranged as the tensor-core
+ * kernel's operand tiles (one contiguous blob per out-channel tile and K stage:
+ * 128 x 32 channels at T = 4, 64 x 16 at T = 8, in the kernel's swizzled
+ * shared-memory order, scaled by the inverse DFT's factors 1/T and 2/T), so each
+ * pipeline stage is one copy.
  */
 EQL_API size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t plan);
 
@@ -154,7 +156,7 @@ EQL_API eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t plan, const vo
                                           const void* W_hat, void* dX, void* stream);
 
 /* Workspace bytes eqlinear_backward_weight needs for N rows (FP32 partial
- * spectra of the split reduction over rows). */
+ * spectra of the split reduction over rows; large enough for either kernel). */
 EQL_API size_t eqlinear_backward_weight_workspace_bytes(eqlinear_plan_t plan, int64_t N);
 
 /*
@@ -162,7 +164,10 @@ EQL_API size_t eqlinear_backward_weight_workspace_bytes(eqlinear_plan_t plan, in
  *   dW[d][c][u] = sum_{n,s} dY[n, d*T+s] * X[n, c*T + (s+u) mod T]
  *   dbias[d]    = sum_{n,s} dY[n, d*T+s]
  * computed per frequency as a reduction over the N rows (FP32, fixed order, so
- * results are bitwise reproducible for a given N), then one inverse DFT.
+ * results are bitwise reproducible for a given N), then one inverse DFT.  FP16
+ * plans with T = 4, C and D multiples of 16 and 16-byte aligned X and dY run on
+ * the tensor cores (the group DFTs of X and dY rounded once to FP16, FP32
+ * accumulation); other plans on CUDA cores in FP32.
  *   X [N][C*T], dY [N][D*T], dW [D][C][T] (plan dtype, overwritten),
  *   dbias [D] or NULL, workspace >= eqlinear_backward_weight_workspace_bytes.
  * N = 0 writes zeros to dW and dbias.
