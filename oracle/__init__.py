@@ -74,6 +74,8 @@ def _load():
             lib.eqlo_backward_weight_pairs.argtypes = [ctypes.c_int, i64, i64, i64, dp, dp,
                                                        i64, lp, lp, dp]
             lib.eqlo_backward_weight_pairs.restype = None
+            lib.eqlo_gelu.argtypes = [i64, dp]
+            lib.eqlo_gelu.restype = None
             lib.eqlo_p4_transform_matrices.argtypes = [dp, dp]
             lib.eqlo_p4_transform_matrices.restype = None
             _lib = lib
@@ -99,15 +101,28 @@ def _shapes(T: int, X: np.ndarray, W: np.ndarray):
     return X.shape[0], C, D
 
 
-def forward(T: int, X, W, bias=None, return_macs: bool = False):
-    """Y[N, D*T] in float64 from X[N, C*T], W[D, C, T], bias[D] or None."""
+def forward(T: int, X, W, bias=None, return_macs: bool = False, act: str = "none"):
+    """Y[N, D*T] in float64 from X[N, C*T], W[D, C, T], bias[D] or None;
+    act="gelu" applies the exact GELU to every output feature (EQ-MLP block)."""
+    if act not in ("none", "gelu"):
+        raise ValueError(f"unknown activation {act!r}")
     lib = _load()
     X, W = _f64(X), _f64(W)
     N, C, D = _shapes(T, X, W)
     b = None if bias is None else _f64(bias)
     Y = np.empty((N, D * T), dtype=np.float64)
     macs = lib.eqlo_forward(T, N, C, D, _ptr(X), _ptr(W), _ptr(b), _ptr(Y))
+    if act == "gelu":
+        lib.eqlo_gelu(Y.size, _ptr(Y))
     return (Y, macs) if return_macs else Y
+
+
+def gelu(y):
+    """The activation alone, elementwise, in float64 (for pins and composition)."""
+    lib = _load()
+    y = _f64(y).copy()
+    lib.eqlo_gelu(y.size, _ptr(y))
+    return y
 
 
 def forward_spectral(T: int, X, W, bias=None, return_macs: bool = False):

@@ -68,6 +68,16 @@ int64_t eqlo_forward(int T, int64_t N, int64_t C, int64_t D, const double* X, co
   return N * D * T * C * T;
 }
 
+/* The EQ-MLP block's activation, applied elementwise to a forward output:
+ * GELU(y) = y * Phi(y) = 0.5 * y * (1 + erf(y / sqrt(2))), the exact (erf) form.
+ * A pointwise function of each output feature commutes with the cyclic shift of
+ * the group axis, so the block stays equivariant ("Key insight"; the pages'
+ * network-level models are ViT/Swin, whose MLP blocks use this activation). */
+void eqlo_gelu(int64_t n, double* y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) y[i] = 0.5 * y[i] * (1.0 + erf(y[i] / sqrt(2.0)));
+}
+
 /* Gradient of the forward with respect to X:
  *   dX[n,c,t] = sum_{d,s} dY[n,d,s] * W[d,c,(t-s) mod T]. */
 int64_t eqlo_backward_input(int T, int64_t N, int64_t C, int64_t D, const double* dY,

@@ -242,3 +242,33 @@ def test_pins_catch_planted_index_mistake(oracle_mod):
     wrong = np.array([[sum(W[0, 0, (s - t) % T] * X[0, t] for t in range(T)) for s in range(T)]])
     assert not np.allclose(wrong, oracle_mod.forward(T, X, W, None))
     np.testing.assert_array_equal(oracle_mod.forward(T, X, W, None), [[5, 8, 11, 6]])
+
+
+# --- the EQ-MLP block's activation (exact GELU) ------------------------------------
+
+def test_gelu_matches_normal_cdf_closed_form(oracle_mod):
+    """GELU(y) = y * Phi(y): pinned to scipy's normal CDF, an independent routine."""
+    from scipy.special import ndtr
+    y = np.concatenate([np.linspace(-8.0, 8.0, 161), [0.0, 1.0, -1.0, 1e-8, -30.0, 30.0]])
+    ref = y * ndtr(y)
+    got = oracle_mod.gelu(y)
+    assert np.max(np.abs(got - ref)) <= 1e-14
+    assert got[-6] == 0.0 and abs(got[-5] - 0.8413447460685429) < 1e-15
+    assert abs(got[-2]) < 1e-190  # GELU(-30) = -30 * Phi(-30), about -1.5e-196
+    assert got[-1] == 30.0
+
+
+def test_forward_gelu_is_gelu_of_forward_and_equivariant(oracle_mod):
+    rng = np.random.default_rng(21)
+    T, N, C, D = 4, 9, 5, 6
+    X = rng.standard_normal((N, C * T))
+    W = rng.standard_normal((D, C, T)) / np.sqrt(C * T)
+    b = 0.1 * rng.standard_normal(D)
+    from scipy.special import ndtr
+    plain = oracle_mod.forward(T, X, W, b)
+    Y = oracle_mod.forward(T, X, W, b, act="gelu")
+    assert np.max(np.abs(Y - plain * ndtr(plain))) <= 1e-14
+    for r in range(T):
+        Xr = np.roll(X.reshape(N, C, T), r, axis=2).reshape(N, C * T)
+        Yr = oracle_mod.forward(T, Xr, W, b, act="gelu")
+        assert np.max(np.abs(Yr - np.roll(Y.reshape(N, D, T), r, axis=2).reshape(N, D * T))) <= 1e-12
