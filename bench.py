@@ -10,7 +10,7 @@ from pinned host memory and the result read back, inside the timed region.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
        [--workload p4_vitb_mlp_f16|p4_vitb_proj_f32|p4_vith_fc1_f16|c8_1024_f16|
-                   p4_vith_fc1_fwd_bwd_f16]
+                   p4_vith_fc1_fwd_bwd_f16|p4_vitb_mlp_block_f16]
 Under torchrun (N > 1) every rank runs its own copy of the workload (weak
 scaling; rows are independent, so no collective is on the data path).
 """
@@ -42,8 +42,15 @@ PIPELINES = {
     "p4_vith_fc1_f16": ["p4_vith_fc1_f16"],
     "c8_1024_f16": ["c8_1024_f16"],
     "p4_vith_fc1_fwd_bwd_f16": ["p4_vith_fc1_f16"],
+    "p4_vitb_mlp_block_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
 }
 BACKWARD = {"p4_vith_fc1_fwd_bwd_f16"}
+# per-layer output activation (fused into that layer's epilogue); default none
+ACTS = {"p4_vitb_mlp_block_f16": ["gelu", "none"]}
+
+
+def acts_of(workload):
+    return ACTS.get(workload, ["none"] * len(PIPELINES[workload]))
 DESCR = {
     "p4_vitb_mlp_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
                        "C=768->D=192, T=4",
@@ -52,6 +59,8 @@ DESCR = {
     "c8_1024_f16": "cyclic T=8 EQ-Linear fp16: N=16384, C=D=128",
     "p4_vith_fc1_fwd_bwd_f16": "p4 EQ-Linear fp16 ViT-H fc1 forward + dX + dW: N=8224, "
                                "C=320->D=1280, T=4",
+    "p4_vitb_mlp_block_f16": "p4 EQ-MLP block fp16 ViT-B: N=12608, EQ-Linear 192->768 + bias + "
+                             "GELU (fused), EQ-Linear 768->192 + bias, T=4",
 }
 
 
@@ -197,16 +206,17 @@ def dist_init():
     return world, rank, local
 
 
-def oracle_sample(pipeline, rows: int, backward: bool = False):
+def oracle_sample(pipeline, rows: int, backward: bool = False, acts=None):
     """Time the float64 oracle on `rows` rows of the step's ops; returns (seconds, rows)."""
     import oracle
     oracle.build()
     layers = [(WORKLOADS[name], make_inputs(WORKLOADS[name], rows=rows, need_dy=backward))
               for name in pipeline]
+    acts = acts or ["none"] * len(layers)
     x = layers[0][1]["X"].astype(np.float64)
     t0 = time.perf_counter()
-    for w, inp in layers:
-        x = oracle.forward(w.T, x, inp["W"], inp["bias"])
+    for (w, inp), act in zip(layers, acts):
+        x = oracle.forward(w.T, x, inp["W"], inp["bias"], act=act)
     if backward:
         w, inp = layers[0]
         oracle.backward_input(w.T, inp["dY"], inp["W"])
@@ -214,8 +224,8 @@ def oracle_sample(pipeline, rows: int, backward: bool = False):
     return time.perf_counter() - t0, rows
 
 
-def calibrated_oracle_rows(pipeline, target_s: float, backward: bool = False) -> int:
-    t, r = oracle_sample(pipeline, 16, backward)
+def calibrated_oracle_rows(pipeline, target_s: float, backward: bool = False, acts=None) -> int:
+    t, r = oracle_sample(pipeline, 16, backward, acts)
     n_full = WORKLOADS[pipeline[0]].N
     return int(max(16, min(n_full, 16 * target_s / max(t, 1e-6))))
 
@@ -229,10 +239,11 @@ def run_reference(args, workload):
     pipeline = PIPELINES[workload]
     backward = workload in BACKWARD
     per_step_s = max(1.0, 120.0 / max(1, args.steps + args.warmup))
-    rows = calibrated_oracle_rows(pipeline, min(per_step_s, 20.0), backward)
+    acts = acts_of(workload)
+    rows = calibrated_oracle_rows(pipeline, min(per_step_s, 20.0), backward, acts)
     for _ in range(args.warmup):
-        oracle_sample(pipeline, rows, backward)
-    times = [oracle_sample(pipeline, rows, backward)[0] for _ in range(args.steps)]
+        oracle_sample(pipeline, rows, backward, acts)
+    times = [oracle_sample(pipeline, rows, backward, acts)[0] for _ in range(args.steps)]
     total = sum(times)
     value = rows * args.steps / total
     w0 = WORKLOADS[pipeline[0]]
@@ -255,6 +266,76 @@ def run_reference(args, workload):
 
 def wgrad_flops(w) -> float:
     return layer_flops(w)  # same per-frequency products, reduced over rows
+
+
+def dense_flops(w) -> float:
+    return 2.0 * w.N * (w.C * w.T) * (w.D * w.T)
+
+
+def dense_comparator(pipeline, backward, xs, dys, nsets, steps, rank, acts=None):
+    """Same-GPU dense baseline: torch F.linear (cuBLAS) on the replicated
+    (D*T x C*T) matrix M[(d,s),(c,t)] = W[d,c,(t-s) mod T] in the same dtype, GEMM
+    time only (M built outside the timed region); for the training step also
+    dX = dY M and the dense weight-gradient GEMM dY^T X."""
+    import torch
+    import torch.nn.functional as F
+    stream = torch.cuda.current_stream()
+    Ms, bs = [], []
+    for w in pipeline:
+        inp = make_inputs(w.with_(seed=w.seed + 1000 * rank), rows=1)
+        W = torch.from_numpy(inp["W"]).cuda()
+        M = torch.empty((w.D, w.T, w.C, w.T), dtype=W.dtype, device="cuda")
+        for sh in range(w.T):
+            M[:, sh] = torch.roll(W, shifts=sh, dims=2)
+        Ms.append(M.reshape(w.D * w.T, w.C * w.T))
+        bs.append(torch.from_numpy(inp["bias"]).cuda().repeat_interleave(w.T) if w.bias else None)
+    outs = []
+
+    def step(i, events=None):
+        def mark():
+            if events is not None:
+                events.append(torch.cuda.Event(enable_timing=True))
+                events[-1].record(stream)
+        x = xs[i % nsets]
+        for li in range(len(pipeline)):
+            mark()
+            x = F.linear(x, Ms[li], bs[li])
+            if acts and acts[li] == "gelu":
+                x = F.gelu(x)
+            mark()
+        if backward:
+            dy = dys[i % nsets]
+            mark()
+            dx = dy @ Ms[0]
+            mark()
+            mark()
+            dw = dy.t() @ xs[i % nsets]
+            mark()
+            del dx, dw
+        del x
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    ev = []
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        step(3 + i, ev)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    nops = len(ev) // 2 // steps
+    op_ms = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1])
+                      for j in range(len(ev) // 2)]).reshape(steps, nops).mean(axis=0)
+    flops = sum(dense_flops(w) for w in pipeline) + (2 * dense_flops(pipeline[0]) if backward else 0)
+    return {"kind": "dense F.linear on the replicated (D*T x C*T) matrix, cuBLAS, same dtype, "
+                    "GEMM time only" + ("; training step adds dY@M and dY^T@X" if backward else "")
+                    + ("; F.gelu after the layers that fuse it" if acts and "gelu" in acts else ""),
+            "value": pipeline[0].N / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "op_ms": [round(float(m), 5) for m in op_ms],
+            "tflops": flops / (ms / 1e3) / 1e12}
 
 
 def run_ours(args, workload):
@@ -307,10 +388,11 @@ def run_ours(args, workload):
 
     # the ops of one step: (label, kernel, flops, algorithmic bytes, callable(set index))
     ops = []
+    acts = acts_of(workload)
     for li, w in enumerate(pipeline):
         def fwd(i, li=li):
             x = xs[i % nsets] if li == 0 else outs[i % nsets][li - 1]
-            plans[li].forward(x, whats[li], biases[li], out=outs[i % nsets][li])
+            plans[li].forward(x, whats[li], biases[li], out=outs[i % nsets][li], act=acts[li])
         ops.append(("forward", plans[li].forward_kernel_name(N), layer_flops(w), layer_bytes(w),
                     fwd))
     if backward:
@@ -448,11 +530,16 @@ def run_ours(args, workload):
         roof["launch_ms"] = mean_launch_ms
         roof["kernel"] = f"eqlinear_{dlabel}[{dkern}]"
         roof["step_share"] = dms / float(mean_ms.sum())
+        comparator = None
+        if not args.no_dense:
+            comparator = dense_comparator(pipeline, backward, xs, dys if backward else None,
+                                          nsets, min(args.steps, 200), rank, acts)
+            comparator["ours_over_dense"] = value / comparator["value"]
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             import oracle
-            rows = calibrated_oracle_rows(PIPELINES[workload], 10.0, backward)
-            secs, rows = oracle_sample(PIPELINES[workload], rows, backward)
+            rows = calibrated_oracle_rows(PIPELINES[workload], 10.0, backward, acts_of(workload))
+            secs, rows = oracle_sample(PIPELINES[workload], rows, backward, acts_of(workload))
             cpu = {"value": rows / secs, "unit": "tokens/s", "cores": oracle.threads_used(),
                    "kind": "oracle",
                    "sample": f"{rows} of {N} rows through every op of the step, float64, "
@@ -464,6 +551,9 @@ def run_ours(args, workload):
             "scaling": "weak", "vs_baseline": None,
             "dtype": "f16" if dt == torch.float16 else "f32", "data": "synthetic",
             "tflops": flops * args.steps * world / (elapsed_ms / 1e3) / 1e12,
+            "tflops_dense_equiv": (sum(dense_flops(w) for w in pipeline)
+                                   + (2 * dense_flops(pipeline[0]) if backward else 0))
+                                  * args.steps * world / (elapsed_ms / 1e3) / 1e12,
             "config": {"workload": DESCR[workload], "global_batch": N * world, "seq_len": None,
                        "parallelism": f"replicas x{world} (rows independent)",
                        "l2": f"{nsets} rotating input/output sets of {per_set / 2**20:.0f} MiB "
@@ -472,6 +562,7 @@ def run_ours(args, workload):
             "op_ms": [round(float(m), 5) for m in mean_ms],
             "roofline": roof,
             "cpu_baseline": cpu,
+            "dense_comparator": comparator,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
             "gpu_launches": args.steps * sum(2 if label == "backward_weight" else 1
@@ -495,6 +586,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(PIPELINES), default="p4_vitb_mlp_f16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense F.linear comparator")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps, reported as run
     if args.impl == "reference":

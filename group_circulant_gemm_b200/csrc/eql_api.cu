@@ -69,14 +69,14 @@ const void* adj_tiles(const eqlinear_plan_s* p, const void* W_hat) {
 //   other : planes [P][Cin][Cout]  (CUDA-core operand)
 eqlinear_status_t run_forward_like(eqlinear_plan_s* p, const void* X, int64_t N, int Cin,
                                    int Cout, const void* tiles, const void* other,
-                                   const void* bias, void* Y, cudaStream_t st) {
+                                   const void* bias, void* Y, int act, cudaStream_t st) {
   const bool tc_ok = has_tiles(p) && eql::fwd_tc_supported(p->T, to_dt(p->dtype), N, Cin, Cout);
   if (p->kernel == EQL_KERNEL_TCGEN05 && !tc_ok) return EQL_ERR_UNSUPPORTED;
   if (p->kernel != EQL_KERNEL_SIMT && tc_ok)
     return from_cuda(eql::launch_fwd_tc(p->T, X, N, Cin, Cout, tiles, bias, Y, p->status,
-                                        p->num_sms, p->debug_drop_w_stage, st));
+                                        p->num_sms, p->debug_drop_w_stage, act, st));
   return from_cuda(eql::launch_fwd_simt(p->T, to_dt(p->dtype), X, N, Cin, Cout, other, bias, Y,
-                                        p->tw, st));
+                                        p->tw, act, st));
 }
 
 eqlinear_status_t check_plan_device(const eqlinear_plan_s* p) {
@@ -212,7 +212,14 @@ eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, voi
 
 eqlinear_status_t eqlinear_forward(eqlinear_plan_t p, const void* X, int64_t N,
                                    const void* W_hat, const void* bias, void* Y, void* stream) {
+  return eqlinear_forward_act(p, X, N, W_hat, bias, EQL_ACT_NONE, Y, stream);
+}
+
+eqlinear_status_t eqlinear_forward_act(eqlinear_plan_t p, const void* X, int64_t N,
+                                       const void* W_hat, const void* bias, eqlinear_act_t act,
+                                       void* Y, void* stream) {
   if (!p || N < 0) return EQL_ERR_INVALID_ARG;
+  if (act != EQL_ACT_NONE && act != EQL_ACT_GELU) return EQL_ERR_INVALID_ARG;
   if (N == 0) return EQL_OK;
   if (!X || !W_hat || !Y) return EQL_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(W_hat) || !aligned16(Y) || (bias && !aligned16(bias)))
@@ -220,7 +227,7 @@ eqlinear_status_t eqlinear_forward(eqlinear_plan_t p, const void* X, int64_t N,
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
   return run_forward_like(p, X, N, p->C, p->D, fwd_tiles(p, W_hat), adj_block(p, W_hat), bias,
-                          Y, (cudaStream_t)stream);
+                          Y, (int)act, (cudaStream_t)stream);
 }
 
 eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int64_t N,
@@ -234,7 +241,7 @@ eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int
   // dX is the forward-shaped product with the adjoint weights: input width D,
   // output width C; the CUDA-core path reads the forward block [P][D][C].
   return run_forward_like(p, dY, N, p->D, p->C, adj_tiles(p, W_hat), fwd_block(p, W_hat),
-                          nullptr, dX, (cudaStream_t)stream);
+                          nullptr, dX, 0, (cudaStream_t)stream);
 }
 
 // Enough for either kernel, so the size does not depend on which one runs.

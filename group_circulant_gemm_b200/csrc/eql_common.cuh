@@ -100,4 +100,37 @@ __device__ __forceinline__ void group_idft(const float (&p)[T], float (&y)[T], c
   }
 }
 
+// Output activation of the EQ-MLP block: 0 = none, 1 = GELU (exact erf form),
+// y * Phi(y) = 0.5 y (1 + erf(y / sqrt 2)), in FP32 before the output rounding.
+// A pointwise function of each output feature commutes with the group shift.
+// erf is evaluated with Abramowitz & Stegun, Handbook of Mathematical Functions,
+// formula 7.1.26 (|error| <= 1.5e-7 on the whole line):
+//   1 - erf(x) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2),
+//   t = 1 / (1 + p x), x >= 0, with erf(-x) = -erf(x),
+// which gives 1 + erf(x) without cancellation on the negative side.
+__device__ __forceinline__ float gelu_erf(float y) {
+  const float x = fabsf(y) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, x, 1.0f));
+  float q = fmaf(t, 1.061405429f, -1.453152027f);
+  q = fmaf(t, q, 1.421413741f);
+  q = fmaf(t, q, -0.284496736f);
+  q = fmaf(t, q, 0.254829592f);
+  const float r = t * q * __expf(-x * x);  // 1 - erf(|y| / sqrt 2)
+  return 0.5f * y * (y >= 0.f ? 2.0f - r : r);
+}
+
+template <int ACT>
+__device__ __forceinline__ float act_fn(float y) {
+  if constexpr (ACT == 1) {
+    return gelu_erf(y);
+  } else {
+    return y;
+  }
+}
+
+// Runtime-selected form for the CUDA-core kernels.
+__device__ __forceinline__ float apply_act(float y, int act) {
+  return act == 1 ? gelu_erf(y) : y;
+}
+
 }  // namespace eql

@@ -20,9 +20,10 @@ cudaError_t launch_prepare(int T, DType dt, const void* W, int C, int D, void* f
 //   X [N][Cin*T] -> Y [N][Cout*T]; Wt = planes [P][Cin][Cout] of the OTHER block
 //   (adjoint block for the forward pass, forward block for dX): the kernel takes
 //   Re from the Re planes and Im from the "-Im" slots, which hold the right sign.
+// act: output activation (0 none, 1 GELU), applied after the bias.
 cudaError_t launch_fwd_simt(int T, DType dt, const void* X, int64_t N, int Cin, int Cout,
                             const void* Wt, const void* bias, void* Y, const Twiddles& tw,
-                            cudaStream_t st);
+                            int act, cudaStream_t st);
 
 // CUDA-core weight gradient: split reduction over rows into FP32 partial spectra,
 // then a finalize kernel (sum in fixed split order, inverse DFT, cast).
@@ -53,7 +54,7 @@ bool fwd_tc_supported(int T, DType dt, int64_t N, int Cin, int Cout);
 // so its bounded waits expire and the kernel reports a timeout.
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
-                          int num_sms, int drop_w_stage, cudaStream_t st);
+                          int num_sms, int drop_w_stage, int act, cudaStream_t st);
 
 // tcgen05/TMEM tensor-core weight gradient for T = 4, FP16: FP32 partial
 // spectra part[splits][4][C][D] and bias partials bpart[splits][D], finished by

@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(const In* __restrict__ X,
                                                        int Cin, int Cout,
                                                        const In* __restrict__ Wt,
                                                        const In* __restrict__ bias,
-                                                       In* __restrict__ Y, Twiddles tw) {
+                                                       In* __restrict__ Y, Twiddles tw, int act) {
   using S = Spec<T>;
   using G = SimtTile<T>;
   __shared__ __align__(16) float xs[T][G::BK][G::XS];
@@ -224,7 +224,8 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(const In* __restrict__ X,
       group_idft<T>(acc[m][dd], y, tw);
       const float b = bias ? to_f32(bias[d]) : 0.f;
 #pragma unroll
-      for (int s = 0; s < T; ++s) Y[row * ldy + (int64_t)d * T + s] = from_f32<In>(y[s] + b);
+      for (int s = 0; s < T; ++s)
+        Y[row * ldy + (int64_t)d * T + s] = from_f32<In>(apply_act(y[s] + b, act));
     }
   }
 }
@@ -418,7 +419,7 @@ cudaError_t launch_prepare(int T, DType dt, const void* W, int C, int D, void* f
 
 cudaError_t launch_fwd_simt(int T, DType dt, const void* X, int64_t N, int Cin, int Cout,
                             const void* Wt, const void* bias, void* Y, const Twiddles& tw,
-                            cudaStream_t st) {
+                            int act, cudaStream_t st) {
   if (N == 0) return cudaSuccess;
   return dispatch_T(T, [&](auto tc) {
     constexpr int TT = decltype(tc)::value;
@@ -429,11 +430,11 @@ cudaError_t launch_fwd_simt(int T, DType dt, const void* X, int64_t N, int Cin, 
     if (dt == DType::F32)
       fwd_simt_kernel<TT, float><<<grid, 256, 0, st>>>((const float*)X, N, Cin, Cout,
                                                        (const float*)Wt, (const float*)bias,
-                                                       (float*)Y, tw);
+                                                       (float*)Y, tw, act);
     else
       fwd_simt_kernel<TT, __half><<<grid, 256, 0, st>>>((const __half*)X, N, Cin, Cout,
                                                         (const __half*)Wt, (const __half*)bias,
-                                                        (__half*)Y, tw);
+                                                        (__half*)Y, tw, act);
     return cudaGetLastError();
   });
 }

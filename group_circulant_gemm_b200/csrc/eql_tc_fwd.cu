@@ -232,7 +232,7 @@ __device__ __forceinline__ void xf_write(uint8_t* slot, int xt, const uint4 (&v)
 // FP16 output (four 16-byte pieces, in Y's channel-major, group-minor order).
 // Plane p of out-channel c sits in TMEM column p * BD + c.
 // ---------------------------------------------------------------------------
-template <int T, int BD>
+template <int T, int BD, int ACT>
 __device__ __forceinline__ void epi_half(uint32_t lane_addr, int c0, const __half* bsm,
                                          uint4 (&o)[4]) {
   constexpr int NCH = 32 / T;
@@ -266,8 +266,8 @@ __device__ __forceinline__ void epi_half(uint32_t lane_addr, int c0, const __hal
       const float y2 = __uint_as_float(v[1][i]);
       const float yr = __uint_as_float(v[2][i]), yi = __uint_as_float(v[3][i]);
       const float e = s + y2, od = s - y2;
-      w[2 * i] = pack_h2(e + yr, od - yi);
-      w[2 * i + 1] = pack_h2(e - yr, od + yi);
+      w[2 * i] = pack_h2(act_fn<ACT>(e + yr), act_fn<ACT>(od - yi));
+      w[2 * i + 1] = pack_h2(act_fn<ACT>(e - yr), act_fn<ACT>(od + yi));
     }
 #pragma unroll
     for (int m = 0; m < 4; ++m) o[m] = make_uint4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
@@ -288,13 +288,15 @@ __device__ __forceinline__ void epi_half(uint32_t lane_addr, int c0, const __hal
       const float B1 = h * (Yv[2] - Yv[3] - Yv[6] - Yv[7]);
       const float B2 = Yv[7] - Yv[3];
       const float B3 = h * (-Yv[2] - Yv[3] + Yv[6] - Yv[7]);
-      o[i] = make_uint4(pack_h2(A0 + B0, A1 + B1), pack_h2(A2 + B2, A3 + B3),
-                        pack_h2(A0 - B0, A1 - B1), pack_h2(A2 - B2, A3 - B3));
+      o[i] = make_uint4(pack_h2(act_fn<ACT>(A0 + B0), act_fn<ACT>(A1 + B1)),
+                        pack_h2(act_fn<ACT>(A2 + B2), act_fn<ACT>(A3 + B3)),
+                        pack_h2(act_fn<ACT>(A0 - B0), act_fn<ACT>(A1 - B1)),
+                        pack_h2(act_fn<ACT>(A2 - B2), act_fn<ACT>(A3 - B3)));
     }
   }
 }
 
-template <int T>
+template <int T, int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     eq_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                      const __grid_constant__ CUtensorMap map_y, const uint8_t* __restrict__ wtiles,
@@ -465,14 +467,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (d0 >= Cout) break;  // warp-uniform: Cout is a multiple of 16
         const __half* bs = bsm + sc * kSliceCh;
         uint4 o[4];
-        epi_half<T, BD>(lane_addr, c0, bs, o);
+        epi_half<T, BD, ACT>(lane_addr, c0, bs, o);
         // the previous slice's store has finished reading the buffer
         if (lane == 0) bulk_wait_read_all();
         __syncwarp();
 #pragma unroll
         for (int m = 0; m < 4; ++m)
           *reinterpret_cast<uint4*>(my_row + ((m ^ (lane & 7)) << 4)) = o[m];
-        epi_half<T, BD>(lane_addr, c0 + 32 / T, bs + 32 / T, o);
+        epi_half<T, BD, ACT>(lane_addr, c0 + 32 / T, bs + 32 / T, o);
 #pragma unroll
         for (int m = 0; m < 4; ++m)
           *reinterpret_cast<uint4*>(my_row + (((4 + m) ^ (lane & 7)) << 4)) = o[m];
@@ -606,7 +608,7 @@ cudaError_t launch_tile_weights(int T, const void* planes, int Cin, int Cout, vo
 
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
-                          int num_sms, int drop_w_stage, cudaStream_t st) {
+                          int num_sms, int drop_w_stage, int act, cudaStream_t st) {
   if (!fwd_tc_supported(T, DType::F16, N, Cin, Cout)) return cudaErrorNotSupported;
   if (!Wtiles) return cudaErrorNotSupported;
 
@@ -645,14 +647,16 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
     ti.drop_w = drop_w_stage;
     static bool attr_set = false;
     if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute(eq_fwd_tc_kernel<TT>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           S::SMEM_BYTES);
-      if (e != cudaSuccess) return e;
+      for (auto fn : {eq_fwd_tc_kernel<TT, 0>, eq_fwd_tc_kernel<TT, 1>}) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             S::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+      }
       attr_set = true;
     }
     const int grid = ti.num_tiles < num_sms ? ti.num_tiles : num_sms;
-    eq_fwd_tc_kernel<TT><<<grid, kThreads, S::SMEM_BYTES, st>>>(
+    auto kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1> : eq_fwd_tc_kernel<TT, 0>;
+    kernel<<<grid, kThreads, S::SMEM_BYTES, st>>>(
         mx, my, static_cast<const uint8_t*>(Wtiles), static_cast<const __half*>(bias), N, Cin,
         Cout, ti, status);
     return cudaGetLastError();

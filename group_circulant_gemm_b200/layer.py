@@ -59,14 +59,20 @@ class EqLinearPlan:
         _n.eqlinear_prepare_weights(self.handle, W, out)
         return out
 
-    def forward(self, X, W_hat, bias=None, out=None) -> torch.Tensor:
+    def forward(self, X, W_hat, bias=None, out=None, act: str = "none") -> torch.Tensor:
+        """Y = act(EQ-Linear(X) + bias); act is "none" or "gelu" (fused in the epilogue)."""
         N = X.shape[0]
         self._check(X, (N, self.C * self.T), "X")
         if bias is not None:
             self._check(bias, (self.D,), "bias")
+        if act not in _n.ACT:
+            raise ValueError(f"unknown activation {act!r}")
         if out is None:
             out = torch.empty((N, self.D * self.T), dtype=self.dtype, device=X.device)
-        _n.eqlinear_forward(self.handle, X, N, W_hat, bias, out)
+        if act == "none":
+            _n.eqlinear_forward(self.handle, X, N, W_hat, bias, out)
+        else:
+            _n.eqlinear_forward_act(self.handle, X, N, W_hat, bias, _n.ACT[act], out)
         return out
 
     def backward_input(self, dY, W_hat, out=None) -> torch.Tensor:

@@ -24,7 +24,8 @@ EXPORTED = (
     "eqlinear_version", "eqlinear_status_string", "eqlinear_plan_create",
     "eqlinear_plan_destroy", "eqlinear_plan_set_kernel", "eqlinear_forward_kernel_name",
     "eqlinear_backward_weight_kernel_name", "eqlinear_prepared_weight_bytes",
-    "eqlinear_prepare_weights", "eqlinear_forward", "eqlinear_backward_input",
+    "eqlinear_prepare_weights", "eqlinear_forward", "eqlinear_forward_act",
+    "eqlinear_backward_input",
     "eqlinear_backward_weight_workspace_bytes", "eqlinear_backward_weight",
     "eqlinear_get_status", "eqlinear_backward_weight_noalloc",
 )
@@ -54,6 +55,7 @@ def _load() -> ctypes.CDLL:
         "eqlinear_prepared_weight_bytes": ([vp], sz),
         "eqlinear_prepare_weights": ([vp, vp, vp, vp], i32),
         "eqlinear_forward": ([vp, vp, i64, vp, vp, vp, vp], i32),
+        "eqlinear_forward_act": ([vp, vp, i64, vp, vp, i32, vp, vp], i32),
         "eqlinear_backward_input": ([vp, vp, i64, vp, vp, vp], i32),
         "eqlinear_backward_weight_workspace_bytes": ([vp, i64], sz),
         "eqlinear_backward_weight": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
@@ -135,6 +137,14 @@ def eqlinear_prepare_weights(plan: int, W, W_hat, stream=None) -> None:
 def eqlinear_forward(plan: int, X, N: int, W_hat, bias, Y, stream=None) -> None:
     _check(_lib.eqlinear_forward(plan, _ptr(X), N, _ptr(W_hat), _ptr(bias), _ptr(Y),
                                  _stream(stream)), "eqlinear_forward")
+
+
+ACT = {"none": 0, "gelu": 1}
+
+
+def eqlinear_forward_act(plan: int, X, N: int, W_hat, bias, act: int, Y, stream=None) -> None:
+    _check(_lib.eqlinear_forward_act(plan, _ptr(X), N, _ptr(W_hat), _ptr(bias), act, _ptr(Y),
+                                     _stream(stream)), "eqlinear_forward_act")
 
 
 def eqlinear_backward_input(plan: int, dY, N: int, W_hat, dX, stream=None) -> None:

@@ -146,6 +146,28 @@ EQL_API eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t plan, const v
 EQL_API eqlinear_status_t eqlinear_forward(eqlinear_plan_t plan, const void* X, int64_t N,
                                    const void* W_hat, const void* bias, void* Y, void* stream);
 
+/* Output activation applied by eqlinear_forward_act. */
+typedef enum {
+  EQL_ACT_NONE = 0,
+  EQL_ACT_GELU = 1  /* GELU(y) = y * Phi(y) = 0.5 y (1 + erf(y / sqrt 2)), exact erf form */
+} eqlinear_act_t;
+
+/*
+ * Forward pass with an elementwise activation fused into the epilogue, the
+ * first half of an EQ-MLP block (the pages' network-level Flash EQ-ViT/Swin
+ * models stack EQ-Linear layers in MLP blocks, "Results / network level"):
+ *   Y[n, d*T+s] = act(bias[d] + sum_{c,t} W[d][c][(t-s) mod T] * X[n, c*T+t])
+ * A pointwise function of each output feature commutes with the cyclic shift
+ * of the group axis, so the block stays equivariant.  The activation runs in
+ * FP32 on the accumulated value and is followed by the single rounding to the
+ * plan dtype.  Same arguments, layouts and errors as eqlinear_forward, plus
+ * EQL_ERR_INVALID_ARG for an unknown act.  eqlinear_forward is this call with
+ * EQL_ACT_NONE.
+ */
+EQL_API eqlinear_status_t eqlinear_forward_act(eqlinear_plan_t plan, const void* X, int64_t N,
+                                               const void* W_hat, const void* bias,
+                                               eqlinear_act_t act, void* Y, void* stream);
+
 /*
  * Gradient with respect to the input ("Implementation": backward pass):
  *   dX[n, c*T+t] = sum_{d,s} dY[n, d*T+s] * W[d][c][(t-s) mod T]

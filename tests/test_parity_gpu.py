@@ -292,3 +292,55 @@ def test_error_paths():
                      Wh.data_ptr(), None, ws.data_ptr(), 16, st)
     assert s == n.EQL_ERR_WORKSPACE
     assert p.status() == 0
+
+
+# --- fused activation (EQ-MLP block: EQ-Linear + bias + GELU in the epilogue) ------
+
+ACT_CASES = [
+    # T, N, C, D, dtype, kernel
+    (4, 333, 192, 768, "f16", "tcgen05"),
+    (4, 261, 80, 208, "f16", "tcgen05"),
+    (8, 389, 128, 128, "f16", "tcgen05"),
+    (4, 256, 16, 16, "f32", "simt"),
+    (3, 129, 7, 33, "f16", "simt"),
+]
+
+
+@pytest.mark.parametrize("T,N,C,D,dtype,kernel", ACT_CASES)
+def test_forward_gelu_matches_oracle(T, N, C, D, dtype, kernel):
+    w = Workload("act", T, N, C, D, dtype, True, 900 + T + N)
+    inp = make_inputs(w)
+    p = _plan(w, kernel)
+    assert p.forward_kernel_name(N) == kernel
+    Wh = p.prepare_weights(_dev(inp["W"]))
+    Y = p.forward(_dev(inp["X"]), Wh, _dev(inp["bias"]), act="gelu")
+    assert p.status() == 0
+    ref = oracle.forward(T, inp["X"], inp["W"], inp["bias"], act="gelu")
+    assert _rel(Y.double().cpu().numpy(), ref) <= TOL[dtype]
+
+
+def test_forward_gelu_equivariant_on_gpu():
+    w = Workload("acteq", 4, 512, 64, 128, "f16", True, 77)
+    inp = make_inputs(w)
+    p = _plan(w)
+    Wh = p.prepare_weights(_dev(inp["W"]))
+    N, C, D, T = w.N, w.C, w.D, w.T
+    X = inp["X"]
+    Y = p.forward(_dev(X), Wh, _dev(inp["bias"]), act="gelu").float().cpu().numpy()
+    for r in range(1, T):
+        Xr = np.roll(X.reshape(N, C, T), r, axis=2).reshape(N, C * T)
+        Yr = p.forward(_dev(Xr), Wh, _dev(inp["bias"]), act="gelu").float().cpu().numpy()
+        Yroll = np.roll(Y.reshape(N, D, T), r, axis=2).reshape(N, D * T)
+        assert np.max(np.abs(Yr - Yroll)) <= TOL["f16"] * np.max(np.abs(Y))
+
+
+def test_forward_act_rejects_unknown_activation():
+    from group_circulant_gemm_b200 import native as n
+    w = Workload("actbad", 4, 16, 16, 16, "f16", True, 3)
+    p = _plan(w)
+    X = torch.zeros((16, 64), dtype=torch.float16, device="cuda")
+    Y = torch.empty((16, 64), dtype=torch.float16, device="cuda")
+    Wh = p.prepare_weights(_dev(make_inputs(w)["W"]))
+    s = n.raw_status("eqlinear_forward_act", p.handle, X.data_ptr(), 16, Wh.data_ptr(), None, 7,
+                     Y.data_ptr(), None)
+    assert s == 1  # EQL_ERR_INVALID_ARG
