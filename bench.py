@@ -91,11 +91,10 @@ KERNEL_SOURCES = {
     "backward_weight": ("eql_tc_wgrad.cu", "eql_tc_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("forward", "ae950bd8670fee35"): {"p4_vitb_mlp_f16": 61.63e6, "c8_1024_f16": 35.61e6,
-                                      "p4_vith_fc1_fwd_bwd_f16": 69.94e6},
+    ("forward", "e01149104234b8ee"): {"p4_vitb_mlp_f16": 58.94e6, "c8_1024_f16": 34.02e6,
+                                      "p4_vith_fc1_fwd_bwd_f16": 70.12e6},
     ("backward_weight", "bfa7d6c1a4d80534"): {"p4_vith_fc1_fwd_bwd_f16": 108.84e6},
 }
-
 
 def kernel_traffic(family: str, workload: str):
     import hashlib
@@ -538,7 +537,7 @@ def run_ours(args, workload):
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             import oracle
-            rows = calibrated_oracle_rows(PIPELINES[workload], 10.0, backward, acts_of(workload))
+            rows = calibrated_oracle_rows(PIPELINES[workload], 15.0, backward, acts_of(workload))
             secs, rows = oracle_sample(PIPELINES[workload], rows, backward, acts_of(workload))
             cpu = {"value": rows / secs, "unit": "tokens/s", "cores": oracle.threads_used(),
                    "kind": "oracle",
