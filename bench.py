@@ -10,7 +10,7 @@ from pinned host memory and the result read back, inside the timed region.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
        [--workload p4_vitb_mlp_f16|p4_vitb_proj_f32|p4_vith_fc1_f16|c8_1024_f16|
-                   p4_vith_fc1_fwd_bwd_f16|p4_vitb_mlp_block_f16]
+                   p4_vith_fc1_fwd_bwd_f16|p4_vitb_mlp_block_f16|p4_vitb_mlp_spectral_f16]
 Under torchrun (N > 1) every rank runs its own copy of the workload (weak
 scaling; rows are independent, so no collective is on the data path).
 """
@@ -43,7 +43,11 @@ PIPELINES = {
     "c8_1024_f16": ["c8_1024_f16"],
     "p4_vith_fc1_fwd_bwd_f16": ["p4_vith_fc1_f16"],
     "p4_vitb_mlp_block_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
+    "p4_vitb_mlp_spectral_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
 }
+# two-layer pipelines whose intermediate stays in the frequency domain (the first
+# layer's epilogue writes the second layer's operand planes)
+SPECTRAL = {"p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectral_f16"}
 BACKWARD = {"p4_vith_fc1_fwd_bwd_f16"}
 # per-layer output activation (fused into that layer's epilogue); default none
 ACTS = {"p4_vitb_mlp_block_f16": ["gelu", "none"]}
@@ -60,7 +64,11 @@ DESCR = {
     "p4_vith_fc1_fwd_bwd_f16": "p4 EQ-Linear fp16 ViT-H fc1 forward + dX + dW: N=8224, "
                                "C=320->D=1280, T=4",
     "p4_vitb_mlp_block_f16": "p4 EQ-MLP block fp16 ViT-B: N=12608, EQ-Linear 192->768 + bias + "
-                             "GELU (fused), EQ-Linear 768->192 + bias, T=4",
+                             "GELU (fused), EQ-Linear 768->192 + bias, T=4; intermediate kept as "
+                             "the second layer's spectral planes",
+    "p4_vitb_mlp_spectral_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
+                                "C=768->D=192, T=4; intermediate kept as the second layer's "
+                                "spectral planes",
 }
 
 
@@ -388,10 +396,23 @@ def run_ours(args, workload):
     # the ops of one step: (label, kernel, flops, algorithmic bytes, callable(set index))
     ops = []
     acts = acts_of(workload)
+    spectral = workload in SPECTRAL
+    if spectral:
+        # the first layer writes the second layer's input planes [4, N, H]
+        outs = [[torch.empty((4, N, pipeline[0].D), dtype=dt, device="cuda"), o[1]]
+                for o in outs]
     for li, w in enumerate(pipeline):
         def fwd(i, li=li):
             x = xs[i % nsets] if li == 0 else outs[i % nsets][li - 1]
-            plans[li].forward(x, whats[li], biases[li], out=outs[i % nsets][li], act=acts[li])
+            if spectral and li == 0:
+                plans[li].forward_to_spectral(x, whats[li], biases[li], act=acts[li],
+                                              out=outs[i % nsets][li])
+            elif spectral and li == 1:
+                plans[li].forward_from_spectral(x, whats[li], biases[li], act=acts[li],
+                                                out=outs[i % nsets][li])
+            else:
+                plans[li].forward(x, whats[li], biases[li], out=outs[i % nsets][li],
+                                  act=acts[li])
         ops.append(("forward", plans[li].forward_kernel_name(N), layer_flops(w), layer_bytes(w),
                     fwd))
     if backward:

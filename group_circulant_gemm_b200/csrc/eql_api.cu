@@ -74,7 +74,7 @@ eqlinear_status_t run_forward_like(eqlinear_plan_s* p, const void* X, int64_t N,
   if (p->kernel == EQL_KERNEL_TCGEN05 && !tc_ok) return EQL_ERR_UNSUPPORTED;
   if (p->kernel != EQL_KERNEL_SIMT && tc_ok)
     return from_cuda(eql::launch_fwd_tc(p->T, X, N, Cin, Cout, tiles, bias, Y, p->status,
-                                        p->num_sms, p->debug_drop_w_stage, act, st));
+                                        p->num_sms, p->debug_drop_w_stage, act, 0, st));
   return from_cuda(eql::launch_fwd_simt(p->T, to_dt(p->dtype), X, N, Cin, Cout, other, bias, Y,
                                         p->tw, act, st));
 }
@@ -228,6 +228,46 @@ eqlinear_status_t eqlinear_forward_act(eqlinear_plan_t p, const void* X, int64_t
   if (s != EQL_OK) return s;
   return run_forward_like(p, X, N, p->C, p->D, fwd_tiles(p, W_hat), adj_block(p, W_hat), bias,
                           Y, (int)act, (cudaStream_t)stream);
+}
+
+static bool spectral_ok(eqlinear_plan_t p, int64_t N) {
+  return p->T == 4 && p->dtype == EQL_F16 && p->kernel != EQL_KERNEL_SIMT && has_tiles(p) &&
+         eql::fwd_tc_supported(p->T, to_dt(p->dtype), N, p->C, p->D);
+}
+
+size_t eqlinear_spectral_bytes(eqlinear_plan_t p, int64_t N) {
+  if (!p || N < 0) return 0;
+  return (size_t)4 * (size_t)N * (size_t)p->D * 2;
+}
+
+static eqlinear_status_t forward_spectral_io(eqlinear_plan_t p, const void* X, int64_t N,
+                                             const void* W_hat, const void* bias,
+                                             eqlinear_act_t act, void* Y, int io, void* stream) {
+  if (!p || N < 0) return EQL_ERR_INVALID_ARG;
+  if (act != EQL_ACT_NONE && act != EQL_ACT_GELU) return EQL_ERR_INVALID_ARG;
+  if (N == 0) return EQL_OK;
+  if (!X || !W_hat || !Y) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_hat) || !aligned16(Y) || (bias && !aligned16(bias)))
+    return EQL_ERR_ALIGNMENT;
+  if (!spectral_ok(p, N)) return EQL_ERR_UNSUPPORTED;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_fwd_tc(p->T, X, N, p->C, p->D, fwd_tiles(p, W_hat), bias, Y,
+                                      p->status, p->num_sms, p->debug_drop_w_stage, (int)act, io,
+                                      (cudaStream_t)stream));
+}
+
+eqlinear_status_t eqlinear_forward_to_spectral(eqlinear_plan_t p, const void* X, int64_t N,
+                                               const void* W_hat, const void* bias,
+                                               eqlinear_act_t act, void* Xhat_next,
+                                               void* stream) {
+  return forward_spectral_io(p, X, N, W_hat, bias, act, Xhat_next, 1, stream);
+}
+
+eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t p, const void* Xhat, int64_t N,
+                                                 const void* W_hat, const void* bias,
+                                                 eqlinear_act_t act, void* Y, void* stream) {
+  return forward_spectral_io(p, Xhat, N, W_hat, bias, act, Y, 2, stream);
 }
 
 eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int64_t N,

@@ -52,9 +52,12 @@ cudaError_t launch_tile_weights(int T, const void* planes /* [P][Cout][Cin] */, 
 bool fwd_tc_supported(int T, DType dt, int64_t N, int Cin, int Cout);
 // drop_w_stage >= 0 is a test-only fault: CTA 0 never issues that weight stage,
 // so its bounded waits expire and the kernel reports a timeout.
+// io (T = 4 only beyond 0): 0 = spatial X and Y; 1 = Y written as the next
+// layer's spectral planes [4][N][Cout] (the group DFT of act(y): X0, X2, Xr, Xi);
+// 2 = X read as spectral planes [4][N][Cin] produced that way.
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
-                          int num_sms, int drop_w_stage, int act, cudaStream_t st);
+                          int num_sms, int drop_w_stage, int act, int io, cudaStream_t st);
 
 // tcgen05/TMEM tensor-core weight gradient for T = 4, FP16: FP32 partial
 // spectra part[splits][4][C][D] and bias partials bpart[splits][D], finished by

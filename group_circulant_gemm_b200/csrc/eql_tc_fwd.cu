@@ -56,6 +56,9 @@ constexpr int kXfWarp0 = 12;     // warps 12..19
 constexpr int kXfWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kStgBytes = 4096;  // per epilogue warp: 32 rows x 128 B of Y
+// Input/output forms (T = 4): spatial X and Y; Y written as the next layer's
+// spectral operand planes; X read as spectral operand planes.
+constexpr int kIoSpatial = 0, kIoSpectralOut = 1, kIoSpectralIn = 2;
 
 // Per-group shape of the pipeline.
 template <int T>
@@ -296,7 +299,47 @@ __device__ __forceinline__ void epi_half(uint32_t lane_addr, int c0, const __hal
   }
 }
 
-template <int T, int ACT>
+// T = 4 epilogue of 8 out-channels written as the NEXT layer's input in the
+// frequency domain: per channel the four outputs y_s = act(IDFT + bias) are
+// transformed again, X0 = y0+y1+y2+y3, X2 = y0-y1+y2-y3, Xr = y0-y2, Xi = y3-y1
+// (FP32, one rounding to FP16); o[p] = plane p of the 8 channels (16 bytes).
+template <int BD, int ACT>
+__device__ __forceinline__ void epi_half_spec(uint32_t lane_addr, int c0, const __half* bsm,
+                                              uint4 (&o)[4]) {
+  uint32_t v[4][8];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) tmem_ld_32x32b<8>(lane_addr + p * BD + c0, v[p]);
+  const uint4 bb = *reinterpret_cast<const uint4*>(bsm);
+  const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+  tmem_wait_ld();
+  uint32_t pl[4][4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const float2 bf = unpack_h2(bw[m]);
+    float q[4][2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int i = 2 * m + e;
+      const float sb = __uint_as_float(v[0][i]) + (e ? bf.y : bf.x);
+      const float y2 = __uint_as_float(v[1][i]);
+      const float yr = __uint_as_float(v[2][i]), yi = __uint_as_float(v[3][i]);
+      const float ev = sb + y2, od = sb - y2;
+      const float z0 = act_fn<ACT>(ev + yr), z1 = act_fn<ACT>(od - yi);
+      const float z2 = act_fn<ACT>(ev - yr), z3 = act_fn<ACT>(od + yi);
+      const float a = z0 + z2, b = z1 + z3;
+      q[0][e] = a + b;
+      q[1][e] = a - b;
+      q[2][e] = z0 - z2;
+      q[3][e] = z3 - z1;
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) pl[p][m] = pack_h2(q[p][0], q[p][1]);
+  }
+#pragma unroll
+  for (int p = 0; p < 4; ++p) o[p] = make_uint4(pl[p][0], pl[p][1], pl[p][2], pl[p][3]);
+}
+
+template <int T, int ACT, int IO>
 __global__ void __launch_bounds__(kThreads, 1)
     eq_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                      const __grid_constant__ CUtensorMap map_y, const uint8_t* __restrict__ wtiles,
@@ -363,9 +406,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!is_raw && blockIdx.x == 0 && (int)it == ti.drop_w) continue;  // injected fault
           if (is_raw) {
             mbar_expect_tx(&full[s], X_STAGE_BYTES);
-            // 3-D view of X: (64 halves, 128-byte chunk of the row, row); a stage is
-            // chunks 2ks, 2ks+1 of 128 rows
-            tma_load_3d(sbase + S::OFF_X + s * X_STAGE_BYTES, &map_x, &full[s], 0, 2 * ks, row0);
+            if constexpr (IO == kIoSpectralIn) {
+              // planes [4][N][Cin] of the previous layer: (32 channels, 128 rows, 4 planes)
+              // land as the four K-major 64-byte-swizzled operand planes of this stage
+              tma_load_3d(sbase + S::OFF_X + s * X_STAGE_BYTES, &map_x, &full[s], S::BK * ks,
+                          row0, 0);
+            } else {
+              // 3-D view of X: (64 halves, 128-byte chunk of the row, row); a stage is
+              // chunks 2ks, 2ks+1 of 128 rows
+              tma_load_3d(sbase + S::OFF_X + s * X_STAGE_BYTES, &map_x, &full[s], 0, 2 * ks,
+                          row0);
+            }
           } else {
             // one pre-arranged blob per (out-channel tile, K stage)
             mbar_expect_tx(&full[s], S::W_STAGE_BYTES);
@@ -395,7 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int ks = 0; ks < ti.k_stages; ++ks, ++it) {
           const int sx = it % X_ST, sw = it % S::W_ST;
-          if (!(ok = wait_bounded(&bars->x_ready[sx], (it / X_ST) & 1, abort_flag, status))) break;
+          uint64_t* xbar = (IO == kIoSpectralIn) ? &bars->x_full[sx] : &bars->x_ready[sx];
+          if (!(ok = wait_bounded(xbar, (it / X_ST) & 1, abort_flag, status))) break;
           if (!(ok = wait_bounded(&bars->w_full[sw], (it / S::W_ST) & 1, abort_flag, status)))
             break;
           tc_fence_after();
@@ -466,6 +518,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int d0 = dbase + sc * kSliceCh;          // out-channel
         if (d0 >= Cout) break;  // warp-uniform: Cout is a multiple of 16
         const __half* bs = bsm + sc * kSliceCh;
+        if constexpr (IO == kIoSpectralOut) {
+          // staging [plane][32 rows][32 B], 32-byte swizzle (16-byte piece ^ (row / 4) % 2)
+          uint4 o[4];
+          epi_half_spec<BD, ACT>(lane_addr, c0, bs, o);
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          const int sw = (lane >> 2) & 1;
+#pragma unroll
+          for (int p = 0; p < 4; ++p)
+            *reinterpret_cast<uint4*>(stg + p * 1024 + lane * 32 + ((0 ^ sw) << 4)) = o[p];
+          epi_half_spec<BD, ACT>(lane_addr, c0 + 8, bs + 8, o);
+#pragma unroll
+          for (int p = 0; p < 4; ++p)
+            *reinterpret_cast<uint4*>(stg + p * 1024 + lane * 32 + ((1 ^ sw) << 4)) = o[p];
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            if (row0 < N) tma_store_3d(&map_y, stg_s, d0, (int)row0, 0);
+            bulk_commit();
+          }
+          continue;
+        }
         uint4 o[4];
         epi_half<T, BD, ACT>(lane_addr, c0, bs, o);
         // the previous slice's store has finished reading the buffer
@@ -491,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
-  } else if (warp >= kXfWarp0) {
+  } else if (warp >= kXfWarp0 && IO != kIoSpectralIn) {
     // ---------------- transform: group DFT into the operand planes ----------------
     const int xt = threadIdx.x - kXfWarp0 * 32;  // 0..255
     uint32_t it = 0;
@@ -606,38 +680,76 @@ cudaError_t launch_tile_weights(int T, const void* planes, int Cin, int Cout, vo
   });
 }
 
+namespace {
+
+// Spectral planes [4][N][channels] (FP16), viewed as (channel, row, plane).
+bool encode_planes_map(CUtensorMap* m, void* base, int channels, int64_t N, uint32_t box_ch,
+                       uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto encode = encode_fn();
+  cuuint64_t dims[3] = {(cuuint64_t)channels, (cuuint64_t)N, 4};
+  cuuint64_t strides[2] = {(cuuint64_t)channels * 2, (cuuint64_t)N * channels * 2};
+  cuuint32_t box[3] = {box_ch, box_rows, 4};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, base, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int TT, int ACT, int IO>
+cudaError_t set_smem_attr() {
+  return cudaFuncSetAttribute(eq_fwd_tc_kernel<TT, ACT, IO>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, Shape<TT>::SMEM_BYTES);
+}
+
+}  // namespace
+
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
-                          int num_sms, int drop_w_stage, int act, cudaStream_t st) {
+                          int num_sms, int drop_w_stage, int act, int io, cudaStream_t st) {
   if (!fwd_tc_supported(T, DType::F16, N, Cin, Cout)) return cudaErrorNotSupported;
   if (!Wtiles) return cudaErrorNotSupported;
+  if (io != kIoSpatial && T != 4) return cudaErrorNotSupported;
+  if (act != 0 && act != 1) return cudaErrorInvalidValue;
 
   auto encode = encode_fn();
   if (!encode) return cudaErrorNotSupported;
   return dispatch_tc(T, [&](auto tcst) {
     constexpr int TT = decltype(tcst)::value;
     using S = Shape<TT>;
-    CUtensorMap mx;
-    // X row = Cin*T/64 chunks of 64 halves (128 B); box = 2 chunks x 128 rows
-    cuuint64_t dims[3] = {64, (cuuint64_t)Cin * TT / 64, (cuuint64_t)N};
-    cuuint64_t strides[2] = {128, (cuuint64_t)Cin * TT * 2};
-    cuuint32_t box[3] = {64, 2, BM};
     cuuint32_t estr[3] = {1, 1, 1};
-    if (encode(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(X), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-    // Y row = Cout*T/64 chunks of 128 B; store box = 1 chunk x 32 rows
+    CUtensorMap mx;
+    if (io == kIoSpectralIn) {
+      // planes of the previous layer: box = 32 channels (64 B) x 128 rows x 4 planes
+      if (!encode_planes_map(&mx, const_cast<void*>(X), Cin, N, S::BK, BM,
+                             CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    } else {
+      // X row = Cin*T/64 chunks of 64 halves (128 B); box = 2 chunks x 128 rows
+      cuuint64_t dims[3] = {64, (cuuint64_t)Cin * TT / 64, (cuuint64_t)N};
+      cuuint64_t strides[2] = {128, (cuuint64_t)Cin * TT * 2};
+      cuuint32_t box[3] = {64, 2, BM};
+      if (encode(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(X), dims, strides,
+                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
     CUtensorMap my;
-    cuuint64_t ydims[3] = {64, (cuuint64_t)Cout * TT / 64, (cuuint64_t)N};
-    cuuint64_t ystrides[2] = {128, (cuuint64_t)Cout * TT * 2};
-    cuuint32_t ybox[3] = {64, 1, 32};
-    if (encode(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, Y, ydims, ystrides, ybox, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
+    if (io == kIoSpectralOut) {
+      // planes for the next layer: store box = 16 channels (32 B) x 32 rows x 4 planes
+      if (!encode_planes_map(&my, Y, Cout, N, 16, 32, CU_TENSOR_MAP_SWIZZLE_32B))
+        return cudaErrorInvalidValue;
+    } else {
+      // Y row = Cout*T/64 chunks of 128 B; store box = 1 chunk x 32 rows
+      cuuint64_t ydims[3] = {64, (cuuint64_t)Cout * TT / 64, (cuuint64_t)N};
+      cuuint64_t ystrides[2] = {128, (cuuint64_t)Cout * TT * 2};
+      cuuint32_t ybox[3] = {64, 1, 32};
+      if (encode(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, Y, ydims, ystrides, ybox, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
     TileInfo ti;
     ti.n_dt = (Cout + S::BD - 1) / S::BD;
     const int64_t n_rt = (N + BM - 1) / BM;
@@ -647,15 +759,27 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
     ti.drop_w = drop_w_stage;
     static bool attr_set = false;
     if (!attr_set) {
-      for (auto fn : {eq_fwd_tc_kernel<TT, 0>, eq_fwd_tc_kernel<TT, 1>}) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             S::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
+      cudaError_t e = set_smem_attr<TT, 0, kIoSpatial>();
+      if (e == cudaSuccess) e = set_smem_attr<TT, 1, kIoSpatial>();
+      if constexpr (TT == 4) {
+        if (e == cudaSuccess) e = set_smem_attr<TT, 0, kIoSpectralOut>();
+        if (e == cudaSuccess) e = set_smem_attr<TT, 1, kIoSpectralOut>();
+        if (e == cudaSuccess) e = set_smem_attr<TT, 0, kIoSpectralIn>();
+        if (e == cudaSuccess) e = set_smem_attr<TT, 1, kIoSpectralIn>();
       }
+      if (e != cudaSuccess) return e;
       attr_set = true;
     }
     const int grid = ti.num_tiles < num_sms ? ti.num_tiles : num_sms;
-    auto kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1> : eq_fwd_tc_kernel<TT, 0>;
+    auto kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1, kIoSpatial> : eq_fwd_tc_kernel<TT, 0, kIoSpatial>;
+    if constexpr (TT == 4) {
+      if (io == kIoSpectralOut)
+        kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1, kIoSpectralOut>
+                          : eq_fwd_tc_kernel<TT, 0, kIoSpectralOut>;
+      else if (io == kIoSpectralIn)
+        kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1, kIoSpectralIn>
+                          : eq_fwd_tc_kernel<TT, 0, kIoSpectralIn>;
+    }
     kernel<<<grid, kThreads, S::SMEM_BYTES, st>>>(
         mx, my, static_cast<const uint8_t*>(Wtiles), static_cast<const __half*>(bias), N, Cin,
         Cout, ti, status);

@@ -75,6 +75,31 @@ class EqLinearPlan:
             _n.eqlinear_forward_act(self.handle, X, N, W_hat, bias, _n.ACT[act], out)
         return out
 
+    def forward_to_spectral(self, X, W_hat, bias=None, act: str = "none",
+                            out=None) -> torch.Tensor:
+        """act(EQ-Linear(X) + bias) as the next p4 layer's input planes [4, N, D]."""
+        N = X.shape[0]
+        self._check(X, (N, self.C * self.T), "X")
+        if bias is not None:
+            self._check(bias, (self.D,), "bias")
+        if out is None:
+            out = torch.empty((4, N, self.D), dtype=self.dtype, device=X.device)
+        self._check(out, (4, N, self.D), "out")
+        _n.eqlinear_forward_to_spectral(self.handle, X, N, W_hat, bias, _n.ACT[act], out)
+        return out
+
+    def forward_from_spectral(self, Xhat, W_hat, bias=None, act: str = "none",
+                              out=None) -> torch.Tensor:
+        """EQ-Linear forward of an input given as spectral planes [4, N, C]."""
+        N = Xhat.shape[1]
+        self._check(Xhat, (4, N, self.C), "Xhat")
+        if bias is not None:
+            self._check(bias, (self.D,), "bias")
+        if out is None:
+            out = torch.empty((N, self.D * self.T), dtype=self.dtype, device=Xhat.device)
+        _n.eqlinear_forward_from_spectral(self.handle, Xhat, N, W_hat, bias, _n.ACT[act], out)
+        return out
+
     def backward_input(self, dY, W_hat, out=None) -> torch.Tensor:
         N = dY.shape[0]
         self._check(dY, (N, self.D * self.T), "dY")

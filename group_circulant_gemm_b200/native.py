@@ -25,6 +25,7 @@ EXPORTED = (
     "eqlinear_plan_destroy", "eqlinear_plan_set_kernel", "eqlinear_forward_kernel_name",
     "eqlinear_backward_weight_kernel_name", "eqlinear_prepared_weight_bytes",
     "eqlinear_prepare_weights", "eqlinear_forward", "eqlinear_forward_act",
+    "eqlinear_spectral_bytes", "eqlinear_forward_to_spectral", "eqlinear_forward_from_spectral",
     "eqlinear_backward_input",
     "eqlinear_backward_weight_workspace_bytes", "eqlinear_backward_weight",
     "eqlinear_get_status", "eqlinear_backward_weight_noalloc",
@@ -56,6 +57,9 @@ def _load() -> ctypes.CDLL:
         "eqlinear_prepare_weights": ([vp, vp, vp, vp], i32),
         "eqlinear_forward": ([vp, vp, i64, vp, vp, vp, vp], i32),
         "eqlinear_forward_act": ([vp, vp, i64, vp, vp, i32, vp, vp], i32),
+        "eqlinear_spectral_bytes": ([vp, i64], ctypes.c_size_t),
+        "eqlinear_forward_to_spectral": ([vp, vp, i64, vp, vp, i32, vp, vp], i32),
+        "eqlinear_forward_from_spectral": ([vp, vp, i64, vp, vp, i32, vp, vp], i32),
         "eqlinear_backward_input": ([vp, vp, i64, vp, vp, vp], i32),
         "eqlinear_backward_weight_workspace_bytes": ([vp, i64], sz),
         "eqlinear_backward_weight": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
@@ -145,6 +149,24 @@ ACT = {"none": 0, "gelu": 1}
 def eqlinear_forward_act(plan: int, X, N: int, W_hat, bias, act: int, Y, stream=None) -> None:
     _check(_lib.eqlinear_forward_act(plan, _ptr(X), N, _ptr(W_hat), _ptr(bias), act, _ptr(Y),
                                      _stream(stream)), "eqlinear_forward_act")
+
+
+def eqlinear_spectral_bytes(plan: int, N: int) -> int:
+    return _lib.eqlinear_spectral_bytes(plan, N)
+
+
+def eqlinear_forward_to_spectral(plan: int, X, N: int, W_hat, bias, act: int, Xhat,
+                                 stream=None) -> None:
+    _check(_lib.eqlinear_forward_to_spectral(plan, _ptr(X), N, _ptr(W_hat), _ptr(bias), act,
+                                             _ptr(Xhat), _stream(stream)),
+           "eqlinear_forward_to_spectral")
+
+
+def eqlinear_forward_from_spectral(plan: int, Xhat, N: int, W_hat, bias, act: int, Y,
+                                   stream=None) -> None:
+    _check(_lib.eqlinear_forward_from_spectral(plan, _ptr(Xhat), N, _ptr(W_hat), _ptr(bias), act,
+                                               _ptr(Y), _stream(stream)),
+           "eqlinear_forward_from_spectral")
 
 
 def eqlinear_backward_input(plan: int, dY, N: int, W_hat, dX, stream=None) -> None:

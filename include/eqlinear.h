@@ -169,6 +169,35 @@ EQL_API eqlinear_status_t eqlinear_forward_act(eqlinear_plan_t plan, const void*
                                                eqlinear_act_t act, void* Y, void* stream);
 
 /*
+ * Two-layer EQ-MLP block with the intermediate kept in the frequency domain
+ * ("Algorithmic approach": the layer is a per-frequency product between a
+ * forward and an inverse group DFT; when one EQ-Linear feeds another, the
+ * second layer's forward DFT can be taken by the first layer's epilogue).
+ *
+ * eqlinear_forward_to_spectral writes, instead of Y, the group DFT of
+ * act(Y) as four FP16 planes Xhat[4][N][D] (plane 0: sum over s, 1: alternating
+ * sum, 2: y0 - y2, 3: y3 - y1; FP32 arithmetic, one rounding), which is the
+ * input a following p4 layer multiplies directly.  eqlinear_forward_from_spectral
+ * is the forward of a layer whose input arrives as such planes Xhat[4][N][C]
+ * (Y [N][D*T], optional bias and act as in eqlinear_forward_act).  Chaining the
+ * two equals eqlinear_forward_act followed by eqlinear_forward up to rounding.
+ *
+ * Only FP16 plans with T = 4 and C, D multiples of 16 (the tensor-core path);
+ * others return EQL_ERR_UNSUPPORTED, as does a plan forced to the CUDA-core
+ * kernels.  Buffers: eqlinear_spectral_bytes(plan, N) = 4 * N * D * 2 bytes for
+ * the output of eqlinear_forward_to_spectral (the same size as Y).
+ */
+EQL_API size_t eqlinear_spectral_bytes(eqlinear_plan_t plan, int64_t N);
+EQL_API eqlinear_status_t eqlinear_forward_to_spectral(eqlinear_plan_t plan, const void* X,
+                                                       int64_t N, const void* W_hat,
+                                                       const void* bias, eqlinear_act_t act,
+                                                       void* Xhat_next, void* stream);
+EQL_API eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t plan, const void* Xhat,
+                                                         int64_t N, const void* W_hat,
+                                                         const void* bias, eqlinear_act_t act,
+                                                         void* Y, void* stream);
+
+/*
  * Gradient with respect to the input ("Implementation": backward pass):
  *   dX[n, c*T+t] = sum_{d,s} dY[n, d*T+s] * W[d][c][(t-s) mod T]
  * which is the same group-circulant product with the transposed weights and the

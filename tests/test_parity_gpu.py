@@ -344,3 +344,66 @@ def test_forward_act_rejects_unknown_activation():
     s = n.raw_status("eqlinear_forward_act", p.handle, X.data_ptr(), 16, Wh.data_ptr(), None, 7,
                      Y.data_ptr(), None)
     assert s == 1  # EQL_ERR_INVALID_ARG
+
+
+# --- two-layer block with the intermediate in the frequency domain -------------------
+
+def _planes_of(Y, H):
+    """float64 group DFT of a [N, H*4] activation: planes [4, N, H] in the kernel's order."""
+    g = Y.reshape(Y.shape[0], H, 4)
+    return np.stack([g.sum(axis=2), g[..., 0] - g[..., 1] + g[..., 2] - g[..., 3],
+                     g[..., 0] - g[..., 2], g[..., 3] - g[..., 1]])
+
+
+BLOCK_CASES = [
+    # N, C, H (hidden), D2, act
+    (333, 192, 768, 192, "gelu"),
+    (300, 48, 144, 80, "none"),
+    (129, 16, 16, 32, "gelu"),
+    (1, 32, 64, 48, "none"),
+]
+
+
+@pytest.mark.parametrize("N,C,H,D2,act", BLOCK_CASES)
+def test_spectral_block_matches_oracle(N, C, H, D2, act):
+    w1 = Workload("blk1", 4, N, C, H, "f16", True, 1300 + N + C)
+    w2 = Workload("blk2", 4, N, H, D2, "f16", True, 1400 + N + H)
+    in1, in2 = make_inputs(w1), make_inputs(w2, rows=1)
+    p1, p2 = _plan(w1), _plan(w2)
+    Wh1, Wh2 = p1.prepare_weights(_dev(in1["W"])), p2.prepare_weights(_dev(in2["W"]))
+    Xh = p1.forward_to_spectral(_dev(in1["X"]), Wh1, _dev(in1["bias"]), act=act)
+    assert tuple(Xh.shape) == (4, N, H)
+    Y1 = oracle.forward(4, in1["X"], in1["W"], in1["bias"], act=act)
+    assert _rel(Xh.double().cpu().numpy(), _planes_of(Y1, H)) <= TOL["f16"]
+    Y = p2.forward_from_spectral(Xh, Wh2, _dev(in2["bias"]))
+    assert p1.status() == 0 and p2.status() == 0
+    ref = oracle.forward(4, Y1, in2["W"], in2["bias"])
+    assert _rel(Y.double().cpu().numpy(), ref) <= TOL["f16"]
+
+
+def test_spectral_block_full_size_sampled_rows():
+    w1, w2 = WORKLOADS["p4_vitb_fc1_f16"], WORKLOADS["p4_vitb_fc2_f16"]
+    in1, in2 = make_inputs(w1), make_inputs(w2, rows=1)
+    p1, p2 = _plan(w1), _plan(w2)
+    Wh1, Wh2 = p1.prepare_weights(_dev(in1["W"])), p2.prepare_weights(_dev(in2["W"]))
+    Xh = p1.forward_to_spectral(_dev(in1["X"]), Wh1, _dev(in1["bias"]), act="gelu")
+    Y = p2.forward_from_spectral(Xh, Wh2, _dev(in2["bias"])).double().cpu().numpy()
+    assert p1.status() == 0 and p2.status() == 0
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([rng.choice(w1.N, 40, replace=False),
+                                     np.arange(w1.N - 8, w1.N), np.arange(8)]))
+    Y1 = oracle.forward(4, in1["X"][rows], in1["W"], in1["bias"], act="gelu")
+    ref = oracle.forward(4, Y1, in2["W"], in2["bias"])
+    assert _rel(Y[rows], ref) <= TOL["f16"]
+
+
+def test_spectral_entry_points_reject_unsupported_plans():
+    from group_circulant_gemm_b200 import native as n
+    w = Workload("blkbad", 8, 16, 16, 16, "f16", True, 3)  # T = 8: no spectral form
+    p = _plan(w)
+    X = torch.zeros((16, 128), dtype=torch.float16, device="cuda")
+    Xh = torch.zeros((4, 16, 16), dtype=torch.float16, device="cuda")
+    Wh = p.prepare_weights(_dev(make_inputs(w)["W"]))
+    s = n.raw_status("eqlinear_forward_to_spectral", p.handle, X.data_ptr(), 16, Wh.data_ptr(),
+                     None, 0, Xh.data_ptr(), None)
+    assert s == 2  # EQL_ERR_UNSUPPORTED
