@@ -149,7 +149,8 @@ EQL_API eqlinear_status_t eqlinear_forward(eqlinear_plan_t plan, const void* X, 
 /* Output activation applied by eqlinear_forward_act. */
 typedef enum {
   EQL_ACT_NONE = 0,
-  EQL_ACT_GELU = 1  /* GELU(y) = y * Phi(y) = 0.5 y (1 + erf(y / sqrt 2)), exact erf form */
+  EQL_ACT_GELU = 1  /* GELU(y) = y * Phi(y) = 0.5 y (1 + erf(y / sqrt 2)), exact erf form
+                       (erf within 3e-7, Abramowitz & Stegun 7.1.28) */
 } eqlinear_act_t;
 
 /*
