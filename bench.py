@@ -99,7 +99,7 @@ KERNEL_SOURCES = {
     "backward_weight": ("eql_tc_wgrad.cu", "eql_tc_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("forward", "e01149104234b8ee"): {"p4_vitb_mlp_f16": 58.94e6, "c8_1024_f16": 34.02e6,
+    ("forward", "edcf01d7b2cb736c"): {"p4_vitb_mlp_f16": 58.94e6, "c8_1024_f16": 34.02e6,
                                       "p4_vith_fc1_fwd_bwd_f16": 70.12e6},
     ("backward_weight", "bfa7d6c1a4d80534"): {"p4_vith_fc1_fwd_bwd_f16": 108.84e6},
 }

@@ -1,6 +1,6 @@
 // tcgen05/TMEM tensor-core forward of the cyclic-group EQ-Linear layer for
 // T = 4 (the p4 rotation group) and T = 8, FP16 in, FP32 accumulate, FP16 out,
-// for sm_100a.
+// for sm_100a.  Also used for dX (the same product with the adjoint weights).
 //
 // What it computes (Flash EQ-Linear summary, "Algorithmic approach" items 1-3
 // and "Specialisation for p4"): per row n and input channel c the real DFT of
@@ -11,13 +11,19 @@
 //   complex k:  Y_kr = Xr_k Br_k^T - Xi_k Bi_k^T,  Y_ki = Xr_k Bi_k^T + Xi_k Br_k^T
 //   y[s] = (Y_0 + (-1)^s Y_{T/2}) / T + (2/T) sum_k (Y_kr cos(2 pi k s/T) - Y_ki sin(2 pi k s/T))
 // For T = 4 the transforms are adds only (X0 = x0+x1+x2+x3, X2 = x0-x1+x2-x3,
-// Xr = x0-x2, Xi = x3-x1) and the inverse uses the factors 1/4 and 1/2; for
-// T = 8 a radix-2 split leaves one non-dyadic twiddle, sqrt(2)/2.
+// Xr = x0-x2, Xi = x3-x1); for T = 8 a radix-2 split leaves one non-dyadic
+// twiddle, sqrt(2)/2.  The inverse's factors 1/T and 2/T are folded into the
+// weight tiles, so the epilogue is adds only.
+//
+// Template parameters: ACT = output activation (0 none, 1 GELU, fused into the
+// epilogue); IO (T = 4) = spatial X and Y, or Y written as the next layer's
+// spectral operand planes [4][N][Cout], or X read as such planes (then the TMA
+// box lands directly as the operand planes and the transform warps are idle).
 //
 // Design (one persistent CTA per SM; tile = 128 rows x BD out-channels; K stage
 // = BK input channels, whose raw X tile is always 128 rows x 256 B = 32 KB):
 //   warp 0      TMA producer: the raw X tile of a stage, one 3-D box
-//               (64 halves x 2 row chunks x 128 rows, 128B-swizzled).
+//               (64 halves x 2 row chunks x 128 rows, 128B-swizzled), 3-deep ring.
 //   warp 2      weight producer: one bulk copy per stage of a blob that
 //               prepare_weights pre-arranged in the MMA operand layout.
 //   warp 1      TMEM allocator; lane 0 issues the MMAs of each K step:
@@ -26,8 +32,11 @@
 //   warps 12-19 transform: group DFT in FP32, one rounding to FP16, written as
 //               T K-major swizzled operand planes over the raw tile of the same
 //               slot (the planes take exactly the raw tile's 32 KB).
-//   warps 4-11  epilogue: tcgen05.ld of the T accumulators, inverse DFT, bias,
-//               FP16 pack, 16-byte global stores.
+//   warps 4-11  epilogue: the tile's biases staged in shared memory while the
+//               main loop runs; tcgen05.ld 32x32b (one row per lane), inverse
+//               DFT + bias (+ activation), FP16 pack into a per-warp 4 KB
+//               staging buffer, one TMA store per 32 rows x 128 bytes of Y (or
+//               per 32 rows x 16 channels x 4 planes for spectral output).
 // TMEM (T * BD = 512 columns): real frequency 0 at [0, BD), real frequency T/2
 // at [BD, 2 BD), complex frequency k at [2 BD k, 2 BD k + 2 BD) as (re | im).
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the CTA
