@@ -203,20 +203,6 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// 16 TMEM lanes x 256 bits: thread t gets lanes (t/4) and (t/4 + 8) of the
-// addressed 16-lane group, columns 2*(t%4) and 2*(t%4)+1 -> regs
-// {lane t/4: col, col+1, lane t/4+8: col, col+1}.
-#define EQL_TMEM_LD_16x256(taddr, r)                                                   \
-  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0, %1, %2, %3}, [%4];"         \
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])                         \
-               : "r"(taddr))
-// The .x2 form repeats the pattern for the next 8 columns in regs 4..7.
-#define EQL_TMEM_LD_16x256_X2(taddr, r)                                                    \
-  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"    \
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),    \
-                 "=r"(r[6]), "=r"(r[7])                                                    \
-               : "r"(taddr))
-
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);  // a -> low half, b -> high half
   uint32_t u;
