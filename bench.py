@@ -101,7 +101,6 @@ KERNEL_SOURCES = {
 NCU_TRAFFIC = {
     ("forward", "7f61d3dc196bce45"): {"p4_vitb_mlp_f16": 58.94e6, "c8_1024_f16": 34.02e6,
                                       "p4_vith_fc1_fwd_bwd_f16": 70.12e6},
-    ("backward_weight", "308cf9f20b2e3fd0"): {"p4_vith_fc1_fwd_bwd_f16": 108.84e6},
 }
 
 def kernel_traffic(family: str, workload: str):

@@ -308,16 +308,9 @@ eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t p, const void* X, con
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  if (wgrad_use_tc(p, N, X, dY)) {
-    const int splits = eql::wgrad_tc_splits(N, p->C, p->D, p->num_sms);
-    float* part = static_cast<float*>(workspace);
-    float* bpart = part + (size_t)splits * 4 * p->C * p->D;
-    s = from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, part, bpart, splits, p->status,
-                                       p->num_sms, st));
-    if (s != EQL_OK) return s;
-    return from_cuda(eql::launch_wgrad_tc_finalize(part, bpart, splits, p->C, p->D, dW, dbias,
-                                                   p->tw, st));
-  }
+  if (wgrad_use_tc(p, N, X, dY))
+    return from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, workspace, dW, dbias, p->status,
+                                          p->num_sms, p->tw, st));
   const int splits = eql::wgrad_simt_splits(p->T, N, p->C, p->D, p->num_sms);
   return from_cuda(eql::launch_wgrad_simt(p->T, to_dt(p->dtype), X, dY, N, p->C, p->D, dW,
                                           dbias, static_cast<float*>(workspace), splits, p->tw,

@@ -59,16 +59,14 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
                           int num_sms, int drop_w_stage, int act, int io, cudaStream_t st);
 
-// tcgen05/TMEM tensor-core weight gradient for T = 4, FP16: FP32 partial
-// spectra part[splits][4][C][D] and bias partials bpart[splits][D], finished by
-// launch_wgrad_tc_finalize.  X and dY must be 16-byte aligned (TMA).
+// tcgen05/TMEM tensor-core weight gradient for T = 4, FP16: stream-K over
+// (tile, 32-row stage) ranges, FP32 partial slots in `workspace`, then a
+// fixed-order finalize (inverse DFT, cast) into dW [D][C][4] and dbias [D].
+// X and dY must be 16-byte aligned (TMA).  N = 0 is handled by the caller.
 bool wgrad_tc_supported(int T, DType dt, int64_t N, int C, int D, const void* X, const void* dY);
-int wgrad_tc_splits(int64_t N, int C, int D, int num_sms);
 size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms);
-cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D, float* part,
-                            float* bpart, int splits, int* status, int num_sms, cudaStream_t st);
-cudaError_t launch_wgrad_tc_finalize(const float* part, const float* bpart, int splits, int C,
-                                     int D, void* dW, void* dbias, const Twiddles& tw,
-                                     cudaStream_t st);
+cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
+                            void* workspace, void* dW, void* dbias, int* status, int num_sms,
+                            const Twiddles& tw, cudaStream_t st);
 
 }  // namespace eql

@@ -7,14 +7,19 @@
 // G2 = g0-g1+g2-g3, Gr = g0-g2, Gi = g3-g1, likewise for X):
 //   Q0 = G0^T Xh0,  Q2 = G2^T Xh2,
 //   Qr = Gr^T Xr + Gi^T Xi,  Qi = Gr^T Xi - Gi^T Xr        (D x C each, K = rows)
-// summed over the row range of one work unit and stored as the FP32 partial
-// planes part[split][4][C][D] (out-channel fastest, so each warp store writes 32
-// consecutive floats); dbias partials are the FP32 column sums of G0.  A
-// finalize kernel adds the splits in a fixed order, applies the inverse group
-// DFT and casts, so the result is deterministic.
+// summed over a range of rows and stored as FP32 partial planes; dbias partials
+// are the FP32 column sums of G0.  A finalize kernel adds a tile's partials in a
+// fixed order, applies the inverse group DFT and casts, so the result is
+// deterministic.
 //
-// Design (one persistent CTA per SM; work unit = 128 out-channels x 128
-// in-channels x one row range; stage = 32 rows):
+// Work split (stream-K over rows): the (tile, 32-row stage) space, tile = 128
+// out-channels x 128 in-channels, is cut into equal contiguous ranges, one per
+// CTA, so every SM does the same number of stages.  A range can end one tile
+// and start the next; each piece (a "segment") accumulates in TMEM and writes
+// its own partial slot part[tile][j][4][128 c][128 d] (j = which of the tile's
+// ranges; out-channel fastest, so each warp store writes 128 contiguous bytes).
+//
+// Design (one CTA per SM; stage = 32 rows):
 //   warp 0      TMA producer: per stage one 3-D box of dY (32 rows x 1 KB: the
 //               128 out-channels x 4 group elements of the tile) and one of X.
 //   warp 1      TMEM allocator; lane 0 issues the MMAs: M = out-channel, N =
@@ -67,29 +72,45 @@ struct WgBars {
 static_assert(sizeof(WgBars) <= 512, "barrier block");
 
 struct WgInfo {
-  int n_dt, n_ct;       // out-channel and in-channel tiles
-  int num_units;        // n_dt * n_ct * splits
-  int64_t rows_per_split;  // multiple of WG_BR
+  int n_dt, n_ct;      // out-channel and in-channel tiles
+  int spt;             // 32-row stages per tile, ceil(N / 32)
+  int per_unit;        // stages per CTA range
+  int maxj;            // partial slots per tile
+  int64_t total;       // tiles * spt
 };
 
+// One segment of a CTA's range: stages [r0 / 32, r0 / 32 + stages) of one tile.
 struct Unit {
-  int z, dt, ct;
+  int dt, ct, tile, slot;  // slot = tile * maxj + (range index within the tile)
   int64_t r0;
   int stages;
 };
-__device__ __forceinline__ Unit decode(int u, const WgInfo& wi, int64_t N) {
-  Unit x;
-  const int tiles = wi.n_dt * wi.n_ct;
-  x.z = u / tiles;
-  const int t = u % tiles;
-  x.dt = t / wi.n_ct;
-  x.ct = t % wi.n_ct;
-  x.r0 = (int64_t)x.z * wi.rows_per_split;
-  int64_t end = x.r0 + wi.rows_per_split;
-  if (end > N) end = N;
-  x.stages = (int)((end - x.r0 + WG_BR - 1) / WG_BR);
-  return x;
+
+__host__ __device__ inline int first_range_of_tile(int64_t tile, const WgInfo& wi) {
+  return (int)(tile * wi.spt / wi.per_unit);
 }
+
+struct SegIter {
+  int64_t g, g1;
+  int u;
+  __device__ SegIter(const WgInfo& wi, int u_) : u(u_) {
+    g = (int64_t)u * wi.per_unit;
+    g1 = g + wi.per_unit < wi.total ? g + wi.per_unit : wi.total;
+  }
+  __device__ bool next(const WgInfo& wi, Unit& x) {
+    if (g >= g1) return false;
+    x.tile = (int)(g / wi.spt);
+    const int s0 = (int)(g % wi.spt);
+    const int64_t room = wi.spt - s0;
+    x.stages = (int)(room < g1 - g ? room : g1 - g);
+    x.dt = x.tile / wi.n_ct;
+    x.ct = x.tile % wi.n_ct;
+    x.slot = x.tile * wi.maxj + (u - first_range_of_tile(x.tile, wi));
+    x.r0 = (int64_t)s0 * WG_BR;
+    g += x.stages;
+    return true;
+  }
+};
 
 // One transform item: rows 8q..8q+7 of the raw tile, channel pair pd = 8w + j.
 // The raw tile is [row][128-byte chunk][128 B] with 128-byte swizzle (16-byte
@@ -196,8 +217,9 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       for (int s = 0; s < WG_ST; ++s) issued_phase[s] = -1;
       uint32_t it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < wi.num_units; u += gridDim.x) {
-        const Unit un = decode(u, wi, N);
+      SegIter si(wi, blockIdx.x);
+      Unit un;
+      while (ok && si.next(wi, un)) {
         for (int s = 0; s < un.stages; ++s, ++it) {
           const int slot = it % WG_ST;
           const uint32_t ph = (it / WG_ST) & 1;
@@ -224,8 +246,9 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       const uint32_t id_n1 = idesc_f16(128, WG_BC);
       const uint32_t id_n1_neg = idesc_f16(128, WG_BC, true);
       const uint32_t id_n2 = idesc_f16(128, 2 * WG_BC);
-      for (int u = blockIdx.x; ok && u < wi.num_units; u += gridDim.x, ++ucount) {
-        const Unit un = decode(u, wi, N);
+      SegIter si(wi, blockIdx.x);
+      Unit un;
+      for (; ok && si.next(wi, un); ++ucount) {
         if (!(ok = wait_bounded(&bars->acc_empty, (ucount & 1) ^ 1, abort_flag, status))) break;
         tc_fence_after();
         for (int s = 0; s < un.stages; ++s, ++it) {
@@ -262,15 +285,18 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     // and each of the 16 stores writes 32 consecutive out-channels (128 B).
     const int q = warp & 3;
     uint32_t ucount = 0;
-    for (int u = blockIdx.x; u < wi.num_units; u += gridDim.x, ++ucount) {
-      const Unit un = decode(u, wi, N);
+    SegIter si(wi, blockIdx.x);
+    Unit un;
+    for (; si.next(wi, un); ++ucount) {
       if (!warp_wait(&bars->acc_full, ucount & 1, abort_flag, status)) break;
       tc_fence_after();
-      const int d = un.dt * WG_BD + 32 * q + lane;
+      const int dl = 32 * q + lane;  // out-channel within the tile
+      const int d = un.dt * WG_BD + dl;
       const uint32_t lrow = tmem + ((uint32_t)(32 * q) << 16);
+      float* slot_base = part + (int64_t)un.slot * (4 * WG_BC * WG_BD);
 #pragma unroll 1
       for (int p = 0; p < 4; ++p) {
-        float* dst_plane = part + ((int64_t)un.z * 4 + p) * D * C;
+        float* dst_plane = slot_base + p * (WG_BC * WG_BD);
 #pragma unroll 1
         for (int gq = 0; gq < WG_BC / 16; ++gq) {
           const int c = un.ct * WG_BC + 16 * gq;
@@ -281,7 +307,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
           if (d < D) {
 #pragma unroll
             for (int k = 0; k < 16; ++k)
-              dst_plane[(int64_t)(c + k) * D + d] = __uint_as_float(r[k]);
+              dst_plane[(16 * gq + k) * WG_BD + dl] = __uint_as_float(r[k]);
           }
         }
       }
@@ -295,8 +321,9 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     const int j = lane & 7, q = lane >> 3;
     uint32_t it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < wi.num_units; u += gridDim.x) {
-      const Unit un = decode(u, wi, N);
+    SegIter si(wi, blockIdx.x);
+    Unit un;
+    while (ok && si.next(wi, un)) {
       float bsum[2] = {0.f, 0.f}, unused[2] = {0.f, 0.f};
       for (int s = 0; s < un.stages; ++s, ++it) {
         const int slot = it % WG_ST;
@@ -322,9 +349,9 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
         bsum[e] += __shfl_xor_sync(0xffffffffu, bsum[e], 16);
       }
       if (grp == 0 && un.ct == 0 && q == 0) {
-        const int d = un.dt * WG_BD + 2 * (8 * w + j);
-        if (d < D) bpart[(int64_t)un.z * D + d] = bsum[0];
-        if (d + 1 < D) bpart[(int64_t)un.z * D + d + 1] = bsum[1];
+        const int dl = 2 * (8 * w + j);
+        bpart[(int64_t)un.slot * WG_BD + dl] = bsum[0];
+        bpart[(int64_t)un.slot * WG_BD + dl + 1] = bsum[1];
       }
     }
   }
@@ -337,30 +364,40 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
   }
 }
 
-// Sum of the split partials (fixed order), inverse group DFT, cast:
-// dW[d][c][u] from part[split][4][C][D]; dbias[d] from bpart[split][D].
+// Sum of a tile's partial slots (fixed order), inverse group DFT, cast:
+// dW[d][c][u] from part[tile][j][4][128 c][128 d]; dbias[d] from
+// bpart[tile][j][128] of the tiles with in-channel tile 0.
 __global__ void wgrad_tc_finalize_kernel(const float* __restrict__ part,
-                                         const float* __restrict__ bpart, int splits, int C, int D,
-                                         __half* __restrict__ dW, __half* __restrict__ dbias,
-                                         Twiddles tw) {
+                                         const float* __restrict__ bpart, WgInfo wi, int C,
+                                         int D, __half* __restrict__ dW,
+                                         __half* __restrict__ dbias, Twiddles tw) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // c * D + d
-  const int64_t plane = (int64_t)D * C;
-  if (idx < plane) {
+  if (idx < (int64_t)D * C) {
+    const int c = (int)(idx / D), d = (int)(idx % D);
+    const int tile = (d / WG_BD) * wi.n_ct + c / WG_BC;
+    const int first = first_range_of_tile(tile, wi);
+    const int last = (int)(((int64_t)tile * wi.spt + wi.spt - 1) / wi.per_unit);
+    const int64_t off = (int64_t)(c % WG_BC) * WG_BD + (d % WG_BD);
     float qv[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int z = 0; z < splits; ++z) {
+    for (int j = 0; j <= last - first; ++j) {
+      const float* slot = part + ((int64_t)tile * wi.maxj + j) * (4 * WG_BC * WG_BD);
 #pragma unroll
-      for (int p = 0; p < 4; ++p) qv[p] += part[((int64_t)z * 4 + p) * plane + idx];
+      for (int p = 0; p < 4; ++p) qv[p] += slot[p * (WG_BC * WG_BD) + off];
     }
     float wv[4];
     group_idft<4>(qv, wv, tw);
-    const int64_t c = idx / D, d = idx % D;
-    __half2* out = reinterpret_cast<__half2*>(dW + (d * C + c) * 4);
+    __half2* out = reinterpret_cast<__half2*>(dW + ((int64_t)d * C + c) * 4);
     out[0] = __floats2half2_rn(wv[0], wv[1]);
     out[1] = __floats2half2_rn(wv[2], wv[3]);
   }
   if (dbias && idx < D) {
+    const int d = (int)idx;
+    const int tile = (d / WG_BD) * wi.n_ct;
+    const int first = first_range_of_tile(tile, wi);
+    const int last = (int)(((int64_t)tile * wi.spt + wi.spt - 1) / wi.per_unit);
     float b = 0.f;
-    for (int z = 0; z < splits; ++z) b += bpart[(int64_t)z * D + idx];
+    for (int j = 0; j <= last - first; ++j)
+      b += bpart[((int64_t)tile * wi.maxj + j) * WG_BD + d % WG_BD];
     dbias[idx] = __float2half_rn(b);
   }
 }
@@ -379,9 +416,33 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int channels, int64_t N) 
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int64_t wgrad_tc_rows_per_split(int64_t N, int splits) {
-  const int64_t per = (N + splits - 1) / splits;
-  return (per + WG_BR - 1) / WG_BR * WG_BR;
+// The stream-K layout for N rows: equal contiguous ranges of (tile, stage), one
+// per CTA, and the number of partial slots a tile can need.
+bool wgrad_tc_layout(int64_t N, int C, int D, int num_sms, WgInfo* wi, int* grid) {
+  if (N <= 0) return false;
+  wi->n_dt = (D + WG_BD - 1) / WG_BD;
+  wi->n_ct = (C + WG_BC - 1) / WG_BC;
+  const int64_t spt = (N + WG_BR - 1) / WG_BR;
+  if (spt > 0x3fffffffLL) return false;
+  wi->spt = (int)spt;
+  wi->total = (int64_t)wi->n_dt * wi->n_ct * spt;
+  const int64_t want = std::min<int64_t>(num_sms, wi->total);
+  int64_t per = (wi->total + want - 1) / want;
+  // at least 16 stages (512 rows) per range, or a whole tile, so the 256 KB
+  // partial a range writes is amortised
+  per = std::max<int64_t>(per, std::min<int64_t>(spt, 16));
+  if (per > 0x3fffffffLL) return false;
+  wi->per_unit = (int)per;
+  *grid = (int)((wi->total + per - 1) / per);
+  // slots per tile: the number of ranges that touch it (exact maximum)
+  const int64_t tiles = (int64_t)wi->n_dt * wi->n_ct;
+  int64_t maxj = 1;
+  for (int64_t t = 0; t < tiles; ++t) {
+    const int64_t first = t * spt / per, last = (t * spt + spt - 1) / per;
+    maxj = std::max(maxj, last - first + 1);
+  }
+  wi->maxj = (int)maxj;
+  return true;
 }
 
 }  // namespace
@@ -392,45 +453,25 @@ bool wgrad_tc_supported(int T, DType dt, int64_t N, int C, int D, const void* X,
          ((reinterpret_cast<uintptr_t>(dY) & 15) == 0);
 }
 
-int wgrad_tc_splits(int64_t N, int C, int D, int num_sms) {
-  if (N <= 0) return 0;
-  const int tiles = ((D + WG_BD - 1) / WG_BD) * ((C + WG_BC - 1) / WG_BC);
-  int64_t s = std::max(1, num_sms / tiles);
-  s = std::min<int64_t>(s, (N + WG_BR - 1) / WG_BR);
-  // drop splits that the rounding of the row range leaves empty
-  const int64_t rows = wgrad_tc_rows_per_split(N, (int)s);
-  return (int)((N + rows - 1) / rows);
-}
-
 size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms) {
-  const int s = wgrad_tc_splits(N, C, D, num_sms);
-  return (size_t)std::max(s, 1) * ((size_t)4 * C * D + D) * sizeof(float);
+  WgInfo wi;
+  int grid = 0;
+  if (!wgrad_tc_layout(N, C, D, num_sms, &wi, &grid)) return 0;
+  const size_t slots = (size_t)wi.n_dt * wi.n_ct * wi.maxj;
+  return slots * ((size_t)4 * WG_BC * WG_BD + WG_BD) * sizeof(float);
 }
 
-cudaError_t launch_wgrad_tc_finalize(const float* part, const float* bpart, int splits, int C,
-                                     int D, void* dW, void* dbias, const Twiddles& tw,
-                                     cudaStream_t st) {
-  const int64_t total = std::max<int64_t>((int64_t)C * D, D);
-  const unsigned blocks = (unsigned)((total + 255) / 256);
-  wgrad_tc_finalize_kernel<<<blocks, 256, 0, st>>>(part, bpart, splits, C, D,
-                                                    static_cast<__half*>(dW),
-                                                    static_cast<__half*>(dbias), tw);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D, float* part,
-                            float* bpart, int splits, int* status, int num_sms, cudaStream_t st) {
-  if (N <= 0 || splits <= 0) return cudaSuccess;
+cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
+                            void* workspace, void* dW, void* dbias, int* status, int num_sms,
+                            const Twiddles& tw, cudaStream_t st) {
+  WgInfo wi;
+  int grid = 0;
+  if (!wgrad_tc_layout(N, C, D, num_sms, &wi, &grid)) return cudaErrorInvalidValue;
   CUtensorMap mg, mx;
   if (!encode_rows_map(&mg, dY, D, N) || !encode_rows_map(&mx, X, C, N))
     return cudaErrorInvalidValue;
-  WgInfo wi;
-  wi.n_dt = (D + WG_BD - 1) / WG_BD;
-  wi.n_ct = (C + WG_BC - 1) / WG_BC;
-  wi.rows_per_split = wgrad_tc_rows_per_split(N, splits);
-  const int64_t units = (int64_t)wi.n_dt * wi.n_ct * splits;
-  if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
-  wi.num_units = (int)units;
+  float* part = static_cast<float*>(workspace);
+  float* bpart = part + (size_t)wi.n_dt * wi.n_ct * wi.maxj * (4 * WG_BC * WG_BD);
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(wgrad_tc_kernel,
@@ -438,8 +479,12 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int grid = wi.num_units < num_sms ? wi.num_units : num_sms;
   wgrad_tc_kernel<<<grid, WG_THREADS, WG_SMEM, st>>>(mg, mx, N, C, D, wi, part, bpart, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t total = std::max<int64_t>((int64_t)C * D, D);
+  wgrad_tc_finalize_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+      part, bpart, wi, C, D, static_cast<__half*>(dW), static_cast<__half*>(dbias), tw);
   return cudaGetLastError();
 }
 
