@@ -12,7 +12,10 @@ Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|referenc
        [--workload p4_vitb_mlp_f16|p4_vitb_proj_f32|p4_vith_fc1_f16|c8_1024_f16|
                    p4_vith_fc1_fwd_bwd_f16|p4_vitb_mlp_block_f16|p4_vitb_mlp_spectral_f16]
 Under torchrun (N > 1) every rank runs its own copy of the workload (weak
-scaling; rows are independent, so no collective is on the data path).
+scaling; rows are independent, so no collective is on the forward path).  The
+training workload is then data parallel: each rank's FP32 weight gradient is
+summed over ranks by one NCCL all-reduce, queued behind dW while dX runs, and
+rounded once.
 """
 from __future__ import annotations
 
@@ -355,6 +358,7 @@ def run_ours(args, workload):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     from group_circulant_gemm_b200 import EqLinearPlan
+    from group_circulant_gemm_b200.parallel import allreduce_grad_buffer
 
     backward = workload in BACKWARD
     pipeline = [WORKLOADS[n] for n in PIPELINES[workload]]
@@ -384,12 +388,16 @@ def run_ours(args, workload):
     xs = [torch.from_numpy(x_host).cuda() for _ in range(nsets)]
     outs = [[torch.empty((N, w.D * w.T), dtype=dt, device="cuda") for w in pipeline]
             for _ in range(nsets)]
+    # data parallel: every rank trains on its own rows; the weight gradient is
+    # summed over ranks in FP32 (one NCCL all-reduce) and rounded once
+    dp = backward and (world > 1 or args.dp_path)
     if backward:
         w0 = pipeline[0]
         dys = [torch.from_numpy(dy_host).cuda() for _ in range(nsets)]
         dxs = [torch.empty((N, w0.C * w0.T), dtype=dt, device="cuda") for _ in range(nsets)]
-        dW = torch.empty((w0.D, w0.C, w0.T), dtype=dt, device="cuda")
-        db = torch.empty((w0.D,), dtype=dt, device="cuda")
+        gbuf = plans[0].grad_buffer(dt)
+        dW, db = plans[0].split_grad(gbuf)
+        gbuf32 = plans[0].grad_buffer(torch.float32) if dp else None
         ws = torch.empty(max(16, plans[0].workspace_bytes(N)), dtype=torch.uint8, device="cuda")
 
     # the ops of one step: (label, kernel, flops, algorithmic bytes, callable(set index))
@@ -416,17 +424,36 @@ def run_ours(args, workload):
                     fwd))
     if backward:
         w0 = pipeline[0]
+        pending = []
 
         def bwd_x(i):
             plans[0].backward_input(dys[i % nsets], whats[0], out=dxs[i % nsets])
 
         def bwd_w(i):
-            plans[0].backward_weight(xs[i % nsets], dys[i % nsets], dW=dW, dbias=db, workspace=ws)
+            if dp:
+                plans[0].backward_weight_f32(xs[i % nsets], dys[i % nsets], buf=gbuf32,
+                                             workspace=ws)
+                # queued behind dW; dX runs on the compute stream meanwhile
+                pending.append(allreduce_grad_buffer(gbuf32, async_op=True))
+            else:
+                plans[0].backward_weight(xs[i % nsets], dys[i % nsets], dW=dW, dbias=db,
+                                         workspace=ws)
+
+        def grad_sync(i):
+            handle = pending.pop()
+            if handle is not None:  # None: one rank, nothing was reduced
+                handle.wait()
+            plans[0].cast_from_f32(gbuf32, out=gbuf)
         nb = es * (N * w0.C * w0.T + N * w0.D * w0.T)
-        ops.append(("backward_input", plans[0].forward_kernel_name(N), layer_flops(w0),
-                    nb + es * 1.25 * w0.C * w0.D * w0.T, bwd_x))
-        ops.append(("backward_weight", plans[0].backward_weight_kernel_name(N), wgrad_flops(w0),
-                    nb + es * w0.D * w0.C * w0.T, bwd_w))
+        op_dx = ("backward_input", plans[0].forward_kernel_name(N), layer_flops(w0),
+                 nb + es * 1.25 * w0.C * w0.D * w0.T, bwd_x)
+        op_dw = ("backward_weight", plans[0].backward_weight_kernel_name(N), wgrad_flops(w0),
+                 nb + es * w0.D * w0.C * w0.T, bwd_w)
+        if dp:
+            ops += [op_dw, op_dx, ("weight_grad_allreduce", "nccl+cast", 0.0,
+                                   (4 + es) * gbuf.numel(), grad_sync)]
+        else:
+            ops += [op_dx, op_dw]
 
     def step(i, events=None):
         for _, _, _, _, fn in ops:
@@ -477,7 +504,7 @@ def run_ours(args, workload):
     if backward:
         dy_pin = torch.from_numpy(dy_host).pin_memory()
         dx_pin = torch.empty(tuple(dxs[0].shape), dtype=dt).pin_memory()
-        dw_pin = torch.empty(tuple(dW.shape), dtype=dt).pin_memory()
+        dw_pin = torch.empty(tuple(gbuf.shape), dtype=dt).pin_memory()
         h2d += dy_pin.numel() * dy_pin.element_size()
         d2h += (dx_pin.numel() + dw_pin.numel()) * dx_pin.element_size()
 
@@ -489,7 +516,7 @@ def run_ours(args, workload):
         y_pin.copy_(outs[0][-1], non_blocking=True)
         if backward:
             dx_pin.copy_(dxs[0], non_blocking=True)
-            dw_pin.copy_(dW, non_blocking=True)
+            dw_pin.copy_(gbuf, non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -574,7 +601,9 @@ def run_ours(args, workload):
                                    + (2 * dense_flops(pipeline[0]) if backward else 0))
                                   * args.steps * world / (elapsed_ms / 1e3) / 1e12,
             "config": {"workload": DESCR[workload], "global_batch": N * world, "seq_len": None,
-                       "parallelism": f"replicas x{world} (rows independent)",
+                       "parallelism": (f"data parallel x{world}: rows sharded, dW/dbias "
+                                       "FP32 NCCL all-reduce overlapped with dX"
+                                       if dp else f"replicas x{world} (rows independent)"),
                        "l2": f"{nsets} rotating input/output sets of {per_set / 2**20:.0f} MiB "
                              "(> 2x L2)",
                        "kernels": [f"{label}[{k}]" for label, k, _, _, _ in ops]},
@@ -586,6 +615,7 @@ def run_ours(args, workload):
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
             "gpu_launches": args.steps * sum(2 if label == "backward_weight" else 1
                                              for label, _, _, _, _ in ops),
+            # (the all-reduce op counts its cast kernel; NCCL's own kernel is not ours)
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
@@ -606,6 +636,9 @@ def main():
     ap.add_argument("--workload", choices=list(PIPELINES), default="p4_vitb_mlp_f16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense F.linear comparator")
+    ap.add_argument("--dp-path", action="store_true",
+                    help="training workload: take the data-parallel weight-gradient path "
+                         "(FP32 sums, reduction over ranks, one cast) even on one rank")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps, reported as run
     if args.impl == "reference":

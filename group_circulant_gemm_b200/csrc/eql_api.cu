@@ -294,9 +294,10 @@ size_t eqlinear_backward_weight_workspace_bytes(eqlinear_plan_t p, int64_t N) {
   return need;
 }
 
-eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t p, const void* X, const void* dY,
-                                           int64_t N, void* dW, void* dbias, void* workspace,
-                                           size_t workspace_bytes, void* stream) {
+static eqlinear_status_t backward_weight_impl(eqlinear_plan_t p, const void* X, const void* dY,
+                                              int64_t N, void* dW, void* dbias, void* workspace,
+                                              size_t workspace_bytes, eql::DType out_dt,
+                                              void* stream) {
   if (!p || N < 0 || !dW) return EQL_ERR_INVALID_ARG;
   if (N > 0 && (!X || !dY)) return EQL_ERR_INVALID_ARG;
   if ((X && !aligned16(X)) || (dY && !aligned16(dY)) || !aligned16(dW) ||
@@ -309,12 +310,44 @@ eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t p, const void* X, con
   if (s != EQL_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   if (wgrad_use_tc(p, N, X, dY))
-    return from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, workspace, dW, dbias, p->status,
-                                          p->num_sms, p->tw, st));
+    return from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, workspace, out_dt, dW, dbias,
+                                          p->status, p->num_sms, p->tw, st));
   const int splits = eql::wgrad_simt_splits(p->T, N, p->C, p->D, p->num_sms);
-  return from_cuda(eql::launch_wgrad_simt(p->T, to_dt(p->dtype), X, dY, N, p->C, p->D, dW,
-                                          dbias, static_cast<float*>(workspace), splits, p->tw,
-                                          st));
+  return from_cuda(eql::launch_wgrad_simt(p->T, to_dt(p->dtype), out_dt, X, dY, N, p->C, p->D,
+                                          dW, dbias, static_cast<float*>(workspace), splits,
+                                          p->tw, st));
+}
+
+eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t p, const void* X, const void* dY,
+                                           int64_t N, void* dW, void* dbias, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  if (!p) return EQL_ERR_INVALID_ARG;
+  return backward_weight_impl(p, X, dY, N, dW, dbias, workspace, workspace_bytes,
+                              to_dt(p->dtype), stream);
+}
+
+eqlinear_status_t eqlinear_backward_weight_f32(eqlinear_plan_t p, const void* X, const void* dY,
+                                               int64_t N, float* dW, float* dbias,
+                                               void* workspace, size_t workspace_bytes,
+                                               void* stream) {
+  return backward_weight_impl(p, X, dY, N, dW, dbias, workspace, workspace_bytes,
+                              eql::DType::F32, stream);
+}
+
+eqlinear_status_t eqlinear_cast_from_f32(eqlinear_plan_t p, const float* src, int64_t count,
+                                         void* dst, void* stream) {
+  if (!p || count < 0) return EQL_ERR_INVALID_ARG;
+  if (count == 0) return EQL_OK;
+  if (!src || !dst) return EQL_ERR_INVALID_ARG;
+  const char* s0 = reinterpret_cast<const char*>(src);
+  const char* d0 = static_cast<const char*>(dst);
+  const size_t sb = (size_t)count * sizeof(float), db = (size_t)count * elem_size(p->dtype);
+  const bool same_f32 = s0 == d0 && p->dtype == EQL_F32;  // a no-op
+  if (!same_f32 && s0 < d0 + db && d0 < s0 + sb) return EQL_ERR_INVALID_ARG;  // overlap
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_cast_from_f32(to_dt(p->dtype), src, dst, count,
+                                             (cudaStream_t)stream));
 }
 
 eqlinear_status_t eqlinear_get_status(eqlinear_plan_t p, void* stream) {

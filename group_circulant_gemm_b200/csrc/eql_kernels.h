@@ -26,16 +26,17 @@ cudaError_t launch_fwd_simt(int T, DType dt, const void* X, int64_t N, int Cin, 
                             int act, cudaStream_t st);
 
 // CUDA-core weight gradient: split reduction over rows into FP32 partial spectra,
-// then a finalize kernel (sum in fixed split order, inverse DFT, cast).
+// then a finalize kernel (sum in fixed split order, inverse DFT, cast to out_dt).
 int wgrad_simt_splits(int T, int64_t N, int C, int D, int num_sms);
 size_t wgrad_simt_workspace(int T, int64_t N, int C, int D, int num_sms);
-cudaError_t launch_wgrad_simt(int T, DType dt, const void* X, const void* dY, int64_t N, int C,
-                              int D, void* dW, void* dbias, float* ws, int splits,
-                              const Twiddles& tw, cudaStream_t st);
+cudaError_t launch_wgrad_simt(int T, DType dt, DType out_dt, const void* X, const void* dY,
+                              int64_t N, int C, int D, void* dW, void* dbias, float* ws,
+                              int splits, const Twiddles& tw, cudaStream_t st);
 
 // Finalize of a split weight-gradient reduction: partial spectra
-// part[split][T planes][D][C] (+ bias partials [split][D]) -> dW[D][C][T], dbias[D].
-cudaError_t launch_wgrad_finalize(int T, DType dt, const float* part, const float* bpart,
+// part[split][T planes][D][C] (+ bias partials [split][D]) -> dW[D][C][T], dbias[D]
+// in out_dt.
+cudaError_t launch_wgrad_finalize(int T, DType out_dt, const float* part, const float* bpart,
                                   int splits, int C, int D, void* dW, void* dbias,
                                   const Twiddles& tw, cudaStream_t st);
 
@@ -61,12 +62,17 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
 
 // tcgen05/TMEM tensor-core weight gradient for T = 4, FP16: stream-K over
 // (tile, 32-row stage) ranges, FP32 partial slots in `workspace`, then a
-// fixed-order finalize (inverse DFT, cast) into dW [D][C][4] and dbias [D].
-// X and dY must be 16-byte aligned (TMA).  N = 0 is handled by the caller.
+// fixed-order finalize (inverse DFT, cast to out_dt: F16 or F32) into
+// dW [D][C][4] and dbias [D].  X and dY must be 16-byte aligned (TMA).  N = 0 is
+// handled by the caller.
 bool wgrad_tc_supported(int T, DType dt, int64_t N, int C, int D, const void* X, const void* dY);
 size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms);
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
-                            void* workspace, void* dW, void* dbias, int* status, int num_sms,
-                            const Twiddles& tw, cudaStream_t st);
+                            void* workspace, DType out_dt, void* dW, void* dbias, int* status,
+                            int num_sms, const Twiddles& tw, cudaStream_t st);
+
+// dst[i] = src[i] rounded to nearest-even in dt (a copy for F32), i < n.
+cudaError_t launch_cast_from_f32(DType dt, const float* src, void* dst, int64_t n,
+                                 cudaStream_t st);
 
 }  // namespace eql

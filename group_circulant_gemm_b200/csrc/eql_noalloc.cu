@@ -71,8 +71,9 @@ extern "C" eqlinear_status_t eqlinear_backward_weight_noalloc(eqlinear_plan_t p,
   const int fit = (int)(kScratchFloats / per_split);
   if (splits > fit) splits = fit;
   const eql::DType dt = p->dtype == EQL_F32 ? eql::DType::F32 : eql::DType::F16;
-  const cudaError_t e = eql::launch_wgrad_simt(p->T, dt, X, dY, N, p->C, p->D, dW, dbias,
-                                               scratch, splits, p->tw, (cudaStream_t)stream);
+  const cudaError_t e = eql::launch_wgrad_simt(p->T, dt, dt, X, dY, N, p->C, p->D, dW,
+                                               dbias, scratch, splits, p->tw,
+                                               (cudaStream_t)stream);
   if (e == cudaSuccess) return EQL_OK;
   return e == cudaErrorNotSupported ? EQL_ERR_UNSUPPORTED : EQL_ERR_CUDA;
 }

@@ -452,14 +452,14 @@ size_t wgrad_simt_workspace(int T, int64_t N, int C, int D, int num_sms) {
   return (size_t)splits * ((size_t)T * C * D + D) * sizeof(float);
 }
 
-cudaError_t launch_wgrad_finalize(int T, DType dt, const float* part, const float* bpart,
+cudaError_t launch_wgrad_finalize(int T, DType out_dt, const float* part, const float* bpart,
                                   int splits, int C, int D, void* dW, void* dbias,
                                   const Twiddles& tw, cudaStream_t st) {
   const int64_t total = std::max<int64_t>((int64_t)C * D, D);
   const unsigned blocks = (unsigned)((total + 255) / 256);
   return dispatch_T(T, [&](auto tc) {
     constexpr int TT = decltype(tc)::value;
-    if (dt == DType::F32)
+    if (out_dt == DType::F32)
       wgrad_finalize_kernel<TT, float><<<blocks, 256, 0, st>>>(part, bpart, splits, C, D,
                                                                (float*)dW, (float*)dbias, tw);
     else
@@ -469,9 +469,9 @@ cudaError_t launch_wgrad_finalize(int T, DType dt, const float* part, const floa
   });
 }
 
-cudaError_t launch_wgrad_simt(int T, DType dt, const void* X, const void* dY, int64_t N, int C,
-                              int D, void* dW, void* dbias, float* ws, int splits,
-                              const Twiddles& tw, cudaStream_t st) {
+cudaError_t launch_wgrad_simt(int T, DType dt, DType out_dt, const void* X, const void* dY,
+                              int64_t N, int C, int D, void* dW, void* dbias, float* ws,
+                              int splits, const Twiddles& tw, cudaStream_t st) {
   float* part = ws;
   float* bpart = ws + (size_t)splits * T * C * D;
   if (N > 0) {
@@ -491,7 +491,49 @@ cudaError_t launch_wgrad_simt(int T, DType dt, const void* X, const void* dY, in
     });
     if (e != cudaSuccess) return e;
   }
-  return launch_wgrad_finalize(T, dt, part, bpart, N > 0 ? splits : 0, C, D, dW, dbias, tw, st);
+  return launch_wgrad_finalize(T, out_dt, part, bpart, N > 0 ? splits : 0, C, D, dW, dbias, tw,
+                               st);
+}
+
+namespace {
+
+// Four elements per thread (16-byte loads, 8-byte stores) when both pointers
+// allow it, else one.
+__global__ void cast_from_f32_kernel(const float* __restrict__ src, __half* __restrict__ dst,
+                                     int64_t n, int vec) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  int64_t done = 0;
+  if (vec) {
+    const int64_t n4 = n / 4;
+    for (int64_t i = t0; i < n4; i += stride) {
+      const float4 v = reinterpret_cast<const float4*>(src)[i];
+      const __half2 lo = __floats2half2_rn(v.x, v.y), hi = __floats2half2_rn(v.z, v.w);
+      uint2 o;
+      o.x = *reinterpret_cast<const uint32_t*>(&lo);
+      o.y = *reinterpret_cast<const uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(dst)[i] = o;
+    }
+    done = n4 * 4;
+  }
+  for (int64_t i = done + t0; i < n; i += stride) dst[i] = __float2half_rn(src[i]);
+}
+
+}  // namespace
+
+cudaError_t launch_cast_from_f32(DType dt, const float* src, void* dst, int64_t n,
+                                 cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  if (dt == DType::F32) {
+    if (static_cast<const void*>(src) == dst) return cudaSuccess;
+    return cudaMemcpyAsync(dst, src, (size_t)n * sizeof(float), cudaMemcpyDeviceToDevice, st);
+  }
+  const int vec = ((reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
+                   (reinterpret_cast<uintptr_t>(dst) & 7) == 0) ? 1 : 0;
+  const int64_t want = ((vec ? n / 4 : n) + 255) / 256;
+  const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, 148 * 8));
+  cast_from_f32_kernel<<<blocks, 256, 0, st>>>(src, static_cast<__half*>(dst), n, vec);
+  return cudaGetLastError();
 }
 
 }  // namespace eql

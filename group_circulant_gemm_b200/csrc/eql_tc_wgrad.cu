@@ -364,13 +364,25 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
   }
 }
 
-// Sum of a tile's partial slots (fixed order), inverse group DFT, cast:
+__device__ __forceinline__ void store_dw4(__half* p, const float* w) {
+  __half2* out = reinterpret_cast<__half2*>(p);
+  out[0] = __floats2half2_rn(w[0], w[1]);
+  out[1] = __floats2half2_rn(w[2], w[3]);
+}
+__device__ __forceinline__ void store_dw4(float* p, const float* w) {
+  *reinterpret_cast<float4*>(p) = make_float4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ void store_one(__half* p, float v) { *p = __float2half_rn(v); }
+__device__ __forceinline__ void store_one(float* p, float v) { *p = v; }
+
+// Sum of a tile's partial slots (fixed order), inverse group DFT, cast to Out:
 // dW[d][c][u] from part[tile][j][4][128 c][128 d]; dbias[d] from
 // bpart[tile][j][128] of the tiles with in-channel tile 0.
+template <typename Out>
 __global__ void wgrad_tc_finalize_kernel(const float* __restrict__ part,
                                          const float* __restrict__ bpart, WgInfo wi, int C,
-                                         int D, __half* __restrict__ dW,
-                                         __half* __restrict__ dbias, Twiddles tw) {
+                                         int D, Out* __restrict__ dW, Out* __restrict__ dbias,
+                                         Twiddles tw) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // c * D + d
   if (idx < (int64_t)D * C) {
     const int c = (int)(idx / D), d = (int)(idx % D);
@@ -386,9 +398,7 @@ __global__ void wgrad_tc_finalize_kernel(const float* __restrict__ part,
     }
     float wv[4];
     group_idft<4>(qv, wv, tw);
-    __half2* out = reinterpret_cast<__half2*>(dW + ((int64_t)d * C + c) * 4);
-    out[0] = __floats2half2_rn(wv[0], wv[1]);
-    out[1] = __floats2half2_rn(wv[2], wv[3]);
+    store_dw4(dW + ((int64_t)d * C + c) * 4, wv);
   }
   if (dbias && idx < D) {
     const int d = (int)idx;
@@ -398,7 +408,7 @@ __global__ void wgrad_tc_finalize_kernel(const float* __restrict__ part,
     float b = 0.f;
     for (int j = 0; j <= last - first; ++j)
       b += bpart[((int64_t)tile * wi.maxj + j) * WG_BD + d % WG_BD];
-    dbias[idx] = __float2half_rn(b);
+    store_one(dbias + idx, b);
   }
 }
 
@@ -462,8 +472,8 @@ size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms) {
 }
 
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
-                            void* workspace, void* dW, void* dbias, int* status, int num_sms,
-                            const Twiddles& tw, cudaStream_t st) {
+                            void* workspace, DType out_dt, void* dW, void* dbias, int* status,
+                            int num_sms, const Twiddles& tw, cudaStream_t st) {
   WgInfo wi;
   int grid = 0;
   if (!wgrad_tc_layout(N, C, D, num_sms, &wi, &grid)) return cudaErrorInvalidValue;
@@ -483,8 +493,13 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t total = std::max<int64_t>((int64_t)C * D, D);
-  wgrad_tc_finalize_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
-      part, bpart, wi, C, D, static_cast<__half*>(dW), static_cast<__half*>(dbias), tw);
+  const unsigned fblocks = (unsigned)((total + 255) / 256);
+  if (out_dt == DType::F32)
+    wgrad_tc_finalize_kernel<float><<<fblocks, 256, 0, st>>>(
+        part, bpart, wi, C, D, static_cast<float*>(dW), static_cast<float*>(dbias), tw);
+  else
+    wgrad_tc_finalize_kernel<__half><<<fblocks, 256, 0, st>>>(
+        part, bpart, wi, C, D, static_cast<__half*>(dW), static_cast<__half*>(dbias), tw);
   return cudaGetLastError();
 }
 

@@ -126,5 +126,49 @@ class EqLinearPlan:
                                     workspace.numel() * workspace.element_size())
         return dW, dbias
 
+    # --- data-parallel weight gradient: FP32 per-rank sums, one reduction, one cast
+
+    def grad_offset(self) -> int:
+        """Element offset of dbias in a flat gradient buffer (dW first, padded to 8)."""
+        return (self.D * self.C * self.T + 7) // 8 * 8
+
+    def grad_buffer(self, dtype: torch.dtype = torch.float32, device="cuda") -> torch.Tensor:
+        """A zeroed flat buffer holding dW [D, C, T] then dbias [D], so one
+        collective reduces both."""
+        return torch.zeros(self.grad_offset() + self.D, dtype=dtype, device=device)
+
+    def split_grad(self, buf: torch.Tensor):
+        """(dW, dbias) views of a flat gradient buffer."""
+        off = self.grad_offset()
+        return buf[:self.D * self.C * self.T].view(self.D, self.C, self.T), buf[off:off + self.D]
+
+    def backward_weight_f32(self, X, dY, buf=None, workspace=None) -> torch.Tensor:
+        """This rank's dW and dbias as FP32 sums in a flat buffer (before the cast)."""
+        N = X.shape[0]
+        self._check(X, (N, self.C * self.T), "X")
+        self._check(dY, (N, self.D * self.T), "dY")
+        if buf is None:
+            buf = self.grad_buffer(torch.float32, X.device)
+        if buf.dtype != torch.float32 or buf.numel() != self.grad_offset() + self.D:
+            raise ValueError("buf must be a flat FP32 gradient buffer of this plan")
+        dW, db = self.split_grad(buf)
+        nb = self.workspace_bytes(N)
+        if workspace is None:
+            workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=X.device)
+        _n.eqlinear_backward_weight_f32(self.handle, X, dY, N, dW, db, workspace,
+                                        workspace.numel() * workspace.element_size())
+        return buf
+
+    def cast_from_f32(self, src: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+        """Round an FP32 tensor to the plan dtype on the GPU (nearest-even)."""
+        if not src.is_cuda or src.dtype != torch.float32 or not src.is_contiguous():
+            raise ValueError("src must be a contiguous CUDA FP32 tensor")
+        if out is None:
+            out = torch.empty(tuple(src.shape), dtype=self.dtype, device=src.device)
+        if out.dtype != self.dtype or out.numel() != src.numel() or not out.is_contiguous():
+            raise ValueError("out must be a contiguous tensor of the plan dtype, same size")
+        _n.eqlinear_cast_from_f32(self.handle, src, src.numel(), out)
+        return out
+
     def status(self) -> int:
         return _n.eqlinear_get_status(self.handle)

@@ -29,6 +29,7 @@ EXPORTED = (
     "eqlinear_backward_input",
     "eqlinear_backward_weight_workspace_bytes", "eqlinear_backward_weight",
     "eqlinear_get_status", "eqlinear_backward_weight_noalloc",
+    "eqlinear_backward_weight_f32", "eqlinear_cast_from_f32",
 )
 
 
@@ -65,6 +66,8 @@ def _load() -> ctypes.CDLL:
         "eqlinear_backward_weight": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
         "eqlinear_get_status": ([vp, vp], i32),
         "eqlinear_backward_weight_noalloc": ([vp, vp, vp, i64, vp, vp, vp], i32),
+        "eqlinear_backward_weight_f32": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
+        "eqlinear_cast_from_f32": ([vp, vp, i64, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -183,6 +186,18 @@ def eqlinear_backward_weight(plan: int, X, dY, N: int, dW, dbias, workspace,
     _check(_lib.eqlinear_backward_weight(plan, _ptr(X), _ptr(dY), N, _ptr(dW), _ptr(dbias),
                                          _ptr(workspace), workspace_bytes, _stream(stream)),
            "eqlinear_backward_weight")
+
+
+def eqlinear_backward_weight_f32(plan: int, X, dY, N: int, dW, dbias, workspace,
+                                 workspace_bytes: int, stream=None) -> None:
+    _check(_lib.eqlinear_backward_weight_f32(plan, _ptr(X), _ptr(dY), N, _ptr(dW), _ptr(dbias),
+                                             _ptr(workspace), workspace_bytes, _stream(stream)),
+           "eqlinear_backward_weight_f32")
+
+
+def eqlinear_cast_from_f32(plan: int, src, count: int, dst, stream=None) -> None:
+    _check(_lib.eqlinear_cast_from_f32(plan, _ptr(src), count, _ptr(dst), _stream(stream)),
+           "eqlinear_cast_from_f32")
 
 
 def eqlinear_backward_weight_noalloc(plan: int, X, dY, N: int, dW, dbias, stream=None) -> None:

@@ -2,8 +2,12 @@
 
 The layer's forward and input gradient shard over the N rows with no exchange
 at all; the weight gradient of a row-sharded batch is the sum over ranks of
-each rank's partial dW (and dbias), one all-reduce.  These helpers hold that
-host logic; the arithmetic runs in the CUDA library on each rank.
+each rank's partial dW (and dbias), one all-reduce.  Each rank writes its FP32
+sums into one flat buffer (``EqLinearPlan.backward_weight_f32``), the buffer is
+summed over ranks in FP32, and one cast rounds it (``cast_from_f32``), so the
+ranks' contributions meet before the single rounding a one-rank run has.
+These helpers hold that host logic; the arithmetic runs in the CUDA library on
+each rank.
 """
 from __future__ import annotations
 
@@ -29,15 +33,16 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
-def allreduce_weight_grad(dW: torch.Tensor, dbias: torch.Tensor | None = None):
-    """Sum per-rank partial weight gradients in FP32; returns tensors in dW's dtype."""
+def allreduce_grad_buffer(buf: torch.Tensor, async_op: bool = False):
+    """Sum a flat FP32 gradient buffer (dW then dbias) over ranks, in place.
+
+    With ``async_op`` the reduction is queued behind the work already on the
+    current stream and a handle is returned; ``handle.wait()`` makes the current
+    stream wait for it, so independent kernels (dX) can run in between.  Returns
+    None when there is nothing to reduce (one rank).
+    """
+    if buf.dtype != torch.float32:
+        raise ValueError("the data-parallel gradient is reduced in FP32")
     if not dist.is_initialized() or dist.get_world_size() == 1:
-        return dW, dbias
-    acc = dW.float()
-    dist.all_reduce(acc, op=dist.ReduceOp.SUM)
-    out_b = None
-    if dbias is not None:
-        bacc = dbias.float()
-        dist.all_reduce(bacc, op=dist.ReduceOp.SUM)
-        out_b = bacc.to(dbias.dtype)
-    return acc.to(dW.dtype), out_b
+        return None
+    return dist.all_reduce(buf, op=dist.ReduceOp.SUM, async_op=async_op)

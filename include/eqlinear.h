@@ -229,6 +229,36 @@ EQL_API eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t plan, const v
                                            size_t workspace_bytes, void* stream);
 
 /*
+ * Data-parallel form of the weight gradient.  dW and dbias are sums over rows,
+ * so a batch split by rows across ranks has dW = the sum over ranks of each
+ * rank's dW.  To add the ranks' contributions in FP32 (one rounding to the plan
+ * dtype at the end, as for a single rank), each rank calls
+ * eqlinear_backward_weight_f32 on its rows, the ranks sum the FP32 results
+ * (an all-reduce), and eqlinear_cast_from_f32 rounds the sum.  The page
+ * describing the layer trains on one device and has no counterpart to these
+ * two calls.
+ *
+ * eqlinear_backward_weight_f32: the same computation, kernels and arguments as
+ * eqlinear_backward_weight, except that dW [D][C][T] and dbias [D] (or NULL)
+ * are FP32 whatever the plan dtype: the fixed-order FP32 sums before the final
+ * cast.  Rounding that output to the plan dtype gives exactly what
+ * eqlinear_backward_weight writes.  dW must be 16-byte aligned.
+ */
+EQL_API eqlinear_status_t eqlinear_backward_weight_f32(eqlinear_plan_t plan, const void* X,
+                                                       const void* dY, int64_t N, float* dW,
+                                                       float* dbias, void* workspace,
+                                                       size_t workspace_bytes, void* stream);
+
+/*
+ * dst[i] = src[i] rounded to nearest-even in the plan dtype, for i < count
+ * (a copy for FP32 plans).  src: count FP32 values on the plan's device; dst:
+ * count values of the plan dtype; the two must not overlap (an FP32 plan may
+ * pass dst == src, which does nothing).  Asynchronous on `stream`.
+ */
+EQL_API eqlinear_status_t eqlinear_cast_from_f32(eqlinear_plan_t plan, const float* src,
+                                                 int64_t count, void* dst, void* stream);
+
+/*
  * Weight gradient for callers that cannot allocate device memory.  The page
  * describing the layer has no counterpart to this call; it exists for users of
  * this library whose device memory is all owned by another allocator or fixed
