@@ -41,6 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # workload name -> list of layer workloads applied in sequence (output feeds the next)
 PIPELINES = {
     "p4_vitb_mlp_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
+    "p4_vitb_mlp_2calls_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
     "p4_vitb_proj_f32": ["p4_vitb_proj_f32"],
     "p4_vith_fc1_f16": ["p4_vith_fc1_f16"],
     "c8_1024_f16": ["c8_1024_f16"],
@@ -52,6 +53,9 @@ PIPELINES = {
 # layer's epilogue writes the second layer's operand planes)
 SPECTRAL = {"p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectral_f16"}
 BACKWARD = {"p4_vith_fc1_fwd_bwd_f16"}
+# two-layer pipelines run as one chained launch (eqlinear_forward_chain: both
+# layers' tiles in one dynamic queue; bitwise the two separate calls)
+CHAINED = {"p4_vitb_mlp_f16", "p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectral_f16"}
 # per-layer output activation (fused into that layer's epilogue); default none
 ACTS = {"p4_vitb_mlp_block_f16": ["gelu", "none"]}
 
@@ -60,7 +64,9 @@ def acts_of(workload):
     return ACTS.get(workload, ["none"] * len(PIPELINES[workload]))
 DESCR = {
     "p4_vitb_mlp_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
-                       "C=768->D=192, T=4",
+                       "C=768->D=192, T=4; both layers in one chained launch",
+    "p4_vitb_mlp_2calls_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
+                              "C=768->D=192, T=4; one launch per layer",
     "p4_vitb_proj_f32": "p4 EQ-Linear fp32 ViT-B projection: N=12608, C=D=192, T=4",
     "p4_vith_fc1_f16": "p4 EQ-Linear fp16 ViT-H fc1: N=8224, C=320->D=1280, T=4",
     "c8_1024_f16": "cyclic T=8 EQ-Linear fp16: N=16384, C=D=128",
@@ -68,10 +74,10 @@ DESCR = {
                                "C=320->D=1280, T=4",
     "p4_vitb_mlp_block_f16": "p4 EQ-MLP block fp16 ViT-B: N=12608, EQ-Linear 192->768 + bias + "
                              "GELU (fused), EQ-Linear 768->192 + bias, T=4; intermediate kept as "
-                             "the second layer's spectral planes",
+                             "the second layer's spectral planes; one chained launch",
     "p4_vitb_mlp_spectral_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
                                 "C=768->D=192, T=4; intermediate kept as the second layer's "
-                                "spectral planes",
+                                "spectral planes; one chained launch",
 }
 
 
@@ -90,21 +96,15 @@ def layer_bytes(w) -> float:
     return es * (w.N * w.C * w.T + w.N * w.D * w.T + planes * w.C * w.D + w.D)
 
 
-# DRAM traffic per forward launch (dram__bytes_read.sum + dram__bytes_write.sum),
-# from the ncu captures summarised in profiles/, valid only for the kernel source
-# they were taken on (SHA-256 prefix of csrc/eql_tc_fwd.cu); any other source
-# reports null.
 # DRAM bytes (read + write) per launch of the step's dominant kernel, from the
 # ncu captures summarised under profiles/, keyed by a hash of the kernel's
 # sources: a changed kernel reports null until it is captured again.
 KERNEL_SOURCES = {
-    "forward": ("eql_tc_fwd.cu", "eql_tc_common.cuh"),
+    "forward": ("eql_tc_fwd.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
+    "forward_chain": ("eql_tc_chain.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
     "backward_weight": ("eql_tc_wgrad.cu", "eql_tc_common.cuh"),
 }
-NCU_TRAFFIC = {
-    ("forward", "7f61d3dc196bce45"): {"p4_vitb_mlp_f16": 58.94e6, "c8_1024_f16": 34.02e6,
-                                      "p4_vith_fc1_fwd_bwd_f16": 70.12e6},
-}
+NCU_TRAFFIC = {}
 
 def kernel_traffic(family: str, workload: str):
     import hashlib
@@ -357,7 +357,7 @@ def run_ours(args, workload):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    from group_circulant_gemm_b200 import EqLinearPlan
+    from group_circulant_gemm_b200 import EqLinearPlan, forward_chain, native
     from group_circulant_gemm_b200.parallel import allreduce_grad_buffer
 
     backward = workload in BACKWARD
@@ -408,7 +408,19 @@ def run_ours(args, workload):
         # the first layer writes the second layer's input planes [4, N, H]
         outs = [[torch.empty((4, N, pipeline[0].D), dtype=dt, device="cuda"), o[1]]
                 for o in outs]
-    for li, w in enumerate(pipeline):
+    chained = workload in CHAINED
+    if chained:
+        ws_chain = torch.zeros(max(16, native.eqlinear_chain_workspace_bytes(
+            plans[0].handle, plans[1].handle, N)), dtype=torch.uint8, device="cuda")
+
+        def fwd_chain(i):
+            o = outs[i % nsets]
+            forward_chain(plans[0], plans[1], xs[i % nsets], whats[0], biases[0], whats[1],
+                          biases[1], act=acts[0], spectral=spectral, H=o[0], Y=o[1],
+                          workspace=ws_chain)
+        ops.append(("forward_chain", "tcgen05", sum(layer_flops(w) for w in pipeline),
+                    sum(layer_bytes(w) for w in pipeline), fwd_chain))
+    for li, w in enumerate([] if chained else pipeline):
         def fwd(i, li=li):
             x = xs[i % nsets] if li == 0 else outs[i % nsets][li - 1]
             if spectral and li == 0:

@@ -7,12 +7,12 @@ of ``native`` or ``EqLinearPlan`` does, and raises if it is missing.
 """
 import importlib
 
-__all__ = ["EqLinearPlan", "native", "synth"]
+__all__ = ["EqLinearPlan", "forward_chain", "native", "synth"]
 
 
 def __getattr__(name):
-    if name == "EqLinearPlan":
-        return importlib.import_module(".layer", __name__).EqLinearPlan
+    if name in ("EqLinearPlan", "forward_chain"):
+        return getattr(importlib.import_module(".layer", __name__), name)
     if name in ("native", "synth", "layer", "build"):
         return importlib.import_module("." + name, __name__)
     raise AttributeError(name)

@@ -270,6 +270,51 @@ eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t p, const void* 
   return forward_spectral_io(p, Xhat, N, W_hat, bias, act, Y, 2, stream);
 }
 
+// Both layers must be p4 FP16 plans with tensor-core tiles whose widths chain.
+static eqlinear_status_t chain_check(eqlinear_plan_t a, eqlinear_plan_t b, int64_t N) {
+  if (!a || !b || N < 0) return EQL_ERR_INVALID_ARG;
+  if (a->D != b->C || a->device != b->device) return EQL_ERR_INVALID_ARG;
+  const bool ok = a->T == 4 && b->T == 4 && a->dtype == EQL_F16 && b->dtype == EQL_F16 &&
+                  a->kernel != EQL_KERNEL_SIMT && b->kernel != EQL_KERNEL_SIMT &&
+                  has_tiles(a) && has_tiles(b);
+  if (!ok) return EQL_ERR_UNSUPPORTED;
+  if (N > 0 && (!eql::fwd_tc_supported(4, eql::DType::F16, N, a->C, a->D) ||
+                !eql::fwd_tc_supported(4, eql::DType::F16, N, b->C, b->D)))
+    return EQL_ERR_UNSUPPORTED;
+  return EQL_OK;
+}
+
+size_t eqlinear_chain_workspace_bytes(eqlinear_plan_t first, eqlinear_plan_t second, int64_t N) {
+  if (chain_check(first, second, N) != EQL_OK) return 0;
+  return std::max<size_t>(eql::chain_tc_sync_bytes(N), 16);
+}
+
+eqlinear_status_t eqlinear_forward_chain(eqlinear_plan_t first, eqlinear_plan_t second,
+                                         const void* X, int64_t N, const void* W1_hat,
+                                         const void* bias1, eqlinear_act_t act1,
+                                         const void* W2_hat, const void* bias2,
+                                         int spectral_intermediate, void* H, void* Y,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+  eqlinear_status_t s = chain_check(first, second, N);
+  if (s != EQL_OK) return s;
+  if (act1 != EQL_ACT_NONE && act1 != EQL_ACT_GELU) return EQL_ERR_INVALID_ARG;
+  if (spectral_intermediate != 0 && spectral_intermediate != 1) return EQL_ERR_INVALID_ARG;
+  if (N == 0) return EQL_OK;
+  if (!X || !W1_hat || !W2_hat || !H || !Y) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W1_hat) || !aligned16(W2_hat) || !aligned16(H) ||
+      !aligned16(Y) || (bias1 && !aligned16(bias1)) || (bias2 && !aligned16(bias2)) ||
+      (workspace && !aligned16(workspace)))
+    return EQL_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < eqlinear_chain_workspace_bytes(first, second, N))
+    return EQL_ERR_WORKSPACE;
+  s = check_plan_device(first);
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_chain_tc(
+      X, N, first->C, first->D, second->D, fwd_tiles(first, W1_hat), bias1,
+      fwd_tiles(second, W2_hat), bias2, H, Y, static_cast<int*>(workspace), first->status,
+      first->num_sms, (int)act1, spectral_intermediate, (cudaStream_t)stream));
+}
+
 eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int64_t N,
                                           const void* W_hat, void* dX, void* stream) {
   if (!p || N < 0) return EQL_ERR_INVALID_ARG;

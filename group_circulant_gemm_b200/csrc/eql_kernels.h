@@ -71,6 +71,16 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
                             void* workspace, DType out_dt, void* dW, void* dbias, int* status,
                             int num_sms, const Twiddles& tw, cudaStream_t st);
 
+// Two chained T = 4 FP16 layers (C0 -> C1 -> C2) in one persistent launch with a
+// dynamic tile queue: H = act1(L1(X)) (spatial [N][C1*4], or spectral planes
+// [4][N][C1] when `spectral`), Y = L2(H).  `sync` holds chain_tc_sync_bytes(N)
+// bytes of counters that must be zero at launch; the kernel leaves them zero.
+size_t chain_tc_sync_bytes(int64_t N);
+cudaError_t launch_chain_tc(const void* X, int64_t N, int C0, int C1, int C2,
+                            const void* W1tiles, const void* b1, const void* W2tiles,
+                            const void* b2, void* H, void* Y, int* sync, int* status, int num_sms,
+                            int act1, int spectral, cudaStream_t st);
+
 // dst[i] = src[i] rounded to nearest-even in dt (a copy for F32), i < n.
 cudaError_t launch_cast_from_f32(DType dt, const float* src, void* dst, int64_t n,
                                  cudaStream_t st);

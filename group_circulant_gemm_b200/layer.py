@@ -172,3 +172,32 @@ class EqLinearPlan:
 
     def status(self) -> int:
         return _n.eqlinear_get_status(self.handle)
+
+
+def forward_chain(first: EqLinearPlan, second: EqLinearPlan, X, W1_hat, bias1, W2_hat, bias2,
+                  act: str = "none", spectral: bool = False, H=None, Y=None, workspace=None):
+    """Two chained layers in one launch: H = act(first(X)), Y = second(H).
+
+    Returns (H, Y); H is [N, D1*T], or the spectral planes [4, N, D1] when
+    ``spectral``.  Bitwise equal to the two separate calls.  A ``workspace``
+    passed in must be zero-filled before its first use (each call leaves it
+    zero).
+    """
+    N = X.shape[0]
+    first._check(X, (N, first.C * first.T), "X")
+    if second.C != first.D:
+        raise ValueError("the second layer's input width must be the first layer's output width")
+    shape_h = (4, N, first.D) if spectral else (N, first.D * first.T)
+    if H is None:
+        H = torch.empty(shape_h, dtype=first.dtype, device=X.device)
+    if Y is None:
+        Y = torch.empty((N, second.D * second.T), dtype=second.dtype, device=X.device)
+    nb = _n.eqlinear_chain_workspace_bytes(first.handle, second.handle, N)
+    if workspace is None:
+        # counters that must start at zero; each call leaves them zero again
+        workspace = torch.zeros(max(nb, 16), dtype=torch.uint8, device=X.device)
+    _n.eqlinear_forward_chain(first.handle, second.handle, X, N, W1_hat, bias1, _n.ACT[act],
+                              W2_hat, bias2, 1 if spectral else 0, H, Y, workspace,
+                              workspace.numel() * workspace.element_size())
+    return H, Y
+

@@ -30,6 +30,7 @@ EXPORTED = (
     "eqlinear_backward_weight_workspace_bytes", "eqlinear_backward_weight",
     "eqlinear_get_status", "eqlinear_backward_weight_noalloc",
     "eqlinear_backward_weight_f32", "eqlinear_cast_from_f32",
+    "eqlinear_chain_workspace_bytes", "eqlinear_forward_chain",
 )
 
 
@@ -68,6 +69,9 @@ def _load() -> ctypes.CDLL:
         "eqlinear_backward_weight_noalloc": ([vp, vp, vp, i64, vp, vp, vp], i32),
         "eqlinear_backward_weight_f32": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
         "eqlinear_cast_from_f32": ([vp, vp, i64, vp, vp], i32),
+        "eqlinear_chain_workspace_bytes": ([vp, vp, i64], sz),
+        "eqlinear_forward_chain": ([vp, vp, vp, i64, vp, vp, i32, vp, vp, i32, vp, vp, vp, sz,
+                                    vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -198,6 +202,20 @@ def eqlinear_backward_weight_f32(plan: int, X, dY, N: int, dW, dbias, workspace,
 def eqlinear_cast_from_f32(plan: int, src, count: int, dst, stream=None) -> None:
     _check(_lib.eqlinear_cast_from_f32(plan, _ptr(src), count, _ptr(dst), _stream(stream)),
            "eqlinear_cast_from_f32")
+
+
+def eqlinear_chain_workspace_bytes(first: int, second: int, N: int) -> int:
+    return _lib.eqlinear_chain_workspace_bytes(first, second, N)
+
+
+def eqlinear_forward_chain(first: int, second: int, X, N: int, W1_hat, bias1, act1: int, W2_hat,
+                           bias2, spectral_intermediate: int, H, Y, workspace,
+                           workspace_bytes: int, stream=None) -> None:
+    _check(_lib.eqlinear_forward_chain(first, second, _ptr(X), N, _ptr(W1_hat), _ptr(bias1),
+                                       act1, _ptr(W2_hat), _ptr(bias2), spectral_intermediate,
+                                       _ptr(H), _ptr(Y), _ptr(workspace), workspace_bytes,
+                                       _stream(stream)),
+           "eqlinear_forward_chain")
 
 
 def eqlinear_backward_weight_noalloc(plan: int, X, dY, N: int, dW, dbias, stream=None) -> None:

@@ -199,6 +199,45 @@ EQL_API eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t plan, c
                                                          void* Y, void* stream);
 
 /*
+ * Two chained layers in one launch (the MLP pair of a Flash EQ-ViT block):
+ *   H = act1(layer first (X))     H: [N][D1*T], or with spectral_intermediate = 1
+ *                                    the planes [4][N][D1] of
+ *                                    eqlinear_forward_to_spectral
+ *   Y = layer second (H)          Y: [N][D2*T], no activation
+ * first: C0 -> D1 channels, second: D1 -> D2 (second's C must equal first's D).
+ * The results, H included, are bitwise those of the two separate calls
+ * (eqlinear_forward_act then eqlinear_forward, or eqlinear_forward_to_spectral
+ * then eqlinear_forward_from_spectral): every tile runs the same arithmetic.
+ * What changes is the schedule: both layers' tiles form one queue that the
+ * GPU's CTAs take from as they become free, and a second-layer tile starts as
+ * soon as the first-layer tiles of its 128 rows are stored, so neither layer's
+ * last partial wave leaves SMs idle.
+ *
+ * Both plans: T = 4, FP16, C and D multiples of 16, not forced to the CUDA
+ * cores, on the same device; otherwise EQL_ERR_UNSUPPORTED (EQL_ERR_INVALID_ARG
+ * for widths that do not chain).  W1_hat, W2_hat: the plans' prepared weights;
+ * bias1, bias2: [D1], [D2] or NULL; act1: EQL_ACT_NONE or EQL_ACT_GELU.  All
+ * pointers 16-byte aligned; H must not overlap X or Y.  workspace: at least
+ * eqlinear_chain_workspace_bytes(first, second, N) bytes of device memory
+ * (int32 counters: the task queue and one per 128 rows), owned by the caller,
+ * ZERO-FILLED before its first use (e.g. cudaMemset) and not shared by calls
+ * that may run at the same time.  Every call that completes leaves the counters
+ * zero again, so the same workspace serves the next call (of any N up to its
+ * size) with no clearing.  After a call that reports EQL_ERR_TIMEOUT through
+ * eqlinear_get_status(first, ...), zero the workspace again before reusing it.
+ * Asynchronous on `stream`.  N = 0 does nothing.
+ */
+EQL_API size_t eqlinear_chain_workspace_bytes(eqlinear_plan_t first, eqlinear_plan_t second,
+                                              int64_t N);
+EQL_API eqlinear_status_t eqlinear_forward_chain(eqlinear_plan_t first, eqlinear_plan_t second,
+                                                 const void* X, int64_t N, const void* W1_hat,
+                                                 const void* bias1, eqlinear_act_t act1,
+                                                 const void* W2_hat, const void* bias2,
+                                                 int spectral_intermediate, void* H, void* Y,
+                                                 void* workspace, size_t workspace_bytes,
+                                                 void* stream);
+
+/*
  * Gradient with respect to the input ("Implementation": backward pass):
  *   dX[n, c*T+t] = sum_{d,s} dY[n, d*T+s] * W[d][c][(t-s) mod T]
  * which is the same group-circulant product with the transposed weights and the
