@@ -104,7 +104,11 @@ KERNEL_SOURCES = {
     "forward_chain": ("eql_tc_chain.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
     "backward_weight": ("eql_tc_wgrad.cu", "eql_tc_common.cuh"),
 }
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("forward", "5facc1d5cf0b65aa"): {"p4_vitb_mlp_2calls_f16": 58.89e6, "c8_1024_f16": 34.06e6,
+                                      "p4_vith_fc1_fwd_bwd_f16": 69.86e6},
+    ("forward_chain", "79e08cb6e9db3b65"): {"p4_vitb_mlp_f16": 81.76e6},
+}
 
 def kernel_traffic(family: str, workload: str):
     import hashlib
