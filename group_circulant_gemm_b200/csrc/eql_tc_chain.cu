@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kL2Planes = SPEC != 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < X_ST; ++s) {
+    for (int s = 0; s < S::X_ST; ++s) {
       mbar_init(&bars->x_full[s], 1);
       mbar_init(&bars->x_read[s], kXfWarps);
       mbar_init(&bars->x_ready[s], kXfWarps);
@@ -192,8 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------- X producer and task fetcher -------
     if (lane == 0) {
-      int issued_phase[X_ST];
-      for (int s = 0; s < X_ST; ++s) issued_phase[s] = -1;
+      int issued_phase[S::X_ST];
+      for (int s = 0; s < S::X_ST; ++s) issued_phase[s] = -1;
       uint32_t it = 0, n = 0;
       bool ok = true;
       while (ok) {
@@ -212,8 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             !(ok = wait_row(&sync[2 + t.r], ci.flag_target, abort_flag, status)))
           break;
         for (int ks = 0; ks < ks_n; ++ks, ++it) {
-          const int sx = it % X_ST;
-          const uint32_t ph = (it / X_ST) & 1;
+          const int sx = it % S::X_ST;
+          const uint32_t ph = (it / S::X_ST) & 1;
           if (!(ok = wait_bounded(&bars->x_empty[sx], ph ^ 1, abort_flag, status))) break;
           mbar_expect_tx(&bars->x_full[sx], X_STAGE_BYTES);
           const uint32_t dst = sbase + S::OFF_X + sx * X_STAGE_BYTES;
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) {
-        for (int s = 0; s < X_ST; ++s)
+        for (int s = 0; s < S::X_ST; ++s)
           if (issued_phase[s] >= 0) drain_wait(&bars->x_full[s], (uint32_t)issued_phase[s]);
       }
     }
@@ -277,9 +277,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait_bounded(&bars->acc_empty, (tcount & 1) ^ 1, abort_flag, status))) break;
         tc_fence_after();
         for (int ks = 0; ks < ks_n; ++ks, ++it) {
-          const int sx = it % X_ST, sw = it % S::W_ST;
+          const int sx = it % S::X_ST, sw = it % S::W_ST;
           uint64_t* xbar = planes_in ? &bars->x_full[sx] : &bars->x_ready[sx];
-          if (!(ok = wait_bounded(xbar, (it / X_ST) & 1, abort_flag, status))) break;
+          if (!(ok = wait_bounded(xbar, (it / S::X_ST) & 1, abort_flag, status))) break;
           if (!(ok = wait_bounded(&bars->w_full[sw], (it / S::W_ST) & 1, abort_flag, status)))
             break;
           tc_fence_after();
@@ -374,14 +374,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       for (int ks = 0; ks < ks_n; ++ks, ++it) {
-        const int sx = it % X_ST;
-        if (!(ok = warp_wait(&bars->x_full[sx], (it / X_ST) & 1, abort_flag, status))) break;
+        const int sx = it % S::X_ST;
+        if (!(ok = warp_wait(&bars->x_full[sx], (it / S::X_ST) & 1, abort_flag, status))) break;
         uint8_t* slot = smem + S::OFF_X + sx * X_STAGE_BYTES;
         uint4 v[8];
         xf_read<4>(slot, xt, v);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->x_read[sx]);
-        if (!(ok = warp_wait(&bars->x_read[sx], (it / X_ST) & 1, abort_flag, status))) break;
+        if (!(ok = warp_wait(&bars->x_read[sx], (it / S::X_ST) & 1, abort_flag, status))) break;
         xf_write<4>(slot, xt, v);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();

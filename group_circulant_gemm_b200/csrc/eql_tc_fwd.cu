@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < X_ST; ++s) {
+    for (int s = 0; s < S::X_ST; ++s) {
       mbar_init(&bars->x_full[s], 1);          // raw tile landed (TMA bytes)
       mbar_init(&bars->x_read[s], kXfWarps);   // every transform warp holds its raw pieces
       mbar_init(&bars->x_ready[s], kXfWarps);  // operand planes written (transform warps)
@@ -107,10 +107,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------- producers: warp 0 raw X (TMA, 3-D box), warp 2 weight tiles (bulk copy) -------
     if (lane == 0) {
       const bool is_raw = (warp == 0);
-      const int depth = is_raw ? X_ST : S::W_ST;
+      const int depth = is_raw ? S::X_ST : S::W_ST;
       uint64_t* full = is_raw ? bars->x_full : bars->w_full;
       uint64_t* empty = is_raw ? bars->x_empty : bars->w_empty;
-      int issued_phase[X_ST > S::W_ST ? X_ST : S::W_ST];  // last phase issued per slot
+      int issued_phase[S::X_ST > S::W_ST ? S::X_ST : S::W_ST];  // last phase issued per slot
       for (int s = 0; s < depth; ++s) issued_phase[s] = -1;
       uint32_t it = 0;
       bool ok = true;
@@ -163,9 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait_bounded(&bars->acc_empty, (tcount & 1) ^ 1, abort_flag, status))) break;
         tc_fence_after();
         for (int ks = 0; ks < ti.k_stages; ++ks, ++it) {
-          const int sx = it % X_ST, sw = it % S::W_ST;
+          const int sx = it % S::X_ST, sw = it % S::W_ST;
           uint64_t* xbar = (IO == kIoSpectralIn) ? &bars->x_full[sx] : &bars->x_ready[sx];
-          if (!(ok = wait_bounded(xbar, (it / X_ST) & 1, abort_flag, status))) break;
+          if (!(ok = wait_bounded(xbar, (it / S::X_ST) & 1, abort_flag, status))) break;
           if (!(ok = wait_bounded(&bars->w_full[sw], (it / S::W_ST) & 1, abort_flag, status)))
             break;
           tc_fence_after();
@@ -239,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < ti.num_tiles; tile += gridDim.x) {
       for (int ks = 0; ks < ti.k_stages; ++ks, ++it) {
-        const int sx = it % X_ST;
-        if (!(ok = warp_wait(&bars->x_full[sx], (it / X_ST) & 1, abort_flag, status))) break;
+        const int sx = it % S::X_ST;
+        if (!(ok = warp_wait(&bars->x_full[sx], (it / S::X_ST) & 1, abort_flag, status))) break;
         uint8_t* slot = smem + S::OFF_X + sx * X_STAGE_BYTES;
         uint4 v[8];
         xf_read<T>(slot, xt, v);
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (an mbarrier rather than a named barrier, so the wait stays bounded)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->x_read[sx]);
-        if (!(ok = warp_wait(&bars->x_read[sx], (it / X_ST) & 1, abort_flag, status))) break;
+        if (!(ok = warp_wait(&bars->x_read[sx], (it / S::X_ST) & 1, abort_flag, status))) break;
         xf_write<T>(slot, xt, v);
         // make the generic-proxy stores visible to the tensor core (async proxy)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
