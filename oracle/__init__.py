@@ -20,6 +20,10 @@ What each function computes, and the passage of the "Flash EQ-Linear" summary
   ("Specialisation for p4", bullet 3: 6 real GEMMs, 16/6 fewer MACs).
 * :func:`p4_transform_matrices` -- the real 4x4 DFT / inverse-DFT pair for the
   p4 group ("Specialisation for p4", bullets 1-2: coefficients 0, +-1, +-1/2).
+* :func:`conv_forward` -- the group-circulant convolution ("Limitations and
+  future work" names equivariant convolution as the next operator; no formula
+  is given): the EQ-Linear's channel mixing at every tap of a KH x KW kernel,
+  stride 1, zero padding.
 
 Every function is pinned by tests/test_oracle_pins.py against values fixed by
 something other than this code (dense replicated matmul, numpy FFT, closed
@@ -78,6 +82,10 @@ def _load():
             lib.eqlo_gelu.restype = None
             lib.eqlo_p4_transform_matrices.argtypes = [dp, dp]
             lib.eqlo_p4_transform_matrices.restype = None
+            lib.eqlo_conv_forward.argtypes = [ctypes.c_int, i64, i64, i64, i64, i64,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, dp, dp, dp, dp]
+            lib.eqlo_conv_forward.restype = i64
             _lib = lib
     return _lib
 
@@ -192,6 +200,25 @@ def p4_transform_matrices():
     G = np.empty((4, 4), dtype=np.float64)
     lib.eqlo_p4_transform_matrices(_ptr(F), _ptr(G))
     return F, G
+
+
+def conv_forward(T: int, X, Wc, bias=None, pad=(0, 0), return_macs: bool = False):
+    """Y[N, Ho, Wo, D*T] in float64 from X[N, H, W, C*T], Wc[KH, KW, D, C, T],
+    bias[D] or None, zero padding pad = (ph, pw), stride 1."""
+    X, Wc = _f64(X), _f64(Wc)
+    KH, KW, D, C, TW = Wc.shape
+    if TW != T or X.ndim != 4 or X.shape[3] != C * T:
+        raise ValueError("X must be [N, H, W, C*T] and Wc [KH, KW, D, C, T]")
+    N, H, Wd = X.shape[:3]
+    ph, pw = pad
+    Ho, Wo = H + 2 * ph - KH + 1, Wd + 2 * pw - KW + 1
+    if Ho <= 0 or Wo <= 0:
+        raise ValueError("empty output")
+    b = None if bias is None else _f64(bias)
+    Y = np.empty((N, Ho, Wo, D * T), dtype=np.float64)
+    macs = _load().eqlo_conv_forward(T, N, H, Wd, C, D, KH, KW, ph, pw, _ptr(X), _ptr(Wc),
+                                     _ptr(b), _ptr(Y))
+    return (Y, macs) if return_macs else Y
 
 
 def threads_used() -> int:

@@ -242,3 +242,54 @@ void eqlo_p4_transform_matrices(double* F, double* G) {
     if (fabs(G[i] * 4.0 - qg) < 1e-12) G[i] = qg / 4.0;
   }
 }
+
+/*
+ * Group-circulant convolution, the plain definition (the pages name equivariant
+ * convolution as the natural next operator for the per-frequency method,
+ * "Limitations and future work"; they give no formula).  Reading: the
+ * EQ-Linear's group-circulant channel mixing at every tap of a KH x KW kernel,
+ * stride 1, zero padding (ph, pw):
+ *   Y[n][oy][ox][d*T+s] = bias[d] + sum_{i<KH, j<KW} sum_{c,t}
+ *       Wc[i][j][d][c][(t-s) mod T] * X[n][oy+i-ph][ox+j-pw][c*T+t]
+ * with X zero outside the H x Wd image.  A cyclic shift of every pixel's group
+ * axis shifts the output's group axis the same way, as for the EQ-Linear, and
+ * the operator commutes with translations away from the border.
+ * Layouts: X [N][H][Wd][C*T], Wc [KH][KW][D][C][T], bias [D] or NULL,
+ * Y [N][Ho][Wo][D*T] with Ho = H + 2 ph - KH + 1, Wo = Wd + 2 pw - KW + 1.
+ * Returns the number of real multiply-adds taken inside the image.
+ */
+int64_t eqlo_conv_forward(int T, int64_t N, int64_t H, int64_t Wd, int64_t C, int64_t D,
+                          int KH, int KW, int ph, int pw, const double* X, const double* Wc,
+                          const double* bias, double* Y) {
+  const int64_t Ho = H + 2 * ph - KH + 1, Wo = Wd + 2 * pw - KW + 1;
+  if (Ho <= 0 || Wo <= 0) return 0;
+  int64_t macs = 0;
+#pragma omp parallel for collapse(2) schedule(static) reduction(+ : macs)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t oy = 0; oy < Ho; ++oy) {
+      for (int64_t ox = 0; ox < Wo; ++ox) {
+        double* y = Y + ((n * Ho + oy) * Wo + ox) * D * T;
+        for (int64_t d = 0; d < D; ++d) {
+          for (int s = 0; s < T; ++s) {
+            double acc = 0.0;
+            for (int i = 0; i < KH; ++i) {
+              const int64_t iy = oy + i - ph;
+              if (iy < 0 || iy >= H) continue;
+              for (int j = 0; j < KW; ++j) {
+                const int64_t ix = ox + j - pw;
+                if (ix < 0 || ix >= Wd) continue;
+                const double* x = X + ((n * H + iy) * Wd + ix) * C * T;
+                const double* w = Wc + (((int64_t)i * KW + j) * D + d) * C * T;
+                for (int64_t c = 0; c < C; ++c)
+                  for (int t = 0; t < T; ++t) acc += w[c * T + wrap(t - s, T)] * x[c * T + t];
+                macs += C * T;
+              }
+            }
+            y[d * T + s] = acc + (bias ? bias[d] : 0.0);
+          }
+        }
+      }
+    }
+  }
+  return macs;
+}
