@@ -315,6 +315,81 @@ eqlinear_status_t eqlinear_forward_chain(eqlinear_plan_t first, eqlinear_plan_t 
       first->num_sms, (int)act1, spectral_intermediate, (cudaStream_t)stream));
 }
 
+// ---- group-circulant convolution ----------------------------------------------
+
+static bool conv_plan_ok(eqlinear_plan_t p) {
+  return p && p->T == 4 && p->dtype == EQL_F16 && p->kernel != EQL_KERNEL_SIMT && has_tiles(p);
+}
+static size_t conv_tap_tiles(eqlinear_plan_t p) { return eql::tc_tile_bytes(4, p->C, p->D); }
+static size_t conv_tap_planes(eqlinear_plan_t p) {
+  return (size_t)eql::spec_planes(4) * plane_elems(p) * elem_size(p->dtype);
+}
+
+size_t eqlinear_conv_prepared_weight_bytes(eqlinear_plan_t p, int KH, int KW) {
+  if (!conv_plan_ok(p) || KH < 1 || KW < 1 || KH > 15 || KW > 15) return 0;
+  // per tap: operand tiles (read by the kernel, all taps first) and the forward
+  // and adjoint planes they are made from
+  return (size_t)KH * KW * (conv_tap_tiles(p) + 2 * conv_tap_planes(p));
+}
+
+eqlinear_status_t eqlinear_conv_prepare_weights(eqlinear_plan_t p, int KH, int KW,
+                                                const void* Wc, void* Wc_hat, void* stream) {
+  if (!p || !Wc || !Wc_hat || KH < 1 || KW < 1 || KH > 15 || KW > 15)
+    return EQL_ERR_INVALID_ARG;
+  if (!conv_plan_ok(p)) return EQL_ERR_UNSUPPORTED;
+  if (!aligned16(Wc) || !aligned16(Wc_hat)) return EQL_ERR_ALIGNMENT;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int taps = KH * KW;
+  char* tiles = static_cast<char*>(Wc_hat);
+  char* planes = tiles + (size_t)taps * conv_tap_tiles(p);
+  const size_t w_tap = (size_t)p->D * p->C * 4 * elem_size(p->dtype);
+  for (int tap = 0; tap < taps; ++tap) {
+    char* fwd = planes + (size_t)tap * 2 * conv_tap_planes(p);
+    char* adj = fwd + conv_tap_planes(p);
+    s = from_cuda(eql::launch_prepare(4, to_dt(p->dtype), static_cast<const char*>(Wc) + tap * w_tap,
+                                      p->C, p->D, fwd, adj, p->tw, st));
+    if (s != EQL_OK) return s;
+    s = from_cuda(eql::launch_tile_weights(4, fwd, p->C, p->D,
+                                           tiles + (size_t)tap * conv_tap_tiles(p), st));
+    if (s != EQL_OK) return s;
+  }
+  return EQL_OK;
+}
+
+size_t eqlinear_conv_workspace_bytes(eqlinear_plan_t p, int64_t N, int H, int W) {
+  if (!conv_plan_ok(p) || N < 0 || H < 0 || W < 0) return 0;
+  return std::max<size_t>(eql::conv_tc_planes_bytes(N, H, W, p->C), 16);
+}
+
+eqlinear_status_t eqlinear_conv_forward(eqlinear_plan_t p, const void* X, int64_t N, int H, int W,
+                                        int KH, int KW, int pad_h, int pad_w,
+                                        const void* Wc_hat, const void* bias, eqlinear_act_t act,
+                                        void* Y, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  if (!p || N < 0 || H < 1 || W < 1 || KH < 1 || KW < 1 || pad_h < 0 || pad_w < 0)
+    return EQL_ERR_INVALID_ARG;
+  if (act != EQL_ACT_NONE && act != EQL_ACT_GELU) return EQL_ERR_INVALID_ARG;
+  if (!conv_plan_ok(p)) return EQL_ERR_UNSUPPORTED;
+  if ((int64_t)H + 2 * pad_h - KH + 1 < 1 || (int64_t)W + 2 * pad_w - KW + 1 < 1)
+    return EQL_ERR_INVALID_ARG;
+  if (N == 0) return EQL_OK;
+  if (!eql::conv_tc_supported(4, to_dt(p->dtype), N, H, W, p->C, p->D, KH, KW, pad_h, pad_w))
+    return EQL_ERR_UNSUPPORTED;
+  if (!X || !Wc_hat || !Y) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Wc_hat) || !aligned16(Y) || (bias && !aligned16(bias)) ||
+      (workspace && !aligned16(workspace)))
+    return EQL_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < eqlinear_conv_workspace_bytes(p, N, H, W))
+    return EQL_ERR_WORKSPACE;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_conv_tc(X, N, H, W, p->C, p->D, KH, KW, pad_h, pad_w, Wc_hat, bias,
+                                       Y, workspace, p->status, p->num_sms, (int)act,
+                                       (cudaStream_t)stream));
+}
+
 eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int64_t N,
                                           const void* W_hat, void* dX, void* stream) {
   if (!p || N < 0) return EQL_ERR_INVALID_ARG;

@@ -81,6 +81,17 @@ cudaError_t launch_chain_tc(const void* X, int64_t N, int C0, int C1, int C2,
                             const void* b2, void* H, void* Y, int* sync, int* status, int num_sms,
                             int act1, int spectral, cudaStream_t st);
 
+// Group-circulant convolution (T = 4, FP16): X [N][H][W][C*4] -> Y [N][Ho][Wo][D*4],
+// KH x KW taps, stride 1, zero padding (ph, pw).  Wtiles: one forward tile block
+// (tc_tile_bytes(4, C, D)) per tap, tap-major; planes: conv_tc_planes_bytes of
+// scratch for the group DFT of X.
+bool conv_tc_supported(int T, DType dt, int64_t N, int H, int W, int C, int D, int KH, int KW,
+                       int ph, int pw);
+size_t conv_tc_planes_bytes(int64_t N, int H, int W, int C);
+cudaError_t launch_conv_tc(const void* X, int64_t N, int H, int W, int C, int D, int KH, int KW,
+                           int ph, int pw, const void* Wtiles, const void* bias, void* Y,
+                           void* planes, int* status, int num_sms, int act, cudaStream_t st);
+
 // dst[i] = src[i] rounded to nearest-even in dt (a copy for F32), i < n.
 cudaError_t launch_cast_from_f32(DType dt, const float* src, void* dst, int64_t n,
                                  cudaStream_t st);

@@ -335,13 +335,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t.layer == 0) {
         if constexpr (SPEC)
           epi_slices<4, BD, ACT1, kIoSpectralOut>(lane_addr, ch, lane, stg, bsm, dbase, Cout,
-                                                  row0, ci.N, &map_h_store);
+                                                  PlaneStore{&map_h_store, row0, ci.N});
         else
-          epi_slices<4, BD, ACT1, kIoSpatial>(lane_addr, ch, lane, stg, bsm, dbase, Cout, row0,
-                                              ci.N, &map_h_store);
+          epi_slices<4, BD, ACT1, kIoSpatial>(lane_addr, ch, lane, stg, bsm, dbase, Cout,
+                                              RowStore<4>{&map_h_store, row0, ci.N});
       } else {
-        epi_slices<4, BD, 0, kIoSpatial>(lane_addr, ch, lane, stg, bsm, dbase, Cout, row0, ci.N,
-                                         &map_y);
+        epi_slices<4, BD, 0, kIoSpatial>(lane_addr, ch, lane, stg, bsm, dbase, Cout,
+                                         RowStore<4>{&map_y, row0, ci.N});
       }
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);

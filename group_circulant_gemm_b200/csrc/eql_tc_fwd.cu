@@ -226,7 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&bars->acc_full, tcount & 1, abort_flag, status)) break;
       tc_fence_after();
       const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-      epi_slices<T, BD, ACT, IO>(lane_addr, ch, lane, stg, bsm, dbase, Cout, row0, N, &map_y);
+      epi_slices<T, BD, ACT, IO>(lane_addr, ch, lane, stg, bsm, dbase, Cout,
+                                 StoreOf<T, IO>{&map_y, row0, N});
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
     }

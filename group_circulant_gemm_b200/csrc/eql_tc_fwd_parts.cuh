@@ -4,6 +4,8 @@
 // staged X tile into operand planes, and the inverse-DFT epilogue.
 #pragma once
 
+#include <type_traits>
+
 #include "eql_tc_common.cuh"
 
 namespace eql {
@@ -314,11 +316,12 @@ __device__ __forceinline__ void epi_half_spec(uint32_t lane_addr, int c0, const 
 // Epilogue of one tile for one epilogue warp: its TMEM lane quarter (lane_addr),
 // out-channel half ch, in slices of 64/T out-channels (16 channels for spectral
 // output); each slice is staged in the warp's 4 KB buffer and written by one TMA
-// store.  bsm holds the half's biases; dbase is the half's first out-channel.
-template <int T, int BD, int ACT, int IO>
+// store, store(staging address, first out-channel of the slice), issued by lane 0.
+// bsm holds the half's biases; dbase is the half's first out-channel.
+template <int T, int BD, int ACT, int IO, class Store>
 __device__ __forceinline__ void epi_slices(uint32_t lane_addr, int ch, int lane, uint8_t* stg,
-                                           const __half* bsm, int dbase, int Cout, int64_t row0,
-                                           int64_t N, const CUtensorMap* map_y) {
+                                           const __half* bsm, int dbase, int Cout,
+                                           const Store& store) {
   constexpr int kSliceCh = 64 / T;
   constexpr int kSlices = (BD / 2) / kSliceCh;
   const uint32_t stg_s = smem_u32(stg);
@@ -346,7 +349,7 @@ __device__ __forceinline__ void epi_slices(uint32_t lane_addr, int ch, int lane,
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) {
-        if (row0 < N) tma_store_3d(map_y, stg_s, d0, (int)row0, 0);
+        store(stg_s, d0);
         bulk_commit();
       }
       continue;
@@ -367,11 +370,32 @@ __device__ __forceinline__ void epi_slices(uint32_t lane_addr, int ch, int lane,
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
     if (lane == 0) {
-      if (row0 < N) tma_store_3d(map_y, stg_s, 0, d0 * T / 64, (int)row0);
+      store(stg_s, d0);
       bulk_commit();
     }
   }
 }
+
+// Stores of a row-tile epilogue: 32 rows starting at row0 of an [N][Cout*T]
+// activation (3-D map: 64 halves, 128-byte chunk, row), or of spectral planes
+// [4][N][Cout] (3-D map: channel, row, plane).
+template <int T>
+struct RowStore {
+  const CUtensorMap* map;
+  int64_t row0, N;
+  __device__ __forceinline__ void operator()(uint32_t src, int d0) const {
+    if (row0 < N) tma_store_3d(map, src, 0, d0 * T / 64, (int)row0);
+  }
+};
+struct PlaneStore {
+  const CUtensorMap* map;
+  int64_t row0, N;
+  __device__ __forceinline__ void operator()(uint32_t src, int d0) const {
+    if (row0 < N) tma_store_3d(map, src, d0, (int)row0, 0);
+  }
+};
+template <int T, int IO>
+using StoreOf = typename std::conditional<IO == kIoSpectralOut, PlaneStore, RowStore<T>>::type;
 
 }  // namespace ftc
 }  // namespace eql

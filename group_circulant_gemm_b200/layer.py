@@ -126,6 +126,38 @@ class EqLinearPlan:
                                     workspace.numel() * workspace.element_size())
         return dW, dbias
 
+    # --- group-circulant convolution (KH x KW taps, stride 1, zero padding)
+
+    def conv_prepare_weights(self, Wc: torch.Tensor, out: torch.Tensor | None = None):
+        """Wc [KH, KW, D, C, T] -> prepared convolution weights."""
+        KH, KW = int(Wc.shape[0]), int(Wc.shape[1])
+        self._check(Wc, (KH, KW, self.D, self.C, self.T), "Wc")
+        nbytes = _n.eqlinear_conv_prepared_weight_bytes(self.handle, KH, KW)
+        if nbytes == 0:
+            raise ValueError("this plan has no convolution kernel (T = 4, FP16, C and D "
+                             "multiples of 16)")
+        if out is None:
+            out = torch.empty(nbytes // Wc.element_size(), dtype=self.dtype, device=Wc.device)
+        _n.eqlinear_conv_prepare_weights(self.handle, KH, KW, Wc, out)
+        return out
+
+    def conv_forward(self, X, Wc_hat, KH: int, KW: int, bias=None, pad=(0, 0), act="none",
+                     out=None, workspace=None) -> torch.Tensor:
+        """X [N, H, W, C*T] -> Y [N, Ho, Wo, D*T]."""
+        N, H, W = (int(v) for v in X.shape[:3])
+        self._check(X, (N, H, W, self.C * self.T), "X")
+        ph, pw = pad
+        Ho, Wo = H + 2 * ph - KH + 1, W + 2 * pw - KW + 1
+        if out is None:
+            out = torch.empty((N, Ho, Wo, self.D * self.T), dtype=self.dtype, device=X.device)
+        nb = _n.eqlinear_conv_workspace_bytes(self.handle, N, H, W)
+        if workspace is None:
+            workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=X.device)
+        _n.eqlinear_conv_forward(self.handle, X, N, H, W, KH, KW, ph, pw, Wc_hat, bias,
+                                 _n.ACT[act], out, workspace,
+                                 workspace.numel() * workspace.element_size())
+        return out
+
     # --- data-parallel weight gradient: FP32 per-rank sums, one reduction, one cast
 
     def grad_offset(self) -> int:

@@ -31,6 +31,8 @@ EXPORTED = (
     "eqlinear_get_status", "eqlinear_backward_weight_noalloc",
     "eqlinear_backward_weight_f32", "eqlinear_cast_from_f32",
     "eqlinear_chain_workspace_bytes", "eqlinear_forward_chain",
+    "eqlinear_conv_prepared_weight_bytes", "eqlinear_conv_prepare_weights",
+    "eqlinear_conv_workspace_bytes", "eqlinear_conv_forward",
 )
 
 
@@ -70,6 +72,11 @@ def _load() -> ctypes.CDLL:
         "eqlinear_backward_weight_f32": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
         "eqlinear_cast_from_f32": ([vp, vp, i64, vp, vp], i32),
         "eqlinear_chain_workspace_bytes": ([vp, vp, i64], sz),
+        "eqlinear_conv_prepared_weight_bytes": ([vp, i32, i32], sz),
+        "eqlinear_conv_prepare_weights": ([vp, i32, i32, vp, vp, vp], i32),
+        "eqlinear_conv_workspace_bytes": ([vp, i64, i32, i32], sz),
+        "eqlinear_conv_forward": ([vp, vp, i64, i32, i32, i32, i32, i32, i32, vp, vp, i32, vp,
+                                   vp, sz, vp], i32),
         "eqlinear_forward_chain": ([vp, vp, vp, i64, vp, vp, i32, vp, vp, i32, vp, vp, vp, sz,
                                     vp], i32),
     }
@@ -216,6 +223,29 @@ def eqlinear_forward_chain(first: int, second: int, X, N: int, W1_hat, bias1, ac
                                        _ptr(H), _ptr(Y), _ptr(workspace), workspace_bytes,
                                        _stream(stream)),
            "eqlinear_forward_chain")
+
+
+def eqlinear_conv_prepared_weight_bytes(plan: int, KH: int, KW: int) -> int:
+    return _lib.eqlinear_conv_prepared_weight_bytes(plan, KH, KW)
+
+
+def eqlinear_conv_prepare_weights(plan: int, KH: int, KW: int, Wc, Wc_hat, stream=None) -> None:
+    _check(_lib.eqlinear_conv_prepare_weights(plan, KH, KW, _ptr(Wc), _ptr(Wc_hat),
+                                              _stream(stream)),
+           "eqlinear_conv_prepare_weights")
+
+
+def eqlinear_conv_workspace_bytes(plan: int, N: int, H: int, W: int) -> int:
+    return _lib.eqlinear_conv_workspace_bytes(plan, N, H, W)
+
+
+def eqlinear_conv_forward(plan: int, X, N: int, H: int, W: int, KH: int, KW: int, pad_h: int,
+                          pad_w: int, Wc_hat, bias, act: int, Y, workspace, workspace_bytes: int,
+                          stream=None) -> None:
+    _check(_lib.eqlinear_conv_forward(plan, _ptr(X), N, H, W, KH, KW, pad_h, pad_w,
+                                      _ptr(Wc_hat), _ptr(bias), act, _ptr(Y), _ptr(workspace),
+                                      workspace_bytes, _stream(stream)),
+           "eqlinear_conv_forward")
 
 
 def eqlinear_backward_weight_noalloc(plan: int, X, dY, N: int, dW, dbias, stream=None) -> None:

@@ -238,6 +238,43 @@ EQL_API eqlinear_status_t eqlinear_forward_chain(eqlinear_plan_t first, eqlinear
                                                  void* stream);
 
 /*
+ * Group-circulant convolution.  The pages name equivariant convolution as the
+ * natural next operator for the per-frequency method ("Limitations and future
+ * work") and give no formula; this library's reading is the layer's
+ * group-circulant channel mixing at every tap of a KH x KW kernel, stride 1,
+ * zero padding:
+ *   Y[n][oy][ox][d*T+s] = act(bias[d] + sum_{i<KH, j<KW} sum_{c,t}
+ *       Wc[i][j][d][c][(t-s) mod T] * X[n][oy+i-pad_h][ox+j-pad_w][c*T+t])
+ * with X zero outside the H x W image; Ho = H + 2 pad_h - KH + 1,
+ * Wo = W + 2 pad_w - KW + 1.  Like the layer it commutes with the cyclic shift
+ * of every pixel's group axis, and with translations away from the border.
+ *
+ * Plans: T = 4, FP16, C and D multiples of 16, not forced to the CUDA cores
+ * (otherwise EQL_ERR_UNSUPPORTED).  KH, KW in 1..15, 0 <= pad < kernel size.
+ *   eqlinear_conv_prepared_weight_bytes(plan, KH, KW): size of Wc_hat.
+ *   eqlinear_conv_prepare_weights: Wc [KH][KW][D][C][T] (tap-major; each tap a
+ *     contiguous [D][C][T] block) -> Wc_hat, once per weight update.
+ *   eqlinear_conv_workspace_bytes(plan, N, H, W): scratch of eqlinear_conv_forward
+ *     (the group DFT of X as FP16 planes, 4 * N * H * W * C * 2 bytes).
+ *   eqlinear_conv_forward: X [N][H][W][C*T] (feature index c*T+t, pixels
+ *     row-major), Y [N][Ho][Wo][D*T], bias [D] or NULL, act as in
+ *     eqlinear_forward_act.  All pointers 16-byte aligned; the caller owns every
+ *     buffer.  Asynchronous on `stream`.  N = 0 does nothing.
+ * A 1 x 1 kernel with no padding computes exactly eqlinear_forward on the N*H*W
+ * pixels.
+ */
+EQL_API size_t eqlinear_conv_prepared_weight_bytes(eqlinear_plan_t plan, int KH, int KW);
+EQL_API eqlinear_status_t eqlinear_conv_prepare_weights(eqlinear_plan_t plan, int KH, int KW,
+                                                        const void* Wc, void* Wc_hat,
+                                                        void* stream);
+EQL_API size_t eqlinear_conv_workspace_bytes(eqlinear_plan_t plan, int64_t N, int H, int W);
+EQL_API eqlinear_status_t eqlinear_conv_forward(eqlinear_plan_t plan, const void* X, int64_t N,
+                                                int H, int W, int KH, int KW, int pad_h,
+                                                int pad_w, const void* Wc_hat, const void* bias,
+                                                eqlinear_act_t act, void* Y, void* workspace,
+                                                size_t workspace_bytes, void* stream);
+
+/*
  * Gradient with respect to the input ("Implementation": backward pass):
  *   dX[n, c*T+t] = sum_{d,s} dY[n, d*T+s] * W[d][c][(t-s) mod T]
  * which is the same group-circulant product with the transposed weights and the
