@@ -9,8 +9,10 @@ resident in HBM; `e2e` = the same through the C ABI with the step's input copied
 from pinned host memory and the result read back, inside the timed region.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--workload p4_vitb_mlp_f16|p4_vitb_proj_f32|p4_vith_fc1_f16|c8_1024_f16|
-                   p4_vith_fc1_fwd_bwd_f16|p4_vitb_mlp_block_f16|p4_vitb_mlp_spectral_f16]
+       [--workload p4_vitb_mlp_f16|p4_vitb_mlp_2calls_f16|p4_vitb_proj_f32|p4_vith_fc1_f16|
+                   c8_1024_f16|p4_vith_fc1_fwd_bwd_f16|p4_vitb_mlp_block_f16|
+                   p4_vitb_mlp_spectral_f16|p4_conv3x3_f16] [--dp-path] [--no-dense]
+       [--no-cpu-baseline]
 Under torchrun (N > 1) every rank runs its own copy of the workload (weak
 scaling; rows are independent, so no collective is on the forward path).  The
 training workload is then data parallel: each rank's FP32 weight gradient is
@@ -32,7 +34,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from group_circulant_gemm_b200.synth import WORKLOADS, make_inputs  # noqa: E402
+from group_circulant_gemm_b200.synth import (CONV_WORKLOADS, WORKLOADS,  # noqa: E402
+                                             make_conv_inputs, make_inputs)
 
 METRIC = "EQ-Linear fwd tokens/s + TFLOP/s (T=4, fp16/fp32) and % of tensor roofline"
 L2_BYTES = 126 * 1024 * 1024
@@ -102,6 +105,7 @@ def layer_bytes(w) -> float:
 KERNEL_SOURCES = {
     "forward": ("eql_tc_fwd.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
     "forward_chain": ("eql_tc_chain.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
+    "conv": ("eql_tc_conv.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
     "backward_weight": ("eql_tc_wgrad.cu", "eql_tc_common.cuh"),
 }
 NCU_TRAFFIC = {
@@ -643,13 +647,254 @@ def run_ours(args, workload):
     return 0
 
 
+CONV_DESCR = {
+    "p4_conv3x3_f16": "p4 group-circulant convolution fp16: 64 images 56x56, C=64->D=64 per "
+                      "group element (256 -> 256 features), 3x3 taps, stride 1, zero padding 1, "
+                      "T=4",
+}
+
+
+def conv_flops(w) -> float:
+    """Algorithmic FLOPs: the layer's 12*C*D per output pixel and tap (6 real GEMMs)."""
+    return 12.0 * w.N * w.Ho * w.Wo * w.C * w.D * w.KH * w.KW
+
+
+def conv_dense_flops(w) -> float:
+    return 2.0 * w.N * w.Ho * w.Wo * (w.C * w.T) * (w.D * w.T) * w.KH * w.KW
+
+
+def conv_oracle_sample(w, images: int):
+    import oracle
+    oracle.build()
+    inp = make_conv_inputs(w, images=images)
+    t0 = time.perf_counter()
+    oracle.conv_forward(w.T, inp["X"], inp["Wc"], inp["bias"], pad=(w.ph, w.pw))
+    return time.perf_counter() - t0
+
+
+def conv_oracle_images(w, target_s: float) -> int:
+    t1 = conv_oracle_sample(w, 1)
+    return int(max(1, min(w.N, target_s / max(t1, 1e-6))))
+
+
+def run_conv_reference(args, workload):
+    import oracle
+    world, rank, _ = dist_init()
+    if rank != 0:
+        return 0
+    w = CONV_WORKLOADS[workload]
+    per_step_s = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+    images = conv_oracle_images(w, min(per_step_s, 20.0))
+    for _ in range(args.warmup):
+        conv_oracle_sample(w, images)
+    times = [conv_oracle_sample(w, images) for _ in range(args.steps)]
+    total = sum(times)
+    value = images * w.Ho * w.Wo * args.steps / total
+    sample = f"{images} of {w.N} images per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": CONV_DESCR[workload], "images_per_step": images,
+                   "global_batch": w.N, "seq_len": None, "parallelism": "none (host oracle)",
+                   "tokens": "output pixels"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads_used(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_conv(args, workload):
+    """The convolution step: one eqlinear_conv_forward (planes pre-pass + tap-loop
+    kernel) over the whole batch; tokens = output pixels."""
+    import torch
+    import torch.distributed as dist
+    import torch.nn.functional as F
+
+    world, rank, local = dist_init()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from group_circulant_gemm_b200 import EqLinearPlan
+
+    w = CONV_WORKLOADS[workload]
+    inp = make_conv_inputs(w.with_(seed=w.seed + 1000 * rank))
+    p = EqLinearPlan(w.T, w.C, w.D, torch.float16)
+    Wc = torch.from_numpy(inp["Wc"]).cuda()
+    Wh = p.conv_prepare_weights(Wc)
+    bias = torch.from_numpy(inp["bias"]).cuda()
+    x_host = inp["X"]
+    pixels = w.N * w.Ho * w.Wo
+    per_set = x_host.nbytes + pixels * w.D * w.T * 2
+    nsets = max(2, int(np.ceil(2 * L2_BYTES / per_set)))
+    xs = [torch.from_numpy(x_host).cuda() for _ in range(nsets)]
+    ys = [torch.empty((w.N, w.Ho, w.Wo, w.D * w.T), dtype=torch.float16, device="cuda")
+          for _ in range(nsets)]
+    from group_circulant_gemm_b200 import native
+    ws = torch.empty(native.eqlinear_conv_workspace_bytes(p.handle, w.N, w.H, w.W),
+                     dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i, events=None):
+        if events is not None:
+            events.append(torch.cuda.Event(enable_timing=True))
+            events[-1].record(stream)
+        p.conv_forward(xs[i % nsets], Wh, w.KH, w.KW, bias, pad=(w.ph, w.pw),
+                       out=ys[i % nsets], workspace=ws)
+        if events is not None:
+            events.append(torch.cuda.Event(enable_timing=True))
+            events[-1].record(stream)
+
+    clocks = ClockSampler(local)
+    if rank == 0:
+        clocks.start()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert p.status() == 0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark(0)
+    ev = []
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, ev)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(1)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if rank == 0 else {}
+    elapsed_ms = t0.elapsed_time(t1)
+    launch_ms = float(np.mean([ev[2 * j].elapsed_time(ev[2 * j + 1])
+                               for j in range(len(ev) // 2)]))
+
+    x_pin = torch.from_numpy(x_host).pin_memory()
+    y_pin = torch.empty(tuple(ys[0].shape), dtype=torch.float16).pin_memory()
+
+    def e2e_step():
+        xs[0].copy_(x_pin, non_blocking=True)
+        step(0)
+        y_pin.copy_(ys[0], non_blocking=True)
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    assert p.status() == 0
+    times = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms = times.tolist()
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        flops = conv_flops(w)
+        value = world * pixels * args.steps / (elapsed_ms / 1e3)
+        achieved = flops / (launch_ms / 1e3) / 1e12
+        nbytes = x_host.nbytes + pixels * w.D * w.T * 2 + inp["Wc"].nbytes
+        hbm = nbytes / (launch_ms / 1e3) / 1e9
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "traffic": kernel_traffic("conv", workload),
+                "peak_source": f"{peak_src} dense bf16 burst (fp16 runs at the same rate)",
+                "hbm_gbs": hbm, "hbm_frac": hbm / peaks["hbm_gbs"], "launch_ms": launch_ms,
+                "kernel": "eqlinear_conv_forward[planes pre-pass + tcgen05 tap loop]",
+                "step_share": 1.0}
+        comparator = None
+        if not args.no_dense:
+            # cuDNN on the replicated dense kernel K[(d,s),(c,t),i,j] = Wc[i,j,d,c,(t-s) mod T]
+            K = torch.stack([torch.roll(Wc, shifts=sh, dims=4) for sh in range(w.T)])
+            K = K.permute(3, 0, 4, 5, 1, 2).reshape(w.D * w.T, w.C * w.T, w.KH, w.KW)
+            K = K.contiguous(memory_format=torch.channels_last)
+            brep = bias.repeat_interleave(w.T)
+
+            def dense(i):
+                return F.conv2d(xs[i % nsets].permute(0, 3, 1, 2), K, brep,
+                                padding=(w.ph, w.pw))
+            for i in range(3):
+                dense(i)
+            torch.cuda.synchronize()
+            d0 = torch.cuda.Event(enable_timing=True)
+            d1 = torch.cuda.Event(enable_timing=True)
+            nd = min(args.steps, 100)
+            d0.record(stream)
+            for i in range(nd):
+                dense(i)
+            d1.record(stream)
+            torch.cuda.synchronize()
+            dms = d0.elapsed_time(d1) / nd
+            comparator = {"kind": "dense F.conv2d (cuDNN, channels-last) with the replicated "
+                                  "(D*T x C*T x KH x KW) kernel, same dtype",
+                          "value": pixels / (dms / 1e3), "unit": "tokens/s",
+                          "ms_per_step": dms,
+                          "tflops": conv_dense_flops(w) / (dms / 1e3) / 1e12}
+            comparator["ours_over_dense"] = value / world / comparator["value"]
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            images = conv_oracle_images(w, 15.0)
+            secs = conv_oracle_sample(w, images)
+            cpu = {"value": images * w.Ho * w.Wo / secs, "unit": "tokens/s",
+                   "cores": oracle.threads_used(), "kind": "oracle",
+                   "sample": f"{images} of {w.N} images, float64, {secs:.1f} s"}
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "tflops": flops * args.steps * world / (elapsed_ms / 1e3) / 1e12,
+            "tflops_dense_equiv": conv_dense_flops(w) * args.steps * world
+                                  / (elapsed_ms / 1e3) / 1e12,
+            "config": {"workload": CONV_DESCR[workload], "global_batch": w.N * world,
+                       "seq_len": None, "tokens": "output pixels",
+                       "parallelism": f"replicas x{world} (images independent)",
+                       "l2": f"{nsets} rotating input/output sets of {per_set / 2**20:.0f} MiB "
+                             "(> 2x L2)",
+                       "kernels": ["conv_forward[tcgen05]"]},
+            "op_ms": [round(launch_ms, 5)],
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "dense_comparator": comparator,
+            "e2e": {"value": world * pixels * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(x_pin.numel() * 2),
+                    "d2h_bytes_per_step": int(y_pin.numel() * 2)},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    p.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(PIPELINES), default="p4_vitb_mlp_f16")
+    ap.add_argument("--workload", choices=list(PIPELINES) + list(CONV_WORKLOADS),
+                    default="p4_vitb_mlp_f16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense F.linear comparator")
     ap.add_argument("--dp-path", action="store_true",
@@ -657,6 +902,10 @@ def main():
                          "(FP32 sums, reduction over ranks, one cast) even on one rank")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps, reported as run
+    if args.workload in CONV_WORKLOADS:
+        if args.impl == "reference":
+            return run_conv_reference(args, args.workload)
+        return run_conv(args, args.workload)
     if args.impl == "reference":
         return run_reference(args, args.workload)
     return run_ours(args, args.workload)

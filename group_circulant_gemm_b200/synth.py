@@ -84,3 +84,59 @@ def make_arrays(seed: int, T: int, N: int, C: int, D: int, dtype: str = "f32",
                 bias: bool = True, need_dy: bool = False):
     """Ad-hoc shape with the same recipe (used for edge-case tests)."""
     return make_inputs(Workload("adhoc", T, N, C, D, dtype, bias, seed), need_dy=need_dy)
+
+
+@dataclass(frozen=True)
+class ConvWorkload:
+    """A group-circulant convolution: N images of H x W pixels, C -> D channels per
+    group element, KH x KW taps, stride 1, zero padding (ph, pw)."""
+    name: str
+    T: int
+    N: int
+    H: int
+    W: int
+    C: int
+    D: int
+    KH: int
+    KW: int
+    ph: int
+    pw: int
+    dtype: str = "f16"
+    seed: int = 1300
+
+    @property
+    def Ho(self) -> int:
+        return self.H + 2 * self.ph - self.KH + 1
+
+    @property
+    def Wo(self) -> int:
+        return self.W + 2 * self.pw - self.KW + 1
+
+    def with_(self, **kw) -> "ConvWorkload":
+        return replace(self, **kw)
+
+
+# A ResNet-stage shape for p4 feature maps (64 images, 56 x 56, 64 -> 64
+# channels per group element, 3 x 3): the pages measure no convolution, so this
+# is a plain choice of a common CNN stage, not a published benchmark.
+CONV_WORKLOADS = {
+    "p4_conv3x3_f16": ConvWorkload("p4_conv3x3_f16", 4, 64, 56, 56, 64, 64, 3, 3, 1, 1, "f16",
+                                   1300),
+}
+
+
+def make_conv_inputs(w: ConvWorkload, images: int | None = None):
+    """dict(X [N, H, W, C*T], Wc [KH, KW, D, C, T], bias [D]) with the layer's recipe:
+    float64 normal draws in the order X, Wc, bias from default_rng(seed),
+    Wc ~ N(0, 1/(C*T*KH*KW)), bias ~ N(0, 0.01), cast to the dtype.  ``images``
+    keeps a prefix of the images (drawn in full first)."""
+    rng = np.random.default_rng(w.seed)
+    X = rng.standard_normal((w.N, w.H, w.W, w.C * w.T))
+    Wc = rng.standard_normal((w.KH, w.KW, w.D, w.C, w.T)) * np.sqrt(
+        1.0 / (w.C * w.T * w.KH * w.KW))
+    b = rng.standard_normal((w.D,)) * np.sqrt(0.01)
+    if images is not None:
+        X = X[:images]
+    dt = np.float16 if w.dtype == "f16" else np.float32
+    return {"X": np.ascontiguousarray(X.astype(dt)), "Wc": np.ascontiguousarray(Wc.astype(dt)),
+            "bias": np.ascontiguousarray(b.astype(dt))}
