@@ -112,6 +112,7 @@ NCU_TRAFFIC = {
     ("forward", "5facc1d5cf0b65aa"): {"p4_vitb_mlp_2calls_f16": 58.89e6, "c8_1024_f16": 34.06e6,
                                       "p4_vith_fc1_fwd_bwd_f16": 69.86e6},
     ("forward_chain", "79e08cb6e9db3b65"): {"p4_vitb_mlp_f16": 81.76e6},
+    ("conv", "0fd00f0424229b1e"): {"p4_conv3x3_f16": 160.16e6},
 }
 
 def kernel_traffic(family: str, workload: str):
