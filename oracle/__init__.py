@@ -20,6 +20,10 @@ What each function computes, and the passage of the "Flash EQ-Linear" summary
   ("Specialisation for p4", bullet 3: 6 real GEMMs, 16/6 fewer MACs).
 * :func:`p4_transform_matrices` -- the real 4x4 DFT / inverse-DFT pair for the
   p4 group ("Specialisation for p4", bullets 1-2: coefficients 0, +-1, +-1/2).
+* :func:`d4_forward` -- the layer over the dihedral group D4 (p4m), the
+  reflection group named in "Limitations and future work" (no formula given):
+  the group cross-correlation ``Y[n,d,g] = bias[d] + sum_{c,h} W[d,c,g^-1 h]
+  X[n,c,h]`` with elements ``g = a + 4b`` for ``r^a m^b``.
 * :func:`conv_forward` -- the group-circulant convolution ("Limitations and
   future work" names equivariant convolution as the next operator; no formula
   is given): the EQ-Linear's channel mixing at every tap of a KH x KW kernel,
@@ -86,6 +90,8 @@ def _load():
                                               ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int, dp, dp, dp, dp]
             lib.eqlo_conv_forward.restype = i64
+            lib.eqlo_d4_forward.argtypes = [i64, i64, i64, dp, dp, dp, dp]
+            lib.eqlo_d4_forward.restype = i64
             _lib = lib
     return _lib
 
@@ -200,6 +206,24 @@ def p4_transform_matrices():
     G = np.empty((4, 4), dtype=np.float64)
     lib.eqlo_p4_transform_matrices(_ptr(F), _ptr(G))
     return F, G
+
+
+def d4_forward(X, W, bias=None, return_macs: bool = False, act: str = "none"):
+    """Y[N, D*8] in float64 from X[N, C*8], W[D, C, 8], bias[D] or None: the layer
+    over D4, feature index c*8 + g with g = a + 4b for r^a m^b."""
+    if act not in ("none", "gelu"):
+        raise ValueError(act)
+    X, W = _f64(X), _f64(W)
+    D, C, G = W.shape
+    if G != 8 or X.ndim != 2 or X.shape[1] != C * 8:
+        raise ValueError("X must be [N, C*8] and W [D, C, 8]")
+    N = X.shape[0]
+    b = None if bias is None else _f64(bias)
+    Y = np.empty((N, D * 8), dtype=np.float64)
+    macs = _load().eqlo_d4_forward(N, C, D, _ptr(X), _ptr(W), _ptr(b), _ptr(Y))
+    if act == "gelu":
+        _load().eqlo_gelu(Y.size, _ptr(Y))
+    return (Y, macs) if return_macs else Y
 
 
 def conv_forward(T: int, X, Wc, bias=None, pad=(0, 0), return_macs: bool = False):

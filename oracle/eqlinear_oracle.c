@@ -293,3 +293,45 @@ int64_t eqlo_conv_forward(int T, int64_t N, int64_t H, int64_t Wd, int64_t C, in
   }
   return macs;
 }
+
+/*
+ * EQ-Linear over the dihedral group D4 (p4m: the four 90-degree rotations and
+ * their compositions with a mirror), the reflection group the pages name as the
+ * natural generalisation of the p4 method ("Limitations and future work"; no
+ * formula is given).  Reading: the same group-circulant weight structure with
+ * the cyclic shift replaced by the group law, i.e. a group cross-correlation
+ * over the regular representation:
+ *   Y[n][d*8+g] = bias[d] + sum_{c,h} W[d][c][g^-1 h] * X[n][c*8+h]
+ * Group elements are indexed g = a + 4 b for r^a m^b (a = 0..3 quarter turns,
+ * b = 1 with the mirror), with m r m = r^-1, so
+ *   (r^a m^b)(r^c m^e) = r^(a + (-1)^b c) m^(b+e),   (r^a m^b)^-1 = r^(-(-1)^b a) m^b.
+ * With W[d][c][u] = 0 for mirrored u and X zero on mirrored h, the rotation
+ * outputs equal the cyclic T = 4 layer.  Returns the number of real
+ * multiply-adds (N * D * C * 64).
+ */
+static int d4_mul(int g, int h) {
+  const int a = g & 3, b = g >> 2, c = h & 3, e = h >> 2;
+  const int rot = (a + (b ? -c : c)) & 3;
+  return rot + 4 * (b ^ e);
+}
+static int d4_inv(int g) {
+  const int a = g & 3, b = g >> 2;
+  return (b ? a : ((4 - a) & 3)) + 4 * b;
+}
+
+int64_t eqlo_d4_forward(int64_t N, int64_t C, int64_t D, const double* X, const double* W,
+                        const double* bias, double* Y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t d = 0; d < D; ++d) {
+      for (int g = 0; g < 8; ++g) {
+        const int gi = d4_inv(g);
+        double acc = 0.0;
+        for (int64_t c = 0; c < C; ++c)
+          for (int h = 0; h < 8; ++h) acc += W[(d * C + c) * 8 + d4_mul(gi, h)] * X[(n * C + c) * 8 + h];
+        Y[(n * D + d) * 8 + g] = acc + (bias ? bias[d] : 0.0);
+      }
+    }
+  }
+  return N * D * C * 64;
+}
