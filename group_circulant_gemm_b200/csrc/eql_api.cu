@@ -54,8 +54,10 @@ const void* adj_block(const eqlinear_plan_s* p, const void* W_hat) {
 bool has_tiles(const eqlinear_plan_s* p) {
   return eql::tc_tiles_wanted(p->T, to_dt(p->dtype), p->C, p->D);
 }
-// tensor-core operand tiles: forward (Cin = C, Cout = D) then adjoint (Cin = D, Cout = C)
+// tensor-core operand tiles: forward (Cin = C, Cout = D) then adjoint (Cin = D, Cout = C);
+// a D4 plan holds its 8 spectrum planes then the forward tiles only
 const void* fwd_tiles(const eqlinear_plan_s* p, const void* W_hat) {
+  if (p->group == 1) return static_cast<const char*>(W_hat) + 8 * plane_elems(p) * 2;
   return static_cast<const char*>(W_hat) +
          2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
 }
@@ -150,6 +152,18 @@ void eqlinear_plan_destroy(eqlinear_plan_t p) {
   delete p;
 }
 
+eqlinear_status_t eqlinear_plan_create_dihedral4(int C, int D, eqlinear_dtype_t dtype,
+                                                 eqlinear_plan_t* out) {
+  eqlinear_status_t s = eqlinear_plan_create(8, C, D, dtype, out);
+  if (s == EQL_OK) (*out)->group = 1;
+  return s;
+}
+
+// The D4 layer runs on the tensor cores only (FP16, C and D multiples of 16).
+static bool d4_ok(eqlinear_plan_t p) {
+  return p->dtype == EQL_F16 && p->kernel != EQL_KERNEL_SIMT && has_tiles(p);
+}
+
 eqlinear_status_t eqlinear_plan_set_kernel(eqlinear_plan_t p, eqlinear_kernel_t which) {
   if (!p) return EQL_ERR_INVALID_ARG;
   if (which != EQL_KERNEL_AUTO && which != EQL_KERNEL_SIMT && which != EQL_KERNEL_TCGEN05)
@@ -161,6 +175,7 @@ eqlinear_status_t eqlinear_plan_set_kernel(eqlinear_plan_t p, eqlinear_kernel_t 
 const char* eqlinear_forward_kernel_name(eqlinear_plan_t p, int64_t N) {
   if (!p) return "unsupported";
   const bool tc_ok = has_tiles(p) && eql::fwd_tc_supported(p->T, to_dt(p->dtype), N, p->C, p->D);
+  if (p->group == 1) return d4_ok(p) && tc_ok ? "tcgen05" : "unsupported";
   if (p->kernel == EQL_KERNEL_TCGEN05) return tc_ok ? "tcgen05" : "unsupported";
   if (p->kernel == EQL_KERNEL_AUTO && tc_ok) return "tcgen05";
   return "simt";
@@ -177,7 +192,7 @@ static bool wgrad_use_tc(eqlinear_plan_t p, int64_t N, const void* X, const void
 }
 
 const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t p, int64_t N) {
-  if (!p) return "unsupported";
+  if (!p || p->group == 1) return "unsupported";
   const void* aligned = reinterpret_cast<const void*>(uintptr_t(256));
   const bool tc_ok = wgrad_tc_ok(p, N, aligned, aligned);
   if (p->kernel == EQL_KERNEL_TCGEN05) return tc_ok ? "tcgen05" : "unsupported";
@@ -187,6 +202,8 @@ const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t p, int64_t N) {
 
 size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t p) {
   if (!p) return 0;
+  if (p->group == 1)
+    return d4_ok(p) ? 8 * plane_elems(p) * 2 + eql::tc_tile_bytes(8, p->C, p->D) : 0;
   size_t bytes = 2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
   if (has_tiles(p)) bytes += eql::tc_tile_bytes(p->T, p->C, p->D) + eql::tc_tile_bytes(p->T, p->D, p->C);
   return bytes;
@@ -201,6 +218,13 @@ eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, voi
   void* fwd = W_hat;
   void* adj = const_cast<void*>(adj_block(p, W_hat));
   cudaStream_t st = (cudaStream_t)stream;
+  if (p->group == 1) {
+    if (!d4_ok(p)) return EQL_ERR_UNSUPPORTED;
+    s = from_cuda(eql::launch_prepare_d4(W, p->C, p->D, fwd, st));
+    if (s != EQL_OK) return s;
+    return from_cuda(eql::launch_tile_weights(8, fwd, p->C, p->D,
+                                              const_cast<void*>(fwd_tiles(p, W_hat)), st, 1));
+  }
   s = from_cuda(eql::launch_prepare(p->T, to_dt(p->dtype), W, p->C, p->D, fwd, adj, p->tw, st));
   if (s != EQL_OK || !has_tiles(p)) return s;
   s = from_cuda(eql::launch_tile_weights(p->T, fwd, p->C, p->D, const_cast<void*>(fwd_tiles(p, W_hat)),
@@ -226,6 +250,13 @@ eqlinear_status_t eqlinear_forward_act(eqlinear_plan_t p, const void* X, int64_t
     return EQL_ERR_ALIGNMENT;
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
+  if (p->group == 1) {
+    if (!d4_ok(p) || !eql::fwd_tc_supported(8, to_dt(p->dtype), N, p->C, p->D))
+      return EQL_ERR_UNSUPPORTED;
+    return from_cuda(eql::launch_fwd_tc(8, X, N, p->C, p->D, fwd_tiles(p, W_hat), bias, Y,
+                                        p->status, p->num_sms, p->debug_drop_w_stage, (int)act,
+                                        0, (cudaStream_t)stream, 1));
+  }
   return run_forward_like(p, X, N, p->C, p->D, fwd_tiles(p, W_hat), adj_block(p, W_hat), bias,
                           Y, (int)act, (cudaStream_t)stream);
 }
@@ -393,6 +424,7 @@ eqlinear_status_t eqlinear_conv_forward(eqlinear_plan_t p, const void* X, int64_
 eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int64_t N,
                                           const void* W_hat, void* dX, void* stream) {
   if (!p || N < 0) return EQL_ERR_INVALID_ARG;
+  if (p->group == 1) return EQL_ERR_UNSUPPORTED;
   if (N == 0) return EQL_OK;
   if (!dY || !W_hat || !dX) return EQL_ERR_INVALID_ARG;
   if (!aligned16(dY) || !aligned16(W_hat) || !aligned16(dX)) return EQL_ERR_ALIGNMENT;
@@ -419,6 +451,7 @@ static eqlinear_status_t backward_weight_impl(eqlinear_plan_t p, const void* X, 
                                               size_t workspace_bytes, eql::DType out_dt,
                                               void* stream) {
   if (!p || N < 0 || !dW) return EQL_ERR_INVALID_ARG;
+  if (p->group == 1) return EQL_ERR_UNSUPPORTED;
   if (N > 0 && (!X || !dY)) return EQL_ERR_INVALID_ARG;
   if ((X && !aligned16(X)) || (dY && !aligned16(dY)) || !aligned16(dW) ||
       (dbias && !aligned16(dbias)) || (workspace && !aligned16(workspace)))

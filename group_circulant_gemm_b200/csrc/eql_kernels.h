@@ -48,7 +48,10 @@ cudaError_t launch_wgrad_finalize(int T, DType out_dt, const float* part, const 
 bool tc_tiles_wanted(int T, DType dt, int C, int D);
 size_t tc_tile_bytes(int T, int Cin, int Cout);
 cudaError_t launch_tile_weights(int T, const void* planes /* [P][Cout][Cin] */, int Cin,
-                                int Cout, void* tiles, cudaStream_t st);
+                                int Cout, void* tiles, cudaStream_t st, int group = 0);
+// The dihedral group D4 (T = 8 layout, group = 1): its weight spectrum in the
+// tile regions' order, W [D][C][8] -> planes [8][D][C] (FP16).
+cudaError_t launch_prepare_d4(const void* W, int C, int D, void* planes, cudaStream_t st);
 // Returns cudaErrorNotSupported when the shape does not fit the kernel.
 bool fwd_tc_supported(int T, DType dt, int64_t N, int Cin, int Cout);
 // drop_w_stage >= 0 is a test-only fault: CTA 0 never issues that weight stage,
@@ -58,7 +61,8 @@ bool fwd_tc_supported(int T, DType dt, int64_t N, int Cin, int Cout);
 // 2 = X read as spectral planes [4][N][Cin] produced that way.
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
-                          int num_sms, int drop_w_stage, int act, int io, cudaStream_t st);
+                          int num_sms, int drop_w_stage, int act, int io, cudaStream_t st,
+                          int group = 0);
 
 // tcgen05/TMEM tensor-core weight gradient for T = 4, FP16: stream-K over
 // (tile, 32-row stage) ranges, FP32 partial slots in `workspace`, then a

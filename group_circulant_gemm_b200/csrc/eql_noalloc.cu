@@ -52,6 +52,7 @@ extern "C" eqlinear_status_t eqlinear_backward_weight_noalloc(eqlinear_plan_t p,
                                                               void* dW, void* dbias,
                                                               void* stream) {
   if (!p || N < 0 || !dW) return EQL_ERR_INVALID_ARG;
+  if (p->group == 1) return EQL_ERR_UNSUPPORTED;  // the D4 layer has no backward
   if (N > 0 && (!X || !dY)) return EQL_ERR_INVALID_ARG;
   if ((X && !aligned16(X)) || (dY && !aligned16(dY)) || !aligned16(dW) ||
       (dbias && !aligned16(dbias)))

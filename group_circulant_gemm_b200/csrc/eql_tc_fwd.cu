@@ -57,7 +57,7 @@ namespace {
 using namespace tc;
 using namespace ftc;
 
-template <int T, int ACT, int IO>
+template <int T, int ACT, int IO, int G = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     eq_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                      const __grid_constant__ CUtensorMap map_y, const uint8_t* __restrict__ wtiles,
@@ -177,6 +177,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
             auto A = [&](int p) { return desc_kmajor<S::ROWB>(pl + p * S::PLANE_BYTES + ko); };
             auto B = [&](int p) { return desc_kmajor<S::ROWB>(wr + p * S::WREG_BYTES + ko); };
+            if constexpr (G == 1) {
+              // D4: four characters (N = BD each), then the 2 x 2 block
+              // Y[i][k] = sum_j X[i][j] W[k][j]: per (i, j) one N = 2 BD MMA into
+              // [Y[i][0] | Y[i][1]] with weight regions 4+2j (k = 0), 5+2j (k = 1)
+#pragma unroll
+              for (int p = 0; p < 4; ++p) umma(tmem + p * BD, A(p), B(p), id_n1, acc);
+#pragma unroll
+              for (int i = 0; i < 2; ++i) {
+                umma(tmem + 4 * BD + 2 * BD * i, A(4 + 2 * i), B(4), id_n2, acc);
+                umma(tmem + 4 * BD + 2 * BD * i, A(5 + 2 * i), B(6), id_n2, 1u);
+              }
+              continue;
+            }
             // real frequencies 0 and T/2
             umma(tmem + 0, A(0), B(0), id_n1, acc);
             umma(tmem + BD, A(1), B(1), id_n1, acc);
@@ -226,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&bars->acc_full, tcount & 1, abort_flag, status)) break;
       tc_fence_after();
       const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-      epi_slices<T, BD, ACT, IO>(lane_addr, ch, lane, stg, bsm, dbase, Cout,
-                                 StoreOf<T, IO>{&map_y, row0, N});
+      epi_slices<T, BD, ACT, IO, StoreOf<T, IO>, G>(lane_addr, ch, lane, stg, bsm, dbase, Cout,
+                                                    StoreOf<T, IO>{&map_y, row0, N});
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
     }
@@ -250,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->x_read[sx]);
         if (!(ok = warp_wait(&bars->x_read[sx], (it / S::X_ST) & 1, abort_flag, status))) break;
-        xf_write<T>(slot, xt, v);
+        xf_write<T, G>(slot, xt, v);
         // make the generic-proxy stores visible to the tensor core (async proxy)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
@@ -273,10 +286,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // image: blob (dt, ks) = regions 0..T-1 (prepared planes 0..T-1: real frequency
 // 0, real frequency T/2, then Re and Im of each complex frequency), each BD rows
 // x BK channels in the K-major swizzled layout the MMAs read; rows and channels
-// past the matrix are zero.  One thread per 16-byte piece.
+// past the matrix are zero.  One thread per 16-byte piece.  Regions below nreal
+// hold one-dimensional frequencies (inverse factor 1/T), the others entries of
+// two-dimensional ones (2/T): nreal = 2 for the cyclic groups of even order, 4 for D4.
 template <int T>
 __global__ void tile_weights_kernel(const __half* __restrict__ planes, int Cin, int Cout,
-                                    int n_ks, int64_t n_chunks, uint4* __restrict__ tiles) {
+                                    int n_ks, int64_t n_chunks, int nreal,
+                                    uint4* __restrict__ tiles) {
   using S = Shape<T>;
   constexpr int kPieces = S::ROWB / 16;  // 16-byte pieces per row
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -292,7 +308,7 @@ __global__ void tile_weights_kernel(const __half* __restrict__ planes, int Cin, 
     v = *reinterpret_cast<const uint4*>(planes + ((int64_t)region * Cout + d) * Cin + c0);
     // the inverse DFT's factors 1/T (real frequencies) and 2/T (complex), exact
     // powers of two, applied here so the epilogue needs no multiplies by them
-    const __half2 s = __float2half2_rn(region < 2 ? 1.f / T : 2.f / T);
+    const __half2 s = __float2half2_rn(region < nreal ? 1.f / T : 2.f / T);
     __half2* h = reinterpret_cast<__half2*>(&v);
 #pragma unroll
     for (int i = 0; i < 4; ++i) h[i] = __hmul2(h[i], s);
@@ -335,7 +351,8 @@ size_t tc_tile_bytes(int T, int Cin, int Cout) {
 }
 
 cudaError_t launch_tile_weights(int T, const void* planes, int Cin, int Cout, void* tiles,
-                                cudaStream_t st) {
+                                cudaStream_t st, int group) {
+  if (group != 0 && T != 8) return cudaErrorNotSupported;
   return dispatch_tc(T, [&](auto tcst) {
     constexpr int TT = decltype(tcst)::value;
     using S = Shape<TT>;
@@ -343,7 +360,8 @@ cudaError_t launch_tile_weights(int T, const void* planes, int Cin, int Cout, vo
     const int64_t n_chunks = (int64_t)tc_tile_bytes(TT, Cin, Cout) / 16;
     const unsigned blocks = (unsigned)((n_chunks + 255) / 256);
     tile_weights_kernel<TT><<<blocks, 256, 0, st>>>(static_cast<const __half*>(planes), Cin, Cout,
-                                                    n_ks, n_chunks, static_cast<uint4*>(tiles));
+                                                    n_ks, n_chunks, group ? 4 : 2,
+                                                    static_cast<uint4*>(tiles));
     return cudaGetLastError();
   });
 }
@@ -363,20 +381,53 @@ bool encode_planes_map(CUtensorMap* m, void* base, int channels, int64_t N, uint
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int TT, int ACT, int IO>
+template <int TT, int ACT, int IO, int G = 0>
 cudaError_t set_smem_attr() {
-  return cudaFuncSetAttribute(eq_fwd_tc_kernel<TT, ACT, IO>,
+  return cudaFuncSetAttribute(eq_fwd_tc_kernel<TT, ACT, IO, G>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, Shape<TT>::SMEM_BYTES);
+}
+
+// D4 weight spectrum, in the tile regions' order: W^(rho) = sum_u W(u) rho(u)
+// for the characters (+,+), (+,-), (-,+), (-,-) and the 2 x 2 entries 00, 10,
+// 01, 11 (region 4 + 2j + k holds entry [k][j]); FP32, one rounding.
+// W [D][C][8] -> planes [8][D][C].  One thread per (d, c).
+__global__ void prepare_d4_kernel(const __half* __restrict__ W, int C, int D,
+                                  __half* __restrict__ planes) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t plane = (int64_t)C * D;
+  if (idx >= plane) return;
+  float x[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) x[u] = __half2float(W[idx * 8 + u]);
+  const float e0 = x[0] + x[2], o0 = x[1] + x[3], e1 = x[4] + x[6], o1 = x[5] + x[7];
+  const float d0 = x[0] - x[2], d1 = x[1] - x[3], d4 = x[4] - x[6], d5 = x[5] - x[7];
+  const float v[8] = {(e0 + o0) + (e1 + o1), (e0 + o0) - (e1 + o1), (e0 - o0) + (e1 - o1),
+                      (e0 - o0) - (e1 - o1),
+                      d0 + d4,   // [0][0]
+                      d1 + d5,   // [1][0]
+                      d5 - d1,   // [0][1]
+                      d0 - d4};  // [1][1]
+#pragma unroll
+  for (int r = 0; r < 8; ++r) planes[r * plane + idx] = __float2half_rn(v[r]);
 }
 
 }  // namespace
 
+cudaError_t launch_prepare_d4(const void* W, int C, int D, void* planes, cudaStream_t st) {
+  const int64_t total = (int64_t)C * D;
+  prepare_d4_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+      static_cast<const __half*>(W), C, D, static_cast<__half*>(planes));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
-                          int num_sms, int drop_w_stage, int act, int io, cudaStream_t st) {
+                          int num_sms, int drop_w_stage, int act, int io, cudaStream_t st,
+                          int group) {
   if (!fwd_tc_supported(T, DType::F16, N, Cin, Cout)) return cudaErrorNotSupported;
   if (!Wtiles) return cudaErrorNotSupported;
   if (io != kIoSpatial && T != 4) return cudaErrorNotSupported;
+  if (group != 0 && (T != 8 || io != kIoSpatial)) return cudaErrorNotSupported;
   if (act != 0 && act != 1) return cudaErrorInvalidValue;
 
   auto encode = encode_fn();
@@ -434,6 +485,9 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
         if (e == cudaSuccess) e = set_smem_attr<TT, 1, kIoSpectralOut>();
         if (e == cudaSuccess) e = set_smem_attr<TT, 0, kIoSpectralIn>();
         if (e == cudaSuccess) e = set_smem_attr<TT, 1, kIoSpectralIn>();
+      } else {
+        if (e == cudaSuccess) e = set_smem_attr<TT, 0, kIoSpatial, 1>();
+        if (e == cudaSuccess) e = set_smem_attr<TT, 1, kIoSpatial, 1>();
       }
       if (e != cudaSuccess) return e;
       attr_set = true;
@@ -447,6 +501,10 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
       else if (io == kIoSpectralIn)
         kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1, kIoSpectralIn>
                           : eq_fwd_tc_kernel<TT, 0, kIoSpectralIn>;
+    } else {
+      if (group == 1)
+        kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1, kIoSpatial, 1>
+                          : eq_fwd_tc_kernel<TT, 0, kIoSpatial, 1>;
     }
     kernel<<<grid, kThreads, S::SMEM_BYTES, st>>>(
         mx, my, static_cast<const uint8_t*>(Wtiles), static_cast<const __half*>(bias), N, Cin,

@@ -125,7 +125,9 @@ __device__ __forceinline__ void xf_read(const uint8_t* slot, int xt, uint4 (&v)[
   }
 }
 
-template <int T>
+// G = 1 (T = 8 layout): the group is the dihedral group D4, element g = a + 4b
+// for r^a m^b; the planes are its Fourier coefficients (below).
+template <int T, int G = 0>
 __device__ __forceinline__ void xf_write(uint8_t* slot, int xt, const uint4 (&v)[8]) {
   using S = Shape<T>;
   if constexpr (T == 4) {
@@ -179,6 +181,24 @@ __device__ __forceinline__ void xf_write(uint8_t* slot, int xt, const uint4 (&v)
       for (int hh = 0; hh < 2; ++hh) {
         const uint4 w = v[2 * pr + hh];
         const float2 p01 = f2(w.x), p23 = f2(w.y), p45 = f2(w.z), p67 = f2(w.w);
+        if constexpr (G == 1) {
+          // D4: X^(rho) = sum_g x_g rho(g).  Characters chi(r) = +-1, chi(m) = +-1
+          // (planes 0..3: (+,+), (+,-), (-,+), (-,-)); the 2 x 2 representation
+          // r -> [[0,-1],[1,0]], m -> diag(1,-1) (planes 4..7: entries 00, 01, 10, 11).
+          const float e0 = p01.x + p23.x, o0 = p01.y + p23.y;  // x0+x2, x1+x3
+          const float e1 = p45.x + p67.x, o1 = p45.y + p67.y;  // x4+x6, x5+x7
+          const float d0 = p01.x - p23.x, d1 = p01.y - p23.y;  // x0-x2, x1-x3
+          const float d4 = p45.x - p67.x, d5 = p45.y - p67.y;  // x4-x6, x5-x7
+          val[0][hh] = (e0 + o0) + (e1 + o1);
+          val[1][hh] = (e0 + o0) - (e1 + o1);
+          val[2][hh] = (e0 - o0) + (e1 - o1);
+          val[3][hh] = (e0 - o0) - (e1 - o1);
+          val[4][hh] = d0 + d4;
+          val[5][hh] = d5 - d1;
+          val[6][hh] = d1 + d5;
+          val[7][hh] = d0 - d4;
+          continue;
+        }
         const float a0 = p01.x + p45.x, a1 = p01.y + p45.y, a2 = p23.x + p67.x, a3 = p23.y + p67.y;
         const float b0 = p01.x - p45.x, b1 = p01.y - p45.y, b2 = p23.x - p67.x, b3 = p23.y - p67.y;
         const float s13 = h * (b1 - b3), t13 = h * (b1 + b3);
@@ -209,7 +229,7 @@ __device__ __forceinline__ void xf_write(uint8_t* slot, int xt, const uint4 (&v)
 // FP16 output (four 16-byte pieces, in Y's channel-major, group-minor order).
 // Plane p of out-channel c sits in TMEM column p * BD + c.
 // ---------------------------------------------------------------------------
-template <int T, int BD, int ACT>
+template <int T, int BD, int ACT, int G = 0>
 __device__ __forceinline__ void epi_half(uint32_t lane_addr, int c0, const __half* bsm,
                                          uint4 (&o)[4]) {
   constexpr int NCH = 32 / T;
@@ -257,6 +277,19 @@ __device__ __forceinline__ void epi_half(uint32_t lane_addr, int c0, const __hal
       float Yv[8];
 #pragma unroll
       for (int p = 0; p < 8; ++p) Yv[p] = __uint_as_float(v[p][i]);
+      if constexpr (G == 1) {
+        // D4, accumulators arrive scaled (characters by 1/8, the 2 x 2 block by 2/8):
+        // y(g) = sum_p chi_p(g) c_p + sum_{i,k} rho(g)_ik m_ik  (+ bias), g = a + 4b
+        const float s = Yv[0] + b[i];
+        const float P = s + Yv[2], Q = s - Yv[2], U = Yv[1] + Yv[3], V = Yv[1] - Yv[3];
+        const float E = Yv[4] + Yv[7], F = Yv[6] - Yv[5], Gm = Yv[4] - Yv[7],
+                    H = Yv[5] + Yv[6];
+        o[i] = make_uint4(pack_h2(act_fn<ACT>(P + U + E), act_fn<ACT>(Q + V + F)),
+                          pack_h2(act_fn<ACT>(P + U - E), act_fn<ACT>(Q + V - F)),
+                          pack_h2(act_fn<ACT>(P - U + Gm), act_fn<ACT>(Q - V + H)),
+                          pack_h2(act_fn<ACT>(P - U - Gm), act_fn<ACT>(Q - V - H)));
+        continue;
+      }
       const float s = Yv[0] + b[i];
       const float E = s + Yv[1], O = s - Yv[1];
       const float A0 = E + Yv[4], A2 = E - Yv[4];
@@ -318,7 +351,7 @@ __device__ __forceinline__ void epi_half_spec(uint32_t lane_addr, int c0, const 
 // output); each slice is staged in the warp's 4 KB buffer and written by one TMA
 // store, store(staging address, first out-channel of the slice), issued by lane 0.
 // bsm holds the half's biases; dbase is the half's first out-channel.
-template <int T, int BD, int ACT, int IO, class Store>
+template <int T, int BD, int ACT, int IO, class Store, int G = 0>
 __device__ __forceinline__ void epi_slices(uint32_t lane_addr, int ch, int lane, uint8_t* stg,
                                            const __half* bsm, int dbase, int Cout,
                                            const Store& store) {
@@ -355,14 +388,14 @@ __device__ __forceinline__ void epi_slices(uint32_t lane_addr, int ch, int lane,
       continue;
     }
     uint4 o[4];
-    epi_half<T, BD, ACT>(lane_addr, c0, bs, o);
+    epi_half<T, BD, ACT, G>(lane_addr, c0, bs, o);
     // the previous slice's store has finished reading the buffer
     if (lane == 0) bulk_wait_read_all();
     __syncwarp();
 #pragma unroll
     for (int m = 0; m < 4; ++m)
       *reinterpret_cast<uint4*>(my_row + ((m ^ (lane & 7)) << 4)) = o[m];
-    epi_half<T, BD, ACT>(lane_addr, c0 + 32 / T, bs + 32 / T, o);
+    epi_half<T, BD, ACT, G>(lane_addr, c0 + 32 / T, bs + 32 / T, o);
 #pragma unroll
     for (int m = 0; m < 4; ++m)
       *reinterpret_cast<uint4*>(my_row + (((4 + m) ^ (lane & 7)) << 4)) = o[m];

@@ -15,13 +15,24 @@ _KERNEL = {"auto": _n.EQL_KERNEL_AUTO, "simt": _n.EQL_KERNEL_SIMT,
 
 
 class EqLinearPlan:
-    """A plan for the EQ-Linear layer of group order T, C -> D channels."""
+    """A plan for the EQ-Linear layer of group order T, C -> D channels.
 
-    def __init__(self, T: int, C: int, D: int, dtype: torch.dtype, kernel: str = "auto"):
+    ``group="dihedral4"`` makes the layer over the dihedral group D4 instead of
+    the cyclic group (T must be 8; forward only, FP16)."""
+
+    def __init__(self, T: int, C: int, D: int, dtype: torch.dtype, kernel: str = "auto",
+                 group: str = "cyclic"):
         if dtype not in _DT:
             raise ValueError(f"unsupported dtype {dtype}")
-        self.T, self.C, self.D, self.dtype = T, C, D, dtype
-        self.handle = _n.eqlinear_plan_create(T, C, D, _DT[dtype])
+        self.T, self.C, self.D, self.dtype, self.group = T, C, D, dtype, group
+        if group == "dihedral4":
+            if T != 8:
+                raise ValueError("D4 has eight elements: T must be 8")
+            self.handle = _n.eqlinear_plan_create_dihedral4(C, D, _DT[dtype])
+        elif group == "cyclic":
+            self.handle = _n.eqlinear_plan_create(T, C, D, _DT[dtype])
+        else:
+            raise ValueError(f"unknown group {group}")
         self.set_kernel(kernel)
 
     def set_kernel(self, kernel: str) -> None:

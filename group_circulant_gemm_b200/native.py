@@ -33,6 +33,7 @@ EXPORTED = (
     "eqlinear_chain_workspace_bytes", "eqlinear_forward_chain",
     "eqlinear_conv_prepared_weight_bytes", "eqlinear_conv_prepare_weights",
     "eqlinear_conv_workspace_bytes", "eqlinear_conv_forward",
+    "eqlinear_plan_create_dihedral4",
 )
 
 
@@ -53,6 +54,7 @@ def _load() -> ctypes.CDLL:
         "eqlinear_version": ([], i32),
         "eqlinear_status_string": ([i32], ctypes.c_char_p),
         "eqlinear_plan_create": ([i32, i32, i32, i32, ctypes.POINTER(vp)], i32),
+        "eqlinear_plan_create_dihedral4": ([i32, i32, i32, ctypes.POINTER(vp)], i32),
         "eqlinear_plan_destroy": ([vp], None),
         "eqlinear_plan_set_kernel": ([vp, i32], i32),
         "eqlinear_forward_kernel_name": ([vp, i64], ctypes.c_char_p),
@@ -124,6 +126,13 @@ def eqlinear_status_string(status: int) -> str:
 def eqlinear_plan_create(T: int, C: int, D: int, dtype: int) -> int:
     out = ctypes.c_void_p()
     _check(_lib.eqlinear_plan_create(T, C, D, dtype, ctypes.byref(out)), "eqlinear_plan_create")
+    return out.value
+
+
+def eqlinear_plan_create_dihedral4(C: int, D: int, dtype: int) -> int:
+    out = ctypes.c_void_p()
+    _check(_lib.eqlinear_plan_create_dihedral4(C, D, dtype, ctypes.byref(out)),
+           "eqlinear_plan_create_dihedral4")
     return out.value
 
 

@@ -91,6 +91,26 @@ EQL_API const char* eqlinear_status_string(eqlinear_status_t status);
 EQL_API eqlinear_status_t eqlinear_plan_create(int T, int C, int D, eqlinear_dtype_t dtype,
                                        eqlinear_plan_t* out);
 
+/*
+ * A plan for the layer over the dihedral group D4 (p4m: quarter turns and a
+ * mirror; the pages name reflection groups as the natural generalisation,
+ * "Limitations and future work", without a formula).  Reading: the same
+ * group-circulant weight structure with the group law in place of the cyclic
+ * shift,
+ *   Y[n, d*8+g] = bias[d] + sum_{c,h} W[d][c][g^-1 h] * X[n, c*8+h],
+ * group element g = a + 4b for r^a m^b (m r m = r^-1).  D4 is not abelian: its
+ * Fourier transform has four characters and one 2 x 2 representation (entries
+ * 0, +-1, so the transforms are adds), and the per-frequency products are four
+ * real GEMMs plus a 2 x 2 block product (eight), 12 real products per (row,
+ * in-channel, out-channel) against the dense 64.
+ * Supported: FP16, C and D multiples of 16, forward only (eqlinear_forward and
+ * eqlinear_forward_act on the tensor cores); eqlinear_prepared_weight_bytes is
+ * 0 and every other call returns EQL_ERR_UNSUPPORTED for other plans of this
+ * kind.  W [D][C][8], X [N][C*8], Y [N][D*8].  Free with eqlinear_plan_destroy.
+ */
+EQL_API eqlinear_status_t eqlinear_plan_create_dihedral4(int C, int D, eqlinear_dtype_t dtype,
+                                                        eqlinear_plan_t* out);
+
 /* Free the plan and its status word.  NULL is ignored.  The caller must make
  * sure no call using the plan is still running on any stream. */
 EQL_API void eqlinear_plan_destroy(eqlinear_plan_t plan);
