@@ -11,7 +11,8 @@ from pinned host memory and the result read back, inside the timed region.
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
        [--workload p4_vitb_mlp_f16|p4_vitb_mlp_2calls_f16|p4_vitb_proj_f32|p4_vith_fc1_f16|
                    c8_1024_f16|p4_vith_fc1_fwd_bwd_f16|p4_vitb_mlp_block_f16|
-                   p4_vitb_mlp_spectral_f16|p4_conv3x3_f16] [--dp-path] [--no-dense]
+                   p4_vitb_mlp_spectral_f16|p4m_vitb_mlp_f16|p4_conv3x3_f16] [--dp-path]
+       [--no-dense]
        [--no-cpu-baseline]
 Under torchrun (N > 1) every rank runs its own copy of the workload (weak
 scaling; rows are independent, so no collective is on the forward path).  The
@@ -51,7 +52,11 @@ PIPELINES = {
     "p4_vith_fc1_fwd_bwd_f16": ["p4_vith_fc1_f16"],
     "p4_vitb_mlp_block_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
     "p4_vitb_mlp_spectral_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
+    "p4m_vitb_mlp_f16": ["p4m_vitb_fc1_f16", "p4m_vitb_fc2_f16"],
 }
+# pipelines whose layers are over the dihedral group D4 (T = 8 elements) instead
+# of the cyclic group
+DIHEDRAL = {"p4m_vitb_mlp_f16"}
 # two-layer pipelines whose intermediate stays in the frequency domain (the first
 # layer's epilogue writes the second layer's operand planes)
 SPECTRAL = {"p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectral_f16"}
@@ -81,11 +86,21 @@ DESCR = {
     "p4_vitb_mlp_spectral_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
                                 "C=768->D=192, T=4; intermediate kept as the second layer's "
                                 "spectral planes; one chained launch",
+    "p4m_vitb_mlp_f16": "p4m (dihedral D4, 8 elements) EQ-Linear fp16 ViT-B MLP pair: N=12608, "
+                        "C=96->D=384 then C=384->D=96 per group element (768->3072->768 "
+                        "features); one launch per layer",
 }
 
 
+def is_d4(w) -> bool:
+    return w.name.startswith("p4m_")
+
+
 def layer_flops(w) -> float:
-    """Algorithmic FLOPs of one forward: 2 * (real GEMMs per frequency plan) * N*C*D."""
+    """Algorithmic FLOPs of one forward: 2 * (real GEMMs per frequency plan) * N*C*D
+    (D4: four characters and a 2 x 2 block, 4 + 8 real GEMMs)."""
+    if is_d4(w):
+        return 2.0 * 12 * w.N * w.C * w.D
     nr = 2 if w.T % 2 == 0 else 1
     nc = (w.T - nr) // 2
     return 2.0 * (nr + 4 * nc) * w.N * w.C * w.D
@@ -95,7 +110,7 @@ def layer_bytes(w) -> float:
     """Algorithmic HBM bytes of one forward: read X, prepared weights, bias; write Y."""
     es = 2 if w.dtype == "f16" else 4
     nr = 2 if w.T % 2 == 0 else 1
-    planes = w.T + (w.T - nr) // 2
+    planes = 8 if is_d4(w) else w.T + (w.T - nr) // 2
     return es * (w.N * w.C * w.T + w.N * w.D * w.T + planes * w.C * w.D + w.D)
 
 
@@ -177,13 +192,17 @@ class ClockSampler:
             return
         self._nvml = nv
 
+        def one():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                self.samples.append((time.perf_counter(), sm, mx, int(reasons(h))))
+            except Exception:
+                pass
+        self._one = one
+
         def run():
             while not self._stop.is_set():
-                try:
-                    sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
-                    self.samples.append((time.perf_counter(), sm, mx, int(reasons(h))))
-                except Exception:
-                    pass
+                one()
                 time.sleep(0.002)
 
         self._thread = threading.Thread(target=run, daemon=True)
@@ -191,6 +210,14 @@ class ClockSampler:
 
     def mark(self, which: int):
         self.window[which] = time.perf_counter()
+
+    def sample_now(self):
+        """One sample from the calling thread (the timed loop calls this every few
+        launches, while the GPU works through the queue, so a short timed region
+        is covered even when the polling thread is not scheduled)."""
+        one = getattr(self, "_one", None)
+        if one is not None:
+            one()
 
     def stop(self):
         out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
@@ -217,6 +244,29 @@ class ClockSampler:
         return out
 
 
+def capture_graphs(step, nsets):
+    """One CUDA graph per rotating input/output set, each holding one step's
+    launches, so the timed region replays them without per-launch host work."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for k in range(nsets):
+            step(k)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graphs = []
+    for k in range(nsets):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(k)
+        graphs.append(g)
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    return graphs
+
+
 def dist_init():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -234,7 +284,10 @@ def oracle_sample(pipeline, rows: int, backward: bool = False, acts=None):
     x = layers[0][1]["X"].astype(np.float64)
     t0 = time.perf_counter()
     for (w, inp), act in zip(layers, acts):
-        x = oracle.forward(w.T, x, inp["W"], inp["bias"], act=act)
+        if is_d4(w):
+            x = oracle.d4_forward(x, inp["W"], inp["bias"], act=act)
+        else:
+            x = oracle.forward(w.T, x, inp["W"], inp["bias"], act=act)
     if backward:
         w, inp = layers[0]
         oracle.backward_input(w.T, inp["dY"], inp["W"])
@@ -290,7 +343,7 @@ def dense_flops(w) -> float:
     return 2.0 * w.N * (w.C * w.T) * (w.D * w.T)
 
 
-def dense_comparator(pipeline, backward, xs, dys, nsets, steps, rank, acts=None):
+def dense_comparator(pipeline, backward, xs, dys, nsets, steps, rank, acts=None, eager=False):
     """Same-GPU dense baseline: torch F.linear (cuBLAS) on the replicated
     (D*T x C*T) matrix M[(d,s),(c,t)] = W[d,c,(t-s) mod T] in the same dtype, GEMM
     time only (M built outside the timed region); for the training step also
@@ -303,8 +356,20 @@ def dense_comparator(pipeline, backward, xs, dys, nsets, steps, rank, acts=None)
         inp = make_inputs(w.with_(seed=w.seed + 1000 * rank), rows=1)
         W = torch.from_numpy(inp["W"]).cuda()
         M = torch.empty((w.D, w.T, w.C, w.T), dtype=W.dtype, device="cuda")
-        for sh in range(w.T):
-            M[:, sh] = torch.roll(W, shifts=sh, dims=2)
+        if is_d4(w):
+            # M[(d,g),(c,h)] = W[d, c, g^-1 h] with g = a + 4b for r^a m^b (m r m = r^-1)
+            def mul(g, h):
+                a, bb, c, e = g & 3, g >> 2, h & 3, h >> 2
+                return ((a + (-c if bb else c)) & 3) + 4 * (bb ^ e)
+
+            def inv(g):
+                return ((g & 3) if g >> 2 else (-(g & 3)) & 3) + 4 * (g >> 2)
+            for g in range(8):
+                idx = torch.tensor([mul(inv(g), h) for h in range(8)], device="cuda")
+                M[:, g] = W[:, :, idx]
+        else:
+            for sh in range(w.T):
+                M[:, sh] = torch.roll(W, shifts=sh, dims=2)
         Ms.append(M.reshape(w.D * w.T, w.C * w.T))
         bs.append(torch.from_numpy(inp["bias"]).cuda().repeat_interleave(w.T) if w.bias else None)
     outs = []
@@ -335,18 +400,30 @@ def dense_comparator(pipeline, backward, xs, dys, nsets, steps, rank, acts=None)
     for i in range(3):
         step(i)
     torch.cuda.synchronize()
+    # timed the same way as our step: CUDA graph replays, per-op times from an
+    # eager pass with events
+    graphs = None if eager else capture_graphs(step, nsets)
     ev = []
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(steps):
-        step(3 + i, ev)
+        if graphs is not None:
+            graphs[(3 + i) % nsets].replay()
+        else:
+            step(3 + i, ev)
     t1.record(stream)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / steps
-    nops = len(ev) // 2 // steps
+    op_steps = steps
+    if graphs is not None:
+        op_steps = min(steps, 50)
+        for i in range(op_steps):
+            step(3 + i, ev)
+        torch.cuda.synchronize()
+    nops = len(ev) // 2 // op_steps
     op_ms = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1])
-                      for j in range(len(ev) // 2)]).reshape(steps, nops).mean(axis=0)
+                      for j in range(len(ev) // 2)]).reshape(op_steps, nops).mean(axis=0)
     flops = sum(dense_flops(w) for w in pipeline) + (2 * dense_flops(pipeline[0]) if backward else 0)
     return {"kind": "dense F.linear on the replicated (D*T x C*T) matrix, cuBLAS, same dtype, "
                     "GEMM time only" + ("; training step adds dY@M and dY^T@X" if backward else "")
@@ -380,7 +457,7 @@ def run_ours(args, workload):
     plans, whats, biases = [], [], []
     for w in pipeline:
         inp = make_inputs(w.with_(seed=w.seed + 1000 * rank), rows=1)
-        p = EqLinearPlan(w.T, w.C, w.D, dt)
+        p = EqLinearPlan(w.T, w.C, w.D, dt, group="dihedral4" if is_d4(w) else "cyclic")
         W = torch.from_numpy(inp["W"]).cuda()
         plans.append(p)
         whats.append(p.prepare_weights(W))
@@ -497,6 +574,12 @@ def run_ours(args, workload):
     for p in plans:
         assert p.status() == 0
 
+    # the timed steps replay CUDA graphs (one per rotating set); the data-parallel
+    # training step, whose all-reduce is queued asynchronously, runs eagerly
+    graphs = None if (dp or args.eager) else capture_graphs(step, nsets)
+    for p in plans:
+        assert p.status() == 0
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -506,7 +589,12 @@ def run_ours(args, workload):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(args.steps):
-        step(args.warmup + i, ev)
+        if graphs is not None:
+            graphs[(args.warmup + i) % nsets].replay()
+        else:
+            step(args.warmup + i, ev)
+        if rank == 0 and i % 16 == 15:
+            clocks.sample_now()
     t1.record(stream)
     torch.cuda.synchronize()
     clocks.mark(1)
@@ -514,8 +602,18 @@ def run_ours(args, workload):
         dist.barrier()
     clk = clocks.stop() if rank == 0 else {}
     elapsed_ms = t0.elapsed_time(t1)
+    op_steps = args.steps
+    if graphs is not None:
+        # per-launch times: an eager pass with events around every launch
+        op_steps = min(args.steps, 100)
+        for i in range(op_steps):
+            step(args.warmup + i, ev)
+        torch.cuda.synchronize()
     launch_ms = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1])
-                          for j in range(len(ev) // 2)]).reshape(args.steps, len(ops))
+                          for j in range(len(ev) // 2)]).reshape(op_steps, len(ops))
+    timing = ("CUDA graph replay of each step (one graph per rotating set); per-launch times "
+              f"from {op_steps} eager steps with events around each launch"
+              if graphs is not None else "eager launches with events around each launch")
 
     # end to end through the ABI: pinned host inputs -> device, the step, results -> host
     x_pin = torch.from_numpy(x_host).pin_memory()
@@ -600,7 +698,7 @@ def run_ours(args, workload):
         comparator = None
         if not args.no_dense:
             comparator = dense_comparator(pipeline, backward, xs, dys if backward else None,
-                                          nsets, min(args.steps, 200), rank, acts)
+                                          nsets, min(args.steps, 200), rank, acts, args.eager)
             comparator["ours_over_dense"] = value / comparator["value"]
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -627,7 +725,8 @@ def run_ours(args, workload):
                                        if dp else f"replicas x{world} (rows independent)"),
                        "l2": f"{nsets} rotating input/output sets of {per_set / 2**20:.0f} MiB "
                              "(> 2x L2)",
-                       "kernels": [f"{label}[{k}]" for label, k, _, _, _ in ops]},
+                       "kernels": [f"{label}[{k}]" for label, k, _, _, _ in ops],
+                       "timing": timing},
             "op_ms": [round(float(m), 5) for m in mean_ms],
             "roofline": roof,
             "cpu_baseline": cpu,
@@ -758,6 +857,7 @@ def run_conv(args, workload):
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
+    graphs = None if args.eager else capture_graphs(step, nsets)
     assert p.status() == 0
     if world > 1:
         dist.barrier()
@@ -768,7 +868,12 @@ def run_conv(args, workload):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(args.steps):
-        step(args.warmup + i, ev)
+        if graphs is not None:
+            graphs[(args.warmup + i) % nsets].replay()
+        else:
+            step(args.warmup + i, ev)
+        if rank == 0 and i % 16 == 15:
+            clocks.sample_now()
     t1.record(stream)
     torch.cuda.synchronize()
     clocks.mark(1)
@@ -776,8 +881,17 @@ def run_conv(args, workload):
         dist.barrier()
     clk = clocks.stop() if rank == 0 else {}
     elapsed_ms = t0.elapsed_time(t1)
+    op_steps = args.steps
+    if graphs is not None:
+        op_steps = min(args.steps, 100)
+        for i in range(op_steps):
+            step(args.warmup + i, ev)
+        torch.cuda.synchronize()
     launch_ms = float(np.mean([ev[2 * j].elapsed_time(ev[2 * j + 1])
                                for j in range(len(ev) // 2)]))
+    timing = ("CUDA graph replay of each step (one graph per rotating set); per-call time "
+              f"from {op_steps} eager steps with events around each call"
+              if graphs is not None else "eager launches with events around each call")
 
     x_pin = torch.from_numpy(x_host).pin_memory()
     y_pin = torch.empty(tuple(ys[0].shape), dtype=torch.float16).pin_memory()
@@ -833,12 +947,16 @@ def run_conv(args, workload):
             for i in range(3):
                 dense(i)
             torch.cuda.synchronize()
+            dgraphs = None if args.eager else capture_graphs(lambda i: dense(i), nsets)
             d0 = torch.cuda.Event(enable_timing=True)
             d1 = torch.cuda.Event(enable_timing=True)
             nd = min(args.steps, 100)
             d0.record(stream)
             for i in range(nd):
-                dense(i)
+                if dgraphs is not None:
+                    dgraphs[i % nsets].replay()
+                else:
+                    dense(i)
             d1.record(stream)
             torch.cuda.synchronize()
             dms = d0.elapsed_time(d1) / nd
@@ -869,7 +987,7 @@ def run_conv(args, workload):
                        "parallelism": f"replicas x{world} (images independent)",
                        "l2": f"{nsets} rotating input/output sets of {per_set / 2**20:.0f} MiB "
                              "(> 2x L2)",
-                       "kernels": ["conv_forward[tcgen05]"]},
+                       "kernels": ["conv_forward[tcgen05]"], "timing": timing},
             "op_ms": [round(launch_ms, 5)],
             "roofline": roof,
             "cpu_baseline": cpu,
@@ -898,6 +1016,8 @@ def main():
                     default="p4_vitb_mlp_f16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense F.linear comparator")
+    ap.add_argument("--eager", action="store_true",
+                    help="time eager launches instead of replaying CUDA graphs of the step")
     ap.add_argument("--dp-path", action="store_true",
                     help="training workload: take the data-parallel weight-gradient path "
                          "(FP32 sums, reduction over ranks, one cast) even on one rank")

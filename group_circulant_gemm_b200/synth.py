@@ -50,6 +50,10 @@ WORKLOADS = {
     "p4_vitb_fc2_f16": Workload("p4_vitb_fc2_f16", 4, 12608, 768, 192, "f16", True, 1236),
     "p4_vith_fc1_f16": Workload("p4_vith_fc1_f16", 4, 8224, 320, 1280, "f16", True, 1237),
     "c8_1024_f16": Workload("c8_1024_f16", 8, 16384, 128, 128, "f16", True, 1238),
+    # the ViT-B MLP pair over the dihedral group D4 (8 elements): 768 -> 3072 -> 768
+    # features as 96 -> 384 -> 96 channels per group element
+    "p4m_vitb_fc1_f16": Workload("p4m_vitb_fc1_f16", 8, 12608, 96, 384, "f16", True, 1239),
+    "p4m_vitb_fc2_f16": Workload("p4m_vitb_fc2_f16", 8, 12608, 384, 96, "f16", True, 1239),
 }
 
 
