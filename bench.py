@@ -124,10 +124,11 @@ KERNEL_SOURCES = {
     "backward_weight": ("eql_tc_wgrad.cu", "eql_tc_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("forward", "5facc1d5cf0b65aa"): {"p4_vitb_mlp_2calls_f16": 58.89e6, "c8_1024_f16": 34.06e6,
-                                      "p4_vith_fc1_fwd_bwd_f16": 69.86e6},
-    ("forward_chain", "79e08cb6e9db3b65"): {"p4_vitb_mlp_f16": 81.76e6},
-    ("conv", "0fd00f0424229b1e"): {"p4_conv3x3_f16": 160.16e6},
+    ("forward", "bfd6f056114c3e22"): {"p4_vitb_mlp_2calls_f16": 58.98e6, "c8_1024_f16": 33.94e6,
+                                      "p4_vith_fc1_fwd_bwd_f16": 69.82e6,
+                                      "p4m_vitb_mlp_f16": 58.07e6},
+    ("forward_chain", "033fd47b5cd211f5"): {"p4_vitb_mlp_f16": 86.94e6},
+    ("conv", "c700b6d872d52cc5"): {"p4_conv3x3_f16": 160.33e6},
 }
 
 def kernel_traffic(family: str, workload: str):
