@@ -60,9 +60,11 @@ using namespace ftc;
 template <int T, int ACT, int IO, int G = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     eq_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x,
-                     const __grid_constant__ CUtensorMap map_y, const uint8_t* __restrict__ wtiles,
-                     const __half* __restrict__ bias, int64_t N, int Cin, int Cout, TileInfo ti,
-                     int* status) {
+                     const __grid_constant__ CUtensorMap map_y,
+                     const __grid_constant__ CUtensorMap map_x_half,
+                     const __grid_constant__ CUtensorMap map_y_half,
+                     const uint8_t* __restrict__ wtiles, const __half* __restrict__ bias,
+                     int64_t N, int Cin, int Cout, TileInfo ti, int* status) {
   using S = Shape<T>;
   constexpr int BD = S::BD;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -114,15 +116,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < depth; ++s) issued_phase[s] = -1;
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < ti.num_tiles; tile += gridDim.x) {
-        const int row0 = (tile / ti.n_dt) * BM;
-        const int dt = tile % ti.n_dt;
+      for (int u = blockIdx.x; ok && u < ti.num_units; u += gridDim.x) {
+        const UnitPos up = unit_pos(u, ti);
+        const int row0 = (int)up.row0;
+        const int dt = up.dt;
         for (int ks = 0; ks < ti.k_stages; ++ks, ++it) {
           const int s = it % depth;
           const uint32_t ph = (it / depth) & 1;
           if (!(ok = wait_bounded(&empty[s], ph ^ 1, abort_flag, status))) break;
           if (!is_raw && blockIdx.x == 0 && (int)it == ti.drop_w) continue;  // injected fault
           if (is_raw) {
+            if constexpr (IO == kIoSpatial && T == 4) {
+              if (up.half >= 0) {
+                // a 64-row half unit: the first 64 rows of the raw layout
+                mbar_expect_tx(&full[s], X_STAGE_BYTES / 2);
+                tma_load_3d(sbase + S::OFF_X + s * X_STAGE_BYTES, &map_x_half, &full[s], 0,
+                            2 * ks, row0);
+                issued_phase[s] = (int)ph;
+                continue;
+              }
+            }
             mbar_expect_tx(&full[s], X_STAGE_BYTES);
             if constexpr (IO == kIoSpectralIn) {
               // planes [4][N][Cin] of the previous layer: (32 channels, 128 rows, 4 planes)
@@ -156,10 +169,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      const uint32_t id_n1 = idesc_f16(BM, BD);
-      const uint32_t id_n1_neg = idesc_f16(BM, BD, true);
-      const uint32_t id_n2 = idesc_f16(BM, 2 * BD);
-      for (int tile = blockIdx.x; ok && tile < ti.num_tiles; tile += gridDim.x, ++tcount) {
+      for (int u = blockIdx.x; ok && u < ti.num_units; u += gridDim.x, ++tcount) {
+        // a half unit (T = 4 only) multiplies its 64 rows with M = 64 MMAs
+        int mrows = BM;
+        if constexpr (T == 4) mrows = unit_pos(u, ti).half >= 0 ? 64 : BM;
+        const uint32_t id_n1 = idesc_f16(mrows, BD);
+        const uint32_t id_n1_neg = idesc_f16(mrows, BD, true);
+        const uint32_t id_n2 = idesc_f16(mrows, 2 * BD);
         if (!(ok = wait_bounded(&bars->acc_empty, (tcount & 1) ^ 1, abort_flag, status))) break;
         tc_fence_after();
         for (int ks = 0; ks < ti.k_stages; ++ks, ++it) {
@@ -225,9 +241,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* stg = smem + S::OFF_STG + (warp - kEpiWarp0) * kStgBytes;
     __half* bsm = reinterpret_cast<__half*>(smem + S::OFF_BIAS + (warp - kEpiWarp0) * 128);
     uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < ti.num_tiles; tile += gridDim.x, ++tcount) {
-      const int64_t row0 = (int64_t)(tile / ti.n_dt) * BM + 32 * q;
-      const int dbase = (tile % ti.n_dt) * BD + (BD / 2) * ch;
+    for (int u = blockIdx.x; u < ti.num_units; u += gridDim.x, ++tcount) {
+      const UnitPos up = unit_pos(u, ti);
+      // M = 128: TMEM lane 32q + l holds row 32q + l; M = 64 (half unit, T = 4 only):
+      // lanes 32q .. 32q + 15 hold rows 16q .. 16q + 15
+      const bool half = T == 4 && up.half >= 0;
+      const int64_t row0 = up.row0 + (half ? 16 * q : 32 * q);
+      const int dbase = up.dt * BD + (BD / 2) * ch;
       // stage this warp's BD/2 biases while the mainloop runs (lane l: channels 2l, 2l+1)
       if (2 * lane < BD / 2) {
         const int d = dbase + 2 * lane;
@@ -239,8 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&bars->acc_full, tcount & 1, abort_flag, status)) break;
       tc_fence_after();
       const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-      epi_slices<T, BD, ACT, IO, StoreOf<T, IO>, G>(lane_addr, ch, lane, stg, bsm, dbase, Cout,
-                                                    StoreOf<T, IO>{&map_y, row0, N});
+      epi_slices<T, BD, ACT, IO, StoreOf<T, IO>, G>(
+          lane_addr, ch, lane, stg, bsm, dbase, Cout,
+          StoreOf<T, IO>{half ? &map_y_half : &map_y, row0, N});
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
     }
@@ -251,19 +272,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int xt = threadIdx.x - kXfWarp0 * 32;  // 0..255
     uint32_t it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < ti.num_tiles; tile += gridDim.x) {
+    for (int u = blockIdx.x; ok && u < ti.num_units; u += gridDim.x) {
+      // a half unit (T = 4 only) has rows 0..63: threads 128..255 (whole warps) idle
+      bool idle = false;
+      if constexpr (T == 4) idle = unit_pos(u, ti).half >= 0 && xt >= 128;
       for (int ks = 0; ks < ti.k_stages; ++ks, ++it) {
         const int sx = it % S::X_ST;
         if (!(ok = warp_wait(&bars->x_full[sx], (it / S::X_ST) & 1, abort_flag, status))) break;
         uint8_t* slot = smem + S::OFF_X + sx * X_STAGE_BYTES;
         uint4 v[8];
-        xf_read<T>(slot, xt, v);
+        if (!idle) xf_read<T>(slot, xt, v);
         // every raw piece of the slot is in registers before any plane overwrites it
         // (an mbarrier rather than a named barrier, so the wait stays bounded)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->x_read[sx]);
         if (!(ok = warp_wait(&bars->x_read[sx], (it / S::X_ST) & 1, abort_flag, status))) break;
-        xf_write<T, G>(slot, xt, v);
+        if (!idle) xf_write<T, G>(slot, xt, v);
         // make the generic-proxy stores visible to the tensor core (async proxy)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
@@ -436,7 +460,7 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
     constexpr int TT = decltype(tcst)::value;
     using S = Shape<TT>;
     cuuint32_t estr[3] = {1, 1, 1};
-    CUtensorMap mx;
+    CUtensorMap mx, mx_half, my_half;
     if (io == kIoSpectralIn) {
       // planes of the previous layer: box = 32 channels (64 B) x 128 rows x 4 planes
       if (!encode_planes_map(&mx, const_cast<void*>(X), Cin, N, S::BK, BM,
@@ -449,6 +473,13 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
       cuuint32_t box[3] = {64, 2, BM};
       if (encode(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(X), dims, strides,
                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+      // half units: 64 rows
+      cuuint32_t hbox[3] = {64, 2, 64};
+      if (encode(&mx_half, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(X), dims,
+                 strides, hbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
@@ -468,6 +499,17 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+      // half units: an epilogue warp stores 16 rows
+      cuuint32_t yhbox[3] = {64, 1, 16};
+      if (encode(&my_half, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, Y, ydims, ystrides, yhbox, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+    if (io != kIoSpatial) {  // no half units with spectral input or output
+      mx_half = mx;
+      my_half = my;
     }
     TileInfo ti;
     ti.n_dt = (Cout + S::BD - 1) / S::BD;
@@ -476,6 +518,18 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
     ti.num_tiles = (int)(n_rt * ti.n_dt);
     ti.k_stages = (Cin + S::BK - 1) / S::BK;
     ti.drop_w = drop_w_stage;
+    // The last partial wave (rem tiles) runs as 2 * rem half units when that still
+    // fits in one wave: a half unit moves about 0.6 of a tile's shared-memory
+    // traffic (its MMAs cost as much as a whole tile's), so the wave ends sooner.
+    ti.full = ti.num_tiles;
+    ti.num_units = ti.num_tiles;
+    if (io == kIoSpatial && TT == 4) {  // T = 8 tiles keep their registers for the transform
+      const int rem = ti.num_tiles >= num_sms ? ti.num_tiles % num_sms : ti.num_tiles;
+      if (rem > 0 && 2 * rem <= num_sms) {
+        ti.full = ti.num_tiles - rem;
+        ti.num_units = ti.full + 2 * rem;
+      }
+    }
     static bool attr_set = false;
     if (!attr_set) {
       cudaError_t e = set_smem_attr<TT, 0, kIoSpatial>();
@@ -492,7 +546,7 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
       if (e != cudaSuccess) return e;
       attr_set = true;
     }
-    const int grid = ti.num_tiles < num_sms ? ti.num_tiles : num_sms;
+    const int grid = ti.num_units < num_sms ? ti.num_units : num_sms;
     auto kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1, kIoSpatial> : eq_fwd_tc_kernel<TT, 0, kIoSpatial>;
     if constexpr (TT == 4) {
       if (io == kIoSpectralOut)
@@ -507,8 +561,8 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           : eq_fwd_tc_kernel<TT, 0, kIoSpatial, 1>;
     }
     kernel<<<grid, kThreads, S::SMEM_BYTES, st>>>(
-        mx, my, static_cast<const uint8_t*>(Wtiles), static_cast<const __half*>(bias), N, Cin,
-        Cout, ti, status);
+        mx, my, mx_half, my_half, static_cast<const uint8_t*>(Wtiles),
+        static_cast<const __half*>(bias), N, Cin, Cout, ti, status);
     return cudaGetLastError();
   });
 }

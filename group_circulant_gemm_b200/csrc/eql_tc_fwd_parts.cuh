@@ -88,7 +88,35 @@ struct TileInfo {
   int num_tiles;  // row tiles x d tiles
   int k_stages;   // ceil(Cin / BK)
   int drop_w;     // fault injection for tests: CTA 0 never issues weight stage drop_w (-1: off)
+  // Work units: [0, full) are whole tiles; the remaining tiles (the last partial
+  // wave) are split into two 64-row halves each, so that wave spreads over twice
+  // as many SMs: num_units = full + 2 * (num_tiles - full).
+  int full;
+  int num_units;
 };
+
+// Position of work unit u: first row, out-channel tile, and which half
+// (-1: the whole 128-row tile; 0, 1: rows 0-63, 64-127, computed with M = 64 MMAs).
+struct UnitPos {
+  int64_t row0;
+  int dt, half;
+};
+__device__ __forceinline__ UnitPos unit_pos(int u, const TileInfo& ti) {
+  int tile, half;
+  if (u < ti.full) {
+    tile = u;
+    half = -1;
+  } else {
+    const int h = u - ti.full;
+    tile = ti.full + (h >> 1);
+    half = h & 1;
+  }
+  UnitPos p;
+  p.dt = tile % ti.n_dt;
+  p.half = half;
+  p.row0 = (int64_t)(tile / ti.n_dt) * BM + (half > 0 ? 64 : 0);
+  return p;
+}
 
 // ---------------------------------------------------------------------------
 // Transform: the raw stage is [row][128-byte chunk c][128 B], every 128-byte

@@ -407,3 +407,24 @@ def test_spectral_entry_points_reject_unsupported_plans():
     s = n.raw_status("eqlinear_forward_to_spectral", p.handle, X.data_ptr(), 16, Wh.data_ptr(),
                      None, 0, Xh.data_ptr(), None)
     assert s == 2  # EQL_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("N,C,D", [(151 * 128 - 51, 64, 128), (150 * 128, 32, 256), (300, 64, 128)])
+def test_last_wave_half_units_match_oracle(N, C, D):
+    """Tiles of the last partial wave run as two 64-row halves (M = 64 MMAs): every row
+    of the split tiles, and a sample of whole-tile rows, against the oracle."""
+    w = Workload("halves", 4, N, C, D, "f16", True, 700 + N)
+    inp = make_inputs(w)
+    p = _plan(w, "tcgen05")
+    Wh = p.prepare_weights(_dev(inp["W"]))
+    Y = p.forward(_dev(inp["X"]), Wh, _dev(inp["bias"])).double().cpu().numpy()
+    assert p.status() == 0
+    n_dt = (D + 127) // 128
+    tiles = ((N + 127) // 128) * n_dt
+    rem = tiles % 148 if tiles >= 148 else tiles
+    first_split_row = ((tiles - rem) // n_dt) * 128
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([np.arange(first_split_row, N),
+                                     rng.integers(0, max(first_split_row, 1), 64)]))
+    ref = oracle.forward(4, inp["X"][rows], inp["W"], inp["bias"])
+    assert _rel(Y[rows], ref) <= TOL["f16"]
