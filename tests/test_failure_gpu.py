@@ -43,3 +43,34 @@ def test_dropped_weight_stage_times_out_and_context_survives():
     ref = oracle.forward(4, inp["X"], inp["W"], inp["bias"])
     rel = np.max(np.abs(Y.double().cpu().numpy() - ref)) / np.max(np.abs(ref))
     assert rel <= 2e-3
+
+
+def test_chained_launch_row_wait_times_out_and_recovers():
+    """The chained two-layer launch waits (bounded) for the layer-1 tiles of a row
+    before a layer-2 tile reads them.  Starting the task counter past the first
+    layer-1 tile (a workspace the host planted) leaves row 0's layer-2 tile waiting
+    for a tile nobody computes: the wait gives up after ~2 s, the status word
+    reports EQL_ERR_TIMEOUT, the kernel's last CTA still clears the counters, and
+    the next call with the same workspace is correct."""
+    from group_circulant_gemm_b200 import EqLinearPlan, forward_chain
+    from group_circulant_gemm_b200 import native as n
+    N, C0, C1, C2 = 20 * 128, 64, 128, 64
+    w1 = Workload("chf1", 4, N, C0, C1, "f16", True, 51)
+    w2 = Workload("chf2", 4, N, C1, C2, "f16", True, 52)
+    in1, in2 = make_inputs(w1), make_inputs(w2, rows=1)
+    p1 = EqLinearPlan(4, C0, C1, torch.float16)
+    p2 = EqLinearPlan(4, C1, C2, torch.float16)
+    wh1 = p1.prepare_weights(torch.from_numpy(in1["W"]).cuda())
+    wh2 = p2.prepare_weights(torch.from_numpy(in2["W"]).cuda())
+    X = torch.from_numpy(in1["X"]).cuda()
+    b1, b2 = torch.from_numpy(in1["bias"]).cuda(), torch.from_numpy(in2["bias"]).cuda()
+    ws = torch.zeros(n.eqlinear_chain_workspace_bytes(p1.handle, p2.handle, N),
+                     dtype=torch.uint8, device="cuda")
+    ws.view(torch.int32)[0] = 1  # skip task 0: the layer-1 tile of row 0
+    forward_chain(p1, p2, X, wh1, b1, wh2, b2, workspace=ws)
+    assert p1.status() == n.EQL_ERR_TIMEOUT
+    assert int(ws.view(torch.int32).abs().sum().item()) == 0
+    H, Y = forward_chain(p1, p2, X, wh1, b1, wh2, b2, workspace=ws)
+    assert p1.status() == n.EQL_OK
+    Y_ref = p2.forward(p1.forward(X, wh1, b1), wh2, b2)
+    assert torch.equal(Y.view(torch.int16), Y_ref.view(torch.int16))
