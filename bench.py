@@ -471,6 +471,11 @@ def run_ours(args, workload):
     per_set = sum(N * w.C * w.T * es + N * w.D * w.T * es for w in pipeline)
     if backward:
         per_set += sum(N * w.D * w.T * es + N * w.C * w.T * es for w in pipeline)
+    # training: the forward and dX kernels save the group spectra of X and dY
+    # (the same sizes) for the weight gradient, unless --wgrad-transform
+    saved = backward and not args.wgrad_transform
+    if saved:
+        per_set += sum(N * w.C * w.T * es + N * w.D * w.T * es for w in pipeline[:1])
     nsets = max(2, int(np.ceil(2 * L2_BYTES / per_set)))
     xs = [torch.from_numpy(x_host).cuda() for _ in range(nsets)]
     outs = [[torch.empty((N, w.D * w.T), dtype=dt, device="cuda") for w in pipeline]
@@ -486,6 +491,9 @@ def run_ours(args, workload):
         dW, db = plans[0].split_grad(gbuf)
         gbuf32 = plans[0].grad_buffer(torch.float32) if dp else None
         ws = torch.empty(max(16, plans[0].workspace_bytes(N)), dtype=torch.uint8, device="cuda")
+        if saved:
+            xhats = [torch.empty((4, N, w0.C), dtype=dt, device="cuda") for _ in range(nsets)]
+            ghats = [torch.empty((4, N, w0.D), dtype=dt, device="cuda") for _ in range(nsets)]
 
     # the ops of one step: (label, kernel, flops, algorithmic bytes, callable(set index))
     ops = []
@@ -516,27 +524,42 @@ def run_ours(args, workload):
             elif spectral and li == 1:
                 plans[li].forward_from_spectral(x, whats[li], biases[li], act=acts[li],
                                                 out=outs[i % nsets][li])
+            elif saved and li == 0:
+                plans[li].forward_save_spectrum(x, whats[li], biases[li], act=acts[li],
+                                                out=outs[i % nsets][li], Xhat=xhats[i % nsets])
             else:
                 plans[li].forward(x, whats[li], biases[li], out=outs[i % nsets][li],
                                   act=acts[li])
-        ops.append(("forward", plans[li].forward_kernel_name(N), layer_flops(w), layer_bytes(w),
-                    fwd))
+        # a saved spectrum is one more write of X's size
+        extra = es * w.N * w.C * w.T if saved and li == 0 else 0
+        ops.append(("forward", plans[li].forward_kernel_name(N), layer_flops(w),
+                    layer_bytes(w) + extra, fwd))
     if backward:
         w0 = pipeline[0]
         pending = []
 
         def bwd_x(i):
-            plans[0].backward_input(dys[i % nsets], whats[0], out=dxs[i % nsets])
+            if saved:
+                plans[0].backward_input_save_spectrum(dys[i % nsets], whats[0],
+                                                      out=dxs[i % nsets], dYhat=ghats[i % nsets])
+            else:
+                plans[0].backward_input(dys[i % nsets], whats[0], out=dxs[i % nsets])
 
         def bwd_w(i):
+            # the weight gradient reads the spectra (or X and dY: the same bytes)
+            a = xhats[i % nsets] if saved else xs[i % nsets]
+            g = ghats[i % nsets] if saved else dys[i % nsets]
             if dp:
-                plans[0].backward_weight_f32(xs[i % nsets], dys[i % nsets], buf=gbuf32,
-                                             workspace=ws)
+                if saved:
+                    plans[0].backward_weight_from_spectra_f32(a, g, buf=gbuf32, workspace=ws)
+                else:
+                    plans[0].backward_weight_f32(a, g, buf=gbuf32, workspace=ws)
                 # queued behind dW; dX runs on the compute stream meanwhile
                 pending.append(allreduce_grad_buffer(gbuf32, async_op=True))
+            elif saved:
+                plans[0].backward_weight_from_spectra(a, g, dW=dW, dbias=db, workspace=ws)
             else:
-                plans[0].backward_weight(xs[i % nsets], dys[i % nsets], dW=dW, dbias=db,
-                                         workspace=ws)
+                plans[0].backward_weight(a, g, dW=dW, dbias=db, workspace=ws)
 
         def grad_sync(i):
             handle = pending.pop()
@@ -545,12 +568,16 @@ def run_ours(args, workload):
             plans[0].cast_from_f32(gbuf32, out=gbuf)
         nb = es * (N * w0.C * w0.T + N * w0.D * w0.T)
         op_dx = ("backward_input", plans[0].forward_kernel_name(N), layer_flops(w0),
-                 nb + es * 1.25 * w0.C * w0.D * w0.T, bwd_x)
+                 nb + es * 1.25 * w0.C * w0.D * w0.T + (es * N * w0.D * w0.T if saved else 0),
+                 bwd_x)
         op_dw = ("backward_weight", plans[0].backward_weight_kernel_name(N), wgrad_flops(w0),
                  nb + es * w0.D * w0.C * w0.T, bwd_w)
         if dp:
-            ops += [op_dw, op_dx, ("weight_grad_allreduce", "nccl+cast", 0.0,
-                                   (4 + es) * gbuf.numel(), grad_sync)]
+            # dW from saved spectra needs dX's saved dY spectrum, so it follows dX;
+            # the transforming dW goes first and its all-reduce overlaps dX
+            first_two = [op_dx, op_dw] if saved else [op_dw, op_dx]
+            ops += first_two + [("weight_grad_allreduce", "nccl+cast", 0.0,
+                                 (4 + es) * gbuf.numel(), grad_sync)]
         else:
             ops += [op_dx, op_dw]
 
@@ -1019,6 +1046,9 @@ def main():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense F.linear comparator")
     ap.add_argument("--eager", action="store_true",
                     help="time eager launches instead of replaying CUDA graphs of the step")
+    ap.add_argument("--wgrad-transform", action="store_true",
+                    help="training workload: the weight gradient transforms X and dY itself "
+                         "instead of reading the spectra the forward and dX kernels saved")
     ap.add_argument("--dp-path", action="store_true",
                     help="training workload: take the data-parallel weight-gradient path "
                          "(FP32 sums, reduction over ranks, one cast) even on one rank")

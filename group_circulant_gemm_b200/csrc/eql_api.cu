@@ -421,6 +421,46 @@ eqlinear_status_t eqlinear_conv_forward(eqlinear_plan_t p, const void* X, int64_
                                        (cudaStream_t)stream));
 }
 
+// The forward-shaped product (Cin -> Cout) with the input's group spectrum
+// also written to `spectrum` [4][N][Cin]: tensor cores only (T = 4, FP16).
+static eqlinear_status_t save_spectrum_io(eqlinear_plan_t p, const void* X, int64_t N, int Cin,
+                                          int Cout, const void* tiles, const void* bias,
+                                          eqlinear_act_t act, void* Y, void* spectrum,
+                                          void* stream) {
+  if (!p || N < 0) return EQL_ERR_INVALID_ARG;
+  if (act != EQL_ACT_NONE && act != EQL_ACT_GELU) return EQL_ERR_INVALID_ARG;
+  if (!(p->T == 4 && p->group == 0 && p->dtype == EQL_F16 && p->kernel != EQL_KERNEL_SIMT &&
+        has_tiles(p)))
+    return EQL_ERR_UNSUPPORTED;
+  if (N == 0) return EQL_OK;
+  if (!X || !tiles || !Y || !spectrum) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(tiles) || !aligned16(Y) || !aligned16(spectrum) ||
+      (bias && !aligned16(bias)))
+    return EQL_ERR_ALIGNMENT;
+  if (!eql::fwd_tc_supported(4, eql::DType::F16, N, Cin, Cout)) return EQL_ERR_UNSUPPORTED;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_fwd_tc(4, X, N, Cin, Cout, tiles, bias, Y, p->status, p->num_sms,
+                                      p->debug_drop_w_stage, (int)act, 3, (cudaStream_t)stream,
+                                      0, spectrum));
+}
+
+eqlinear_status_t eqlinear_forward_save_spectrum(eqlinear_plan_t p, const void* X, int64_t N,
+                                                 const void* W_hat, const void* bias,
+                                                 eqlinear_act_t act, void* Y, void* Xhat,
+                                                 void* stream) {
+  if (!p || !W_hat) return EQL_ERR_INVALID_ARG;
+  return save_spectrum_io(p, X, N, p->C, p->D, fwd_tiles(p, W_hat), bias, act, Y, Xhat, stream);
+}
+
+eqlinear_status_t eqlinear_backward_input_save_spectrum(eqlinear_plan_t p, const void* dY,
+                                                        int64_t N, const void* W_hat, void* dX,
+                                                        void* dYhat, void* stream) {
+  if (!p || !W_hat) return EQL_ERR_INVALID_ARG;
+  return save_spectrum_io(p, dY, N, p->D, p->C, adj_tiles(p, W_hat), nullptr, EQL_ACT_NONE, dX,
+                          dYhat, stream);
+}
+
 eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int64_t N,
                                           const void* W_hat, void* dX, void* stream) {
   if (!p || N < 0) return EQL_ERR_INVALID_ARG;
@@ -446,23 +486,34 @@ size_t eqlinear_backward_weight_workspace_bytes(eqlinear_plan_t p, int64_t N) {
   return need;
 }
 
+// spectra = true: X and dY are the group spectra [4][N][C] and [4][N][D] that
+// the save-spectrum calls wrote (tensor cores only; C and D multiples of 64).
 static eqlinear_status_t backward_weight_impl(eqlinear_plan_t p, const void* X, const void* dY,
                                               int64_t N, void* dW, void* dbias, void* workspace,
                                               size_t workspace_bytes, eql::DType out_dt,
-                                              void* stream) {
+                                              void* stream, bool spectra = false) {
   if (!p || N < 0 || !dW) return EQL_ERR_INVALID_ARG;
   if (p->group == 1) return EQL_ERR_UNSUPPORTED;
   if (N > 0 && (!X || !dY)) return EQL_ERR_INVALID_ARG;
   if ((X && !aligned16(X)) || (dY && !aligned16(dY)) || !aligned16(dW) ||
       (dbias && !aligned16(dbias)) || (workspace && !aligned16(workspace)))
     return EQL_ERR_ALIGNMENT;
-  if (p->kernel == EQL_KERNEL_TCGEN05 && !wgrad_tc_ok(p, N, X, dY)) return EQL_ERR_UNSUPPORTED;
+  if (spectra && !(p->T == 4 && p->dtype == EQL_F16 && p->kernel != EQL_KERNEL_SIMT &&
+                   p->C % 64 == 0 && p->D % 64 == 0))
+    return EQL_ERR_UNSUPPORTED;
+  if (!spectra && p->kernel == EQL_KERNEL_TCGEN05 && !wgrad_tc_ok(p, N, X, dY))
+    return EQL_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < eqlinear_backward_weight_workspace_bytes(p, N))
     return EQL_ERR_WORKSPACE;
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  if (wgrad_use_tc(p, N, X, dY))
+  if (spectra && N > 0) {
+    if (!eql::wgrad_tc_planes_supported(N, p->C, p->D, X, dY)) return EQL_ERR_UNSUPPORTED;
+    return from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, workspace, out_dt, dW, dbias,
+                                          p->status, p->num_sms, p->tw, st, true));
+  }
+  if (!spectra && wgrad_use_tc(p, N, X, dY))
     return from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, workspace, out_dt, dW, dbias,
                                           p->status, p->num_sms, p->tw, st));
   const int splits = eql::wgrad_simt_splits(p->T, N, p->C, p->D, p->num_sms);
@@ -485,6 +536,24 @@ eqlinear_status_t eqlinear_backward_weight_f32(eqlinear_plan_t p, const void* X,
                                                void* stream) {
   return backward_weight_impl(p, X, dY, N, dW, dbias, workspace, workspace_bytes,
                               eql::DType::F32, stream);
+}
+
+eqlinear_status_t eqlinear_backward_weight_from_spectra(eqlinear_plan_t p, const void* Xhat,
+                                                        const void* dYhat, int64_t N, void* dW,
+                                                        void* dbias, void* workspace,
+                                                        size_t workspace_bytes, void* stream) {
+  if (!p) return EQL_ERR_INVALID_ARG;
+  return backward_weight_impl(p, Xhat, dYhat, N, dW, dbias, workspace, workspace_bytes,
+                              to_dt(p->dtype), stream, true);
+}
+
+eqlinear_status_t eqlinear_backward_weight_from_spectra_f32(eqlinear_plan_t p, const void* Xhat,
+                                                            const void* dYhat, int64_t N,
+                                                            float* dW, float* dbias,
+                                                            void* workspace,
+                                                            size_t workspace_bytes, void* stream) {
+  return backward_weight_impl(p, Xhat, dYhat, N, dW, dbias, workspace, workspace_bytes,
+                              eql::DType::F32, stream, true);
 }
 
 eqlinear_status_t eqlinear_cast_from_f32(eqlinear_plan_t p, const float* src, int64_t count,

@@ -58,11 +58,13 @@ bool fwd_tc_supported(int T, DType dt, int64_t N, int Cin, int Cout);
 // so its bounded waits expire and the kernel reports a timeout.
 // io (T = 4 only beyond 0): 0 = spatial X and Y; 1 = Y written as the next
 // layer's spectral planes [4][N][Cout] (the group DFT of act(y): X0, X2, Xr, Xi);
-// 2 = X read as spectral planes [4][N][Cin] produced that way.
+// 2 = X read as spectral planes [4][N][Cin] produced that way; 3 = spatial X
+// and Y, and X's group spectrum written to `spectrum` [4][N][Cin] (FP16, the
+// same planes order), which must be non-null exactly for io = 3.
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
                           int num_sms, int drop_w_stage, int act, int io, cudaStream_t st,
-                          int group = 0);
+                          int group = 0, void* spectrum = nullptr);
 
 // tcgen05/TMEM tensor-core weight gradient for T = 4, FP16: stream-K over
 // (tile, 32-row stage) ranges, FP32 partial slots in `workspace`, then a
@@ -71,9 +73,14 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
 // handled by the caller.
 bool wgrad_tc_supported(int T, DType dt, int64_t N, int C, int D, const void* X, const void* dY);
 size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms);
+// planes = true: X and dY are instead their group spectra as FP16 planes
+// [4][N][C] and [4][N][D] (as the forward and dX kernels save them); needs
+// C % 64 == 0 and D % 64 == 0 (wgrad_tc_planes_supported).
+bool wgrad_tc_planes_supported(int64_t N, int C, int D, const void* Xhat, const void* Ghat);
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
                             void* workspace, DType out_dt, void* dW, void* dbias, int* status,
-                            int num_sms, const Twiddles& tw, cudaStream_t st);
+                            int num_sms, const Twiddles& tw, cudaStream_t st,
+                            bool planes = false);
 
 // Two chained T = 4 FP16 layers (C0 -> C1 -> C2) in one persistent launch with a
 // dynamic tile queue: H = act1(L1(X)) (spatial [N][C1*4], or spectral planes

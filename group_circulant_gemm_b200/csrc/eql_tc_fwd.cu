@@ -18,7 +18,10 @@
 // Template parameters: ACT = output activation (0 none, 1 GELU, fused into the
 // epilogue); IO (T = 4) = spatial X and Y, or Y written as the next layer's
 // spectral operand planes [4][N][Cout], or X read as such planes (then the TMA
-// box lands directly as the operand planes and the transform warps are idle).
+// box lands directly as the operand planes and the transform warps are idle),
+// or spatial X and Y with X's spectrum saved: warp 3 stores transformed stages
+// (one TMA box of 32 channels x 128 rows x 4 planes each; stage ks by the
+// out-channel tile ks % n_dt) before their slots are released.
 //
 // Design (one persistent CTA per SM; tile = 128 rows x BD out-channels; K stage
 // = BK input channels, whose raw X tile is always 128 rows x 256 B = 32 KB):
@@ -63,6 +66,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap map_y,
                      const __grid_constant__ CUtensorMap map_x_half,
                      const __grid_constant__ CUtensorMap map_y_half,
+                     const __grid_constant__ CUtensorMap map_p,
                      const uint8_t* __restrict__ wtiles, const __half* __restrict__ bias,
                      int64_t N, int Cin, int Cout, TileInfo ti, int* status) {
   using S = Shape<T>;
@@ -81,7 +85,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->x_full[s], 1);          // raw tile landed (TMA bytes)
       mbar_init(&bars->x_read[s], kXfWarps);   // every transform warp holds its raw pieces
       mbar_init(&bars->x_ready[s], kXfWarps);  // operand planes written (transform warps)
-      mbar_init(&bars->x_empty[s], 1);         // MMAs done with the planes (tcgen05.commit)
+      // MMAs done with the planes (tcgen05.commit), and with a saved spectrum its
+      // store has read them
+      mbar_init(&bars->x_empty[s], IO == kIoSaveSpectrum ? 2 : 1);
     }
     for (int s = 0; s < S::W_ST; ++s) {
       mbar_init(&bars->w_full[s], 1);
@@ -267,6 +273,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
+  } else if (IO == kIoSaveSpectrum && warp == 3) {
+    // ---------------- spectrum store ----------------
+    // Every out-channel tile of a row tile transforms the same X stages; stage ks
+    // is stored by tile ks % n_dt, so each tile stores an equal share.  A stored
+    // slot is released once the store has read it, checked one stage later
+    // (wait_group.read 1) so the store overlaps the next stage.
+    if (lane == 0) {
+      uint32_t it = 0;
+      int pending = -1;  // slot whose store may still be reading it
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < ti.num_units; u += gridDim.x) {
+        const UnitPos up = unit_pos(u, ti);
+        for (int ks = 0; ks < ti.k_stages; ++ks, ++it) {
+          const int sx = it % S::X_ST;
+          if (!(ok = wait_bounded(&bars->x_ready[sx], (it / S::X_ST) & 1, abort_flag, status)))
+            break;
+          if (ks % ti.n_dt == up.dt) {
+            // the transform warps fenced their plane stores to the async proxy before
+            // arriving on x_ready; rows past N and channels past Cin are clipped
+            tma_store_3d(&map_p, sbase + S::OFF_X + sx * X_STAGE_BYTES, S::BK * ks,
+                         (int)up.row0, 0);
+            bulk_commit();
+            if (pending >= 0) {
+              bulk_wait_read_1();
+              mbar_arrive(&bars->x_empty[pending]);
+            }
+            pending = sx;
+          } else {
+            if (pending >= 0) {
+              bulk_wait_read_all();
+              mbar_arrive(&bars->x_empty[pending]);
+              pending = -1;
+            }
+            mbar_arrive(&bars->x_empty[sx]);
+          }
+        }
+      }
+      bulk_wait_all();
+      if (pending >= 0) mbar_arrive(&bars->x_empty[pending]);
+    }
+    __syncwarp();
   } else if (warp >= kXfWarp0 && IO != kIoSpectralIn) {
     // ---------------- transform: group DFT into the operand planes ----------------
     const int xt = threadIdx.x - kXfWarp0 * 32;  // 0..255
@@ -447,10 +494,11 @@ cudaError_t launch_prepare_d4(const void* W, int C, int D, void* planes, cudaStr
 cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           const void* Wtiles, const void* bias, void* Y, int* status,
                           int num_sms, int drop_w_stage, int act, int io, cudaStream_t st,
-                          int group) {
+                          int group, void* spectrum) {
   if (!fwd_tc_supported(T, DType::F16, N, Cin, Cout)) return cudaErrorNotSupported;
   if (!Wtiles) return cudaErrorNotSupported;
   if (io != kIoSpatial && T != 4) return cudaErrorNotSupported;
+  if ((io == kIoSaveSpectrum) != (spectrum != nullptr)) return cudaErrorInvalidValue;
   if (group != 0 && (T != 8 || io != kIoSpatial)) return cudaErrorNotSupported;
   if (act != 0 && act != 1) return cudaErrorInvalidValue;
 
@@ -507,6 +555,12 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     }
+    CUtensorMap mp = mx;
+    if (io == kIoSaveSpectrum) {
+      // the input's spectrum: store box = 32 channels (64 B) x 128 rows x 4 planes
+      if (!encode_planes_map(&mp, spectrum, Cin, N, S::BK, BM, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    }
     if (io != kIoSpatial) {  // no half units with spectral input or output
       mx_half = mx;
       my_half = my;
@@ -539,6 +593,8 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
         if (e == cudaSuccess) e = set_smem_attr<TT, 1, kIoSpectralOut>();
         if (e == cudaSuccess) e = set_smem_attr<TT, 0, kIoSpectralIn>();
         if (e == cudaSuccess) e = set_smem_attr<TT, 1, kIoSpectralIn>();
+        if (e == cudaSuccess) e = set_smem_attr<TT, 0, kIoSaveSpectrum>();
+        if (e == cudaSuccess) e = set_smem_attr<TT, 1, kIoSaveSpectrum>();
       } else {
         if (e == cudaSuccess) e = set_smem_attr<TT, 0, kIoSpatial, 1>();
         if (e == cudaSuccess) e = set_smem_attr<TT, 1, kIoSpatial, 1>();
@@ -555,13 +611,16 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
       else if (io == kIoSpectralIn)
         kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1, kIoSpectralIn>
                           : eq_fwd_tc_kernel<TT, 0, kIoSpectralIn>;
+      else if (io == kIoSaveSpectrum)
+        kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1, kIoSaveSpectrum>
+                          : eq_fwd_tc_kernel<TT, 0, kIoSaveSpectrum>;
     } else {
       if (group == 1)
         kernel = act == 1 ? eq_fwd_tc_kernel<TT, 1, kIoSpatial, 1>
                           : eq_fwd_tc_kernel<TT, 0, kIoSpatial, 1>;
     }
     kernel<<<grid, kThreads, S::SMEM_BYTES, st>>>(
-        mx, my, mx_half, my_half, static_cast<const uint8_t*>(Wtiles),
+        mx, my, mx_half, my_half, mp, static_cast<const uint8_t*>(Wtiles),
         static_cast<const __half*>(bias), N, Cin, Cout, ti, status);
     return cudaGetLastError();
   });

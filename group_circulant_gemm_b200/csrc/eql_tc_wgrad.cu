@@ -14,10 +14,15 @@
 //
 // Work split (stream-K over rows): the (tile, 32-row stage) space, tile = 128
 // out-channels x 128 in-channels, is cut into equal contiguous ranges, one per
-// CTA, so every SM does the same number of stages.  A range can end one tile
-// and start the next; each piece (a "segment") accumulates in TMEM and writes
-// its own partial slot part[tile][j][4][128 c][128 d] (j = which of the tile's
-// ranges; out-channel fastest, so each warp store writes 128 contiguous bytes).
+// CTA, so every SM does the same number of stages.  The space is ordered row
+// block by row block (block = as many stages as a range, the last block
+// shorter), then tile, then stage: the CTAs that run at the same time then
+// read the same rows, so each row of X (read once per out-channel tile) and of
+// dY (once per in-channel tile) comes from DRAM about once and from L2 after.
+// A range can end one (block, tile) pair and start the next; each piece (a
+// "segment") accumulates in TMEM and writes its own partial slot
+// part[pair][j][4][128 c][128 d] (j = which of the pair's ranges; out-channel
+// fastest, so each warp store writes 128 contiguous bytes).
 //
 // Design (one CTA per SM; stage = 32 rows):
 //   warp 0      TMA producer: per stage one 3-D box of dY (32 rows x 1 KB: the
@@ -37,6 +42,19 @@
 // TMEM (512 columns): Q0 at [0,128), Q2 at [128,256), Qr at [256,384), Qi at
 // [384,512).  Every mbarrier wait is bounded (about 2 s); on expiry the CTA sets
 // the plan's status word, drains what it issued and returns.
+//
+// Planes variant (PL): the group DFTs of X and dY arrive precomputed as FP16
+// planes [4][N][C] and [4][N][D] (written by the forward and dX kernels while
+// they transform the same tensors), so no transform runs here.  A ring slot is
+// 16 rows: one 4-D TMA box per operand, (64 channels, 16 rows, 2 blocks of 64
+// channels, 4 planes), 128-byte swizzled, landing as [plane][block][16 rows]
+// [128 B]: the rows are the MMA's K dimension and the channels are contiguous,
+// i.e. MN-major operands (64-channel blocks 2 KB apart, 8-row groups 1 KB
+// apart, so the N = 256 [Xr | Xi] operand spans planes 2 and 3 at a uniform
+// stride).  Warps 8-11 sum plane 0 of dY's spectrum for dbias; warps 4-7 and
+// 12-15 drain planes 0-1 and 2-3 of the accumulators.  Needs C and D
+// multiples of 64.
+
 #include <algorithm>
 
 #include "eql_kernels.h"
@@ -58,13 +76,39 @@ constexpr uint32_t WG_PLANE = 128 * WG_ROWB; // one operand plane (128 channels)
 constexpr uint32_t WG_OFF_BAR = WG_ST * WG_STAGE;
 constexpr uint32_t WG_SMEM = WG_OFF_BAR + 512 + 1024;
 constexpr int WG_THREADS = 768;
+// Planes variant: no transform warps; warps 8..11 sum dbias, warps 4..7 and
+// 12..15 drain the accumulators.  Its ring holds 6 slots of 16 rows (one MMA K
+// step, 32 KB) in the same 192 KB, so more bytes stay in flight.
+constexpr int WG_THREADS_PL = 512;
+constexpr int WG_BIASW = 4;
+constexpr int PL_SUB = 1;                         // slots per 32-row stage
+constexpr int PL_ST = 3;                          // ring depth
+constexpr int PL_ROWS = WG_BR / PL_SUB;           // 16 rows per slot
+constexpr uint32_t PL_BLOCK = PL_ROWS * 128;      // 64 channels x 16 rows (the LBO)
+constexpr uint32_t PL_PLANE = 2 * PL_BLOCK;       // 128 channels
+constexpr uint32_t PL_TILE = 4 * PL_PLANE;        // one operand's 4 planes
+constexpr uint32_t PL_SLOT = 2 * PL_TILE;         // dY spectrum, then X spectrum
+constexpr int WG_RING_MAX = PL_ST;
 constexpr int WG_EPI0 = 4, WG_EPIW = 4;      // warps 4..7: one per TMEM lane quarter
 constexpr int WG_XF0 = 8, WG_XFW = 8;        // warps 8..15 (dY tile), 16..23 (X tile)
 static_assert(4 * WG_PLANE == WG_TILE, "planes replace the raw tile in place");
+static_assert(PL_ST * PL_SLOT == WG_ST * WG_STAGE, "both rings fill the same bytes");
 static_assert(WG_SMEM <= 232448, "shared memory budget");
 
+// MN-major operand of a planes slot: 64-channel blocks `lbo` bytes apart, 8-row
+// K groups 1 KB apart (SBO), 128-byte swizzle (layout type 2), descriptor v1.
+__device__ __forceinline__ uint64_t desc_mn128(uint32_t saddr, uint32_t lbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(lbo >> 4) << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// kind::f16 instruction descriptor with both operands MN-major (bits 15, 16).
+__host__ __device__ constexpr uint32_t idesc_f16_mn(int M, int N, bool negate_a = false) {
+  return idesc_f16(M, N, negate_a) | (1u << 15) | (1u << 16);
+}
+
 struct WgBars {
-  uint64_t full[WG_ST], read_g[WG_ST], read_x[WG_ST], ready[WG_ST], empty[WG_ST];
+  uint64_t full[WG_RING_MAX], read_g[WG_RING_MAX], read_x[WG_RING_MAX], ready[WG_RING_MAX],
+      empty[WG_RING_MAX];
   uint64_t acc_full, acc_empty, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -74,20 +118,33 @@ static_assert(sizeof(WgBars) <= 512, "barrier block");
 struct WgInfo {
   int n_dt, n_ct;      // out-channel and in-channel tiles
   int spt;             // 32-row stages per tile, ceil(N / 32)
+  int bst;             // stages per row block (the last block: spt - (nb - 1) * bst)
+  int nb;              // row blocks
   int per_unit;        // stages per CTA range
-  int maxj;            // partial slots per tile
+  int maxj;            // partial slots per (block, tile) pair
   int64_t total;       // tiles * spt
 };
 
 // One segment of a CTA's range: stages [r0 / 32, r0 / 32 + stages) of one tile.
 struct Unit {
-  int dt, ct, tile, slot;  // slot = tile * maxj + (range index within the tile)
+  int dt, ct, tile, slot;  // slot = pair * maxj + (range index within the pair)
   int64_t r0;
   int stages;
 };
 
-__host__ __device__ inline int first_range_of_tile(int64_t tile, const WgInfo& wi) {
-  return (int)(tile * wi.spt / wi.per_unit);
+__host__ __device__ inline int block_len(int b, const WgInfo& wi) {
+  return b == wi.nb - 1 ? wi.spt - b * wi.bst : wi.bst;
+}
+// Global index of the first stage of pair (block b, tile t).
+__host__ __device__ inline int64_t pair_start(int b, int t, const WgInfo& wi) {
+  return (int64_t)b * (wi.n_dt * wi.n_ct) * wi.bst + (int64_t)t * block_len(b, wi);
+}
+// The CTA ranges that touch pair (b, t): first .. last.
+__host__ __device__ inline int first_range_of_pair(int b, int t, const WgInfo& wi) {
+  return (int)(pair_start(b, t, wi) / wi.per_unit);
+}
+__host__ __device__ inline int last_range_of_pair(int b, int t, const WgInfo& wi) {
+  return (int)((pair_start(b, t, wi) + block_len(b, wi) - 1) / wi.per_unit);
 }
 
 struct SegIter {
@@ -99,14 +156,19 @@ struct SegIter {
   }
   __device__ bool next(const WgInfo& wi, Unit& x) {
     if (g >= g1) return false;
-    x.tile = (int)(g / wi.spt);
-    const int s0 = (int)(g % wi.spt);
-    const int64_t room = wi.spt - s0;
+    const int tiles = wi.n_dt * wi.n_ct;
+    const int64_t per_block = (int64_t)tiles * wi.bst;
+    const int b = (int)(g / per_block < wi.nb - 1 ? g / per_block : wi.nb - 1);
+    const int64_t off = g - (int64_t)b * per_block;
+    const int len = block_len(b, wi);
+    x.tile = (int)(off / len);
+    const int s0 = (int)(off % len);
+    const int64_t room = len - s0;
     x.stages = (int)(room < g1 - g ? room : g1 - g);
     x.dt = x.tile / wi.n_ct;
     x.ct = x.tile % wi.n_ct;
-    x.slot = x.tile * wi.maxj + (u - first_range_of_tile(x.tile, wi));
-    x.r0 = (int64_t)s0 * WG_BR;
+    x.slot = (b * tiles + x.tile) * wi.maxj + (u - first_range_of_pair(b, x.tile, wi));
+    x.r0 = ((int64_t)b * wi.bst + s0) * WG_BR;
     g += x.stages;
     return true;
   }
@@ -172,7 +234,8 @@ __device__ __forceinline__ void wg_transform(uint8_t* tile, int w, int j, int q,
   }
 }
 
-__global__ void __launch_bounds__(WG_THREADS, 1)
+template <bool PL>
+__global__ void __launch_bounds__(PL ? WG_THREADS_PL : WG_THREADS, 1)
     wgrad_tc_kernel(const __grid_constant__ CUtensorMap map_g,
                     const __grid_constant__ CUtensorMap map_x, int64_t N, int C, int D,
                     WgInfo wi, float* __restrict__ part, float* __restrict__ bpart, int* status) {
@@ -183,17 +246,23 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
   int* abort_flag = &bars->abort_flag;
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  constexpr int RING = PL ? PL_ST : WG_ST;           // ring slots
+  constexpr int SUB = PL ? PL_SUB : 1;               // slots per 32-row stage
+  constexpr uint32_t SLOT = PL ? PL_SLOT : WG_STAGE;  // bytes per slot
+  constexpr uint32_t TILEB = PL ? PL_TILE : WG_TILE;  // one operand's bytes in a slot
+  constexpr int EPIW = PL ? 2 * WG_EPIW : WG_EPIW;   // accumulator-draining warps
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < WG_ST; ++s) {
+    for (int s = 0; s < RING; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->read_g[s], WG_XFW);
       mbar_init(&bars->read_x[s], WG_XFW);
       mbar_init(&bars->ready[s], 2 * WG_XFW);
-      mbar_init(&bars->empty[s], 1);
+      // PL: the MMA commit and the dbias warps both release the slot
+      mbar_init(&bars->empty[s], PL ? 1 + WG_BIASW : 1);
     }
     mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->acc_empty, WG_EPIW * 32);
+    mbar_init(&bars->acc_empty, EPIW * 32);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -213,29 +282,35 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      int issued_phase[WG_ST];
-      for (int s = 0; s < WG_ST; ++s) issued_phase[s] = -1;
+      int issued_phase[RING];
+      for (int s = 0; s < RING; ++s) issued_phase[s] = -1;
       uint32_t it = 0;
       bool ok = true;
       SegIter si(wi, blockIdx.x);
       Unit un;
       while (ok && si.next(wi, un)) {
-        for (int s = 0; s < un.stages; ++s, ++it) {
-          const int slot = it % WG_ST;
-          const uint32_t ph = (it / WG_ST) & 1;
+        for (int s = 0; ok && s < un.stages * SUB; ++s, ++it) {
+          const int slot = it % RING;
+          const uint32_t ph = (it / RING) & 1;
           if (!(ok = wait_bounded(&bars->empty[slot], ph ^ 1, abort_flag, status))) break;
-          mbar_expect_tx(&bars->full[slot], WG_STAGE);
-          const int row = (int)(un.r0 + (int64_t)WG_BR * s);
-          const uint32_t dst = sbase + slot * WG_STAGE;
-          // 3-D views (64 halves, 128-byte chunk of the row, row); a unit's tile is
-          // chunks 8*tile .. 8*tile+7 (128 channels x 4 group elements)
-          tma_load_3d(dst, &map_g, &bars->full[slot], 0, 8 * un.dt, row);
-          tma_load_3d(dst + WG_TILE, &map_x, &bars->full[slot], 0, 8 * un.ct, row);
+          mbar_expect_tx(&bars->full[slot], SLOT);
+          const int row = (int)(un.r0 + (int64_t)(WG_BR / SUB) * s);
+          const uint32_t dst = sbase + slot * SLOT;
+          if constexpr (PL) {
+            // 4-D planes views (64 channels, row, 64-channel block, plane)
+            tma_load_4d(dst, &map_g, &bars->full[slot], 0, row, 2 * un.dt, 0);
+            tma_load_4d(dst + TILEB, &map_x, &bars->full[slot], 0, row, 2 * un.ct, 0);
+          } else {
+            // 3-D views (64 halves, 128-byte chunk of the row, row); a unit's tile is
+            // chunks 8*tile .. 8*tile+7 (128 channels x 4 group elements)
+            tma_load_3d(dst, &map_g, &bars->full[slot], 0, 8 * un.dt, row);
+            tma_load_3d(dst + WG_TILE, &map_x, &bars->full[slot], 0, 8 * un.ct, row);
+          }
           issued_phase[slot] = (int)ph;
         }
       }
       if (!ok)
-        for (int s = 0; s < WG_ST; ++s)
+        for (int s = 0; s < RING; ++s)
           if (issued_phase[s] >= 0) drain_wait(&bars->full[s], (uint32_t)issued_phase[s]);
     }
   } else if (warp == 1) {
@@ -243,27 +318,35 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     if (lane == 0) {
       uint32_t it = 0, ucount = 0;
       bool ok = true;
-      const uint32_t id_n1 = idesc_f16(128, WG_BC);
-      const uint32_t id_n1_neg = idesc_f16(128, WG_BC, true);
-      const uint32_t id_n2 = idesc_f16(128, 2 * WG_BC);
+      const uint32_t id_n1 = PL ? idesc_f16_mn(128, WG_BC) : idesc_f16(128, WG_BC);
+      const uint32_t id_n1_neg =
+          PL ? idesc_f16_mn(128, WG_BC, true) : idesc_f16(128, WG_BC, true);
+      const uint32_t id_n2 = PL ? idesc_f16_mn(128, 2 * WG_BC) : idesc_f16(128, 2 * WG_BC);
       SegIter si(wi, blockIdx.x);
       Unit un;
       for (; ok && si.next(wi, un); ++ucount) {
         if (!(ok = wait_bounded(&bars->acc_empty, (ucount & 1) ^ 1, abort_flag, status))) break;
         tc_fence_after();
-        for (int s = 0; s < un.stages; ++s, ++it) {
-          const int slot = it % WG_ST;
-          if (!(ok = wait_bounded(&bars->ready[slot], (it / WG_ST) & 1, abort_flag, status)))
-            break;
+        for (int s = 0; s < un.stages * SUB; ++s, ++it) {
+          const int slot = it % RING;
+          uint64_t* rbar = PL ? &bars->full[slot] : &bars->ready[slot];
+          if (!(ok = wait_bounded(rbar, (it / RING) & 1, abort_flag, status))) break;
           tc_fence_after();
-          const uint32_t g = sbase + slot * WG_STAGE;  // G planes (A: rows = out-channels)
-          const uint32_t x = g + WG_TILE;              // Xh planes (B: rows = in-channels)
+          const uint32_t g = sbase + slot * SLOT;  // G planes (A: M = out-channels)
+          const uint32_t x = g + TILEB;            // Xh planes (B: N = in-channels)
 #pragma unroll
-          for (int kk = 0; kk < WG_BR / 16; ++kk) {
-            const uint32_t ko = 32u * kk;
+          for (int kk = 0; kk < WG_BR / 16 / SUB; ++kk) {
             const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-            auto A = [&](int p) { return desc_kmajor<WG_ROWB>(g + p * WG_PLANE + ko); };
-            auto B = [&](int p) { return desc_kmajor<WG_ROWB>(x + p * WG_PLANE + ko); };
+            // transform path: K-major planes, K step = 32 B of a row; planes path:
+            // MN-major planes, K step = 16 rows x 128 B
+            auto A = [&](int p) {
+              return PL ? desc_mn128(g + p * PL_PLANE + 2048u * kk, PL_BLOCK)
+                        : desc_kmajor<WG_ROWB>(g + p * WG_PLANE + 32u * kk);
+            };
+            auto B = [&](int p) {
+              return PL ? desc_mn128(x + p * PL_PLANE + 2048u * kk, PL_BLOCK)
+                        : desc_kmajor<WG_ROWB>(x + p * WG_PLANE + 32u * kk);
+            };
             umma(tmem + 0, A(0), B(0), id_n1, acc);              // Q0
             umma(tmem + WG_BC, A(1), B(1), id_n1, acc);          // Q2
             umma(tmem + 2 * WG_BC, A(2), B(2), id_n2, acc);      // [Qr|Qi] += Gr [Xr|Xi]
@@ -278,12 +361,16 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       drain_wait(&bars->drain, 0);
     }
     __syncwarp();
-  } else if (warp >= WG_EPI0 && warp < WG_EPI0 + WG_EPIW) {
+  } else if ((warp >= WG_EPI0 && warp < WG_EPI0 + WG_EPIW) ||
+             (PL && warp >= WG_XF0 + WG_BIASW && warp < WG_XF0 + WG_BIASW + WG_EPIW)) {
     // ---------------- epilogue: accumulators -> FP32 partial planes ----------------
     // Warp w reads TMEM lane quarter q = w % 4: lane l holds out-channel
-    // 32q + l; a 32x32b load gives it 16 consecutive in-channels of one plane,
-    // and each of the 16 stores writes 32 consecutive out-channels (128 B).
+    // 32q + l; two 32x32b loads (one wait) give it 32 consecutive in-channels
+    // of one plane, and each store writes 32 consecutive out-channels (128 B).
+    // Planes variant: warps 4-7 take planes 0-1, warps 12-15 planes 2-3.
     const int q = warp & 3;
+    const int p0 = PL ? (warp >= WG_XF0 ? 2 : 0) : 0;
+    const int p1 = PL ? p0 + 2 : 4;
     uint32_t ucount = 0;
     SegIter si(wi, blockIdx.x);
     Unit un;
@@ -295,26 +382,61 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       const uint32_t lrow = tmem + ((uint32_t)(32 * q) << 16);
       float* slot_base = part + (int64_t)un.slot * (4 * WG_BC * WG_BD);
 #pragma unroll 1
-      for (int p = 0; p < 4; ++p) {
+      for (int p = p0; p < p1; ++p) {
         float* dst_plane = slot_base + p * (WG_BC * WG_BD);
 #pragma unroll 1
-        for (int gq = 0; gq < WG_BC / 16; ++gq) {
+        for (int gq = 0; gq < WG_BC / 16; gq += 2) {
           const int c = un.ct * WG_BC + 16 * gq;
           if (c >= C) break;  // warp-uniform; C % 16 == 0: the 16 columns are all in range
-          uint32_t r[16];
+          const bool two = c + 16 < C;  // the second group of 16 columns is in range
+          uint32_t r[16], r2[16];
           tmem_ld_32x32b<16>(lrow + p * WG_BC + 16 * gq, r);
+          if (two) tmem_ld_32x32b<16>(lrow + p * WG_BC + 16 * gq + 16, r2);
           tmem_wait_ld();
           if (d < D) {
 #pragma unroll
             for (int k = 0; k < 16; ++k)
               dst_plane[(16 * gq + k) * WG_BD + dl] = __uint_as_float(r[k]);
+            if (two) {
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
+                dst_plane[(16 * gq + 16 + k) * WG_BD + dl] = __uint_as_float(r2[k]);
+            }
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
     }
-  } else if (warp >= WG_XF0) {
+  } else if (PL && warp >= WG_XF0 && warp < WG_XF0 + WG_BIASW) {
+    // ---------------- planes variant: dbias partials from plane 0 of dY's spectrum ----------------
+    // thread = out-channel dl of the tile; plane 0 sits at [block dl / 64][row][128 B],
+    // 16-byte piece (dl % 64) / 8 swizzled with row % 8
+    const int dl = (warp - WG_XF0) * 32 + lane;
+    uint32_t it = 0;
+    bool ok = true;
+    SegIter si(wi, blockIdx.x);
+    Unit un;
+    while (ok && si.next(wi, un)) {
+      float b = 0.f;
+      for (int s = 0; s < un.stages * SUB; ++s, ++it) {
+        const int slot = it % RING;
+        if (!(ok = warp_wait(&bars->full[slot], (it / RING) & 1, abort_flag, status))) break;
+        if (un.ct == 0) {
+          const uint8_t* blk = smem + slot * SLOT + (dl >> 6) * PL_BLOCK;
+          const int piece = (dl & 63) >> 3, within = (dl & 7) * 2;
+#pragma unroll 8
+          for (int r = 0; r < PL_ROWS; ++r)
+            b += __half2float(
+                *reinterpret_cast<const __half*>(blk + r * 128 + ((piece ^ (r & 7)) << 4) + within));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->empty[slot]);
+      }
+      if (!ok) break;
+      if (un.ct == 0) bpart[(int64_t)un.slot * WG_BD + dl] = b;
+    }
+  } else if (!PL && warp >= WG_XF0) {
     // ---------------- transform: group DFT, transposed into the operand planes ----------------
     const int grp = (warp - WG_XF0) >> 3;  // 0: dY tile (and the dbias sums), 1: X tile
     const int w = (warp - WG_XF0) & 7;     // raw chunk = channel pairs 8w..8w+7
@@ -375,9 +497,9 @@ __device__ __forceinline__ void store_dw4(float* p, const float* w) {
 __device__ __forceinline__ void store_one(__half* p, float v) { *p = __float2half_rn(v); }
 __device__ __forceinline__ void store_one(float* p, float v) { *p = v; }
 
-// Sum of a tile's partial slots (fixed order), inverse group DFT, cast to Out:
-// dW[d][c][u] from part[tile][j][4][128 c][128 d]; dbias[d] from
-// bpart[tile][j][128] of the tiles with in-channel tile 0.
+// Sum of a tile's partial slots (fixed order: row block, then range), inverse
+// group DFT, cast to Out: dW[d][c][u] from part[pair][j][4][128 c][128 d];
+// dbias[d] from bpart[pair][j][128] of the tiles with in-channel tile 0.
 template <typename Out>
 __global__ void wgrad_tc_finalize_kernel(const float* __restrict__ part,
                                          const float* __restrict__ bpart, WgInfo wi, int C,
@@ -387,14 +509,16 @@ __global__ void wgrad_tc_finalize_kernel(const float* __restrict__ part,
   if (idx < (int64_t)D * C) {
     const int c = (int)(idx / D), d = (int)(idx % D);
     const int tile = (d / WG_BD) * wi.n_ct + c / WG_BC;
-    const int first = first_range_of_tile(tile, wi);
-    const int last = (int)(((int64_t)tile * wi.spt + wi.spt - 1) / wi.per_unit);
     const int64_t off = (int64_t)(c % WG_BC) * WG_BD + (d % WG_BD);
     float qv[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j <= last - first; ++j) {
-      const float* slot = part + ((int64_t)tile * wi.maxj + j) * (4 * WG_BC * WG_BD);
+    for (int b = 0; b < wi.nb; ++b) {
+      const int pair = b * wi.n_dt * wi.n_ct + tile;
+      const int n = last_range_of_pair(b, tile, wi) - first_range_of_pair(b, tile, wi);
+      for (int j = 0; j <= n; ++j) {
+        const float* slot = part + ((int64_t)pair * wi.maxj + j) * (4 * WG_BC * WG_BD);
 #pragma unroll
-      for (int p = 0; p < 4; ++p) qv[p] += slot[p * (WG_BC * WG_BD) + off];
+        for (int p = 0; p < 4; ++p) qv[p] += slot[p * (WG_BC * WG_BD) + off];
+      }
     }
     float wv[4];
     group_idft<4>(qv, wv, tw);
@@ -403,11 +527,12 @@ __global__ void wgrad_tc_finalize_kernel(const float* __restrict__ part,
   if (dbias && idx < D) {
     const int d = (int)idx;
     const int tile = (d / WG_BD) * wi.n_ct;
-    const int first = first_range_of_tile(tile, wi);
-    const int last = (int)(((int64_t)tile * wi.spt + wi.spt - 1) / wi.per_unit);
     float b = 0.f;
-    for (int j = 0; j <= last - first; ++j)
-      b += bpart[((int64_t)tile * wi.maxj + j) * WG_BD + d % WG_BD];
+    for (int rb = 0; rb < wi.nb; ++rb) {
+      const int pair = rb * wi.n_dt * wi.n_ct + tile;
+      const int n = last_range_of_pair(rb, tile, wi) - first_range_of_pair(rb, tile, wi);
+      for (int j = 0; j <= n; ++j) b += bpart[((int64_t)pair * wi.maxj + j) * WG_BD + d % WG_BD];
+    }
     store_one(dbias + idx, b);
   }
 }
@@ -421,6 +546,23 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int channels, int64_t N) 
   cuuint32_t box[3] = {64, 8, WG_BR};
   cuuint32_t estr[3] = {1, 1, 1};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Spectral planes [4][N][channels] viewed as (64 channels, row, 64-channel
+// block, plane); box = (64, 16 rows, 2 blocks, 4 planes), 128-byte swizzle.
+// The block dimension steps by 128 B inside a row, so channels % 64 == 0 keeps
+// every block inside its row.
+bool encode_planes4_map(CUtensorMap* m, const void* base, int channels, int64_t N) {
+  auto encode = encode_fn();
+  if (!encode || channels % 64 != 0) return false;
+  cuuint64_t dims[4] = {64, (cuuint64_t)N, (cuuint64_t)channels / 64, 4};
+  cuuint64_t strides[3] = {(cuuint64_t)channels * 2, 128, (cuuint64_t)N * channels * 2};
+  cuuint32_t box[4] = {64, PL_ROWS, 2, 4};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides,
                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -444,13 +586,17 @@ bool wgrad_tc_layout(int64_t N, int C, int D, int num_sms, WgInfo* wi, int* grid
   if (per > 0x3fffffffLL) return false;
   wi->per_unit = (int)per;
   *grid = (int)((wi->total + per - 1) / per);
-  // slots per tile: the number of ranges that touch it (exact maximum)
-  const int64_t tiles = (int64_t)wi->n_dt * wi->n_ct;
+  // row blocks of one range's length: in every full block, range u covers
+  // exactly pair u, so the CTAs of a block step through its rows together
+  wi->bst = (int)std::min<int64_t>(per, spt);
+  wi->nb = (int)((spt + wi->bst - 1) / wi->bst);
+  // slots per pair: the number of ranges that touch it (exact maximum)
+  const int tiles = wi->n_dt * wi->n_ct;
   int64_t maxj = 1;
-  for (int64_t t = 0; t < tiles; ++t) {
-    const int64_t first = t * spt / per, last = (t * spt + spt - 1) / per;
-    maxj = std::max(maxj, last - first + 1);
-  }
+  for (int b = 0; b < wi->nb; ++b)
+    for (int t = 0; t < tiles; ++t)
+      maxj = std::max<int64_t>(maxj, last_range_of_pair(b, t, *wi) -
+                                         first_range_of_pair(b, t, *wi) + 1);
   wi->maxj = (int)maxj;
   return true;
 }
@@ -467,29 +613,46 @@ size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms) {
   WgInfo wi;
   int grid = 0;
   if (!wgrad_tc_layout(N, C, D, num_sms, &wi, &grid)) return 0;
-  const size_t slots = (size_t)wi.n_dt * wi.n_ct * wi.maxj;
+  const size_t slots = (size_t)wi.nb * wi.n_dt * wi.n_ct * wi.maxj;
   return slots * ((size_t)4 * WG_BC * WG_BD + WG_BD) * sizeof(float);
+}
+
+bool wgrad_tc_planes_supported(int64_t N, int C, int D, const void* Xhat, const void* Ghat) {
+  return wgrad_tc_supported(4, DType::F16, N, C, D, Xhat, Ghat) && C % 64 == 0 && D % 64 == 0;
 }
 
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
                             void* workspace, DType out_dt, void* dW, void* dbias, int* status,
-                            int num_sms, const Twiddles& tw, cudaStream_t st) {
+                            int num_sms, const Twiddles& tw, cudaStream_t st, bool planes) {
   WgInfo wi;
   int grid = 0;
   if (!wgrad_tc_layout(N, C, D, num_sms, &wi, &grid)) return cudaErrorInvalidValue;
+  if (planes && (C % 64 != 0 || D % 64 != 0)) return cudaErrorNotSupported;
   CUtensorMap mg, mx;
-  if (!encode_rows_map(&mg, dY, D, N) || !encode_rows_map(&mx, X, C, N))
+  if (planes) {
+    if (!encode_planes4_map(&mg, dY, D, N) || !encode_planes4_map(&mx, X, C, N))
+      return cudaErrorInvalidValue;
+  } else if (!encode_rows_map(&mg, dY, D, N) || !encode_rows_map(&mx, X, C, N)) {
     return cudaErrorInvalidValue;
+  }
   float* part = static_cast<float*>(workspace);
-  float* bpart = part + (size_t)wi.n_dt * wi.n_ct * wi.maxj * (4 * WG_BC * WG_BD);
+  float* bpart = part + (size_t)wi.nb * wi.n_dt * wi.n_ct * wi.maxj * (4 * WG_BC * WG_BD);
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(wgrad_tc_kernel,
+    cudaError_t e = cudaFuncSetAttribute(wgrad_tc_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(wgrad_tc_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  wgrad_tc_kernel<<<grid, WG_THREADS, WG_SMEM, st>>>(mg, mx, N, C, D, wi, part, bpart, status);
+  if (planes)
+    wgrad_tc_kernel<true><<<grid, WG_THREADS_PL, WG_SMEM, st>>>(mg, mx, N, C, D, wi, part, bpart,
+                                                                status);
+  else
+    wgrad_tc_kernel<false><<<grid, WG_THREADS, WG_SMEM, st>>>(mg, mx, N, C, D, wi, part, bpart,
+                                                              status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t total = std::max<int64_t>((int64_t)C * D, D);

@@ -137,6 +137,73 @@ class EqLinearPlan:
                                     workspace.numel() * workspace.element_size())
         return dW, dbias
 
+    # --- training with saved spectra (the weight gradient runs no transform)
+
+    def forward_save_spectrum(self, X, W_hat, bias=None, act: str = "none", out=None,
+                              Xhat=None):
+        """(forward(X), Xhat): Xhat [4, N, C] is X's group spectrum, kept for
+        backward_weight_from_spectra."""
+        N = X.shape[0]
+        self._check(X, (N, self.C * self.T), "X")
+        if bias is not None:
+            self._check(bias, (self.D,), "bias")
+        if out is None:
+            out = torch.empty((N, self.D * self.T), dtype=self.dtype, device=X.device)
+        if Xhat is None:
+            Xhat = torch.empty((4, N, self.C), dtype=self.dtype, device=X.device)
+        self._check(out, (N, self.D * self.T), "out")
+        self._check(Xhat, (4, N, self.C), "Xhat")
+        _n.eqlinear_forward_save_spectrum(self.handle, X, N, W_hat, bias, _n.ACT[act], out, Xhat)
+        return out, Xhat
+
+    def backward_input_save_spectrum(self, dY, W_hat, out=None, dYhat=None):
+        """(backward_input(dY), dYhat): dYhat [4, N, D] is dY's group spectrum."""
+        N = dY.shape[0]
+        self._check(dY, (N, self.D * self.T), "dY")
+        if out is None:
+            out = torch.empty((N, self.C * self.T), dtype=self.dtype, device=dY.device)
+        if dYhat is None:
+            dYhat = torch.empty((4, N, self.D), dtype=self.dtype, device=dY.device)
+        self._check(out, (N, self.C * self.T), "out")
+        self._check(dYhat, (4, N, self.D), "dYhat")
+        _n.eqlinear_backward_input_save_spectrum(self.handle, dY, N, W_hat, out, dYhat)
+        return out, dYhat
+
+    def backward_weight_from_spectra(self, Xhat, dYhat, dW=None, dbias=None, workspace=None,
+                                     want_bias=True):
+        N = Xhat.shape[1]
+        self._check(Xhat, (4, N, self.C), "Xhat")
+        self._check(dYhat, (4, N, self.D), "dYhat")
+        if dW is None:
+            dW = torch.empty((self.D, self.C, self.T), dtype=self.dtype, device=Xhat.device)
+        if dbias is None and want_bias:
+            dbias = torch.empty((self.D,), dtype=self.dtype, device=Xhat.device)
+        if workspace is None:
+            workspace = torch.empty(max(self.workspace_bytes(N), 16), dtype=torch.uint8,
+                                    device=Xhat.device)
+        _n.eqlinear_backward_weight_from_spectra(self.handle, Xhat, dYhat, N, dW, dbias,
+                                                 workspace,
+                                                 workspace.numel() * workspace.element_size())
+        return dW, dbias
+
+    def backward_weight_from_spectra_f32(self, Xhat, dYhat, buf=None, workspace=None):
+        """backward_weight_f32 from the saved spectra."""
+        N = Xhat.shape[1]
+        self._check(Xhat, (4, N, self.C), "Xhat")
+        self._check(dYhat, (4, N, self.D), "dYhat")
+        if buf is None:
+            buf = self.grad_buffer(torch.float32, Xhat.device)
+        if buf.dtype != torch.float32 or buf.numel() != self.grad_offset() + self.D:
+            raise ValueError("buf must be a flat FP32 gradient buffer of this plan")
+        dW, db = self.split_grad(buf)
+        if workspace is None:
+            workspace = torch.empty(max(self.workspace_bytes(N), 16), dtype=torch.uint8,
+                                    device=Xhat.device)
+        _n.eqlinear_backward_weight_from_spectra_f32(self.handle, Xhat, dYhat, N, dW, db,
+                                                     workspace,
+                                                     workspace.numel() * workspace.element_size())
+        return buf
+
     # --- group-circulant convolution (KH x KW taps, stride 1, zero padding)
 
     def conv_prepare_weights(self, Wc: torch.Tensor, out: torch.Tensor | None = None):

@@ -34,6 +34,8 @@ EXPORTED = (
     "eqlinear_conv_prepared_weight_bytes", "eqlinear_conv_prepare_weights",
     "eqlinear_conv_workspace_bytes", "eqlinear_conv_forward",
     "eqlinear_plan_create_dihedral4",
+    "eqlinear_forward_save_spectrum", "eqlinear_backward_input_save_spectrum",
+    "eqlinear_backward_weight_from_spectra", "eqlinear_backward_weight_from_spectra_f32",
 )
 
 
@@ -73,6 +75,11 @@ def _load() -> ctypes.CDLL:
         "eqlinear_backward_weight_noalloc": ([vp, vp, vp, i64, vp, vp, vp], i32),
         "eqlinear_backward_weight_f32": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
         "eqlinear_cast_from_f32": ([vp, vp, i64, vp, vp], i32),
+        "eqlinear_forward_save_spectrum": ([vp, vp, i64, vp, vp, i32, vp, vp, vp], i32),
+        "eqlinear_backward_input_save_spectrum": ([vp, vp, i64, vp, vp, vp, vp], i32),
+        "eqlinear_backward_weight_from_spectra": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
+        "eqlinear_backward_weight_from_spectra_f32": ([vp, vp, vp, i64, vp, vp, vp, sz, vp],
+                                                      i32),
         "eqlinear_chain_workspace_bytes": ([vp, vp, i64], sz),
         "eqlinear_conv_prepared_weight_bytes": ([vp, i32, i32], sz),
         "eqlinear_conv_prepare_weights": ([vp, i32, i32, vp, vp, vp], i32),
@@ -213,6 +220,37 @@ def eqlinear_backward_weight_f32(plan: int, X, dY, N: int, dW, dbias, workspace,
     _check(_lib.eqlinear_backward_weight_f32(plan, _ptr(X), _ptr(dY), N, _ptr(dW), _ptr(dbias),
                                              _ptr(workspace), workspace_bytes, _stream(stream)),
            "eqlinear_backward_weight_f32")
+
+
+def eqlinear_forward_save_spectrum(plan: int, X, N: int, W_hat, bias, act: int, Y, Xhat,
+                                   stream=None) -> None:
+    _check(_lib.eqlinear_forward_save_spectrum(plan, _ptr(X), N, _ptr(W_hat), _ptr(bias), act,
+                                               _ptr(Y), _ptr(Xhat), _stream(stream)),
+           "eqlinear_forward_save_spectrum")
+
+
+def eqlinear_backward_input_save_spectrum(plan: int, dY, N: int, W_hat, dX, dYhat,
+                                          stream=None) -> None:
+    _check(_lib.eqlinear_backward_input_save_spectrum(plan, _ptr(dY), N, _ptr(W_hat), _ptr(dX),
+                                                      _ptr(dYhat), _stream(stream)),
+           "eqlinear_backward_input_save_spectrum")
+
+
+def eqlinear_backward_weight_from_spectra(plan: int, Xhat, dYhat, N: int, dW, dbias, workspace,
+                                          workspace_bytes: int, stream=None) -> None:
+    _check(_lib.eqlinear_backward_weight_from_spectra(plan, _ptr(Xhat), _ptr(dYhat), N, _ptr(dW),
+                                                      _ptr(dbias), _ptr(workspace),
+                                                      workspace_bytes, _stream(stream)),
+           "eqlinear_backward_weight_from_spectra")
+
+
+def eqlinear_backward_weight_from_spectra_f32(plan: int, Xhat, dYhat, N: int, dW, dbias,
+                                              workspace, workspace_bytes: int,
+                                              stream=None) -> None:
+    _check(_lib.eqlinear_backward_weight_from_spectra_f32(plan, _ptr(Xhat), _ptr(dYhat), N,
+                                                          _ptr(dW), _ptr(dbias), _ptr(workspace),
+                                                          workspace_bytes, _stream(stream)),
+           "eqlinear_backward_weight_from_spectra_f32")
 
 
 def eqlinear_cast_from_f32(plan: int, src, count: int, dst, stream=None) -> None:

@@ -346,6 +346,54 @@ EQL_API eqlinear_status_t eqlinear_backward_weight_f32(eqlinear_plan_t plan, con
                                                        size_t workspace_bytes, void* stream);
 
 /*
+ * Training with saved input spectra.  The weight gradient is a sum over rows
+ * of per-frequency products of the group DFTs of X and dY ("Algorithmic
+ * approach": the backward pass reuses the per-frequency structure); the
+ * forward and the input-gradient kernels already form exactly those DFTs as
+ * their tensor-core operands.  These calls keep them, so the weight gradient
+ * multiplies them directly and runs no transform of its own:
+ *
+ * eqlinear_forward_save_spectrum: eqlinear_forward_act (Y bitwise the same),
+ *   and also Xhat [4][N][C], the group DFT of X (plane 0: x0+x1+x2+x3, 1:
+ *   x0-x1+x2-x3, 2: x0-x2, 3: x3-x1; FP32 arithmetic, one rounding to FP16),
+ *   the planes order of eqlinear_forward_to_spectral.
+ * eqlinear_backward_input_save_spectrum: eqlinear_backward_input (dX bitwise
+ *   the same), and also dYhat [4][N][D], the group DFT of dY in that order.
+ * eqlinear_backward_weight_from_spectra (and _f32, as eqlinear_backward_weight
+ *   _f32): eqlinear_backward_weight from Xhat and dYhat instead of X and dY,
+ *   with the same workspace (eqlinear_backward_weight_workspace_bytes).  dW's
+ *   operands are the same FP16 values the transforming kernel forms; dbias sums
+ *   dYhat's plane 0 (already rounded to FP16) instead of the FP32 sums.
+ *   A layer whose input arrives as the planes of eqlinear_forward_to_spectral
+ *   may pass them as its Xhat.
+ *
+ * Tensor cores only: FP16 plans with T = 4 and C, D multiples of 16 (the save
+ * calls) or of 64 (the weight gradient), not forced to the CUDA cores;
+ * otherwise EQL_ERR_UNSUPPORTED.  Xhat takes 4 * N * C * 2 bytes (as X),
+ * dYhat 4 * N * D * 2 (as dY); all pointers 16-byte aligned; a spectrum must
+ * not overlap the call's other buffers.  N = 0: the save calls do nothing and
+ * the weight gradient writes zeros.
+ */
+EQL_API eqlinear_status_t eqlinear_forward_save_spectrum(eqlinear_plan_t plan, const void* X,
+                                                         int64_t N, const void* W_hat,
+                                                         const void* bias, eqlinear_act_t act,
+                                                         void* Y, void* Xhat, void* stream);
+EQL_API eqlinear_status_t eqlinear_backward_input_save_spectrum(eqlinear_plan_t plan,
+                                                                const void* dY, int64_t N,
+                                                                const void* W_hat, void* dX,
+                                                                void* dYhat, void* stream);
+EQL_API eqlinear_status_t eqlinear_backward_weight_from_spectra(eqlinear_plan_t plan,
+                                                                const void* Xhat,
+                                                                const void* dYhat, int64_t N,
+                                                                void* dW, void* dbias,
+                                                                void* workspace,
+                                                                size_t workspace_bytes,
+                                                                void* stream);
+EQL_API eqlinear_status_t eqlinear_backward_weight_from_spectra_f32(
+    eqlinear_plan_t plan, const void* Xhat, const void* dYhat, int64_t N, float* dW, float* dbias,
+    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * dst[i] = src[i] rounded to nearest-even in the plan dtype, for i < count
  * (a copy for FP32 plans).  src: count FP32 values on the plan's device; dst:
  * count values of the plan dtype; the two must not overlap (an FP32 plan may
