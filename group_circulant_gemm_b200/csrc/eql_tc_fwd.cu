@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap map_x_half,
                      const __grid_constant__ CUtensorMap map_y_half,
                      const __grid_constant__ CUtensorMap map_p,
+                     const __grid_constant__ CUtensorMap map_p_half,
                      const uint8_t* __restrict__ wtiles, const __half* __restrict__ bias,
                      int64_t N, int Cin, int Cout, TileInfo ti, int* status) {
   using S = Shape<T>;
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bounded(&empty[s], ph ^ 1, abort_flag, status))) break;
           if (!is_raw && blockIdx.x == 0 && (int)it == ti.drop_w) continue;  // injected fault
           if (is_raw) {
-            if constexpr (IO == kIoSpatial && T == 4) {
+            if constexpr ((IO == kIoSpatial || IO == kIoSaveSpectrum) && T == 4) {
               if (up.half >= 0) {
                 // a 64-row half unit: the first 64 rows of the raw layout
                 mbar_expect_tx(&full[s], X_STAGE_BYTES / 2);
@@ -292,8 +293,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ks % ti.n_dt == up.dt) {
             // the transform warps fenced their plane stores to the async proxy before
             // arriving on x_ready; rows past N and channels past Cin are clipped
-            tma_store_3d(&map_p, sbase + S::OFF_X + sx * X_STAGE_BYTES, S::BK * ks,
-                         (int)up.row0, 0);
+            const uint32_t src = sbase + S::OFF_X + sx * X_STAGE_BYTES;
+            if (T == 4 && up.half >= 0) {
+              // a 64-row half unit fills rows 0..63 of each plane: one box per plane
+              for (int p = 0; p < 4; ++p)
+                tma_store_3d(&map_p_half, src + p * S::PLANE_BYTES, S::BK * ks, (int)up.row0,
+                             p);
+            } else {
+              tma_store_3d(&map_p, src, S::BK * ks, (int)up.row0, 0);
+            }
             bulk_commit();
             if (pending >= 0) {
               bulk_wait_read_1();
@@ -441,11 +449,11 @@ namespace {
 
 // Spectral planes [4][N][channels] (FP16), viewed as (channel, row, plane).
 bool encode_planes_map(CUtensorMap* m, void* base, int channels, int64_t N, uint32_t box_ch,
-                       uint32_t box_rows, CUtensorMapSwizzle swz) {
+                       uint32_t box_rows, CUtensorMapSwizzle swz, uint32_t box_planes = 4) {
   auto encode = encode_fn();
   cuuint64_t dims[3] = {(cuuint64_t)channels, (cuuint64_t)N, 4};
   cuuint64_t strides[2] = {(cuuint64_t)channels * 2, (cuuint64_t)N * channels * 2};
-  cuuint32_t box[3] = {box_ch, box_rows, 4};
+  cuuint32_t box[3] = {box_ch, box_rows, box_planes};
   cuuint32_t estr[3] = {1, 1, 1};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, base, dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -555,13 +563,17 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     }
-    CUtensorMap mp = mx;
+    CUtensorMap mp = mx, mp_half = mx;
     if (io == kIoSaveSpectrum) {
-      // the input's spectrum: store box = 32 channels (64 B) x 128 rows x 4 planes
-      if (!encode_planes_map(&mp, spectrum, Cin, N, S::BK, BM, CU_TENSOR_MAP_SWIZZLE_64B))
+      // the input's spectrum: store box = 32 channels (64 B) x 128 rows x 4 planes,
+      // for half units 32 channels x 64 rows x 1 plane
+      if (!encode_planes_map(&mp, spectrum, Cin, N, S::BK, BM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+          !encode_planes_map(&mp_half, spectrum, Cin, N, S::BK, 64, CU_TENSOR_MAP_SWIZZLE_64B,
+                             1))
         return cudaErrorInvalidValue;
     }
-    if (io != kIoSpatial) {  // no half units with spectral input or output
+    const bool halves_ok = io == kIoSpatial || io == kIoSaveSpectrum;
+    if (!halves_ok) {  // no half units with spectral input or output
       mx_half = mx;
       my_half = my;
     }
@@ -577,7 +589,7 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
     // traffic (its MMAs cost as much as a whole tile's), so the wave ends sooner.
     ti.full = ti.num_tiles;
     ti.num_units = ti.num_tiles;
-    if (io == kIoSpatial && TT == 4) {  // T = 8 tiles keep their registers for the transform
+    if (halves_ok && TT == 4) {  // T = 8 tiles keep their registers for the transform
       const int rem = ti.num_tiles >= num_sms ? ti.num_tiles % num_sms : ti.num_tiles;
       if (rem > 0 && 2 * rem <= num_sms) {
         ti.full = ti.num_tiles - rem;
@@ -620,7 +632,7 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
                           : eq_fwd_tc_kernel<TT, 0, kIoSpatial, 1>;
     }
     kernel<<<grid, kThreads, S::SMEM_BYTES, st>>>(
-        mx, my, mx_half, my_half, mp, static_cast<const uint8_t*>(Wtiles),
+        mx, my, mx_half, my_half, mp, mp_half, static_cast<const uint8_t*>(Wtiles),
         static_cast<const __half*>(bias), N, Cin, Cout, ti, status);
     return cudaGetLastError();
   });

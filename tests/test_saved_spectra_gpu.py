@@ -146,6 +146,9 @@ def test_training_step_full_size_from_spectra():
     _, dYhat = p.backward_input_save_spectrum(dY, Wh)
     dW, db = p.backward_weight_from_spectra(Xhat, dYhat)
     assert p.status() == 0
+    # both saved spectra in full (the last partial wave runs as 64-row half units)
+    _check_planes(Xhat.cpu().numpy(), _planes_ref(inp["X"], C))
+    _check_planes(dYhat.cpu().numpy(), _planes_ref(inp["dY"], D))
     rng = np.random.default_rng(5301)
     d_idx = np.concatenate([[0, D - 1, 127, 128], rng.integers(0, D, 28)]).astype(np.int64)
     c_idx = np.concatenate([[0, C - 1, 255, 256], rng.integers(0, C, 28)]).astype(np.int64)
