@@ -124,11 +124,14 @@ KERNEL_SOURCES = {
     "backward_weight": ("eql_tc_wgrad.cu", "eql_tc_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("forward", "bfd6f056114c3e22"): {"p4_vitb_mlp_2calls_f16": 58.98e6, "c8_1024_f16": 33.94e6,
-                                      "p4_vith_fc1_fwd_bwd_f16": 69.82e6,
-                                      "p4m_vitb_mlp_f16": 58.07e6},
-    ("forward_chain", "033fd47b5cd211f5"): {"p4_vitb_mlp_f16": 86.94e6},
-    ("conv", "c700b6d872d52cc5"): {"p4_conv3x3_f16": 160.33e6},
+    ("forward", "4458390a32641562"): {"p4_vitb_mlp_2calls_f16": 58.33e6, "c8_1024_f16": 33.95e6,
+                                      "p4_vith_fc1_f16": 48.86e6,
+                                      "p4_vith_fc1_fwd_bwd_f16": 107.56e6,
+                                      "p4m_vitb_mlp_f16": 57.75e6},
+    ("forward_chain", "350ff7855a00971d"): {"p4_vitb_mlp_f16": 89.45e6,
+                                            "p4_vitb_mlp_spectral_f16": 89.27e6,
+                                            "p4_vitb_mlp_block_f16": 85.77e6},
+    ("conv", "e00676af90759f5d"): {"p4_conv3x3_f16": 160.12e6},
 }
 
 def kernel_traffic(family: str, workload: str):

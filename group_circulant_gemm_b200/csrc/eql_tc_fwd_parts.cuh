@@ -25,8 +25,8 @@ constexpr uint32_t kStgBytes = 4096;  // per epilogue warp: 32 rows x 128 B of Y
 // Input/output forms (T = 4): spatial X and Y; Y written as the next layer's
 // spectral operand planes; X read as spectral operand planes.
 // kIoSaveSpectrum: spatial X and Y, and the input's group spectrum (the operand
-// planes the transform makes) also written to [4][N][Cin] by the first
-// out-channel tile of each row tile, for a later weight gradient.
+// planes the transform makes) also written to [4][N][Cin], for a later weight
+// gradient.
 constexpr int kIoSpatial = 0, kIoSpectralOut = 1, kIoSpectralIn = 2, kIoSaveSpectrum = 3;
 
 // Per-group shape of the pipeline.

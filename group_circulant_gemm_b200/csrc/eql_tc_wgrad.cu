@@ -139,12 +139,14 @@ __host__ __device__ inline int block_len(int b, const WgInfo& wi) {
 __host__ __device__ inline int64_t pair_start(int b, int t, const WgInfo& wi) {
   return (int64_t)b * (wi.n_dt * wi.n_ct) * wi.bst + (int64_t)t * block_len(b, wi);
 }
-// The CTA ranges that touch pair (b, t): first .. last.
+// The CTA ranges that touch pair (b, t): first .. last.  The layout keeps the
+// stage count below 2^31, so 32-bit unsigned division suffices (the finalize
+// evaluates these per output element).
 __host__ __device__ inline int first_range_of_pair(int b, int t, const WgInfo& wi) {
-  return (int)(pair_start(b, t, wi) / wi.per_unit);
+  return (int)((uint32_t)pair_start(b, t, wi) / (uint32_t)wi.per_unit);
 }
 __host__ __device__ inline int last_range_of_pair(int b, int t, const WgInfo& wi) {
-  return (int)((pair_start(b, t, wi) + block_len(b, wi) - 1) / wi.per_unit);
+  return (int)((uint32_t)(pair_start(b, t, wi) + block_len(b, wi) - 1) / (uint32_t)wi.per_unit);
 }
 
 struct SegIter {
@@ -487,9 +489,10 @@ __global__ void __launch_bounds__(PL ? WG_THREADS_PL : WG_THREADS, 1)
 }
 
 __device__ __forceinline__ void store_dw4(__half* p, const float* w) {
-  __half2* out = reinterpret_cast<__half2*>(p);
-  out[0] = __floats2half2_rn(w[0], w[1]);
-  out[1] = __floats2half2_rn(w[2], w[3]);
+  // one 8-byte store (p is 8-byte aligned: dW is 16-byte aligned, entries are 4 halves)
+  const __half2 lo = __floats2half2_rn(w[0], w[1]), hi = __floats2half2_rn(w[2], w[3]);
+  *reinterpret_cast<uint2*>(p) =
+      make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
 }
 __device__ __forceinline__ void store_dw4(float* p, const float* w) {
   *reinterpret_cast<float4*>(p) = make_float4(w[0], w[1], w[2], w[3]);
@@ -500,40 +503,55 @@ __device__ __forceinline__ void store_one(float* p, float v) { *p = v; }
 // Sum of a tile's partial slots (fixed order: row block, then range), inverse
 // group DFT, cast to Out: dW[d][c][u] from part[pair][j][4][128 c][128 d];
 // dbias[d] from bpart[pair][j][128] of the tiles with in-channel tile 0.
+// A block takes 32 out-channels x 8 in-channels (inside one 128 x 128 tile), one
+// entry per thread: lanes read the partials along d, the results pass through
+// shared memory, and groups of 8 lanes write dW along c (each entry 4
+// contiguous values), so both sides are coalesced.
+constexpr int FZ_D = 32, FZ_C = 8;
 template <typename Out>
-__global__ void wgrad_tc_finalize_kernel(const float* __restrict__ part,
-                                         const float* __restrict__ bpart, WgInfo wi, int C,
-                                         int D, Out* __restrict__ dW, Out* __restrict__ dbias,
-                                         Twiddles tw) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // c * D + d
-  if (idx < (int64_t)D * C) {
-    const int c = (int)(idx / D), d = (int)(idx % D);
-    const int tile = (d / WG_BD) * wi.n_ct + c / WG_BC;
-    const int64_t off = (int64_t)(c % WG_BC) * WG_BD + (d % WG_BD);
-    float qv[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int b = 0; b < wi.nb; ++b) {
-      const int pair = b * wi.n_dt * wi.n_ct + tile;
-      const int n = last_range_of_pair(b, tile, wi) - first_range_of_pair(b, tile, wi);
-      for (int j = 0; j <= n; ++j) {
-        const float* slot = part + ((int64_t)pair * wi.maxj + j) * (4 * WG_BC * WG_BD);
+__global__ void __launch_bounds__(256)
+    wgrad_tc_finalize_kernel(const float* __restrict__ part, const float* __restrict__ bpart,
+                             WgInfo wi, int C, int D, Out* __restrict__ dW,
+                             Out* __restrict__ dbias, Twiddles tw) {
+  __shared__ __align__(16) float s[FZ_C][FZ_D * 4 + 4];  // [c][d][u], rows padded by 16 B
+  const int d0 = blockIdx.x * FZ_D, c0 = blockIdx.y * FZ_C;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;  // 8 warps
+  const int tile = (d0 / WG_BD) * wi.n_ct + c0 / WG_BC;
+  {
+    const int d = d0 + lane, c = c0 + w;  // lane = out-channel, warp = in-channel
+    if (d < D && c < C) {
+      const int64_t off = (int64_t)(c % WG_BC) * WG_BD + (d % WG_BD);
+      float qv[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int b = 0; b < wi.nb; ++b) {
+        const int pair = b * wi.n_dt * wi.n_ct + tile;
+        const int n = last_range_of_pair(b, tile, wi) - first_range_of_pair(b, tile, wi);
+        for (int j = 0; j <= n; ++j) {
+          const float* slot = part + ((int64_t)pair * wi.maxj + j) * (4 * WG_BC * WG_BD);
 #pragma unroll
-        for (int p = 0; p < 4; ++p) qv[p] += slot[p * (WG_BC * WG_BD) + off];
+          for (int p = 0; p < 4; ++p) qv[p] += slot[p * (WG_BC * WG_BD) + off];
+        }
       }
+      float wv[4];
+      group_idft<4>(qv, wv, tw);
+      *reinterpret_cast<float4*>(&s[w][4 * lane]) = make_float4(wv[0], wv[1], wv[2], wv[3]);
     }
-    float wv[4];
-    group_idft<4>(qv, wv, tw);
-    store_dw4(dW + ((int64_t)d * C + c) * 4, wv);
   }
-  if (dbias && idx < D) {
-    const int d = (int)idx;
-    const int tile = (d / WG_BD) * wi.n_ct;
+  __syncthreads();
+  {
+    const int cl = threadIdx.x & (FZ_C - 1), dl = threadIdx.x / FZ_C;
+    const int c = c0 + cl, d = d0 + dl;
+    if (d < D && c < C) store_dw4(dW + ((int64_t)d * C + c) * 4, &s[cl][4 * dl]);
+  }
+  if (dbias && blockIdx.y == 0 && w == 0 && d0 + lane < D) {
+    const int d = d0 + lane;
+    const int tile0 = (d / WG_BD) * wi.n_ct;
     float b = 0.f;
     for (int rb = 0; rb < wi.nb; ++rb) {
-      const int pair = rb * wi.n_dt * wi.n_ct + tile;
-      const int n = last_range_of_pair(rb, tile, wi) - first_range_of_pair(rb, tile, wi);
+      const int pair = rb * wi.n_dt * wi.n_ct + tile0;
+      const int n = last_range_of_pair(rb, tile0, wi) - first_range_of_pair(rb, tile0, wi);
       for (int j = 0; j <= n; ++j) b += bpart[((int64_t)pair * wi.maxj + j) * WG_BD + d % WG_BD];
     }
-    store_one(dbias + idx, b);
+    store_one(dbias + d, b);
   }
 }
 
@@ -578,6 +596,7 @@ bool wgrad_tc_layout(int64_t N, int C, int D, int num_sms, WgInfo* wi, int* grid
   if (spt > 0x3fffffffLL) return false;
   wi->spt = (int)spt;
   wi->total = (int64_t)wi->n_dt * wi->n_ct * spt;
+  if (wi->total > 0x7fffffffLL) return false;  // stage indices stay 32-bit
   const int64_t want = std::min<int64_t>(num_sms, wi->total);
   int64_t per = (wi->total + want - 1) / want;
   // at least 16 stages (512 rows) per range, or a whole tile, so the 256 KB
@@ -655,13 +674,12 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
                                                               status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t total = std::max<int64_t>((int64_t)C * D, D);
-  const unsigned fblocks = (unsigned)((total + 255) / 256);
+  const dim3 fgrid((D + FZ_D - 1) / FZ_D, (C + FZ_C - 1) / FZ_C);
   if (out_dt == DType::F32)
-    wgrad_tc_finalize_kernel<float><<<fblocks, 256, 0, st>>>(
+    wgrad_tc_finalize_kernel<float><<<fgrid, 256, 0, st>>>(
         part, bpart, wi, C, D, static_cast<float*>(dW), static_cast<float*>(dbias), tw);
   else
-    wgrad_tc_finalize_kernel<__half><<<fblocks, 256, 0, st>>>(
+    wgrad_tc_finalize_kernel<__half><<<fgrid, 256, 0, st>>>(
         part, bpart, wi, C, D, static_cast<__half*>(dW), static_cast<__half*>(dbias), tw);
   return cudaGetLastError();
 }
