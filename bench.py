@@ -3,8 +3,8 @@
 
 Default workload: the p4 (T=4) FP16 ViT-B MLP pair, N = 12608 rows (64 images x
 197 tokens), layer 1 C=192 -> D=768 (768 -> 3072 features), layer 2 C=768 ->
-D=192 (3072 -> 768) applied to layer 1's output.  One step = both forward
-launches.  `value` = rows (tokens) per second over the whole job, inputs
+D=192 (3072 -> 768) applied to layer 1's output.  One step = both layers, as
+one chained launch.  `value` = rows (tokens) per second over the whole job, inputs
 resident in HBM; `e2e` = the same through the C ABI with the step's input copied
 from pinned host memory and the result read back, inside the timed region.
 
@@ -12,13 +12,14 @@ Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|referenc
        [--workload p4_vitb_mlp_f16|p4_vitb_mlp_2calls_f16|p4_vitb_proj_f32|p4_vith_fc1_f16|
                    c8_1024_f16|p4_vith_fc1_fwd_bwd_f16|p4_vitb_mlp_block_f16|
                    p4_vitb_mlp_spectral_f16|p4m_vitb_mlp_f16|p4_conv3x3_f16] [--dp-path]
-       [--no-dense]
-       [--no-cpu-baseline]
+       [--wgrad-transform] [--no-dense] [--no-cpu-baseline] [--eager]
+The training workload (p4_vith_fc1_fwd_bwd_f16) is forward, dX and dW; the
+forward and dX kernels save the group spectra of X and dY, which dW multiplies
+directly (--wgrad-transform: dW transforms X and dY itself).
 Under torchrun (N > 1) every rank runs its own copy of the workload (weak
 scaling; rows are independent, so no collective is on the forward path).  The
 training workload is then data parallel: each rank's FP32 weight gradient is
-summed over ranks by one NCCL all-reduce, queued behind dW while dX runs, and
-rounded once.
+summed over ranks by one NCCL all-reduce and rounded once.
 """
 from __future__ import annotations
 
