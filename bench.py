@@ -713,7 +713,11 @@ def run_ours(args, workload):
         if dkern == "tcgen05":
             peak = peaks["bf16_tflops"]
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": kernel_traffic(dlabel, workload),
+                    "frac": achieved / peak,
+                    # the training step's forward family stores spectra unless
+                    # --wgrad-transform: its counters were taken in that mode only
+                    "traffic": (None if backward and args.wgrad_transform
+                                else kernel_traffic(dlabel, workload)),
                     "peak_source": f"{peak_src} dense bf16 burst (fp16 runs at the same rate)"}
         else:
             # CUDA-core FP32 FMA peak: 148 SMs x 128 FMA/clk x 2 FLOP x max SM clock
