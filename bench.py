@@ -491,8 +491,10 @@ def run_ours(args, workload):
         w0 = pipeline[0]
         dys = [torch.from_numpy(dy_host).cuda() for _ in range(nsets)]
         dxs = [torch.empty((N, w0.C * w0.T), dtype=dt, device="cuda") for _ in range(nsets)]
-        gbuf = plans[0].grad_buffer(dt)
-        dW, db = plans[0].split_grad(gbuf)
+        # two gradient buffers (set i uses i % 2) so that the end-to-end loop can
+        # copy one step's dW out while the next step computes
+        gbufs = [plans[0].grad_buffer(dt) for _ in range(2)]
+        gbuf = gbufs[0]
         gbuf32 = plans[0].grad_buffer(torch.float32) if dp else None
         ws = torch.empty(max(16, plans[0].workspace_bytes(N)), dtype=torch.uint8, device="cuda")
         if saved:
@@ -560,10 +562,12 @@ def run_ours(args, workload):
                     plans[0].backward_weight_f32(a, g, buf=gbuf32, workspace=ws)
                 # queued behind dW; dX runs on the compute stream meanwhile
                 pending.append(allreduce_grad_buffer(gbuf32, async_op=True))
-            elif saved:
-                plans[0].backward_weight_from_spectra(a, g, dW=dW, dbias=db, workspace=ws)
             else:
-                plans[0].backward_weight(a, g, dW=dW, dbias=db, workspace=ws)
+                dW, db = plans[0].split_grad(gbufs[i % 2])
+                if saved:
+                    plans[0].backward_weight_from_spectra(a, g, dW=dW, dbias=db, workspace=ws)
+                else:
+                    plans[0].backward_weight(a, g, dW=dW, dbias=db, workspace=ws)
 
         def grad_sync(i):
             handle = pending.pop()
@@ -659,19 +663,21 @@ def run_ours(args, workload):
         h2d += dy_pin.numel() * dy_pin.element_size()
         d2h += (dx_pin.numel() + dw_pin.numel()) * dx_pin.element_size()
 
-    # Forward workloads overlap each step's copies with the neighbouring steps'
-    # compute: copy-in, compute and copy-out streams over two device input/output
-    # sets, ordered by events (a set is refilled only after the step two back has
-    # read it and its output only after that step's copy-out).  The training step
-    # runs its copies and kernels in order on one stream (dW has one buffer).
-    s_in = torch.cuda.Stream() if not backward else stream
-    s_out = torch.cuda.Stream() if not backward else stream
+    # Each step's copies overlap the neighbouring steps' compute: copy-in,
+    # compute and copy-out streams over two device input/output sets, ordered by
+    # events (a set is refilled only after the step two back has read it, and
+    # its outputs are overwritten only after that step's copy-out).  The
+    # data-parallel training step keeps its copies and kernels in order on one
+    # stream (its all-reduce and cast share one buffer).
+    piped = not dp
+    s_in = torch.cuda.Stream() if piped else stream
+    s_out = torch.cuda.Stream() if piped else stream
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_c = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
 
     def e2e_step(k):
-        if backward:
+        if not piped:
             xs[0].copy_(x_pin, non_blocking=True)
             dys[0].copy_(dy_pin, non_blocking=True)
             step(0)
@@ -684,6 +690,8 @@ def run_ours(args, workload):
             if k >= 2:
                 s_in.wait_event(ev_c[j])
             xs[j].copy_(x_pin, non_blocking=True)
+            if backward:
+                dys[j].copy_(dy_pin, non_blocking=True)
             ev_in[j].record(s_in)
         stream.wait_event(ev_in[j])
         if k >= 2:
@@ -693,6 +701,9 @@ def run_ours(args, workload):
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_c[j])
             y_pin.copy_(outs[j][-1], non_blocking=True)
+            if backward:
+                dx_pin.copy_(dxs[j], non_blocking=True)
+                dw_pin.copy_(gbufs[j], non_blocking=True)
             ev_out[j].record(s_out)
 
     for k in range(2):
@@ -795,7 +806,7 @@ def run_ours(args, workload):
             "dense_comparator": comparator,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                    "copies": ("in order with the kernels on one stream" if backward else
+                    "copies": ("in order with the kernels on one stream" if dp else
                                "overlapped with the neighbouring steps' kernels (copy-in, "
                                "compute, copy-out streams; two device sets)")},
             "gpu_launches": args.steps * sum(2 if label == "backward_weight" else 1
