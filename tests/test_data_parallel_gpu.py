@@ -123,3 +123,25 @@ def test_cast_from_f32_edges():
     assert native.raw_status("eqlinear_cast_from_f32", q.handle, x.data_ptr(), 10,
                              x.data_ptr(), None) == native.EQL_OK
     assert torch.equal(x, torch.arange(10, dtype=torch.float32, device="cuda"))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_emulated_ranks_from_saved_spectra(world):
+    """The training step's form: each rank saves the spectra of its rows in the
+    forward and dX calls and writes FP32 sums from them; the FP32 total, cast
+    once, meets the oracle on the whole batch."""
+    w = Workload("dpspec", 4, 2501, 128, 192, "f16", True, 4343)
+    inp = make_inputs(w, need_dy=True)
+    p = _plan(w)
+    Wh = p.prepare_weights(_dev(inp["W"]))
+    total = p.grad_buffer(torch.float32)
+    for r in range(world):
+        a, b = row_shard(w.N, world, r)
+        _, xhat = p.forward_save_spectrum(_dev(inp["X"][a:b]), Wh)
+        _, ghat = p.backward_input_save_spectrum(_dev(inp["dY"][a:b]), Wh)
+        total += p.backward_weight_from_spectra_f32(xhat, ghat)
+    dW, db = p.split_grad(p.cast_from_f32(total))
+    assert p.status() == 0
+    rdW, rdb = oracle.backward_weight(4, inp["X"], inp["dY"], w.D)
+    assert _rel(dW.double().cpu().numpy(), rdW) <= TOL["f16"]
+    assert _rel(db.double().cpu().numpy(), rdb) <= TOL["f16"]
