@@ -46,11 +46,11 @@
 // Planes variant (PL): the group DFTs of X and dY arrive precomputed as FP16
 // planes [4][N][C] and [4][N][D] (written by the forward and dX kernels while
 // they transform the same tensors), so no transform runs here.  A ring slot is
-// 16 rows: one 4-D TMA box per operand, (64 channels, 16 rows, 2 blocks of 64
-// channels, 4 planes), 128-byte swizzled, landing as [plane][block][16 rows]
-// [128 B]: the rows are the MMA's K dimension and the channels are contiguous,
-// i.e. MN-major operands (64-channel blocks 2 KB apart, 8-row groups 1 KB
-// apart, so the N = 256 [Xr | Xi] operand spans planes 2 and 3 at a uniform
+// one 32-row stage: one 4-D TMA box per operand, (64 channels, 32 rows, 2 blocks
+// of 64 channels, 4 planes), 128-byte swizzled, landing as [plane][block][32
+// rows][128 B]: the rows are the MMA's K dimension and the channels are
+// contiguous, i.e. MN-major operands (64-channel blocks 4 KB apart, 8-row groups
+// 1 KB apart, so the N = 256 [Xr | Xi] operand spans planes 2 and 3 at a uniform
 // stride).  Warps 8-11 sum plane 0 of dY's spectrum for dbias; warps 4-7 and
 // 12-15 drain planes 0-1 and 2-3 of the accumulators.  Needs C and D
 // multiples of 64.
@@ -77,14 +77,14 @@ constexpr uint32_t WG_OFF_BAR = WG_ST * WG_STAGE;
 constexpr uint32_t WG_SMEM = WG_OFF_BAR + 512 + 1024;
 constexpr int WG_THREADS = 768;
 // Planes variant: no transform warps; warps 8..11 sum dbias, warps 4..7 and
-// 12..15 drain the accumulators.  Its ring holds 6 slots of 16 rows (one MMA K
-// step, 32 KB) in the same 192 KB, so more bytes stay in flight.
+// 12..15 drain the accumulators.  Its ring has the same 192 KB; PL_SUB = 2
+// would split each stage into two 16-row slots (6 deep), which measured slower.
 constexpr int WG_THREADS_PL = 512;
 constexpr int WG_BIASW = 4;
 constexpr int PL_SUB = 1;                         // slots per 32-row stage
-constexpr int PL_ST = 3;                          // ring depth
-constexpr int PL_ROWS = WG_BR / PL_SUB;           // 16 rows per slot
-constexpr uint32_t PL_BLOCK = PL_ROWS * 128;      // 64 channels x 16 rows (the LBO)
+constexpr int PL_ST = 3 * PL_SUB;                 // ring depth
+constexpr int PL_ROWS = WG_BR / PL_SUB;           // rows per slot
+constexpr uint32_t PL_BLOCK = PL_ROWS * 128;      // 64 channels x PL_ROWS rows (the LBO)
 constexpr uint32_t PL_PLANE = 2 * PL_BLOCK;       // 128 channels
 constexpr uint32_t PL_TILE = 4 * PL_PLANE;        // one operand's 4 planes
 constexpr uint32_t PL_SLOT = 2 * PL_TILE;         // dY spectrum, then X spectrum
@@ -570,7 +570,7 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int channels, int64_t N) 
 }
 
 // Spectral planes [4][N][channels] viewed as (64 channels, row, 64-channel
-// block, plane); box = (64, 16 rows, 2 blocks, 4 planes), 128-byte swizzle.
+// block, plane); box = (64, PL_ROWS rows, 2 blocks, 4 planes), 128-byte swizzle.
 // The block dimension steps by 128 B inside a row, so channels % 64 == 0 keeps
 // every block inside its row.
 bool encode_planes4_map(CUtensorMap* m, const void* base, int channels, int64_t N) {
