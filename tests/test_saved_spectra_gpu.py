@@ -208,3 +208,27 @@ def test_saved_spectra_error_paths():
     torch.cuda.synchronize()
     assert float(dW0.abs().sum()) == 0.0 and float(db0.abs().sum()) == 0.0
     assert p.status() == 0
+
+
+def test_dw_from_the_spectral_intermediate():
+    """A layer whose input arrives as the previous layer's spectral planes
+    (eqlinear_forward_to_spectral) passes those planes as its Xhat: dW then
+    equals the oracle's on the spatial input they represent (the inverse p4
+    transform of the planes, float64)."""
+    from group_circulant_gemm_b200 import EqLinearPlan
+    N, C0, C1, C2 = 777, 64, 128, 64
+    w1 = Workload("sp1", 4, N, C0, C1, "f16", True, 5400)
+    w2 = Workload("sp2", 4, N, C1, C2, "f16", True, 5401)
+    in1, in2 = make_inputs(w1), make_inputs(w2, need_dy=True)
+    p1 = EqLinearPlan(4, C0, C1, torch.float16)
+    p2 = EqLinearPlan(4, C1, C2, torch.float16)
+    Wh1, Wh2 = p1.prepare_weights(_dev(in1["W"])), p2.prepare_weights(_dev(in2["W"]))
+    H = p1.forward_to_spectral(_dev(in1["X"]), Wh1, _dev(in1["bias"]), act="gelu")
+    _, g2 = p2.backward_input_save_spectrum(_dev(in2["dY"]), Wh2)
+    dW, db = p2.backward_weight_from_spectra(H, g2)
+    assert p1.status() == 0 and p2.status() == 0
+    _, G = oracle.p4_transform_matrices()
+    Hs = np.einsum("tp,pnc->nct", G, H.double().cpu().numpy()).reshape(N, C1 * 4)
+    ref_w, ref_b = oracle.backward_weight(4, Hs, in2["dY"], C2)
+    assert _rel(dW.double().cpu().numpy(), ref_w) <= TOL16
+    assert _rel(db.double().cpu().numpy(), ref_b) <= TOL16
