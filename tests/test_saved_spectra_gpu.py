@@ -66,6 +66,7 @@ def _margins_intact(buf, pad, n):
 CASES = [
     # N, C, D, act
     (333, 64, 128, "none"),
+    (4096, 16, 48, "none"),     # the smallest widths the save calls take, whole row tiles
     (129, 128, 64, "gelu"),
     (1000, 192, 768, "none"),
     (1, 64, 64, "none"),
@@ -98,6 +99,8 @@ WG_CASES = [
     (1, 64, 64),
     (4097, 320, 192),
     (2000, 64, 384),
+    (8223, 64, 64),      # many row blocks, a ragged last stage
+    (129, 1024, 64),     # wide input: 8 in-channel tiles
 ]
 
 
