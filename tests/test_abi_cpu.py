@@ -76,6 +76,15 @@ def test_null_plan_calls_are_rejected(native):
     assert native.raw_status("eqlinear_backward_input", None, None, 4, None, None, None) == \
         native.EQL_ERR_INVALID_ARG
     assert native.raw_status("eqlinear_get_status", None, None) == native.EQL_ERR_INVALID_ARG
+    # the training-with-saved-spectra entries
+    assert native.raw_status("eqlinear_forward_save_spectrum", None, None, 4, None, None, 0,
+                             None, None, None) == native.EQL_ERR_INVALID_ARG
+    assert native.raw_status("eqlinear_backward_input_save_spectrum", None, None, 4, None, None,
+                             None, None) == native.EQL_ERR_INVALID_ARG
+    for name in ("eqlinear_backward_weight_from_spectra",
+                 "eqlinear_backward_weight_from_spectra_f32"):
+        assert native.raw_status(name, None, None, None, 4, None, None, None, 0, None) == \
+            native.EQL_ERR_INVALID_ARG
     assert native.eqlinear_prepared_weight_bytes(None) == 0
     assert native.eqlinear_backward_weight_workspace_bytes(None, 10) == 0
     native.eqlinear_plan_destroy(None)
