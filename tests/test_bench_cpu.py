@@ -1,0 +1,54 @@
+"""The bench's workload tables and algorithmic accounting (CPU only).
+
+The FLOP counts are the method's (per row: two real GEMMs per real frequency
+and four per complex frequency, "Algorithmic approach" item 2; D4: four
+characters and the 2 x 2 block), the dense comparator's are 2·N·(C·T)·(D·T);
+the traffic table must point at existing kernel sources.
+"""
+import os
+
+import bench
+from group_circulant_gemm_b200.synth import WORKLOADS
+
+
+def test_every_pipeline_resolves_and_chains():
+    for name, layers in bench.PIPELINES.items():
+        ws = [WORKLOADS[n] for n in layers]
+        for a, b in zip(ws, ws[1:]):
+            assert a.D == b.C and a.T == b.T and a.N == b.N, name
+        assert name in bench.DESCR, name
+    for name in bench.CHAINED | bench.SPECTRAL:
+        assert len(bench.PIPELINES[name]) == 2, name
+    for name in bench.BACKWARD:
+        assert name in bench.PIPELINES
+
+
+def test_flop_counts():
+    w4 = WORKLOADS["p4_vitb_fc1_f16"]      # T = 4: 2 real + 1 complex frequency
+    assert bench.layer_flops(w4) == 2.0 * 6 * w4.N * w4.C * w4.D
+    w8 = WORKLOADS["c8_1024_f16"]          # T = 8: 2 real + 3 complex
+    assert bench.layer_flops(w8) == 2.0 * 14 * w8.N * w8.C * w8.D
+    wd = WORKLOADS["p4m_vitb_fc1_f16"]     # D4: 4 characters + 2 x 2 block
+    assert bench.layer_flops(wd) == 2.0 * 12 * wd.N * wd.C * wd.D
+    # the dense layer the method replaces: 16·N·C·D multiply-adds at T = 4 against
+    # the method's 6·N·C·D
+    assert bench.dense_flops(w4) == 2.0 * w4.N * (w4.C * 4) * (w4.D * 4)
+    assert bench.wgrad_flops(w4) == bench.layer_flops(w4)
+
+
+def test_layer_bytes_counts_inputs_weights_outputs():
+    w = WORKLOADS["p4_vith_fc1_f16"]
+    planes = 4 + 1  # T = 4: frequencies 0 and 2, Re/Im of frequency 1, and -Im
+    assert bench.layer_bytes(w) == 2 * (w.N * w.C * 4 + w.N * w.D * 4 + planes * w.C * w.D + w.D)
+
+
+def test_traffic_table_refers_to_existing_sources():
+    csrc = os.path.join(bench.ROOT, "group_circulant_gemm_b200", "csrc")
+    for family, files in bench.KERNEL_SOURCES.items():
+        for f in files:
+            assert os.path.exists(os.path.join(csrc, f)), (family, f)
+    for (family, _), per_workload in bench.NCU_TRAFFIC.items():
+        assert family in bench.KERNEL_SOURCES
+        for workload, nbytes in per_workload.items():
+            assert workload in bench.PIPELINES or workload in bench.CONV_WORKLOADS
+            assert 1e6 < nbytes < 1e9
