@@ -9,6 +9,13 @@
 //   then for k = 1..NC : Re V[k], Im V[k]         (NC complex frequencies)
 // The prepared weights add NC more planes holding -Im of each complex frequency,
 // so that a tensor-core B operand can be a contiguous stack of planes.
+//
+// Range: every stored plane (prepared weights, and the input planes the
+// tensor-core kernels form or save) holds the DFT divided by Tp, the smallest
+// power of two >= T.  |V[k]| <= T max|v|, so a stored value never exceeds the
+// largest input magnitude and legal FP16 inputs cannot overflow to inf in an
+// FP16 plane; the division and the matching multiplication by Tp in every
+// consumer are exact (powers of two).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -37,6 +44,11 @@ struct Spec {
   // number of real multiply-adds per (row, out-channel, in-channel)
   static constexpr int macs = NR + 4 * NC;
 };
+
+// Tp: smallest power of two >= T; stored planes are the DFT times 1/Tp.
+__host__ __device__ constexpr int plane_pow2(int T) { return T <= 1 ? 1 : 2 * plane_pow2((T + 1) / 2); }
+template <int T>
+__host__ __device__ constexpr float plane_scale() { return 1.0f / plane_pow2(T); }
 
 __host__ __device__ inline int spec_nr(int T) { return (T % 2 == 0) ? 2 : 1; }
 __host__ __device__ inline int spec_nc(int T) { return (T - spec_nr(T)) / 2; }

@@ -17,7 +17,8 @@ namespace {
 
 // ---------------------------------------------------------------------------
 // prepare: W[D][C][T] -> forward planes [P][D][C] = conj(DFT(W)), adjoint planes
-// [P][C][D] = DFT(W) transposed.  One thread per (d, c).
+// [P][C][D] = DFT(W) transposed, both times 1/Tp (exact; the stored range never
+// exceeds max|W|).  One thread per (d, c).
 // conj(DFT(w))[k] = sum_u w[u] e^{+2 pi i k u/T}: Re = sum w cos, Im = +sum w sin.
 // ---------------------------------------------------------------------------
 template <int T, typename In>
@@ -59,10 +60,11 @@ __global__ void prepare_kernel(const In* __restrict__ W, int C, int D, In* __res
     im_adj[S::negim(k)] = b; // adjoint -Im
   }
   const int64_t plane = (int64_t)C * D;
+  constexpr float sc = plane_scale<T>();
 #pragma unroll
   for (int j = 0; j < S::P; ++j) {
-    fwd[j * plane + (int64_t)d * C + c] = from_f32<In>(re[j]);
-    adj[j * plane + (int64_t)c * D + d] = from_f32<In>(im_adj[j]);
+    fwd[j * plane + (int64_t)d * C + c] = from_f32<In>(re[j] * sc);
+    adj[j * plane + (int64_t)c * D + d] = from_f32<In>(im_adj[j] * sc);
   }
 }
 
@@ -147,7 +149,9 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(const In* __restrict__ X,
         // spectral plane j -> prepared plane: Re planes as-is, Im from the -Im slot
         int src = j;
         if (j >= S::NR && ((j - S::NR) & 1)) src = S::negim((j - S::NR) / 2 + 1);
-        if (c < Cin && d < Cout) v = to_f32(Wt[src * plane + (int64_t)c * Cout + d]);
+        // the stored planes carry 1/Tp: undo it exactly here
+        if (c < Cin && d < Cout)
+          v = to_f32(Wt[src * plane + (int64_t)c * Cout + d]) * (float)plane_pow2(T);
       }
       wreg[i] = v;
     }

@@ -79,8 +79,9 @@ struct PixelStore {
 };
 
 // Group DFT of every pixel's group vectors: X [P][C*4] -> planes [4][P][C]
-// (X0 = x0+x1+x2+x3, X2 = x0-x1+x2-x3, Xr = x0-x2, Xi = x3-x1; FP32, one
-// rounding).  One thread per pixel and 8 channels.
+// (X0 = x0+x1+x2+x3, X2 = x0-x1+x2-x3, Xr = x0-x2, Xi = x3-x1, each times 1/4
+// like every stored plane; FP32, one rounding).  One thread per pixel and 8
+// channels.
 __global__ void conv_planes_kernel(const uint4* __restrict__ X, int64_t P, int C,
                                    uint4* __restrict__ planes) {
   const int groups = C / 8;
@@ -100,10 +101,10 @@ __global__ void conv_planes_kernel(const uint4* __restrict__ X, int64_t P, int C
       const float2 lo = unpack_h2(w4[2 * hh]), hi = unpack_h2(w4[2 * hh + 1]);
       const float x0 = lo.x, x1 = lo.y, x2 = hi.x, x3 = hi.y;
       const float a = x0 + x2, b = x1 + x3;
-      f0[hh] = a + b;
-      fh[hh] = a - b;
-      fr[hh] = x0 - x2;
-      fi[hh] = x3 - x1;
+      f0[hh] = (a + b) * 0.25f;
+      fh[hh] = (a - b) * 0.25f;
+      fr[hh] = (x0 - x2) * 0.25f;
+      fi[hh] = (x3 - x1) * 0.25f;
     }
     o[0][q] = pack_h2(f0[0], f0[1]);
     o[1][q] = pack_h2(fh[0], fh[1]);

@@ -12,8 +12,10 @@
 //   y[s] = (Y_0 + (-1)^s Y_{T/2}) / T + (2/T) sum_k (Y_kr cos(2 pi k s/T) - Y_ki sin(2 pi k s/T))
 // For T = 4 the transforms are adds only (X0 = x0+x1+x2+x3, X2 = x0-x1+x2-x3,
 // Xr = x0-x2, Xi = x3-x1); for T = 8 a radix-2 split leaves one non-dyadic
-// twiddle, sqrt(2)/2.  The inverse's factors 1/T and 2/T are folded into the
-// weight tiles, so the epilogue is adds only.
+// twiddle, sqrt(2)/2.  Both operands' planes hold the DFT times 1/T (exact), so
+// an FP16 plane never exceeds the largest input magnitude (no overflow for any
+// finite FP16 input); the epilogue multiplies the accumulators by T (real
+// frequencies) and 2T (complex), which gives the inverse's 1/T and 2/T terms.
 //
 // Template parameters: ACT = output activation (0 none, 1 GELU, fused into the
 // epilogue); IO (T = 4) = spatial X and Y, or Y written as the next layer's
@@ -365,13 +367,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // image: blob (dt, ks) = regions 0..T-1 (prepared planes 0..T-1: real frequency
 // 0, real frequency T/2, then Re and Im of each complex frequency), each BD rows
 // x BK channels in the K-major swizzled layout the MMAs read; rows and channels
-// past the matrix are zero.  One thread per 16-byte piece.  Regions below nreal
-// hold one-dimensional frequencies (inverse factor 1/T), the others entries of
-// two-dimensional ones (2/T): nreal = 2 for the cyclic groups of even order, 4 for D4.
+// past the matrix are zero.  One thread per 16-byte piece.  The values are the
+// prepared planes unchanged (the DFT times 1/T); the epilogue applies the
+// inverse transform's factors.
 template <int T>
 __global__ void tile_weights_kernel(const __half* __restrict__ planes, int Cin, int Cout,
-                                    int n_ks, int64_t n_chunks, int nreal,
-                                    uint4* __restrict__ tiles) {
+                                    int n_ks, int64_t n_chunks, uint4* __restrict__ tiles) {
   using S = Shape<T>;
   constexpr int kPieces = S::ROWB / 16;  // 16-byte pieces per row
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -383,15 +384,8 @@ __global__ void tile_weights_kernel(const __half* __restrict__ planes, int Cin, 
   const int dt = (int)(blob / n_ks), ks = (int)(blob % n_ks);
   const int d = dt * S::BD + r, c0 = ks * S::BK + piece * 8;
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
-  if (d < Cout && c0 < Cin) {  // Cin % 16 == 0: the 8 channels are all in range
+  if (d < Cout && c0 < Cin)  // Cin % 16 == 0: the 8 channels are all in range
     v = *reinterpret_cast<const uint4*>(planes + ((int64_t)region * Cout + d) * Cin + c0);
-    // the inverse DFT's factors 1/T (real frequencies) and 2/T (complex), exact
-    // powers of two, applied here so the epilogue needs no multiplies by them
-    const __half2 s = __float2half2_rn(region < nreal ? 1.f / T : 2.f / T);
-    __half2* h = reinterpret_cast<__half2*>(&v);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __hmul2(h[i], s);
-  }
   // swizzle: piece ^= (byte offset of the row >> 7) within the swizzle span
   const int swz = ((r * S::ROWB) >> 7) & (kPieces - 1);
   const int64_t dst_byte = blob * S::W_STAGE_BYTES + (int64_t)region * S::WREG_BYTES +
@@ -439,8 +433,7 @@ cudaError_t launch_tile_weights(int T, const void* planes, int Cin, int Cout, vo
     const int64_t n_chunks = (int64_t)tc_tile_bytes(TT, Cin, Cout) / 16;
     const unsigned blocks = (unsigned)((n_chunks + 255) / 256);
     tile_weights_kernel<TT><<<blocks, 256, 0, st>>>(static_cast<const __half*>(planes), Cin, Cout,
-                                                    n_ks, n_chunks, group ? 4 : 2,
-                                                    static_cast<uint4*>(tiles));
+                                                    n_ks, n_chunks, static_cast<uint4*>(tiles));
     return cudaGetLastError();
   });
 }
@@ -468,7 +461,8 @@ cudaError_t set_smem_attr() {
 
 // D4 weight spectrum, in the tile regions' order: W^(rho) = sum_u W(u) rho(u)
 // for the characters (+,+), (+,-), (-,+), (-,-) and the 2 x 2 entries 00, 10,
-// 01, 11 (region 4 + 2j + k holds entry [k][j]); FP32, one rounding.
+// 01, 11 (region 4 + 2j + k holds entry [k][j]), times 1/8 like every stored
+// plane (exact); FP32, one rounding.
 // W [D][C][8] -> planes [8][D][C].  One thread per (d, c).
 __global__ void prepare_d4_kernel(const __half* __restrict__ W, int C, int D,
                                   __half* __restrict__ planes) {
@@ -487,7 +481,7 @@ __global__ void prepare_d4_kernel(const __half* __restrict__ W, int C, int D,
                       d5 - d1,   // [0][1]
                       d0 - d4};  // [1][1]
 #pragma unroll
-  for (int r = 0; r < 8; ++r) planes[r * plane + idx] = __float2half_rn(v[r]);
+  for (int r = 0; r < 8; ++r) planes[r * plane + idx] = __float2half_rn(v[r] * 0.125f);
 }
 
 }  // namespace

@@ -126,7 +126,10 @@ __device__ __forceinline__ UnitPos unit_pos(int u, const TileInfo& ti) {
 // line L = 2r + c swizzled by (L % 8).  A thread reads eight 16-byte pieces and,
 // once every transform warp holds its pieces, writes its share of the planes.
 // Lane mapping: an 8-lane phase covers 4 rows x both chunks, so its swizzled
-// reads and writes hit 8 distinct bank groups.
+// reads and writes hit 8 distinct bank groups.  The planes are the DFT times
+// 1/T (T = 4, 8: exact), so an FP16 plane never exceeds the largest input
+// magnitude; the weight planes carry the same factor and the epilogue
+// multiplies it out.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 f2(uint32_t u) { return unpack_h2(u); }
 
@@ -177,11 +180,12 @@ __device__ __forceinline__ void xf_write(uint8_t* slot, int xt, const uint4 (&v)
         for (int hh = 0; hh < 2; ++hh) {
           const float2 lo = f2(w4[2 * hh]), hi = f2(w4[2 * hh + 1]);
           const float x0 = lo.x, x1 = lo.y, x2 = hi.x, x3 = hi.y;
+          // stored planes carry 1/4 (exact), so |plane| <= max|x|
           const float a = x0 + x2, b = x1 + x3;
-          f0[hh] = a + b;
-          fh[hh] = a - b;
-          fr[hh] = x0 - x2;
-          fi[hh] = x3 - x1;
+          f0[hh] = (a + b) * 0.25f;
+          fh[hh] = (a - b) * 0.25f;
+          fr[hh] = (x0 - x2) * 0.25f;
+          fi[hh] = (x3 - x1) * 0.25f;
         }
         o0[i] = pack_h2(f0[0], f0[1]);
         o2[i] = pack_h2(fh[0], fh[1]);
@@ -242,8 +246,9 @@ __device__ __forceinline__ void xf_write(uint8_t* slot, int xt, const uint4 (&v)
         val[6][hh] = b0 - s13;
         val[7][hh] = b2 - t13;
       }
+      // stored planes carry 1/8 (exact), so |plane| <= max|x|
 #pragma unroll
-      for (int p = 0; p < 8; ++p) o[p][pr] = pack_h2(val[p][0], val[p][1]);
+      for (int p = 0; p < 8; ++p) o[p][pr] = pack_h2(val[p][0] * 0.125f, val[p][1] * 0.125f);
     }
     // K-major 32 B rows: 16-byte piece c at (c ^ ((r / 4) % 2))
     const uint32_t off = r * 32 + ((c ^ ((r >> 2) & 1)) << 4);
@@ -285,14 +290,16 @@ __device__ __forceinline__ void epi_half(uint32_t lane_addr, int c0, const __hal
   }
   tmem_wait_ld();
   if constexpr (T == 4) {
-    // accumulators arrive scaled (Y0/4, Y2/4, Yr/2, Yi/2):
+    // Both operands carry 1/4, so the accumulators hold Y/16; the exact factors 4
+    // (real frequencies) and 8 (complex) give the inverse transform's scaled terms
+    // Y0' = Y0/4, Y2' = Y2/4, Yr' = Yr/2, Yi' = Yi/2:
     // y0 = Y0'+Y2'+Yr', y1 = Y0'-Y2'-Yi', y2 = Y0'+Y2'-Yr', y3 = Y0'-Y2'+Yi' (+ bias)
     uint32_t w[2 * NCH];
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
-      const float s = __uint_as_float(v[0][i]) + b[i];
-      const float y2 = __uint_as_float(v[1][i]);
-      const float yr = __uint_as_float(v[2][i]), yi = __uint_as_float(v[3][i]);
+      const float s = fmaf(4.f, __uint_as_float(v[0][i]), b[i]);
+      const float y2 = 4.f * __uint_as_float(v[1][i]);
+      const float yr = 8.f * __uint_as_float(v[2][i]), yi = 8.f * __uint_as_float(v[3][i]);
       const float e = s + y2, od = s - y2;
       w[2 * i] = pack_h2(act_fn<ACT>(e + yr), act_fn<ACT>(od - yi));
       w[2 * i + 1] = pack_h2(act_fn<ACT>(e - yr), act_fn<ACT>(od + yi));
@@ -300,16 +307,20 @@ __device__ __forceinline__ void epi_half(uint32_t lane_addr, int c0, const __hal
 #pragma unroll
     for (int m = 0; m < 4; ++m) o[m] = make_uint4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
   } else {
-    // accumulators arrive scaled (frequencies 0 and 4 by 1/8, complex by 1/4);
-    // y_s = A_s + B_s, y_{s+4} = A_s - B_s (A: frequencies 0, 2, 4; B: 1, 3)
+    // Both operands carry 1/8, so the accumulators hold Y/64; the exact factors 8
+    // (frequencies 0 and 4) and 16 (complex) give the inverse transform's terms
+    // Y/8 and Y/4.  y_s = A_s + B_s, y_{s+4} = A_s - B_s (A: frequencies 0, 2, 4;
+    // B: 1, 3)
     const float h = 0.70710678118654752f;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       float Yv[8];
+      // cyclic T = 8: planes 0, 1 real; D4: planes 0..3 characters (both x 8)
+      constexpr int kReal = (G == 1) ? 4 : 2;
 #pragma unroll
-      for (int p = 0; p < 8; ++p) Yv[p] = __uint_as_float(v[p][i]);
+      for (int p = 0; p < 8; ++p) Yv[p] = (p < kReal ? 8.f : 16.f) * __uint_as_float(v[p][i]);
       if constexpr (G == 1) {
-        // D4, accumulators arrive scaled (characters by 1/8, the 2 x 2 block by 2/8):
+        // D4, after the factors: characters' terms Y/8, the 2 x 2 block's Y/4:
         // y(g) = sum_p chi_p(g) c_p + sum_{i,k} rho(g)_ik m_ik  (+ bias), g = a + 4b
         const float s = Yv[0] + b[i];
         const float P = s + Yv[2], Q = s - Yv[2], U = Yv[1] + Yv[3], V = Yv[1] - Yv[3];
@@ -339,8 +350,9 @@ __device__ __forceinline__ void epi_half(uint32_t lane_addr, int c0, const __hal
 
 // T = 4 epilogue of 8 out-channels written as the NEXT layer's input in the
 // frequency domain: per channel the four outputs y_s = act(IDFT + bias) are
-// transformed again, X0 = y0+y1+y2+y3, X2 = y0-y1+y2-y3, Xr = y0-y2, Xi = y3-y1
-// (FP32, one rounding to FP16); o[p] = plane p of the 8 channels (16 bytes).
+// transformed again, X0 = y0+y1+y2+y3, X2 = y0-y1+y2-y3, Xr = y0-y2, Xi = y3-y1,
+// each times 1/4 (FP32, one rounding to FP16); o[p] = plane p of the 8 channels
+// (16 bytes).
 template <int BD, int ACT>
 __device__ __forceinline__ void epi_half_spec(uint32_t lane_addr, int c0, const __half* bsm,
                                               uint4 (&o)[4]) {
@@ -358,17 +370,19 @@ __device__ __forceinline__ void epi_half_spec(uint32_t lane_addr, int c0, const 
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int i = 2 * m + e;
-      const float sb = __uint_as_float(v[0][i]) + (e ? bf.y : bf.x);
-      const float y2 = __uint_as_float(v[1][i]);
-      const float yr = __uint_as_float(v[2][i]), yi = __uint_as_float(v[3][i]);
+      // accumulators hold Y/16: factors 4 and 8 as in epi_half
+      const float sb = fmaf(4.f, __uint_as_float(v[0][i]), e ? bf.y : bf.x);
+      const float y2 = 4.f * __uint_as_float(v[1][i]);
+      const float yr = 8.f * __uint_as_float(v[2][i]), yi = 8.f * __uint_as_float(v[3][i]);
       const float ev = sb + y2, od = sb - y2;
       const float z0 = act_fn<ACT>(ev + yr), z1 = act_fn<ACT>(od - yi);
       const float z2 = act_fn<ACT>(ev - yr), z3 = act_fn<ACT>(od + yi);
+      // the next layer's planes carry 1/4 like every stored plane
       const float a = z0 + z2, b = z1 + z3;
-      q[0][e] = a + b;
-      q[1][e] = a - b;
-      q[2][e] = z0 - z2;
-      q[3][e] = z3 - z1;
+      q[0][e] = (a + b) * 0.25f;
+      q[1][e] = (a - b) * 0.25f;
+      q[2][e] = (z0 - z2) * 0.25f;
+      q[3][e] = (z3 - z1) * 0.25f;
     }
 #pragma unroll
     for (int p = 0; p < 4; ++p) pl[p][m] = pack_h2(q[p][0], q[p][1]);

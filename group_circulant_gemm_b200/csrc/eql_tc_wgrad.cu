@@ -10,7 +10,9 @@
 // summed over a range of rows and stored as FP32 partial planes; dbias partials
 // are the FP32 column sums of G0.  A finalize kernel adds a tile's partials in a
 // fixed order, applies the inverse group DFT and casts, so the result is
-// deterministic.
+// deterministic.  The FP16 operand planes hold G/4 and Xh/4 (exact), like every
+// stored plane of the library, so no legal FP16 input overflows them; the
+// partials are therefore Q/16 and the finalize multiplies by 16.
 //
 // Work split (stream-K over rows): the (tile, 32-row stage) space, tile = 128
 // out-channels x 128 in-channels, is cut into equal contiguous ranges, one per
@@ -207,7 +209,12 @@ __device__ __forceinline__ void wg_transform(uint8_t* tile, int w, int j, int q,
         p2[h] = s02 - s13;
         pr[h] = g0 - g2;
         pi[h] = g3 - g1;
-        if (kBias) bsum[e] += p0[h];
+        if (kBias) bsum[e] += p0[h];  // dbias: the unscaled FP32 G0
+        // stored planes carry 1/4 (exact)
+        p0[h] *= 0.25f;
+        p2[h] *= 0.25f;
+        pr[h] *= 0.25f;
+        pi[h] *= 0.25f;
       }
       o[0][e][m] = pack_h2(p0[0], p0[1]);
       o[1][e][m] = pack_h2(p2[0], p2[1]);
@@ -436,7 +443,8 @@ __global__ void __launch_bounds__(PL ? WG_THREADS_PL : WG_THREADS, 1)
         if (lane == 0) mbar_arrive(&bars->empty[slot]);
       }
       if (!ok) break;
-      if (un.ct == 0) bpart[(int64_t)un.slot * WG_BD + dl] = b;
+      // the saved plane 0 holds G0/4: the sum times 4 (exact) is the sum of G0
+      if (un.ct == 0) bpart[(int64_t)un.slot * WG_BD + dl] = 4.f * b;
     }
   } else if (!PL && warp >= WG_XF0) {
     // ---------------- transform: group DFT, transposed into the operand planes ----------------
@@ -531,6 +539,9 @@ __global__ void __launch_bounds__(256)
           for (int p = 0; p < 4; ++p) qv[p] += slot[p * (WG_BC * WG_BD) + off];
         }
       }
+      // both operand planes carried 1/4: the partial sums are Q/16
+#pragma unroll
+      for (int p = 0; p < 4; ++p) qv[p] *= 16.f;
       float wv[4];
       group_idft<4>(qv, wv, tw);
       *reinterpret_cast<float4*>(&s[w][4 * lane]) = make_float4(wv[0], wv[1], wv[2], wv[3]);

@@ -144,3 +144,50 @@ def make_conv_inputs(w: ConvWorkload, images: int | None = None):
     dt = np.float16 if w.dtype == "f16" else np.float32
     return {"X": np.ascontiguousarray(X.astype(dt)), "Wc": np.ascontiguousarray(Wc.astype(dt)),
             "bias": np.ascontiguousarray(b.astype(dt))}
+
+
+# Extreme group vectors for the FP16 range tests: for each group order, sign
+# patterns that put the largest possible magnitude into one frequency
+# (constant, alternating, and the sign patterns of the first harmonics).  Plain
+# integer tables: a planted group is amplitude * pattern.
+RANGE_PATTERNS = {
+    3: [[1, 1, 1], [1, -1, -1], [0, 1, -1]],
+    4: [[1, 1, 1, 1], [1, -1, 1, -1], [1, 0, -1, 0], [0, -1, 0, 1], [1, 1, -1, -1]],
+    8: [[1] * 8, [1, -1] * 4, [1, 1, 0, -1, -1, -1, 0, 1], [0, -1, -1, -1, 0, 1, 1, 1],
+        [1, 0, -1, 0] * 2, [1, -1, 0, 1, -1, 1, 0, -1], [1, 1, -1, -1] * 2],
+}
+
+
+def make_range_inputs(seed: int, T: int, N: int, C: int, D: int,
+                      x=(1.0, 0.0), w=(1.0, 0.0), dy=(1.0, 0.0), need_dy: bool = False,
+                      dtype: str = "f16"):
+    """Inputs that reach the edge of the FP16 range.
+
+    Each of X [N, C*T], W [D, C, T], dY [N, D*T] is given as (fill, amp): every
+    entry is first drawn as fill * U(-1, 1) (W's fill also times 1/sqrt(C*T)),
+    then about one group vector in four is replaced by amp * (a random pattern
+    of RANGE_PATTERNS[T]) * (random sign), so that a group's DFT reaches T * amp.
+    bias ~ N(0, 0.01).  Draw order: X, W, bias, dY, each array's uniform fill,
+    then its group mask, pattern choice and signs.  Cast with round-to-nearest."""
+    rng = np.random.default_rng(seed)
+    pats = np.asarray(RANGE_PATTERNS[T], dtype=np.float64)
+
+    def draw(shape_groups, fill, amp):
+        a = rng.uniform(-1.0, 1.0, shape_groups + (T,)) * fill
+        mask = rng.uniform(0.0, 1.0, shape_groups) < 0.25
+        which = rng.integers(0, len(pats), shape_groups)
+        sign = np.where(rng.uniform(0.0, 1.0, shape_groups) < 0.5, -1.0, 1.0)
+        if amp > 0:
+            a = np.where(mask[..., None], amp * sign[..., None] * pats[which], a)
+        return a
+
+    X = draw((N, C), *x).reshape(N, C * T)
+    W = draw((D, C), w[0] / np.sqrt(C * T), w[1])
+    b = rng.standard_normal((D,)) * np.sqrt(0.01)
+    dY = draw((N, D), *dy).reshape(N, D * T) if need_dy else None
+    dt = np.float32 if dtype == "f32" else np.float16
+    out = {"X": np.ascontiguousarray(X.astype(dt)), "W": np.ascontiguousarray(W.astype(dt)),
+           "bias": np.ascontiguousarray(b.astype(dt))}
+    if dY is not None:
+        out["dY"] = np.ascontiguousarray(dY.astype(dt))
+    return out

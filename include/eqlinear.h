@@ -135,12 +135,14 @@ EQL_API const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t plan, i
  * (even T); Re and Im of each complex frequency k = 1..n_cplx; then -Im of each
  * complex frequency.  Forward planes hold conj(DFT(W)) (the correlation form of
  * the convolution theorem), adjoint planes hold DFT(W) transposed, used for dX.
+ * Every plane is stored times 1/Tp, Tp the smallest power of two >= T (exact):
+ * a DFT coefficient is at most T max|W| in magnitude, so a stored value never
+ * exceeds max|W| and no finite FP16 weight overflows its plane.
  * For FP16 plans with T = 4 or 8 and C, D multiples of 16 two more blocks
  * follow: the forward and adjoint planes re-arranged as the tensor-core
  * kernel's operand tiles (one contiguous blob per out-channel tile and K stage:
  * 128 x 32 channels at T = 4, 64 x 16 at T = 8, in the kernel's swizzled
- * shared-memory order, scaled by the inverse DFT's factors 1/T and 2/T), so each
- * pipeline stage is one copy.
+ * shared-memory order, the same values), so each pipeline stage is one copy.
  */
 EQL_API size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t plan);
 
@@ -196,9 +198,11 @@ EQL_API eqlinear_status_t eqlinear_forward_act(eqlinear_plan_t plan, const void*
  * second layer's forward DFT can be taken by the first layer's epilogue).
  *
  * eqlinear_forward_to_spectral writes, instead of Y, the group DFT of
- * act(Y) as four FP16 planes Xhat[4][N][D] (plane 0: sum over s, 1: alternating
- * sum, 2: y0 - y2, 3: y3 - y1; FP32 arithmetic, one rounding), which is the
- * input a following p4 layer multiplies directly.  eqlinear_forward_from_spectral
+ * act(Y) as four FP16 planes Xhat[4][N][D], each value times 1/4 (plane 0: sum
+ * over s, 1: alternating sum, 2: y0 - y2, 3: y3 - y1, then / 4; FP32 arithmetic,
+ * one rounding; the factor keeps every plane within max|act(Y)|, so no finite
+ * FP16 activation overflows), which is the input a following p4 layer
+ * multiplies directly.  eqlinear_forward_from_spectral
  * is the forward of a layer whose input arrives as such planes Xhat[4][N][C]
  * (Y [N][D*T], optional bias and act as in eqlinear_forward_act).  Chaining the
  * two equals eqlinear_forward_act followed by eqlinear_forward up to rounding.
@@ -275,7 +279,7 @@ EQL_API eqlinear_status_t eqlinear_forward_chain(eqlinear_plan_t first, eqlinear
  *   eqlinear_conv_prepare_weights: Wc [KH][KW][D][C][T] (tap-major; each tap a
  *     contiguous [D][C][T] block) -> Wc_hat, once per weight update.
  *   eqlinear_conv_workspace_bytes(plan, N, H, W): scratch of eqlinear_conv_forward
- *     (the group DFT of X as FP16 planes, 4 * N * H * W * C * 2 bytes).
+ *     (the group DFT of X times 1/4 as FP16 planes, 4 * N * H * W * C * 2 bytes).
  *   eqlinear_conv_forward: X [N][H][W][C*T] (feature index c*T+t, pixels
  *     row-major), Y [N][Ho][Wo][D*T], bias [D] or NULL, act as in
  *     eqlinear_forward_act.  All pointers 16-byte aligned; the caller owns every
@@ -354,16 +358,17 @@ EQL_API eqlinear_status_t eqlinear_backward_weight_f32(eqlinear_plan_t plan, con
  * multiplies them directly and runs no transform of its own:
  *
  * eqlinear_forward_save_spectrum: eqlinear_forward_act (Y bitwise the same),
- *   and also Xhat [4][N][C], the group DFT of X (plane 0: x0+x1+x2+x3, 1:
- *   x0-x1+x2-x3, 2: x0-x2, 3: x3-x1; FP32 arithmetic, one rounding to FP16),
- *   the planes order of eqlinear_forward_to_spectral.
+ *   and also Xhat [4][N][C], the group DFT of X times 1/4 (plane 0:
+ *   (x0+x1+x2+x3)/4, 1: (x0-x1+x2-x3)/4, 2: (x0-x2)/4, 3: (x3-x1)/4; FP32
+ *   arithmetic, one rounding to FP16; no finite FP16 input overflows), the
+ *   planes order and scale of eqlinear_forward_to_spectral.
  * eqlinear_backward_input_save_spectrum: eqlinear_backward_input (dX bitwise
  *   the same), and also dYhat [4][N][D], the group DFT of dY in that order.
  * eqlinear_backward_weight_from_spectra (and _f32, as eqlinear_backward_weight
  *   _f32): eqlinear_backward_weight from Xhat and dYhat instead of X and dY,
  *   with the same workspace (eqlinear_backward_weight_workspace_bytes).  dW's
  *   operands are the same FP16 values the transforming kernel forms; dbias sums
- *   dYhat's plane 0 (already rounded to FP16) instead of the FP32 sums.
+ *   dYhat's plane 0 (already rounded to FP16) times 4 instead of the FP32 sums.
  *   A layer whose input arrives as the planes of eqlinear_forward_to_spectral
  *   may pass them as its Xhat.
  *

@@ -349,10 +349,11 @@ def test_forward_act_rejects_unknown_activation():
 # --- two-layer block with the intermediate in the frequency domain -------------------
 
 def _planes_of(Y, H):
-    """float64 group DFT of a [N, H*4] activation: planes [4, N, H] in the kernel's order."""
+    """float64 group DFT of a [N, H*4] activation: planes [4, N, H] in the kernel's order,
+    times 1/4 (the scale of every stored plane)."""
     g = Y.reshape(Y.shape[0], H, 4)
-    return np.stack([g.sum(axis=2), g[..., 0] - g[..., 1] + g[..., 2] - g[..., 3],
-                     g[..., 0] - g[..., 2], g[..., 3] - g[..., 1]])
+    return 0.25 * np.stack([g.sum(axis=2), g[..., 0] - g[..., 1] + g[..., 2] - g[..., 3],
+                            g[..., 0] - g[..., 2], g[..., 3] - g[..., 1]])
 
 
 BLOCK_CASES = [

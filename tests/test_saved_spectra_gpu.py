@@ -3,7 +3,7 @@
 The forward and dX kernels can also store the group DFTs they form (of X and
 of dY); the weight gradient then multiplies those planes directly.  Checks:
   * Y and dX are bitwise those of the plain calls;
-  * the saved planes are the real 4-point DFT of the input rows (the oracle's
+  * the saved planes are the real 4-point DFT of the input rows times 1/4 (the oracle's
     p4 transform matrix, float64) up to the one FP16 rounding;
   * dW and dbias from the spectra match the float64 oracle (FP16 tolerance
     2e-3 of max|ref|) and the transforming weight-gradient kernel;
@@ -39,10 +39,11 @@ def _setup(N, C, D, seed):
 
 
 def _planes_ref(rows, channels):
-    """float64 planes [4, N, channels] of rows [N, channels * 4]."""
+    """float64 planes [4, N, channels] of rows [N, channels * 4], times 1/4 (the scale
+    of every stored plane)."""
     F, _ = oracle.p4_transform_matrices()
     x = rows.astype(np.float64).reshape(rows.shape[0], channels, 4)
-    return np.einsum("pt,nct->pnc", F, x)
+    return 0.25 * np.einsum("pt,nct->pnc", F, x)
 
 
 def _check_planes(got, ref):
@@ -231,7 +232,8 @@ def test_dw_from_the_spectral_intermediate():
     dW, db = p2.backward_weight_from_spectra(H, g2)
     assert p1.status() == 0 and p2.status() == 0
     _, G = oracle.p4_transform_matrices()
-    Hs = np.einsum("tp,pnc->nct", G, H.double().cpu().numpy()).reshape(N, C1 * 4)
+    # the planes carry 1/4: four times them are the plain DFT that G inverts
+    Hs = np.einsum("tp,pnc->nct", G, 4.0 * H.double().cpu().numpy()).reshape(N, C1 * 4)
     ref_w, ref_b = oracle.backward_weight(4, Hs, in2["dY"], C2)
     assert _rel(dW.double().cpu().numpy(), ref_w) <= TOL16
     assert _rel(db.double().cpu().numpy(), ref_b) <= TOL16
