@@ -414,18 +414,24 @@ EQL_API eqlinear_status_t eqlinear_cast_from_f32(eqlinear_plan_t plan, const flo
  * at start-up, or who must not call cudaMalloc/cudaFree (those calls can
  * synchronise the whole device) on a latency-critical path.
  *
- * Computes exactly what eqlinear_backward_weight computes (same arguments minus
- * the workspace), but keeps the FP32 partial spectra of the split reduction in a
- * scratch array that the library reserves statically: 16 MiB (4,194,304 floats)
- * per GPU on which the library is loaded, held until the process exits.
+ * Computes what eqlinear_backward_weight computes (same arguments minus the
+ * workspace), always with the CUDA-core kernels (wgrad_simt + finalize), and
+ * keeps the FP32 partial spectra of their split reduction over rows in a
+ * scratch array that the library reserves statically: 16 MiB (4,194,304
+ * floats) per GPU on which the library is loaded, held until the process exits.
+ *   - Kernels: for FP16 plans with T = 4 the workspace entry runs the tensor
+ *     cores, so the two can differ in rounding (both within the FP16 accuracy
+ *     target) and in speed; a plan forced to EQL_KERNEL_TCGEN05 is rejected
+ *     with EQL_ERR_UNSUPPORTED.
  *   - Size limit: one row split needs T*C*D + D floats; plans above 4,194,304
  *     floats are rejected with EQL_ERR_WORKSPACE before anything is launched.
- *     When the usual number of splits does not fit, fewer splits are used, so
- *     results can differ from eqlinear_backward_weight in rounding only.
+ *     When the usual number of splits does not fit, fewer splits are used (at
+ *     T = 4, C = 320, D = 1280 only 2 fit, so the row reduction runs on fewer,
+ *     longer CTAs and is several times slower than the workspace entry).
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
- *   - The first call on each device looks up the scratch array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *   - The first call in each CUDA context looks up the scratch array's device
+ *     address (cudaGetSymbolAddress) in that context and remembers it; make that
+ *     first call before any stream capture.
  *   - Every call on a GPU shares the one scratch array and leaves its contents
  *     behind; each call writes every scratch element before reading it, so no
  *     clearing is needed, but calls whose executions overlap on the GPU (other
