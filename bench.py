@@ -306,17 +306,75 @@ def calibrated_oracle_rows(pipeline, target_s: float, backward: bool = False, ac
     return int(max(16, min(n_full, 16 * target_s / max(t, 1e-6))))
 
 
+def reference_step_seconds(args) -> float:
+    """Host-oracle seconds per step of the reference arm: the whole run (warm-up
+    + timed steps) takes about two minutes, at most 20 s a step, unless
+    --ref-seconds sets it."""
+    if args.ref_seconds is not None:
+        return max(1e-3, args.ref_seconds)
+    return min(20.0, max(1.0, 120.0 / max(1, args.steps + args.warmup)))
+
+
+def layer_cpu_baseline(workload, backward: bool, N: int) -> dict:
+    """The oracle on the host cores, a calibrated sample (~15 s with all threads,
+    ~5 s with one) through every op of the step; rows/s."""
+    import oracle
+    pipeline, acts = PIPELINES[workload], acts_of(workload)
+    rows = calibrated_oracle_rows(pipeline, 15.0, backward, acts)
+    secs, rows = oracle_sample(pipeline, rows, backward, acts)
+    cores = oracle.threads_used()
+    oracle.set_threads(1)
+    try:
+        rows1 = calibrated_oracle_rows(pipeline, 5.0, backward, acts)
+        secs1, rows1 = oracle_sample(pipeline, rows1, backward, acts)
+    finally:
+        oracle.set_threads(None)
+    return {"value": rows / secs, "unit": "tokens/s", "cores": cores,
+            "cpu_model": oracle.cpu_model(), "kind": "oracle",
+            "sample": f"{rows} of {N} rows through every op of the step, float64, "
+                      f"{secs:.1f} s",
+            "value_1thread": rows1 / secs1,
+            "sample_1thread": f"{rows1} rows, 1 thread, {secs1:.1f} s"}
+
+
+def conv_cpu_baseline(w) -> dict:
+    """The convolution oracle on the host cores (~15 s) and on one thread (~5 s)."""
+    import oracle
+    images = conv_oracle_images(w, 15.0)
+    secs = conv_oracle_sample(w, images)
+    cores = oracle.threads_used()
+    oracle.set_threads(1)
+    try:
+        images1 = conv_oracle_images(w, 5.0)
+        secs1 = conv_oracle_sample(w, images1)
+    finally:
+        oracle.set_threads(None)
+    return {"value": images * w.Ho * w.Wo / secs, "unit": "tokens/s", "cores": cores,
+            "cpu_model": oracle.cpu_model(), "kind": "oracle",
+            "sample": f"{images} of {w.N} images, float64, {secs:.1f} s",
+            "value_1thread": images1 * w.Ho * w.Wo / secs1,
+            "sample_1thread": f"{images1} images, 1 thread, {secs1:.1f} s"}
+
+
+def use_all_host_cores(world: int) -> None:
+    """Under a launcher with several ranks (torchrun sets OMP_NUM_THREADS=1 per
+    rank) rank 0 runs the host oracle alone, so it gets every core it may use."""
+    if world > 1:
+        import oracle
+        oracle.set_threads(len(os.sched_getaffinity(0)))
+
+
 def run_reference(args, workload):
     """Reference arm: the float64 oracle on the host cores, bounded sample per step."""
     import oracle
     world, rank, _ = dist_init()
     if rank != 0:
         return 0
+    use_all_host_cores(world)
     pipeline = PIPELINES[workload]
     backward = workload in BACKWARD
-    per_step_s = max(1.0, 120.0 / max(1, args.steps + args.warmup))
     acts = acts_of(workload)
-    rows = calibrated_oracle_rows(pipeline, min(per_step_s, 20.0), backward, acts)
+    rows = calibrated_oracle_rows(pipeline, reference_step_seconds(args), backward, acts)
     for _ in range(args.warmup):
         oracle_sample(pipeline, rows, backward, acts)
     times = [oracle_sample(pipeline, rows, backward, acts)[0] for _ in range(args.steps)]
@@ -325,13 +383,13 @@ def run_reference(args, workload):
     w0 = WORKLOADS[pipeline[0]]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": DESCR[workload], "rows_per_step": rows, "global_batch": w0.N,
                    "seq_len": None, "parallelism": "none (host oracle)"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads_used(),
-                         "kind": "oracle",
+                         "cpu_model": oracle.cpu_model(), "kind": "oracle",
                          "sample": f"{rows} of {w0.N} rows per step through every layer"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -775,13 +833,7 @@ def run_ours(args, workload):
             comparator["ours_over_dense"] = value / comparator["value"]
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            import oracle
-            rows = calibrated_oracle_rows(PIPELINES[workload], 15.0, backward, acts_of(workload))
-            secs, rows = oracle_sample(PIPELINES[workload], rows, backward, acts_of(workload))
-            cpu = {"value": rows / secs, "unit": "tokens/s", "cores": oracle.threads_used(),
-                   "kind": "oracle",
-                   "sample": f"{rows} of {N} rows through every op of the step, float64, "
-                             f"{secs:.1f} s"}
+            cpu = layer_cpu_baseline(workload, backward, N)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -858,9 +910,9 @@ def run_conv_reference(args, workload):
     world, rank, _ = dist_init()
     if rank != 0:
         return 0
+    use_all_host_cores(world)
     w = CONV_WORKLOADS[workload]
-    per_step_s = max(1.0, 120.0 / max(1, args.steps + args.warmup))
-    images = conv_oracle_images(w, min(per_step_s, 20.0))
+    images = conv_oracle_images(w, reference_step_seconds(args))
     for _ in range(args.warmup):
         conv_oracle_sample(w, images)
     times = [conv_oracle_sample(w, images) for _ in range(args.steps)]
@@ -869,14 +921,14 @@ def run_conv_reference(args, workload):
     sample = f"{images} of {w.N} images per step"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": CONV_DESCR[workload], "images_per_step": images,
                    "global_batch": w.N, "seq_len": None, "parallelism": "none (host oracle)",
                    "tokens": "output pixels"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads_used(),
-                         "kind": "oracle", "sample": sample},
+                         "cpu_model": oracle.cpu_model(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -1062,12 +1114,7 @@ def run_conv(args, workload):
             comparator["ours_over_dense"] = value / world / comparator["value"]
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            import oracle
-            images = conv_oracle_images(w, 15.0)
-            secs = conv_oracle_sample(w, images)
-            cpu = {"value": images * w.Ho * w.Wo / secs, "unit": "tokens/s",
-                   "cores": oracle.threads_used(), "kind": "oracle",
-                   "sample": f"{images} of {w.N} images, float64, {secs:.1f} s"}
+            cpu = conv_cpu_baseline(w)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -1102,6 +1149,21 @@ def run_conv(args, workload):
     return 0
 
 
+def spawn_ranks(n: int) -> int:
+    """Run this same command as n ranks on this node (torch.distributed.run,
+    rendezvous on 127.0.0.1), so that --gpus N without a launcher still runs N
+    ranks; rank 0 prints the result line.  Returns the launcher's exit code."""
+    import socket
+    import subprocess
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", f"--master-port={port}",
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1120,8 +1182,19 @@ def main():
     ap.add_argument("--dp-path", action="store_true",
                     help="training workload: take the data-parallel weight-gradient path "
                          "(FP32 sums, reduction over ranks, one cast) even on one rank")
+    ap.add_argument("--ref-seconds", type=float, default=None,
+                    help="reference arm: host-oracle seconds per step (default: about two "
+                         "minutes for the whole run, at most 20 s a step)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps, reported as run
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        # not launched by torchrun: start one rank per GPU ourselves
+        return spawn_ranks(args.gpus)
+    if env_world is not None and int(env_world) != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={env_world}; launch one rank per "
+              "GPU (torchrun --nproc-per-node N) with --gpus N", file=sys.stderr, flush=True)
+        return 2
     if args.workload in CONV_WORKLOADS:
         if args.impl == "reference":
             return run_conv_reference(args, args.workload)

@@ -211,6 +211,7 @@ size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t p) {
 
 eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, void* W_hat,
                                            void* stream) {
+  EQL_TRACE();
   if (!p || !W || !W_hat) return EQL_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(W_hat)) return EQL_ERR_ALIGNMENT;
   eqlinear_status_t s = check_plan_device(p);
@@ -236,12 +237,14 @@ eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, voi
 
 eqlinear_status_t eqlinear_forward(eqlinear_plan_t p, const void* X, int64_t N,
                                    const void* W_hat, const void* bias, void* Y, void* stream) {
+  EQL_TRACE();
   return eqlinear_forward_act(p, X, N, W_hat, bias, EQL_ACT_NONE, Y, stream);
 }
 
 eqlinear_status_t eqlinear_forward_act(eqlinear_plan_t p, const void* X, int64_t N,
                                        const void* W_hat, const void* bias, eqlinear_act_t act,
                                        void* Y, void* stream) {
+  EQL_TRACE();
   if (!p || N < 0) return EQL_ERR_INVALID_ARG;
   if (act != EQL_ACT_NONE && act != EQL_ACT_GELU) return EQL_ERR_INVALID_ARG;
   if (N == 0) return EQL_OK;
@@ -292,12 +295,14 @@ eqlinear_status_t eqlinear_forward_to_spectral(eqlinear_plan_t p, const void* X,
                                                const void* W_hat, const void* bias,
                                                eqlinear_act_t act, void* Xhat_next,
                                                void* stream) {
+  EQL_TRACE();
   return forward_spectral_io(p, X, N, W_hat, bias, act, Xhat_next, 1, stream);
 }
 
 eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t p, const void* Xhat, int64_t N,
                                                  const void* W_hat, const void* bias,
                                                  eqlinear_act_t act, void* Y, void* stream) {
+  EQL_TRACE();
   return forward_spectral_io(p, Xhat, N, W_hat, bias, act, Y, 2, stream);
 }
 
@@ -326,6 +331,7 @@ eqlinear_status_t eqlinear_forward_chain(eqlinear_plan_t first, eqlinear_plan_t 
                                          const void* W2_hat, const void* bias2,
                                          int spectral_intermediate, void* H, void* Y,
                                          void* workspace, size_t workspace_bytes, void* stream) {
+  EQL_TRACE();
   eqlinear_status_t s = chain_check(first, second, N);
   if (s != EQL_OK) return s;
   if (act1 != EQL_ACT_NONE && act1 != EQL_ACT_GELU) return EQL_ERR_INVALID_ARG;
@@ -365,6 +371,7 @@ size_t eqlinear_conv_prepared_weight_bytes(eqlinear_plan_t p, int KH, int KW) {
 
 eqlinear_status_t eqlinear_conv_prepare_weights(eqlinear_plan_t p, int KH, int KW,
                                                 const void* Wc, void* Wc_hat, void* stream) {
+  EQL_TRACE();
   if (!p || !Wc || !Wc_hat || KH < 1 || KW < 1 || KH > 15 || KW > 15)
     return EQL_ERR_INVALID_ARG;
   if (!conv_plan_ok(p)) return EQL_ERR_UNSUPPORTED;
@@ -399,6 +406,7 @@ eqlinear_status_t eqlinear_conv_forward(eqlinear_plan_t p, const void* X, int64_
                                         const void* Wc_hat, const void* bias, eqlinear_act_t act,
                                         void* Y, void* workspace, size_t workspace_bytes,
                                         void* stream) {
+  EQL_TRACE();
   if (!p || N < 0 || H < 1 || W < 1 || KH < 1 || KW < 1 || pad_h < 0 || pad_w < 0)
     return EQL_ERR_INVALID_ARG;
   if (act != EQL_ACT_NONE && act != EQL_ACT_GELU) return EQL_ERR_INVALID_ARG;
@@ -449,6 +457,7 @@ eqlinear_status_t eqlinear_forward_save_spectrum(eqlinear_plan_t p, const void* 
                                                  const void* W_hat, const void* bias,
                                                  eqlinear_act_t act, void* Y, void* Xhat,
                                                  void* stream) {
+  EQL_TRACE();
   if (!p || !W_hat) return EQL_ERR_INVALID_ARG;
   return save_spectrum_io(p, X, N, p->C, p->D, fwd_tiles(p, W_hat), bias, act, Y, Xhat, stream);
 }
@@ -456,6 +465,7 @@ eqlinear_status_t eqlinear_forward_save_spectrum(eqlinear_plan_t p, const void* 
 eqlinear_status_t eqlinear_backward_input_save_spectrum(eqlinear_plan_t p, const void* dY,
                                                         int64_t N, const void* W_hat, void* dX,
                                                         void* dYhat, void* stream) {
+  EQL_TRACE();
   if (!p || !W_hat) return EQL_ERR_INVALID_ARG;
   return save_spectrum_io(p, dY, N, p->D, p->C, adj_tiles(p, W_hat), nullptr, EQL_ACT_NONE, dX,
                           dYhat, stream);
@@ -463,6 +473,7 @@ eqlinear_status_t eqlinear_backward_input_save_spectrum(eqlinear_plan_t p, const
 
 eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int64_t N,
                                           const void* W_hat, void* dX, void* stream) {
+  EQL_TRACE();
   if (!p || N < 0) return EQL_ERR_INVALID_ARG;
   if (p->group == 1) return EQL_ERR_UNSUPPORTED;
   if (N == 0) return EQL_OK;
@@ -525,6 +536,7 @@ static eqlinear_status_t backward_weight_impl(eqlinear_plan_t p, const void* X, 
 eqlinear_status_t eqlinear_backward_weight(eqlinear_plan_t p, const void* X, const void* dY,
                                            int64_t N, void* dW, void* dbias, void* workspace,
                                            size_t workspace_bytes, void* stream) {
+  EQL_TRACE();
   if (!p) return EQL_ERR_INVALID_ARG;
   return backward_weight_impl(p, X, dY, N, dW, dbias, workspace, workspace_bytes,
                               to_dt(p->dtype), stream);
@@ -534,6 +546,7 @@ eqlinear_status_t eqlinear_backward_weight_f32(eqlinear_plan_t p, const void* X,
                                                int64_t N, float* dW, float* dbias,
                                                void* workspace, size_t workspace_bytes,
                                                void* stream) {
+  EQL_TRACE();
   return backward_weight_impl(p, X, dY, N, dW, dbias, workspace, workspace_bytes,
                               eql::DType::F32, stream);
 }
@@ -542,6 +555,7 @@ eqlinear_status_t eqlinear_backward_weight_from_spectra(eqlinear_plan_t p, const
                                                         const void* dYhat, int64_t N, void* dW,
                                                         void* dbias, void* workspace,
                                                         size_t workspace_bytes, void* stream) {
+  EQL_TRACE();
   if (!p) return EQL_ERR_INVALID_ARG;
   return backward_weight_impl(p, Xhat, dYhat, N, dW, dbias, workspace, workspace_bytes,
                               to_dt(p->dtype), stream, true);
@@ -552,12 +566,14 @@ eqlinear_status_t eqlinear_backward_weight_from_spectra_f32(eqlinear_plan_t p, c
                                                             float* dW, float* dbias,
                                                             void* workspace,
                                                             size_t workspace_bytes, void* stream) {
+  EQL_TRACE();
   return backward_weight_impl(p, Xhat, dYhat, N, dW, dbias, workspace, workspace_bytes,
                               eql::DType::F32, stream, true);
 }
 
 eqlinear_status_t eqlinear_cast_from_f32(eqlinear_plan_t p, const float* src, int64_t count,
                                          void* dst, void* stream) {
+  EQL_TRACE();
   if (!p || count < 0) return EQL_ERR_INVALID_ARG;
   if (count == 0) return EQL_OK;
   if (!src || !dst) return EQL_ERR_INVALID_ARG;
@@ -573,6 +589,7 @@ eqlinear_status_t eqlinear_cast_from_f32(eqlinear_plan_t p, const float* src, in
 }
 
 eqlinear_status_t eqlinear_get_status(eqlinear_plan_t p, void* stream) {
+  EQL_TRACE();
   if (!p) return EQL_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   if (cudaStreamSynchronize(st) != cudaSuccess) return EQL_ERR_CUDA;

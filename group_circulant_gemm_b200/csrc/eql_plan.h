@@ -1,8 +1,21 @@
 // Internal definition of the opaque plan handle of include/eqlinear.h.
 #pragma once
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/eqlinear.h"
 #include "eql_common.cuh"
+
+// One NVTX range per ABI call, named after the entry point (seen by Nsight
+// tools and by ncu's --nvtx filters; header-only NVTX does nothing when no
+// tool is attached).
+struct EqlTraceRange {
+  explicit EqlTraceRange(const char* name) { nvtxRangePushA(name); }
+  ~EqlTraceRange() { nvtxRangePop(); }
+  EqlTraceRange(const EqlTraceRange&) = delete;
+  EqlTraceRange& operator=(const EqlTraceRange&) = delete;
+};
+#define EQL_TRACE() EqlTraceRange eql_trace_range_(__func__)
 
 struct eqlinear_plan_s {
   int T, C, D;

@@ -92,6 +92,8 @@ def _load():
             lib.eqlo_conv_forward.restype = i64
             lib.eqlo_d4_forward.argtypes = [i64, i64, i64, dp, dp, dp, dp]
             lib.eqlo_d4_forward.restype = i64
+            lib.eqlo_set_threads.argtypes = [ctypes.c_int]
+            lib.eqlo_set_threads.restype = None
             _lib = lib
     return _lib
 
@@ -245,8 +247,44 @@ def conv_forward(T: int, X, Wc, bias=None, pad=(0, 0), return_macs: bool = False
     return (Y, macs) if return_macs else Y
 
 
+_threads_override = None
+
+
+def set_threads(n: int | None) -> None:
+    """Run the parallel loops on n threads (None: back to the default count).
+    Timing only: every loop writes disjoint outputs, so results do not change."""
+    global _threads_override
+    _load().eqlo_set_threads(int(n) if n else _default_threads())
+    _threads_override = int(n) if n else None
+
+
+def _default_threads() -> int:
+    env = os.environ.get("OMP_NUM_THREADS")
+    if env:
+        try:
+            return max(1, int(env.split(",")[0]))
+        except ValueError:
+            pass
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (first 'model name' line of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def threads_used() -> int:
     """Threads OpenMP will use for the parallel loops (OMP_NUM_THREADS or cores)."""
+    if _threads_override:
+        return _threads_override
     env = os.environ.get("OMP_NUM_THREADS")
     if env:
         try:

@@ -48,6 +48,20 @@
 
 static long wrap(long i, long T) { return ((i % T) + T) % T; }
 
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Threads of the parallel loops that follow (timing only; no effect on any
+ * result, every loop writes disjoint outputs in a fixed order). */
+void eqlo_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* Forward, the plain definition.  Returns the number of real multiply-adds. */
 int64_t eqlo_forward(int T, int64_t N, int64_t C, int64_t D, const double* X, const double* W,
                      const double* bias, double* Y) {

@@ -6,9 +6,12 @@ characters and the 2 x 2 block), the dense comparator's are 2·N·(C·T)·(D·T)
 the traffic table must point at existing kernel sources.
 """
 import os
+import sys
 
 import bench
 from group_circulant_gemm_b200.synth import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_every_pipeline_resolves_and_chains():
@@ -52,3 +55,34 @@ def test_traffic_table_refers_to_existing_sources():
         for workload, nbytes in per_workload.items():
             assert workload in bench.PIPELINES or workload in bench.CONV_WORKLOADS
             assert 1e6 < nbytes < 1e9
+
+
+def _run_bench(args, env_extra=None, timeout=300):
+    import json
+    import subprocess
+    env = dict(os.environ)
+    env.pop("WORLD_SIZE", None)
+    env.update(env_extra or {})
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], env=env,
+                       capture_output=True, text=True, timeout=timeout, cwd=ROOT)
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    return r.returncode, lines, r.stderr
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """--gpus 2 without a launcher starts two ranks itself (torch.distributed.run on
+    127.0.0.1); the host-oracle reference arm needs no GPU, so the path runs here:
+    rank 0 prints one line for a world of two, the other rank prints nothing."""
+    rc, lines, err = _run_bench(["--gpus", "2", "--impl", "reference", "--steps", "1",
+                                 "--warmup", "3", "--ref-seconds", "0.01"])
+    assert rc == 0, err[-2000:]
+    assert len(lines) == 1 and lines[0]["impl"] == "reference"
+    assert lines[0]["n_gpus"] == 2
+    assert lines[0]["cpu_baseline"]["cores"] >= 1 and lines[0]["cpu_baseline"]["cpu_model"]
+
+
+def test_gpus_flag_disagreeing_with_the_launcher_fails_loudly():
+    rc, lines, err = _run_bench(["--gpus", "2", "--impl", "reference", "--steps", "1",
+                                 "--ref-seconds", "0.01"], {"WORLD_SIZE": "3"}, timeout=120)
+    assert rc != 0 and not lines
+    assert "WORLD_SIZE=3" in err
