@@ -64,6 +64,16 @@ const void* fwd_tiles(const eqlinear_plan_s* p, const void* W_hat) {
 const void* adj_tiles(const eqlinear_plan_s* p, const void* W_hat) {
   return static_cast<const char*>(fwd_tiles(p, W_hat)) + eql::tc_tile_bytes(p->T, p->C, p->D);
 }
+// p4 FP16 plans also hold the pair kernel's weight stages (forward, then adjoint)
+bool has_pair_tiles(const eqlinear_plan_s* p) {
+  return p->group == 0 && p->T == 4 && has_tiles(p);
+}
+const void* pair_fwd_tiles(const eqlinear_plan_s* p, const void* W_hat) {
+  return static_cast<const char*>(adj_tiles(p, W_hat)) + eql::tc_tile_bytes(p->T, p->D, p->C);
+}
+const void* pair_adj_tiles(const eqlinear_plan_s* p, const void* W_hat) {
+  return static_cast<const char*>(pair_fwd_tiles(p, W_hat)) + eql::pair_tile_bytes(p->C, p->D);
+}
 
 // Forward-shaped product used by both eqlinear_forward (Cin=C, Cout=D) and
 // eqlinear_backward_input (Cin=D, Cout=C).
@@ -206,6 +216,7 @@ size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t p) {
     return d4_ok(p) ? 8 * plane_elems(p) * 2 + eql::tc_tile_bytes(8, p->C, p->D) : 0;
   size_t bytes = 2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
   if (has_tiles(p)) bytes += eql::tc_tile_bytes(p->T, p->C, p->D) + eql::tc_tile_bytes(p->T, p->D, p->C);
+  if (has_pair_tiles(p)) bytes += eql::pair_tile_bytes(p->C, p->D) + eql::pair_tile_bytes(p->D, p->C);
   return bytes;
 }
 
@@ -231,8 +242,14 @@ eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, voi
   s = from_cuda(eql::launch_tile_weights(p->T, fwd, p->C, p->D, const_cast<void*>(fwd_tiles(p, W_hat)),
                                          st));
   if (s != EQL_OK) return s;
-  return from_cuda(eql::launch_tile_weights(p->T, adj, p->D, p->C,
-                                            const_cast<void*>(adj_tiles(p, W_hat)), st));
+  s = from_cuda(eql::launch_tile_weights(p->T, adj, p->D, p->C,
+                                         const_cast<void*>(adj_tiles(p, W_hat)), st));
+  if (s != EQL_OK || !has_pair_tiles(p)) return s;
+  s = from_cuda(eql::launch_pair_tile_weights(fwd, p->C, p->D,
+                                              const_cast<void*>(pair_fwd_tiles(p, W_hat)), st));
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_pair_tile_weights(adj, p->D, p->C,
+                                                 const_cast<void*>(pair_adj_tiles(p, W_hat)), st));
 }
 
 eqlinear_status_t eqlinear_forward(eqlinear_plan_t p, const void* X, int64_t N,
@@ -304,6 +321,69 @@ eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t p, const void* 
                                                  eqlinear_act_t act, void* Y, void* stream) {
   EQL_TRACE();
   return forward_spectral_io(p, Xhat, N, W_hat, bias, act, Y, 2, stream);
+}
+
+size_t eqlinear_tiled_spectrum_bytes(eqlinear_plan_t p, int64_t N, int channels) {
+  if (!p || N < 0 || channels <= 0) return 0;
+  return eql::tiled_planes_bytes(N, channels);
+}
+
+// Tiled spectral input through the pair kernel: forward (adjoint = false:
+// Cin = C, Cout = D, bias and act allowed) or dX (adjoint: Cin = D, Cout = C).
+static eqlinear_status_t pair_io(eqlinear_plan_t p, const void* Xt, int64_t N, const void* W_hat,
+                                 const void* bias, eqlinear_act_t act, void* out,
+                                 int spectral_out, bool adjoint, void* stream) {
+  if (!p || N < 0) return EQL_ERR_INVALID_ARG;
+  if (act != EQL_ACT_NONE && act != EQL_ACT_GELU) return EQL_ERR_INVALID_ARG;
+  if (N == 0) return EQL_OK;
+  if (!Xt || !W_hat || !out) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(Xt) || !aligned16(W_hat) || !aligned16(out) || (bias && !aligned16(bias)))
+    return EQL_ERR_ALIGNMENT;
+  const int Cin = adjoint ? p->D : p->C, Cout = adjoint ? p->C : p->D;
+  if (!has_pair_tiles(p) || p->kernel == EQL_KERNEL_SIMT ||
+      !eql::pair_tc_supported(N, Cin, Cout))
+    return EQL_ERR_UNSUPPORTED;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_pair_tc(Xt, N, Cin, Cout,
+                                       adjoint ? pair_adj_tiles(p, W_hat) : pair_fwd_tiles(p, W_hat),
+                                       bias, out, p->status, p->num_sms, (int)act, spectral_out,
+                                       (cudaStream_t)stream));
+}
+
+eqlinear_status_t eqlinear_group_dft(eqlinear_plan_t p, const void* X, int64_t N, int channels,
+                                     void* Xt, void* stream) {
+  EQL_TRACE();
+  if (!p || N < 0) return EQL_ERR_INVALID_ARG;
+  if (channels != p->C && channels != p->D) return EQL_ERR_INVALID_ARG;
+  if (p->T != 4 || p->dtype != EQL_F16 || p->group != 0 || channels % 16 != 0)
+    return EQL_ERR_UNSUPPORTED;
+  if (N == 0) return EQL_OK;
+  if (!X || !Xt) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Xt)) return EQL_ERR_ALIGNMENT;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_group_dft_tiled(X, N, channels, Xt, (cudaStream_t)stream));
+}
+
+eqlinear_status_t eqlinear_forward_tiled(eqlinear_plan_t p, const void* Xt, int64_t N,
+                                         const void* W_hat, const void* bias, eqlinear_act_t act,
+                                         void* Y, void* stream) {
+  EQL_TRACE();
+  return pair_io(p, Xt, N, W_hat, bias, act, Y, 0, false, stream);
+}
+
+eqlinear_status_t eqlinear_forward_tiled_next(eqlinear_plan_t p, const void* Xt, int64_t N,
+                                              const void* W_hat, const void* bias,
+                                              eqlinear_act_t act, void* Yt_next, void* stream) {
+  EQL_TRACE();
+  return pair_io(p, Xt, N, W_hat, bias, act, Yt_next, 1, false, stream);
+}
+
+eqlinear_status_t eqlinear_backward_input_tiled(eqlinear_plan_t p, const void* dYt, int64_t N,
+                                                const void* W_hat, void* dX, void* stream) {
+  EQL_TRACE();
+  return pair_io(p, dYt, N, W_hat, nullptr, EQL_ACT_NONE, dX, 0, true, stream);
 }
 
 // Both layers must be p4 FP16 plans with tensor-core tiles whose widths chain.

@@ -103,6 +103,27 @@ cudaError_t launch_conv_tc(const void* X, int64_t N, int H, int W, int C, int D,
                            int ph, int pw, const void* Wtiles, const void* bias, void* Y,
                            void* planes, int* status, int num_sms, int act, cudaStream_t st);
 
+// Tiled planes: the group DFT of p4 rows stored as the pair kernel's
+// shared-memory operand image (rows padded to a multiple of 128; per plane and
+// 16-channel block, 32-byte rows with the 32-byte swizzle; see eql_tc_pair.cu).
+int64_t tiled_rows(int64_t N);
+size_t tiled_planes_bytes(int64_t N, int channels);
+// X [N][C*4] -> tiled planes of X (times 1/4), C a multiple of 16.
+cudaError_t launch_group_dft_tiled(const void* X, int64_t N, int C, void* out, cudaStream_t st);
+
+// Pair-CTA (cta_group::2) tensor-core forward for T = 4, FP16, from tiled
+// input planes: Y [N][Cout*4] or, with spectral_out, the next layer's tiled
+// planes.  Weights: the pair kernel's own stage image (launch_pair_tile_weights
+// from a block of prepared planes [5][Cout][Cin]).  Returns
+// cudaErrorNotSupported for shapes it does not take (Cin, Cout multiples of 16).
+bool pair_tc_supported(int64_t N, int Cin, int Cout);
+size_t pair_tile_bytes(int Cin, int Cout);
+cudaError_t launch_pair_tile_weights(const void* planes, int Cin, int Cout, void* tiles,
+                                     cudaStream_t st);
+cudaError_t launch_pair_tc(const void* Xt, int64_t N, int Cin, int Cout, const void* tiles,
+                           const void* bias, void* Y, int* status, int num_sms, int act,
+                           int spectral_out, cudaStream_t st);
+
 // dst[i] = src[i] rounded to nearest-even in dt (a copy for F32), i < n.
 cudaError_t launch_cast_from_f32(DType dt, const float* src, void* dst, int64_t n,
                                  cudaStream_t st);

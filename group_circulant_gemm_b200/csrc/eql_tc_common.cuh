@@ -63,8 +63,12 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* b, uint32_t parity
   return ok != 0;
 }
 // Bounded wait: false if the CTA aborted or the wait timed out (then aborts it).
-static __device__ __noinline__ bool wait_bounded(uint64_t* b, uint32_t parity, int* abort_flag, int* status) {
-  if (mbar_try_wait(b, parity)) return true;
+// The loop lives out of line; the test for an already completed phase is
+// inlined (below), so a pipeline whose stages are ready pays no call: in a
+// kernel near its register limit, a call per stage costs hundreds of cycles
+// of saves and restores, several times the tensor core's time per K step.
+static __device__ __noinline__ bool wait_bounded_slow(uint64_t* b, uint32_t parity,
+                                                      int* abort_flag, int* status) {
   const uint64_t t0 = gtimer();
   while (true) {
     if (mbar_try_wait_sleep(b, parity, 200000u)) return true;
@@ -75,6 +79,11 @@ static __device__ __noinline__ bool wait_bounded(uint64_t* b, uint32_t parity, i
       return false;
     }
   }
+}
+__device__ __forceinline__ bool wait_bounded(uint64_t* b, uint32_t parity, int* abort_flag,
+                                             int* status) {
+  if (mbar_try_wait(b, parity)) return true;
+  return wait_bounded_slow(b, parity, abort_flag, status);
 }
 // Warp-uniform bounded wait: every lane polls, then the warp agrees, so a lane
 // that gave up cannot leave the others waiting at a warp-synchronous point.

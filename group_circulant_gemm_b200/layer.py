@@ -111,6 +111,60 @@ class EqLinearPlan:
         _n.eqlinear_forward_from_spectral(self.handle, Xhat, N, W_hat, bias, _n.ACT[act], out)
         return out
 
+    # --- the frequency-domain form on tiled planes (see eqlinear_group_dft)
+
+    def tiled_shape(self, N: int, channels: int):
+        """Shape of tiled planes of N rows: (4 planes, channels/16 blocks, Np rows,
+        16 halves per row in the swizzled order of the header), Np = N rounded up
+        to a multiple of 128."""
+        return (4, channels // 16, (N + 127) // 128 * 128, 16)
+
+    def group_dft(self, X, out=None) -> torch.Tensor:
+        """Tiled planes of X [N, c*4] (c = C for an input, D for an upstream gradient)."""
+        N = X.shape[0]
+        c = X.shape[1] // self.T
+        if c not in (self.C, self.D) or X.shape[1] != c * self.T:
+            raise ValueError(f"X must be [N, C*T] or [N, D*T], got {tuple(X.shape)}")
+        self._check(X, (N, c * self.T), "X")
+        if out is None:
+            out = torch.empty(self.tiled_shape(N, c), dtype=self.dtype, device=X.device)
+        self._check(out, self.tiled_shape(N, c), "out")
+        _n.eqlinear_group_dft(self.handle, X, N, c, out)
+        return out
+
+    def forward_tiled(self, Xt, N: int, W_hat, bias=None, act: str = "none",
+                      out=None) -> torch.Tensor:
+        """Y [N, D*T] from the tiled planes of X."""
+        self._check(Xt, self.tiled_shape(N, self.C), "Xt")
+        if bias is not None:
+            self._check(bias, (self.D,), "bias")
+        if out is None:
+            out = torch.empty((N, self.D * self.T), dtype=self.dtype, device=Xt.device)
+        self._check(out, (N, self.D * self.T), "out")
+        _n.eqlinear_forward_tiled(self.handle, Xt, N, W_hat, bias, _n.ACT[act], out)
+        return out
+
+    def forward_tiled_next(self, Xt, N: int, W_hat, bias=None, act: str = "none",
+                           out=None) -> torch.Tensor:
+        """The tiled planes of act(Y) (the next p4 layer's input) from those of X."""
+        self._check(Xt, self.tiled_shape(N, self.C), "Xt")
+        if bias is not None:
+            self._check(bias, (self.D,), "bias")
+        if out is None:
+            out = torch.empty(self.tiled_shape(N, self.D), dtype=self.dtype, device=Xt.device)
+        self._check(out, self.tiled_shape(N, self.D), "out")
+        _n.eqlinear_forward_tiled_next(self.handle, Xt, N, W_hat, bias, _n.ACT[act], out)
+        return out
+
+    def backward_input_tiled(self, dYt, N: int, W_hat, out=None) -> torch.Tensor:
+        """dX [N, C*T] from the tiled planes of dY."""
+        self._check(dYt, self.tiled_shape(N, self.D), "dYt")
+        if out is None:
+            out = torch.empty((N, self.C * self.T), dtype=self.dtype, device=dYt.device)
+        self._check(out, (N, self.C * self.T), "out")
+        _n.eqlinear_backward_input_tiled(self.handle, dYt, N, W_hat, out)
+        return out
+
     def backward_input(self, dY, W_hat, out=None) -> torch.Tensor:
         N = dY.shape[0]
         self._check(dY, (N, self.D * self.T), "dY")

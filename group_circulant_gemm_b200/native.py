@@ -36,6 +36,8 @@ EXPORTED = (
     "eqlinear_plan_create_dihedral4",
     "eqlinear_forward_save_spectrum", "eqlinear_backward_input_save_spectrum",
     "eqlinear_backward_weight_from_spectra", "eqlinear_backward_weight_from_spectra_f32",
+    "eqlinear_tiled_spectrum_bytes", "eqlinear_group_dft", "eqlinear_forward_tiled",
+    "eqlinear_forward_tiled_next", "eqlinear_backward_input_tiled",
 )
 
 
@@ -68,6 +70,11 @@ def _load() -> ctypes.CDLL:
         "eqlinear_spectral_bytes": ([vp, i64], ctypes.c_size_t),
         "eqlinear_forward_to_spectral": ([vp, vp, i64, vp, vp, i32, vp, vp], i32),
         "eqlinear_forward_from_spectral": ([vp, vp, i64, vp, vp, i32, vp, vp], i32),
+        "eqlinear_tiled_spectrum_bytes": ([vp, i64, i32], sz),
+        "eqlinear_group_dft": ([vp, vp, i64, i32, vp, vp], i32),
+        "eqlinear_forward_tiled": ([vp, vp, i64, vp, vp, i32, vp, vp], i32),
+        "eqlinear_forward_tiled_next": ([vp, vp, i64, vp, vp, i32, vp, vp], i32),
+        "eqlinear_backward_input_tiled": ([vp, vp, i64, vp, vp, vp], i32),
         "eqlinear_backward_input": ([vp, vp, i64, vp, vp, vp], i32),
         "eqlinear_backward_weight_workspace_bytes": ([vp, i64], sz),
         "eqlinear_backward_weight": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
@@ -197,6 +204,35 @@ def eqlinear_forward_from_spectral(plan: int, Xhat, N: int, W_hat, bias, act: in
     _check(_lib.eqlinear_forward_from_spectral(plan, _ptr(Xhat), N, _ptr(W_hat), _ptr(bias), act,
                                                _ptr(Y), _stream(stream)),
            "eqlinear_forward_from_spectral")
+
+
+def eqlinear_tiled_spectrum_bytes(plan: int, N: int, channels: int) -> int:
+    return _lib.eqlinear_tiled_spectrum_bytes(plan, N, channels)
+
+
+def eqlinear_group_dft(plan: int, X, N: int, channels: int, Xt, stream=None) -> None:
+    _check(_lib.eqlinear_group_dft(plan, _ptr(X), N, channels, _ptr(Xt), _stream(stream)),
+           "eqlinear_group_dft")
+
+
+def eqlinear_forward_tiled(plan: int, Xt, N: int, W_hat, bias, act: int, Y,
+                           stream=None) -> None:
+    _check(_lib.eqlinear_forward_tiled(plan, _ptr(Xt), N, _ptr(W_hat), _ptr(bias), act, _ptr(Y),
+                                       _stream(stream)),
+           "eqlinear_forward_tiled")
+
+
+def eqlinear_forward_tiled_next(plan: int, Xt, N: int, W_hat, bias, act: int, Yt,
+                                stream=None) -> None:
+    _check(_lib.eqlinear_forward_tiled_next(plan, _ptr(Xt), N, _ptr(W_hat), _ptr(bias), act,
+                                            _ptr(Yt), _stream(stream)),
+           "eqlinear_forward_tiled_next")
+
+
+def eqlinear_backward_input_tiled(plan: int, dYt, N: int, W_hat, dX, stream=None) -> None:
+    _check(_lib.eqlinear_backward_input_tiled(plan, _ptr(dYt), N, _ptr(W_hat), _ptr(dX),
+                                              _stream(stream)),
+           "eqlinear_backward_input_tiled")
 
 
 def eqlinear_backward_input(plan: int, dY, N: int, W_hat, dX, stream=None) -> None:

@@ -143,6 +143,9 @@ EQL_API const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t plan, i
  * kernel's operand tiles (one contiguous blob per out-channel tile and K stage:
  * 128 x 32 channels at T = 4, 64 x 16 at T = 8, in the kernel's swizzled
  * shared-memory order, the same values), so each pipeline stage is one copy.
+ * At T = 4 two more follow: the same planes as the two-SM spectral kernel's
+ * stages (forward, then adjoint; per 128 out-channels and 16 input channels,
+ * each SM's half of the weights: 2 x 12 KB).
  */
 EQL_API size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t plan);
 
@@ -221,6 +224,50 @@ EQL_API eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t plan, c
                                                          int64_t N, const void* W_hat,
                                                          const void* bias, eqlinear_act_t act,
                                                          void* Y, void* stream);
+
+/*
+ * The layer in the frequency domain, as separate steps ("Algorithmic approach"
+ * items 1-3: forward group DFT, per-frequency products, inverse DFT): the
+ * input's DFT is formed once by eqlinear_group_dft and kept in HBM as "tiled
+ * planes"; the products and the inverse then run in a kernel that copies those
+ * planes straight into the tensor cores' operand layout, two SMs per 256-row
+ * tile (tcgen05 cta_group::2), and can write its output as the next layer's
+ * tiled planes, so a chain of p4 layers stays in the frequency domain.
+ *
+ * Tiled planes of a [N][c*4] array: the four planes of eqlinear_forward_to_spectral
+ * (X0, X2, Xr, Xi, each times 1/4) stored as the kernel's shared-memory image.
+ * Rows are padded to Np = N rounded up to a multiple of 128; element (plane p,
+ * row n, channel j) is the FP16 value at byte offset
+ *   ((p * (c / 16) + j / 16) * Np + n) * 32 + 16 * (((j % 16) / 8) ^ ((n / 4) % 2))
+ *   + 2 * (j % 8).
+ * eqlinear_tiled_spectrum_bytes(plan, N, c) = 4 * Np * c * 2 bytes.
+ *
+ * eqlinear_group_dft: X [N][channels*4] -> tiled planes (rows N..Np-1 zero);
+ *   channels is the plan's C (a layer input) or D (an upstream gradient).
+ * eqlinear_forward_tiled: tiled planes of X [N][C*4] -> Y [N][D*4], bias and
+ *   act as in eqlinear_forward_act.
+ * eqlinear_forward_tiled_next: the same, written as the tiled planes of act(Y)
+ *   (padding rows N..Np-1 hold values of no meaning).
+ * eqlinear_backward_input_tiled: tiled planes of dY [N][D*4] -> dX [N][C*4].
+ * Each equals eqlinear_forward_act / eqlinear_backward_input up to the rounding
+ * of the planes.  FP16 plans with T = 4 and C, D multiples of 16, not forced to
+ * the CUDA cores (else EQL_ERR_UNSUPPORTED); channels not C or D:
+ * EQL_ERR_INVALID_ARG; all pointers 16-byte aligned; outputs must not overlap
+ * inputs; N = 0 is a no-op.
+ */
+EQL_API size_t eqlinear_tiled_spectrum_bytes(eqlinear_plan_t plan, int64_t N, int channels);
+EQL_API eqlinear_status_t eqlinear_group_dft(eqlinear_plan_t plan, const void* X, int64_t N,
+                                             int channels, void* Xt, void* stream);
+EQL_API eqlinear_status_t eqlinear_forward_tiled(eqlinear_plan_t plan, const void* Xt,
+                                                 int64_t N, const void* W_hat, const void* bias,
+                                                 eqlinear_act_t act, void* Y, void* stream);
+EQL_API eqlinear_status_t eqlinear_forward_tiled_next(eqlinear_plan_t plan, const void* Xt,
+                                                      int64_t N, const void* W_hat,
+                                                      const void* bias, eqlinear_act_t act,
+                                                      void* Yt_next, void* stream);
+EQL_API eqlinear_status_t eqlinear_backward_input_tiled(eqlinear_plan_t plan, const void* dYt,
+                                                        int64_t N, const void* W_hat, void* dX,
+                                                        void* stream);
 
 /*
  * Two chained layers in one launch (the MLP pair of a Flash EQ-ViT block):
