@@ -380,6 +380,42 @@ eqlinear_status_t eqlinear_forward_tiled_next(eqlinear_plan_t p, const void* Xt,
   return pair_io(p, Xt, N, W_hat, bias, act, Yt_next, 1, false, stream);
 }
 
+size_t eqlinear_chain_tiled_workspace_bytes(eqlinear_plan_t first, eqlinear_plan_t second,
+                                            int64_t N) {
+  if (!first || !second || N < 0) return 0;
+  return eql::pair_chain_sync_bytes(N);
+}
+
+eqlinear_status_t eqlinear_forward_chain_tiled(eqlinear_plan_t a, eqlinear_plan_t b,
+                                               const void* Xt, int64_t N, const void* W1_hat,
+                                               const void* bias1, eqlinear_act_t act1,
+                                               const void* W2_hat, const void* bias2, void* Ht,
+                                               void* Y, void* workspace, size_t workspace_bytes,
+                                               void* stream) {
+  EQL_TRACE();
+  if (!a || !b || N < 0) return EQL_ERR_INVALID_ARG;
+  if (act1 != EQL_ACT_NONE && act1 != EQL_ACT_GELU) return EQL_ERR_INVALID_ARG;
+  if (a->D != b->C || a->device != b->device) return EQL_ERR_INVALID_ARG;
+  if (!has_pair_tiles(a) || !has_pair_tiles(b) || a->kernel == EQL_KERNEL_SIMT ||
+      b->kernel == EQL_KERNEL_SIMT)
+    return EQL_ERR_UNSUPPORTED;
+  if (N == 0) return EQL_OK;
+  if (!Xt || !W1_hat || !W2_hat || !Ht || !Y || !workspace) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(Xt) || !aligned16(W1_hat) || !aligned16(W2_hat) || !aligned16(Ht) ||
+      !aligned16(Y) || (bias1 && !aligned16(bias1)) || (bias2 && !aligned16(bias2)) ||
+      !aligned16(workspace))
+    return EQL_ERR_ALIGNMENT;
+  if (workspace_bytes < eql::pair_chain_sync_bytes(N)) return EQL_ERR_WORKSPACE;
+  if (!eql::pair_tc_supported(N, a->C, a->D) || !eql::pair_tc_supported(N, b->C, b->D))
+    return EQL_ERR_UNSUPPORTED;
+  eqlinear_status_t s = check_plan_device(a);
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_pair_chain_tc(
+      Xt, N, a->C, a->D, b->D, pair_fwd_tiles(a, W1_hat), bias1, pair_fwd_tiles(b, W2_hat), bias2,
+      Ht, Y, static_cast<int*>(workspace), a->status, a->num_sms, (int)act1,
+      (cudaStream_t)stream));
+}
+
 eqlinear_status_t eqlinear_backward_input_tiled(eqlinear_plan_t p, const void* dYt, int64_t N,
                                                 const void* W_hat, void* dX, void* stream) {
   EQL_TRACE();

@@ -123,6 +123,15 @@ cudaError_t launch_pair_tile_weights(const void* planes, int Cin, int Cout, void
 cudaError_t launch_pair_tc(const void* Xt, int64_t N, int Cin, int Cout, const void* tiles,
                            const void* bias, void* Y, int* status, int num_sms, int act,
                            int spectral_out, cudaStream_t st);
+// Two chained p4 layers on SM pairs (C0 -> C1 -> C2) in one persistent launch
+// with a dynamic tile queue: Ht = tiled planes of act1(L1(X)), Y = L2(H) spatial.
+// `sync` holds pair_chain_sync_bytes(N) bytes of counters, zero at launch and
+// left zero.
+size_t pair_chain_sync_bytes(int64_t N);
+cudaError_t launch_pair_chain_tc(const void* Xt, int64_t N, int C0, int C1, int C2,
+                                 const void* W1tiles, const void* b1, const void* W2tiles,
+                                 const void* b2, void* Ht, void* Y, int* sync, int* status,
+                                 int num_sms, int act1, cudaStream_t st);
 
 // dst[i] = src[i] rounded to nearest-even in dt (a copy for F32), i < n.
 cudaError_t launch_cast_from_f32(DType dt, const float* src, void* dst, int64_t n,

@@ -365,3 +365,26 @@ def forward_chain(first: EqLinearPlan, second: EqLinearPlan, X, W1_hat, bias1, W
                               workspace.numel() * workspace.element_size())
     return H, Y
 
+
+
+def forward_chain_tiled(first: EqLinearPlan, second: EqLinearPlan, Xt, N: int, W1_hat, bias1,
+                        W2_hat, bias2, act: str = "none", Ht=None, Y=None, workspace=None):
+    """Two chained layers on tiled planes in one launch: Ht = tiled planes of
+    act(first(X)), Y = second(H) [N, D2*T], from Xt = first.group_dft(X).
+    Bitwise equal to first.forward_tiled_next then second.forward_tiled.  A
+    ``workspace`` passed in must be zero-filled before its first use (each call
+    leaves it zero)."""
+    first._check(Xt, first.tiled_shape(N, first.C), "Xt")
+    if second.C != first.D:
+        raise ValueError("the second layer's input width must be the first layer's output width")
+    if Ht is None:
+        Ht = torch.empty(first.tiled_shape(N, first.D), dtype=first.dtype, device=Xt.device)
+    if Y is None:
+        Y = torch.empty((N, second.D * second.T), dtype=second.dtype, device=Xt.device)
+    nb = _n.eqlinear_chain_tiled_workspace_bytes(first.handle, second.handle, N)
+    if workspace is None:
+        workspace = torch.zeros(max(nb, 16), dtype=torch.uint8, device=Xt.device)
+    _n.eqlinear_forward_chain_tiled(first.handle, second.handle, Xt, N, W1_hat, bias1,
+                                    _n.ACT[act], W2_hat, bias2, Ht, Y, workspace,
+                                    workspace.numel() * workspace.element_size())
+    return Ht, Y

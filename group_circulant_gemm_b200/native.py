@@ -38,6 +38,7 @@ EXPORTED = (
     "eqlinear_backward_weight_from_spectra", "eqlinear_backward_weight_from_spectra_f32",
     "eqlinear_tiled_spectrum_bytes", "eqlinear_group_dft", "eqlinear_forward_tiled",
     "eqlinear_forward_tiled_next", "eqlinear_backward_input_tiled",
+    "eqlinear_chain_tiled_workspace_bytes", "eqlinear_forward_chain_tiled",
 )
 
 
@@ -75,6 +76,9 @@ def _load() -> ctypes.CDLL:
         "eqlinear_forward_tiled": ([vp, vp, i64, vp, vp, i32, vp, vp], i32),
         "eqlinear_forward_tiled_next": ([vp, vp, i64, vp, vp, i32, vp, vp], i32),
         "eqlinear_backward_input_tiled": ([vp, vp, i64, vp, vp, vp], i32),
+        "eqlinear_chain_tiled_workspace_bytes": ([vp, vp, i64], sz),
+        "eqlinear_forward_chain_tiled": ([vp, vp, vp, i64, vp, vp, i32, vp, vp, vp, vp, vp, sz,
+                                          vp], i32),
         "eqlinear_backward_input": ([vp, vp, i64, vp, vp, vp], i32),
         "eqlinear_backward_weight_workspace_bytes": ([vp, i64], sz),
         "eqlinear_backward_weight": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
@@ -227,6 +231,20 @@ def eqlinear_forward_tiled_next(plan: int, Xt, N: int, W_hat, bias, act: int, Yt
     _check(_lib.eqlinear_forward_tiled_next(plan, _ptr(Xt), N, _ptr(W_hat), _ptr(bias), act,
                                             _ptr(Yt), _stream(stream)),
            "eqlinear_forward_tiled_next")
+
+
+def eqlinear_chain_tiled_workspace_bytes(first: int, second: int, N: int) -> int:
+    return _lib.eqlinear_chain_tiled_workspace_bytes(first, second, N)
+
+
+def eqlinear_forward_chain_tiled(first: int, second: int, Xt, N: int, W1_hat, bias1, act1: int,
+                                 W2_hat, bias2, Ht, Y, workspace, workspace_bytes: int,
+                                 stream=None) -> None:
+    _check(_lib.eqlinear_forward_chain_tiled(first, second, _ptr(Xt), N, _ptr(W1_hat),
+                                             _ptr(bias1), act1, _ptr(W2_hat), _ptr(bias2),
+                                             _ptr(Ht), _ptr(Y), _ptr(workspace), workspace_bytes,
+                                             _stream(stream)),
+           "eqlinear_forward_chain_tiled")
 
 
 def eqlinear_backward_input_tiled(plan: int, dYt, N: int, W_hat, dX, stream=None) -> None:

@@ -270,6 +270,32 @@ EQL_API eqlinear_status_t eqlinear_backward_input_tiled(eqlinear_plan_t plan, co
                                                         void* stream);
 
 /*
+ * Two chained layers on tiled planes in one launch (the MLP pair of a Flash
+ * EQ-ViT block, kept in the frequency domain between the layers):
+ *   Ht = tiled planes of act1(first(X))   (as eqlinear_forward_tiled_next)
+ *   Y  = second(H)                        (as eqlinear_forward_tiled), Y [N][D2*4]
+ * from Xt, the tiled planes of X [N][C0*4] (eqlinear_group_dft).  Results are
+ * bitwise those of the two separate calls; the tiles of both layers share one
+ * queue, so neither layer's last partial wave leaves SMs idle.  Ht is the
+ * caller's buffer (eqlinear_tiled_spectrum_bytes(first, N, first's D)).
+ * workspace: eqlinear_chain_tiled_workspace_bytes(first, second, N) bytes of
+ * int32 counters that must be zero before the first call; each call leaves
+ * them zero (after a timeout reported by eqlinear_get_status, zero them again).
+ * Plans: p4 FP16 with C, D multiples of 16, second's C = first's D, same device,
+ * not forced to the CUDA cores (else EQL_ERR_UNSUPPORTED / EQL_ERR_INVALID_ARG);
+ * EQL_ERR_WORKSPACE for a short workspace; pointers 16-byte aligned.
+ */
+EQL_API size_t eqlinear_chain_tiled_workspace_bytes(eqlinear_plan_t first, eqlinear_plan_t second,
+                                                    int64_t N);
+EQL_API eqlinear_status_t eqlinear_forward_chain_tiled(eqlinear_plan_t first,
+                                                       eqlinear_plan_t second, const void* Xt,
+                                                       int64_t N, const void* W1_hat,
+                                                       const void* bias1, eqlinear_act_t act1,
+                                                       const void* W2_hat, const void* bias2,
+                                                       void* Ht, void* Y, void* workspace,
+                                                       size_t workspace_bytes, void* stream);
+
+/*
  * Two chained layers in one launch (the MLP pair of a Flash EQ-ViT block):
  *   H = act1(layer first (X))     H: [N][D1*T], or with spectral_intermediate = 1
  *                                    the planes [4][N][D1] of

@@ -157,3 +157,80 @@ def test_tiled_entries_reject_what_they_do_not_take():
     p.set_kernel("auto")
     assert n.raw_status("eqlinear_forward_tiled", p.handle, None, 0, Wh.data_ptr(), None, 0,
                         None, None) == n.EQL_OK
+
+
+CHAIN_CASES = [
+    # N, C0, C1, C2, act
+    (333, 64, 128, 64, "none"),
+    (1000, 192, 768, 192, "gelu"),
+    (257, 48, 80, 32, "none"),
+    (1, 16, 32, 16, "gelu"),
+    (2600, 128, 256, 128, "none"),   # more tasks than pairs: the queue wraps
+]
+
+
+@pytest.mark.parametrize("N,C0,C1,C2,act", CHAIN_CASES)
+def test_tiled_chain_equals_two_calls_bitwise(N, C0, C1, C2, act):
+    from group_circulant_gemm_b200.layer import forward_chain_tiled
+    w1 = Workload("c1", 4, N, C0, C1, "f16", True, 3500 + N)
+    w2 = Workload("c2", 4, N, C1, C2, "f16", True, 3600 + N)
+    in1, in2 = make_inputs(w1), make_inputs(w2, rows=1)
+    p1, p2 = _plan(4, C0, C1), _plan(4, C1, C2)
+    Wh1, Wh2 = p1.prepare_weights(_dev(in1["W"])), p2.prepare_weights(_dev(in2["W"]))
+    b1, b2 = _dev(in1["bias"]), _dev(in2["bias"])
+    Xt = p1.group_dft(_dev(in1["X"]))
+    ws = torch.zeros(native.eqlinear_chain_tiled_workspace_bytes(p1.handle, p2.handle, N) + 64,
+                     dtype=torch.uint8, device="cuda")
+    for _ in range(2):  # the second call reuses the workspace the first left zero
+        Ht, Y = forward_chain_tiled(p1, p2, Xt, N, Wh1, b1, Wh2, b2, act=act, workspace=ws)
+        assert p1.status() == 0 and p2.status() == 0
+        assert int(ws.abs().sum()) == 0
+    Ht_ref = p1.forward_tiled_next(Xt, N, Wh1, b1, act=act)
+    Y_ref = p2.forward_tiled(Ht_ref, N, Wh2, b2)
+    got_h, _ = _untile(Ht, N, C1)
+    ref_h, _ = _untile(Ht_ref, N, C1)
+    assert np.array_equal(got_h, ref_h)
+    assert torch.equal(Y, Y_ref)
+    if N <= 1000:
+        H = oracle.forward(4, in1["X"], in1["W"], in1["bias"], act=act)
+        assert _rel(Y.double().cpu().numpy(), oracle.forward(4, H, in2["W"], in2["bias"])) <= TOL
+
+
+def test_tiled_chain_full_size_sampled_rows():
+    from group_circulant_gemm_b200.layer import forward_chain_tiled
+    w1, w2 = WORKLOADS["p4_vitb_fc1_f16"], WORKLOADS["p4_vitb_fc2_f16"]
+    in1, in2 = make_inputs(w1), make_inputs(w2, rows=1)
+    p1, p2 = _plan(4, w1.C, w1.D), _plan(4, w2.C, w2.D)
+    Wh1, Wh2 = p1.prepare_weights(_dev(in1["W"])), p2.prepare_weights(_dev(in2["W"]))
+    N = w1.N
+    Xt = p1.group_dft(_dev(in1["X"]))
+    _, Y = forward_chain_tiled(p1, p2, Xt, N, Wh1, _dev(in1["bias"]), Wh2, _dev(in2["bias"]))
+    Y = Y.double().cpu().numpy()
+    assert p1.status() == 0 and p2.status() == 0
+    rng = np.random.default_rng(11)
+    rows = np.unique(np.concatenate([rng.choice(N, 48, replace=False), np.arange(N - 8, N),
+                                     np.arange(8), np.arange(252, 260)]))
+    H = oracle.forward(4, in1["X"][rows], in1["W"], in1["bias"])
+    assert _rel(Y[rows], oracle.forward(4, H, in2["W"], in2["bias"])) <= TOL
+
+
+def test_tiled_chain_rejects_bad_arguments():
+    p1, p2, p3 = _plan(4, 32, 64), _plan(4, 64, 32), _plan(4, 48, 32)
+    N = 100
+    Xt = torch.zeros(p1.tiled_shape(N, 32), dtype=torch.float16, device="cuda")
+    Ht = torch.zeros(p1.tiled_shape(N, 64), dtype=torch.float16, device="cuda")
+    Y = torch.zeros((N, 128), dtype=torch.float16, device="cuda")
+    W1 = torch.zeros(native.eqlinear_prepared_weight_bytes(p1.handle) // 2, dtype=torch.float16,
+                     device="cuda")
+    W2 = torch.zeros(native.eqlinear_prepared_weight_bytes(p2.handle) // 2, dtype=torch.float16,
+                     device="cuda")
+    nb = native.eqlinear_chain_tiled_workspace_bytes(p1.handle, p2.handle, N)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+
+    def call(a, b, wsb=nb):
+        return native.raw_status("eqlinear_forward_chain_tiled", a.handle, b.handle, Xt.data_ptr(),
+                                 N, W1.data_ptr(), None, 0, W2.data_ptr(), None, Ht.data_ptr(),
+                                 Y.data_ptr(), ws.data_ptr(), wsb, None)
+
+    assert call(p1, p3) == native.EQL_ERR_INVALID_ARG      # widths do not chain
+    assert call(p1, p2, nb - 4) == native.EQL_ERR_WORKSPACE
