@@ -3,13 +3,15 @@
 
 Default workload: the p4 (T=4) FP16 ViT-B MLP pair, N = 12608 rows (64 images x
 197 tokens), layer 1 C=192 -> D=768 (768 -> 3072 features), layer 2 C=768 ->
-D=192 (3072 -> 768) applied to layer 1's output.  One step = both layers, as
-one chained launch.  `value` = rows (tokens) per second over the whole job, inputs
+D=192 (3072 -> 768) applied to layer 1's output.  One step = the group DFT of X
+into tiled spectral planes, then both layers as one chained launch on SM pairs
+(the first layer's epilogue writes the second layer's planes).  `value` = rows (tokens) per second over the whole job, inputs
 resident in HBM; `e2e` = the same through the C ABI with the step's input copied
 from pinned host memory and the result read back, inside the timed region.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--workload p4_vitb_mlp_f16|p4_vitb_mlp_2calls_f16|p4_vitb_proj_f32|p4_vith_fc1_f16|
+       [--workload p4_vitb_mlp_f16|p4_vitb_mlp_fused_f16|p4_vitb_mlp_2calls_f16|
+                   p4_vitb_proj_f32|p4_vith_fc1_f16|
                    c8_1024_f16|p4_vith_fc1_fwd_bwd_f16|p4_vitb_mlp_block_f16|
                    p4_vitb_mlp_spectral_f16|p4m_vitb_mlp_f16|p4_conv3x3_f16] [--dp-path]
        [--wgrad-transform] [--no-dense] [--no-cpu-baseline] [--eager]
@@ -46,6 +48,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # workload name -> list of layer workloads applied in sequence (output feeds the next)
 PIPELINES = {
     "p4_vitb_mlp_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
+    "p4_vitb_mlp_fused_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
     "p4_vitb_mlp_2calls_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
     "p4_vitb_proj_f32": ["p4_vitb_proj_f32"],
     "p4_vith_fc1_f16": ["p4_vith_fc1_f16"],
@@ -64,7 +67,11 @@ SPECTRAL = {"p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectral_f16"}
 BACKWARD = {"p4_vith_fc1_fwd_bwd_f16"}
 # two-layer pipelines run as one chained launch (eqlinear_forward_chain: both
 # layers' tiles in one dynamic queue; bitwise the two separate calls)
-CHAINED = {"p4_vitb_mlp_f16", "p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectral_f16"}
+CHAINED = {"p4_vitb_mlp_fused_f16", "p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectral_f16"}
+# two-layer pipelines run on tiled spectral planes: one group-DFT launch, then both
+# layers in one chained launch on SM pairs (eqlinear_group_dft +
+# eqlinear_forward_chain_tiled; bitwise the per-layer tiled calls)
+TILED = {"p4_vitb_mlp_f16"}
 # per-layer output activation (fused into that layer's epilogue); default none
 ACTS = {"p4_vitb_mlp_block_f16": ["gelu", "none"]}
 
@@ -73,7 +80,11 @@ def acts_of(workload):
     return ACTS.get(workload, ["none"] * len(PIPELINES[workload]))
 DESCR = {
     "p4_vitb_mlp_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
-                       "C=768->D=192, T=4; both layers in one chained launch",
+                       "C=768->D=192, T=4; group DFT of X to tiled planes, then both layers "
+                       "in one chained launch on SM pairs",
+    "p4_vitb_mlp_fused_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
+                             "C=768->D=192, T=4; both layers in one chained launch, the "
+                             "group transforms fused into the GEMM kernel",
     "p4_vitb_mlp_2calls_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
                               "C=768->D=192, T=4; one launch per layer",
     "p4_vitb_proj_f32": "p4 EQ-Linear fp32 ViT-B projection: N=12608, C=D=192, T=4",
@@ -123,16 +134,18 @@ KERNEL_SOURCES = {
     "forward_chain": ("eql_tc_chain.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
     "conv": ("eql_tc_conv.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
     "backward_weight": ("eql_tc_wgrad.cu", "eql_tc_common.cuh"),
+    "forward_chain_tiled": ("eql_tc_pair.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
 }
 NCU_TRAFFIC = {
     ("forward", "4458390a32641562"): {"p4_vitb_mlp_2calls_f16": 58.33e6, "c8_1024_f16": 33.95e6,
                                       "p4_vith_fc1_f16": 48.86e6,
                                       "p4_vith_fc1_fwd_bwd_f16": 107.56e6,
                                       "p4m_vitb_mlp_f16": 57.75e6},
-    ("forward_chain", "350ff7855a00971d"): {"p4_vitb_mlp_f16": 89.45e6,
+    ("forward_chain", "350ff7855a00971d"): {"p4_vitb_mlp_fused_f16": 89.45e6,
                                             "p4_vitb_mlp_spectral_f16": 89.27e6,
                                             "p4_vitb_mlp_block_f16": 85.77e6},
     ("conv", "e00676af90759f5d"): {"p4_conv3x3_f16": 160.12e6},
+    ("forward_chain_tiled", "5f6ce7da20fa529c"): {"p4_vitb_mlp_f16": 92.44e6},
 }
 
 def kernel_traffic(family: str, workload: str):
@@ -507,6 +520,7 @@ def run_ours(args, workload):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     from group_circulant_gemm_b200 import EqLinearPlan, forward_chain, native
+    from group_circulant_gemm_b200.layer import forward_chain_tiled
     from group_circulant_gemm_b200.parallel import allreduce_grad_buffer
 
     backward = workload in BACKWARD
@@ -531,6 +545,10 @@ def run_ours(args, workload):
 
     # rotating input/output sets so the step's working set leaves L2 between steps
     per_set = sum(N * w.C * w.T * es + N * w.D * w.T * es for w in pipeline)
+    tiled = workload in TILED
+    if tiled:
+        # X's tiled planes (rows padded to the kernel's 128-row tile)
+        per_set += int(np.prod(plans[0].tiled_shape(N, pipeline[0].C))) * es
     if backward:
         per_set += sum(N * w.D * w.T * es + N * w.C * w.T * es for w in pipeline)
     # training: the forward and dX kernels save the group spectra of X and dY
@@ -568,6 +586,30 @@ def run_ours(args, workload):
         outs = [[torch.empty((4, N, pipeline[0].D), dtype=dt, device="cuda"), o[1]]
                 for o in outs]
     chained = workload in CHAINED
+    if tiled:
+        # the intermediate is the second layer's tiled planes, written by the first
+        # layer's epilogue
+        w1, w2 = pipeline
+        xts = [torch.empty(plans[0].tiled_shape(N, w1.C), dtype=dt, device="cuda")
+               for _ in range(nsets)]
+        outs = [[torch.empty(plans[0].tiled_shape(N, w1.D), dtype=dt, device="cuda"), o[1]]
+                for o in outs]
+        ws_tiled = torch.zeros(max(16, native.eqlinear_chain_tiled_workspace_bytes(
+            plans[0].handle, plans[1].handle, N)), dtype=torch.uint8, device="cuda")
+
+        def group_dft(i):
+            plans[0].group_dft(xs[i % nsets], out=xts[i % nsets])
+
+        def fwd_chain_tiled(i):
+            o = outs[i % nsets]
+            forward_chain_tiled(plans[0], plans[1], xts[i % nsets], N, whats[0], biases[0],
+                                whats[1], biases[1], act=acts[0], Ht=o[0], Y=o[1],
+                                workspace=ws_tiled)
+        # the transform reads X and writes its planes (the same bytes); its
+        # additions are not counted as the method's FLOPs
+        ops.append(("group_dft", "simt", 0.0, 2.0 * es * N * w1.C * w1.T, group_dft))
+        ops.append(("forward_chain_tiled", "tcgen05", sum(layer_flops(w) for w in pipeline),
+                    sum(layer_bytes(w) for w in pipeline), fwd_chain_tiled))
     if chained:
         ws_chain = torch.zeros(max(16, native.eqlinear_chain_workspace_bytes(
             plans[0].handle, plans[1].handle, N)), dtype=torch.uint8, device="cuda")
@@ -579,7 +621,7 @@ def run_ours(args, workload):
                           workspace=ws_chain)
         ops.append(("forward_chain", "tcgen05", sum(layer_flops(w) for w in pipeline),
                     sum(layer_bytes(w) for w in pipeline), fwd_chain))
-    for li, w in enumerate([] if chained else pipeline):
+    for li, w in enumerate([] if chained or tiled else pipeline):
         def fwd(i, li=li):
             x = xs[i % nsets] if li == 0 else outs[i % nsets][li - 1]
             if spectral and li == 0:

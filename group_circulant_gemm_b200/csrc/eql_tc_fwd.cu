@@ -28,9 +28,11 @@
 // Design (one persistent CTA per SM; tile = 128 rows x BD out-channels; K stage
 // = BK input channels, whose raw X tile is always 128 rows x 256 B = 32 KB):
 //   warp 0      TMA producer: the raw X tile of a stage, one 3-D box
-//               (64 halves x 2 row chunks x 128 rows, 128B-swizzled), 3-deep ring.
+//               (64 halves x 2 row chunks x 128 rows, 128B-swizzled), into a
+//               ring of Cfg<T>::X_ST slots (4 at T = 4, 3 at T = 8).
 //   warp 2      weight producer: one bulk copy per stage of a blob that
-//               prepare_weights pre-arranged in the MMA operand layout.
+//               prepare_weights pre-arranged in the MMA operand layout, into a
+//               ring of Cfg<T>::W_ST slots (2 at T = 4, 6 at T = 8).
 //   warp 1      TMEM allocator; lane 0 issues the MMAs of each K step:
 //               N = BD for each real frequency, N = 2 BD for Xr_k [Br_k|Bi_k],
 //               and N = BD for -Xi_k Bi_k (negate-A bit) and Xi_k Br_k.

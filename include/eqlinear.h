@@ -144,8 +144,8 @@ EQL_API const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t plan, i
  * 128 x 32 channels at T = 4, 64 x 16 at T = 8, in the kernel's swizzled
  * shared-memory order, the same values), so each pipeline stage is one copy.
  * At T = 4 two more follow: the same planes as the two-SM spectral kernel's
- * stages (forward, then adjoint; per 128 out-channels and 16 input channels,
- * each SM's half of the weights: 2 x 12 KB).
+ * stages (forward, then adjoint; per 128 out-channels and 32 input channels,
+ * each SM's 64 out-channels of the four planes X0, X2, Re, Im: 2 x 16 KB).
  */
 EQL_API size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t plan);
 

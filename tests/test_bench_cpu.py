@@ -20,7 +20,7 @@ def test_every_pipeline_resolves_and_chains():
         for a, b in zip(ws, ws[1:]):
             assert a.D == b.C and a.T == b.T and a.N == b.N, name
         assert name in bench.DESCR, name
-    for name in bench.CHAINED | bench.SPECTRAL:
+    for name in bench.CHAINED | bench.SPECTRAL | bench.TILED:
         assert len(bench.PIPELINES[name]) == 2, name
     for name in bench.BACKWARD:
         assert name in bench.PIPELINES
