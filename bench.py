@@ -285,6 +285,47 @@ def capture_graphs(step, nsets):
     return graphs
 
 
+def graph_op_times(step, nsets, op_steps, first):
+    """Per-launch device times of each op of a step, from CUDA graphs that hold
+    the step with event-record nodes around every launch (one graph per rotating
+    set).  Each replay runs alone (synchronised after it), so a launch's time
+    holds no host work: in eager launches the event before a kernel can complete
+    while the host is still encoding that kernel's arguments.  Returns an array
+    [op_steps, ops], or None when events cannot be captured (then the caller
+    times eager launches)."""
+    import torch
+    try:
+        gs, evs = [], []
+        for k in range(nsets):
+            e = []
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(first + k, e, external=True)
+            gs.append(g)
+            evs.append(e)
+        rows = []
+        for i in range(op_steps):
+            k = i % nsets
+            gs[k].replay()
+            torch.cuda.synchronize()
+            e = evs[k]
+            rows.append([e[2 * j].elapsed_time(e[2 * j + 1]) for j in range(len(e) // 2)])
+        return np.array(rows)
+    except Exception as exc:  # noqa: BLE001 - fall back to eager timing, say so
+        print(f"per-launch timing inside graphs unavailable ({exc}); timing eager launches",
+              file=sys.stderr)
+        return None
+
+
+def new_event(external: bool = False):
+    """A timing event recorded on the current stream (inside a graph capture,
+    `external` makes the record a node of the graph)."""
+    import torch
+    e = torch.cuda.Event(enable_timing=True, external=external)
+    e.record()
+    return e
+
+
 def dist_init():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -450,11 +491,10 @@ def dense_comparator(pipeline, backward, xs, dys, nsets, steps, rank, acts=None,
         bs.append(torch.from_numpy(inp["bias"]).cuda().repeat_interleave(w.T) if w.bias else None)
     outs = []
 
-    def step(i, events=None):
+    def step(i, events=None, external=False):
         def mark():
             if events is not None:
-                events.append(torch.cuda.Event(enable_timing=True))
-                events[-1].record(stream)
+                events.append(new_event(external))
         x = xs[i % nsets]
         for li in range(len(pipeline)):
             mark()
@@ -492,14 +532,19 @@ def dense_comparator(pipeline, backward, xs, dys, nsets, steps, rank, acts=None,
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / steps
     op_steps = steps
+    per_op = None
     if graphs is not None:
         op_steps = min(steps, 50)
-        for i in range(op_steps):
-            step(3 + i, ev)
-        torch.cuda.synchronize()
-    nops = len(ev) // 2 // op_steps
-    op_ms = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1])
-                      for j in range(len(ev) // 2)]).reshape(op_steps, nops).mean(axis=0)
+        per_op = graph_op_times(step, nsets, op_steps, 3)
+        if per_op is None:
+            for i in range(op_steps):
+                step(3 + i, ev)
+            torch.cuda.synchronize()
+    if per_op is None:
+        nops = len(ev) // 2 // op_steps
+        per_op = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1])
+                           for j in range(len(ev) // 2)]).reshape(op_steps, nops)
+    op_ms = per_op.mean(axis=0)
     flops = sum(dense_flops(w) for w in pipeline) + (2 * dense_flops(pipeline[0]) if backward else 0)
     return {"kind": "dense F.linear on the replicated (D*T x C*T) matrix, cuBLAS, same dtype, "
                     "GEMM time only" + ("; training step adds dY@M and dY^T@X" if backward else "")
@@ -689,15 +734,13 @@ def run_ours(args, workload):
         else:
             ops += [op_dx, op_dw]
 
-    def step(i, events=None):
+    def step(i, events=None, external=False):
         for _, _, _, _, fn in ops:
             if events is not None:
-                events.append(torch.cuda.Event(enable_timing=True))
-                events[-1].record(stream)
+                events.append(new_event(external))
             fn(i)
             if events is not None:
-                events.append(torch.cuda.Event(enable_timing=True))
-                events[-1].record(stream)
+                events.append(new_event(external))
 
     kernel_names = [k for _, k, _, _, _ in ops]
     # the clock sampler runs from the start of warm-up to the end of the timed region
@@ -739,16 +782,26 @@ def run_ours(args, workload):
     clk = clocks.stop() if rank == 0 else {}
     elapsed_ms = t0.elapsed_time(t1)
     op_steps = args.steps
+    launch_ms = None
     if graphs is not None:
-        # per-launch times: an eager pass with events around every launch
+        # per-launch times: the step's graphs again, with event nodes around every
+        # launch (eager launches if events cannot be captured)
         op_steps = min(args.steps, 100)
-        for i in range(op_steps):
-            step(args.warmup + i, ev)
-        torch.cuda.synchronize()
-    launch_ms = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1])
-                          for j in range(len(ev) // 2)]).reshape(op_steps, len(ops))
+        launch_ms = graph_op_times(step, nsets, op_steps, args.warmup)
+        if launch_ms is None:
+            for i in range(op_steps):
+                step(args.warmup + i, ev)
+            torch.cuda.synchronize()
+        for p in plans:
+            assert p.status() == 0
+    in_graph = launch_ms is not None
+    if launch_ms is None:
+        launch_ms = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1])
+                              for j in range(len(ev) // 2)]).reshape(op_steps, len(ops))
     timing = ("CUDA graph replay of each step (one graph per rotating set); per-launch times "
-              f"from {op_steps} eager steps with events around each launch"
+              + (f"from {op_steps} replays of the step's graphs with event nodes around each "
+                 "launch" if in_graph else
+                 f"from {op_steps} eager steps with events around each launch")
               if graphs is not None else "eager launches with events around each launch")
 
     # end to end through the ABI: pinned host inputs -> device, the step, results -> host
@@ -1011,15 +1064,13 @@ def run_conv(args, workload):
                      dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step(i, events=None):
+    def step(i, events=None, external=False):
         if events is not None:
-            events.append(torch.cuda.Event(enable_timing=True))
-            events[-1].record(stream)
+            events.append(new_event(external))
         p.conv_forward(xs[i % nsets], Wh, w.KH, w.KW, bias, pad=(w.ph, w.pw),
                        out=ys[i % nsets], workspace=ws)
         if events is not None:
-            events.append(torch.cuda.Event(enable_timing=True))
-            events[-1].record(stream)
+            events.append(new_event(external))
 
     clocks = ClockSampler(local)
     if rank == 0:
@@ -1052,15 +1103,21 @@ def run_conv(args, workload):
     clk = clocks.stop() if rank == 0 else {}
     elapsed_ms = t0.elapsed_time(t1)
     op_steps = args.steps
+    per_call = None
     if graphs is not None:
         op_steps = min(args.steps, 100)
-        for i in range(op_steps):
-            step(args.warmup + i, ev)
-        torch.cuda.synchronize()
-    launch_ms = float(np.mean([ev[2 * j].elapsed_time(ev[2 * j + 1])
-                               for j in range(len(ev) // 2)]))
+        per_call = graph_op_times(step, nsets, op_steps, args.warmup)
+        if per_call is None:
+            for i in range(op_steps):
+                step(args.warmup + i, ev)
+            torch.cuda.synchronize()
+    in_graph = per_call is not None
+    if per_call is None:
+        per_call = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(len(ev) // 2)])
+    launch_ms = float(np.mean(per_call))
     timing = ("CUDA graph replay of each step (one graph per rotating set); per-call time "
-              f"from {op_steps} eager steps with events around each call"
+              + (f"from {op_steps} replays of the step's graphs with event nodes around the "
+                 "call" if in_graph else f"from {op_steps} eager steps with events around each call")
               if graphs is not None else "eager launches with events around each call")
 
     x_pin = torch.from_numpy(x_host).pin_memory()
