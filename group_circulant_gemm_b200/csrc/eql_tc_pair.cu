@@ -69,6 +69,34 @@ namespace {
 using namespace tc;
 using namespace ftc;
 
+// Programmatic dependent launch: a kernel launched with launch_dependent may
+// start while the previous kernel in the stream is finishing; it calls
+// grid_dependency_wait (which returns once that kernel has completed and its
+// memory is visible) before touching global memory.  grid_launch_dependents
+// lets the next such kernel launch once every CTA of this one has called it or
+// exited.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 constexpr int PR_BD = 128;                       // out-channels per tile
 constexpr int PR_KC = 16;                        // input channels per K step
 constexpr int PR_KSS = 2;                        // K steps per stage (32 channels)
@@ -377,6 +405,7 @@ struct PairSched {
   int total;         // tasks
   int lag;           // (chain) layer-1 row blocks queued ahead of layer 2
   int flag_target;   // (chain) counter value of a complete layer-1 row block
+  int npairs;        // (chain) clusters in the grid
   PairLayer L[2];
 };
 struct PairTask {
@@ -442,8 +471,11 @@ __device__ __noinline__ bool ring_wait(uint64_t* b, uint32_t parity, int* abort_
 }
 
 // Bounded wait until a layer-1 row block is stored, then order the TMA loads
-// that follow after the acquire.
-__device__ __noinline__ bool pair_wait_row(const int* flag, int target, int* abort_flag,
+// that follow after the acquire.  Each of the block's `consumers` waiters then
+// adds one; the last of them returns the counter to zero (nothing reads it
+// again in this launch), so a launch leaves its counters zero without a pass
+// over them at the end.
+__device__ __noinline__ bool pair_wait_row(int* flag, int target, int consumers, int* abort_flag,
                                            int* status) {
   const uint64_t t0 = gtimer();
   while (true) {
@@ -451,6 +483,7 @@ __device__ __noinline__ bool pair_wait_row(const int* flag, int target, int* abo
     asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
     if (v >= target) {
       asm volatile("fence.proxy.async.global;" ::: "memory");
+      if (atomicAdd(flag, 1) == target + consumers - 1) atomicExch(flag, 0);
       return true;
     }
     if (*(volatile int*)abort_flag) return false;
@@ -481,6 +514,9 @@ struct TaskSource {
     ++n;
     if (!wait_bounded(&ring->empty[q], ph ^ 1, abort_flag, status)) return false;
     const int v = atomicAdd(counter, 1);
+    // every pair's leader stops at its first id past the end, so the counter's
+    // last value is total + npairs - 1: that fetch returns it to zero
+    if (v == sc.total + sc.npairs - 1) atomicExch(counter, 0);
     *id = v < sc.total ? v : -1;
     ring->id[q] = *id;
     const uint32_t peer_id = peer_addr(smem_u32(&ring->id[q]), 1);
@@ -599,7 +635,13 @@ __device__ __forceinline__ void pair_epilogue(uint32_t lane_addr, int ch, int la
 
 // CHAIN = 0: one layer, output IO1 with ACT1.  CHAIN = 1: layer 1 writes H as
 // tiled planes with ACT1, layer 2 writes Y spatially; `sync` = [next task,
-// CTAs finished, one counter per row block], zero at launch and left zero.
+// unused, one counter per row block], zero at launch and left zero (the last
+// fetch of the task counter and the last waiter on a row counter reset them).
+//
+// Launched as a programmatic dependent of the previous kernel in the stream:
+// the prologue (barriers, TMEM allocation) overlaps that kernel's last wave,
+// and griddepcontrol.wait, which returns once that kernel has completed and
+// its writes are visible, comes before the first global-memory access.
 template <int ACT1, int IO1, int CHAIN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
     eq_pair_tc_kernel(const __grid_constant__ CUtensorMap map_x1,
@@ -647,6 +689,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before any remote arrive or TMA completion
   tc_fence_after();
+  grid_dependency_wait();
   const uint32_t tmem = bars->tmem_base;
   TaskSource<CHAIN> src{ring, peer_addr(smem_u32(&ring->empty[0]), 0), sync, 0u, pair, npairs};
 
@@ -670,7 +713,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
         const CUtensorMap* mw = t.layer ? &map_w2 : &map_w1;
         const int row = t.prow * 256 + 128 * (int)rank;
         if (CHAIN && t.layer == 1 &&
-            !(ok = pair_wait_row(&sync[2 + t.prow], sc.flag_target, abort_flag, status)))
+            !(ok = pair_wait_row(&sync[2 + t.prow], sc.flag_target, 2 * sc.L[1].n_dt,
+                                 abort_flag, status)))
           break;
         for (int ks = 0; ks < L.n_ks; ++ks, ++it) {
           const int s = it % PR_ST;
@@ -794,6 +838,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
     __syncwarp();
   }
 
+  grid_launch_dependents();  // this CTA has no more work: the next kernel may launch
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // no CTA leaves while its pair may still touch its shared memory
@@ -801,17 +846,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols));
-  }
-  if (CHAIN && threadIdx.x == 0) {
-    // every role of this CTA is done with the counters; the last CTA clears them
-    __threadfence();
-    if (atomicAdd(&sync[1], 1) == (int)gridDim.x - 1) {
-      __threadfence();
-      for (int i = 0; i < sc.n_prow; ++i) sync[2 + i] = 0;
-      sync[0] = 0;
-      __threadfence();
-      sync[1] = 0;
-    }
   }
 }
 
@@ -854,6 +888,8 @@ __global__ void pair_tile_weights_kernel(const __half* __restrict__ planes, int 
 __global__ void group_dft_tiled_kernel(const uint4* __restrict__ X, int64_t N, int64_t Np, int C,
                                        uint8_t* __restrict__ out) {
   constexpr int G = 4;  // channel blocks per warp
+  grid_dependency_wait();
+  grid_launch_dependents();
   const int KB = C / 16;
   const int KBG = (KB + G - 1) / G;
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -964,9 +1000,9 @@ cudaError_t launch_group_dft_tiled(const void* X, int64_t N, int C, void* out, c
   if (C % 16 != 0) return cudaErrorInvalidValue;
   const int64_t Np = tiled_rows(N);
   const int64_t threads = Np / 4 * ((C / 16 + 3) / 4) * 32;
-  group_dft_tiled_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-      static_cast<const uint4*>(X), N, Np, C, static_cast<uint8_t*>(out));
-  return cudaGetLastError();
+  return launch_dependent(group_dft_tiled_kernel, dim3((unsigned)((threads + 255) / 256)),
+                          dim3(256), 0, st, static_cast<const uint4*>(X), N, Np, C,
+                          static_cast<uint8_t*>(out));
 }
 
 bool pair_tc_supported(int64_t N, int Cin, int Cout) {
@@ -1059,8 +1095,8 @@ cudaError_t launch_pair_tc(const void* Xt, int64_t N, int Cin, int Cout, const v
                                     : eq_pair_tc_kernel<0, kIoSpatial, 0>);
   int npairs = pair_capacity((const void*)kernel, num_sms);
   if (npairs > sc.total) npairs = sc.total;
-  kernel<<<2 * npairs, PR_THREADS, PR_SMEM, st>>>(mx, mw, my, mx, mw, my, sc, nullptr, status);
-  return cudaGetLastError();
+  return launch_dependent(kernel, dim3(2 * npairs), dim3(PR_THREADS), PR_SMEM, st, mx, mw, my, mx,
+                          mw, my, sc, (int*)nullptr, status);
 }
 
 size_t pair_chain_sync_bytes(int64_t N) { return (size_t)(2 + (N + 255) / 256) * sizeof(int); }
@@ -1101,8 +1137,9 @@ cudaError_t launch_pair_chain_tc(const void* Xt, int64_t N, int C0, int C1, int 
   if (lag < wave) lag = wave;
   sc.lag = lag < sc.n_prow ? lag : sc.n_prow;
   sc.flag_target = 2 * kEpiWarps * sc.L[0].n_dt;
-  kernel<<<2 * npairs, PR_THREADS, PR_SMEM, st>>>(mx1, mw1, mh_st, mh_ld, mw2, my, sc, sync, status);
-  return cudaGetLastError();
+  sc.npairs = npairs;
+  return launch_dependent(kernel, dim3(2 * npairs), dim3(PR_THREADS), PR_SMEM, st, mx1, mw1, mh_st,
+                          mh_ld, mw2, my, sc, sync, status);
 }
 
 }  // namespace eql
