@@ -121,9 +121,9 @@ constexpr uint32_t PR_OFF_BAR = PR_OFF_BIAS + kEpiWarps * 128;
 constexpr uint32_t PR_SMEM = PR_OFF_BAR + 512 + 1024;
 static_assert(PR_STAGE % 1024 == 0, "stage slots stay 1024-byte aligned");
 static_assert(PR_SMEM <= 232448, "shared memory budget");
-// weight regions of a K step (byte offsets): this CTA's 64 rows (out-channels
-// 64 * rank ..) of A0, A2, Br, Bi
-constexpr uint32_t PR_R0 = 0, PR_R1 = 64 * PR_ROWB, PR_R2 = 128 * PR_ROWB, PR_R3 = 192 * PR_ROWB;
+// weight regions of a K step: this CTA's 64 rows (out-channels 64 * rank ..) of
+// A0, A2, Br, Bi, each 64 x 32 B (a narrow tile: 32 rows each, out-channels
+// 32 * rank ..)
 
 struct PairBars {
   uint64_t full[PR_ST];   // leader: both CTAs' bytes of a stage landed
@@ -397,8 +397,16 @@ struct PairLayer {
   int n_dt;   // out-channel tiles
   int n_ks;   // stages of 32 input channels
   int Cout;
+  int narrow;        // the last out-channel tile holds <= 64 channels: N = 64 products
+  int narrow_line0;  // weight-tile line where that tile's stages start
   const __half* bias;
 };
+// The last out-channel tile of a layer whose remainder is at most 64 channels
+// runs N = 64 products (each SM 32 weight rows per plane): half the weight bytes
+// and tensor time of a zero-padded 128-channel tile.
+__device__ __forceinline__ bool pair_narrow(const PairLayer& L, int dt) {
+  return L.narrow && dt == L.n_dt - 1;
+}
 struct PairSched {
   int64_t N;
   int n_prow;        // 256-row blocks
@@ -569,6 +577,13 @@ __device__ __forceinline__ void pair_epilogue(uint32_t lane_addr, int ch, int la
                                               uint32_t stg_s, const __half* bsm, int dbase,
                                               int Cout, uint32_t acc_empty_leader,
                                               const Store& store) {
+  if (dbase >= Cout) {
+    // the narrow last tile: this warp's 64 columns hold no output channel
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) arrive_remote_relaxed(acc_empty_leader);
+    return;
+  }
   // read the whole tile share out of TMEM: slices 0-1 into staging, 2-7 held;
   // each slice's TMEM load is issued before the previous slice is computed, so
   // one wait::ld covers it while that computation runs
@@ -721,12 +736,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
           const uint32_t ph = (it / PR_ST) & 1;
           if (!(ok = wait_bounded(&bars->empty[s], ph ^ 1, abort_flag, status))) break;
           const uint32_t full_leader = peer_addr(smem_u32(&bars->full[s]), 0);
-          if (rank == 0) mbar_expect_tx(&bars->full[s], 2 * PR_STAGE);
+          const bool nar = pair_narrow(L, t.dt);
+          if (rank == 0)
+            mbar_expect_tx(&bars->full[s], 2 * (PR_XBYTES + (nar ? PR_WBYTES / 2 : PR_WBYTES)));
           const uint32_t slot = sbase + s * PR_STAGE;
           // planes: lines row/4 .. +32 of channel blocks 2ks, 2ks+1, all four planes
           tma_load_4d_pair(slot, mx, full_leader, 0, row / 4, PR_KSS * ks, 0);
-          const int wline = ((t.dt * L.n_ks + ks) * 2 + (int)rank) * PR_WLINES;
-          tma_load_2d_pair(slot + PR_XBYTES, mw, full_leader, 0, wline);
+          // this CTA's weight rows of the stage, boxes of 64 lines (8 KB)
+          if (nar) {
+            const int wline = L.narrow_line0 + (ks * 2 + (int)rank) * (PR_WLINES / 2);
+            tma_load_2d_pair(slot + PR_XBYTES, mw, full_leader, 0, wline);
+          } else {
+            const int wline = ((t.dt * L.n_ks + ks) * 2 + (int)rank) * PR_WLINES;
+            tma_load_2d_pair(slot + PR_XBYTES, mw, full_leader, 0, wline);
+            tma_load_2d_pair(slot + PR_XBYTES + PR_WBYTES / 2, mw, full_leader, 0,
+                             wline + PR_WLINES / 2);
+          }
           issued_phase[s] = (int)ph;
         }
       }
@@ -744,8 +769,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
     // ~70 cycles a tcgen05.mma costs its issuing thread are paid twice in parallel.
     if (rank == 0 && lane == 0) {
       const int who = warp == 1 ? 0 : 1;
-      const uint32_t id_n1 = idesc_f16(256, PR_BD);
-      const uint32_t id_neg = idesc_f16(256, PR_BD, true);
+      const uint32_t id_full = idesc_f16(256, PR_BD), id_full_neg = idesc_f16(256, PR_BD, true);
+      const uint32_t id_nar = idesc_f16(256, PR_BD / 2), id_nar_neg = idesc_f16(256, PR_BD / 2, true);
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       while (ok) {
@@ -753,6 +778,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
         if (!(ok = src.take1(sc, &id, abort_flag, status)) || id < 0) break;
         const PairTask t = pair_decode<CHAIN>(id, sc);
         const int n_ks = sc.L[t.layer].n_ks;
+        // a narrow tile: N = 64, this CTA's 32 rows per weight plane
+        const bool nar = pair_narrow(sc.L[t.layer], t.dt);
+        const uint32_t id_n1 = nar ? id_nar : id_full, id_neg = nar ? id_nar_neg : id_full_neg;
+        const uint32_t w_kstep = nar ? PR_WKS / 2 : PR_WKS;
+        const uint32_t w_plane = nar ? 32 * PR_ROWB : 64 * PR_ROWB;
         if (!(ok = wait_bounded(&bars->acc_empty, (tcount & 1) ^ 1, abort_flag, status))) break;
         tc_fence_after();
         for (int ks = 0; ks < n_ks; ++ks, ++it) {
@@ -762,19 +792,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
           const uint32_t xs = sbase + s * PR_STAGE, ws = xs + PR_XBYTES;
 #pragma unroll
           for (int kk = 0; kk < PR_KSS; ++kk) {
-            const uint32_t xa = xs + kk * PR_XBLK, wb = ws + kk * PR_WKS;
+            const uint32_t xa = xs + kk * PR_XBLK, wb = ws + kk * w_kstep;
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
             const uint64_t xr = desc_kmajor<32>(xa + 2 * PR_XPLANE);
             const uint64_t xi = desc_kmajor<32>(xa + 3 * PR_XPLANE);
-            const uint64_t br = desc_kmajor<32>(wb + PR_R2), bi = desc_kmajor<32>(wb + PR_R3);
+            const uint64_t br = desc_kmajor<32>(wb + 2 * w_plane);
+            const uint64_t bi = desc_kmajor<32>(wb + 3 * w_plane);
             if (who == 0) {
               umma_pair(tmem + 0, desc_kmajor<32>(xa + 0 * PR_XPLANE),
-                        desc_kmajor<32>(wb + PR_R0), id_n1, acc);                   // Y0
+                        desc_kmajor<32>(wb), id_n1, acc);                           // Y0
               umma_pair(tmem + 2 * PR_BD, xr, br, id_n1, acc);                      // Y1r
               umma_pair(tmem + 2 * PR_BD, xi, bi, id_neg, 1u);                      // -Xi Bi
             } else {
               umma_pair(tmem + PR_BD, desc_kmajor<32>(xa + 1 * PR_XPLANE),
-                        desc_kmajor<32>(wb + PR_R1), id_n1, acc);                   // Y2
+                        desc_kmajor<32>(wb + w_plane), id_n1, acc);                 // Y2
               umma_pair(tmem + 3 * PR_BD, xr, bi, id_n1, acc);                      // Y1i
               umma_pair(tmem + 3 * PR_BD, xi, br, id_n1, 1u);
             }
@@ -850,30 +881,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PR_THREADS, 1)
 }
 
 // Prepared planes [P][Cout][Cin] (P = 5 at T = 4: A0, A2, Br, Bi, -Bi) -> the
-// pair kernel's weight stages: blob (dt, stage, rank) = two K steps (channels
-// 32*stage + 16*kk ..+16) of 256 rows x 16 channels (32 bytes, 32-byte swizzle:
-// 16-byte piece ^= (row / 4) % 2): rows 64j .. 64j+63 hold plane j (A0, A2, Br,
-// Bi) at out-channels dt*128 + 64*rank + (row % 64); zero past the matrix.  One
-// thread per 16-byte piece.
+// pair kernel's weight stages.  A 128-channel tile: blob (dt, stage, rank) =
+// two K steps (channels 32*stage + 16*kk ..+16) of 256 rows x 16 channels (32
+// bytes, 32-byte swizzle: 16-byte piece ^= (row / 4) % 2); rows 64j .. 64j+63
+// hold plane j (A0, A2, Br, Bi) at out-channels dt*128 + 64*rank + (row % 64).
+// The narrow last tile (<= 64 channels, after the full ones): blob (stage,
+// rank) = two K steps of 128 rows, rows 32j .. 32j+31 = plane j at out-channels
+// dt*128 + 32*rank + (row % 32).  Zero past the matrix.  One thread per 16-byte
+// piece.
 __global__ void pair_tile_weights_kernel(const __half* __restrict__ planes, int Cin, int Cout,
-                                         int n_ks, int64_t n_pieces, uint4* __restrict__ tiles) {
+                                         int n_ks, int n_full, int64_t n_pieces,
+                                         uint4* __restrict__ tiles) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n_pieces) return;
-  const int piece = (int)(idx & 1);
-  const int r = (int)((idx >> 1) % PR_WROWS);
-  const int64_t kblob = (idx >> 1) / PR_WROWS;  // (dt, stage, rank, kk)
+  const int64_t full_pieces = (int64_t)n_full * n_ks * 2 * (PR_WBYTES / 16);
+  const bool nar = idx >= full_pieces;
+  const int64_t j = nar ? idx - full_pieces : idx;
+  const int rows = nar ? PR_WROWS / 2 : PR_WROWS;  // rows of one K step of a blob
+  const int piece = (int)(j & 1);
+  const int r = (int)((j >> 1) % rows);
+  const int64_t kblob = (j >> 1) / rows;  // (dt, stage, rank, kk), narrow: (stage, rank, kk)
   const int kk = (int)(kblob % PR_KSS);
   const int64_t blob = kblob / PR_KSS;
   const int rank = (int)(blob & 1);
   const int64_t dk = blob >> 1;
-  const int dt = (int)(dk / n_ks), ks = (int)(dk % n_ks) * PR_KSS + kk;
-  const int plane = r >> 6;
-  const int d = dt * PR_BD + 64 * rank + (r & 63);
+  const int dt = nar ? n_full : (int)(dk / n_ks);
+  const int ks = (int)(dk % n_ks) * PR_KSS + kk;
+  const int per = rows / 4;  // rows per plane
+  const int plane = r / per;
+  const int d = dt * PR_BD + per * rank + (r % per);
   const int c0 = ks * PR_KC + piece * 8;
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
   if (d < Cout && c0 < Cin)  // Cin % 16 == 0: the 8 channels are all in range
     v = *reinterpret_cast<const uint4*>(planes + ((int64_t)plane * Cout + d) * Cin + c0);
-  const int64_t dst = kblob * PR_WKS + r * PR_ROWB + ((piece ^ ((r >> 2) & 1)) << 4);
+  const int64_t base = nar ? full_pieces * 16 : 0;
+  const int64_t dst = base + kblob * (rows * PR_ROWB) + r * PR_ROWB + ((piece ^ ((r >> 2) & 1)) << 4);
   tiles[dst >> 4] = v;
 }
 
@@ -1010,18 +1052,28 @@ bool pair_tc_supported(int64_t N, int Cin, int Cout) {
          Cout >= 16;
 }
 
+namespace {
+// out-channel tiles of a layer: full 128-channel tiles, then a narrow one when
+// the remainder is at most 64 channels
+int pair_n_dt(int Cout) { return (Cout + PR_BD - 1) / PR_BD; }
+bool pair_has_narrow(int Cout) { return Cout - (pair_n_dt(Cout) - 1) * PR_BD <= PR_BD / 2; }
+int pair_n_ks(int Cin) { return (Cin + PR_KC * PR_KSS - 1) / (PR_KC * PR_KSS); }
+}  // namespace
+
 size_t pair_tile_bytes(int Cin, int Cout) {
-  const int kst = PR_KC * PR_KSS;
-  const size_t n_dt = (size_t)(Cout + PR_BD - 1) / PR_BD, n_st = (size_t)(Cin + kst - 1) / kst;
-  return n_dt * n_st * 2 * PR_WBYTES;
+  const size_t n_st = (size_t)pair_n_ks(Cin);
+  const size_t nar = pair_has_narrow(Cout) ? 1 : 0, n_full = (size_t)pair_n_dt(Cout) - nar;
+  return n_full * n_st * 2 * PR_WBYTES + nar * n_st * 2 * (PR_WBYTES / 2);
 }
 
 cudaError_t launch_pair_tile_weights(const void* planes, int Cin, int Cout, void* tiles,
                                      cudaStream_t st) {
-  const int n_ks = (Cin + PR_KC * PR_KSS - 1) / (PR_KC * PR_KSS);  // stages
+  const int n_ks = pair_n_ks(Cin);
+  const int n_full = pair_n_dt(Cout) - (pair_has_narrow(Cout) ? 1 : 0);
   const int64_t n_pieces = (int64_t)pair_tile_bytes(Cin, Cout) / 16;
   pair_tile_weights_kernel<<<(unsigned)((n_pieces + 255) / 256), 256, 0, st>>>(
-      static_cast<const __half*>(planes), Cin, Cout, n_ks, n_pieces, static_cast<uint4*>(tiles));
+      static_cast<const __half*>(planes), Cin, Cout, n_ks, n_full, n_pieces,
+      static_cast<uint4*>(tiles));
   return cudaGetLastError();
 }
 
@@ -1032,7 +1084,7 @@ bool encode_pair_weights(CUtensorMap* m, const void* tiles, int Cin, int Cout) {
   const uint64_t lines = pair_tile_bytes(Cin, Cout) / 128;
   cuuint64_t dims[2] = {64, (cuuint64_t)lines};
   cuuint64_t strides[1] = {128};
-  cuuint32_t box[2] = {64, PR_WLINES};
+  cuuint32_t box[2] = {64, PR_WLINES / 2};
   cuuint32_t estr[2] = {1, 1};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(tiles), dims, strides,
                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -1054,9 +1106,11 @@ bool encode_rows_store(CUtensorMap* m, void* Y, int Cout, int64_t N) {
 
 PairLayer pair_layer(int Cin, int Cout, const void* bias) {
   PairLayer L;
-  L.n_dt = (Cout + PR_BD - 1) / PR_BD;
-  L.n_ks = (Cin + PR_KC * PR_KSS - 1) / (PR_KC * PR_KSS);  // a last half stage reads zeros
+  L.n_dt = pair_n_dt(Cout);
+  L.n_ks = pair_n_ks(Cin);  // a last half stage reads zeros
   L.Cout = Cout;
+  L.narrow = pair_has_narrow(Cout) ? 1 : 0;
+  L.narrow_line0 = (L.n_dt - L.narrow) * L.n_ks * 2 * PR_WLINES;
   L.bias = static_cast<const __half*>(bias);
   return L;
 }
