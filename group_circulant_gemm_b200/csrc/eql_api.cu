@@ -74,6 +74,18 @@ const void* pair_fwd_tiles(const eqlinear_plan_s* p, const void* W_hat) {
 const void* pair_adj_tiles(const eqlinear_plan_s* p, const void* W_hat) {
   return static_cast<const char*>(pair_fwd_tiles(p, W_hat)) + eql::pair_tile_bytes(p->C, p->D);
 }
+// p4 FP32 plans with C, D multiples of 8 hold the 3xTF32 pair kernel's weight
+// stages after their planes (forward, then adjoint)
+bool has_tf32_tiles(const eqlinear_plan_s* p) {
+  return p->group == 0 && p->T == 4 && p->dtype == EQL_F32 && p->C % 8 == 0 && p->D % 8 == 0;
+}
+const void* tf32_fwd_tiles(const eqlinear_plan_s* p, const void* W_hat) {
+  return static_cast<const char*>(W_hat) +
+         2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
+}
+const void* tf32_adj_tiles(const eqlinear_plan_s* p, const void* W_hat) {
+  return static_cast<const char*>(tf32_fwd_tiles(p, W_hat)) + eql::pair_tf32_tile_bytes(p->C, p->D);
+}
 
 // Forward-shaped product used by both eqlinear_forward (Cin=C, Cout=D) and
 // eqlinear_backward_input (Cin=D, Cout=C).
@@ -217,6 +229,8 @@ size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t p) {
   size_t bytes = 2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
   if (has_tiles(p)) bytes += eql::tc_tile_bytes(p->T, p->C, p->D) + eql::tc_tile_bytes(p->T, p->D, p->C);
   if (has_pair_tiles(p)) bytes += eql::pair_tile_bytes(p->C, p->D) + eql::pair_tile_bytes(p->D, p->C);
+  if (has_tf32_tiles(p))
+    bytes += eql::pair_tf32_tile_bytes(p->C, p->D) + eql::pair_tf32_tile_bytes(p->D, p->C);
   return bytes;
 }
 
@@ -238,6 +252,14 @@ eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, voi
                                               const_cast<void*>(fwd_tiles(p, W_hat)), st, 1));
   }
   s = from_cuda(eql::launch_prepare(p->T, to_dt(p->dtype), W, p->C, p->D, fwd, adj, p->tw, st));
+  if (s == EQL_OK && has_tf32_tiles(p)) {
+    s = from_cuda(eql::launch_pair_tf32_tile_weights(
+        fwd, p->C, p->D, const_cast<void*>(tf32_fwd_tiles(p, W_hat)), st));
+    if (s == EQL_OK)
+      s = from_cuda(eql::launch_pair_tf32_tile_weights(
+          adj, p->D, p->C, const_cast<void*>(tf32_adj_tiles(p, W_hat)), st));
+    return s;
+  }
   if (s != EQL_OK || !has_tiles(p)) return s;
   s = from_cuda(eql::launch_tile_weights(p->T, fwd, p->C, p->D, const_cast<void*>(fwd_tiles(p, W_hat)),
                                          st));
@@ -325,6 +347,7 @@ eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t p, const void* 
 
 size_t eqlinear_tiled_spectrum_bytes(eqlinear_plan_t p, int64_t N, int channels) {
   if (!p || N < 0 || channels <= 0) return 0;
+  if (p->dtype == EQL_F32) return eql::tiled_tf32_planes_bytes(N, channels);
   return eql::tiled_planes_bytes(N, channels);
 }
 
@@ -340,6 +363,17 @@ static eqlinear_status_t pair_io(eqlinear_plan_t p, const void* Xt, int64_t N, c
   if (!aligned16(Xt) || !aligned16(W_hat) || !aligned16(out) || (bias && !aligned16(bias)))
     return EQL_ERR_ALIGNMENT;
   const int Cin = adjoint ? p->D : p->C, Cout = adjoint ? p->C : p->D;
+  if (p->dtype == EQL_F32) {
+    // 3xTF32 on SM pairs; the output is spatial only
+    if (!has_tf32_tiles(p) || p->kernel == EQL_KERNEL_SIMT || spectral_out ||
+        !eql::pair_tf32_supported(N, Cin, Cout))
+      return EQL_ERR_UNSUPPORTED;
+    eqlinear_status_t s = check_plan_device(p);
+    if (s != EQL_OK) return s;
+    return from_cuda(eql::launch_pair_tf32(
+        Xt, N, Cin, Cout, adjoint ? tf32_adj_tiles(p, W_hat) : tf32_fwd_tiles(p, W_hat), bias, out,
+        p->status, p->num_sms, (int)act, (cudaStream_t)stream));
+  }
   if (!has_pair_tiles(p) || p->kernel == EQL_KERNEL_SIMT ||
       !eql::pair_tc_supported(N, Cin, Cout))
     return EQL_ERR_UNSUPPORTED;
@@ -356,13 +390,14 @@ eqlinear_status_t eqlinear_group_dft(eqlinear_plan_t p, const void* X, int64_t N
   EQL_TRACE();
   if (!p || N < 0) return EQL_ERR_INVALID_ARG;
   if (channels != p->C && channels != p->D) return EQL_ERR_INVALID_ARG;
-  if (p->T != 4 || p->dtype != EQL_F16 || p->group != 0 || channels % 16 != 0)
-    return EQL_ERR_UNSUPPORTED;
+  const bool f32 = p->dtype == EQL_F32;
+  if (p->T != 4 || p->group != 0 || channels % (f32 ? 8 : 16) != 0) return EQL_ERR_UNSUPPORTED;
   if (N == 0) return EQL_OK;
   if (!X || !Xt) return EQL_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Xt)) return EQL_ERR_ALIGNMENT;
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
+  if (f32) return from_cuda(eql::launch_group_dft_tf32(X, N, channels, Xt, (cudaStream_t)stream));
   return from_cuda(eql::launch_group_dft_tiled(X, N, channels, Xt, (cudaStream_t)stream));
 }
 

@@ -133,6 +133,20 @@ cudaError_t launch_pair_chain_tc(const void* Xt, int64_t N, int C0, int C1, int 
                                  const void* b2, void* Ht, void* Y, int* sync, int* status,
                                  int num_sms, int act1, cudaStream_t st);
 
+// FP32 p4 layer on SM pairs with 3xTF32 split precision (eql_tc_pair32.cu):
+// tiled hi/lo planes of the input (8 planes, 8 FP32 channels per 32-byte row),
+// weight stages from prepared FP32 planes [5][Cout][Cin], Y [N][Cout*4] FP32.
+// Cin, Cout multiples of 8.
+bool pair_tf32_supported(int64_t N, int Cin, int Cout);
+size_t tiled_tf32_planes_bytes(int64_t N, int channels);
+size_t pair_tf32_tile_bytes(int Cin, int Cout);
+cudaError_t launch_pair_tf32_tile_weights(const void* planes, int Cin, int Cout, void* tiles,
+                                          cudaStream_t st);
+cudaError_t launch_group_dft_tf32(const void* X, int64_t N, int C, void* out, cudaStream_t st);
+cudaError_t launch_pair_tf32(const void* Xt, int64_t N, int Cin, int Cout, const void* tiles,
+                             const void* bias, void* Y, int* status, int num_sms, int act,
+                             cudaStream_t st);
+
 // dst[i] = src[i] rounded to nearest-even in dt (a copy for F32), i < n.
 cudaError_t launch_cast_from_f32(DType dt, const float* src, void* dst, int64_t n,
                                  cudaStream_t st);

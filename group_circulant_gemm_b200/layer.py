@@ -114,10 +114,14 @@ class EqLinearPlan:
     # --- the frequency-domain form on tiled planes (see eqlinear_group_dft)
 
     def tiled_shape(self, N: int, channels: int):
-        """Shape of tiled planes of N rows: (4 planes, channels/16 blocks, Np rows,
-        16 halves per row in the swizzled order of the header), Np = N rounded up
-        to a multiple of 128."""
-        return (4, channels // 16, (N + 127) // 128 * 128, 16)
+        """Shape of tiled planes of N rows, Np = N rounded up to a multiple of 128.
+        FP16: (4 planes, channels/16 blocks, Np rows, 16 halves per row in the
+        swizzled order of the header).  FP32: (8 planes = the TF32 hi parts of the
+        four, then the lo parts, channels/8 blocks, Np rows, 8 floats per row)."""
+        Np = (N + 127) // 128 * 128
+        if self.dtype == torch.float32:
+            return (8, channels // 8, Np, 8)
+        return (4, channels // 16, Np, 16)
 
     def group_dft(self, X, out=None) -> torch.Tensor:
         """Tiled planes of X [N, c*4] (c = C for an input, D for an upstream gradient)."""
