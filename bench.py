@@ -51,6 +51,7 @@ PIPELINES = {
     "p4_vitb_mlp_fused_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
     "p4_vitb_mlp_2calls_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
     "p4_vitb_proj_f32": ["p4_vitb_proj_f32"],
+    "p4_vitb_proj_f32_simt": ["p4_vitb_proj_f32"],
     "p4_vith_fc1_f16": ["p4_vith_fc1_f16"],
     "c8_1024_f16": ["c8_1024_f16"],
     "p4_vith_fc1_fwd_bwd_f16": ["p4_vith_fc1_f16"],
@@ -72,6 +73,9 @@ CHAINED = {"p4_vitb_mlp_fused_f16", "p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectr
 # layers in one chained launch on SM pairs (eqlinear_group_dft +
 # eqlinear_forward_chain_tiled; bitwise the per-layer tiled calls)
 TILED = {"p4_vitb_mlp_f16"}
+# FP32 layers on the tensor cores with 3xTF32 split precision: one group-DFT
+# launch (TF32 hi/lo planes), then the pair kernel (eqlinear_forward_tiled)
+TILED_F32 = {"p4_vitb_proj_f32"}
 # per-layer output activation (fused into that layer's epilogue); default none
 ACTS = {"p4_vitb_mlp_block_f16": ["gelu", "none"]}
 
@@ -87,7 +91,10 @@ DESCR = {
                              "group transforms fused into the GEMM kernel",
     "p4_vitb_mlp_2calls_f16": "p4 EQ-Linear fp16 ViT-B MLP pair: N=12608, C=192->D=768 then "
                               "C=768->D=192, T=4; one launch per layer",
-    "p4_vitb_proj_f32": "p4 EQ-Linear fp32 ViT-B projection: N=12608, C=D=192, T=4",
+    "p4_vitb_proj_f32": "p4 EQ-Linear fp32 ViT-B projection: N=12608, C=D=192, T=4; group DFT "
+                        "to TF32 hi/lo planes, then 3xTF32 products on SM-pair tensor cores",
+    "p4_vitb_proj_f32_simt": "p4 EQ-Linear fp32 ViT-B projection: N=12608, C=D=192, T=4; FP32 FMA "
+                             "on the CUDA cores",
     "p4_vith_fc1_f16": "p4 EQ-Linear fp16 ViT-H fc1: N=8224, C=320->D=1280, T=4",
     "c8_1024_f16": "cyclic T=8 EQ-Linear fp16: N=16384, C=D=128",
     "p4_vith_fc1_fwd_bwd_f16": "p4 EQ-Linear fp16 ViT-H fc1 forward + dX + dW: N=8224, "
@@ -591,6 +598,10 @@ def run_ours(args, workload):
     # rotating input/output sets so the step's working set leaves L2 between steps
     per_set = sum(N * w.C * w.T * es + N * w.D * w.T * es for w in pipeline)
     tiled = workload in TILED
+    tiled32 = workload in TILED_F32
+    if tiled32:
+        # the TF32 hi/lo planes of X (8 planes, rows padded to the 128-row tile)
+        per_set += int(np.prod(plans[0].tiled_shape(N, pipeline[0].C))) * 4
     if tiled:
         # X's tiled planes (rows padded to the kernel's 128-row tile)
         per_set += int(np.prod(plans[0].tiled_shape(N, pipeline[0].C))) * es
@@ -666,7 +677,24 @@ def run_ours(args, workload):
                           workspace=ws_chain)
         ops.append(("forward_chain", "tcgen05", sum(layer_flops(w) for w in pipeline),
                     sum(layer_bytes(w) for w in pipeline), fwd_chain))
-    for li, w in enumerate([] if chained or tiled else pipeline):
+    if tiled32:
+        w0 = pipeline[0]
+        xts = [torch.empty(plans[0].tiled_shape(N, w0.C), dtype=dt, device="cuda")
+               for _ in range(nsets)]
+
+        def group_dft32(i):
+            plans[0].group_dft(xs[i % nsets], out=xts[i % nsets])
+
+        def fwd_tf32(i):
+            plans[0].forward_tiled(xts[i % nsets], N, whats[0], biases[0], act=acts[0],
+                                   out=outs[i % nsets][0])
+        # the transform reads X and writes hi and lo planes (twice X's bytes); the
+        # products read both planes, the weights' hi/lo stages, and write Y
+        ops.append(("group_dft", "simt", 0.0, 3.0 * es * N * w0.C * w0.T, group_dft32))
+        ops.append(("forward_tiled", "tcgen05-3xtf32", layer_flops(w0),
+                    es * (2 * N * w0.C * w0.T + N * w0.D * w0.T + 2 * 4 * w0.C * w0.D + w0.D),
+                    fwd_tf32))
+    for li, w in enumerate([] if chained or tiled or tiled32 else pipeline):
         def fwd(i, li=li):
             x = xs[i % nsets] if li == 0 else outs[i % nsets][li - 1]
             if spectral and li == 0:
@@ -900,7 +928,16 @@ def run_ours(args, workload):
         flops_per_launch = dflops / dcount
         bytes_per_launch = dbytes / dcount
         achieved = flops_per_launch / (mean_launch_ms / 1e3) / 1e12
-        if dkern == "tcgen05":
+        if dkern == "tcgen05-3xtf32":
+            # TF32 peak from the measured BF16 one and the nominal TF32:BF16 ratio
+            # (1.1 : 2.25 PFLOP/s dense); the split precision runs three TF32
+            # products per product of the method, so 1/3 is this path's ceiling
+            peak = peaks["bf16_tflops"] * 1.1 / 2.25
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": kernel_traffic(dlabel, workload),
+                    "peak_source": f"{peak_src} dense bf16 burst x 1.1/2.25 (TF32)",
+                    "mma_flops_per_method_flop": 3}
+        elif dkern == "tcgen05":
             peak = peaks["bf16_tflops"]
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak,
