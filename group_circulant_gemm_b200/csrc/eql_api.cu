@@ -83,6 +83,20 @@ const void* tf32_fwd_tiles(const eqlinear_plan_s* p, const void* W_hat) {
   return static_cast<const char*>(W_hat) +
          2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
 }
+// FP16 T = 8 plans (cyclic or D4) with C, D multiples of 16 also hold the
+// eight-plane pair kernel's weight stages: cyclic forward then adjoint, after
+// the one-CTA tiles; D4 forward only, after its forward tiles
+bool has_pair8_tiles(const eqlinear_plan_s* p) {
+  return p->T == 8 && p->dtype == EQL_F16 && p->C % 16 == 0 && p->D % 16 == 0 && has_tiles(p);
+}
+const void* pair8_fwd_tiles(const eqlinear_plan_s* p, const void* W_hat) {
+  if (p->group == 1)
+    return static_cast<const char*>(fwd_tiles(p, W_hat)) + eql::tc_tile_bytes(8, p->C, p->D);
+  return static_cast<const char*>(adj_tiles(p, W_hat)) + eql::tc_tile_bytes(p->T, p->D, p->C);
+}
+const void* pair8_adj_tiles(const eqlinear_plan_s* p, const void* W_hat) {
+  return static_cast<const char*>(pair8_fwd_tiles(p, W_hat)) + eql::pair8_tile_bytes(p->C, p->D);
+}
 const void* tf32_adj_tiles(const eqlinear_plan_s* p, const void* W_hat) {
   return static_cast<const char*>(tf32_fwd_tiles(p, W_hat)) + eql::pair_tf32_tile_bytes(p->C, p->D);
 }
@@ -225,12 +239,15 @@ const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t p, int64_t N) {
 size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t p) {
   if (!p) return 0;
   if (p->group == 1)
-    return d4_ok(p) ? 8 * plane_elems(p) * 2 + eql::tc_tile_bytes(8, p->C, p->D) : 0;
+    return d4_ok(p) ? 8 * plane_elems(p) * 2 + eql::tc_tile_bytes(8, p->C, p->D) +
+                          (has_pair8_tiles(p) ? eql::pair8_tile_bytes(p->C, p->D) : 0)
+                    : 0;
   size_t bytes = 2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
   if (has_tiles(p)) bytes += eql::tc_tile_bytes(p->T, p->C, p->D) + eql::tc_tile_bytes(p->T, p->D, p->C);
   if (has_pair_tiles(p)) bytes += eql::pair_tile_bytes(p->C, p->D) + eql::pair_tile_bytes(p->D, p->C);
   if (has_tf32_tiles(p))
     bytes += eql::pair_tf32_tile_bytes(p->C, p->D) + eql::pair_tf32_tile_bytes(p->D, p->C);
+  if (has_pair8_tiles(p)) bytes += eql::pair8_tile_bytes(p->C, p->D) + eql::pair8_tile_bytes(p->D, p->C);
   return bytes;
 }
 
@@ -248,8 +265,11 @@ eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, voi
     if (!d4_ok(p)) return EQL_ERR_UNSUPPORTED;
     s = from_cuda(eql::launch_prepare_d4(W, p->C, p->D, fwd, st));
     if (s != EQL_OK) return s;
-    return from_cuda(eql::launch_tile_weights(8, fwd, p->C, p->D,
-                                              const_cast<void*>(fwd_tiles(p, W_hat)), st, 1));
+    s = from_cuda(eql::launch_tile_weights(8, fwd, p->C, p->D,
+                                           const_cast<void*>(fwd_tiles(p, W_hat)), st, 1));
+    if (s != EQL_OK || !has_pair8_tiles(p)) return s;
+    return from_cuda(eql::launch_pair8_tile_weights(
+        fwd, p->C, p->D, const_cast<void*>(pair8_fwd_tiles(p, W_hat)), st));
   }
   s = from_cuda(eql::launch_prepare(p->T, to_dt(p->dtype), W, p->C, p->D, fwd, adj, p->tw, st));
   if (s == EQL_OK && has_tf32_tiles(p)) {
@@ -266,6 +286,14 @@ eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, voi
   if (s != EQL_OK) return s;
   s = from_cuda(eql::launch_tile_weights(p->T, adj, p->D, p->C,
                                          const_cast<void*>(adj_tiles(p, W_hat)), st));
+  if (s == EQL_OK && has_pair8_tiles(p)) {
+    s = from_cuda(eql::launch_pair8_tile_weights(
+        fwd, p->C, p->D, const_cast<void*>(pair8_fwd_tiles(p, W_hat)), st));
+    if (s == EQL_OK)
+      s = from_cuda(eql::launch_pair8_tile_weights(
+          adj, p->D, p->C, const_cast<void*>(pair8_adj_tiles(p, W_hat)), st));
+    return s;
+  }
   if (s != EQL_OK || !has_pair_tiles(p)) return s;
   s = from_cuda(eql::launch_pair_tile_weights(fwd, p->C, p->D,
                                               const_cast<void*>(pair_fwd_tiles(p, W_hat)), st));
@@ -348,6 +376,7 @@ eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t p, const void* 
 size_t eqlinear_tiled_spectrum_bytes(eqlinear_plan_t p, int64_t N, int channels) {
   if (!p || N < 0 || channels <= 0) return 0;
   if (p->dtype == EQL_F32) return eql::tiled_tf32_planes_bytes(N, channels);
+  if (p->T == 8) return eql::tiled8_planes_bytes(N, channels);
   return eql::tiled_planes_bytes(N, channels);
 }
 
@@ -363,6 +392,17 @@ static eqlinear_status_t pair_io(eqlinear_plan_t p, const void* Xt, int64_t N, c
   if (!aligned16(Xt) || !aligned16(W_hat) || !aligned16(out) || (bias && !aligned16(bias)))
     return EQL_ERR_ALIGNMENT;
   const int Cin = adjoint ? p->D : p->C, Cout = adjoint ? p->C : p->D;
+  if (p->T == 8) {
+    // eight-plane pair kernel; spatial output; D4 plans have no adjoint stages
+    if (!has_pair8_tiles(p) || p->kernel == EQL_KERNEL_SIMT || spectral_out ||
+        (adjoint && p->group == 1) || !eql::pair8_supported(N, Cin, Cout))
+      return EQL_ERR_UNSUPPORTED;
+    eqlinear_status_t s = check_plan_device(p);
+    if (s != EQL_OK) return s;
+    return from_cuda(eql::launch_pair8_tc(
+        Xt, N, Cin, Cout, adjoint ? pair8_adj_tiles(p, W_hat) : pair8_fwd_tiles(p, W_hat), bias,
+        out, p->status, p->num_sms, (int)act, p->group, (cudaStream_t)stream));
+  }
   if (p->dtype == EQL_F32) {
     // 3xTF32 on SM pairs; the output is spatial only
     if (!has_tf32_tiles(p) || p->kernel == EQL_KERNEL_SIMT || spectral_out ||
@@ -391,13 +431,18 @@ eqlinear_status_t eqlinear_group_dft(eqlinear_plan_t p, const void* X, int64_t N
   if (!p || N < 0) return EQL_ERR_INVALID_ARG;
   if (channels != p->C && channels != p->D) return EQL_ERR_INVALID_ARG;
   const bool f32 = p->dtype == EQL_F32;
-  if (p->T != 4 || p->group != 0 || channels % (f32 ? 8 : 16) != 0) return EQL_ERR_UNSUPPORTED;
+  const bool eight = p->T == 8 && !f32 && channels % 16 == 0;
+  if (!eight && (p->T != 4 || p->group != 0 || channels % (f32 ? 8 : 16) != 0))
+    return EQL_ERR_UNSUPPORTED;
   if (N == 0) return EQL_OK;
   if (!X || !Xt) return EQL_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Xt)) return EQL_ERR_ALIGNMENT;
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
   if (f32) return from_cuda(eql::launch_group_dft_tf32(X, N, channels, Xt, (cudaStream_t)stream));
+  if (eight)
+    return from_cuda(
+        eql::launch_group_dft8_tiled(X, N, channels, p->group, Xt, (cudaStream_t)stream));
   return from_cuda(eql::launch_group_dft_tiled(X, N, channels, Xt, (cudaStream_t)stream));
 }
 

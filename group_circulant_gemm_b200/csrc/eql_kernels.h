@@ -147,6 +147,21 @@ cudaError_t launch_pair_tf32(const void* Xt, int64_t N, int Cin, int Cout, const
                              const void* bias, void* Y, int* status, int num_sms, int act,
                              cudaStream_t st);
 
+// Eight-plane layers on SM pairs (eql_tc_pair8.cu): cyclic T = 8 (group 0) and
+// the dihedral group D4 (group 1), FP16: tiled planes of the group Fourier
+// transform (8 planes, 16 channels per 32-byte row), weight stages from 8
+// prepared planes [.][Cout][Cin], Y [N][Cout*8].  Cin, Cout multiples of 16.
+bool pair8_supported(int64_t N, int Cin, int Cout);
+size_t tiled8_planes_bytes(int64_t N, int channels);
+size_t pair8_tile_bytes(int Cin, int Cout);
+cudaError_t launch_pair8_tile_weights(const void* planes, int Cin, int Cout, void* tiles,
+                                      cudaStream_t st);
+cudaError_t launch_group_dft8_tiled(const void* X, int64_t N, int C, int group, void* out,
+                                    cudaStream_t st);
+cudaError_t launch_pair8_tc(const void* Xt, int64_t N, int Cin, int Cout, const void* tiles,
+                            const void* bias, void* Y, int* status, int num_sms, int act,
+                            int group, cudaStream_t st);
+
 // dst[i] = src[i] rounded to nearest-even in dt (a copy for F32), i < n.
 cudaError_t launch_cast_from_f32(DType dt, const float* src, void* dst, int64_t n,
                                  cudaStream_t st);

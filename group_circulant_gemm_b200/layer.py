@@ -116,11 +116,14 @@ class EqLinearPlan:
     def tiled_shape(self, N: int, channels: int):
         """Shape of tiled planes of N rows, Np = N rounded up to a multiple of 128.
         FP16: (4 planes, channels/16 blocks, Np rows, 16 halves per row in the
-        swizzled order of the header).  FP32: (8 planes = the TF32 hi parts of the
-        four, then the lo parts, channels/8 blocks, Np rows, 8 floats per row)."""
+        swizzled order of the header); 8 planes at T = 8 (cyclic or D4).  FP32: (8
+        planes = the TF32 hi parts of the four, then the lo parts, channels/8
+        blocks, Np rows, 8 floats per row)."""
         Np = (N + 127) // 128 * 128
         if self.dtype == torch.float32:
             return (8, channels // 8, Np, 8)
+        if self.T == 8:
+            return (8, channels // 16, Np, 16)
         return (4, channels // 16, Np, 16)
 
     def group_dft(self, X, out=None) -> torch.Tensor:
