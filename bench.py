@@ -11,9 +11,10 @@ from pinned host memory and the result read back, inside the timed region.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
        [--workload p4_vitb_mlp_f16|p4_vitb_mlp_fused_f16|p4_vitb_mlp_2calls_f16|
-                   p4_vitb_proj_f32|p4_vith_fc1_f16|
-                   c8_1024_f16|p4_vith_fc1_fwd_bwd_f16|p4_vitb_mlp_block_f16|
-                   p4_vitb_mlp_spectral_f16|p4m_vitb_mlp_f16|p4_conv3x3_f16] [--dp-path]
+                   p4_vitb_proj_f32|p4_vitb_proj_f32_simt|p4_vith_fc1_f16|
+                   c8_1024_f16|c8_1024_tiled_f16|p4_vith_fc1_fwd_bwd_f16|
+                   p4_vitb_mlp_block_f16|p4_vitb_mlp_spectral_f16|p4m_vitb_mlp_f16|
+                   p4m_vitb_mlp_fused_f16|p4_conv3x3_f16] [--dp-path]
        [--wgrad-transform] [--no-dense] [--no-cpu-baseline] [--eager]
 The training workload (p4_vith_fc1_fwd_bwd_f16) is forward, dX and dW; the
 forward and dX kernels save the group spectra of X and dY, which dW multiplies
@@ -54,14 +55,16 @@ PIPELINES = {
     "p4_vitb_proj_f32_simt": ["p4_vitb_proj_f32"],
     "p4_vith_fc1_f16": ["p4_vith_fc1_f16"],
     "c8_1024_f16": ["c8_1024_f16"],
+    "c8_1024_tiled_f16": ["c8_1024_f16"],
     "p4_vith_fc1_fwd_bwd_f16": ["p4_vith_fc1_f16"],
     "p4_vitb_mlp_block_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
     "p4_vitb_mlp_spectral_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
     "p4m_vitb_mlp_f16": ["p4m_vitb_fc1_f16", "p4m_vitb_fc2_f16"],
+    "p4m_vitb_mlp_fused_f16": ["p4m_vitb_fc1_f16", "p4m_vitb_fc2_f16"],
 }
 # pipelines whose layers are over the dihedral group D4 (T = 8 elements) instead
 # of the cyclic group
-DIHEDRAL = {"p4m_vitb_mlp_f16"}
+DIHEDRAL = {"p4m_vitb_mlp_f16", "p4m_vitb_mlp_fused_f16"}
 # two-layer pipelines whose intermediate stays in the frequency domain (the first
 # layer's epilogue writes the second layer's operand planes)
 SPECTRAL = {"p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectral_f16"}
@@ -73,9 +76,11 @@ CHAINED = {"p4_vitb_mlp_fused_f16", "p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectr
 # layers in one chained launch on SM pairs (eqlinear_group_dft +
 # eqlinear_forward_chain_tiled; bitwise the per-layer tiled calls)
 TILED = {"p4_vitb_mlp_f16"}
-# FP32 layers on the tensor cores with 3xTF32 split precision: one group-DFT
-# launch (TF32 hi/lo planes), then the pair kernel (eqlinear_forward_tiled)
-TILED_F32 = {"p4_vitb_proj_f32"}
+# layers in the frequency-domain form, one layer at a time: per layer a group
+# Fourier transform launch (tiled planes; TF32 hi/lo planes for FP32), then the
+# pair kernel (eqlinear_forward_tiled): the FP32 layer with 3xTF32 split
+# precision, the cyclic T = 8 layer and the D4 layers with eight planes
+TILED_LAYERS = {"p4_vitb_proj_f32", "c8_1024_tiled_f16", "p4m_vitb_mlp_f16"}
 # per-layer output activation (fused into that layer's epilogue); default none
 ACTS = {"p4_vitb_mlp_block_f16": ["gelu", "none"]}
 
@@ -96,7 +101,10 @@ DESCR = {
     "p4_vitb_proj_f32_simt": "p4 EQ-Linear fp32 ViT-B projection: N=12608, C=D=192, T=4; FP32 FMA "
                              "on the CUDA cores",
     "p4_vith_fc1_f16": "p4 EQ-Linear fp16 ViT-H fc1: N=8224, C=320->D=1280, T=4",
-    "c8_1024_f16": "cyclic T=8 EQ-Linear fp16: N=16384, C=D=128",
+    "c8_1024_f16": "cyclic T=8 EQ-Linear fp16: N=16384, C=D=128; group DFT fused into the "
+                   "one-CTA GEMM kernel",
+    "c8_1024_tiled_f16": "cyclic T=8 EQ-Linear fp16: N=16384, C=D=128; group DFT to eight tiled "
+                         "planes, then the products on SM pairs",
     "p4_vith_fc1_fwd_bwd_f16": "p4 EQ-Linear fp16 ViT-H fc1 forward + dX + dW: N=8224, "
                                "C=320->D=1280, T=4",
     "p4_vitb_mlp_block_f16": "p4 EQ-MLP block fp16 ViT-B: N=12608, EQ-Linear 192->768 + bias + "
@@ -107,7 +115,11 @@ DESCR = {
                                 "spectral planes; one chained launch",
     "p4m_vitb_mlp_f16": "p4m (dihedral D4, 8 elements) EQ-Linear fp16 ViT-B MLP pair: N=12608, "
                         "C=96->D=384 then C=384->D=96 per group element (768->3072->768 "
-                        "features); one launch per layer",
+                        "features); per layer the group Fourier transform to eight tiled "
+                        "planes, then the products on SM pairs",
+    "p4m_vitb_mlp_fused_f16": "p4m (dihedral D4, 8 elements) EQ-Linear fp16 ViT-B MLP pair: "
+                              "N=12608, C=96->D=384 then C=384->D=96 per group element; one "
+                              "launch of the fused one-CTA kernel per layer",
 }
 
 
@@ -598,10 +610,11 @@ def run_ours(args, workload):
     # rotating input/output sets so the step's working set leaves L2 between steps
     per_set = sum(N * w.C * w.T * es + N * w.D * w.T * es for w in pipeline)
     tiled = workload in TILED
-    tiled32 = workload in TILED_F32
-    if tiled32:
-        # the TF32 hi/lo planes of X (8 planes, rows padded to the 128-row tile)
-        per_set += int(np.prod(plans[0].tiled_shape(N, pipeline[0].C))) * 4
+    tiled_layers = workload in TILED_LAYERS
+    if tiled_layers:
+        # every layer input's tiled planes (rows padded to the 128-row tile)
+        per_set += sum(int(np.prod(plans[li].tiled_shape(N, w.C))) * es
+                       for li, w in enumerate(pipeline))
     if tiled:
         # X's tiled planes (rows padded to the kernel's 128-row tile)
         per_set += int(np.prod(plans[0].tiled_shape(N, pipeline[0].C))) * es
@@ -677,24 +690,26 @@ def run_ours(args, workload):
                           workspace=ws_chain)
         ops.append(("forward_chain", "tcgen05", sum(layer_flops(w) for w in pipeline),
                     sum(layer_bytes(w) for w in pipeline), fwd_chain))
-    if tiled32:
-        w0 = pipeline[0]
-        xts = [torch.empty(plans[0].tiled_shape(N, w0.C), dtype=dt, device="cuda")
-               for _ in range(nsets)]
+    if tiled_layers:
+        # planes / input bytes: the FP32 form stores TF32 hi and lo parts
+        pf = 2 if dt == torch.float32 else 1
+        tkern = "tcgen05-3xtf32" if dt == torch.float32 else "tcgen05"
+        xts = [[torch.empty(plans[li].tiled_shape(N, w.C), dtype=dt, device="cuda")
+                for li, w in enumerate(pipeline)] for _ in range(nsets)]
+        for li, w in enumerate(pipeline):
+            def dft_l(i, li=li):
+                x = xs[i % nsets] if li == 0 else outs[i % nsets][li - 1]
+                plans[li].group_dft(x, out=xts[i % nsets][li])
 
-        def group_dft32(i):
-            plans[0].group_dft(xs[i % nsets], out=xts[i % nsets])
-
-        def fwd_tf32(i):
-            plans[0].forward_tiled(xts[i % nsets], N, whats[0], biases[0], act=acts[0],
-                                   out=outs[i % nsets][0])
-        # the transform reads X and writes hi and lo planes (twice X's bytes); the
-        # products read both planes, the weights' hi/lo stages, and write Y
-        ops.append(("group_dft", "simt", 0.0, 3.0 * es * N * w0.C * w0.T, group_dft32))
-        ops.append(("forward_tiled", "tcgen05-3xtf32", layer_flops(w0),
-                    es * (2 * N * w0.C * w0.T + N * w0.D * w0.T + 2 * 4 * w0.C * w0.D + w0.D),
-                    fwd_tf32))
-    for li, w in enumerate([] if chained or tiled or tiled32 else pipeline):
+            def fwd_l(i, li=li):
+                plans[li].forward_tiled(xts[i % nsets][li], N, whats[li], biases[li],
+                                        act=acts[li], out=outs[i % nsets][li])
+            # the transform reads the input and writes its planes; the products read
+            # the planes and the weight stages and write the output
+            ops.append(("group_dft", "simt", 0.0, (1 + pf) * es * N * w.C * w.T, dft_l))
+            ops.append(("forward_tiled", tkern, layer_flops(w),
+                        layer_bytes(w) + (pf - 1) * es * N * w.C * w.T, fwd_l))
+    for li, w in enumerate([] if chained or tiled or tiled_layers else pipeline):
         def fwd(i, li=li):
             x = xs[i % nsets] if li == 0 else outs[i % nsets][li - 1]
             if spectral and li == 0:
