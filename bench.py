@@ -153,18 +153,17 @@ KERNEL_SOURCES = {
     "forward_chain": ("eql_tc_chain.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
     "conv": ("eql_tc_conv.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
     "backward_weight": ("eql_tc_wgrad.cu", "eql_tc_common.cuh"),
-    "forward_chain_tiled": ("eql_tc_pair.cu", "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
+    "forward_chain_tiled": ("eql_tc_pair.cu", "eql_tc_pair_common.cuh", "eql_tc_fwd_parts.cuh",
+                            "eql_tc_common.cuh"),
+    "forward_tiled": ("eql_tc_pair32.cu", "eql_tc_pair8.cu", "eql_tc_pair_common.cuh",
+                      "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
 }
 NCU_TRAFFIC = {
-    ("forward", "4458390a32641562"): {"p4_vitb_mlp_2calls_f16": 58.33e6, "c8_1024_f16": 33.95e6,
-                                      "p4_vith_fc1_f16": 48.86e6,
-                                      "p4_vith_fc1_fwd_bwd_f16": 107.56e6,
-                                      "p4m_vitb_mlp_f16": 57.75e6},
-    ("forward_chain", "350ff7855a00971d"): {"p4_vitb_mlp_fused_f16": 89.45e6,
-                                            "p4_vitb_mlp_spectral_f16": 89.27e6,
-                                            "p4_vitb_mlp_block_f16": 85.77e6},
-    ("conv", "e00676af90759f5d"): {"p4_conv3x3_f16": 160.12e6},
-    ("forward_chain_tiled", "5f6ce7da20fa529c"): {"p4_vitb_mlp_f16": 92.44e6},
+    ("forward", "443ba94f5b306a59"): {"p4_vitb_mlp_2calls_f16": 58.96e6, "c8_1024_f16": 34.20e6, "p4_vith_fc1_f16": 51.20e6, "p4_vith_fc1_fwd_bwd_f16": 109.13e6, "p4m_vitb_mlp_fused_f16": 57.79e6},
+    ("forward_chain", "246b0f491b3357c1"): {"p4_vitb_mlp_fused_f16": 89.59e6, "p4_vitb_mlp_spectral_f16": 80.93e6, "p4_vitb_mlp_block_f16": 81.74e6},
+    ("conv", "30f615e6470be609"): {"p4_conv3x3_f16": 162.29e6},
+    ("forward_chain_tiled", "46882cfee44bc9af"): {"p4_vitb_mlp_f16": 103.14e6},
+    ("forward_tiled", "99717903cdc1492d"): {"p4_vitb_proj_f32": 85.78e6, "p4m_vitb_mlp_f16": 58.38e6, "c8_1024_tiled_f16": 34.38e6},
 }
 
 def kernel_traffic(family: str, workload: str):
