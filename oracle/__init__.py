@@ -92,6 +92,10 @@ def _load():
             lib.eqlo_conv_forward.restype = i64
             lib.eqlo_d4_forward.argtypes = [i64, i64, i64, dp, dp, dp, dp]
             lib.eqlo_d4_forward.restype = i64
+            lib.eqlo_d4_backward_input.argtypes = [i64, i64, i64, dp, dp, dp]
+            lib.eqlo_d4_backward_input.restype = i64
+            lib.eqlo_d4_backward_weight.argtypes = [i64, i64, i64, dp, dp, dp, dp]
+            lib.eqlo_d4_backward_weight.restype = i64
             lib.eqlo_set_threads.argtypes = [ctypes.c_int]
             lib.eqlo_set_threads.restype = None
             _lib = lib
@@ -226,6 +230,33 @@ def d4_forward(X, W, bias=None, return_macs: bool = False, act: str = "none"):
     if act == "gelu":
         _load().eqlo_gelu(Y.size, _ptr(Y))
     return (Y, macs) if return_macs else Y
+
+
+def d4_backward_input(dY, W):
+    """dX[N, C*8] in float64 from dY[N, D*8] and W[D, C, 8]: the gradient of
+    d4_forward with respect to X."""
+    dY, W = _f64(dY), _f64(W)
+    D, C, G = W.shape
+    if G != 8 or dY.ndim != 2 or dY.shape[1] != D * 8:
+        raise ValueError("dY must be [N, D*8] and W [D, C, 8]")
+    N = dY.shape[0]
+    dX = np.empty((N, C * 8), dtype=np.float64)
+    _load().eqlo_d4_backward_input(N, C, D, _ptr(dY), _ptr(W), _ptr(dX))
+    return dX
+
+
+def d4_backward_weight(X, dY, D: int):
+    """(dW[D, C, 8], dbias[D]) in float64 from X[N, C*8] and dY[N, D*8]: the
+    gradients of d4_forward with respect to W and the bias."""
+    X, dY = _f64(X), _f64(dY)
+    N = X.shape[0]
+    C = X.shape[1] // 8
+    if X.shape[1] != C * 8 or dY.shape != (N, D * 8):
+        raise ValueError("shape mismatch")
+    dW = np.empty((D, C, 8), dtype=np.float64)
+    db = np.empty((D,), dtype=np.float64)
+    _load().eqlo_d4_backward_weight(N, C, D, _ptr(X), _ptr(dY), _ptr(dW), _ptr(db))
+    return dW, db
 
 
 def conv_forward(T: int, X, Wc, bias=None, pad=(0, 0), return_macs: bool = False):

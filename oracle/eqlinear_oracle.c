@@ -349,3 +349,49 @@ int64_t eqlo_d4_forward(int64_t N, int64_t C, int64_t D, const double* X, const 
   }
   return N * D * C * 64;
 }
+
+/*
+ * Gradients of the D4 layer (the definition above, differentiated term by term):
+ *   dX[n][c*8+h] = sum_{d,g} W[d][c][g^-1 h] * dY[n][d*8+g]
+ *   dW[d][c][u]  = sum_{n,g} dY[n][d*8+g] * X[n][c*8+g u]     (h = g u)
+ *   dbias[d]     = sum_{n,g} dY[n][d*8+g]
+ * Each returns the number of real multiply-adds (N * D * C * 64).
+ */
+int64_t eqlo_d4_backward_input(int64_t N, int64_t C, int64_t D, const double* dY,
+                               const double* W, double* dX) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t c = 0; c < C; ++c) {
+      for (int h = 0; h < 8; ++h) {
+        double acc = 0.0;
+        for (int64_t d = 0; d < D; ++d)
+          for (int g = 0; g < 8; ++g)
+            acc += W[(d * C + c) * 8 + d4_mul(d4_inv(g), h)] * dY[(n * D + d) * 8 + g];
+        dX[(n * C + c) * 8 + h] = acc;
+      }
+    }
+  }
+  return N * D * C * 64;
+}
+
+int64_t eqlo_d4_backward_weight(int64_t N, int64_t C, int64_t D, const double* X,
+                                const double* dY, double* dW, double* dbias) {
+#pragma omp parallel for schedule(static)
+  for (int64_t dc = 0; dc < D * C; ++dc) {
+    const int64_t d = dc / C, c = dc % C;
+    for (int u = 0; u < 8; ++u) {
+      double acc = 0.0;
+      for (int64_t n = 0; n < N; ++n)
+        for (int g = 0; g < 8; ++g)
+          acc += dY[(n * D + d) * 8 + g] * X[(n * C + c) * 8 + d4_mul(g, u)];
+      dW[dc * 8 + u] = acc;
+    }
+  }
+  for (int64_t d = 0; d < D; ++d) {
+    double acc = 0.0;
+    for (int64_t n = 0; n < N; ++n)
+      for (int g = 0; g < 8; ++g) acc += dY[(n * D + d) * 8 + g];
+    dbias[d] = acc;
+  }
+  return N * D * C * 64;
+}
