@@ -84,8 +84,8 @@ const void* tf32_fwd_tiles(const eqlinear_plan_s* p, const void* W_hat) {
          2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
 }
 // FP16 T = 8 plans (cyclic or D4) with C, D multiples of 16 also hold the
-// eight-plane pair kernel's weight stages: cyclic forward then adjoint, after
-// the one-CTA tiles; D4 forward only, after its forward tiles
+// eight-plane pair kernel's weight stages, forward then adjoint: cyclic after the
+// one-CTA tiles, D4 after its forward tiles
 bool has_pair8_tiles(const eqlinear_plan_s* p) {
   return p->T == 8 && p->dtype == EQL_F16 && p->C % 16 == 0 && p->D % 16 == 0 && has_tiles(p);
 }
@@ -228,7 +228,8 @@ static bool wgrad_use_tc(eqlinear_plan_t p, int64_t N, const void* X, const void
 }
 
 const char* eqlinear_backward_weight_kernel_name(eqlinear_plan_t p, int64_t N) {
-  if (!p || p->group == 1) return "unsupported";
+  if (!p) return "unsupported";
+  if (p->group == 1) return p->kernel == EQL_KERNEL_TCGEN05 ? "unsupported" : "simt";
   const void* aligned = reinterpret_cast<const void*>(uintptr_t(256));
   const bool tc_ok = wgrad_tc_ok(p, N, aligned, aligned);
   if (p->kernel == EQL_KERNEL_TCGEN05) return tc_ok ? "tcgen05" : "unsupported";
@@ -240,7 +241,9 @@ size_t eqlinear_prepared_weight_bytes(eqlinear_plan_t p) {
   if (!p) return 0;
   if (p->group == 1)
     return d4_ok(p) ? 8 * plane_elems(p) * 2 + eql::tc_tile_bytes(8, p->C, p->D) +
-                          (has_pair8_tiles(p) ? eql::pair8_tile_bytes(p->C, p->D) : 0)
+                          (has_pair8_tiles(p) ? eql::pair8_tile_bytes(p->C, p->D) +
+                                                    eql::pair8_tile_bytes(p->D, p->C)
+                                              : 0)
                     : 0;
   size_t bytes = 2 * (size_t)eql::spec_planes(p->T) * plane_elems(p) * elem_size(p->dtype);
   if (has_tiles(p)) bytes += eql::tc_tile_bytes(p->T, p->C, p->D) + eql::tc_tile_bytes(p->T, p->D, p->C);
@@ -268,8 +271,11 @@ eqlinear_status_t eqlinear_prepare_weights(eqlinear_plan_t p, const void* W, voi
     s = from_cuda(eql::launch_tile_weights(8, fwd, p->C, p->D,
                                            const_cast<void*>(fwd_tiles(p, W_hat)), st, 1));
     if (s != EQL_OK || !has_pair8_tiles(p)) return s;
-    return from_cuda(eql::launch_pair8_tile_weights(
+    s = from_cuda(eql::launch_pair8_tile_weights(
         fwd, p->C, p->D, const_cast<void*>(pair8_fwd_tiles(p, W_hat)), st));
+    if (s != EQL_OK) return s;
+    return from_cuda(eql::launch_pair8_tile_weights(
+        fwd, p->D, p->C, const_cast<void*>(pair8_adj_tiles(p, W_hat)), st, 1));
   }
   s = from_cuda(eql::launch_prepare(p->T, to_dt(p->dtype), W, p->C, p->D, fwd, adj, p->tw, st));
   if (s == EQL_OK && has_tf32_tiles(p)) {
@@ -393,9 +399,9 @@ static eqlinear_status_t pair_io(eqlinear_plan_t p, const void* Xt, int64_t N, c
     return EQL_ERR_ALIGNMENT;
   const int Cin = adjoint ? p->D : p->C, Cout = adjoint ? p->C : p->D;
   if (p->T == 8) {
-    // eight-plane pair kernel; spatial output; D4 plans have no adjoint stages
+    // eight-plane pair kernel; spatial output
     if (!has_pair8_tiles(p) || p->kernel == EQL_KERNEL_SIMT || spectral_out ||
-        (adjoint && p->group == 1) || !eql::pair8_supported(N, Cin, Cout))
+        !eql::pair8_supported(N, Cin, Cout))
       return EQL_ERR_UNSUPPORTED;
     eqlinear_status_t s = check_plan_device(p);
     if (s != EQL_OK) return s;
@@ -686,6 +692,7 @@ eqlinear_status_t eqlinear_backward_input(eqlinear_plan_t p, const void* dY, int
 // Enough for either kernel, so the size does not depend on which one runs.
 size_t eqlinear_backward_weight_workspace_bytes(eqlinear_plan_t p, int64_t N) {
   if (!p || N < 0) return 0;
+  if (p->group == 1) return eql::d4_wgrad_workspace(N, p->C, p->D, p->num_sms);
   size_t need = eql::wgrad_simt_workspace(p->T, N, p->C, p->D, p->num_sms);
   const void* aligned = reinterpret_cast<const void*>(uintptr_t(256));
   if (wgrad_tc_ok(p, N, aligned, aligned))
@@ -700,7 +707,7 @@ static eqlinear_status_t backward_weight_impl(eqlinear_plan_t p, const void* X, 
                                               size_t workspace_bytes, eql::DType out_dt,
                                               void* stream, bool spectra = false) {
   if (!p || N < 0 || !dW) return EQL_ERR_INVALID_ARG;
-  if (p->group == 1) return EQL_ERR_UNSUPPORTED;
+  if (p->group == 1 && (spectra || p->kernel == EQL_KERNEL_TCGEN05)) return EQL_ERR_UNSUPPORTED;
   if (N > 0 && (!X || !dY)) return EQL_ERR_INVALID_ARG;
   if ((X && !aligned16(X)) || (dY && !aligned16(dY)) || !aligned16(dW) ||
       (dbias && !aligned16(dbias)) || (workspace && !aligned16(workspace)))
@@ -715,6 +722,9 @@ static eqlinear_status_t backward_weight_impl(eqlinear_plan_t p, const void* X, 
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
+  if (p->group == 1)  // D4: CUDA cores
+    return from_cuda(eql::launch_d4_wgrad(X, dY, N, p->C, p->D, out_dt, dW, dbias,
+                                          static_cast<float*>(workspace), p->num_sms, st));
   if (spectra && N > 0) {
     if (!eql::wgrad_tc_planes_supported(N, p->C, p->D, X, dY)) return EQL_ERR_UNSUPPORTED;
     return from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, workspace, out_dt, dW, dbias,

@@ -154,13 +154,22 @@ cudaError_t launch_pair_tf32(const void* Xt, int64_t N, int Cin, int Cout, const
 bool pair8_supported(int64_t N, int Cin, int Cout);
 size_t tiled8_planes_bytes(int64_t N, int channels);
 size_t pair8_tile_bytes(int Cin, int Cout);
+// d4_adjoint: the dX stages of a D4 layer from its forward planes [8][Cout][Cin]
 cudaError_t launch_pair8_tile_weights(const void* planes, int Cin, int Cout, void* tiles,
-                                      cudaStream_t st);
+                                      cudaStream_t st, int d4_adjoint = 0);
 cudaError_t launch_group_dft8_tiled(const void* X, int64_t N, int C, int group, void* out,
                                     cudaStream_t st);
 cudaError_t launch_pair8_tc(const void* Xt, int64_t N, int Cin, int Cout, const void* tiles,
                             const void* bias, void* Y, int* status, int num_sms, int act,
                             int group, cudaStream_t st);
+
+// Weight gradient of the D4 layer on CUDA cores (eql_d4_wgrad.cu): FP16 X [N][C*8]
+// and dY [N][D*8] -> dW [D][C][8] and dbias [D] in out_dt, through FP32
+// partials per row split (d4_wgrad_workspace bytes) summed in a fixed order.
+size_t d4_wgrad_workspace(int64_t N, int C, int D, int num_sms);
+cudaError_t launch_d4_wgrad(const void* X, const void* dY, int64_t N, int C, int D, DType out_dt,
+                            void* dW, void* dbias, float* workspace, int num_sms,
+                            cudaStream_t st);
 
 // dst[i] = src[i] rounded to nearest-even in dt (a copy for F32), i < n.
 cudaError_t launch_cast_from_f32(DType dt, const float* src, void* dst, int64_t n,

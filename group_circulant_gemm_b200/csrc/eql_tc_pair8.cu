@@ -353,13 +353,18 @@ __global__ void group_dft8_tiled_kernel(const uint4* __restrict__ X, int64_t N, 
   }
 }
 
-// Prepared planes [P][Cout][Cin] (the first eight in the kernel's plane order)
-// -> the eight-plane pair kernel's weight stages: blob (dt, ks, rank) = 8 planes
-// x 32 rows x 16 channels (32 bytes, 32-byte swizzle: 16-byte piece ^= (row / 4)
-// % 2); row r of a plane = out-channel dt*64 + 32*rank + r, channels 16ks ..;
-// zero past the matrix.  One thread per 16-byte piece.
+// Prepared planes -> the eight-plane pair kernel's weight stages: blob (dt, ks,
+// rank) = 8 planes x 32 rows x 16 channels (32 bytes, 32-byte swizzle: 16-byte
+// piece ^= (row / 4) % 2); row r of a plane = out-channel dt*64 + 32*rank + r,
+// channels 16ks ..; zero past the matrix.  One thread per 16-byte piece.
+// Normal: planes [P][Cout][Cin], the first eight in the kernel's plane order.
+// Adjoint of a D4 layer (dX = the D4 layer of dY with W'[c][d][v] = W[d][c][v^-1]):
+// its planes are the forward planes [8][Cin][Cout] read transposed, with the
+// 2 x 2 block's off-diagonal entries exchanged (v -> v^-1 maps rho(v) to
+// rho(v)^T and keeps every character).
 __global__ void pair8_tile_weights_kernel(const __half* __restrict__ planes, int Cin, int Cout,
-                                          int n_ks, int64_t n_pieces, uint4* __restrict__ tiles) {
+                                          int n_ks, int64_t n_pieces, int d4_adjoint,
+                                          uint4* __restrict__ tiles) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n_pieces) return;
   const int piece = (int)(idx & 1);
@@ -372,8 +377,17 @@ __global__ void pair8_tile_weights_kernel(const __half* __restrict__ planes, int
   const int d = dt * P8_BD + 32 * rank + r;
   const int c0 = ks * P8_KC + piece * 8;
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
-  if (d < Cout && c0 < Cin)
-    v = *reinterpret_cast<const uint4*>(planes + ((int64_t)plane * Cout + d) * Cin + c0);
+  if (d < Cout && c0 < Cin) {
+    if (!d4_adjoint) {
+      v = *reinterpret_cast<const uint4*>(planes + ((int64_t)plane * Cout + d) * Cin + c0);
+    } else {
+      const int src = plane == 5 ? 6 : (plane == 6 ? 5 : plane);
+      __half e[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) e[i] = planes[((int64_t)src * Cin + c0 + i) * Cout + d];
+      v = *reinterpret_cast<const uint4*>(e);
+    }
+  }
   const int64_t dst = blob * P8_WBYTES + plane * P8_WPL + r * P8_ROWB + ((piece ^ ((r >> 2) & 1)) << 4);
   tiles[dst >> 4] = v;
 }
@@ -417,11 +431,11 @@ size_t pair8_tile_bytes(int Cin, int Cout) {
 }
 
 cudaError_t launch_pair8_tile_weights(const void* planes, int Cin, int Cout, void* tiles,
-                                      cudaStream_t st) {
+                                      cudaStream_t st, int d4_adjoint) {
   if (Cin % 16 != 0 || Cout % 16 != 0) return cudaErrorInvalidValue;
   const int64_t n_pieces = (int64_t)pair8_tile_bytes(Cin, Cout) / 16;
   pair8_tile_weights_kernel<<<(unsigned)((n_pieces + 255) / 256), 256, 0, st>>>(
-      static_cast<const __half*>(planes), Cin, Cout, Cin / P8_KC, n_pieces,
+      static_cast<const __half*>(planes), Cin, Cout, Cin / P8_KC, n_pieces, d4_adjoint,
       static_cast<uint4*>(tiles));
   return cudaGetLastError();
 }

@@ -103,10 +103,19 @@ EQL_API eqlinear_status_t eqlinear_plan_create(int T, int C, int D, eqlinear_dty
  * 0, +-1, so the transforms are adds), and the per-frequency products are four
  * real GEMMs plus a 2 x 2 block product (eight), 12 real products per (row,
  * in-channel, out-channel) against the dense 64.
- * Supported: FP16, C and D multiples of 16, forward only (eqlinear_forward and
- * eqlinear_forward_act on the tensor cores); eqlinear_prepared_weight_bytes is
- * 0 and every other call returns EQL_ERR_UNSUPPORTED for other plans of this
- * kind.  W [D][C][8], X [N][C*8], Y [N][D*8].  Free with eqlinear_plan_destroy.
+ * Supported: FP16, C and D multiples of 16:
+ *   forward: eqlinear_forward and eqlinear_forward_act (fused one-CTA kernel), or
+ *     eqlinear_group_dft + eqlinear_forward_tiled (the Fourier planes as a pass,
+ *     then SM-pair tensor cores);
+ *   dX: eqlinear_group_dft of dY + eqlinear_backward_input_tiled (the D4 layer of
+ *     dY with W'[c][d][v] = W[d][c][v^-1]); eqlinear_backward_input returns
+ *     EQL_ERR_UNSUPPORTED;
+ *   dW and dbias: eqlinear_backward_weight(_f32) on CUDA cores (workspace from
+ *     eqlinear_backward_weight_workspace_bytes; EQL_ERR_UNSUPPORTED when the plan
+ *     is forced to the tensor cores).
+ * For other plans of this kind eqlinear_prepared_weight_bytes is 0 and every
+ * call returns EQL_ERR_UNSUPPORTED.  W [D][C][8], X [N][C*8], Y [N][D*8].  Free
+ * with eqlinear_plan_destroy.
  */
 EQL_API eqlinear_status_t eqlinear_plan_create_dihedral4(int C, int D, eqlinear_dtype_t dtype,
                                                         eqlinear_plan_t* out);
@@ -250,10 +259,25 @@ EQL_API eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t plan, c
  *   (padding rows N..Np-1 hold values of no meaning).
  * eqlinear_backward_input_tiled: tiled planes of dY [N][D*4] -> dX [N][C*4].
  * Each equals eqlinear_forward_act / eqlinear_backward_input up to the rounding
- * of the planes.  FP16 plans with T = 4 and C, D multiples of 16, not forced to
- * the CUDA cores (else EQL_ERR_UNSUPPORTED); channels not C or D:
- * EQL_ERR_INVALID_ARG; all pointers 16-byte aligned; outputs must not overlap
- * inputs; N = 0 is a no-op.
+ * of the planes.  Plans taken (else EQL_ERR_UNSUPPORTED; never a plan forced to
+ * the CUDA cores):
+ *   - p4 FP16, C and D multiples of 16: as above.
+ *   - FP16 with T = 8, cyclic or D4 (eqlinear_plan_create_dihedral4), C and D
+ *     multiples of 16. Eight planes, each times 1/8: cyclic V0, V4, Re/Im of
+ *     V1, V2, V3 of the DFT; D4 the four characters (chi(r), chi(m)) = (+,+),
+ *     (+,-), (-,+), (-,-), then the 2 x 2 representation's entries
+ *     X[i][j] = sum_g x_g rho(g)_ij at plane 4 + 2i + j, with rho(r) =
+ *     [[0,-1],[1,0]] and rho(m) = diag(1,-1). The same tiled layout with p < 8;
+ *     tiled_spectrum_bytes = 8 * Np * c * 2. No _next form.
+ *   - p4 FP32, C and D multiples of 8 (3xTF32 on the tensor cores). Eight
+ *     planes: the TF32 values hi = tf32(v) of X0, X2, Xr, Xi, then the
+ *     residuals lo = tf32(v - hi). 8 FP32 channels per 32-byte row: element
+ *     (q, n, j) at ((q * (c / 8) + j / 8) * Np + n) * 32 +
+ *     16 * (((j % 8) / 4) ^ ((n / 4) % 2)) + 4 * (j % 4);
+ *     tiled_spectrum_bytes = 8 * Np * c * 4. No _next form. The result is within
+ *     the FP32 bar (products hi*hi + lo*hi + hi*lo, FP32 accumulation).
+ * Channels not C or D: EQL_ERR_INVALID_ARG. All pointers must be 16-byte
+ * aligned, and outputs must not overlap inputs. N = 0 is a no-op.
  */
 EQL_API size_t eqlinear_tiled_spectrum_bytes(eqlinear_plan_t plan, int64_t N, int channels);
 EQL_API eqlinear_status_t eqlinear_group_dft(eqlinear_plan_t plan, const void* X, int64_t N,

@@ -100,9 +100,10 @@ def test_d4_unsupported_paths():
     X = torch.zeros(4, 16 * 8, dtype=torch.float16, device="cuda")
     Wh = p.prepare_weights(torch.zeros(16, 16, 8, dtype=torch.float16, device="cuda"))
     dX = torch.empty_like(X)
+    # dX runs through the tiled entries (eqlinear_backward_input_tiled); dW on CUDA cores
     assert native.raw_status("eqlinear_backward_input", p.handle, X.data_ptr(), 4, Wh.data_ptr(),
                              dX.data_ptr(), None) == native.EQL_ERR_UNSUPPORTED
-    assert p.backward_weight_kernel_name(4) == "unsupported"
+    assert p.backward_weight_kernel_name(4) == "simt"
     f32 = _plan(16, 16, torch.float32)
     assert native.eqlinear_prepared_weight_bytes(f32.handle) == 0
     p.set_kernel("simt")

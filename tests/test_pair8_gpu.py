@@ -17,7 +17,8 @@ max|ref|):
   * the T = 8 workload (16384 x 128 -> 128) and the D4 ViT-B MLP layers at full
     size, on sampled rows;
   * agreement with the fused one-CTA kernels;
-  * requests the path does not take are rejected.
+  * requests the path does not take are rejected (D4 dX in this form is checked
+    in test_d4_backward_gpu.py).
 """
 import numpy as np
 import pytest
@@ -148,9 +149,12 @@ def test_eight_plane_tiled_rejects_what_it_does_not_take():
     Xt = torch.zeros(p.tiled_shape(4, 16), dtype=torch.float16, device="cuda")
     X = torch.zeros(4, 128, dtype=torch.float16, device="cuda")
     assert n.eqlinear_tiled_spectrum_bytes(p.handle, 4, 16) == 8 * 128 * 16 * 2
-    # D4 plans hold no adjoint stages: no dX in this form
-    assert n.raw_status("eqlinear_backward_input_tiled", p.handle, Xt.data_ptr(), 4,
-                        Wh.data_ptr(), X.data_ptr(), None) == n.EQL_ERR_UNSUPPORTED
+    # no next-layer planes for D4 either
+    assert n.raw_status("eqlinear_forward_tiled_next", p.handle, Xt.data_ptr(), 4,
+                        Wh.data_ptr(), None, 0, Xt.data_ptr(), None) == n.EQL_ERR_UNSUPPORTED
+    # channels that are not the plan's C or D
+    assert n.raw_status("eqlinear_group_dft", p.handle, X.data_ptr(), 4, 32, Xt.data_ptr(),
+                        None) == n.EQL_ERR_INVALID_ARG
     # the next layer's planes: p4 only
     c = _plan(16, 16)
     Wc = c.prepare_weights(torch.zeros(16, 16, 8, dtype=torch.float16, device="cuda"))
