@@ -96,6 +96,13 @@ def _load():
             lib.eqlo_d4_backward_input.restype = i64
             lib.eqlo_d4_backward_weight.argtypes = [i64, i64, i64, dp, dp, dp, dp]
             lib.eqlo_d4_backward_weight.restype = i64
+            ci = ctypes.c_int
+            lib.eqlo_conv_backward_input.argtypes = [ci, i64, i64, i64, i64, i64, ci, ci, ci, ci,
+                                                     dp, dp, dp]
+            lib.eqlo_conv_backward_input.restype = None
+            lib.eqlo_conv_backward_weight.argtypes = [ci, i64, i64, i64, i64, i64, ci, ci, ci,
+                                                      ci, dp, dp, dp, dp]
+            lib.eqlo_conv_backward_weight.restype = None
             lib.eqlo_set_threads.argtypes = [ctypes.c_int]
             lib.eqlo_set_threads.restype = None
             _lib = lib
@@ -280,6 +287,39 @@ def conv_forward(T: int, X, Wc, bias=None, pad=(0, 0), return_macs: bool = False
 
 _threads_override = None
 
+
+
+def conv_backward_input(T: int, dY, Wc, H: int, W: int, pad=(0, 0)):
+    """dX[N, H, W, C*T] in float64 from dY[N, Ho, Wo, D*T] and Wc[KH, KW, D, C, T]:
+    the gradient of conv_forward with respect to X (input size H x W)."""
+    dY, Wc = _f64(dY), _f64(Wc)
+    KH, KW, D, C, TW = Wc.shape
+    N, Ho, Wo = dY.shape[:3]
+    ph, pw = pad
+    if TW != T or dY.shape[3] != D * T or Ho != H + 2 * ph - KH + 1 or Wo != W + 2 * pw - KW + 1:
+        raise ValueError("shape mismatch")
+    dX = np.empty((N, H, W, C * T), dtype=np.float64)
+    _load().eqlo_conv_backward_input(T, N, H, W, C, D, KH, KW, ph, pw, _ptr(dY), _ptr(Wc),
+                                     _ptr(dX))
+    return dX
+
+
+def conv_backward_weight(T: int, X, dY, KH: int, KW: int, pad=(0, 0)):
+    """(dWc[KH, KW, D, C, T], dbias[D]) in float64 from X[N, H, W, C*T] and
+    dY[N, Ho, Wo, D*T]: the gradients of conv_forward."""
+    X, dY = _f64(X), _f64(dY)
+    N, H, W = X.shape[:3]
+    C = X.shape[3] // T
+    ph, pw = pad
+    Ho, Wo = H + 2 * ph - KH + 1, W + 2 * pw - KW + 1
+    D = dY.shape[3] // T
+    if dY.shape != (N, Ho, Wo, D * T) or X.shape[3] != C * T:
+        raise ValueError("shape mismatch")
+    dWc = np.empty((KH, KW, D, C, T), dtype=np.float64)
+    db = np.empty((D,), dtype=np.float64)
+    _load().eqlo_conv_backward_weight(T, N, H, W, C, D, KH, KW, ph, pw, _ptr(X), _ptr(dY),
+                                      _ptr(dWc), _ptr(db))
+    return dWc, db
 
 def set_threads(n: int | None) -> None:
     """Run the parallel loops on n threads (None: back to the default count).

@@ -309,6 +309,86 @@ int64_t eqlo_conv_forward(int T, int64_t N, int64_t H, int64_t Wd, int64_t C, in
 }
 
 /*
+ * Gradients of the group-circulant convolution (the definition above,
+ * differentiated term by term; taps outside the image contribute nothing):
+ *   dX[n][y][x][c*T+t] = sum_{i,j,d,s} Wc[i][j][d][c][(t-s) mod T]
+ *                                      * dY[n][y-i+ph][x-j+pw][d*T+s]
+ *   dWc[i][j][d][c][u] = sum_{n,oy,ox,s} dY[n][oy][ox][d*T+s]
+ *                                       * X[n][oy+i-ph][ox+j-pw][c*T + (s+u) mod T]
+ *   dbias[d]           = sum_{n,oy,ox,s} dY[n][oy][ox][d*T+s]
+ * dY is [N][Ho][Wo][D*T] with Ho = H + 2 ph - KH + 1, Wo = Wd + 2 pw - KW + 1.
+ */
+void eqlo_conv_backward_input(int T, int64_t N, int64_t H, int64_t Wd, int64_t C, int64_t D,
+                              int KH, int KW, int ph, int pw, const double* dY, const double* Wc,
+                              double* dX) {
+  const int64_t Ho = H + 2 * ph - KH + 1, Wo = Wd + 2 * pw - KW + 1;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t y = 0; y < H; ++y) {
+      for (int64_t x = 0; x < Wd; ++x) {
+        double* dx = dX + ((n * H + y) * Wd + x) * C * T;
+        for (int64_t c = 0; c < C; ++c) {
+          for (int t = 0; t < T; ++t) {
+            double acc = 0.0;
+            for (int i = 0; i < KH; ++i) {
+              const int64_t oy = y - i + ph;
+              if (oy < 0 || oy >= Ho) continue;
+              for (int j = 0; j < KW; ++j) {
+                const int64_t ox = x - j + pw;
+                if (ox < 0 || ox >= Wo) continue;
+                const double* dy = dY + ((n * Ho + oy) * Wo + ox) * D * T;
+                for (int64_t d = 0; d < D; ++d) {
+                  const double* w = Wc + (((int64_t)i * KW + j) * D + d) * C * T + c * T;
+                  for (int s = 0; s < T; ++s) acc += w[wrap(t - s, T)] * dy[d * T + s];
+                }
+              }
+            }
+            dx[c * T + t] = acc;
+          }
+        }
+      }
+    }
+  }
+}
+
+void eqlo_conv_backward_weight(int T, int64_t N, int64_t H, int64_t Wd, int64_t C, int64_t D,
+                               int KH, int KW, int ph, int pw, const double* X, const double* dY,
+                               double* dWc, double* dbias) {
+  const int64_t Ho = H + 2 * ph - KH + 1, Wo = Wd + 2 * pw - KW + 1;
+#pragma omp parallel for collapse(3) schedule(static)
+  for (int i = 0; i < KH; ++i) {
+    for (int j = 0; j < KW; ++j) {
+      for (int64_t d = 0; d < D; ++d) {
+        for (int64_t c = 0; c < C; ++c) {
+          for (int u = 0; u < T; ++u) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+              for (int64_t oy = 0; oy < Ho; ++oy) {
+                const int64_t iy = oy + i - ph;
+                if (iy < 0 || iy >= H) continue;
+                for (int64_t ox = 0; ox < Wo; ++ox) {
+                  const int64_t ix = ox + j - pw;
+                  if (ix < 0 || ix >= Wd) continue;
+                  const double* dy = dY + ((n * Ho + oy) * Wo + ox) * D * T + d * T;
+                  const double* x = X + ((n * H + iy) * Wd + ix) * C * T + c * T;
+                  for (int s = 0; s < T; ++s) acc += dy[s] * x[wrap(s + u, T)];
+                }
+              }
+            dWc[((((int64_t)i * KW + j) * D + d) * C + c) * T + u] = acc;
+          }
+        }
+      }
+    }
+  }
+  for (int64_t d = 0; d < D; ++d) {
+    double acc = 0.0;
+    for (int64_t q = 0; q < N * Ho * Wo; ++q)
+      for (int s = 0; s < T; ++s) acc += dY[q * D * T + d * T + s];
+    dbias[d] = acc;
+  }
+}
+
+/*
  * EQ-Linear over the dihedral group D4 (p4m: the four 90-degree rotations and
  * their compositions with a mirror), the reflection group the pages name as the
  * natural generalisation of the p4 method ("Limitations and future work"; no

@@ -128,3 +128,30 @@ def test_conv_pins_catch_a_planted_direction_mistake(oracle_mod):
     wrong = oracle_mod.conv_forward(T, X, Wc[..., (-np.arange(T)) % T], None, pad=(1, 1))
     assert _rel(wrong, ref) > 1e-3
     assert _rel(oracle_mod.conv_forward(T, X, Wc, None, pad=(1, 1)), ref) < 1e-13
+
+
+@pytest.mark.parametrize("T,N,H,W,C,D,KH,KW,ph,pw", CASES)
+def test_conv_gradients_match_autograd_of_torch_conv2d(oracle_mod, T, N, H, W, C, D, KH, KW,
+                                                       ph, pw):
+    """dX, dWc and dbias against torch autograd (float64) of conv2d on the
+    replicated dense kernel, whose entries are gathered from Wc by rolling the
+    parameter vectors (a differentiable function of Wc)."""
+    X = _rand(11, N, H, W, C * T)
+    Wc = _rand(12, KH, KW, D, C, T)
+    b = _rand(13, D)
+    Ho, Wo = H + 2 * ph - KH + 1, W + 2 * pw - KW + 1
+    dY = _rand(14, N, Ho, Wo, D * T)
+    Xt = torch.tensor(X, requires_grad=True)
+    Wt = torch.tensor(Wc, requires_grad=True)
+    bt = torch.tensor(b, requires_grad=True)
+    # dense kernel [D*T, C*T, KH, KW]: entry ((d,s),(c,t)) = Wc[.., d, c, (t - s) mod T]
+    idx = torch.tensor([[(t - s) % T for t in range(T)] for s in range(T)])  # [s, t]
+    K = Wt[:, :, :, :, idx]                               # [KH, KW, D, C, s, t]
+    K = K.permute(2, 4, 3, 5, 0, 1).reshape(D * T, C * T, KH, KW)
+    Y = F.conv2d(Xt.permute(0, 3, 1, 2), K, bt.repeat_interleave(T), padding=(ph, pw))
+    Y.permute(0, 2, 3, 1).backward(torch.tensor(dY))
+    dX = oracle_mod.conv_backward_input(T, dY, Wc, H, W, pad=(ph, pw))
+    assert _rel(dX, Xt.grad.numpy()) < 1e-12
+    dW, db = oracle_mod.conv_backward_weight(T, X, dY, KH, KW, pad=(ph, pw))
+    assert _rel(dW, Wt.grad.numpy()) < 1e-12
+    assert _rel(db, bt.grad.numpy()) < 1e-12
