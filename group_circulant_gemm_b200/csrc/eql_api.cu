@@ -556,6 +556,11 @@ eqlinear_status_t eqlinear_forward_chain(eqlinear_plan_t first, eqlinear_plan_t 
 
 // ---- group-circulant convolution ----------------------------------------------
 
+static eqlinear_status_t backward_weight_impl(eqlinear_plan_t p, const void* X, const void* dY,
+                                              int64_t N, void* dW, void* dbias, void* workspace,
+                                              size_t workspace_bytes, eql::DType out_dt,
+                                              void* stream, bool spectra);
+
 static bool conv_plan_ok(eqlinear_plan_t p) {
   return p && p->T == 4 && p->dtype == EQL_F16 && p->kernel != EQL_KERNEL_SIMT && has_tiles(p);
 }
@@ -563,12 +568,19 @@ static size_t conv_tap_tiles(eqlinear_plan_t p) { return eql::tc_tile_bytes(4, p
 static size_t conv_tap_planes(eqlinear_plan_t p) {
   return (size_t)eql::spec_planes(4) * plane_elems(p) * elem_size(p->dtype);
 }
+static size_t conv_tap_adj_tiles(eqlinear_plan_t p) { return eql::tc_tile_bytes(4, p->D, p->C); }
+// Wc_hat: [taps x forward tiles][taps x (forward planes, adjoint planes)][taps x adjoint tiles]
+static const char* conv_adj_tiles(eqlinear_plan_t p, int taps, const void* Wc_hat) {
+  return static_cast<const char*>(Wc_hat) +
+         (size_t)taps * (conv_tap_tiles(p) + 2 * conv_tap_planes(p));
+}
 
 size_t eqlinear_conv_prepared_weight_bytes(eqlinear_plan_t p, int KH, int KW) {
   if (!conv_plan_ok(p) || KH < 1 || KW < 1 || KH > 15 || KW > 15) return 0;
-  // per tap: operand tiles (read by the kernel, all taps first) and the forward
-  // and adjoint planes they are made from
-  return (size_t)KH * KW * (conv_tap_tiles(p) + 2 * conv_tap_planes(p));
+  // per tap: operand tiles (read by the kernel, all taps first), the forward
+  // and adjoint planes they are made from, then the adjoint tiles of the flipped
+  // taps (dX)
+  return (size_t)KH * KW * (conv_tap_tiles(p) + 2 * conv_tap_planes(p) + conv_tap_adj_tiles(p));
 }
 
 eqlinear_status_t eqlinear_conv_prepare_weights(eqlinear_plan_t p, int KH, int KW,
@@ -593,6 +605,103 @@ eqlinear_status_t eqlinear_conv_prepare_weights(eqlinear_plan_t p, int KH, int K
     if (s != EQL_OK) return s;
     s = from_cuda(eql::launch_tile_weights(4, fwd, p->C, p->D,
                                            tiles + (size_t)tap * conv_tap_tiles(p), st));
+    if (s != EQL_OK) return s;
+  }
+  // dX is the convolution of dY with the flipped kernel of adjoint taps: tap (i, j)
+  // of it holds the adjoint tiles of tap (KH-1-i, KW-1-j)
+  char* adj_tiles = const_cast<char*>(conv_adj_tiles(p, taps, Wc_hat));
+  for (int tap = 0; tap < taps; ++tap) {
+    const int src = (KH - 1 - tap / KW) * KW + (KW - 1 - tap % KW);
+    const char* adj = planes + (size_t)src * 2 * conv_tap_planes(p) + conv_tap_planes(p);
+    s = from_cuda(eql::launch_tile_weights(4, adj, p->D, p->C,
+                                           adj_tiles + (size_t)tap * conv_tap_adj_tiles(p), st));
+    if (s != EQL_OK) return s;
+  }
+  return EQL_OK;
+}
+
+size_t eqlinear_conv_backward_workspace_bytes(eqlinear_plan_t p, int64_t N, int H, int W, int KH,
+                                              int KW, int pad_h, int pad_w) {
+  if (!conv_plan_ok(p) || N < 0 || H < 1 || W < 1 || KH < 1 || KW < 1 || pad_h < 0 || pad_w < 0)
+    return 0;
+  const int64_t Ho = (int64_t)H + 2 * pad_h - KH + 1, Wo = (int64_t)W + 2 * pad_w - KW + 1;
+  if (Ho < 1 || Wo < 1) return 0;
+  const int64_t rows = N * Ho * Wo;
+  // dX: the group DFT planes of dY; dW: one tap's shifted rows of X, then the
+  // layer weight gradient's scratch for N*Ho*Wo rows
+  const size_t dx = eql::conv_tc_planes_bytes(N, (int)Ho, (int)Wo, p->D);
+  const size_t shifted = ((size_t)rows * p->C * 4 * elem_size(p->dtype) + 255) / 256 * 256;
+  const size_t dw = shifted + eqlinear_backward_weight_workspace_bytes(p, rows);
+  return std::max<size_t>(std::max(dx, dw), 16);
+}
+
+eqlinear_status_t eqlinear_conv_backward_input(eqlinear_plan_t p, const void* dY, int64_t N, int H,
+                                               int W, int KH, int KW, int pad_h, int pad_w,
+                                               const void* Wc_hat, void* dX, void* workspace,
+                                               size_t workspace_bytes, void* stream) {
+  EQL_TRACE();
+  if (!p || N < 0 || H < 1 || W < 1 || KH < 1 || KW < 1 || pad_h < 0 || pad_w < 0)
+    return EQL_ERR_INVALID_ARG;
+  if (!conv_plan_ok(p)) return EQL_ERR_UNSUPPORTED;
+  const int64_t Ho = (int64_t)H + 2 * pad_h - KH + 1, Wo = (int64_t)W + 2 * pad_w - KW + 1;
+  if (Ho < 1 || Wo < 1) return EQL_ERR_INVALID_ARG;
+  if (N == 0) return EQL_OK;
+  const int qh = KH - 1 - pad_h, qw = KW - 1 - pad_w;
+  if (qh < 0 || qw < 0 ||
+      !eql::conv_tc_supported(4, to_dt(p->dtype), N, (int)Ho, (int)Wo, p->D, p->C, KH, KW, qh, qw))
+    return EQL_ERR_UNSUPPORTED;
+  if (!dY || !Wc_hat || !dX) return EQL_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(Wc_hat) || !aligned16(dX) || (workspace && !aligned16(workspace)))
+    return EQL_ERR_ALIGNMENT;
+  if (!workspace ||
+      workspace_bytes < eqlinear_conv_backward_workspace_bytes(p, N, H, W, KH, KW, pad_h, pad_w))
+    return EQL_ERR_WORKSPACE;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  return from_cuda(eql::launch_conv_tc(dY, N, (int)Ho, (int)Wo, p->D, p->C, KH, KW, qh, qw,
+                                       conv_adj_tiles(p, KH * KW, Wc_hat), nullptr, dX, workspace,
+                                       p->status, p->num_sms, 0, (cudaStream_t)stream));
+}
+
+eqlinear_status_t eqlinear_conv_backward_weight(eqlinear_plan_t p, const void* X, int64_t N, int H,
+                                                int W, const void* dY, int KH, int KW, int pad_h,
+                                                int pad_w, void* dWc, void* dbias, void* workspace,
+                                                size_t workspace_bytes, void* stream) {
+  EQL_TRACE();
+  if (!p || N < 0 || H < 1 || W < 1 || KH < 1 || KW < 1 || pad_h < 0 || pad_w < 0)
+    return EQL_ERR_INVALID_ARG;
+  if (!conv_plan_ok(p)) return EQL_ERR_UNSUPPORTED;
+  const int64_t Ho = (int64_t)H + 2 * pad_h - KH + 1, Wo = (int64_t)W + 2 * pad_w - KW + 1;
+  if (Ho < 1 || Wo < 1) return EQL_ERR_INVALID_ARG;
+  if (!dWc) return EQL_ERR_INVALID_ARG;
+  if (N > 0 && (!X || !dY)) return EQL_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || (dY && !aligned16(dY)) || !aligned16(dWc) ||
+      (dbias && !aligned16(dbias)) || (workspace && !aligned16(workspace)))
+    return EQL_ERR_ALIGNMENT;
+  if (!workspace ||
+      workspace_bytes < eqlinear_conv_backward_workspace_bytes(p, N, H, W, KH, KW, pad_h, pad_w))
+    return EQL_ERR_WORKSPACE;
+  eqlinear_status_t s = check_plan_device(p);
+  if (s != EQL_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t rows = N * Ho * Wo;
+  const size_t shifted = ((size_t)rows * p->C * 4 * elem_size(p->dtype) + 255) / 256 * 256;
+  char* xs = static_cast<char*>(workspace);
+  char* ws = xs + shifted;
+  const size_t ws_bytes = workspace_bytes - shifted;
+  const size_t w_tap = (size_t)p->D * p->C * 4 * elem_size(p->dtype);
+  for (int tap = 0; tap < KH * KW; ++tap) {
+    if (N > 0) {
+      s = from_cuda(eql::launch_conv_shift_rows(X, N, H, W, p->C * 4, tap / KW, tap % KW, pad_h,
+                                                pad_w, (int)Ho, (int)Wo, xs, st));
+      if (s != EQL_OK) return s;
+    }
+    // the layer's weight gradient over the tap's rows; dbias (the same for every
+    // tap) with the first tap only
+    s = backward_weight_impl(p, N > 0 ? xs : nullptr, dY, rows,
+                             static_cast<char*>(dWc) + (size_t)tap * w_tap,
+                             tap == 0 ? dbias : nullptr, ws, ws_bytes, to_dt(p->dtype), stream,
+                             false);
     if (s != EQL_OK) return s;
   }
   return EQL_OK;

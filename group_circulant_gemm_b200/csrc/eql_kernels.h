@@ -163,6 +163,11 @@ cudaError_t launch_pair8_tc(const void* Xt, int64_t N, int Cin, int Cout, const 
                             const void* bias, void* Y, int* status, int num_sms, int act,
                             int group, cudaStream_t st);
 
+// Rows of X [N][H][W][c4 halves] shifted by a convolution tap: out[(n*Ho + oy)*Wo + ox]
+// = X[n][oy+i-ph][ox+j-pw] (zero outside the image), c4 a multiple of 8.
+cudaError_t launch_conv_shift_rows(const void* X, int64_t N, int H, int W, int c4, int i, int j,
+                                   int ph, int pw, int Ho, int Wo, void* out, cudaStream_t st);
+
 // Weight gradient of the D4 layer on CUDA cores (eql_d4_wgrad.cu): FP16 X [N][C*8]
 // and dY [N][D*8] -> dW [D][C][8] and dbias [D] in out_dt, through FP32
 // partials per row split (d4_wgrad_workspace bytes) summed in a fixed order.

@@ -385,4 +385,35 @@ cudaError_t launch_conv_tc(const void* X, int64_t N, int H, int W, int C, int D,
   return cudaGetLastError();
 }
 
+namespace {
+// Tap-shifted rows of a pixel tensor (the convolution's weight gradient runs the
+// layer's weight-gradient kernel per tap on these rows): one thread per 16 bytes.
+__global__ void conv_shift_rows_kernel(const uint4* __restrict__ X, int64_t N, int H, int W,
+                                       int c16, int i, int j, int ph, int pw, int Ho, int Wo,
+                                       uint4* __restrict__ out) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = N * Ho * Wo * c16;
+  if (idx >= total) return;
+  const int64_t q = idx / c16;
+  const int k = (int)(idx % c16);
+  const int ox = (int)(q % Wo), oy = (int)((q / Wo) % Ho);
+  const int64_t n = q / ((int64_t)Wo * Ho);
+  const int iy = oy + i - ph, ix = ox + j - pw;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (iy >= 0 && iy < H && ix >= 0 && ix < W) v = X[((n * H + iy) * W + ix) * c16 + k];
+  out[idx] = v;
+}
+}  // namespace
+
+cudaError_t launch_conv_shift_rows(const void* X, int64_t N, int H, int W, int c4, int i, int j,
+                                   int ph, int pw, int Ho, int Wo, void* out, cudaStream_t st) {
+  if (c4 % 8 != 0) return cudaErrorInvalidValue;
+  const int64_t total = N * Ho * Wo * (c4 / 8);
+  if (total == 0) return cudaSuccess;
+  conv_shift_rows_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint4*>(X), N, H, W, c4 / 8, i, j, ph, pw, Ho, Wo,
+      static_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
 }  // namespace eql

@@ -297,6 +297,42 @@ class EqLinearPlan:
                                  workspace.numel() * workspace.element_size())
         return out
 
+    def _conv_bwd_workspace(self, N, H, W, KH, KW, ph, pw, workspace, device):
+        nb = _n.eqlinear_conv_backward_workspace_bytes(self.handle, N, H, W, KH, KW, ph, pw)
+        if nb == 0:
+            raise ValueError("no convolution backward for this plan and shape")
+        if workspace is None:
+            workspace = torch.empty(nb, dtype=torch.uint8, device=device)
+        return workspace
+
+    def conv_backward_input(self, dY, Wc_hat, KH: int, KW: int, H: int, W: int, pad=(0, 0),
+                            out=None, workspace=None) -> torch.Tensor:
+        """dY [N, Ho, Wo, D*T] -> dX [N, H, W, C*T] (the flipped kernel of adjoint taps)."""
+        N = int(dY.shape[0])
+        ph, pw = pad
+        Ho, Wo = H + 2 * ph - KH + 1, W + 2 * pw - KW + 1
+        self._check(dY, (N, Ho, Wo, self.D * self.T), "dY")
+        if out is None:
+            out = torch.empty((N, H, W, self.C * self.T), dtype=self.dtype, device=dY.device)
+        workspace = self._conv_bwd_workspace(N, H, W, KH, KW, ph, pw, workspace, dY.device)
+        _n.eqlinear_conv_backward_input(self.handle, dY, N, H, W, KH, KW, ph, pw, Wc_hat, out,
+                                        workspace, workspace.numel() * workspace.element_size())
+        return out
+
+    def conv_backward_weight(self, X, dY, KH: int, KW: int, pad=(0, 0), workspace=None):
+        """X [N, H, W, C*T], dY [N, Ho, Wo, D*T] -> (dWc [KH, KW, D, C, T], dbias [D])."""
+        N, H, W = (int(v) for v in X.shape[:3])
+        self._check(X, (N, H, W, self.C * self.T), "X")
+        ph, pw = pad
+        Ho, Wo = H + 2 * ph - KH + 1, W + 2 * pw - KW + 1
+        self._check(dY, (N, Ho, Wo, self.D * self.T), "dY")
+        dW = torch.empty((KH, KW, self.D, self.C, self.T), dtype=self.dtype, device=X.device)
+        db = torch.empty(self.D, dtype=self.dtype, device=X.device)
+        workspace = self._conv_bwd_workspace(N, H, W, KH, KW, ph, pw, workspace, X.device)
+        _n.eqlinear_conv_backward_weight(self.handle, X, N, H, W, dY, KH, KW, ph, pw, dW, db,
+                                         workspace, workspace.numel() * workspace.element_size())
+        return dW, db
+
     # --- data-parallel weight gradient: FP32 per-rank sums, one reduction, one cast
 
     def grad_offset(self) -> int:

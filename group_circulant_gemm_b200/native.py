@@ -33,6 +33,8 @@ EXPORTED = (
     "eqlinear_chain_workspace_bytes", "eqlinear_forward_chain",
     "eqlinear_conv_prepared_weight_bytes", "eqlinear_conv_prepare_weights",
     "eqlinear_conv_workspace_bytes", "eqlinear_conv_forward",
+    "eqlinear_conv_backward_workspace_bytes", "eqlinear_conv_backward_input",
+    "eqlinear_conv_backward_weight",
     "eqlinear_plan_create_dihedral4",
     "eqlinear_forward_save_spectrum", "eqlinear_backward_input_save_spectrum",
     "eqlinear_backward_weight_from_spectra", "eqlinear_backward_weight_from_spectra_f32",
@@ -97,6 +99,11 @@ def _load() -> ctypes.CDLL:
         "eqlinear_conv_workspace_bytes": ([vp, i64, i32, i32], sz),
         "eqlinear_conv_forward": ([vp, vp, i64, i32, i32, i32, i32, i32, i32, vp, vp, i32, vp,
                                    vp, sz, vp], i32),
+        "eqlinear_conv_backward_workspace_bytes": ([vp, i64, i32, i32, i32, i32, i32, i32], sz),
+        "eqlinear_conv_backward_input": ([vp, vp, i64, i32, i32, i32, i32, i32, i32, vp, vp,
+                                          vp, sz, vp], i32),
+        "eqlinear_conv_backward_weight": ([vp, vp, i64, i32, i32, vp, i32, i32, i32, i32, vp,
+                                           vp, vp, sz, vp], i32),
         "eqlinear_forward_chain": ([vp, vp, vp, i64, vp, vp, i32, vp, vp, i32, vp, vp, vp, sz,
                                     vp], i32),
     }
@@ -347,6 +354,29 @@ def eqlinear_conv_forward(plan: int, X, N: int, H: int, W: int, KH: int, KW: int
                                       _ptr(Wc_hat), _ptr(bias), act, _ptr(Y), _ptr(workspace),
                                       workspace_bytes, _stream(stream)),
            "eqlinear_conv_forward")
+
+
+def eqlinear_conv_backward_workspace_bytes(plan: int, N: int, H: int, W: int, KH: int, KW: int,
+                                           pad_h: int, pad_w: int) -> int:
+    return _lib.eqlinear_conv_backward_workspace_bytes(plan, N, H, W, KH, KW, pad_h, pad_w)
+
+
+def eqlinear_conv_backward_input(plan: int, dY, N: int, H: int, W: int, KH: int, KW: int,
+                                 pad_h: int, pad_w: int, Wc_hat, dX, workspace,
+                                 workspace_bytes: int, stream=None) -> None:
+    _check(_lib.eqlinear_conv_backward_input(plan, _ptr(dY), N, H, W, KH, KW, pad_h, pad_w,
+                                             _ptr(Wc_hat), _ptr(dX), _ptr(workspace),
+                                             workspace_bytes, _stream(stream)),
+           "eqlinear_conv_backward_input")
+
+
+def eqlinear_conv_backward_weight(plan: int, X, N: int, H: int, W: int, dY, KH: int, KW: int,
+                                  pad_h: int, pad_w: int, dWc, dbias, workspace,
+                                  workspace_bytes: int, stream=None) -> None:
+    _check(_lib.eqlinear_conv_backward_weight(plan, _ptr(X), N, H, W, _ptr(dY), KH, KW, pad_h,
+                                              pad_w, _ptr(dWc), _ptr(dbias), _ptr(workspace),
+                                              workspace_bytes, _stream(stream)),
+           "eqlinear_conv_backward_weight")
 
 
 def eqlinear_backward_weight_noalloc(plan: int, X, dY, N: int, dW, dbias, stream=None) -> None:

@@ -374,7 +374,9 @@ EQL_API eqlinear_status_t eqlinear_forward_chain(eqlinear_plan_t first, eqlinear
  * (otherwise EQL_ERR_UNSUPPORTED).  KH, KW in 1..15, 0 <= pad < kernel size.
  *   eqlinear_conv_prepared_weight_bytes(plan, KH, KW): size of Wc_hat.
  *   eqlinear_conv_prepare_weights: Wc [KH][KW][D][C][T] (tap-major; each tap a
- *     contiguous [D][C][T] block) -> Wc_hat, once per weight update.
+ *     contiguous [D][C][T] block) -> Wc_hat, once per weight update (forward
+ *     tiles, each tap's planes, then the adjoint tiles of the flipped taps that
+ *     eqlinear_conv_backward_input reads).
  *   eqlinear_conv_workspace_bytes(plan, N, H, W): scratch of eqlinear_conv_forward
  *     (the group DFT of X times 1/4 as FP16 planes, 4 * N * H * W * C * 2 bytes).
  *   eqlinear_conv_forward: X [N][H][W][C*T] (feature index c*T+t, pixels
@@ -394,6 +396,43 @@ EQL_API eqlinear_status_t eqlinear_conv_forward(eqlinear_plan_t plan, const void
                                                 int pad_w, const void* Wc_hat, const void* bias,
                                                 eqlinear_act_t act, void* Y, void* workspace,
                                                 size_t workspace_bytes, void* stream);
+
+/*
+ * Gradients of the group-circulant convolution (the definition above,
+ * differentiated; "Implementation": forward and backward passes):
+ *   dX[n][y][x][c*T+t] = sum_{i,j,d,s} Wc[i][j][d][c][(t-s) mod T]
+ *                                      * dY[n][y-i+pad_h][x-j+pad_w][d*T+s]
+ *   dWc[i][j][d][c][u] = sum_{n,oy,ox,s} dY[n][oy][ox][d*T+s]
+ *                                       * X[n][oy+i-pad_h][ox+j-pad_w][c*T + (s+u) mod T]
+ *   dbias[d]           = sum_{n,oy,ox,s} dY[n][oy][ox][d*T+s]
+ * (terms whose pixel falls outside the image are zero).  dY [N][Ho][Wo][D*T].
+ *   eqlinear_conv_backward_input: dX [N][H][W][C*T] is the convolution of dY with
+ *     the spatially flipped kernel of adjoint taps and padding (KH-1-pad_h,
+ *     KW-1-pad_w); it runs the forward's tensor-core kernel with the adjoint
+ *     tiles that eqlinear_conv_prepare_weights also writes into Wc_hat.
+ *   eqlinear_conv_backward_weight: dWc [KH][KW][D][C][T] and dbias [D] (or NULL)
+ *     in the plan dtype. Each tap is the layer's weight gradient between the
+ *     rows of dY and the rows of X shifted by that tap (zero outside the image):
+ *     a gather into the workspace, then the layer's weight-gradient kernel
+ *     (tensor cores when C and D are multiples of 64).
+ *   eqlinear_conv_backward_workspace_bytes(plan, N, H, W, KH, KW, pad_h, pad_w):
+ *     scratch of both calls.
+ * Plans and limits as for eqlinear_conv_forward; all pointers 16-byte aligned;
+ * EQL_ERR_WORKSPACE for a short workspace; N = 0 does nothing.
+ */
+EQL_API size_t eqlinear_conv_backward_workspace_bytes(eqlinear_plan_t plan, int64_t N, int H,
+                                                      int W, int KH, int KW, int pad_h,
+                                                      int pad_w);
+EQL_API eqlinear_status_t eqlinear_conv_backward_input(eqlinear_plan_t plan, const void* dY,
+                                                       int64_t N, int H, int W, int KH, int KW,
+                                                       int pad_h, int pad_w, const void* Wc_hat,
+                                                       void* dX, void* workspace,
+                                                       size_t workspace_bytes, void* stream);
+EQL_API eqlinear_status_t eqlinear_conv_backward_weight(eqlinear_plan_t plan, const void* X,
+                                                        int64_t N, int H, int W, const void* dY,
+                                                        int KH, int KW, int pad_h, int pad_w,
+                                                        void* dWc, void* dbias, void* workspace,
+                                                        size_t workspace_bytes, void* stream);
 
 /*
  * Gradient with respect to the input ("Implementation": backward pass):
