@@ -57,6 +57,7 @@ PIPELINES = {
     "c8_1024_f16": ["c8_1024_f16"],
     "c8_1024_tiled_f16": ["c8_1024_f16"],
     "p4_vith_fc1_fwd_bwd_f16": ["p4_vith_fc1_f16"],
+    "p4_vith_fc1_fwd_bwd_tiled_f16": ["p4_vith_fc1_f16"],
     "p4_vitb_mlp_block_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
     "p4_vitb_mlp_spectral_f16": ["p4_vitb_fc1_f16", "p4_vitb_fc2_f16"],
     "p4m_vitb_mlp_f16": ["p4m_vitb_fc1_f16", "p4m_vitb_fc2_f16"],
@@ -68,7 +69,12 @@ DIHEDRAL = {"p4m_vitb_mlp_f16", "p4m_vitb_mlp_fused_f16"}
 # two-layer pipelines whose intermediate stays in the frequency domain (the first
 # layer's epilogue writes the second layer's operand planes)
 SPECTRAL = {"p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectral_f16"}
-BACKWARD = {"p4_vith_fc1_fwd_bwd_f16"}
+BACKWARD = {"p4_vith_fc1_fwd_bwd_f16", "p4_vith_fc1_fwd_bwd_tiled_f16"}
+# training steps in the frequency-domain form: one group-DFT launch for X (it
+# serves the forward and dW) and one for dY (dX and dW), the products on SM pairs
+# (eqlinear_forward_tiled, eqlinear_backward_input_tiled) and the weight gradient
+# from the two tiled planes (eqlinear_backward_weight_tiled)
+TILED_TRAIN = {"p4_vith_fc1_fwd_bwd_tiled_f16"}
 # two-layer pipelines run as one chained launch (eqlinear_forward_chain: both
 # layers' tiles in one dynamic queue; bitwise the two separate calls)
 CHAINED = {"p4_vitb_mlp_fused_f16", "p4_vitb_mlp_block_f16", "p4_vitb_mlp_spectral_f16"}
@@ -106,7 +112,11 @@ DESCR = {
     "c8_1024_tiled_f16": "cyclic T=8 EQ-Linear fp16: N=16384, C=D=128; group DFT to eight tiled "
                          "planes, then the products on SM pairs",
     "p4_vith_fc1_fwd_bwd_f16": "p4 EQ-Linear fp16 ViT-H fc1 forward + dX + dW: N=8224, "
-                               "C=320->D=1280, T=4",
+                               "C=320->D=1280, T=4; forward and dX in the one-CTA kernel, "
+                               "saving the group spectra that dW reads",
+    "p4_vith_fc1_fwd_bwd_tiled_f16": "p4 EQ-Linear fp16 ViT-H fc1 forward + dX + dW: N=8224, "
+                                     "C=320->D=1280, T=4; group DFTs of X and dY to tiled "
+                                     "planes, forward and dX on SM pairs, dW from the planes",
     "p4_vitb_mlp_block_f16": "p4 EQ-MLP block fp16 ViT-B: N=12608, EQ-Linear 192->768 + bias + "
                              "GELU (fused), EQ-Linear 768->192 + bias, T=4; intermediate kept as "
                              "the second layer's spectral planes; one chained launch",
@@ -157,6 +167,8 @@ KERNEL_SOURCES = {
                             "eql_tc_common.cuh"),
     "forward_tiled": ("eql_tc_pair32.cu", "eql_tc_pair8.cu", "eql_tc_pair_common.cuh",
                       "eql_tc_fwd_parts.cuh", "eql_tc_common.cuh"),
+    "forward_pair": ("eql_tc_pair.cu", "eql_tc_pair_common.cuh", "eql_tc_fwd_parts.cuh",
+                     "eql_tc_common.cuh"),
 }
 NCU_TRAFFIC = {
     ("forward", "443ba94f5b306a59"): {"p4_vitb_mlp_2calls_f16": 58.96e6, "c8_1024_f16": 34.20e6, "p4_vith_fc1_f16": 51.20e6, "p4_vith_fc1_fwd_bwd_f16": 109.13e6, "p4m_vitb_mlp_fused_f16": 57.79e6},
@@ -621,7 +633,12 @@ def run_ours(args, workload):
         per_set += sum(N * w.D * w.T * es + N * w.C * w.T * es for w in pipeline)
     # training: the forward and dX kernels save the group spectra of X and dY
     # (the same sizes) for the weight gradient, unless --wgrad-transform
-    saved = backward and not args.wgrad_transform
+    tiled_train = workload in TILED_TRAIN
+    if tiled_train:
+        # the tiled planes of X and of dY
+        per_set += sum(int(np.prod(plans[0].tiled_shape(N, c))) * es
+                       for c in (pipeline[0].C, pipeline[0].D))
+    saved = backward and not args.wgrad_transform and not tiled_train
     if saved:
         per_set += sum(N * w.C * w.T * es + N * w.D * w.T * es for w in pipeline[:1])
     nsets = max(2, int(np.ceil(2 * L2_BYTES / per_set)))
@@ -708,7 +725,23 @@ def run_ours(args, workload):
             ops.append(("group_dft", "simt", 0.0, (1 + pf) * es * N * w.C * w.T, dft_l))
             ops.append(("forward_tiled", tkern, layer_flops(w),
                         layer_bytes(w) + (pf - 1) * es * N * w.C * w.T, fwd_l))
-    for li, w in enumerate([] if chained or tiled or tiled_layers else pipeline):
+    if tiled_train:
+        w0 = pipeline[0]
+        xts = [torch.empty(plans[0].tiled_shape(N, w0.C), dtype=dt, device="cuda")
+               for _ in range(nsets)]
+        dyts = [torch.empty(plans[0].tiled_shape(N, w0.D), dtype=dt, device="cuda")
+                for _ in range(nsets)]
+
+        def dft_x(i):
+            plans[0].group_dft(xs[i % nsets], out=xts[i % nsets])
+
+        def fwd_t(i):
+            plans[0].forward_tiled(xts[i % nsets], N, whats[0], biases[0], act=acts[0],
+                                   out=outs[i % nsets][0])
+        ops.append(("group_dft", "simt", 0.0, 2.0 * es * N * w0.C * w0.T, dft_x))
+        ops.append(("forward_pair", "tcgen05", layer_flops(w0), layer_bytes(w0), fwd_t))
+    for li, w in enumerate([] if chained or tiled or tiled_layers or tiled_train
+                           else pipeline):
         def fwd(i, li=li):
             x = xs[i % nsets] if li == 0 else outs[i % nsets][li - 1]
             if spectral and li == 0:
@@ -731,8 +764,13 @@ def run_ours(args, workload):
         w0 = pipeline[0]
         pending = []
 
+        def dft_dy(i):
+            plans[0].group_dft(dys[i % nsets], out=dyts[i % nsets])
+
         def bwd_x(i):
-            if saved:
+            if tiled_train:
+                plans[0].backward_input_tiled(dyts[i % nsets], N, whats[0], out=dxs[i % nsets])
+            elif saved:
                 plans[0].backward_input_save_spectrum(dys[i % nsets], whats[0],
                                                       out=dxs[i % nsets], dYhat=ghats[i % nsets])
             else:
@@ -742,8 +780,12 @@ def run_ours(args, workload):
             # the weight gradient reads the spectra (or X and dY: the same bytes)
             a = xhats[i % nsets] if saved else xs[i % nsets]
             g = ghats[i % nsets] if saved else dys[i % nsets]
+            if tiled_train:
+                a, g = xts[i % nsets], dyts[i % nsets]
             if dp:
-                if saved:
+                if tiled_train:
+                    plans[0].backward_weight_tiled_f32(a, g, N, buf=gbuf32, workspace=ws)
+                elif saved:
                     plans[0].backward_weight_from_spectra_f32(a, g, buf=gbuf32, workspace=ws)
                 else:
                     plans[0].backward_weight_f32(a, g, buf=gbuf32, workspace=ws)
@@ -751,7 +793,9 @@ def run_ours(args, workload):
                 pending.append(allreduce_grad_buffer(gbuf32, async_op=True))
             else:
                 dW, db = plans[0].split_grad(gbufs[i % 2])
-                if saved:
+                if tiled_train:
+                    plans[0].backward_weight_tiled(a, g, N, dW=dW, dbias=db, workspace=ws)
+                elif saved:
                     plans[0].backward_weight_from_spectra(a, g, dW=dW, dbias=db, workspace=ws)
                 else:
                     plans[0].backward_weight(a, g, dW=dW, dbias=db, workspace=ws)
@@ -765,16 +809,24 @@ def run_ours(args, workload):
         op_dx = ("backward_input", plans[0].forward_kernel_name(N), layer_flops(w0),
                  nb + es * 1.25 * w0.C * w0.D * w0.T + (es * N * w0.D * w0.T if saved else 0),
                  bwd_x)
+        if tiled_train:
+            # dX reads dY's planes (dY's bytes) and the adjoint weight stages
+            op_dx = ("backward_input_pair", "tcgen05", layer_flops(w0),
+                     nb + es * 1.25 * w0.C * w0.D * w0.T, bwd_x)
         op_dw = ("backward_weight", plans[0].backward_weight_kernel_name(N), wgrad_flops(w0),
                  nb + es * w0.D * w0.C * w0.T, bwd_w)
         if dp:
             # dW from saved spectra needs dX's saved dY spectrum, so it follows dX;
-            # the transforming dW goes first and its all-reduce overlaps dX
+            # the transforming dW (and dW from tiled planes, which needs only dY's
+            # transform) goes first and its all-reduce overlaps dX
             first_two = [op_dx, op_dw] if saved else [op_dw, op_dx]
             ops += first_two + [("weight_grad_allreduce", "nccl+cast", 0.0,
                                  (4 + es) * gbuf.numel(), grad_sync)]
         else:
             ops += [op_dx, op_dw]
+        if tiled_train:
+            ops.insert(len(ops) - (3 if dp else 2),
+                       ("group_dft", "simt", 0.0, 2.0 * es * N * w0.D * w0.T, dft_dy))
 
     def step(i, events=None, external=False):
         for _, _, _, _, fn in ops:
@@ -931,7 +983,8 @@ def run_ours(args, workload):
         mean_ms = launch_ms.mean(axis=0)
         fam = {}
         for j, (label, kern, f, nbytes, _) in enumerate(ops):
-            key = (label if label != "backward_input" else "forward", kern)
+            key = ({"backward_input": "forward", "backward_input_pair": "forward_pair"}
+                   .get(label, label), kern)
             a = fam.setdefault(key, [0.0, 0.0, 0.0, 0])
             a[0] += mean_ms[j]
             a[1] += f

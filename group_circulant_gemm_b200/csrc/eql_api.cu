@@ -559,7 +559,7 @@ eqlinear_status_t eqlinear_forward_chain(eqlinear_plan_t first, eqlinear_plan_t 
 static eqlinear_status_t backward_weight_impl(eqlinear_plan_t p, const void* X, const void* dY,
                                               int64_t N, void* dW, void* dbias, void* workspace,
                                               size_t workspace_bytes, eql::DType out_dt,
-                                              void* stream, bool spectra);
+                                              void* stream, int spectra);
 
 static bool conv_plan_ok(eqlinear_plan_t p) {
   return p && p->T == 4 && p->dtype == EQL_F16 && p->kernel != EQL_KERNEL_SIMT && has_tiles(p);
@@ -701,7 +701,7 @@ eqlinear_status_t eqlinear_conv_backward_weight(eqlinear_plan_t p, const void* X
     s = backward_weight_impl(p, N > 0 ? xs : nullptr, dY, rows,
                              static_cast<char*>(dWc) + (size_t)tap * w_tap,
                              tap == 0 ? dbias : nullptr, ws, ws_bytes, to_dt(p->dtype), stream,
-                             false);
+                             0);
     if (s != EQL_OK) return s;
   }
   return EQL_OK;
@@ -809,20 +809,24 @@ size_t eqlinear_backward_weight_workspace_bytes(eqlinear_plan_t p, int64_t N) {
   return need;
 }
 
-// spectra = true: X and dY are the group spectra [4][N][C] and [4][N][D] that
-// the save-spectrum calls wrote (tensor cores only; C and D multiples of 64).
+// spectra = 1: X and dY are the group spectra [4][N][C] and [4][N][D] that
+// the save-spectrum calls wrote (tensor cores only; C and D multiples of 64);
+// spectra = 2: the tiled planes eqlinear_group_dft writes (C, D multiples of 16).
 static eqlinear_status_t backward_weight_impl(eqlinear_plan_t p, const void* X, const void* dY,
                                               int64_t N, void* dW, void* dbias, void* workspace,
                                               size_t workspace_bytes, eql::DType out_dt,
-                                              void* stream, bool spectra = false) {
+                                              void* stream, int spectra = 0) {
   if (!p || N < 0 || !dW) return EQL_ERR_INVALID_ARG;
   if (p->group == 1 && (spectra || p->kernel == EQL_KERNEL_TCGEN05)) return EQL_ERR_UNSUPPORTED;
   if (N > 0 && (!X || !dY)) return EQL_ERR_INVALID_ARG;
   if ((X && !aligned16(X)) || (dY && !aligned16(dY)) || !aligned16(dW) ||
       (dbias && !aligned16(dbias)) || (workspace && !aligned16(workspace)))
     return EQL_ERR_ALIGNMENT;
-  if (spectra && !(p->T == 4 && p->dtype == EQL_F16 && p->kernel != EQL_KERNEL_SIMT &&
-                   p->C % 64 == 0 && p->D % 64 == 0))
+  if (spectra == 1 && !(p->T == 4 && p->dtype == EQL_F16 && p->kernel != EQL_KERNEL_SIMT &&
+                        p->C % 64 == 0 && p->D % 64 == 0))
+    return EQL_ERR_UNSUPPORTED;
+  if (spectra == 2 && !(p->T == 4 && p->group == 0 && p->dtype == EQL_F16 &&
+                        p->kernel != EQL_KERNEL_SIMT && has_tiles(p)))
     return EQL_ERR_UNSUPPORTED;
   if (!spectra && p->kernel == EQL_KERNEL_TCGEN05 && !wgrad_tc_ok(p, N, X, dY))
     return EQL_ERR_UNSUPPORTED;
@@ -834,10 +838,16 @@ static eqlinear_status_t backward_weight_impl(eqlinear_plan_t p, const void* X, 
   if (p->group == 1)  // D4: CUDA cores
     return from_cuda(eql::launch_d4_wgrad(X, dY, N, p->C, p->D, out_dt, dW, dbias,
                                           static_cast<float*>(workspace), p->num_sms, st));
-  if (spectra && N > 0) {
+  if (spectra == 1 && N > 0) {
     if (!eql::wgrad_tc_planes_supported(N, p->C, p->D, X, dY)) return EQL_ERR_UNSUPPORTED;
     return from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, workspace, out_dt, dW, dbias,
-                                          p->status, p->num_sms, p->tw, st, true));
+                                          p->status, p->num_sms, p->tw, st, 1));
+  }
+  if (spectra == 2 && N > 0) {
+    if (!eql::wgrad_tc_supported(4, eql::DType::F16, N, p->C, p->D, X, dY))
+      return EQL_ERR_UNSUPPORTED;
+    return from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, workspace, out_dt, dW, dbias,
+                                          p->status, p->num_sms, p->tw, st, 2));
   }
   if (!spectra && wgrad_use_tc(p, N, X, dY))
     return from_cuda(eql::launch_wgrad_tc(X, dY, N, p->C, p->D, workspace, out_dt, dW, dbias,
@@ -873,7 +883,7 @@ eqlinear_status_t eqlinear_backward_weight_from_spectra(eqlinear_plan_t p, const
   EQL_TRACE();
   if (!p) return EQL_ERR_INVALID_ARG;
   return backward_weight_impl(p, Xhat, dYhat, N, dW, dbias, workspace, workspace_bytes,
-                              to_dt(p->dtype), stream, true);
+                              to_dt(p->dtype), stream, 1);
 }
 
 eqlinear_status_t eqlinear_backward_weight_from_spectra_f32(eqlinear_plan_t p, const void* Xhat,
@@ -883,7 +893,26 @@ eqlinear_status_t eqlinear_backward_weight_from_spectra_f32(eqlinear_plan_t p, c
                                                             size_t workspace_bytes, void* stream) {
   EQL_TRACE();
   return backward_weight_impl(p, Xhat, dYhat, N, dW, dbias, workspace, workspace_bytes,
-                              eql::DType::F32, stream, true);
+                              eql::DType::F32, stream, 1);
+}
+
+eqlinear_status_t eqlinear_backward_weight_tiled(eqlinear_plan_t p, const void* Xt,
+                                                  const void* dYt, int64_t N, void* dW,
+                                                  void* dbias, void* workspace,
+                                                  size_t workspace_bytes, void* stream) {
+  EQL_TRACE();
+  if (!p) return EQL_ERR_INVALID_ARG;
+  return backward_weight_impl(p, Xt, dYt, N, dW, dbias, workspace, workspace_bytes,
+                              to_dt(p->dtype), stream, 2);
+}
+
+eqlinear_status_t eqlinear_backward_weight_tiled_f32(eqlinear_plan_t p, const void* Xt,
+                                                      const void* dYt, int64_t N, float* dW,
+                                                      float* dbias, void* workspace,
+                                                      size_t workspace_bytes, void* stream) {
+  EQL_TRACE();
+  return backward_weight_impl(p, Xt, dYt, N, dW, dbias, workspace, workspace_bytes,
+                              eql::DType::F32, stream, 2);
 }
 
 eqlinear_status_t eqlinear_cast_from_f32(eqlinear_plan_t p, const float* src, int64_t count,

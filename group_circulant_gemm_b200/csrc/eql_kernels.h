@@ -73,14 +73,15 @@ cudaError_t launch_fwd_tc(int T, const void* X, int64_t N, int Cin, int Cout,
 // handled by the caller.
 bool wgrad_tc_supported(int T, DType dt, int64_t N, int C, int D, const void* X, const void* dY);
 size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms);
-// planes = true: X and dY are instead their group spectra as FP16 planes
+// planes = 1: X and dY are instead their group spectra as FP16 planes
 // [4][N][C] and [4][N][D] (as the forward and dX kernels save them); needs
-// C % 64 == 0 and D % 64 == 0 (wgrad_tc_planes_supported).
+// C % 64 == 0 and D % 64 == 0 (wgrad_tc_planes_supported).  planes = 2: the
+// spectra in the tiled layout of the SM-pair kernels (tiled_rows(N) rows per
+// 16-channel block, as launch_group_dft_tiled writes them); C, D multiples of 16.
 bool wgrad_tc_planes_supported(int64_t N, int C, int D, const void* Xhat, const void* Ghat);
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
                             void* workspace, DType out_dt, void* dW, void* dbias, int* status,
-                            int num_sms, const Twiddles& tw, cudaStream_t st,
-                            bool planes = false);
+                            int num_sms, const Twiddles& tw, cudaStream_t st, int planes = 0);
 
 // Two chained T = 4 FP16 layers (C0 -> C1 -> C2) in one persistent launch with a
 // dynamic tile queue: H = act1(L1(X)) (spatial [N][C1*4], or spectral planes

@@ -286,7 +286,10 @@ struct PairTask {
   int layer, prow, dt;
 };
 
-// One layer: task u = (prow, dt) of layer 0.  Chain: the layer-1 tiles of the
+// One layer: task u = (prow, dt) of layer 0, the full 128-channel tiles of every
+// row block first and a narrow last tile's tasks after them, so a pair that takes
+// a second task takes the cheaper kind (the static list gives pairs 0, 1, ...
+// the tasks npairs, npairs + 1, ... next).  Chain: the layer-1 tiles of the
 // first `lag` row blocks, then per row block k the layer-1 tiles of k and the
 // layer-2 tiles of k - lag, then the rest of layer 2 (every layer-1 tile of a
 // row block precedes that block's layer-2 tiles, and all CTAs are resident, so
@@ -296,8 +299,14 @@ __device__ __forceinline__ PairTask pair_decode(int q, const PairSched& sc) {
   PairTask t;
   if constexpr (!CHAIN) {
     t.layer = 0;
-    t.prow = q / sc.L[0].n_dt;
-    t.dt = q % sc.L[0].n_dt;
+    const int nf = sc.L[0].n_dt - (sc.L[0].narrow ? 1 : 0);  // full tiles per row block
+    if (q < sc.n_prow * nf) {
+      t.prow = q / nf;
+      t.dt = q % nf;
+    } else {
+      t.prow = q - sc.n_prow * nf;
+      t.dt = nf;
+    }
   } else {
     const int n1 = sc.L[0].n_dt, n2 = sc.L[1].n_dt;
     const int a = sc.lag * n1, per = n1 + n2, b = (sc.n_prow - sc.lag) * per;

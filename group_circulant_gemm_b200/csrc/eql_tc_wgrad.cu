@@ -56,6 +56,15 @@
 // stride).  Warps 8-11 sum plane 0 of dY's spectrum for dbias; warps 4-7 and
 // 12-15 drain planes 0-1 and 2-3 of the accumulators.  Needs C and D
 // multiples of 64.
+//
+// Tiled variant (PL, TL): the same spectra in the tiled layout of the SM-pair
+// kernels ([plane][channel / 16][Np rows][16 channels], 32-byte rows stored with
+// the 32-byte swizzle, written by the group-DFT pass).  One 4-D box per operand
+// (8 lines of 4 rows, 8 blocks of 16 channels, 4 planes) lands as [plane][block]
+// [32 rows][32 B], which is already the MN-major 32-byte-swizzled operand image:
+// 16-channel blocks 1 KB apart (LBO), 8-row K groups 256 B apart (SBO), so the
+// N = 256 [Xr | Xi] operand again spans planes 2 and 3 at a uniform stride.
+// Channel counts need only be multiples of 16 (the box reads zeros past C).
 
 #include <algorithm>
 
@@ -102,6 +111,12 @@ static_assert(WG_SMEM <= 232448, "shared memory budget");
 __device__ __forceinline__ uint64_t desc_mn128(uint32_t saddr, uint32_t lbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(lbo >> 4) << 16) |
          ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// MN-major operand of a tiled slot: 16-channel blocks 1 KB apart (LBO), 8-row K
+// groups 256 B apart (SBO), 32-byte swizzle (layout type 6), descriptor v1.
+__device__ __forceinline__ uint64_t desc_mn32(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(1024u >> 4) << 16) |
+         ((uint64_t)(256u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)6u << 61);
 }
 // kind::f16 instruction descriptor with both operands MN-major (bits 15, 16).
 __host__ __device__ constexpr uint32_t idesc_f16_mn(int M, int N, bool negate_a = false) {
@@ -243,7 +258,7 @@ __device__ __forceinline__ void wg_transform(uint8_t* tile, int w, int j, int q,
   }
 }
 
-template <bool PL>
+template <bool PL, bool TL = false>
 __global__ void __launch_bounds__(PL ? WG_THREADS_PL : WG_THREADS, 1)
     wgrad_tc_kernel(const __grid_constant__ CUtensorMap map_g,
                     const __grid_constant__ CUtensorMap map_x, int64_t N, int C, int D,
@@ -305,7 +320,11 @@ __global__ void __launch_bounds__(PL ? WG_THREADS_PL : WG_THREADS, 1)
           mbar_expect_tx(&bars->full[slot], SLOT);
           const int row = (int)(un.r0 + (int64_t)(WG_BR / SUB) * s);
           const uint32_t dst = sbase + slot * SLOT;
-          if constexpr (PL) {
+          if constexpr (PL && TL) {
+            // 4-D tiled views (128-byte line = 4 rows, line, 16-channel block, plane)
+            tma_load_4d(dst, &map_g, &bars->full[slot], 0, row / 4, 8 * un.dt, 0);
+            tma_load_4d(dst + TILEB, &map_x, &bars->full[slot], 0, row / 4, 8 * un.ct, 0);
+          } else if constexpr (PL) {
             // 4-D planes views (64 channels, row, 64-channel block, plane)
             tma_load_4d(dst, &map_g, &bars->full[slot], 0, row, 2 * un.dt, 0);
             tma_load_4d(dst + TILEB, &map_x, &bars->full[slot], 0, row, 2 * un.ct, 0);
@@ -347,13 +366,15 @@ __global__ void __launch_bounds__(PL ? WG_THREADS_PL : WG_THREADS, 1)
           for (int kk = 0; kk < WG_BR / 16 / SUB; ++kk) {
             const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
             // transform path: K-major planes, K step = 32 B of a row; planes path:
-            // MN-major planes, K step = 16 rows x 128 B
+            // MN-major planes, K step = 16 rows x 128 B (tiled: 16 rows x 32 B)
             auto A = [&](int p) {
-              return PL ? desc_mn128(g + p * PL_PLANE + 2048u * kk, PL_BLOCK)
+              return PL ? (TL ? desc_mn32(g + p * PL_PLANE + 512u * kk)
+                              : desc_mn128(g + p * PL_PLANE + 2048u * kk, PL_BLOCK))
                         : desc_kmajor<WG_ROWB>(g + p * WG_PLANE + 32u * kk);
             };
             auto B = [&](int p) {
-              return PL ? desc_mn128(x + p * PL_PLANE + 2048u * kk, PL_BLOCK)
+              return PL ? (TL ? desc_mn32(x + p * PL_PLANE + 512u * kk)
+                              : desc_mn128(x + p * PL_PLANE + 2048u * kk, PL_BLOCK))
                         : desc_kmajor<WG_ROWB>(x + p * WG_PLANE + 32u * kk);
             };
             umma(tmem + 0, A(0), B(0), id_n1, acc);              // Q0
@@ -420,7 +441,8 @@ __global__ void __launch_bounds__(PL ? WG_THREADS_PL : WG_THREADS, 1)
   } else if (PL && warp >= WG_XF0 && warp < WG_XF0 + WG_BIASW) {
     // ---------------- planes variant: dbias partials from plane 0 of dY's spectrum ----------------
     // thread = out-channel dl of the tile; plane 0 sits at [block dl / 64][row][128 B],
-    // 16-byte piece (dl % 64) / 8 swizzled with row % 8
+    // 16-byte piece (dl % 64) / 8 swizzled with row % 8 (tiled: [block dl / 16][row]
+    // [32 B], piece (dl % 16) / 8 swizzled with (row / 4) % 2)
     const int dl = (warp - WG_XF0) * 32 + lane;
     uint32_t it = 0;
     bool ok = true;
@@ -432,12 +454,21 @@ __global__ void __launch_bounds__(PL ? WG_THREADS_PL : WG_THREADS, 1)
         const int slot = it % RING;
         if (!(ok = warp_wait(&bars->full[slot], (it / RING) & 1, abort_flag, status))) break;
         if (un.ct == 0) {
-          const uint8_t* blk = smem + slot * SLOT + (dl >> 6) * PL_BLOCK;
-          const int piece = (dl & 63) >> 3, within = (dl & 7) * 2;
+          if constexpr (TL) {
+            const uint8_t* blk = smem + slot * SLOT + (dl >> 4) * 1024;
+            const int piece = (dl & 15) >> 3, within = (dl & 7) * 2;
 #pragma unroll 8
-          for (int r = 0; r < PL_ROWS; ++r)
-            b += __half2float(
-                *reinterpret_cast<const __half*>(blk + r * 128 + ((piece ^ (r & 7)) << 4) + within));
+            for (int r = 0; r < PL_ROWS; ++r)
+              b += __half2float(*reinterpret_cast<const __half*>(
+                  blk + r * 32 + ((piece ^ ((r >> 2) & 1)) << 4) + within));
+          } else {
+            const uint8_t* blk = smem + slot * SLOT + (dl >> 6) * PL_BLOCK;
+            const int piece = (dl & 63) >> 3, within = (dl & 7) * 2;
+#pragma unroll 8
+            for (int r = 0; r < PL_ROWS; ++r)
+              b += __half2float(*reinterpret_cast<const __half*>(
+                  blk + r * 128 + ((piece ^ (r & 7)) << 4) + within));
+          }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->empty[slot]);
@@ -597,6 +628,24 @@ bool encode_planes4_map(CUtensorMap* m, const void* base, int channels, int64_t 
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tiled planes (tiled_rows(N) rows per 16-channel block) viewed as (64 halves of
+// a 128-byte line, line, 16-channel block, plane); box = (64, 8 lines, 8 blocks,
+// 4 planes), no swizzle (the rows are stored swizzled).
+bool encode_tiled4_map(CUtensorMap* m, const void* base, int channels, int64_t N) {
+  auto encode = encode_fn();
+  if (!encode || channels % 16 != 0) return false;
+  const int64_t Np = tiled_rows(N);
+  const int kb = channels / 16;
+  cuuint64_t dims[4] = {64, (cuuint64_t)(Np / 4), (cuuint64_t)kb, 4};
+  cuuint64_t strides[3] = {128, (cuuint64_t)Np * 32, (cuuint64_t)Np * 32 * kb};
+  cuuint32_t box[4] = {64, PL_ROWS / 4, 8, 4};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The stream-K layout for N rows: equal contiguous ranges of (tile, stage), one
 // per CTA, and the number of partial slots a tile can need.
 bool wgrad_tc_layout(int64_t N, int C, int D, int num_sms, WgInfo* wi, int* grid) {
@@ -653,13 +702,17 @@ bool wgrad_tc_planes_supported(int64_t N, int C, int D, const void* Xhat, const 
 
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
                             void* workspace, DType out_dt, void* dW, void* dbias, int* status,
-                            int num_sms, const Twiddles& tw, cudaStream_t st, bool planes) {
+                            int num_sms, const Twiddles& tw, cudaStream_t st, int planes) {
   WgInfo wi;
   int grid = 0;
   if (!wgrad_tc_layout(N, C, D, num_sms, &wi, &grid)) return cudaErrorInvalidValue;
-  if (planes && (C % 64 != 0 || D % 64 != 0)) return cudaErrorNotSupported;
+  if (planes < 0 || planes > 2) return cudaErrorInvalidValue;
+  if (planes == 1 && (C % 64 != 0 || D % 64 != 0)) return cudaErrorNotSupported;
   CUtensorMap mg, mx;
-  if (planes) {
+  if (planes == 2) {
+    if (!encode_tiled4_map(&mg, dY, D, N) || !encode_tiled4_map(&mx, X, C, N))
+      return cudaErrorInvalidValue;
+  } else if (planes == 1) {
     if (!encode_planes4_map(&mg, dY, D, N) || !encode_planes4_map(&mx, X, C, N))
       return cudaErrorInvalidValue;
   } else if (!encode_rows_map(&mg, dY, D, N) || !encode_rows_map(&mx, X, C, N)) {
@@ -674,10 +727,16 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(wgrad_tc_kernel<true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(wgrad_tc_kernel<true, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  if (planes)
+  if (planes == 2)
+    wgrad_tc_kernel<true, true><<<grid, WG_THREADS_PL, WG_SMEM, st>>>(mg, mx, N, C, D, wi, part,
+                                                                      bpart, status);
+  else if (planes == 1)
     wgrad_tc_kernel<true><<<grid, WG_THREADS_PL, WG_SMEM, st>>>(mg, mx, N, C, D, wi, part, bpart,
                                                                 status);
   else

@@ -172,6 +172,38 @@ class EqLinearPlan:
         _n.eqlinear_backward_input_tiled(self.handle, dYt, N, W_hat, out)
         return out
 
+    def backward_weight_tiled(self, Xt, dYt, N: int, dW=None, dbias=None, workspace=None,
+                              want_bias=True):
+        """(dW [D, C, T], dbias [D]) from the tiled planes of X and dY (group_dft of each)."""
+        self._check(Xt, self.tiled_shape(N, self.C), "Xt")
+        self._check(dYt, self.tiled_shape(N, self.D), "dYt")
+        if dW is None:
+            dW = torch.empty((self.D, self.C, self.T), dtype=self.dtype, device=Xt.device)
+        if dbias is None and want_bias:
+            dbias = torch.empty((self.D,), dtype=self.dtype, device=Xt.device)
+        if workspace is None:
+            workspace = torch.empty(max(self.workspace_bytes(N), 16), dtype=torch.uint8,
+                                    device=Xt.device)
+        _n.eqlinear_backward_weight_tiled(self.handle, Xt, dYt, N, dW, dbias, workspace,
+                                          workspace.numel() * workspace.element_size())
+        return dW, dbias
+
+    def backward_weight_tiled_f32(self, Xt, dYt, N: int, buf=None, workspace=None):
+        """backward_weight_f32 from the tiled planes of X and dY."""
+        self._check(Xt, self.tiled_shape(N, self.C), "Xt")
+        self._check(dYt, self.tiled_shape(N, self.D), "dYt")
+        if buf is None:
+            buf = self.grad_buffer(torch.float32, Xt.device)
+        if buf.dtype != torch.float32 or buf.numel() != self.grad_offset() + self.D:
+            raise ValueError("buf must be a flat FP32 gradient buffer of this plan")
+        dW, db = self.split_grad(buf)
+        if workspace is None:
+            workspace = torch.empty(max(self.workspace_bytes(N), 16), dtype=torch.uint8,
+                                    device=Xt.device)
+        _n.eqlinear_backward_weight_tiled_f32(self.handle, Xt, dYt, N, dW, db, workspace,
+                                              workspace.numel() * workspace.element_size())
+        return buf
+
     def backward_input(self, dY, W_hat, out=None) -> torch.Tensor:
         N = dY.shape[0]
         self._check(dY, (N, self.D * self.T), "dY")

@@ -38,6 +38,7 @@ EXPORTED = (
     "eqlinear_plan_create_dihedral4",
     "eqlinear_forward_save_spectrum", "eqlinear_backward_input_save_spectrum",
     "eqlinear_backward_weight_from_spectra", "eqlinear_backward_weight_from_spectra_f32",
+    "eqlinear_backward_weight_tiled", "eqlinear_backward_weight_tiled_f32",
     "eqlinear_tiled_spectrum_bytes", "eqlinear_group_dft", "eqlinear_forward_tiled",
     "eqlinear_forward_tiled_next", "eqlinear_backward_input_tiled",
     "eqlinear_chain_tiled_workspace_bytes", "eqlinear_forward_chain_tiled",
@@ -91,6 +92,8 @@ def _load() -> ctypes.CDLL:
         "eqlinear_forward_save_spectrum": ([vp, vp, i64, vp, vp, i32, vp, vp, vp], i32),
         "eqlinear_backward_input_save_spectrum": ([vp, vp, i64, vp, vp, vp, vp], i32),
         "eqlinear_backward_weight_from_spectra": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
+        "eqlinear_backward_weight_tiled": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
+        "eqlinear_backward_weight_tiled_f32": ([vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
         "eqlinear_backward_weight_from_spectra_f32": ([vp, vp, vp, i64, vp, vp, vp, sz, vp],
                                                       i32),
         "eqlinear_chain_workspace_bytes": ([vp, vp, i64], sz),
@@ -303,6 +306,22 @@ def eqlinear_backward_weight_from_spectra(plan: int, Xhat, dYhat, N: int, dW, db
                                                       _ptr(dbias), _ptr(workspace),
                                                       workspace_bytes, _stream(stream)),
            "eqlinear_backward_weight_from_spectra")
+
+
+def eqlinear_backward_weight_tiled(plan: int, Xt, dYt, N: int, dW, dbias, workspace,
+                                   workspace_bytes: int, stream=None) -> None:
+    _check(_lib.eqlinear_backward_weight_tiled(plan, _ptr(Xt), _ptr(dYt), N, _ptr(dW),
+                                               _ptr(dbias), _ptr(workspace), workspace_bytes,
+                                               _stream(stream)),
+           "eqlinear_backward_weight_tiled")
+
+
+def eqlinear_backward_weight_tiled_f32(plan: int, Xt, dYt, N: int, dW, dbias, workspace,
+                                       workspace_bytes: int, stream=None) -> None:
+    _check(_lib.eqlinear_backward_weight_tiled_f32(plan, _ptr(Xt), _ptr(dYt), N, _ptr(dW),
+                                                   _ptr(dbias), _ptr(workspace), workspace_bytes,
+                                                   _stream(stream)),
+           "eqlinear_backward_weight_tiled_f32")
 
 
 def eqlinear_backward_weight_from_spectra_f32(plan: int, Xhat, dYhat, N: int, dW, dbias,

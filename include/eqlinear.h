@@ -294,6 +294,34 @@ EQL_API eqlinear_status_t eqlinear_backward_input_tiled(eqlinear_plan_t plan, co
                                                         void* stream);
 
 /*
+ * The weight gradient from tiled planes ("Implementation", bullet 1: the backward
+ * is the same per-frequency product, transposed, summed over rows):
+ * eqlinear_backward_weight_tiled(plan, Xt, dYt, N, dW, dbias, ...) gives
+ * eqlinear_backward_weight of X [N][C*4] and dY [N][D*4] from their tiled
+ * planes Xt and dYt (eqlinear_group_dft of each), so one transform of X serves
+ * the forward and dW, and one of dY serves dX and dW.  dW [D][C][4], dbias [D]
+ * (may be NULL), workspace as eqlinear_backward_weight
+ * (eqlinear_backward_weight_workspace_bytes); _f32 writes FP32 dW and dbias as
+ * eqlinear_backward_weight_f32.  dW's operands are the planes' FP16 values;
+ * dbias sums dYt's plane 0 (rounded to FP16) times 4.  The padding rows of the
+ * planes must be zero, as eqlinear_group_dft leaves them (the planes of
+ * eqlinear_forward_tiled_next do not qualify).
+ *
+ * p4 FP16 plans with C and D multiples of 16, not forced to the CUDA cores;
+ * otherwise EQL_ERR_UNSUPPORTED.  Pointers 16-byte aligned; N = 0 writes zeros.
+ */
+EQL_API eqlinear_status_t eqlinear_backward_weight_tiled(eqlinear_plan_t plan, const void* Xt,
+                                                         const void* dYt, int64_t N, void* dW,
+                                                         void* dbias, void* workspace,
+                                                         size_t workspace_bytes, void* stream);
+EQL_API eqlinear_status_t eqlinear_backward_weight_tiled_f32(eqlinear_plan_t plan,
+                                                             const void* Xt, const void* dYt,
+                                                             int64_t N, float* dW, float* dbias,
+                                                             void* workspace,
+                                                             size_t workspace_bytes,
+                                                             void* stream);
+
+/*
  * Two chained layers on tiled planes in one launch (the MLP pair of a Flash
  * EQ-ViT block, kept in the frequency domain between the layers):
  *   Ht = tiled planes of act1(first(X))   (as eqlinear_forward_tiled_next)

@@ -149,9 +149,9 @@ def test_tiled_entries_reject_what_they_do_not_take():
     p.set_kernel("simt")
     assert n.raw_status("eqlinear_forward_tiled_next", p.handle, Xt.data_ptr(), 64,
                         Wh.data_ptr(), None, 0, Xt.data_ptr(), None) == n.EQL_ERR_UNSUPPORTED
-    # T = 8 plans neither
-    p8 = _plan(8, 16, 16)
-    assert n.raw_status("eqlinear_group_dft", p8.handle, X.data_ptr(), 64, 16, Xt.data_ptr(),
+    # T = 3 plans neither (T = 4 and 8 only)
+    p3 = _plan(3, 16, 16)
+    assert n.raw_status("eqlinear_group_dft", p3.handle, X.data_ptr(), 64, 16, Xt.data_ptr(),
                         None) == n.EQL_ERR_UNSUPPORTED
     # N = 0 is a no-op
     p.set_kernel("auto")
