@@ -173,9 +173,10 @@ KERNEL_SOURCES = {
 NCU_TRAFFIC = {
     ("forward", "443ba94f5b306a59"): {"p4_vitb_mlp_2calls_f16": 58.96e6, "c8_1024_f16": 34.20e6, "p4_vith_fc1_f16": 51.20e6, "p4_vith_fc1_fwd_bwd_f16": 109.13e6, "p4m_vitb_mlp_fused_f16": 57.79e6},
     ("forward_chain", "246b0f491b3357c1"): {"p4_vitb_mlp_fused_f16": 89.59e6, "p4_vitb_mlp_spectral_f16": 80.93e6, "p4_vitb_mlp_block_f16": 81.74e6},
-    ("conv", "30f615e6470be609"): {"p4_conv3x3_f16": 162.29e6},
-    ("forward_chain_tiled", "46882cfee44bc9af"): {"p4_vitb_mlp_f16": 103.14e6},
-    ("forward_tiled", "99717903cdc1492d"): {"p4_vitb_proj_f32": 85.78e6, "p4m_vitb_mlp_f16": 58.38e6, "c8_1024_tiled_f16": 34.38e6},
+    ("conv", "d28bc5734eac2b53"): {"p4_conv3x3_f16": 161.54e6},
+    ("forward_chain_tiled", "6ade53bcfcfaa10b"): {"p4_vitb_mlp_f16": 99.44e6},
+    ("forward_pair", "6ade53bcfcfaa10b"): {"p4_vith_fc1_fwd_bwd_tiled_f16": 96.53e6},
+    ("forward_tiled", "00b0eabab3294aea"): {"p4_vitb_proj_f32": 85.78e6, "p4m_vitb_mlp_f16": 58.38e6, "c8_1024_tiled_f16": 34.38e6},
 }
 
 def kernel_traffic(family: str, workload: str):

@@ -796,39 +796,33 @@ __global__ void pair_tile_weights_kernel(const __half* __restrict__ planes, int 
 
 // Group DFT of p4 rows into tiled planes (layout above): X [N][C*4] -> the
 // four planes, each value times 1/4 (FP32 arithmetic, one rounding), rows
-// N..Np-1 zero.  A warp takes 4 rows and up to 4 blocks of 16 channels.  Per
-// block a lane loads 16 bytes (lane l: row 4r + l/8, channels 2(l%8) and
-// 2(l%8)+1 of the block, all four group elements), so each load instruction
-// reads 4 whole 128-byte row segments; per plane a lane stores the 4 bytes of
-// its two channels, so each store instruction writes 128 contiguous bytes (4
-// rows of 32).  The block loads are all issued before the first is used.
+// N..Np-1 zero.  A thread takes 8 channels of one row (64 bytes of X, four
+// 16-byte loads) and writes one 16-byte half row per plane; a warp takes 16
+// rows of one 16-channel block (lane l: row l/2, channels 8(l%2)..+7), so each
+// of its four plane stores fills 512 contiguous bytes of the tiled layout.
 __global__ void group_dft_tiled_kernel(const uint4* __restrict__ X, int64_t N, int64_t Np, int C,
                                        uint8_t* __restrict__ out) {
-  constexpr int G = 4;  // channel blocks per warp
   grid_dependency_wait();
   grid_launch_dependents();
   const int KB = C / 16;
-  const int KBG = (KB + G - 1) / G;
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (w >= Np / 4 * KBG) return;
+  if (w >= Np / 16 * KB) return;
   const int lane = (int)(threadIdx.x & 31);
-  const int kb0 = (int)(w % KBG) * G;
-  const int64_t n = (w / KBG) * 4 + (lane >> 3);
-  const int piece = lane & 7;
-  uint4 v[G];
+  const int kb = (int)(w % KB), h = lane & 1;
+  const int64_t n = (w / KB) * 16 + (lane >> 1);
+  uint4 v[4];
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    v[g] = make_uint4(0u, 0u, 0u, 0u);
-    if (n < N && kb0 + g < KB) v[g] = X[(n * C * 8 + (int64_t)(kb0 + g) * 128 + piece * 16) / 16];
+  for (int k = 0; k < 4; ++k) {
+    v[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (n < N) v[k] = X[(n * C * 8 + (int64_t)kb * 128 + h * 64) / 16 + k];
   }
-  const int64_t inrow = n * 32 + (((piece >> 2) ^ (int)((n >> 2) & 1)) << 4) + (piece & 3) * 4;
+  uint32_t o[4][4];  // [plane][channel pair k]: channels 8h + 2k, 8h + 2k + 1
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    if (kb0 + g >= KB) break;
-    const uint32_t w4[4] = {v[g].x, v[g].y, v[g].z, v[g].w};
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t w4[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
     float f0[2], fh[2], fr[2], fi[2];
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {  // channel 2*piece + e: x0 x1 | x2 x3
+    for (int e = 0; e < 2; ++e) {  // channel 8h + 2k + e: x0 x1 | x2 x3
       const float2 lo = unpack_h2(w4[2 * e]), hi = unpack_h2(w4[2 * e + 1]);
       const float x0 = lo.x, x1 = lo.y, x2 = hi.x, x3 = hi.y;
       const float a = x0 + x2, b = x1 + x3;
@@ -837,12 +831,16 @@ __global__ void group_dft_tiled_kernel(const uint4* __restrict__ X, int64_t N, i
       fr[e] = (x0 - x2) * 0.25f;
       fi[e] = (x3 - x1) * 0.25f;
     }
-    const uint32_t o[4] = {pack_h2(f0[0], f0[1]), pack_h2(fh[0], fh[1]), pack_h2(fr[0], fr[1]),
-                           pack_h2(fi[0], fi[1])};
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-      *reinterpret_cast<uint32_t*>(out + ((int64_t)p * KB + kb0 + g) * Np * 32 + inrow) = o[p];
+    o[0][k] = pack_h2(f0[0], f0[1]);
+    o[1][k] = pack_h2(fh[0], fh[1]);
+    o[2][k] = pack_h2(fr[0], fr[1]);
+    o[3][k] = pack_h2(fi[0], fi[1]);
   }
+  const int64_t inrow = n * 32 + ((h ^ (int)((n >> 2) & 1)) << 4);
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+    *reinterpret_cast<uint4*>(out + ((int64_t)p * KB + kb) * Np * 32 + inrow) =
+        make_uint4(o[p][0], o[p][1], o[p][2], o[p][3]);
 }
 
 // 4-D view of tiled planes: (64 halves of a 128-byte line, Np/4 lines of a
@@ -916,7 +914,7 @@ cudaError_t launch_group_dft_tiled(const void* X, int64_t N, int C, void* out, c
   if (N <= 0) return cudaSuccess;
   if (C % 16 != 0) return cudaErrorInvalidValue;
   const int64_t Np = tiled_rows(N);
-  const int64_t threads = Np / 4 * ((C / 16 + 3) / 4) * 32;
+  const int64_t threads = Np / 16 * (C / 16) * 32;
   return launch_dependent(group_dft_tiled_kernel, dim3((unsigned)((threads + 255) / 256)),
                           dim3(256), 0, st, static_cast<const uint4*>(X), N, Np, C,
                           static_cast<uint8_t*>(out));

@@ -65,11 +65,24 @@
 // 16-channel blocks 1 KB apart (LBO), 8-row K groups 256 B apart (SBO), so the
 // N = 256 [Xr | Xi] operand again spans planes 2 and 3 at a uniform stride.
 // Channel counts need only be multiples of 16 (the box reads zeros past C).
+//
+// SM-pair variant (wgrad_pair_kernel, tiled planes only): a cluster of two CTAs
+// takes (256 out-channel, 128 in-channel) tiles with tcgen05 cta_group::2 MMAs,
+// M = 256 out-channels (each CTA its own 128 of dY's planes) and N = 128
+// in-channels (each CTA holds 64 of X's): per 32-row stage a CTA loads 48 KB
+// instead of 64 KB for the same MMA work, which is what bounds this kernel (the
+// SMs' L2 ports).  Each CTA writes the partial slot of its own 128 x 128 block;
+// the finalize is shared.  Six N = 128 products per K step on two issuing
+// threads of the leader (the [Xr | Xi] operand of the one-CTA kernel would put
+// Xr and Xi in different CTAs).  The dbias warps of both CTAs read dY's plane 0
+// from their own shared memory once the stage's MMAs have completed (a commit
+// multicast to both CTAs) and release the slot with the MMAs.
 
 #include <algorithm>
 
 #include "eql_kernels.h"
 #include "eql_tc_common.cuh"
+#include "eql_tc_pair_common.cuh"
 
 namespace eql {
 namespace {
@@ -546,16 +559,244 @@ __device__ __forceinline__ void store_one(float* p, float v) { *p = v; }
 // entry per thread: lanes read the partials along d, the results pass through
 // shared memory, and groups of 8 lanes write dW along c (each entry 4
 // contiguous values), so both sides are coalesced.
+// ---------------------------------------------------------------------------
+// SM-pair weight gradient from tiled planes
+// ---------------------------------------------------------------------------
+constexpr int WP_ST = 4;                          // ring depth
+constexpr uint32_t WP_GPLANE = 8 * 1024;          // dY: 8 blocks of 16 out-channels x 32 rows
+constexpr uint32_t WP_XPLANE = 4 * 1024;          // X: this CTA's 4 blocks of 16 in-channels
+constexpr uint32_t WP_G = 4 * WP_GPLANE;          // 32 KB
+constexpr uint32_t WP_STAGE = WP_G + 4 * WP_XPLANE;  // 48 KB
+constexpr uint32_t WP_OFF_BAR = WP_ST * WP_STAGE;
+constexpr uint32_t WP_SMEM = WP_OFF_BAR + 512 + 1024;
+constexpr int WP_THREADS = 512;
+constexpr int WP_EPI0 = 4, WP_EPIW = 8;           // warps 4..11 drain the accumulators
+constexpr int WP_BIAS0 = 12, WP_BIASW = 4;        // warps 12..15 sum dbias
+static_assert(WP_SMEM <= 232448, "shared memory budget");
+static_assert(WP_STAGE % 1024 == 0, "stage slots stay 1024-byte aligned");
+
+struct WpBars {
+  uint64_t full[WP_ST];   // leader: both CTAs' loads of the stage landed
+  uint64_t empty[WP_ST];  // each CTA: the stage's MMAs and its dbias warps are done with it
+  uint64_t done[WP_ST];   // each CTA: the stage's MMAs completed (its data is in place)
+  uint64_t acc_full, acc_empty, drain[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(WpBars) <= 512, "barrier block");
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WP_THREADS, 1)
+    wgrad_pair_kernel(const __grid_constant__ CUtensorMap map_g,
+                      const __grid_constant__ CUtensorMap map_x, int C, int D, WgInfo wi,
+                      float* __restrict__ part, float* __restrict__ bpart, int* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  WpBars* bars = reinterpret_cast<WpBars*>(smem + WP_OFF_BAR);
+  int* abort_flag = &bars->abort_flag;
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cta_rank();
+  const int unit = blockIdx.x >> 1;  // the cluster's stream-K range
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < WP_ST; ++s) {
+      mbar_init(&bars->full[s], 1);              // the leader's producer (both CTAs' bytes)
+      mbar_init(&bars->empty[s], 2 + WP_BIASW);  // both issuers' commits + the dbias warps
+      mbar_init(&bars->done[s], 2);              // both issuers' commits
+    }
+    mbar_init(&bars->acc_full, 2);
+    mbar_init(&bars->acc_empty, 2 * WP_EPIW);  // one arrival per epilogue warp of each CTA
+    mbar_init(&bars->drain[0], 1);
+    mbar_init(&bars->drain[1], 1);
+    bars->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&bars->tmem_base)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive or TMA completion
+  tc_fence_after();
+  grid_dependency_wait();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- producer (both CTAs): own 128 out-channels of dY, own 64 in-channels of X
+    if (lane == 0) {
+      int issued_phase[WP_ST];
+      for (int s = 0; s < WP_ST; ++s) issued_phase[s] = -1;
+      uint32_t it = 0;
+      bool ok = true;
+      SegIter si(wi, unit);
+      Unit un;
+      while (ok && si.next(wi, un)) {
+        for (int s = 0; s < un.stages; ++s, ++it) {
+          const int slot = it % WP_ST;
+          const uint32_t ph = (it / WP_ST) & 1;
+          if (!(ok = wait_bounded(&bars->empty[slot], ph ^ 1, abort_flag, status))) break;
+          const uint32_t full_leader = peer_addr(smem_u32(&bars->full[slot]), 0);
+          if (rank == 0) mbar_expect_tx(&bars->full[slot], 2 * WP_STAGE);
+          const int line = (int)((un.r0 + (int64_t)WG_BR * s) / 4);
+          const uint32_t dst = sbase + slot * WP_STAGE;
+          // (128-byte line = 4 rows, line, 16-channel block, plane)
+          tma_load_4d_pair(dst, &map_g, full_leader, 0, line, 16 * un.dt + 8 * (int)rank, 0);
+          tma_load_4d_pair(dst + WP_G, &map_x, full_leader, 0, line, 8 * un.ct + 4 * (int)rank, 0);
+          issued_phase[slot] = (int)ph;
+        }
+      }
+      if (!ok && rank == 0)
+        for (int s = 0; s < WP_ST; ++s)
+          if (issued_phase[s] >= 0) drain_wait(&bars->full[s], (uint32_t)issued_phase[s]);
+    }
+    __syncwarp();
+  } else if (warp == 1 || warp == 3) {
+    // ---------------- MMA issuers (leader): Q0 and Qr on warp 1, Q2 and Qi on warp 3 ----------------
+    if (rank == 0 && lane == 0) {
+      const int who = warp == 1 ? 0 : 1;
+      const uint32_t id = idesc_f16_mn(256, WG_BC), id_neg = idesc_f16_mn(256, WG_BC, true);
+      uint32_t it = 0, ucount = 0;
+      bool ok = true;
+      SegIter si(wi, unit);
+      Unit un;
+      for (; ok && si.next(wi, un); ++ucount) {
+        if (!(ok = wait_bounded(&bars->acc_empty, (ucount & 1) ^ 1, abort_flag, status))) break;
+        tc_fence_after();
+        for (int s = 0; s < un.stages; ++s, ++it) {
+          const int slot = it % WP_ST;
+          if (!(ok = wait_bounded(&bars->full[slot], (it / WP_ST) & 1, abort_flag, status))) break;
+          tc_fence_after();
+          const uint32_t g = sbase + slot * WP_STAGE, x = g + WP_G;
+#pragma unroll
+          for (int kk = 0; kk < WG_BR / 16; ++kk) {
+            const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t a2 = desc_mn32(g + 2 * WP_GPLANE + 512u * kk);
+            const uint64_t a3 = desc_mn32(g + 3 * WP_GPLANE + 512u * kk);
+            const uint64_t b2 = desc_mn32(x + 2 * WP_XPLANE + 512u * kk);
+            const uint64_t b3 = desc_mn32(x + 3 * WP_XPLANE + 512u * kk);
+            if (who == 0) {
+              umma_pair(tmem + 0, desc_mn32(g + 512u * kk), desc_mn32(x + 512u * kk), id, acc);
+              umma_pair(tmem + 2 * WG_BC, a2, b2, id, acc);        // Qr += Gr Xr
+              umma_pair(tmem + 2 * WG_BC, a3, b3, id, 1u);         // Qr += Gi Xi
+            } else {
+              umma_pair(tmem + WG_BC, desc_mn32(g + WP_GPLANE + 512u * kk),
+                        desc_mn32(x + WP_XPLANE + 512u * kk), id, acc);  // Q2
+              umma_pair(tmem + 3 * WG_BC, a2, b3, id, acc);        // Qi += Gr Xi
+              umma_pair(tmem + 3 * WG_BC, a3, b2, id_neg, 1u);     // Qi -= Gi Xr
+            }
+          }
+          umma_commit_pair(&bars->done[slot], 3);
+          umma_commit_pair(&bars->empty[slot], 3);
+        }
+        if (ok) umma_commit_pair(&bars->acc_full, 3);
+      }
+      // every MMA this thread issued completes before TMEM is freed
+      umma_commit_pair(&bars->drain[who], 1);
+      drain_wait(&bars->drain[who], 0);
+    }
+    __syncwarp();
+  } else if (warp >= WP_EPI0 && warp < WP_EPI0 + WP_EPIW) {
+    // ---------------- epilogue (both CTAs): accumulators -> FP32 partial planes ----------------
+    // lane = out-channel 32q + lane of this CTA's 128; column j = in-channel 128 ct + j
+    const int q = warp & 3;
+    const int p0 = 2 * ((warp - WP_EPI0) >> 2);
+    const uint32_t acc_empty_leader = peer_addr(smem_u32(&bars->acc_empty), 0);
+    uint32_t ucount = 0;
+    SegIter si(wi, unit);
+    Unit un;
+    for (; si.next(wi, un); ++ucount) {
+      if (!warp_wait(&bars->acc_full, ucount & 1, abort_flag, status)) break;
+      tc_fence_after();
+      const int dl = 32 * q + lane;
+      const int d = (2 * un.dt + (int)rank) * WG_BD + dl;
+      const uint32_t lrow = tmem + ((uint32_t)(32 * q) << 16);
+      float* slot_base = part + ((int64_t)un.slot * 2 + rank) * (4 * WG_BC * WG_BD);
+#pragma unroll 1
+      for (int p = p0; p < p0 + 2; ++p) {
+        float* dst_plane = slot_base + p * (WG_BC * WG_BD);
+#pragma unroll 1
+        for (int gq = 0; gq < WG_BC / 16; gq += 2) {
+          const int c = un.ct * WG_BC + 16 * gq;
+          if (c >= C) break;  // warp-uniform; C % 16 == 0
+          const bool two = c + 16 < C;
+          uint32_t r[16], r2[16];
+          tmem_ld_32x32b<16>(lrow + p * WG_BC + 16 * gq, r);
+          if (two) tmem_ld_32x32b<16>(lrow + p * WG_BC + 16 * gq + 16, r2);
+          tmem_wait_ld();
+          if (d < D) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              dst_plane[(16 * gq + k) * WG_BD + dl] = __uint_as_float(r[k]);
+            if (two) {
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
+                dst_plane[(16 * gq + 16 + k) * WG_BD + dl] = __uint_as_float(r2[k]);
+            }
+          }
+        }
+      }
+      // TMEM goes back once every warp of both CTAs has read it (its loads have
+      // completed, so a relaxed arrive suffices)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_remote_relaxed(acc_empty_leader);
+    }
+  } else if (warp >= WP_BIAS0 && warp < WP_BIAS0 + WP_BIASW) {
+    // ---------------- dbias (both CTAs): sums of dY's plane 0, own 128 out-channels ----------------
+    // plane 0 sits at [block dl / 16][row][32 B], piece (dl % 16) / 8 swizzled with (row / 4) % 2
+    const int dl = (warp - WP_BIAS0) * 32 + lane;
+    uint32_t it = 0;
+    bool ok = true;
+    SegIter si(wi, unit);
+    Unit un;
+    while (ok && si.next(wi, un)) {
+      float b = 0.f;
+      for (int s = 0; s < un.stages; ++s, ++it) {
+        const int slot = it % WP_ST;
+        if (!(ok = warp_wait(&bars->done[slot], (it / WP_ST) & 1, abort_flag, status))) break;
+        if (un.ct == 0) {
+          const uint8_t* blk = smem + slot * WP_STAGE + (dl >> 4) * 1024;
+          const int piece = (dl & 15) >> 3, within = (dl & 7) * 2;
+#pragma unroll 8
+          for (int r = 0; r < WG_BR; ++r)
+            b += __half2float(*reinterpret_cast<const __half*>(
+                blk + r * 32 + ((piece ^ ((r >> 2) & 1)) << 4) + within));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->empty[slot]);
+      }
+      if (!ok) break;
+      // the planes hold G0/4: the sum times 4 (exact) is the sum of G0
+      if (un.ct == 0) bpart[((int64_t)un.slot * 2 + rank) * WG_BD + dl] = 4.f * b;
+    }
+  }
+
+  grid_launch_dependents();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its pair may still touch its shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
 constexpr int FZ_D = 32, FZ_C = 8;
 template <typename Out>
 __global__ void __launch_bounds__(256)
     wgrad_tc_finalize_kernel(const float* __restrict__ part, const float* __restrict__ bpart,
                              WgInfo wi, int C, int D, Out* __restrict__ dW,
-                             Out* __restrict__ dbias, Twiddles tw) {
+                             Out* __restrict__ dbias, Twiddles tw, int pairs) {
   __shared__ __align__(16) float s[FZ_C][FZ_D * 4 + 4];  // [c][d][u], rows padded by 16 B
   const int d0 = blockIdx.x * FZ_D, c0 = blockIdx.y * FZ_C;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;  // 8 warps
-  const int tile = (d0 / WG_BD) * wi.n_ct + c0 / WG_BC;
+  // pairs: a stream-K tile is 256 out-channels; its CTA `half` wrote this block
+  const int mult = pairs ? 2 : 1, half = pairs ? (d0 / WG_BD) & 1 : 0;
+  const int tile = (d0 / WG_BD / mult) * wi.n_ct + c0 / WG_BC;
   {
     const int d = d0 + lane, c = c0 + w;  // lane = out-channel, warp = in-channel
     if (d < D && c < C) {
@@ -565,7 +806,8 @@ __global__ void __launch_bounds__(256)
         const int pair = b * wi.n_dt * wi.n_ct + tile;
         const int n = last_range_of_pair(b, tile, wi) - first_range_of_pair(b, tile, wi);
         for (int j = 0; j <= n; ++j) {
-          const float* slot = part + ((int64_t)pair * wi.maxj + j) * (4 * WG_BC * WG_BD);
+          const float* slot =
+              part + (((int64_t)pair * wi.maxj + j) * mult + half) * (4 * WG_BC * WG_BD);
 #pragma unroll
           for (int p = 0; p < 4; ++p) qv[p] += slot[p * (WG_BC * WG_BD) + off];
         }
@@ -586,12 +828,13 @@ __global__ void __launch_bounds__(256)
   }
   if (dbias && blockIdx.y == 0 && w == 0 && d0 + lane < D) {
     const int d = d0 + lane;
-    const int tile0 = (d / WG_BD) * wi.n_ct;
+    const int tile0 = (d / WG_BD / mult) * wi.n_ct;
     float b = 0.f;
     for (int rb = 0; rb < wi.nb; ++rb) {
       const int pair = rb * wi.n_dt * wi.n_ct + tile0;
       const int n = last_range_of_pair(rb, tile0, wi) - first_range_of_pair(rb, tile0, wi);
-      for (int j = 0; j <= n; ++j) b += bpart[((int64_t)pair * wi.maxj + j) * WG_BD + d % WG_BD];
+      for (int j = 0; j <= n; ++j)
+        b += bpart[(((int64_t)pair * wi.maxj + j) * mult + half) * WG_BD + d % WG_BD];
     }
     store_one(dbias + d, b);
   }
@@ -631,14 +874,15 @@ bool encode_planes4_map(CUtensorMap* m, const void* base, int channels, int64_t 
 // Tiled planes (tiled_rows(N) rows per 16-channel block) viewed as (64 halves of
 // a 128-byte line, line, 16-channel block, plane); box = (64, 8 lines, 8 blocks,
 // 4 planes), no swizzle (the rows are stored swizzled).
-bool encode_tiled4_map(CUtensorMap* m, const void* base, int channels, int64_t N) {
+bool encode_tiled4_map(CUtensorMap* m, const void* base, int channels, int64_t N,
+                       uint32_t blocks = 8) {
   auto encode = encode_fn();
   if (!encode || channels % 16 != 0) return false;
   const int64_t Np = tiled_rows(N);
   const int kb = channels / 16;
   cuuint64_t dims[4] = {64, (cuuint64_t)(Np / 4), (cuuint64_t)kb, 4};
   cuuint64_t strides[3] = {128, (cuuint64_t)Np * 32, (cuuint64_t)Np * 32 * kb};
-  cuuint32_t box[4] = {64, PL_ROWS / 4, 8, 4};
+  cuuint32_t box[4] = {64, PL_ROWS / 4, blocks, 4};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides,
                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -648,9 +892,13 @@ bool encode_tiled4_map(CUtensorMap* m, const void* base, int channels, int64_t N
 
 // The stream-K layout for N rows: equal contiguous ranges of (tile, stage), one
 // per CTA, and the number of partial slots a tile can need.
-bool wgrad_tc_layout(int64_t N, int C, int D, int num_sms, WgInfo* wi, int* grid) {
+// pairs: tiles of 256 out-channels, one range per cluster of two SMs.
+bool wgrad_tc_layout(int64_t N, int C, int D, int num_sms, WgInfo* wi, int* grid,
+                     bool pairs = false) {
   if (N <= 0) return false;
-  wi->n_dt = (D + WG_BD - 1) / WG_BD;
+  if (pairs) num_sms /= 2;
+  if (num_sms < 1) return false;
+  wi->n_dt = (D + (pairs ? 2 : 1) * WG_BD - 1) / ((pairs ? 2 : 1) * WG_BD);
   wi->n_ct = (C + WG_BC - 1) / WG_BC;
   const int64_t spt = (N + WG_BR - 1) / WG_BR;
   if (spt > 0x3fffffffLL) return false;
@@ -688,12 +936,17 @@ bool wgrad_tc_supported(int T, DType dt, int64_t N, int C, int D, const void* X,
          ((reinterpret_cast<uintptr_t>(dY) & 15) == 0);
 }
 
+// Enough for the one-CTA layout and the SM-pair one (two 128 x 128 blocks per slot).
 size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms) {
-  WgInfo wi;
-  int grid = 0;
-  if (!wgrad_tc_layout(N, C, D, num_sms, &wi, &grid)) return 0;
-  const size_t slots = (size_t)wi.nb * wi.n_dt * wi.n_ct * wi.maxj;
-  return slots * ((size_t)4 * WG_BC * WG_BD + WG_BD) * sizeof(float);
+  size_t need = 0;
+  for (int pairs = 0; pairs < 2; ++pairs) {
+    WgInfo wi;
+    int grid = 0;
+    if (!wgrad_tc_layout(N, C, D, num_sms, &wi, &grid, pairs != 0)) continue;
+    const size_t slots = (size_t)wi.nb * wi.n_dt * wi.n_ct * wi.maxj * (pairs ? 2 : 1);
+    need = std::max(need, slots * ((size_t)4 * WG_BC * WG_BD + WG_BD) * sizeof(float));
+  }
+  return need;
 }
 
 bool wgrad_tc_planes_supported(int64_t N, int C, int D, const void* Xhat, const void* Ghat) {
@@ -705,12 +958,15 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
                             int num_sms, const Twiddles& tw, cudaStream_t st, int planes) {
   WgInfo wi;
   int grid = 0;
-  if (!wgrad_tc_layout(N, C, D, num_sms, &wi, &grid)) return cudaErrorInvalidValue;
   if (planes < 0 || planes > 2) return cudaErrorInvalidValue;
+  // tiled planes: SM pairs (the one-CTA tiled variant if the pair layout fails)
+  const bool pairs = planes == 2 && wgrad_tc_layout(N, C, D, num_sms, &wi, &grid, true);
+  if (!pairs && !wgrad_tc_layout(N, C, D, num_sms, &wi, &grid)) return cudaErrorInvalidValue;
   if (planes == 1 && (C % 64 != 0 || D % 64 != 0)) return cudaErrorNotSupported;
   CUtensorMap mg, mx;
   if (planes == 2) {
-    if (!encode_tiled4_map(&mg, dY, D, N) || !encode_tiled4_map(&mx, X, C, N))
+    if (!encode_tiled4_map(&mg, dY, D, N) ||
+        !encode_tiled4_map(&mx, X, C, N, pairs ? 4u : 8u))
       return cudaErrorInvalidValue;
   } else if (planes == 1) {
     if (!encode_planes4_map(&mg, dY, D, N) || !encode_planes4_map(&mx, X, C, N))
@@ -719,7 +975,8 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
     return cudaErrorInvalidValue;
   }
   float* part = static_cast<float*>(workspace);
-  float* bpart = part + (size_t)wi.nb * wi.n_dt * wi.n_ct * wi.maxj * (4 * WG_BC * WG_BD);
+  float* bpart =
+      part + (size_t)wi.nb * wi.n_dt * wi.n_ct * wi.maxj * (pairs ? 2 : 1) * (4 * WG_BC * WG_BD);
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(wgrad_tc_kernel<false>,
@@ -730,10 +987,17 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(wgrad_tc_kernel<true, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(wgrad_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               WP_SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  if (planes == 2)
+  if (pairs) {
+    cudaError_t e = launch_dependent(wgrad_pair_kernel, dim3(2 * grid), dim3(WP_THREADS), WP_SMEM,
+                                     st, mg, mx, C, D, wi, part, bpart, status);
+    if (e != cudaSuccess) return e;
+  } else if (planes == 2)
     wgrad_tc_kernel<true, true><<<grid, WG_THREADS_PL, WG_SMEM, st>>>(mg, mx, N, C, D, wi, part,
                                                                       bpart, status);
   else if (planes == 1)
@@ -747,10 +1011,12 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
   const dim3 fgrid((D + FZ_D - 1) / FZ_D, (C + FZ_C - 1) / FZ_C);
   if (out_dt == DType::F32)
     wgrad_tc_finalize_kernel<float><<<fgrid, 256, 0, st>>>(
-        part, bpart, wi, C, D, static_cast<float*>(dW), static_cast<float*>(dbias), tw);
+        part, bpart, wi, C, D, static_cast<float*>(dW), static_cast<float*>(dbias), tw,
+        pairs ? 1 : 0);
   else
     wgrad_tc_finalize_kernel<__half><<<fgrid, 256, 0, st>>>(
-        part, bpart, wi, C, D, static_cast<__half*>(dW), static_cast<__half*>(dbias), tw);
+        part, bpart, wi, C, D, static_cast<__half*>(dW), static_cast<__half*>(dbias), tw,
+        pairs ? 1 : 0);
   return cudaGetLastError();
 }
 
