@@ -87,6 +87,10 @@ TILED = {"p4_vitb_mlp_f16"}
 # pair kernel (eqlinear_forward_tiled): the FP32 layer with 3xTF32 split
 # precision, the cyclic T = 8 layer and the D4 layers with eight planes
 TILED_LAYERS = {"p4_vitb_proj_f32", "c8_1024_tiled_f16", "p4m_vitb_mlp_f16"}
+# of those, pipelines whose layers after the first take their input planes from
+# the previous layer's epilogue (eqlinear_forward_tiled_next): one group-DFT
+# launch per step
+TILED_NEXT = {"p4m_vitb_mlp_f16"}
 # per-layer output activation (fused into that layer's epilogue); default none
 ACTS = {"p4_vitb_mlp_block_f16": ["gelu", "none"]}
 
@@ -125,8 +129,9 @@ DESCR = {
                                 "spectral planes; one chained launch",
     "p4m_vitb_mlp_f16": "p4m (dihedral D4, 8 elements) EQ-Linear fp16 ViT-B MLP pair: N=12608, "
                         "C=96->D=384 then C=384->D=96 per group element (768->3072->768 "
-                        "features); per layer the group Fourier transform to eight tiled "
-                        "planes, then the products on SM pairs",
+                        "features); the group Fourier transform of X to eight tiled "
+                        "planes, fc1 on SM pairs writing fc2's planes from its epilogue, "
+                        "fc2 on SM pairs",
     "p4m_vitb_mlp_fused_f16": "p4m (dihedral D4, 8 elements) EQ-Linear fp16 ViT-B MLP pair: "
                               "N=12608, C=96->D=384 then C=384->D=96 per group element; one "
                               "launch of the fused one-CTA kernel per layer",
@@ -176,7 +181,7 @@ NCU_TRAFFIC = {
     ("conv", "d28bc5734eac2b53"): {"p4_conv3x3_f16": 161.54e6},
     ("forward_chain_tiled", "6ade53bcfcfaa10b"): {"p4_vitb_mlp_f16": 99.44e6},
     ("forward_pair", "6ade53bcfcfaa10b"): {"p4_vith_fc1_fwd_bwd_tiled_f16": 96.53e6},
-    ("forward_tiled", "00b0eabab3294aea"): {"p4_vitb_proj_f32": 85.78e6, "p4m_vitb_mlp_f16": 58.38e6, "c8_1024_tiled_f16": 34.38e6},
+    ("forward_tiled", "2fe2ac1739cebc38"): {"p4_vitb_proj_f32": 85.81e6, "p4m_vitb_mlp_f16": 59.08e6, "c8_1024_tiled_f16": 34.38e6},
 }
 
 def kernel_traffic(family: str, workload: str):
@@ -713,17 +718,25 @@ def run_ours(args, workload):
         tkern = "tcgen05-3xtf32" if dt == torch.float32 else "tcgen05"
         xts = [[torch.empty(plans[li].tiled_shape(N, w.C), dtype=dt, device="cuda")
                 for li, w in enumerate(pipeline)] for _ in range(nsets)]
+        chained_next = workload in TILED_NEXT
         for li, w in enumerate(pipeline):
             def dft_l(i, li=li):
                 x = xs[i % nsets] if li == 0 else outs[i % nsets][li - 1]
                 plans[li].group_dft(x, out=xts[i % nsets][li])
 
             def fwd_l(i, li=li):
-                plans[li].forward_tiled(xts[i % nsets][li], N, whats[li], biases[li],
-                                        act=acts[li], out=outs[i % nsets][li])
+                if chained_next and li + 1 < len(pipeline):
+                    # the next layer's input planes straight from this epilogue
+                    plans[li].forward_tiled_next(xts[i % nsets][li], N, whats[li], biases[li],
+                                                 act=acts[li], out=xts[i % nsets][li + 1])
+                else:
+                    plans[li].forward_tiled(xts[i % nsets][li], N, whats[li], biases[li],
+                                            act=acts[li], out=outs[i % nsets][li])
             # the transform reads the input and writes its planes; the products read
-            # the planes and the weight stages and write the output
-            ops.append(("group_dft", "simt", 0.0, (1 + pf) * es * N * w.C * w.T, dft_l))
+            # the planes and the weight stages and write the output (or the next
+            # layer's planes, the same bytes at T = 8)
+            if li == 0 or not chained_next:
+                ops.append(("group_dft", "simt", 0.0, (1 + pf) * es * N * w.C * w.T, dft_l))
             ops.append(("forward_tiled", tkern, layer_flops(w),
                         layer_bytes(w) + (pf - 1) * es * N * w.C * w.T, fwd_l))
     if tiled_train:

@@ -399,15 +399,16 @@ static eqlinear_status_t pair_io(eqlinear_plan_t p, const void* Xt, int64_t N, c
     return EQL_ERR_ALIGNMENT;
   const int Cin = adjoint ? p->D : p->C, Cout = adjoint ? p->C : p->D;
   if (p->T == 8) {
-    // eight-plane pair kernel; spatial output
-    if (!has_pair8_tiles(p) || p->kernel == EQL_KERNEL_SIMT || spectral_out ||
+    // eight-plane pair kernel; spatial output or the next layer's tiled planes
+    if (!has_pair8_tiles(p) || p->kernel == EQL_KERNEL_SIMT ||
         !eql::pair8_supported(N, Cin, Cout))
       return EQL_ERR_UNSUPPORTED;
     eqlinear_status_t s = check_plan_device(p);
     if (s != EQL_OK) return s;
     return from_cuda(eql::launch_pair8_tc(
         Xt, N, Cin, Cout, adjoint ? pair8_adj_tiles(p, W_hat) : pair8_fwd_tiles(p, W_hat), bias,
-        out, p->status, p->num_sms, (int)act, p->group, (cudaStream_t)stream));
+        out, p->status, p->num_sms, (int)act, p->group, (cudaStream_t)stream,
+        spectral_out ? 1 : 0));
   }
   if (p->dtype == EQL_F32) {
     // 3xTF32 on SM pairs; the output is spatial only

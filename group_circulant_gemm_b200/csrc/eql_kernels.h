@@ -160,9 +160,12 @@ cudaError_t launch_pair8_tile_weights(const void* planes, int Cin, int Cout, voi
                                       cudaStream_t st, int d4_adjoint = 0);
 cudaError_t launch_group_dft8_tiled(const void* X, int64_t N, int C, int group, void* out,
                                     cudaStream_t st);
+// next_planes = 1: Y is instead the tiled planes (tiled8_planes_bytes(N, Cout))
+// of act(Y) for the next layer, as launch_group_dft8_tiled of the spatial output
+// (Y rounded to FP16 first); rows N..Np-1 zero.
 cudaError_t launch_pair8_tc(const void* Xt, int64_t N, int Cin, int Cout, const void* tiles,
                             const void* bias, void* Y, int* status, int num_sms, int act,
-                            int group, cudaStream_t st);
+                            int group, cudaStream_t st, int next_planes = 0);
 
 // Rows of X [N][H][W][c4 halves] shifted by a convolution tap: out[(n*Ho + oy)*Wo + ox]
 // = X[n][oy+i-ph][ox+j-pw] (zero outside the image), c4 a multiple of 8.

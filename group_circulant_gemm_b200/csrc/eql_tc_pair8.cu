@@ -61,7 +61,9 @@ constexpr int P8_WLINES = P8_WBYTES / 128;
 constexpr int P8_ST = 4;
 constexpr int P8_THREADS = 384;
 constexpr int P8_EPI0 = 4;
-constexpr uint32_t P8_STG = 4096;                  // per epilogue warp: 32 rows x 128 B
+// per epilogue warp: 32 rows x 128 B of Y, or (next-layer planes) 8 planes x 32
+// rows x 32 B of one 16-channel block
+constexpr uint32_t P8_STG = 8192;
 constexpr uint32_t P8_OFF_STG = P8_ST * P8_STAGE;
 constexpr uint32_t P8_OFF_BIAS = P8_OFF_STG + kEpiWarps * P8_STG;
 constexpr uint32_t P8_OFF_BAR = P8_OFF_BIAS + kEpiWarps * 128;
@@ -116,9 +118,55 @@ struct P8Sched {
   int64_t N;
   int n_dt, n_ks, Cout, total;
   const __half* bias;
+  int64_t Np;     // rows of the tiled planes
 };
 
-template <int G, int ACT>
+// The group Fourier transform of one channel's eight elements x[t] (FP32), in
+// the plane order of the tiled layout (not yet times 1/8):
+//   G = 0, cyclic T = 8: V0, V4, Re V1, Im V1, Re V2, Im V2, Re V3, Im V3 of
+//   V[k] = sum_t x_t e^{-2 pi i k t / 8} (radix 2: a_t = x_t + x_{t+4},
+//   b_t = x_t - x_{t+4}, one twiddle sqrt(2)/2);
+//   G = 1, D4 (t = a + 4b for r^a m^b): the characters (chi(r), chi(m)) =
+//   (+,+), (+,-), (-,+), (-,-), then X[i][j] = sum_t x_t rho(t)_ij of
+//   r -> [[0,-1],[1,0]], m -> diag(1,-1), at 4 + 2i + j.
+template <int G>
+__device__ __forceinline__ void dft8(const float (&x)[8], float (&val)[8]) {
+  if constexpr (G == 1) {
+    const float e0 = x[0] + x[2], o0 = x[1] + x[3];
+    const float e1 = x[4] + x[6], o1 = x[5] + x[7];
+    const float d0 = x[0] - x[2], d1 = x[1] - x[3];
+    const float d4 = x[4] - x[6], d5 = x[5] - x[7];
+    val[0] = (e0 + o0) + (e1 + o1);
+    val[1] = (e0 + o0) - (e1 + o1);
+    val[2] = (e0 - o0) + (e1 - o1);
+    val[3] = (e0 - o0) - (e1 - o1);
+    val[4] = d0 + d4;
+    val[5] = d5 - d1;
+    val[6] = d1 + d5;
+    val[7] = d0 - d4;
+  } else {
+    const float h = 0.70710678118654752f;
+    const float a0 = x[0] + x[4], a1 = x[1] + x[5], a2 = x[2] + x[6], a3 = x[3] + x[7];
+    const float b0 = x[0] - x[4], b1 = x[1] - x[5], b2 = x[2] - x[6], b3 = x[3] - x[7];
+    // rounded products (never fused into the adds), so every caller forms the
+    // same values
+    const float s13 = __fmul_rn(h, b1 - b3), t13 = __fmul_rn(h, b1 + b3);
+    val[0] = (a0 + a2) + (a1 + a3);
+    val[1] = (a0 + a2) - (a1 + a3);
+    val[2] = b0 + s13;
+    val[3] = -b2 - t13;
+    val[4] = a0 - a2;
+    val[5] = a3 - a1;
+    val[6] = b0 - s13;
+    val[7] = b2 - t13;
+  }
+}
+
+// NEXT = 1: the output is written as the tiled planes of act(Y) (the next
+// layer's input): each value of Y is rounded to FP16 first and then transformed
+// with group_dft8_tiled_kernel's arithmetic (dft8), so the planes are those of
+// the spatial output passed through that kernel; rows N..Np-1 are zero.
+template <int G, int ACT, int NEXT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P8_THREADS, 1)
     eq_pair8_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                        const __grid_constant__ CUtensorMap map_w,
@@ -239,6 +287,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P8_THREADS, 1)
         uint4 oa[4], ob[4];
         epi_half<8, P8_BD, ACT, G>(lane_addr, 32 * ch + 8 * k, bsm + 8 * k, oa);
         epi_half<8, P8_BD, ACT, G>(lane_addr, 32 * ch + 8 * k + 4, bsm + 8 * k + 4, ob);
+        if constexpr (NEXT) {
+          // this lane's row: the 8 channels' Y (FP16) -> 8 planes x 8 channels,
+          // one 16-byte half row per plane, staged as the tiled layout's image
+          // ([plane][32 rows][32 B], halves swapped when (row / 4) % 2); the
+          // 16-channel block goes out as one TMA store after its second half
+          const int64_t n = row0 + lane;
+          {
+            uint32_t pl[8][4];
+#pragma unroll
+            for (int cp = 0; cp < 4; ++cp) {  // channel pair 2cp, 2cp + 1
+              float val[2][8];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int c = 2 * cp + e;
+                const uint4 y = c < 4 ? oa[c] : ob[c - 4];
+                const float2 y01 = unpack_h2(y.x), y23 = unpack_h2(y.y);
+                const float2 y45 = unpack_h2(y.z), y67 = unpack_h2(y.w);
+                const float x[8] = {y01.x, y01.y, y23.x, y23.y, y45.x, y45.y, y67.x, y67.y};
+                dft8<G>(x, val[e]);
+              }
+#pragma unroll
+              for (int p = 0; p < 8; ++p)
+                pl[p][cp] = n < sc.N ? pack_h2(val[0][p] * 0.125f, val[1][p] * 0.125f) : 0u;
+            }
+            const int half = k & 1;  // d0 % 16 / 8: dbase is a multiple of 16
+            if (half == 0) {
+              if (lane == 0) bulk_wait_read_all();  // the previous store has read the staging
+              __syncwarp();
+            }
+            uint8_t* rowp = stg + lane * 32 + ((half ^ ((lane >> 2) & 1)) << 4);
+#pragma unroll
+            for (int p = 0; p < 8; ++p)
+              *reinterpret_cast<uint4*>(rowp + p * 1024) =
+                  make_uint4(pl[p][0], pl[p][1], pl[p][2], pl[p][3]);
+            if (half == 1) {
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              __syncwarp();
+              // rows past Np fall outside the map and are not written
+              if (lane == 0 && row0 < sc.Np) {
+                tma_store_4d(&map_y, stg_s, 0, (int)(row0 / 4), d0 / 16, 0);
+                bulk_commit();
+              }
+            }
+          }
+          continue;
+        }
         if (lane == 0) bulk_wait_read_all();  // the previous store has read the staging
         __syncwarp();
         uint8_t* rowp = stg + lane * 128;
@@ -310,46 +404,21 @@ __global__ void group_dft8_tiled_kernel(const uint4* __restrict__ X, int64_t N, 
     }
   }
   const int64_t inrow = n * 32 + (((piece >> 2) ^ (int)((n >> 2) & 1)) << 4) + (piece & 3) * 4;
-  const float h = 0.70710678118654752f;
 #pragma unroll
   for (int g = 0; g < GB; ++g) {
     if (kb0 + g >= KB) break;
-    float val[8][2];
+    float val[2][8];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const float2 p01 = unpack_h2(v[g][e].x), p23 = unpack_h2(v[g][e].y);
       const float2 p45 = unpack_h2(v[g][e].z), p67 = unpack_h2(v[g][e].w);
-      if constexpr (G == 1) {
-        const float e0 = p01.x + p23.x, o0 = p01.y + p23.y;
-        const float e1 = p45.x + p67.x, o1 = p45.y + p67.y;
-        const float d0 = p01.x - p23.x, d1 = p01.y - p23.y;
-        const float d4 = p45.x - p67.x, d5 = p45.y - p67.y;
-        val[0][e] = (e0 + o0) + (e1 + o1);
-        val[1][e] = (e0 + o0) - (e1 + o1);
-        val[2][e] = (e0 - o0) + (e1 - o1);
-        val[3][e] = (e0 - o0) - (e1 - o1);
-        val[4][e] = d0 + d4;
-        val[5][e] = d5 - d1;
-        val[6][e] = d1 + d5;
-        val[7][e] = d0 - d4;
-      } else {
-        const float a0 = p01.x + p45.x, a1 = p01.y + p45.y, a2 = p23.x + p67.x, a3 = p23.y + p67.y;
-        const float b0 = p01.x - p45.x, b1 = p01.y - p45.y, b2 = p23.x - p67.x, b3 = p23.y - p67.y;
-        const float s13 = h * (b1 - b3), t13 = h * (b1 + b3);
-        val[0][e] = (a0 + a2) + (a1 + a3);
-        val[1][e] = (a0 + a2) - (a1 + a3);
-        val[2][e] = b0 + s13;
-        val[3][e] = -b2 - t13;
-        val[4][e] = a0 - a2;
-        val[5][e] = a3 - a1;
-        val[6][e] = b0 - s13;
-        val[7][e] = b2 - t13;
-      }
+      const float x[8] = {p01.x, p01.y, p23.x, p23.y, p45.x, p45.y, p67.x, p67.y};
+      dft8<G>(x, val[e]);
     }
 #pragma unroll
     for (int p = 0; p < 8; ++p)
       *reinterpret_cast<uint32_t*>(out + ((int64_t)p * KB + kb0 + g) * Np * 32 + inrow) =
-          pack_h2(val[p][0] * 0.125f, val[p][1] * 0.125f);
+          pack_h2(val[0][p] * 0.125f, val[1][p] * 0.125f);
   }
 }
 
@@ -392,9 +461,9 @@ __global__ void pair8_tile_weights_kernel(const __half* __restrict__ planes, int
   tiles[dst >> 4] = v;
 }
 
-template <int G, int ACT>
+template <int G, int ACT, int NEXT>
 cudaError_t set_p8_attr() {
-  return cudaFuncSetAttribute(eq_pair8_tc_kernel<G, ACT>,
+  return cudaFuncSetAttribute(eq_pair8_tc_kernel<G, ACT, NEXT>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, P8_SMEM);
 }
 
@@ -454,7 +523,7 @@ cudaError_t launch_group_dft8_tiled(const void* X, int64_t N, int C, int group, 
 
 cudaError_t launch_pair8_tc(const void* Xt, int64_t N, int Cin, int Cout, const void* tiles,
                             const void* bias, void* Y, int* status, int num_sms, int act,
-                            int group, cudaStream_t st) {
+                            int group, cudaStream_t st, int next_planes) {
   if (!pair8_supported(N, Cin, Cout) || !tiles) return cudaErrorNotSupported;
   if (act != 0 && act != 1) return cudaErrorInvalidValue;
   auto encode = encode_fn();
@@ -483,7 +552,7 @@ cudaError_t launch_pair8_tc(const void* Xt, int64_t N, int Cin, int Cout, const 
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  {
+  if (!next_planes) {
     // Y [N][Cout*8]: (64 halves = 8 channels, Cout/8 chunks, N rows); box = 32 rows
     cuuint64_t dims[3] = {64, (cuuint64_t)(Cout / 8), (cuuint64_t)N};
     cuuint64_t strides[2] = {128, (cuuint64_t)Cout * 8 * 2};
@@ -493,13 +562,28 @@ cudaError_t launch_pair8_tc(const void* Xt, int64_t N, int Cin, int Cout, const 
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
+  } else {
+    // the next layer's tiled planes: (64 halves of a 128-byte line, Np/4 lines,
+    // Cout/16 blocks, 8 planes); box = 8 lines (32 rows) x 1 block x 8 planes
+    cuuint64_t dims[4] = {64, (cuuint64_t)(Np / 4), (cuuint64_t)(Cout / 16), 8};
+    cuuint64_t strides[3] = {128, (cuuint64_t)Np * 32, (cuuint64_t)Np * 32 * (Cout / 16)};
+    cuuint32_t box[4] = {64, 8, 1, 8};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (encode(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, Y, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
   }
   static bool attrs = false;
   if (!attrs) {
-    cudaError_t e = set_p8_attr<0, 0>();
-    if (e == cudaSuccess) e = set_p8_attr<0, 1>();
-    if (e == cudaSuccess) e = set_p8_attr<1, 0>();
-    if (e == cudaSuccess) e = set_p8_attr<1, 1>();
+    cudaError_t e = set_p8_attr<0, 0, 0>();
+    if (e == cudaSuccess) e = set_p8_attr<0, 1, 0>();
+    if (e == cudaSuccess) e = set_p8_attr<1, 0, 0>();
+    if (e == cudaSuccess) e = set_p8_attr<1, 1, 0>();
+    if (e == cudaSuccess) e = set_p8_attr<0, 0, 1>();
+    if (e == cudaSuccess) e = set_p8_attr<0, 1, 1>();
+    if (e == cudaSuccess) e = set_p8_attr<1, 0, 1>();
+    if (e == cudaSuccess) e = set_p8_attr<1, 1, 1>();
     if (e != cudaSuccess) return e;
     attrs = true;
   }
@@ -512,8 +596,14 @@ cudaError_t launch_pair8_tc(const void* Xt, int64_t N, int Cin, int Cout, const 
   if ((int64_t)n_prow * sc.n_dt > 0x7fffffffLL) return cudaErrorInvalidValue;
   sc.total = n_prow * sc.n_dt;
   sc.bias = static_cast<const __half*>(bias);
-  auto kernel = group ? (act ? eq_pair8_tc_kernel<1, 1> : eq_pair8_tc_kernel<1, 0>)
-                      : (act ? eq_pair8_tc_kernel<0, 1> : eq_pair8_tc_kernel<0, 0>);
+  sc.Np = Np;
+  using K = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, P8Sched, int*);
+  const K table[2][2][2] = {
+      {{eq_pair8_tc_kernel<0, 0, 0>, eq_pair8_tc_kernel<0, 0, 1>},
+       {eq_pair8_tc_kernel<0, 1, 0>, eq_pair8_tc_kernel<0, 1, 1>}},
+      {{eq_pair8_tc_kernel<1, 0, 0>, eq_pair8_tc_kernel<1, 0, 1>},
+       {eq_pair8_tc_kernel<1, 1, 0>, eq_pair8_tc_kernel<1, 1, 1>}}};
+  const K kernel = table[group ? 1 : 0][act ? 1 : 0][next_planes ? 1 : 0];
   int npairs = p8_capacity((const void*)kernel, num_sms);
   if (npairs > sc.total) npairs = sc.total;
   return launch_dependent(kernel, dim3(2 * npairs), dim3(P8_THREADS), P8_SMEM, st, mx, mw, my, sc,

@@ -268,7 +268,10 @@ EQL_API eqlinear_status_t eqlinear_forward_from_spectral(eqlinear_plan_t plan, c
  *     (+,-), (-,+), (-,-), then the 2 x 2 representation's entries
  *     X[i][j] = sum_g x_g rho(g)_ij at plane 4 + 2i + j, with rho(r) =
  *     [[0,-1],[1,0]] and rho(m) = diag(1,-1). The same tiled layout with p < 8;
- *     tiled_spectrum_bytes = 8 * Np * c * 2. No _next form.
+ *     tiled_spectrum_bytes = 8 * Np * c * 2. The _next form writes the planes of
+ *     act(Y) rounded to FP16, as eqlinear_group_dft of eqlinear_forward_tiled's
+ *     output (bitwise for D4; cyclic: up to one rounding of Y where the
+ *     sqrt(2)/2 twiddle products round differently), with rows N..Np-1 zero.
  *   - p4 FP32, C and D multiples of 8 (3xTF32 on the tensor cores). Eight
  *     planes: the TF32 values hi = tf32(v) of X0, X2, Xr, Xi, then the
  *     residuals lo = tf32(v - hi). 8 FP32 channels per 32-byte row: element

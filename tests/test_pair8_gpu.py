@@ -17,6 +17,13 @@ max|ref|):
   * the T = 8 workload (16384 x 128 -> 128) and the D4 ViT-B MLP layers at full
     size, on sampled rows;
   * agreement with the fused one-CTA kernels;
+  * eqlinear_forward_tiled_next (the next layer's planes from the epilogue)
+    equals eqlinear_group_dft of eqlinear_forward_tiled's output, padding rows
+    zero: bitwise for D4 (its inverse transform is adds only); for the cyclic
+    group the compiler may fuse the sqrt(2)/2 twiddle products of the inverse
+    into the following adds differently in the two kernels, so a value of Y
+    can differ by one FP16 rounding; and the D4 MLP pair chained that way
+    matches the oracle;
   * requests the path does not take are rejected (D4 dX in this form is checked
     in test_d4_backward_gpu.py).
 """
@@ -149,14 +156,67 @@ def test_eight_plane_tiled_rejects_what_it_does_not_take():
     Xt = torch.zeros(p.tiled_shape(4, 16), dtype=torch.float16, device="cuda")
     X = torch.zeros(4, 128, dtype=torch.float16, device="cuda")
     assert n.eqlinear_tiled_spectrum_bytes(p.handle, 4, 16) == 8 * 128 * 16 * 2
-    # no next-layer planes for D4 either
+    # a plan forced to the CUDA cores has no tiled form
+    p.set_kernel("simt")
     assert n.raw_status("eqlinear_forward_tiled_next", p.handle, Xt.data_ptr(), 4,
                         Wh.data_ptr(), None, 0, Xt.data_ptr(), None) == n.EQL_ERR_UNSUPPORTED
+    p.set_kernel("auto")
     # channels that are not the plan's C or D
     assert n.raw_status("eqlinear_group_dft", p.handle, X.data_ptr(), 4, 32, Xt.data_ptr(),
                         None) == n.EQL_ERR_INVALID_ARG
-    # the next layer's planes: p4 only
-    c = _plan(16, 16)
-    Wc = c.prepare_weights(torch.zeros(16, 16, 8, dtype=torch.float16, device="cuda"))
-    assert n.raw_status("eqlinear_forward_tiled_next", c.handle, Xt.data_ptr(), 4,
-                        Wc.data_ptr(), None, 0, Xt.data_ptr(), None) == n.EQL_ERR_UNSUPPORTED
+    # misaligned output planes
+    bad = torch.zeros(8 * 128 * 16 + 8, dtype=torch.float16, device="cuda")[1:]
+    assert n.raw_status("eqlinear_forward_tiled_next", p.handle, Xt.data_ptr(), 4,
+                        Wh.data_ptr(), None, 0, bad.data_ptr(), None) == n.EQL_ERR_ALIGNMENT
+
+
+NEXT_CASES = [
+    # N, C, D, group, act
+    (333, 32, 64, "dihedral4", "none"),
+    (257, 48, 80, "cyclic", "gelu"),
+    (1000, 96, 384, "dihedral4", "gelu"),
+    (129, 16, 16, "cyclic", "none"),
+]
+
+
+@pytest.mark.parametrize("N,C,D,group,act", NEXT_CASES)
+def test_next_layer_planes_are_the_group_dft_of_the_output(N, C, D, group, act):
+    w = Workload("n8", 8, N, C, D, "f16", True, 8500 + N + C)
+    inp = make_inputs(w)
+    p = _plan(C, D, group)
+    Wh = p.prepare_weights(_dev(inp["W"]))
+    b = _dev(inp["bias"])
+    Xt = p.group_dft(_dev(inp["X"]))
+    Y = p.forward_tiled(Xt, N, Wh, b, act=act)
+    nxt = _plan(D, 16, group)  # a plan whose input width is D
+    ref = nxt.group_dft(Y)
+    got = torch.full(p.tiled_shape(N, D), float("nan"), dtype=torch.float16, device="cuda")
+    p.forward_tiled_next(Xt, N, Wh, b, act=act, out=got)
+    assert p.status() == 0 and nxt.status() == 0
+    if group == "dihedral4":
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    else:
+        g, r = got.double().cpu().numpy(), ref.double().cpu().numpy()
+        assert np.all(np.isfinite(g))
+        # one FP16 rounding of a Y value (2^-10 of |Y|) moves a plane (a signed
+        # mean of the eight) by at most that much, plus the plane's own rounding
+        assert np.max(np.abs(g - r)) <= 2.0 ** -9 * float(Y.abs().max())
+        Np = g.shape[2]
+        assert np.all(g[:, :, N:Np, :] == 0.0)
+
+
+def test_d4_mlp_pair_through_next_layer_planes_matches_the_oracle():
+    """The p4m ViT-B MLP pair (C = 96 -> 384 -> 96 per group element) with the
+    intermediate kept as tiled planes, on sampled rows of the full N = 12608."""
+    w1, w2 = WORKLOADS["p4m_vitb_fc1_f16"], WORKLOADS["p4m_vitb_fc2_f16"]
+    inp1, inp2 = make_inputs(w1), make_inputs(w2)
+    p1, p2 = _plan(w1.C, w1.D, "dihedral4"), _plan(w2.C, w2.D, "dihedral4")
+    W1, W2 = p1.prepare_weights(_dev(inp1["W"])), p2.prepare_weights(_dev(inp2["W"]))
+    b1, b2 = _dev(inp1["bias"]), _dev(inp2["bias"])
+    Ht = p1.forward_tiled_next(p1.group_dft(_dev(inp1["X"])), w1.N, W1, b1)
+    Y = p2.forward_tiled(Ht, w1.N, W2, b2)
+    assert p1.status() == 0 and p2.status() == 0
+    rows = _sampled(w1.N, 83)
+    H = oracle.d4_forward(inp1["X"][rows], inp1["W"], inp1["bias"])
+    ref = oracle.d4_forward(H.astype(np.float16), inp2["W"], inp2["bias"])
+    assert _rel(Y.double().cpu().numpy()[rows], ref) <= TOL16
