@@ -98,7 +98,8 @@ extern "C" eqlinear_status_t eqlinear_backward_weight_noalloc(eqlinear_plan_t p,
                                                               void* stream) {
   EQL_TRACE();
   if (!p || N < 0 || !dW) return EQL_ERR_INVALID_ARG;
-  if (p->group == 1) return EQL_ERR_UNSUPPORTED;  // the D4 layer has no backward
+  // the D4 weight gradient has its own kernel (eqlinear_backward_weight)
+  if (p->group == 1) return EQL_ERR_UNSUPPORTED;
   // this call always runs the CUDA-core kernels; a plan forced to the tensor
   // cores asked for something it cannot give
   if (p->kernel == EQL_KERNEL_TCGEN05) return EQL_ERR_UNSUPPORTED;
