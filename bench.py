@@ -178,7 +178,7 @@ KERNEL_SOURCES = {
 NCU_TRAFFIC = {
     ("forward", "443ba94f5b306a59"): {"p4_vitb_mlp_2calls_f16": 58.96e6, "c8_1024_f16": 34.20e6, "p4_vith_fc1_f16": 51.20e6, "p4_vith_fc1_fwd_bwd_f16": 109.13e6, "p4m_vitb_mlp_fused_f16": 57.79e6},
     ("forward_chain", "246b0f491b3357c1"): {"p4_vitb_mlp_fused_f16": 89.59e6, "p4_vitb_mlp_spectral_f16": 80.93e6, "p4_vitb_mlp_block_f16": 81.74e6},
-    ("conv", "d28bc5734eac2b53"): {"p4_conv3x3_f16": 161.54e6},
+    ("conv", "70beebb2fc455f9a"): {"p4_conv3x3_f16": 161.54e6},
     ("forward_chain_tiled", "6ade53bcfcfaa10b"): {"p4_vitb_mlp_f16": 99.44e6},
     ("forward_pair", "6ade53bcfcfaa10b"): {"p4_vith_fc1_fwd_bwd_tiled_f16": 96.53e6},
     ("forward_tiled", "2fe2ac1739cebc38"): {"p4_vitb_proj_f32": 85.81e6, "p4m_vitb_mlp_f16": 59.08e6, "c8_1024_tiled_f16": 34.38e6},
@@ -1092,11 +1092,15 @@ CONV_DESCR = {
     "p4_conv3x3_f16": "p4 group-circulant convolution fp16: 64 images 56x56, C=64->D=64 per "
                       "group element (256 -> 256 features), 3x3 taps, stride 1, zero padding 1, "
                       "T=4",
+    "p4_conv3x3_fwd_bwd_f16": "p4 group-circulant convolution fp16 training step (forward, dX, "
+                              "dWc + dbias): 64 images 56x56, C=64->D=64 per group element, "
+                              "3x3 taps, stride 1, zero padding 1, T=4",
 }
 
 
 def conv_flops(w) -> float:
-    """Algorithmic FLOPs: the layer's 12*C*D per output pixel and tap (6 real GEMMs)."""
+    """Algorithmic FLOPs of one pass (forward, dX or dWc): the layer's 12*C*D per
+    output pixel and tap (6 real GEMMs)."""
     return 12.0 * w.N * w.Ho * w.Wo * w.C * w.D * w.KH * w.KW
 
 
@@ -1107,9 +1111,12 @@ def conv_dense_flops(w) -> float:
 def conv_oracle_sample(w, images: int):
     import oracle
     oracle.build()
-    inp = make_conv_inputs(w, images=images)
+    inp = make_conv_inputs(w, images=images, need_dy=w.backward)
     t0 = time.perf_counter()
     oracle.conv_forward(w.T, inp["X"], inp["Wc"], inp["bias"], pad=(w.ph, w.pw))
+    if w.backward:
+        oracle.conv_backward_input(w.T, inp["dY"], inp["Wc"], w.H, w.W, pad=(w.ph, w.pw))
+        oracle.conv_backward_weight(w.T, inp["X"], inp["dY"], w.KH, w.KW, pad=(w.ph, w.pw))
     return time.perf_counter() - t0
 
 
@@ -1165,7 +1172,8 @@ def run_conv(args, workload):
     from group_circulant_gemm_b200 import EqLinearPlan
 
     w = CONV_WORKLOADS[workload]
-    inp = make_conv_inputs(w.with_(seed=w.seed + 1000 * rank))
+    bwd = w.backward
+    inp = make_conv_inputs(w.with_(seed=w.seed + 1000 * rank), need_dy=bwd)
     p = EqLinearPlan(w.T, w.C, w.D, torch.float16)
     Wc = torch.from_numpy(inp["Wc"]).cuda()
     Wh = p.conv_prepare_weights(Wc)
@@ -1173,6 +1181,8 @@ def run_conv(args, workload):
     x_host = inp["X"]
     pixels = w.N * w.Ho * w.Wo
     per_set = x_host.nbytes + pixels * w.D * w.T * 2
+    if bwd:
+        per_set += inp["dY"].nbytes + x_host.nbytes  # dY in, dX out
     nsets = max(2, int(np.ceil(2 * L2_BYTES / per_set)))
     xs = [torch.from_numpy(x_host).cuda() for _ in range(nsets)]
     ys = [torch.empty((w.N, w.Ho, w.Wo, w.D * w.T), dtype=torch.float16, device="cuda")
@@ -1182,13 +1192,39 @@ def run_conv(args, workload):
                      dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step(i, events=None, external=False):
-        if events is not None:
-            events.append(new_event(external))
+    def fwd(i):
         p.conv_forward(xs[i % nsets], Wh, w.KH, w.KW, bias, pad=(w.ph, w.pw),
                        out=ys[i % nsets], workspace=ws)
-        if events is not None:
-            events.append(new_event(external))
+    # (label, kernel family, FLOPs, launches, callable)
+    ops = [("conv_forward", "conv", conv_flops(w), 2, fwd)]
+    if bwd:
+        dys = [torch.from_numpy(inp["dY"]).cuda() for _ in range(nsets)]
+        dxs = [torch.empty_like(xs[0]) for _ in range(nsets)]
+        gW = torch.empty((w.KH, w.KW, w.D, w.C, w.T), dtype=torch.float16, device="cuda")
+        gb = torch.empty((w.D,), dtype=torch.float16, device="cuda")
+        wsb = torch.empty(native.eqlinear_conv_backward_workspace_bytes(
+            p.handle, w.N, w.H, w.W, w.KH, w.KW, w.ph, w.pw), dtype=torch.uint8, device="cuda")
+
+        def bwd_x(i):
+            p.conv_backward_input(dys[i % nsets], Wh, w.KH, w.KW, w.H, w.W, pad=(w.ph, w.pw),
+                                  out=dxs[i % nsets], workspace=wsb)
+
+        def bwd_w(i):
+            p.conv_backward_weight(xs[i % nsets], dys[i % nsets], w.KH, w.KW, pad=(w.ph, w.pw),
+                                   workspace=wsb, dW=gW, dbias=gb)
+        # dX: the planes pre-pass of dY and the tap-loop kernel; dWc: X and dY onto
+        # the padded grid, then per tap the layer's weight gradient and its finalize
+        ops += [("conv_backward_input", "conv", conv_flops(w), 2, bwd_x),
+                ("conv_backward_weight", "conv_wgrad", conv_flops(w), 2 + 2 * w.KH * w.KW,
+                 bwd_w)]
+
+    def step(i, events=None, external=False):
+        for _, _, _, _, fn in ops:
+            if events is not None:
+                events.append(new_event(external))
+            fn(i)
+            if events is not None:
+                events.append(new_event(external))
 
     clocks = ClockSampler(local)
     if rank == 0:
@@ -1231,8 +1267,9 @@ def run_conv(args, workload):
             torch.cuda.synchronize()
     in_graph = per_call is not None
     if per_call is None:
-        per_call = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(len(ev) // 2)])
-    launch_ms = float(np.mean(per_call))
+        per_call = np.array([ev[2 * j].elapsed_time(ev[2 * j + 1])
+                             for j in range(len(ev) // 2)]).reshape(-1, len(ops))
+    op_ms = per_call.mean(axis=0)
     timing = ("CUDA graph replay of each step (one graph per rotating set); per-call time "
               + (f"from {op_steps} replays of the step's graphs with event nodes around the "
                  "call" if in_graph else f"from {op_steps} eager steps with events around each call")
@@ -1240,6 +1277,13 @@ def run_conv(args, workload):
 
     x_pin = torch.from_numpy(x_host).pin_memory()
     y_pin = torch.empty(tuple(ys[0].shape), dtype=torch.float16).pin_memory()
+    h2d, d2h = x_pin.numel() * 2, y_pin.numel() * 2
+    if bwd:
+        dy_pin = torch.from_numpy(inp["dY"]).pin_memory()
+        dx_pin = torch.empty(tuple(dxs[0].shape), dtype=torch.float16).pin_memory()
+        dw_pin = torch.empty(tuple(gW.shape), dtype=torch.float16).pin_memory()
+        h2d += dy_pin.numel() * 2
+        d2h += (dx_pin.numel() + dw_pin.numel()) * 2
 
     # copies overlap the neighbouring steps' calls, as in the layer workloads
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
@@ -1253,6 +1297,8 @@ def run_conv(args, workload):
             if k >= 2:
                 s_in.wait_event(ev_c[j])
             xs[j].copy_(x_pin, non_blocking=True)
+            if bwd:
+                dys[j].copy_(dy_pin, non_blocking=True)
             ev_in[j].record(s_in)
         stream.wait_event(ev_in[j])
         if k >= 2:
@@ -1262,6 +1308,9 @@ def run_conv(args, workload):
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_c[j])
             y_pin.copy_(ys[j], non_blocking=True)
+            if bwd:
+                dx_pin.copy_(dxs[j], non_blocking=True)
+                dw_pin.copy_(gW, non_blocking=True)
             ev_out[j].record(s_out)
     for k in range(2):
         e2e_step(k)
@@ -1284,18 +1333,30 @@ def run_conv(args, workload):
 
     if rank == 0:
         peaks, peak_src = load_peaks()
-        flops = conv_flops(w)
+        flops = sum(f for _, _, f, _, _ in ops)
         value = world * pixels * args.steps / (elapsed_ms / 1e3)
-        achieved = flops / (launch_ms / 1e3) / 1e12
+        # dominant kernel family: the forward and dX run the same convolution kernel
+        fam = {}
+        for j, (_, fk, f, _, _) in enumerate(ops):
+            a = fam.setdefault(fk, [0.0, 0.0, 0])
+            a[0] += op_ms[j]
+            a[1] += f
+            a[2] += 1
+        dfam, (fam_ms, dflops, dcount) = max(fam.items(), key=lambda kv: kv[1][0])
+        launch_ms = fam_ms / dcount
+        achieved = dflops / dcount / (launch_ms / 1e3) / 1e12
+        # one convolution pass reads its input and the weights and writes its output
         nbytes = x_host.nbytes + pixels * w.D * w.T * 2 + inp["Wc"].nbytes
         hbm = nbytes / (launch_ms / 1e3) / 1e9
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                "traffic": kernel_traffic("conv", workload),
+                "traffic": kernel_traffic("conv", workload) if dfam == "conv" else None,
                 "peak_source": f"{peak_src} dense bf16 burst (fp16 runs at the same rate)",
                 "hbm_gbs": hbm, "hbm_frac": hbm / peaks["hbm_gbs"], "launch_ms": launch_ms,
-                "kernel": "eqlinear_conv_forward[planes pre-pass + tcgen05 tap loop]",
-                "step_share": 1.0}
+                "kernel": ("eqlinear_conv_forward / conv_backward_input[planes pre-pass + "
+                           "tcgen05 tap loop]" if dfam == "conv" else
+                           "eqlinear_conv_backward_weight[padded grid + per-tap layer dW]"),
+                "step_share": fam_ms / float(op_ms.sum())}
         comparator = None
         if not args.no_dense:
             # cuDNN on the replicated dense kernel K[(d,s),(c,t),i,j] = Wc[i,j,d,c,(t-s) mod T]
@@ -1305,8 +1366,14 @@ def run_conv(args, workload):
             brep = bias.repeat_interleave(w.T)
 
             def dense(i):
-                return F.conv2d(xs[i % nsets].permute(0, 3, 1, 2), K, brep,
-                                padding=(w.ph, w.pw))
+                x = xs[i % nsets].permute(0, 3, 1, 2)
+                y = F.conv2d(x, K, brep, padding=(w.ph, w.pw))
+                if bwd:
+                    g = dys[i % nsets].permute(0, 3, 1, 2)
+                    torch.nn.grad.conv2d_input(x.shape, K, g, padding=(w.ph, w.pw))
+                    torch.nn.grad.conv2d_weight(x, K.shape, g, padding=(w.ph, w.pw))
+                    g.sum(dim=(0, 2, 3))
+                return y
             for i in range(3):
                 dense(i)
             torch.cuda.synchronize()
@@ -1324,10 +1391,13 @@ def run_conv(args, workload):
             torch.cuda.synchronize()
             dms = d0.elapsed_time(d1) / nd
             comparator = {"kind": "dense F.conv2d (cuDNN, channels-last) with the replicated "
-                                  "(D*T x C*T x KH x KW) kernel, same dtype",
+                                  "(D*T x C*T x KH x KW) kernel, same dtype"
+                                  + ("; plus cuDNN's input and weight gradients and the bias "
+                                     "sum" if bwd else ""),
                           "value": pixels / (dms / 1e3), "unit": "tokens/s",
                           "ms_per_step": dms,
-                          "tflops": conv_dense_flops(w) / (dms / 1e3) / 1e12}
+                          "tflops": conv_dense_flops(w) * (3 if bwd else 1) / (dms / 1e3)
+                                    / 1e12}
             comparator["ours_over_dense"] = value / world / comparator["value"]
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -1338,24 +1408,25 @@ def run_conv(args, workload):
             "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
             "tflops": flops * args.steps * world / (elapsed_ms / 1e3) / 1e12,
-            "tflops_dense_equiv": conv_dense_flops(w) * args.steps * world
+            "tflops_dense_equiv": conv_dense_flops(w) * (3 if bwd else 1) * args.steps * world
                                   / (elapsed_ms / 1e3) / 1e12,
             "config": {"workload": CONV_DESCR[workload], "global_batch": w.N * world,
                        "seq_len": None, "tokens": "output pixels",
                        "parallelism": f"replicas x{world} (images independent)",
                        "l2": f"{nsets} rotating input/output sets of {per_set / 2**20:.0f} MiB "
                              "(> 2x L2)",
-                       "kernels": ["conv_forward[tcgen05]"], "timing": timing},
-            "op_ms": [round(launch_ms, 5)],
+                       "kernels": [f"{label}[{fk}]" for label, fk, _, _, _ in ops],
+                       "timing": timing},
+            "op_ms": [round(float(m), 5) for m in op_ms],
             "roofline": roof,
             "cpu_baseline": cpu,
             "dense_comparator": comparator,
             "e2e": {"value": world * pixels * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": int(x_pin.numel() * 2),
-                    "d2h_bytes_per_step": int(y_pin.numel() * 2),
+                    "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h),
                     "copies": "overlapped with the neighbouring steps' calls (copy-in, "
                               "compute, copy-out streams; two device sets)"},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": sum(n for _, _, _, n, _ in ops) * args.steps,
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)

@@ -627,12 +627,19 @@ size_t eqlinear_conv_backward_workspace_bytes(eqlinear_plan_t p, int64_t N, int 
     return 0;
   const int64_t Ho = (int64_t)H + 2 * pad_h - KH + 1, Wo = (int64_t)W + 2 * pad_w - KW + 1;
   if (Ho < 1 || Wo < 1) return 0;
-  const int64_t rows = N * Ho * Wo;
-  // dX: the group DFT planes of dY; dW: one tap's shifted rows of X, then the
-  // layer weight gradient's scratch for N*Ho*Wo rows
+  // dX: the group DFT planes of dY; dW: X and dY on the padded pixel grid, then
+  // the layer weight gradient's scratch for all of its rows
   const size_t dx = eql::conv_tc_planes_bytes(N, (int)Ho, (int)Wo, p->D);
-  const size_t shifted = ((size_t)rows * p->C * 4 * elem_size(p->dtype) + 255) / 256 * 256;
-  const size_t dw = shifted + eqlinear_backward_weight_workspace_bytes(p, rows);
+  const int64_t rows = N * ((int64_t)H + 2 * pad_h) * ((int64_t)W + 2 * pad_w);
+  const size_t xpad = ((size_t)rows * p->C * 4 * elem_size(p->dtype) + 255) / 256 * 256;
+  const size_t gpad = ((size_t)rows * p->D * 4 * elem_size(p->dtype) + 255) / 256 * 256;
+  // the taps' weight gradients run over rows - (i*Wp + j) rows each
+  size_t wg = 0;
+  for (int tap = 0; tap < KH * KW; ++tap) {
+    const int64_t off = (int64_t)(tap / KW) * (W + 2 * pad_w) + tap % KW;
+    wg = std::max(wg, eqlinear_backward_weight_workspace_bytes(p, rows - off));
+  }
+  const size_t dw = xpad + gpad + wg;
   return std::max<size_t>(std::max(dx, dw), 16);
 }
 
@@ -685,21 +692,37 @@ eqlinear_status_t eqlinear_conv_backward_weight(eqlinear_plan_t p, const void* X
   eqlinear_status_t s = check_plan_device(p);
   if (s != EQL_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  const int64_t rows = N * Ho * Wo;
-  const size_t shifted = ((size_t)rows * p->C * 4 * elem_size(p->dtype) + 255) / 256 * 256;
-  char* xs = static_cast<char*>(workspace);
-  char* ws = xs + shifted;
-  const size_t ws_bytes = workspace_bytes - shifted;
-  const size_t w_tap = (size_t)p->D * p->C * 4 * elem_size(p->dtype);
+  // On the padded grid (Hp x Wp per image) X_pad[n,y,x] = X[n, y-ph, x-pw] (zero
+  // outside) and dY_pad[n,y,x] = dY[n,y,x] for y < Ho, x < Wo (zero elsewhere).
+  // Output pixel (n,y,x) of tap (i,j) reads X_pad[n, y+i, x+j]: flattened, the
+  // row i*Wp + j after dY_pad's row, with no wrap (x+j < Wp, y+i < Hp), so
+  // dWc[i][j] is the layer's weight gradient of X_pad shifted by i*Wp + j rows
+  // and dY_pad.  The rows it drops at the end are past the last valid pixel of
+  // dY_pad, hence zero.
+  const int Hp = H + 2 * pad_h, Wp = W + 2 * pad_w;
+  const int64_t rows = N * (int64_t)Hp * Wp;
+  const size_t es = elem_size(p->dtype);
+  const size_t xpad = ((size_t)rows * p->C * 4 * es + 255) / 256 * 256;
+  const size_t gpad = ((size_t)rows * p->D * 4 * es + 255) / 256 * 256;
+  char* xp = static_cast<char*>(workspace);
+  char* gp = xp + xpad;
+  char* ws = gp + gpad;
+  const size_t ws_bytes = workspace_bytes - xpad - gpad;
+  if (N > 0) {
+    s = from_cuda(eql::launch_conv_shift_rows(X, N, H, W, p->C * 4, 0, 0, pad_h, pad_w, Hp, Wp,
+                                              xp, st));
+    if (s != EQL_OK) return s;
+    s = from_cuda(eql::launch_conv_shift_rows(dY, N, (int)Ho, (int)Wo, p->D * 4, 0, 0, 0, 0, Hp,
+                                              Wp, gp, st));
+    if (s != EQL_OK) return s;
+  }
+  const size_t w_tap = (size_t)p->D * p->C * 4 * es;
   for (int tap = 0; tap < KH * KW; ++tap) {
-    if (N > 0) {
-      s = from_cuda(eql::launch_conv_shift_rows(X, N, H, W, p->C * 4, tap / KW, tap % KW, pad_h,
-                                                pad_w, (int)Ho, (int)Wo, xs, st));
-      if (s != EQL_OK) return s;
-    }
-    // the layer's weight gradient over the tap's rows; dbias (the same for every
-    // tap) with the first tap only
-    s = backward_weight_impl(p, N > 0 ? xs : nullptr, dY, rows,
+    const int64_t off = (int64_t)(tap / KW) * Wp + tap % KW;
+    const int64_t n_rows = N > 0 ? rows - off : 0;
+    // dbias (the same for every tap) with the first tap only
+    s = backward_weight_impl(p, N > 0 ? xp + (size_t)off * p->C * 4 * es : nullptr,
+                             N > 0 ? gp : nullptr, n_rows,
                              static_cast<char*>(dWc) + (size_t)tap * w_tap,
                              tap == 0 ? dbias : nullptr, ws, ws_bytes, to_dt(p->dtype), stream,
                              0);

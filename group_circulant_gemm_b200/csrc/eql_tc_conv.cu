@@ -386,8 +386,10 @@ cudaError_t launch_conv_tc(const void* X, int64_t N, int H, int W, int C, int D,
 }
 
 namespace {
-// Tap-shifted rows of a pixel tensor (the convolution's weight gradient runs the
-// layer's weight-gradient kernel per tap on these rows): one thread per 16 bytes.
+// A pixel tensor moved onto another pixel grid: out[n][oy][ox] = X[n][oy + i - ph]
+// [ox + j - pw], zero where that pixel lies outside the image (the convolution's
+// weight gradient puts X and dY on its padded grid this way); one thread per 16
+// bytes.
 __global__ void conv_shift_rows_kernel(const uint4* __restrict__ X, int64_t N, int H, int W,
                                        int c16, int i, int j, int ph, int pw, int Ho, int Wo,
                                        uint4* __restrict__ out) {

@@ -786,6 +786,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WP_THREADS, 1)
 }
 
 constexpr int FZ_D = 32, FZ_C = 8;
+constexpr int FZ_U = 8;  // row blocks summed side by side
 template <typename Out>
 __global__ void __launch_bounds__(256)
     wgrad_tc_finalize_kernel(const float* __restrict__ part, const float* __restrict__ bpart,
@@ -801,17 +802,56 @@ __global__ void __launch_bounds__(256)
     const int d = d0 + lane, c = c0 + w;  // lane = out-channel, warp = in-channel
     if (d < D && c < C) {
       const int64_t off = (int64_t)(c % WG_BC) * WG_BD + (d % WG_BD);
-      float qv[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int b = 0; b < wi.nb; ++b) {
-        const int pair = b * wi.n_dt * wi.n_ct + tile;
-        const int n = last_range_of_pair(b, tile, wi) - first_range_of_pair(b, tile, wi);
-        for (int j = 0; j <= n; ++j) {
-          const float* slot =
-              part + (((int64_t)pair * wi.maxj + j) * mult + half) * (4 * WG_BC * WG_BD);
+      // Row blocks in groups of FZ_U: each block's slots go to their own
+      // accumulators (the first slot's loads of the whole group issued together,
+      // so a thread has FZ_U x 4 loads in flight), then the FZ_U partial sums are
+      // added in a fixed order.  A few output tiles and many row blocks (a small
+      // layer over many rows) would otherwise leave a long chain of dependent
+      // loads per thread.
+      float qa[FZ_U][4];
 #pragma unroll
-          for (int p = 0; p < 4; ++p) qv[p] += slot[p * (WG_BC * WG_BD) + off];
+      for (int u = 0; u < FZ_U; ++u)
+#pragma unroll
+        for (int p = 0; p < 4; ++p) qa[u][p] = 0.f;
+      for (int b0 = 0; b0 < wi.nb; b0 += FZ_U) {
+        float v[FZ_U][4];
+#pragma unroll
+        for (int u = 0; u < FZ_U; ++u) {
+          const int b = b0 + u;
+#pragma unroll
+          for (int p = 0; p < 4; ++p) v[u][p] = 0.f;
+          if (b < wi.nb) {
+            const int pair = b * wi.n_dt * wi.n_ct + tile;
+            const float* slot =
+                part + ((int64_t)pair * wi.maxj * mult + half) * (4 * WG_BC * WG_BD);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) v[u][p] = slot[p * (WG_BC * WG_BD) + off];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < FZ_U; ++u)
+#pragma unroll
+          for (int p = 0; p < 4; ++p) qa[u][p] += v[u][p];
+        // a row block's further slots (ranges that started inside it)
+#pragma unroll
+        for (int u = 0; u < FZ_U; ++u) {
+          const int b = b0 + u;
+          if (b >= wi.nb) continue;
+          const int pair = b * wi.n_dt * wi.n_ct + tile;
+          const int n = last_range_of_pair(b, tile, wi) - first_range_of_pair(b, tile, wi);
+          for (int j = 1; j <= n; ++j) {
+            const float* slot =
+                part + (((int64_t)pair * wi.maxj + j) * mult + half) * (4 * WG_BC * WG_BD);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) qa[u][p] += slot[p * (WG_BC * WG_BD) + off];
+          }
         }
       }
+      float qv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int u = 0; u < FZ_U; ++u)
+#pragma unroll
+        for (int p = 0; p < 4; ++p) qv[p] += qa[u][p];
       // both operand planes carried 1/4: the partial sums are Q/16
 #pragma unroll
       for (int p = 0; p < 4; ++p) qv[p] *= 16.f;
@@ -829,13 +869,23 @@ __global__ void __launch_bounds__(256)
   if (dbias && blockIdx.y == 0 && w == 0 && d0 + lane < D) {
     const int d = d0 + lane;
     const int tile0 = (d / WG_BD / mult) * wi.n_ct;
-    float b = 0.f;
-    for (int rb = 0; rb < wi.nb; ++rb) {
-      const int pair = rb * wi.n_dt * wi.n_ct + tile0;
-      const int n = last_range_of_pair(rb, tile0, wi) - first_range_of_pair(rb, tile0, wi);
-      for (int j = 0; j <= n; ++j)
-        b += bpart[(((int64_t)pair * wi.maxj + j) * mult + half) * WG_BD + d % WG_BD];
+    float ba[FZ_U];
+#pragma unroll
+    for (int u = 0; u < FZ_U; ++u) ba[u] = 0.f;
+    for (int rb0 = 0; rb0 < wi.nb; rb0 += FZ_U) {
+#pragma unroll
+      for (int u = 0; u < FZ_U; ++u) {
+        const int rb = rb0 + u;
+        if (rb >= wi.nb) continue;
+        const int pair = rb * wi.n_dt * wi.n_ct + tile0;
+        const int n = last_range_of_pair(rb, tile0, wi) - first_range_of_pair(rb, tile0, wi);
+        for (int j = 0; j <= n; ++j)
+          ba[u] += bpart[(((int64_t)pair * wi.maxj + j) * mult + half) * WG_BD + d % WG_BD];
+      }
     }
+    float b = 0.f;
+#pragma unroll
+    for (int u = 0; u < FZ_U; ++u) b += ba[u];
     store_one(dbias + d, b);
   }
 }

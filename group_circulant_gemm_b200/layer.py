@@ -351,15 +351,21 @@ class EqLinearPlan:
                                         workspace, workspace.numel() * workspace.element_size())
         return out
 
-    def conv_backward_weight(self, X, dY, KH: int, KW: int, pad=(0, 0), workspace=None):
+    def conv_backward_weight(self, X, dY, KH: int, KW: int, pad=(0, 0), workspace=None,
+                             dW=None, dbias=None):
         """X [N, H, W, C*T], dY [N, Ho, Wo, D*T] -> (dWc [KH, KW, D, C, T], dbias [D])."""
         N, H, W = (int(v) for v in X.shape[:3])
         self._check(X, (N, H, W, self.C * self.T), "X")
         ph, pw = pad
         Ho, Wo = H + 2 * ph - KH + 1, W + 2 * pw - KW + 1
         self._check(dY, (N, Ho, Wo, self.D * self.T), "dY")
-        dW = torch.empty((KH, KW, self.D, self.C, self.T), dtype=self.dtype, device=X.device)
-        db = torch.empty(self.D, dtype=self.dtype, device=X.device)
+        if dW is None:
+            dW = torch.empty((KH, KW, self.D, self.C, self.T), dtype=self.dtype, device=X.device)
+        self._check(dW, (KH, KW, self.D, self.C, self.T), "dW")
+        db = dbias
+        if db is None:
+            db = torch.empty(self.D, dtype=self.dtype, device=X.device)
+        self._check(db, (self.D,), "dbias")
         workspace = self._conv_bwd_workspace(N, H, W, KH, KW, ph, pw, workspace, X.device)
         _n.eqlinear_conv_backward_weight(self.handle, X, N, H, W, dY, KH, KW, ph, pw, dW, db,
                                          workspace, workspace.numel() * workspace.element_size())

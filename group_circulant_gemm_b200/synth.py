@@ -107,6 +107,7 @@ class ConvWorkload:
     pw: int
     dtype: str = "f16"
     seed: int = 1300
+    backward: bool = False  # a training step: forward, dX and dWc
 
     @property
     def Ho(self) -> int:
@@ -126,24 +127,32 @@ class ConvWorkload:
 CONV_WORKLOADS = {
     "p4_conv3x3_f16": ConvWorkload("p4_conv3x3_f16", 4, 64, 56, 56, 64, 64, 3, 3, 1, 1, "f16",
                                    1300),
+    "p4_conv3x3_fwd_bwd_f16": ConvWorkload("p4_conv3x3_fwd_bwd_f16", 4, 64, 56, 56, 64, 64, 3,
+                                           3, 1, 1, "f16", 1300, True),
 }
 
 
-def make_conv_inputs(w: ConvWorkload, images: int | None = None):
-    """dict(X [N, H, W, C*T], Wc [KH, KW, D, C, T], bias [D]) with the layer's recipe:
-    float64 normal draws in the order X, Wc, bias from default_rng(seed),
-    Wc ~ N(0, 1/(C*T*KH*KW)), bias ~ N(0, 0.01), cast to the dtype.  ``images``
-    keeps a prefix of the images (drawn in full first)."""
+def make_conv_inputs(w: ConvWorkload, images: int | None = None, need_dy: bool = False):
+    """dict(X [N, H, W, C*T], Wc [KH, KW, D, C, T], bias [D], and with need_dy
+    dY [N, Ho, Wo, D*T]) with the layer's recipe: float64 normal draws in the
+    order X, Wc, bias, dY from default_rng(seed), Wc ~ N(0, 1/(C*T*KH*KW)),
+    bias ~ N(0, 0.01), dY ~ N(0, 1), cast to the dtype.  ``images`` keeps a
+    prefix of the images (drawn in full first)."""
     rng = np.random.default_rng(w.seed)
     X = rng.standard_normal((w.N, w.H, w.W, w.C * w.T))
     Wc = rng.standard_normal((w.KH, w.KW, w.D, w.C, w.T)) * np.sqrt(
         1.0 / (w.C * w.T * w.KH * w.KW))
     b = rng.standard_normal((w.D,)) * np.sqrt(0.01)
+    dY = rng.standard_normal((w.N, w.Ho, w.Wo, w.D * w.T)) if need_dy else None
     if images is not None:
         X = X[:images]
+        dY = None if dY is None else dY[:images]
     dt = np.float16 if w.dtype == "f16" else np.float32
-    return {"X": np.ascontiguousarray(X.astype(dt)), "Wc": np.ascontiguousarray(Wc.astype(dt)),
-            "bias": np.ascontiguousarray(b.astype(dt))}
+    out = {"X": np.ascontiguousarray(X.astype(dt)), "Wc": np.ascontiguousarray(Wc.astype(dt)),
+           "bias": np.ascontiguousarray(b.astype(dt))}
+    if dY is not None:
+        out["dY"] = np.ascontiguousarray(dY.astype(dt))
+    return out
 
 
 # Extreme group vectors for the FP16 range tests: for each group order, sign

@@ -442,10 +442,12 @@ EQL_API eqlinear_status_t eqlinear_conv_forward(eqlinear_plan_t plan, const void
  *     KW-1-pad_w); it runs the forward's tensor-core kernel with the adjoint
  *     tiles that eqlinear_conv_prepare_weights also writes into Wc_hat.
  *   eqlinear_conv_backward_weight: dWc [KH][KW][D][C][T] and dbias [D] (or NULL)
- *     in the plan dtype. Each tap is the layer's weight gradient between the
- *     rows of dY and the rows of X shifted by that tap (zero outside the image):
- *     a gather into the workspace, then the layer's weight-gradient kernel
- *     (tensor cores when C and D are multiples of 64).
+ *     in the plan dtype. X and dY are copied once into the workspace on the
+ *     padded pixel grid ((H + 2 pad_h) x (W + 2 pad_w) per image: X shifted by
+ *     the padding, dY at the top left, zeros elsewhere); tap (i, j) is then the
+ *     layer's weight gradient between dY's padded rows and X's padded rows
+ *     offset by i (W + 2 pad_w) + j (the layer's weight-gradient kernel, tensor
+ *     cores when the shape allows).
  *   eqlinear_conv_backward_workspace_bytes(plan, N, H, W, KH, KW, pad_h, pad_w):
  *     scratch of both calls.
  * Plans and limits as for eqlinear_conv_forward; all pointers 16-byte aligned;
