@@ -178,7 +178,7 @@ KERNEL_SOURCES = {
 NCU_TRAFFIC = {
     ("forward", "443ba94f5b306a59"): {"p4_vitb_mlp_2calls_f16": 58.96e6, "c8_1024_f16": 34.20e6, "p4_vith_fc1_f16": 51.20e6, "p4_vith_fc1_fwd_bwd_f16": 109.13e6, "p4m_vitb_mlp_fused_f16": 57.79e6},
     ("forward_chain", "246b0f491b3357c1"): {"p4_vitb_mlp_fused_f16": 89.59e6, "p4_vitb_mlp_spectral_f16": 80.93e6, "p4_vitb_mlp_block_f16": 81.74e6},
-    ("conv", "70beebb2fc455f9a"): {"p4_conv3x3_f16": 161.54e6},
+    ("conv", "ae4ea6f4164e2f9d"): {"p4_conv3x3_f16": 161.54e6},
     ("forward_chain_tiled", "6ade53bcfcfaa10b"): {"p4_vitb_mlp_f16": 99.44e6},
     ("forward_pair", "6ade53bcfcfaa10b"): {"p4_vith_fc1_fwd_bwd_tiled_f16": 96.53e6},
     ("forward_tiled", "2fe2ac1739cebc38"): {"p4_vitb_proj_f32": 85.81e6, "p4m_vitb_mlp_f16": 59.08e6, "c8_1024_tiled_f16": 34.38e6},
@@ -1213,9 +1213,13 @@ def run_conv(args, workload):
             p.conv_backward_weight(xs[i % nsets], dys[i % nsets], w.KH, w.KW, pad=(w.ph, w.pw),
                                    workspace=wsb, dW=gW, dbias=gb)
         # dX: the planes pre-pass of dY and the tap-loop kernel; dWc: X and dY onto
-        # the padded grid, then per tap the layer's weight gradient and its finalize
+        # the padded grid (and their group spectra), then per tap the layer's
+        # weight gradient and its finalize
         ops += [("conv_backward_input", "conv", conv_flops(w), 2, bwd_x),
-                ("conv_backward_weight", "conv_wgrad", conv_flops(w), 2 + 2 * w.KH * w.KW,
+                ("conv_backward_weight", "conv_wgrad", conv_flops(w),
+                 # two copies onto the padded grid, (with C and D multiples of 64)
+                 # two spectra passes, and per tap a weight gradient + finalize
+                 2 + (2 if w.C % 64 == 0 and w.D % 64 == 0 else 0) + 2 * w.KH * w.KW,
                  bwd_w)]
 
     def step(i, events=None, external=False):

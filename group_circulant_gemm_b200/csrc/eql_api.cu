@@ -621,6 +621,12 @@ eqlinear_status_t eqlinear_conv_prepare_weights(eqlinear_plan_t p, int KH, int K
   return EQL_OK;
 }
 
+// The convolution's weight gradient multiplies the padded rows' group spectra
+// (computed once) when the tensor-core kernel's planes variant takes the shape.
+static bool conv_wgrad_on_planes(eqlinear_plan_t p) {
+  return p->kernel != EQL_KERNEL_SIMT && p->C % 64 == 0 && p->D % 64 == 0;
+}
+
 size_t eqlinear_conv_backward_workspace_bytes(eqlinear_plan_t p, int64_t N, int H, int W, int KH,
                                               int KW, int pad_h, int pad_w) {
   if (!conv_plan_ok(p) || N < 0 || H < 1 || W < 1 || KH < 1 || KW < 1 || pad_h < 0 || pad_w < 0)
@@ -639,7 +645,10 @@ size_t eqlinear_conv_backward_workspace_bytes(eqlinear_plan_t p, int64_t N, int 
     const int64_t off = (int64_t)(tap / KW) * (W + 2 * pad_w) + tap % KW;
     wg = std::max(wg, eqlinear_backward_weight_workspace_bytes(p, rows - off));
   }
-  const size_t dw = xpad + gpad + wg;
+  // with C and D multiples of 64, the padded rows' group spectra too (as large as
+  // the padded rows)
+  const size_t spectra = conv_wgrad_on_planes(p) ? xpad + gpad : 0;
+  const size_t dw = xpad + gpad + spectra + wg;
   return std::max<size_t>(std::max(dx, dw), 16);
 }
 
@@ -704,10 +713,13 @@ eqlinear_status_t eqlinear_conv_backward_weight(eqlinear_plan_t p, const void* X
   const size_t es = elem_size(p->dtype);
   const size_t xpad = ((size_t)rows * p->C * 4 * es + 255) / 256 * 256;
   const size_t gpad = ((size_t)rows * p->D * 4 * es + 255) / 256 * 256;
+  const bool on_planes = conv_wgrad_on_planes(p) && N > 0;
   char* xp = static_cast<char*>(workspace);
   char* gp = xp + xpad;
-  char* ws = gp + gpad;
-  const size_t ws_bytes = workspace_bytes - xpad - gpad;
+  char* xs = gp + gpad;  // (on_planes) spectra [4][rows][C] and [4][rows][D]
+  char* gs = xs + xpad;
+  char* ws = on_planes ? gs + gpad : gp + gpad;
+  const size_t ws_bytes = workspace_bytes - (size_t)(ws - xp);
   if (N > 0) {
     s = from_cuda(eql::launch_conv_shift_rows(X, N, H, W, p->C * 4, 0, 0, pad_h, pad_w, Hp, Wp,
                                               xp, st));
@@ -717,6 +729,27 @@ eqlinear_status_t eqlinear_conv_backward_weight(eqlinear_plan_t p, const void* X
     if (s != EQL_OK) return s;
   }
   const size_t w_tap = (size_t)p->D * p->C * 4 * es;
+  if (on_planes) {
+    // the padded rows' group spectra once; then per tap the planes variant with
+    // X's spectra read from row i*Wp + j of every plane
+    s = from_cuda(eql::launch_conv_group_planes(xp, rows, p->C, xs, st));
+    if (s != EQL_OK) return s;
+    s = from_cuda(eql::launch_conv_group_planes(gp, rows, p->D, gs, st));
+    if (s != EQL_OK) return s;
+    if (ws_bytes < eqlinear_backward_weight_workspace_bytes(p, rows)) return EQL_ERR_WORKSPACE;
+    s = check_plan_device(p);
+    if (s != EQL_OK) return s;
+    for (int tap = 0; tap < KH * KW; ++tap) {
+      const int64_t off = (int64_t)(tap / KW) * Wp + tap % KW;
+      s = from_cuda(eql::launch_wgrad_tc(xs + (size_t)off * p->C * es, gs, rows - off, p->C,
+                                         p->D, ws, to_dt(p->dtype),
+                                         static_cast<char*>(dWc) + (size_t)tap * w_tap,
+                                         tap == 0 ? dbias : nullptr, p->status, p->num_sms, p->tw,
+                                         st, 1, rows));
+      if (s != EQL_OK) return s;
+    }
+    return EQL_OK;
+  }
   for (int tap = 0; tap < KH * KW; ++tap) {
     const int64_t off = (int64_t)(tap / KW) * Wp + tap % KW;
     const int64_t n_rows = N > 0 ? rows - off : 0;

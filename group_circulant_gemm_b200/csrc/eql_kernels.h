@@ -75,13 +75,15 @@ bool wgrad_tc_supported(int T, DType dt, int64_t N, int C, int D, const void* X,
 size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms);
 // planes = 1: X and dY are instead their group spectra as FP16 planes
 // [4][N][C] and [4][N][D] (as the forward and dX kernels save them); needs
-// C % 64 == 0 and D % 64 == 0 (wgrad_tc_planes_supported).  planes = 2: the
-// spectra in the tiled layout of the SM-pair kernels (tiled_rows(N) rows per
+// C % 64 == 0 and D % 64 == 0 (wgrad_tc_planes_supported).  With plane_rows > N
+// the N rows are read from inside planes of plane_rows rows each.  planes = 2:
+// the spectra in the tiled layout of the SM-pair kernels (tiled_rows(N) rows per
 // 16-channel block, as launch_group_dft_tiled writes them); C, D multiples of 16.
 bool wgrad_tc_planes_supported(int64_t N, int C, int D, const void* Xhat, const void* Ghat);
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
                             void* workspace, DType out_dt, void* dW, void* dbias, int* status,
-                            int num_sms, const Twiddles& tw, cudaStream_t st, int planes = 0);
+                            int num_sms, const Twiddles& tw, cudaStream_t st, int planes = 0,
+                            int64_t plane_rows = 0);
 
 // Two chained T = 4 FP16 layers (C0 -> C1 -> C2) in one persistent launch with a
 // dynamic tile queue: H = act1(L1(X)) (spatial [N][C1*4], or spectral planes
@@ -167,7 +169,12 @@ cudaError_t launch_pair8_tc(const void* Xt, int64_t N, int Cin, int Cout, const 
                             const void* bias, void* Y, int* status, int num_sms, int act,
                             int group, cudaStream_t st, int next_planes = 0);
 
-// Rows of X [N][H][W][c4 halves] shifted by a convolution tap: out[(n*Ho + oy)*Wo + ox]
+// The group DFT of P pixel rows: X [P][C*4] -> planes [4][P][C] (X0, X2, Xr, Xi,
+// each times 1/4; the convolution kernel's pre-pass).
+cudaError_t launch_conv_group_planes(const void* X, int64_t P, int C, void* planes,
+                                     cudaStream_t st);
+
+// X [N][H][W][c4 halves] moved onto an Ho x Wo pixel grid: out[(n*Ho + oy)*Wo + ox]
 // = X[n][oy+i-ph][ox+j-pw] (zero outside the image), c4 a multiple of 8.
 cudaError_t launch_conv_shift_rows(const void* X, int64_t N, int H, int W, int c4, int i, int j,
                                    int ph, int pw, int Ho, int Wo, void* out, cudaStream_t st);

@@ -407,6 +407,16 @@ __global__ void conv_shift_rows_kernel(const uint4* __restrict__ X, int64_t N, i
 }
 }  // namespace
 
+cudaError_t launch_conv_group_planes(const void* X, int64_t P, int C, void* planes,
+                                     cudaStream_t st) {
+  if (C % 8 != 0) return cudaErrorInvalidValue;
+  const int64_t work = P * (C / 8);
+  if (work == 0) return cudaSuccess;
+  conv_planes_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint4*>(X), P, C, static_cast<uint4*>(planes));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_conv_shift_rows(const void* X, int64_t N, int H, int W, int c4, int i, int j,
                                    int ph, int pw, int Ho, int Wo, void* out, cudaStream_t st) {
   if (c4 % 8 != 0) return cudaErrorInvalidValue;

@@ -908,11 +908,15 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int channels, int64_t N) 
 // block, plane); box = (64, PL_ROWS rows, 2 blocks, 4 planes), 128-byte swizzle.
 // The block dimension steps by 128 B inside a row, so channels % 64 == 0 keeps
 // every block inside its row.
-bool encode_planes4_map(CUtensorMap* m, const void* base, int channels, int64_t N) {
+// plane_rows: the rows between one plane and the next (N when the planes are
+// [4][N][channels]; more when N rows are read from inside larger planes).
+bool encode_planes4_map(CUtensorMap* m, const void* base, int channels, int64_t N,
+                        int64_t plane_rows) {
   auto encode = encode_fn();
-  if (!encode || channels % 64 != 0) return false;
+  if (!encode || channels % 64 != 0 || plane_rows < N) return false;
   cuuint64_t dims[4] = {64, (cuuint64_t)N, (cuuint64_t)channels / 64, 4};
-  cuuint64_t strides[3] = {(cuuint64_t)channels * 2, 128, (cuuint64_t)N * channels * 2};
+  cuuint64_t strides[3] = {(cuuint64_t)channels * 2, 128,
+                           (cuuint64_t)plane_rows * channels * 2};
   cuuint32_t box[4] = {64, PL_ROWS, 2, 4};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides,
@@ -1005,7 +1009,8 @@ bool wgrad_tc_planes_supported(int64_t N, int C, int D, const void* Xhat, const 
 
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
                             void* workspace, DType out_dt, void* dW, void* dbias, int* status,
-                            int num_sms, const Twiddles& tw, cudaStream_t st, int planes) {
+                            int num_sms, const Twiddles& tw, cudaStream_t st, int planes,
+                            int64_t plane_rows) {
   WgInfo wi;
   int grid = 0;
   if (planes < 0 || planes > 2) return cudaErrorInvalidValue;
@@ -1019,7 +1024,8 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
         !encode_tiled4_map(&mx, X, C, N, pairs ? 4u : 8u))
       return cudaErrorInvalidValue;
   } else if (planes == 1) {
-    if (!encode_planes4_map(&mg, dY, D, N) || !encode_planes4_map(&mx, X, C, N))
+    const int64_t pr = plane_rows > 0 ? plane_rows : N;
+    if (!encode_planes4_map(&mg, dY, D, N, pr) || !encode_planes4_map(&mx, X, C, N, pr))
       return cudaErrorInvalidValue;
   } else if (!encode_rows_map(&mg, dY, D, N) || !encode_rows_map(&mx, X, C, N)) {
     return cudaErrorInvalidValue;

@@ -9,7 +9,8 @@ KH x KW window, so
     (KH-1-ph, KW-1-pw): eqlinear_conv_backward_input runs the forward
     convolution kernel on those prepared tiles;
   * dWc[i, j] is the layer's weight gradient over the rows of X shifted by tap
-    (i, j) and the rows of dY; dbias is the layer's, once.
+    (i, j) and the rows of dY; dbias is the layer's, once. The library puts X
+    and dY on the padded pixel grid once, so that each tap is a row offset.
 
 FP16 bar: max|gpu - oracle| / max|oracle| <= 2e-3 (the layer's).
 """
@@ -75,7 +76,9 @@ def test_conv_backward_matches_the_oracle(N, H, W, C, D, KH, KW, ph, pw):
 
 
 def test_conv_backward_1x1_is_the_layer_backward():
-    """A 1 x 1 kernel without padding is the layer on N*H*W rows."""
+    """A 1 x 1 kernel without padding is the layer on N*H*W rows. With C and D
+    multiples of 64 the convolution's weight gradient multiplies the rows' group
+    spectra, exactly as the layer's weight gradient from saved spectra does."""
     N, H, W, C, D = 2, 9, 21, 64, 128
     X, Wc, dY = _inputs(N, H, W, C, D, 1, 1, 0, 0, 5100)
     p = _plan(C, D)
@@ -85,7 +88,9 @@ def test_conv_backward_1x1_is_the_layer_backward():
     Wh = p.prepare_weights(_dev(Wc[0, 0]))
     rows = N * H * W
     dX_l = p.backward_input(dYd.view(rows, D * 4), Wh)
-    dW_l, db_l = p.backward_weight(Xd.view(rows, C * 4), dYd.view(rows, D * 4))
+    _, Xhat = p.forward_save_spectrum(Xd.view(rows, C * 4), Wh)
+    _, dYhat = p.backward_input_save_spectrum(dYd.view(rows, D * 4), Wh)
+    dW_l, db_l = p.backward_weight_from_spectra(Xhat, dYhat)
     assert p.status() == 0
     assert _rel(dX.double().cpu().numpy().reshape(rows, -1), dX_l.double().cpu().numpy()) <= 1e-3
     assert torch.equal(dW[0, 0].view(torch.int16), dW_l.view(torch.int16))
