@@ -24,6 +24,26 @@ def test_every_pipeline_resolves_and_chains():
         assert len(bench.PIPELINES[name]) == 2, name
     for name in bench.BACKWARD:
         assert name in bench.PIPELINES
+    # the frequency-domain training step is a training step; a pipeline chained
+    # through next-layer planes runs in the frequency-domain form
+    assert bench.TILED_TRAIN <= bench.BACKWARD
+    assert bench.TILED_NEXT <= bench.TILED_LAYERS
+
+
+def test_every_convolution_workload_is_described():
+    from group_circulant_gemm_b200.synth import CONV_WORKLOADS, make_conv_inputs
+    for name, w in CONV_WORKLOADS.items():
+        assert name in bench.CONV_DESCR, name
+        assert w.Ho >= 1 and w.Wo >= 1
+    # the training step's upstream gradient has the output's shape
+    w = CONV_WORKLOADS["p4_conv3x3_fwd_bwd_f16"]
+    assert w.backward
+    inp = make_conv_inputs(w, images=2, need_dy=True)
+    assert inp["dY"].shape == (2, w.Ho, w.Wo, w.D * w.T)
+    # the forward's inputs do not depend on whether dY is drawn (it comes last)
+    base = make_conv_inputs(CONV_WORKLOADS["p4_conv3x3_f16"], images=2)
+    for k in ("X", "Wc", "bias"):
+        assert (base[k] == inp[k]).all(), k
 
 
 def test_flop_counts():
