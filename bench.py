@@ -1217,9 +1217,10 @@ def run_conv(args, workload):
         # weight gradient and its finalize
         ops += [("conv_backward_input", "conv", conv_flops(w), 2, bwd_x),
                 ("conv_backward_weight", "conv_wgrad", conv_flops(w),
-                 # two copies onto the padded grid, (with C and D multiples of 64)
-                 # two spectra passes, and per tap a weight gradient + finalize
-                 2 + (2 if w.C % 64 == 0 and w.D % 64 == 0 else 0) + 2 * w.KH * w.KW,
+                 # two copies onto the padded grid; with C and D multiples of 64 two
+                 # spectra passes and one weight gradient + finalize for all taps,
+                 # else per tap a weight gradient + finalize
+                 2 + (4 if w.C % 64 == 0 and w.D % 64 == 0 else 2 * w.KH * w.KW),
                  bwd_w)]
 
     def step(i, events=None, external=False):

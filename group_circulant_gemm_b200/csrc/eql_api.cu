@@ -646,8 +646,11 @@ size_t eqlinear_conv_backward_workspace_bytes(eqlinear_plan_t p, int64_t N, int 
     wg = std::max(wg, eqlinear_backward_weight_workspace_bytes(p, rows - off));
   }
   // with C and D multiples of 64, the padded rows' group spectra too (as large as
-  // the padded rows)
-  const size_t spectra = conv_wgrad_on_planes(p) ? xpad + gpad : 0;
+  // the padded rows), and all taps' weight gradients in one launch
+  const bool planes = conv_wgrad_on_planes(p);
+  const size_t spectra = planes ? xpad + gpad : 0;
+  if (planes)
+    wg = std::max(wg, eql::wgrad_tc_conv_workspace(rows, p->C, p->D, KH * KW, p->num_sms));
   const size_t dw = xpad + gpad + spectra + wg;
   return std::max<size_t>(std::max(dx, dw), 16);
 }
@@ -730,25 +733,18 @@ eqlinear_status_t eqlinear_conv_backward_weight(eqlinear_plan_t p, const void* X
   }
   const size_t w_tap = (size_t)p->D * p->C * 4 * es;
   if (on_planes) {
-    // the padded rows' group spectra once; then per tap the planes variant with
-    // X's spectra read from row i*Wp + j of every plane
+    // the padded rows' group spectra once; then one launch of the planes variant
+    // with the taps as in-channel tiles, tap (i, j) reading X's spectra from row
+    // i*Wp + j on
+    if (ws_bytes < eql::wgrad_tc_conv_workspace(rows, p->C, p->D, KH * KW, p->num_sms))
+      return EQL_ERR_WORKSPACE;
     s = from_cuda(eql::launch_conv_group_planes(xp, rows, p->C, xs, st));
     if (s != EQL_OK) return s;
     s = from_cuda(eql::launch_conv_group_planes(gp, rows, p->D, gs, st));
     if (s != EQL_OK) return s;
-    if (ws_bytes < eqlinear_backward_weight_workspace_bytes(p, rows)) return EQL_ERR_WORKSPACE;
-    s = check_plan_device(p);
-    if (s != EQL_OK) return s;
-    for (int tap = 0; tap < KH * KW; ++tap) {
-      const int64_t off = (int64_t)(tap / KW) * Wp + tap % KW;
-      s = from_cuda(eql::launch_wgrad_tc(xs + (size_t)off * p->C * es, gs, rows - off, p->C,
-                                         p->D, ws, to_dt(p->dtype),
-                                         static_cast<char*>(dWc) + (size_t)tap * w_tap,
-                                         tap == 0 ? dbias : nullptr, p->status, p->num_sms, p->tw,
-                                         st, 1, rows));
-      if (s != EQL_OK) return s;
-    }
-    return EQL_OK;
+    return from_cuda(eql::launch_wgrad_tc_conv(xs, gs, rows, p->C, p->D, KH * KW, KW, Wp, ws,
+                                               to_dt(p->dtype), dWc, dbias, p->status,
+                                               p->num_sms, p->tw, st));
   }
   for (int tap = 0; tap < KH * KW; ++tap) {
     const int64_t off = (int64_t)(tap / KW) * Wp + tap % KW;

@@ -80,6 +80,16 @@ size_t wgrad_tc_workspace(int64_t N, int C, int D, int num_sms);
 // the spectra in the tiled layout of the SM-pair kernels (tiled_rows(N) rows per
 // 16-channel block, as launch_group_dft_tiled writes them); C, D multiples of 16.
 bool wgrad_tc_planes_supported(int64_t N, int C, int D, const void* Xhat, const void* Ghat);
+// A convolution's weight gradient in one launch (planes variant): Xs [4][R][C]
+// and Gs [4][R][D] are the group spectra of X and dY on the padded pixel grid
+// (R rows, planes times 1/4); tap t = i*kw + j multiplies Gs's rows with Xs's
+// rows i*wp + j further on, into dW + t*D*C*4 (dW [taps][D][C][4]); dbias once.
+// C and D multiples of 64.
+size_t wgrad_tc_conv_workspace(int64_t R, int C, int D, int taps, int num_sms);
+cudaError_t launch_wgrad_tc_conv(const void* Xs, const void* Gs, int64_t R, int C, int D,
+                                 int taps, int kw, int wp, void* workspace, DType out_dt,
+                                 void* dW, void* dbias, int* status, int num_sms,
+                                 const Twiddles& tw, cudaStream_t st);
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
                             void* workspace, DType out_dt, void* dW, void* dbias, int* status,
                             int num_sms, const Twiddles& tw, cudaStream_t st, int planes = 0,

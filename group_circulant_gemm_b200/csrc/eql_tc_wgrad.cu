@@ -147,6 +147,10 @@ static_assert(sizeof(WgBars) <= 512, "barrier block");
 
 struct WgInfo {
   int n_dt, n_ct;      // out-channel and in-channel tiles
+  // (convolution, planes variant) the in-channel tiles are taps x nct_tap: tile
+  // ct is channel block ct % nct_tap of tap ct / nct_tap, whose X rows are read
+  // (tap / tap_kw) * tap_wp + tap % tap_kw rows further on; one tap otherwise
+  int nct_tap, tap_kw, tap_wp;
   int spt;             // 32-row stages per tile, ceil(N / 32)
   int bst;             // stages per row block (the last block: spt - (nb - 1) * bst)
   int nb;              // row blocks
@@ -154,6 +158,12 @@ struct WgInfo {
   int maxj;            // partial slots per (block, tile) pair
   int64_t total;       // tiles * spt
 };
+
+__host__ __device__ inline int ct_block(int ct, const WgInfo& wi) { return ct % wi.nct_tap; }
+__host__ __device__ inline int ct_row_offset(int ct, const WgInfo& wi) {
+  const int tap = ct / wi.nct_tap;
+  return (tap / wi.tap_kw) * wi.tap_wp + tap % wi.tap_kw;
+}
 
 // One segment of a CTA's range: stages [r0 / 32, r0 / 32 + stages) of one tile.
 struct Unit {
@@ -340,7 +350,8 @@ __global__ void __launch_bounds__(PL ? WG_THREADS_PL : WG_THREADS, 1)
           } else if constexpr (PL) {
             // 4-D planes views (64 channels, row, 64-channel block, plane)
             tma_load_4d(dst, &map_g, &bars->full[slot], 0, row, 2 * un.dt, 0);
-            tma_load_4d(dst + TILEB, &map_x, &bars->full[slot], 0, row, 2 * un.ct, 0);
+            tma_load_4d(dst + TILEB, &map_x, &bars->full[slot], 0, row + ct_row_offset(un.ct, wi),
+                        2 * ct_block(un.ct, wi), 0);
           } else {
             // 3-D views (64 halves, 128-byte chunk of the row, row); a unit's tile is
             // chunks 8*tile .. 8*tile+7 (128 channels x 4 group elements)
@@ -429,7 +440,7 @@ __global__ void __launch_bounds__(PL ? WG_THREADS_PL : WG_THREADS, 1)
         float* dst_plane = slot_base + p * (WG_BC * WG_BD);
 #pragma unroll 1
         for (int gq = 0; gq < WG_BC / 16; gq += 2) {
-          const int c = un.ct * WG_BC + 16 * gq;
+          const int c = ct_block(un.ct, wi) * WG_BC + 16 * gq;
           if (c >= C) break;  // warp-uniform; C % 16 == 0: the 16 columns are all in range
           const bool two = c + 16 < C;  // the second group of 16 columns is in range
           uint32_t r[16], r2[16];
@@ -795,9 +806,11 @@ __global__ void __launch_bounds__(256)
   __shared__ __align__(16) float s[FZ_C][FZ_D * 4 + 4];  // [c][d][u], rows padded by 16 B
   const int d0 = blockIdx.x * FZ_D, c0 = blockIdx.y * FZ_C;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;  // 8 warps
-  // pairs: a stream-K tile is 256 out-channels; its CTA `half` wrote this block
+  // pairs: a stream-K tile is 256 out-channels; its CTA `half` wrote this block.
+  // blockIdx.z: the convolution tap (its dW block follows the previous taps')
   const int mult = pairs ? 2 : 1, half = pairs ? (d0 / WG_BD) & 1 : 0;
-  const int tile = (d0 / WG_BD / mult) * wi.n_ct + c0 / WG_BC;
+  const int tile = (d0 / WG_BD / mult) * wi.n_ct + blockIdx.z * wi.nct_tap + c0 / WG_BC;
+  dW += (size_t)blockIdx.z * D * C * 4;
   {
     const int d = d0 + lane, c = c0 + w;  // lane = out-channel, warp = in-channel
     if (d < D && c < C) {
@@ -866,7 +879,7 @@ __global__ void __launch_bounds__(256)
     const int c = c0 + cl, d = d0 + dl;
     if (d < D && c < C) store_dw4(dW + ((int64_t)d * C + c) * 4, &s[cl][4 * dl]);
   }
-  if (dbias && blockIdx.y == 0 && w == 0 && d0 + lane < D) {
+  if (dbias && blockIdx.y == 0 && blockIdx.z == 0 && w == 0 && d0 + lane < D) {
     const int d = d0 + lane;
     const int tile0 = (d / WG_BD / mult) * wi.n_ct;
     float ba[FZ_U];
@@ -947,13 +960,18 @@ bool encode_tiled4_map(CUtensorMap* m, const void* base, int channels, int64_t N
 // The stream-K layout for N rows: equal contiguous ranges of (tile, stage), one
 // per CTA, and the number of partial slots a tile can need.
 // pairs: tiles of 256 out-channels, one range per cluster of two SMs.
+// taps > 1 (planes variant only): a convolution's taps as in-channel tiles, tap t
+// reading X (t / kw) * wp + t % kw rows further on.
 bool wgrad_tc_layout(int64_t N, int C, int D, int num_sms, WgInfo* wi, int* grid,
-                     bool pairs = false) {
-  if (N <= 0) return false;
+                     bool pairs = false, int taps = 1, int kw = 1, int wp = 0) {
+  if (N <= 0 || taps < 1 || kw < 1) return false;
   if (pairs) num_sms /= 2;
   if (num_sms < 1) return false;
   wi->n_dt = (D + (pairs ? 2 : 1) * WG_BD - 1) / ((pairs ? 2 : 1) * WG_BD);
-  wi->n_ct = (C + WG_BC - 1) / WG_BC;
+  wi->nct_tap = (C + WG_BC - 1) / WG_BC;
+  wi->n_ct = taps * wi->nct_tap;
+  wi->tap_kw = kw;
+  wi->tap_wp = wp;
   const int64_t spt = (N + WG_BR - 1) / WG_BR;
   if (spt > 0x3fffffffLL) return false;
   wi->spt = (int)spt;
@@ -1007,6 +1025,28 @@ bool wgrad_tc_planes_supported(int64_t N, int C, int D, const void* Xhat, const 
   return wgrad_tc_supported(4, DType::F16, N, C, D, Xhat, Ghat) && C % 64 == 0 && D % 64 == 0;
 }
 
+namespace {
+cudaError_t wgrad_attrs() {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(wgrad_tc_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(wgrad_tc_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(wgrad_tc_kernel<true, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(wgrad_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               WP_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  return cudaSuccess;
+}
+}  // namespace
+
 cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int D,
                             void* workspace, DType out_dt, void* dW, void* dbias, int* status,
                             int num_sms, const Twiddles& tw, cudaStream_t st, int planes,
@@ -1033,22 +1073,8 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
   float* part = static_cast<float*>(workspace);
   float* bpart =
       part + (size_t)wi.nb * wi.n_dt * wi.n_ct * wi.maxj * (pairs ? 2 : 1) * (4 * WG_BC * WG_BD);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(wgrad_tc_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(wgrad_tc_kernel<true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(wgrad_tc_kernel<true, true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(wgrad_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               WP_SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t ea = wgrad_attrs();
+  if (ea != cudaSuccess) return ea;
   if (pairs) {
     cudaError_t e = launch_dependent(wgrad_pair_kernel, dim3(2 * grid), dim3(WP_THREADS), WP_SMEM,
                                      st, mg, mx, C, D, wi, part, bpart, status);
@@ -1073,6 +1099,45 @@ cudaError_t launch_wgrad_tc(const void* X, const void* dY, int64_t N, int C, int
     wgrad_tc_finalize_kernel<__half><<<fgrid, 256, 0, st>>>(
         part, bpart, wi, C, D, static_cast<__half*>(dW), static_cast<__half*>(dbias), tw,
         pairs ? 1 : 0);
+  return cudaGetLastError();
+}
+
+size_t wgrad_tc_conv_workspace(int64_t R, int C, int D, int taps, int num_sms) {
+  WgInfo wi;
+  int grid = 0;
+  if (!wgrad_tc_layout(R, C, D, num_sms, &wi, &grid, false, taps, 1, 0)) return 0;
+  const size_t slots = (size_t)wi.nb * wi.n_dt * wi.n_ct * wi.maxj;
+  return slots * ((size_t)4 * WG_BC * WG_BD + WG_BD) * sizeof(float);
+}
+
+cudaError_t launch_wgrad_tc_conv(const void* Xs, const void* Gs, int64_t R, int C, int D,
+                                 int taps, int kw, int wp, void* workspace, DType out_dt,
+                                 void* dW, void* dbias, int* status, int num_sms,
+                                 const Twiddles& tw, cudaStream_t st) {
+  WgInfo wi;
+  int grid = 0;
+  if (C % 64 != 0 || D % 64 != 0) return cudaErrorNotSupported;
+  if (!wgrad_tc_layout(R, C, D, num_sms, &wi, &grid, false, taps, kw, wp))
+    return cudaErrorInvalidValue;
+  // both plane sets whole: a tap's X rows past R read the map's zero fill
+  CUtensorMap mg, mx;
+  if (!encode_planes4_map(&mg, Gs, D, R, R) || !encode_planes4_map(&mx, Xs, C, R, R))
+    return cudaErrorInvalidValue;
+  float* part = static_cast<float*>(workspace);
+  float* bpart = part + (size_t)wi.nb * wi.n_dt * wi.n_ct * wi.maxj * (4 * WG_BC * WG_BD);
+  cudaError_t e = wgrad_attrs();
+  if (e != cudaSuccess) return e;
+  wgrad_tc_kernel<true><<<grid, WG_THREADS_PL, WG_SMEM, st>>>(mg, mx, R, C, D, wi, part, bpart,
+                                                              status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 fgrid((D + FZ_D - 1) / FZ_D, (C + FZ_C - 1) / FZ_C, taps);
+  if (out_dt == DType::F32)
+    wgrad_tc_finalize_kernel<float><<<fgrid, 256, 0, st>>>(
+        part, bpart, wi, C, D, static_cast<float*>(dW), static_cast<float*>(dbias), tw, 0);
+  else
+    wgrad_tc_finalize_kernel<__half><<<fgrid, 256, 0, st>>>(
+        part, bpart, wi, C, D, static_cast<__half*>(dW), static_cast<__half*>(dbias), tw, 0);
   return cudaGetLastError();
 }
 
