@@ -57,6 +57,12 @@
 // 12-15 drain planes 0-1 and 2-3 of the accumulators.  Needs C and D
 // multiples of 64.
 //
+// A convolution's taps (planes variant, launch_wgrad_tc_conv): the spectra of X
+// and dY on the convolution's padded pixel grid, the taps as further in-channel
+// tiles of the same stream-K problem.  Tap t = i * kw + j loads X's rows
+// i * wp + j further on than dY's (the TMA box reads zeros past the end), and
+// the finalize writes tap t's block of dW (grid.z = t).
+//
 // Tiled variant (PL, TL): the same spectra in the tiled layout of the SM-pair
 // kernels ([plane][channel / 16][Np rows][16 channels], 32-byte rows stored with
 // the 32-byte swizzle, written by the group-DFT pass).  One 4-D box per operand

@@ -446,8 +446,10 @@ EQL_API eqlinear_status_t eqlinear_conv_forward(eqlinear_plan_t plan, const void
  *     padded pixel grid ((H + 2 pad_h) x (W + 2 pad_w) per image: X shifted by
  *     the padding, dY at the top left, zeros elsewhere); tap (i, j) is then the
  *     layer's weight gradient between dY's padded rows and X's padded rows
- *     offset by i (W + 2 pad_w) + j (the layer's weight-gradient kernel, tensor
- *     cores when the shape allows).
+ *     offset by i (W + 2 pad_w) + j. With C and D multiples of 64 (and a plan
+ *     not forced to the CUDA cores), the padded rows' group spectra are formed
+ *     once and one tensor-core launch takes all taps; otherwise each tap runs
+ *     the layer's weight-gradient kernel.
  *   eqlinear_conv_backward_workspace_bytes(plan, N, H, W, KH, KW, pad_h, pad_w):
  *     scratch of both calls.
  * Plans and limits as for eqlinear_conv_forward; all pointers 16-byte aligned;
