@@ -97,3 +97,33 @@ def test_plan_create_without_gpu_reports_cuda_error(native):
     out = ctypes.c_void_p()
     assert native.raw_status("eqlinear_plan_create", 4, 16, 16, 0, ctypes.byref(out)) == \
         native.EQL_ERR_CUDA
+
+
+FREQUENCY_DOMAIN_AND_CONV_CALLS = (
+    "eqlinear_group_dft", "eqlinear_forward_tiled", "eqlinear_forward_tiled_next",
+    "eqlinear_backward_input_tiled", "eqlinear_forward_chain_tiled",
+    "eqlinear_backward_weight_tiled", "eqlinear_backward_weight_tiled_f32",
+    "eqlinear_conv_prepare_weights", "eqlinear_conv_forward", "eqlinear_conv_backward_input",
+    "eqlinear_conv_backward_weight", "eqlinear_forward_chain",
+)
+SIZE_QUERIES = (
+    "eqlinear_tiled_spectrum_bytes", "eqlinear_chain_tiled_workspace_bytes",
+    "eqlinear_conv_backward_workspace_bytes", "eqlinear_conv_prepared_weight_bytes",
+    "eqlinear_conv_workspace_bytes", "eqlinear_chain_workspace_bytes",
+)
+
+
+def _null_args(fn):
+    # null for every pointer (the plans included), 1 for every count and flag
+    return [None if t is ctypes.c_void_p else 1 for t in fn.argtypes]
+
+
+def test_frequency_domain_and_convolution_entries_reject_a_null_plan(native):
+    lib = ctypes.CDLL(native.LIB_PATH)
+    for name in FREQUENCY_DOMAIN_AND_CONV_CALLS:
+        fn = getattr(native._lib, name)
+        assert fn(*_null_args(fn)) == native.EQL_ERR_INVALID_ARG, name
+        assert hasattr(lib, name)
+    for name in SIZE_QUERIES:
+        fn = getattr(native._lib, name)
+        assert fn(*_null_args(fn)) == 0, name
