@@ -56,6 +56,8 @@ CASES = [
     (1, 6, 40, 32, 144, 3, 1, 1, 0),
     (1, 1, 1, 16, 16, 3, 3, 1, 1),      # one pixel: only the centre tap sees data
     (3, 8, 16, 80, 208, 2, 2, 1, 0),    # even kernel, asymmetric padding
+    (1, 6, 10, 192, 64, 3, 3, 1, 1),    # two 128-channel tiles per tap in dWc's single launch
+    (2, 5, 7, 128, 192, 3, 2, 1, 0),    # two out-channel tiles, a 3 x 2 kernel
 ]
 
 
